@@ -1,0 +1,190 @@
+"""Seeded synthetic inputs for paged decode.
+
+This module only draws random numbers and shapes. It holds none of the
+method's arithmetic (no slot or block indexing, no attention): block tables
+and slot mappings come from a block pool (the library's, or the oracle's in
+tests), which is handed the seeded free-block order drawn here.
+
+Every tensor is created on the CPU with ``torch.Generator`` seeded per
+workload, already rounded to its storage dtype.
+
+Workloads (shapes follow LLaMA-style decode layers):
+  tiny_fp32_mha        4 seqs, 4 heads, head_dim 64, block 16, lengths {1,17,45,100},
+                       64-block pool; q/k/v ~ N(0,1); scale 1/8
+  llama7b_mha_fp16     64 seqs, 32 heads, head_dim 128, block 16, lengths U{256..2048},
+                       pool 1.1x the blocks needed; q/k/v ~ 0.5 N(0,1); fp16 out
+  gqa_bf16             256 seqs, 32 query / 8 kv heads, head_dim 128, block 16,
+                       lengths log-normal (median 1024, sigma 0.5) clipped to
+                       [128, 4096]; q/k/v ~ N(0,1); fp32 out
+  long_splitk_bf16     8 seqs, 32 query / 8 kv heads, head_dim 128, block 32,
+                       lengths U{32768..131072}, pool exactly the blocks needed;
+                       q,k ~ N(0,1), v ~ U(-1,1); fp32 out
+  parallel_sampling_fp16  16 prompts x 5 branches, 32 heads, head_dim 128, block 16,
+                       1000-token shared prefix, each branch adds U{1..256} tokens;
+                       q/k/v ~ N(0,1); fp16 out
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, replace
+from typing import Dict, Optional
+
+import torch
+
+DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+
+
+@dataclass(frozen=True)
+class Spec:
+    name: str
+    num_seqs: int
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    kv_dtype: str
+    out_dtype: str
+    seed: int
+    # context-length law: ("fixed", [..]) | ("uniform", lo, hi) | ("lognormal", median, sigma, lo, hi)
+    lengths: tuple
+    pool_factor: Optional[float]  # pool = ceil(factor * needed); None = fixed pool_blocks
+    pool_blocks: int = 0
+    q_scale: float = 1.0
+    kv_scale: float = 1.0
+    v_uniform: bool = False
+    partition_size: int = 0  # split-K partition (tokens) the workload is run with; 0 = unsplit
+    # parallel sampling (copy-on-write) workload
+    num_prompts: int = 0
+    branches: int = 0
+    prefix_len: int = 0
+    max_divergent: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.head_dim)
+
+    @property
+    def torch_kv_dtype(self) -> torch.dtype:
+        return DTYPES[self.kv_dtype]
+
+    @property
+    def torch_out_dtype(self) -> torch.dtype:
+        return DTYPES[self.out_dtype]
+
+
+SPECS: Dict[str, Spec] = {
+    "tiny_fp32_mha": Spec("tiny_fp32_mha", 4, 4, 4, 64, 16, "f32", "f32", 3400,
+                          ("fixed", (1, 17, 45, 100)), None, pool_blocks=64),
+    "llama7b_mha_fp16": Spec("llama7b_mha_fp16", 64, 32, 32, 128, 16, "f16", "f16", 3401,
+                             ("uniform", 256, 2048), 1.1, q_scale=0.5, kv_scale=0.5),
+    "gqa_bf16": Spec("gqa_bf16", 256, 32, 8, 128, 16, "bf16", "f32", 3402,
+                     ("lognormal", 1024, 0.5, 128, 4096), 1.1),
+    "long_splitk_bf16": Spec("long_splitk_bf16", 8, 32, 8, 128, 32, "bf16", "f32", 3403,
+                             ("uniform", 32768, 131072), 1.0, v_uniform=True, partition_size=1024),
+    "parallel_sampling_fp16": Spec("parallel_sampling_fp16", 80, 32, 32, 128, 16, "f16", "f16", 3404,
+                                   ("parallel",), None, num_prompts=16, branches=5, prefix_len=1000,
+                                   max_divergent=256),
+}
+
+
+def scaled(spec: Spec, **changes) -> Spec:
+    """A copy of spec with some fields changed (smaller parity cases)."""
+    return replace(spec, **changes)
+
+
+def _normal(gen: torch.Generator, shape, scale: float, dtype: torch.dtype) -> torch.Tensor:
+    out = torch.empty(shape, dtype=dtype)
+    flat = out.view(-1)
+    chunk = 1 << 24
+    for i in range(0, flat.numel(), chunk):
+        n = min(chunk, flat.numel() - i)
+        x = torch.randn(n, generator=gen, dtype=torch.float32)
+        if scale != 1.0:
+            x.mul_(scale)
+        flat[i:i + n] = x.to(dtype)
+    return out
+
+
+def _uniform(gen: torch.Generator, shape, dtype: torch.dtype) -> torch.Tensor:
+    out = torch.empty(shape, dtype=dtype)
+    flat = out.view(-1)
+    chunk = 1 << 24
+    for i in range(0, flat.numel(), chunk):
+        n = min(chunk, flat.numel() - i)
+        x = torch.rand(n, generator=gen, dtype=torch.float32).mul_(2.0).sub_(1.0)
+        flat[i:i + n] = x.to(dtype)
+    return out
+
+
+def context_lengths(spec: Spec, gen: torch.Generator) -> torch.Tensor:
+    law = spec.lengths
+    if law[0] == "fixed":
+        return torch.tensor(law[1], dtype=torch.int32)
+    if law[0] == "uniform":
+        return torch.randint(law[1], law[2] + 1, (spec.num_seqs,), generator=gen, dtype=torch.int64).to(torch.int32)
+    if law[0] == "lognormal":
+        median, sigma, lo, hi = law[1:]
+        z = torch.randn(spec.num_seqs, generator=gen, dtype=torch.float64)
+        x = torch.round(median * torch.exp(sigma * z)).clamp_(lo, hi)
+        return x.to(torch.int32)
+    raise ValueError(law)
+
+
+def make_decode_inputs(spec: Spec) -> dict:
+    """Inputs for one decode step of a non-sampling workload.
+
+    Returns CPU tensors: context_lens [S] int32 (the newest token included);
+    free_order [NB] int32, the order in which the pool hands out physical
+    blocks (a seeded permutation); k_pool/v_pool [NB, Hkv, bs, D] (every slot
+    random; the newest token's slot is overwritten by the slot write);
+    new_key/new_value [S, Hkv, D], the newest token of each sequence;
+    query [S, Hq, D].
+    """
+    assert spec.lengths[0] != "parallel"
+    gen = torch.Generator().manual_seed(spec.seed)
+    dt = spec.torch_kv_dtype
+    ctx = context_lengths(spec, gen)
+    needed = int(sum((int(c) + spec.block_size - 1) // spec.block_size for c in ctx.tolist()))
+    nb = spec.pool_blocks if spec.pool_factor is None else int(math.ceil(spec.pool_factor * needed))
+    nb = max(nb, needed)
+    free_order = torch.randperm(nb, generator=gen).to(torch.int32)
+    shape = (nb, spec.num_kv_heads, spec.block_size, spec.head_dim)
+    k_pool = _normal(gen, shape, spec.kv_scale, dt)
+    v_pool = _uniform(gen, shape, dt) if spec.v_uniform else _normal(gen, shape, spec.kv_scale, dt)
+    kv_shape = (spec.num_seqs, spec.num_kv_heads, spec.head_dim)
+    new_key = _normal(gen, kv_shape, spec.kv_scale, dt)
+    new_value = _uniform(gen, kv_shape, dt) if spec.v_uniform else _normal(gen, kv_shape, spec.kv_scale, dt)
+    query = _normal(gen, (spec.num_seqs, spec.num_heads, spec.head_dim), spec.q_scale, dt)
+    return dict(context_lens=ctx, free_order=free_order, k_pool=k_pool, v_pool=v_pool,
+                new_key=new_key, new_value=new_value, query=query, num_blocks=nb)
+
+
+def make_parallel_sampling_inputs(spec: Spec) -> dict:
+    """Inputs for the parallel-sampling workload: num_prompts prompts of
+    prefix_len tokens, each forked into `branches` branches that append
+    U{1..max_divergent} tokens each, then one decode over every branch.
+
+    Returns CPU tensors: prefix_key/prefix_value [P, prefix_len, Hkv, D];
+    divergent_lens [P, branches] int32; divergent_key/divergent_value
+    [sum(divergent_lens), Hkv, D] in (prompt, branch, token) order;
+    query [P * branches, Hq, D]; free_order [NB] int32; num_blocks.
+    """
+    assert spec.lengths[0] == "parallel"
+    gen = torch.Generator().manual_seed(spec.seed)
+    dt = spec.torch_kv_dtype
+    P, B = spec.num_prompts, spec.branches
+    div = torch.randint(1, spec.max_divergent + 1, (P, B), generator=gen, dtype=torch.int64).to(torch.int32)
+    prefix_blocks = (spec.prefix_len + spec.block_size - 1) // spec.block_size
+    per_branch = (spec.prefix_len + spec.max_divergent + spec.block_size - 1) // spec.block_size + 1
+    nb = P * (prefix_blocks + B * per_branch)
+    free_order = torch.randperm(nb, generator=gen).to(torch.int32)
+    kv = (spec.num_kv_heads, spec.head_dim)
+    prefix_key = _normal(gen, (P, spec.prefix_len) + kv, 1.0, dt)
+    prefix_value = _normal(gen, (P, spec.prefix_len) + kv, 1.0, dt)
+    total = int(div.sum())
+    divergent_key = _normal(gen, (total,) + kv, 1.0, dt)
+    divergent_value = _normal(gen, (total,) + kv, 1.0, dt)
+    query = _normal(gen, (P * B, spec.num_heads, spec.head_dim), 1.0, dt)
+    return dict(prefix_key=prefix_key, prefix_value=prefix_value, divergent_lens=div,
+                divergent_key=divergent_key, divergent_value=divergent_value, query=query,
+                free_order=free_order, num_blocks=nb)
