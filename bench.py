@@ -1,0 +1,472 @@
+"""Benchmark of the paged decode hot path on B200.
+
+A step is one pass of the hot path over one synthetic batch: the copy-on-write
+block copies the batch needs (none for the decode-only workloads), the slot
+write of the step's new tokens, and decode (split-K plus its reduce when the
+partition rule splits the batch). The default workload is the LLaMA-7B-shaped
+fp16 decode layer (64 sequences, 32 heads, head_dim 128, block 16, context
+lengths U{256..2048}).
+
+metric: effective GB/s = algorithmic bytes of the step / device time of the
+step, with
+  decode bytes = sum_s ctx_s * 2 * Hkv * D * elt + S * Hq * D * (elt_q + elt_out)
+                 + 4 * sum_s ceil(ctx_s / bs) + 4 * S
+  slot-write bytes = 2 * T * Hkv * D * elt (read) + the same (write) + 4 * T
+Inputs (>= 1.2 GB of K/V) are larger than L2, so no flush between steps.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1, launch under torchrun: each rank runs its own batch (sequences
+shard across GPUs with no exchange), value = all ranks' bytes / max time.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+DEFAULT_WORKLOAD = "llama7b_mha_fp16"
+METRIC = "paged decode: effective KV GB/s (% of HBM peak) and seq-tokens/s on 1 B200"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def elt(dtype: torch.dtype) -> int:
+    return torch.tensor([], dtype=dtype).element_size()
+
+
+def decode_bytes(spec, ctx: np.ndarray) -> int:
+    """Algorithmic bytes of one decode over the batch (K/V read once, q read,
+    out written, the used table entries and the context lengths read)."""
+    e = elt(spec.torch_kv_dtype)
+    kv = int(ctx.astype(np.int64).sum()) * 2 * spec.num_kv_heads * spec.head_dim * e
+    qo = len(ctx) * spec.num_heads * spec.head_dim * (e + elt(spec.torch_out_dtype))
+    tables = 4 * int(((ctx.astype(np.int64) + spec.block_size - 1) // spec.block_size).sum()) + 4 * len(ctx)
+    return kv + qo + tables
+
+
+def kv_bytes_per_token(num_layers: int, num_kv_heads: int, head_dim: int, elt_bytes: int) -> int:
+    """K and V bytes of one token across all layers (2 * layers * heads * dim * elt)."""
+    return 2 * num_layers * num_kv_heads * head_dim * elt_bytes
+
+
+def write_bytes(spec, num_tokens: int) -> int:
+    row = spec.num_kv_heads * spec.head_dim * elt(spec.torch_kv_dtype)
+    return 2 * 2 * num_tokens * row + 4 * num_tokens
+
+
+def copy_bytes(spec, num_pairs: int) -> int:
+    blk = spec.num_kv_heads * spec.block_size * spec.head_dim * elt(spec.torch_kv_dtype)
+    return 2 * 2 * num_pairs * blk + 16 * num_pairs
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in ("pa_decode.cu", "pa_common.cuh", "pa_internal.h"):
+        with open(os.path.join(ROOT, "paged_kv_cache_340_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "decode_dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    e = rec.get(workload, {}).get(kernel)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.uuid = None
+        try:
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            self.uuid = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.06)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for row in csv.reader(io.StringIO(out)):
+            if len(row) < 8:
+                continue
+            try:
+                sm.append(float(row[0]))
+                mx.append(float(row[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, row[4:8]):
+                if v.strip().lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------ measurement
+
+def build_batch(name: str, rank: int, partition=None):
+    from paged_kv_cache_340_b200.batch import build_decode_batch, build_parallel_sampling_batch, write_prefix
+    from paged_kv_cache_340_b200.workloads import SPECS, make_decode_inputs, make_parallel_sampling_inputs, scaled
+    spec = SPECS[name]
+    if rank:
+        spec = scaled(spec, seed=spec.seed + 1000 * rank)
+    if spec.lengths[0] == "parallel":
+        inp = make_parallel_sampling_inputs(spec)
+        b = build_parallel_sampling_batch(spec, inp, partition_size=partition or 0)
+        write_prefix(b)
+    else:
+        inp = make_decode_inputs(spec)
+        b = build_decode_batch(spec, inp, partition_size=partition)
+    torch.cuda.synchronize()
+    b.host_inputs = inp
+    return spec, b
+
+
+def step_bytes(spec, b) -> dict:
+    d = decode_bytes(spec, b.host_context_lens)
+    w = write_bytes(spec, b.new_key.shape[0])
+    c = copy_bytes(spec, b.cow_pairs.shape[0])
+    return dict(decode=d, write=w, copy=c, total=d + w + c)
+
+
+def launches_per_step(b) -> int:
+    return (1 if b.cow_pairs.shape[0] else 0) + 1 + (2 if b.partition_size else 1)
+
+
+def time_steps(b, steps: int, warmup: int, world: int, sample_clocks=False, device_index=0):
+    """Device time of `steps` steps (max over ranks), and the mean duration of
+    each kernel, from CUDA events on the launching stream."""
+    from paged_kv_cache_340_b200 import pa_copy_blocks, pa_decode, pa_decode_splitk, pa_reshape_and_cache, \
+        pa_splitk_reduce
+    spec = b.spec
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if b.cow_pairs.shape[0]:
+            pa_copy_blocks(b.k_cache, b.v_cache, b.cow_pairs, stream=stream)
+        pa_reshape_and_cache(b.new_key, b.new_value, b.k_cache, b.v_cache, b.slot_mapping, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        if b.partition_size:
+            pa_decode_splitk(b.workspace, b.query, b.k_cache, b.v_cache, b.block_tables, b.context_lens, spec.scale,
+                             b.max_context_len, b.partition_size, stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+            pa_splitk_reduce(b.out, b.workspace, b.context_lens, b.max_context_len, b.partition_size,
+                             stream=stream)
+        else:
+            pa_decode(b.out, b.query, b.k_cache, b.v_cache, b.block_tables, b.context_lens, spec.scale,
+                      stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    # whole-step timing (no per-kernel events inside)
+    sampler = ClockSampler(device_index) if sample_clocks else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.15)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    ms = t0.elapsed_time(t1)
+    ms = max_over_ranks(ms, world)
+    # per-kernel durations over a second pass of the same steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    dec = statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
+    red = statistics.fmean(e[1].elapsed_time(e[2]) for e in evs)
+    return ms / steps, dec, red, clocks
+
+
+def e2e_steps(b, steps: int, warmup: int, world: int):
+    """The same step through the public API with host buffers: every step
+    copies its inputs from pinned host memory (query, new K/V, slots, block
+    tables, context lengths) and reads the output back to pinned memory."""
+    from paged_kv_cache_340_b200.batch import run_step
+    stream = torch.cuda.current_stream()
+    host_in = [(t.cpu().pin_memory(), t) for t in (b.query, b.new_key, b.new_value, b.slot_mapping, b.block_tables,
+                                                    b.context_lens, b.cow_pairs) if t.numel()]
+    host_out = torch.empty(b.out.shape, dtype=b.out.dtype, pin_memory=True)
+    h2d = sum(h.numel() * h.element_size() for h, _ in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+
+    def one():
+        for h, d in host_in:
+            d.copy_(h, non_blocking=True)
+        run_step(b, stream=stream)
+        host_out.copy_(b.out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        one()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(t0.elapsed_time(t1), world) / steps
+    return ms, h2d, d2h
+
+
+# ---------------------------------------------------------- CPU oracle legs
+
+def oracle_sample(spec, b, budget_s: float, start_seq: int = 0):
+    """Times the oracle (as it stands, single-threaded double C) on whole
+    sequences of the batch, from start_seq on, until budget_s of oracle time is
+    spent. Returns (bytes, seconds, sequences). The oracle reads the host
+    copies of the generated inputs; widening to float64 is outside the timed
+    calls."""
+    import oracle
+    oracle.build()
+    if "k_pool" not in b.host_inputs:
+        raise SystemExit("the CPU oracle legs time the decode-only workloads")
+    k = b.host_inputs["k_pool"]
+    v = b.host_inputs["v_pool"]
+    q = b.host_inputs["query"]
+    tot_bytes, tot_s, n_seq = 0, 0.0, 0
+    S = len(b.host_context_lens)
+    s = start_seq
+    while tot_s < budget_s and n_seq < S:
+        L = int(b.host_context_lens[s % S])
+        nb = (L + spec.block_size - 1) // spec.block_size
+        ids = torch.from_numpy(b.host_tables[s % S, :nb].astype(np.int64))
+        kp = k.index_select(0, ids).double().numpy()
+        vp = v.index_select(0, ids).double().numpy()
+        qs = q[s % S:s % S + 1].double().numpy()
+        tab = np.arange(max(nb, 1), dtype=np.int32)[None, :]
+        t = time.perf_counter()
+        oracle.paged_decode(qs, kp, vp, tab, np.array([L], np.int32), spec.scale, spec.block_size)
+        tot_s += time.perf_counter() - t
+        tot_bytes += decode_bytes(spec, np.array([L]))
+        n_seq += 1
+        s += 1
+    return tot_bytes, tot_s, n_seq
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle, timed on the host cores, on the same
+    workload, metric and unit. Rank 0 only."""
+    if rank != 0:
+        return
+    spec, b = build_batch(args.workload, 0)
+    budget = max(0.002, min(2.0, 90.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(spec, b, budget / 4)
+    tot_b, tot_s, seqs = 0, 0.0, 0
+    for i in range(args.steps):
+        nb_, ns_, nq_ = oracle_sample(spec, b, budget, start_seq=i)
+        tot_b += nb_
+        tot_s += ns_
+        seqs += nq_
+    gbs = tot_b / tot_s / 1e9
+    sample = (f"{seqs} whole sequences (all {spec.num_heads} heads each) of the {spec.name} batch over "
+              f"{args.steps} steps, about {budget:.3g} s of oracle time per step; float64 C, one thread")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / max(1, args.steps), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name, "num_seqs": spec.num_seqs, "num_heads": spec.num_heads,
+                   "num_kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim, "block_size": spec.block_size,
+                   "kv_dtype": spec.kv_dtype},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def measure_other(name: str, steps: int, warmup: int):
+    spec, b = build_batch(name, 0)
+    ms, dec, red, _ = time_steps(b, steps, warmup, 1)
+    by = step_bytes(spec, b)
+    peak, _ = peaks()
+    res = {"ms_per_step": round(ms, 4), "GBps": round(by["total"] / ms / 1e6, 1),
+           "pct_of_hbm_peak": round(100 * by["total"] / ms / 1e6 / peak, 1),
+           "decode_kernel_ms": round(dec, 4), "decode_kernel_GBps": round(by["decode"] / dec / 1e6, 1),
+           "partition_size": b.partition_size, "seq_tokens_per_s": round(spec.num_seqs / ms * 1e3, 1)}
+    if b.partition_size:
+        res["reduce_kernel_ms"] = round(red, 4)
+    del b
+    torch.cuda.empty_cache()
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--partition", type=int, default=None, help="force a split-K partition size (0 = unsplit)")
+    ap.add_argument("--no-others", action="store_true", help="skip the other workloads' lines")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    world, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    import paged_kv_cache_340_b200 as pa  # noqa: F401  (fails loudly without the CUDA library)
+
+    spec, b = build_batch(args.workload, rank, args.partition)
+    ms, dec_ms, red_ms, clocks = time_steps(b, args.steps, args.warmup, world, sample_clocks=(rank == 0),
+                                            device_index=local)
+    by = step_bytes(spec, b)
+    peak, peak_kind = peaks()
+    value = world * by["total"] / (ms * 1e-3) / 1e9
+    e2e_ms, h2d, d2h = e2e_steps(b, max(10, args.steps // 4), args.warmup, world)
+    kernel = "pa_decode_splitk" if b.partition_size else "pa_decode"
+    achieved = by["decode"] / (dec_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": spec.kv_dtype, "data": "synthetic",
+        "config": {"workload": spec.name, "num_seqs": spec.num_seqs, "num_heads": spec.num_heads,
+                   "num_kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim, "block_size": spec.block_size,
+                   "context_lens": "U{256..2048}" if spec.name == DEFAULT_WORKLOAD else str(spec.lengths),
+                   "kv_dtype": spec.kv_dtype, "out_dtype": spec.out_dtype, "partition_size": b.partition_size,
+                   "parallelism": f"dp{world} (sequences shard, no exchange)",
+                   "l2": "inputs larger than L2 (K/V >= 1.2 GB per step), no flush",
+                   "step": "copy_blocks (if any) + reshape_and_cache + decode"},
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "seq_tokens_per_s": round(world * spec.num_seqs / (ms * 1e-3), 1),
+        "context_tokens_per_s": round(world * float(b.host_context_lens.sum()) / (ms * 1e-3), 1),
+        "bytes_per_step": by,
+        "e2e": {"value": round(world * by["total"] / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1), "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "kernel_ms": round(dec_ms, 5),
+                     "traffic": recorded_traffic(spec.name, kernel)},
+        "gpu_launches": launches_per_step(b) * args.steps,
+        "clocks": clocks,
+    }
+    if b.partition_size:
+        line["roofline"]["reduce_kernel_ms"] = round(red_ms, 5)
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        nbytes, secs, nseq = oracle_sample(spec, b, 12.0)
+        line["cpu_baseline"] = {"value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{nseq} of {spec.num_seqs} sequences (all heads), decode only; "
+                                          f"float64 C oracle, one thread, {secs:.1f} s"}
+    del b
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_others and args.workload == DEFAULT_WORKLOAD:
+        line["other_workloads"] = {n: measure_other(n, 200, 10) for n in
+                                   ("gqa_bf16", "long_splitk_bf16", "parallel_sampling_fp16")}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,240 @@
+/*
+ * pa.h -- C ABI of the paged KV-cache decode library for NVIDIA B200 (sm_100a).
+ *
+ * A sequence's keys and values live in fixed-size blocks of a shared pool; a
+ * per-sequence block table maps logical block i (tokens i*bs .. i*bs+bs-1) to
+ * a physical block, so no sequence needs contiguous memory.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [P1] "PagedAttention 源码解析：KV Cache 怎么管理" (coreui.cn)
+ *   [P2] "PagedAttention原理与KV Cache显存优化" (xdnf.cn)
+ *   [P3] "Ascend C算子开发高阶实战：实现高性能KV Cache管理与PagedAttention融合算子" (cann.csdn.net)
+ *   [P4] "PagedAttention 实现细节" (pyllm.pages.dev, vLLM series)
+ *   [P5] "Ascend平台下的PageAttention优化实践" (jsqmd.com)
+ *
+ * Conventions for every device entry point:
+ *   - Pointers named *_cache, query, out, key, value, block_tables,
+ *     context_lens, slot_mapping, src_dst_pairs and workspace are DEVICE
+ *     pointers owned by the caller. The library never allocates, frees or
+ *     keeps them.
+ *   - Layouts (row-major, contiguous):
+ *       k_cache, v_cache  [num_blocks, num_kv_heads, block_size, head_dim]
+ *       query, out        [num_seqs, num_heads, head_dim]
+ *       key, value        [num_tokens, num_kv_heads, head_dim]
+ *       block_tables      [num_seqs, max_blocks_per_seq] int32
+ *       context_lens      [num_seqs] int32
+ *       slot_mapping      [num_tokens] int32
+ *     Token t of sequence s is row (block_tables[s][t / block_size], kv head,
+ *     t % block_size) of the pools ([P2] §3.1; [P4] §3.1 index-based kernel).
+ *   - Supported: head_dim 64 or 128; block_size 16 or 32; num_heads a
+ *     multiple of num_kv_heads with num_heads / num_kv_heads in {1, 2, 4, 8}
+ *     (query head h reads kv head h / (num_heads / num_kv_heads)); element
+ *     types PA_F32, PA_F16, PA_BF16. Every device pointer must be 16-byte
+ *     aligned.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream)
+ *     and return PA_OK once the work is enqueued. Arguments are checked on
+ *     the host first; a violation returns a negative pa_status and enqueues
+ *     nothing. A failed launch returns PA_ERR_CUDA.
+ *   - Data errors that only the device can see (a table entry or slot out of
+ *     range, a context longer than its table row) never fault: the kernel
+ *     skips the offending block or token and records a PA_DEVERR_* bit in a
+ *     device error word that pa_read_device_errors() returns.
+ */
+#ifndef PAGED_KV_CACHE_340_B200_PA_H
+#define PAGED_KV_CACHE_340_B200_PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_dtype { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_NULL = -1,            /* a required pointer is NULL */
+    PA_ERR_DTYPE = -2,           /* unsupported element type or output type */
+    PA_ERR_SHAPE = -3,           /* a size is negative or inconsistent */
+    PA_ERR_HEADS = -4,           /* num_heads % num_kv_heads != 0 or group not in {1,2,4,8} */
+    PA_ERR_HEAD_DIM = -5,        /* head_dim not in {64, 128} */
+    PA_ERR_BLOCK_SIZE = -6,      /* block_size not in {16, 32} */
+    PA_ERR_ALIGN = -7,           /* a device pointer is not 16-byte aligned */
+    PA_ERR_PARTITION = -8,       /* partition_size not a positive multiple of block_size */
+    PA_ERR_WORKSPACE = -9,       /* workspace smaller than pa_splitk_workspace_bytes() */
+    PA_ERR_CUDA = -10,           /* a CUDA runtime call or launch failed */
+    PA_ERR_POOL_EXHAUSTED = -11, /* host pool: no free block */
+    PA_ERR_POOL_STATE = -12,     /* host pool: block id out of range or already free */
+    PA_ERR_CAPACITY = -13        /* host pool: caller's table row or output array too small */
+} pa_status;
+
+/* Bits of the device error word (see pa_read_device_errors). */
+#define PA_DEVERR_BLOCK_ID 0x1u  /* table entry outside [0, num_blocks): its tokens were skipped */
+#define PA_DEVERR_SLOT 0x2u      /* slot >= num_blocks * block_size: the token was not written */
+#define PA_DEVERR_CONTEXT 0x4u   /* context_len < 0, or longer than its table row / max_context_len: clamped */
+#define PA_DEVERR_TIMEOUT 0x8u   /* an on-chip pipeline wait ran past its bound: output undefined */
+#define PA_DEVERR_PAIR 0x10u     /* copy pair with an id outside [0, num_blocks): skipped */
+
+/* Text for a pa_status value (static storage, never NULL). */
+const char *pa_status_string(int status);
+
+/* Waits for `stream`, then returns in *flags the PA_DEVERR_* bits recorded
+ * by kernels on the current device since the last call, and clears them.
+ * Returns PA_ERR_CUDA if the synchronisation or copy fails. */
+int pa_read_device_errors(uint32_t *flags, cudaStream_t stream);
+
+/*
+ * pa_reshape_and_cache -- slot write of new tokens.
+ * For each token i with slot = slot_mapping[i] >= 0 and every kv head h:
+ *   k_cache[slot / block_size, h, slot % block_size, :] = key[i, h, :]
+ *   v_cache[slot / block_size, h, slot % block_size, :] = value[i, h, :]
+ * as a bit copy. Negative slots are skipped. Non-negative slots must be
+ * distinct within one call (two writes to one slot race).
+ * [P3] §3.1 and §4.2 (slot_mapping, block_id = slot / block_size,
+ * offset = slot % block_size); [P4] §3.4 (the runner writes each new token's
+ * K/V into its block).
+ * key/value/k_cache/v_cache share dtype `kv_dtype`.
+ */
+int pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
+                         const int32_t *slot_mapping, int num_tokens, int num_blocks,
+                         int num_kv_heads, int head_dim, int block_size, pa_dtype kv_dtype,
+                         cudaStream_t stream);
+
+/*
+ * pa_decode -- fused paged decode attention, one pass, no partitioning.
+ * For each sequence s (L = context_lens[s] tokens) and query head h:
+ *   out[s, h, :] = sum_t softmax_t(scale * query[s, h, :] . K_t) V_t,  t < L,
+ * where K_t, V_t are read in place from the pools through block_tables[s]
+ * (no gathered copy), with fp32 accumulation and a running max and sum.
+ * L == 0 writes zeros. Entries of block_tables[s] past ceil(L / block_size)
+ * are never read. query has dtype kv_dtype; out_dtype is kv_dtype or PA_F32.
+ * [P3] §1.3 (softmax(QK^T / sqrt(d)) V over the gathered history) and §3
+ * (gather and attention fused in one pass, no intermediate written back);
+ * [P4] §3.1 (index-based kernel over key_cache/value_cache
+ * [num_blocks, num_kv_heads, block_size, head_dim]); [P5] §3.2 (inputs
+ * query, key_cache, value_cache, block_tables, context_lens, scale).
+ */
+int pa_decode(void *out, const void *query, const void *k_cache, const void *v_cache,
+              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+              int num_seqs, int num_heads, int num_kv_heads, int head_dim, float scale,
+              int block_size, int num_blocks, pa_dtype kv_dtype, pa_dtype out_dtype,
+              cudaStream_t stream);
+
+/*
+ * Split-K (partitioned) decode for few, long sequences ([P5] §2.3: the
+ * partitioned kernel of the pair). Tokens of sequence s are cut into
+ * partitions of `partition_size` tokens (a multiple of block_size); partition
+ * p covers [p * P, min((p + 1) * P, L)). pa_decode_splitk writes, per
+ * (s, h, p) with a non-empty range:
+ *   m   = max_t scale * q . K_t                          (float)
+ *   l   = sum_t exp(scale * q . K_t - m)                 (float)
+ *   acc = sum_t exp(scale * q . K_t - m) V_t             (float[head_dim])
+ * into `workspace`, laid out as
+ *   ml  float [num_seqs, num_heads, max_parts, 2]   (m, l) at offset 0
+ *   acc float [num_seqs, num_heads, max_parts, head_dim] at byte offset
+ *       pa_splitk_acc_offset(...)
+ * with max_parts = ceil(max_context_len / partition_size). Entries of empty
+ * partitions are not written. max_context_len must bound every
+ * context_lens[s]; longer contexts are clamped (PA_DEVERR_CONTEXT).
+ * pa_splitk_reduce then merges them by log-sum-exp:
+ *   M = max_p m_p,  out = sum_p e^(m_p - M) acc_p / sum_p e^(m_p - M) l_p
+ * (the standard split of the softmax; the pages only name the partitioned
+ * kernel). Both calls must get the same sizes.
+ */
+size_t pa_splitk_workspace_bytes(int num_seqs, int num_heads, int head_dim, int max_context_len,
+                                 int partition_size);
+size_t pa_splitk_acc_offset(int num_seqs, int num_heads, int max_context_len, int partition_size);
+
+int pa_decode_splitk(void *workspace, size_t workspace_bytes, const void *query,
+                     const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                     int max_blocks_per_seq, const int32_t *context_lens, int num_seqs,
+                     int num_heads, int num_kv_heads, int head_dim, float scale, int block_size,
+                     int num_blocks, int max_context_len, int partition_size, pa_dtype kv_dtype,
+                     cudaStream_t stream);
+
+int pa_splitk_reduce(void *out, const void *workspace, size_t workspace_bytes,
+                     const int32_t *context_lens, int num_seqs, int num_heads, int head_dim,
+                     int max_context_len, int partition_size, pa_dtype out_dtype,
+                     cudaStream_t stream);
+
+/*
+ * Partition size this library would pick for a batch: 0 when the
+ * unpartitioned pa_decode already fills the GPU, else a multiple of
+ * block_size. Host-only arithmetic on the sizes given (occupancy rule:
+ * split until there are enough work items for every SM).
+ */
+int pa_choose_partition(int num_seqs, int num_kv_heads, int max_context_len, int block_size,
+                        int head_dim, pa_dtype kv_dtype);
+
+/*
+ * pa_copy_blocks -- copy-on-write block copy. For each pair
+ * (src_dst_pairs[2i], src_dst_pairs[2i+1]) = (src, dst): physical block dst
+ * of both pools becomes a bit copy of block src (all kv heads, all slots).
+ * Preconditions: dst ids distinct, and no dst is also a src in the same call
+ * (all pairs run in parallel). Pairs with an id outside [0, num_blocks) are
+ * skipped (PA_DEVERR_PAIR). src_dst_pairs is a device int64 [num_pairs, 2].
+ * [P4] §3.3 (copy the whole block, device to device, before writing the
+ * copy); [P2] §3.4 (parallel sampling, beam search).
+ */
+int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pairs, int num_pairs,
+                   int num_blocks, int num_kv_heads, int head_dim, int block_size,
+                   pa_dtype kv_dtype, cudaStream_t stream);
+
+/*
+ * Host block pool (no device memory): free list, reference counts and the
+ * copy-on-write decision. These are plain host calls on host memory.
+ * [P2] §3.3-§3.4 and §4.2 (PhysicalBlockPool: allocate sets the count to 1,
+ * free returns a block at count 0; append_token_kv takes a new block when the
+ * cached token count is a multiple of the block size); [P4] §3.3 (write into
+ * a block whose count is above 1: take a new block, copy, drop the old
+ * block's count, give the copy count 1, repoint the table).
+ * A pool is not thread-safe; callers serialise access.
+ */
+typedef struct pa_block_pool pa_block_pool;
+
+enum { PA_POOL_LIFO = 0, PA_POOL_FIFO = 1 };
+
+/* free_order: NULL for 0..num_blocks-1, else a permutation of the ids giving
+ * the initial free list. PA_POOL_LIFO hands out the list's last entry
+ * ([P2] §4.2), PA_POOL_FIFO its first ([P1] §3); freed blocks go to the end.
+ * Returns NULL on bad arguments or if free_order is not a permutation. */
+pa_block_pool *pa_pool_create(int num_blocks, int block_size, int policy,
+                              const int32_t *free_order);
+void pa_pool_destroy(pa_block_pool *pool);
+int pa_pool_num_free(const pa_block_pool *pool);
+/* Reference count of a block (0 = free), or PA_ERR_POOL_STATE for a bad id. */
+int pa_pool_ref_count(const pa_block_pool *pool, int block);
+int pa_pool_allocate(pa_block_pool *pool, int32_t *block_out);
+int pa_pool_share(pa_block_pool *pool, int block);
+int pa_pool_free(pa_block_pool *pool, int block);
+
+/*
+ * Appends n_new tokens to a sequence whose host table row `table` (capacity
+ * max_blocks) and token count *num_tokens describe it. Token t = *num_tokens
+ * goes to table[t / bs] at offset t % bs: a new block is taken when t % bs == 0;
+ * otherwise, if that block's count is above 1, it is copied first (the pair
+ * (old, new) is appended to cow_pairs as two int64, the row is repointed).
+ * slots (nullable) receives each new token's slot. cow_pairs (nullable when
+ * cow_capacity is 0) has room for cow_capacity pairs; *num_cow receives the
+ * count. On an error the tokens appended before it stay appended and
+ * *num_tokens says how many there are.
+ */
+int pa_pool_append(pa_block_pool *pool, int32_t *table, int max_blocks, int32_t *num_tokens,
+                   int n_new, int32_t *slots, int64_t *cow_pairs, int cow_capacity, int *num_cow);
+
+/* Makes dst_table share every block of table (first ceil(num_tokens / bs)
+ * entries): each count goes up by one. */
+int pa_pool_fork(pa_block_pool *pool, const int32_t *table, int num_tokens, int32_t *dst_table,
+                 int max_blocks);
+
+/* Drops the sequence's reference to each of its blocks. */
+int pa_pool_release(pa_block_pool *pool, const int32_t *table, int num_tokens);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_KV_CACHE_340_B200_PA_H */

@@ -1,0 +1,268 @@
+"""Python binding of the paged KV-cache decode library for B200 (sm_100a).
+
+Argument marshalling only: every operation runs in the CUDA kernels of
+``lib/libpa_b200.so`` through its C ABI (``include/pa.h``); functions keep the
+C names. PyTorch supplies device memory and streams. There is no CPU or
+library fallback: if the shared library is missing, importing the binding
+raises.
+
+Layouts (contiguous): k_cache/v_cache [num_blocks, num_kv_heads, block_size,
+head_dim]; query/out [num_seqs, num_heads, head_dim]; key/value
+[num_tokens, num_kv_heads, head_dim]; block_tables [num_seqs,
+max_blocks_per_seq] int32; context_lens [num_seqs] int32; slot_mapping
+[num_tokens] int32; src_dst_pairs [n, 2] int64.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import numpy as np
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libpa_b200.so")
+
+PA_F32, PA_F16, PA_BF16 = 0, 1, 2
+_DT = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
+
+PA_DEVERR_BLOCK_ID = 0x1
+PA_DEVERR_SLOT = 0x2
+PA_DEVERR_CONTEXT = 0x4
+PA_DEVERR_TIMEOUT = 0x8
+PA_DEVERR_PAIR = 0x10
+
+PA_POOL_LIFO, PA_POOL_FIFO = 0, 1
+
+EXPORTED = (
+    "pa_status_string", "pa_read_device_errors", "pa_reshape_and_cache", "pa_decode",
+    "pa_splitk_workspace_bytes", "pa_splitk_acc_offset", "pa_decode_splitk", "pa_splitk_reduce",
+    "pa_choose_partition", "pa_copy_blocks", "pa_pool_create", "pa_pool_destroy", "pa_pool_num_free",
+    "pa_pool_ref_count", "pa_pool_allocate", "pa_pool_share", "pa_pool_free", "pa_pool_append",
+    "pa_pool_fork", "pa_pool_release",
+)
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, what: str, status: int):
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m paged_kv_cache_340_b200._build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, sz, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    sig = {
+        "pa_status_string": (ctypes.c_char_p, [i32]),
+        "pa_read_device_errors": (i32, [ctypes.POINTER(ctypes.c_uint32), vp]),
+        "pa_reshape_and_cache": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
+        "pa_decode": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32, vp]),
+        "pa_splitk_workspace_bytes": (sz, [i32, i32, i32, i32, i32]),
+        "pa_splitk_acc_offset": (sz, [i32, i32, i32, i32]),
+        "pa_decode_splitk": (i32, [vp, sz, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32,
+                                   i32, vp]),
+        "pa_splitk_reduce": (i32, [vp, vp, sz, vp, i32, i32, i32, i32, i32, i32, vp]),
+        "pa_choose_partition": (i32, [i32, i32, i32, i32, i32, i32]),
+        "pa_copy_blocks": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
+        "pa_pool_create": (vp, [i32, i32, i32, i32p]),
+        "pa_pool_destroy": (None, [vp]),
+        "pa_pool_num_free": (i32, [vp]),
+        "pa_pool_ref_count": (i32, [vp, i32]),
+        "pa_pool_allocate": (i32, [vp, i32p]),
+        "pa_pool_share": (i32, [vp, i32]),
+        "pa_pool_free": (i32, [vp, i32]),
+        "pa_pool_append": (i32, [vp, i32p, i32, i32p, i32, i32p, i64p, i32, ctypes.POINTER(ctypes.c_int)]),
+        "pa_pool_fork": (i32, [vp, i32p, i32, i32p, i32]),
+        "pa_pool_release": (i32, [vp, i32p, i32]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def status_string(status: int) -> str:
+    return _lib.pa_status_string(int(status)).decode()
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise PagedAttentionError(what, rc)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise ValueError(f"unsupported dtype {t.dtype}")
+    return _DT[t.dtype]
+
+
+# ------------------------------------------------------------------ device
+
+def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None) -> None:
+    NB, Hkv, bs, D = k_cache.shape
+    rc = _lib.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+                                   slot_mapping.shape[0], NB, Hkv, D, bs, _dtype(k_cache), _stream(stream))
+    _check(rc, "pa_reshape_and_cache")
+
+
+def pa_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale, stream=None) -> None:
+    S, Hq, D = query.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    rc = _lib.pa_decode(_ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                        block_tables.shape[1], _ptr(context_lens), S, Hq, Hkv, D, float(scale), bs, NB,
+                        _dtype(k_cache), _dtype(out), _stream(stream))
+    _check(rc, "pa_decode")
+
+
+def pa_splitk_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, partition_size) -> int:
+    return int(_lib.pa_splitk_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, partition_size))
+
+
+def pa_splitk_acc_offset(num_seqs, num_heads, max_context_len, partition_size) -> int:
+    return int(_lib.pa_splitk_acc_offset(num_seqs, num_heads, max_context_len, partition_size))
+
+
+def pa_decode_splitk(workspace, query, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
+                     partition_size, stream=None) -> None:
+    S, Hq, D = query.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    rc = _lib.pa_decode_splitk(_ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(query),
+                               _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1],
+                               _ptr(context_lens), S, Hq, Hkv, D, float(scale), bs, NB, int(max_context_len),
+                               int(partition_size), _dtype(k_cache), _stream(stream))
+    _check(rc, "pa_decode_splitk")
+
+
+def pa_splitk_reduce(out, workspace, context_lens, max_context_len, partition_size, stream=None) -> None:
+    S, Hq, D = out.shape
+    rc = _lib.pa_splitk_reduce(_ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _ptr(context_lens), S, Hq, D, int(max_context_len), int(partition_size),
+                               _dtype(out), _stream(stream))
+    _check(rc, "pa_splitk_reduce")
+
+
+def pa_choose_partition(num_seqs, num_kv_heads, max_context_len, block_size, head_dim, kv_dtype) -> int:
+    return int(_lib.pa_choose_partition(num_seqs, num_kv_heads, max_context_len, block_size, head_dim,
+                                        _DT[kv_dtype] if isinstance(kv_dtype, torch.dtype) else int(kv_dtype)))
+
+
+def pa_copy_blocks(k_cache, v_cache, src_dst_pairs, stream=None) -> None:
+    NB, Hkv, bs, D = k_cache.shape
+    n = src_dst_pairs.shape[0] if src_dst_pairs is not None else 0
+    rc = _lib.pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(src_dst_pairs) if n else None, n, NB, Hkv, D,
+                             bs, _dtype(k_cache), _stream(stream))
+    _check(rc, "pa_copy_blocks")
+
+
+def pa_read_device_errors(stream=None) -> int:
+    flags = ctypes.c_uint32(0)
+    _check(_lib.pa_read_device_errors(ctypes.byref(flags), _stream(stream)), "pa_read_device_errors")
+    return int(flags.value)
+
+
+def splitk_views(workspace: torch.Tensor, num_seqs, num_heads, head_dim, max_context_len, partition_size):
+    """(ml, acc) float32 views of a split-K workspace, as laid out by pa_decode_splitk:
+    ml [S, Hq, max_parts, 2], acc [S, Hq, max_parts, head_dim]."""
+    mp = -(-max_context_len // partition_size)
+    off = pa_splitk_acc_offset(num_seqs, num_heads, max_context_len, partition_size)
+    flat = workspace.view(torch.uint8)
+    ml = flat[: num_seqs * num_heads * mp * 8].view(torch.float32).view(num_seqs, num_heads, mp, 2)
+    acc = flat[off: off + num_seqs * num_heads * mp * head_dim * 4].view(torch.float32)
+    return ml, acc.view(num_seqs, num_heads, mp, head_dim)
+
+
+# -------------------------------------------------------------- host pool
+
+def _i32p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+class BlockPool:
+    """Host block pool (pa_pool_* calls): free list, reference counts and the
+    copy-on-write decision. Tables are numpy int32 rows owned by the caller."""
+
+    def __init__(self, num_blocks: int, block_size: int, policy: int = PA_POOL_LIFO, free_order=None):
+        self.block_size = block_size
+        self.num_blocks = num_blocks
+        order = None
+        if free_order is not None:
+            self._order = np.ascontiguousarray(np.asarray(free_order, dtype=np.int32))
+            order = _i32p(self._order)
+        h = _lib.pa_pool_create(num_blocks, block_size, policy, order)
+        if not h:
+            raise PagedAttentionError("pa_pool_create", -3)
+        self._h = ctypes.c_void_p(h)
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            _lib.pa_pool_destroy(h)
+            self._h = None
+
+    def num_free(self) -> int:
+        return int(_lib.pa_pool_num_free(self._h))
+
+    def ref_count(self, block: int) -> int:
+        rc = int(_lib.pa_pool_ref_count(self._h, int(block)))
+        if rc < 0:
+            raise PagedAttentionError("pa_pool_ref_count", rc)
+        return rc
+
+    def allocate(self) -> int:
+        b = ctypes.c_int32(-1)
+        _check(_lib.pa_pool_allocate(self._h, ctypes.byref(b)), "pa_pool_allocate")
+        return int(b.value)
+
+    def share(self, block: int) -> None:
+        _check(_lib.pa_pool_share(self._h, int(block)), "pa_pool_share")
+
+    def free(self, block: int) -> None:
+        _check(_lib.pa_pool_free(self._h, int(block)), "pa_pool_free")
+
+    def append(self, table: np.ndarray, num_tokens: int, n_new: int, want_slots: bool = True,
+               cow_capacity: int = 64) -> Tuple[int, Optional[np.ndarray], np.ndarray]:
+        """Appends n_new tokens to the sequence (table row, num_tokens).
+        Returns (new num_tokens, slots int32 [n_new] or None, cow pairs int64 [k, 2])."""
+        assert table.dtype == np.int32 and table.flags["C_CONTIGUOUS"]
+        nt = ctypes.c_int32(num_tokens)
+        slots = np.empty(n_new, np.int32) if want_slots else None
+        cow = np.empty((cow_capacity, 2), np.int64)
+        ncow = ctypes.c_int(0)
+        rc = _lib.pa_pool_append(self._h, _i32p(table), table.shape[0], ctypes.byref(nt), int(n_new),
+                                 _i32p(slots) if slots is not None else None,
+                                 cow.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), cow_capacity,
+                                 ctypes.byref(ncow))
+        _check(rc, "pa_pool_append")
+        return int(nt.value), slots, cow[: ncow.value].copy()
+
+    def fork(self, table: np.ndarray, num_tokens: int, dst: np.ndarray) -> None:
+        _check(_lib.pa_pool_fork(self._h, _i32p(table), int(num_tokens), _i32p(dst), dst.shape[0]), "pa_pool_fork")
+
+    def release(self, table: np.ndarray, num_tokens: int) -> None:
+        _check(_lib.pa_pool_release(self._h, _i32p(table), int(num_tokens)), "pa_pool_release")

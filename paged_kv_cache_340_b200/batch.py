@@ -1,0 +1,184 @@
+"""Host flow of one decode step, on the library's own block pool.
+
+An engine allocates blocks as sequences grow, writes each new token's K/V
+through its slot, copies shared blocks before a sequence writes into them,
+then runs decode. These helpers do that for the synthetic workloads: the pool
+(``BlockPool``, the C++ pa_pool_* calls) hands out blocks in the workload's
+seeded order and yields the block tables, slot mappings and copy-on-write
+pairs; the device calls go through the C ABI.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import (PA_POOL_FIFO, BlockPool, pa_choose_partition, pa_copy_blocks, pa_decode, pa_decode_splitk,
+               pa_reshape_and_cache, pa_splitk_reduce, pa_splitk_workspace_bytes)
+from .workloads import Spec
+
+
+@dataclass
+class DecodeBatch:
+    spec: Spec
+    num_blocks: int
+    k_cache: torch.Tensor       # device [NB, Hkv, bs, D]
+    v_cache: torch.Tensor
+    query: torch.Tensor         # device [S, Hq, D]
+    out: torch.Tensor           # device [S, Hq, D] of spec.out_dtype
+    block_tables: torch.Tensor  # device int32 [S, MB]
+    context_lens: torch.Tensor  # device int32 [S]
+    new_key: torch.Tensor       # device [T, Hkv, D], the tokens written this step
+    new_value: torch.Tensor
+    slot_mapping: torch.Tensor  # device int32 [T]
+    cow_pairs: torch.Tensor     # device int64 [n, 2] (n may be 0)
+    max_context_len: int
+    partition_size: int         # 0 = unpartitioned
+    workspace: Optional[torch.Tensor]
+    host_tables: np.ndarray
+    host_slots: np.ndarray
+    host_cow: np.ndarray
+    host_context_lens: np.ndarray
+
+
+def _blocks(n: int, bs: int) -> int:
+    return (n + bs - 1) // bs
+
+
+def build_decode_batch(spec: Spec, inputs: dict, device="cuda", partition_size: Optional[int] = None,
+                       pool_policy: int = PA_POOL_FIFO) -> DecodeBatch:
+    """Decode step of a non-sampling workload: every sequence already holds
+    context_lens - 1 tokens; its newest token is written through its slot,
+    then all sequences attend over context_lens tokens."""
+    bs = spec.block_size
+    ctx = inputs["context_lens"].numpy().astype(np.int32)
+    S = ctx.shape[0]
+    nb = int(inputs["num_blocks"])
+    mb = max(1, _blocks(int(ctx.max()), bs))
+    pool = BlockPool(nb, bs, pool_policy, free_order=inputs["free_order"].numpy())
+    tables = np.full((S, mb), -1, np.int32)
+    slots = np.empty(S, np.int32)
+    for s in range(S):
+        nt, _, cow = pool.append(tables[s], 0, int(ctx[s]) - 1, want_slots=False)
+        nt, sl, cow2 = pool.append(tables[s], nt, 1)
+        assert cow.size == 0 and cow2.size == 0
+        slots[s] = sl[0]
+    dev = torch.device(device)
+    max_ctx = int(ctx.max())
+    if partition_size is None:
+        partition_size = spec.partition_size or pa_choose_partition(S, spec.num_kv_heads, max_ctx, bs, spec.head_dim,
+                                                                    spec.torch_kv_dtype)
+    ws = None
+    if partition_size:
+        nbytes = pa_splitk_workspace_bytes(S, spec.num_heads, spec.head_dim, max_ctx, partition_size)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    return DecodeBatch(
+        spec=spec, num_blocks=nb,
+        k_cache=inputs["k_pool"].to(dev), v_cache=inputs["v_pool"].to(dev),
+        query=inputs["query"].to(dev),
+        out=torch.empty((S, spec.num_heads, spec.head_dim), dtype=spec.torch_out_dtype, device=dev),
+        block_tables=torch.from_numpy(tables).to(dev), context_lens=torch.from_numpy(ctx).to(dev),
+        new_key=inputs["new_key"].to(dev), new_value=inputs["new_value"].to(dev),
+        slot_mapping=torch.from_numpy(slots).to(dev),
+        cow_pairs=torch.empty((0, 2), dtype=torch.int64, device=dev),
+        max_context_len=max_ctx, partition_size=int(partition_size), workspace=ws,
+        host_tables=tables, host_slots=slots, host_cow=np.empty((0, 2), np.int64), host_context_lens=ctx)
+
+
+@dataclass
+class SamplingBatch(DecodeBatch):
+    prefix_key: torch.Tensor = None     # device [P * prefix_len, Hkv, D]
+    prefix_value: torch.Tensor = None
+    prefix_slots: torch.Tensor = None   # device int32 [P * prefix_len]
+    host_prefix_slots: np.ndarray = None
+
+
+def build_parallel_sampling_batch(spec: Spec, inputs: dict, device="cuda", partition_size: int = 0,
+                                  pool_policy: int = PA_POOL_FIFO) -> SamplingBatch:
+    """Parallel sampling: each prompt's prefix is written once, the prompt is
+    forked into `branches` sequences sharing its blocks, and every branch
+    appends its own tokens (the first write into the shared partial block
+    copies it). Branches are processed in (prompt, branch) order."""
+    bs = spec.block_size
+    P, B, L0 = spec.num_prompts, spec.branches, spec.prefix_len
+    div = inputs["divergent_lens"].numpy().astype(np.int32)
+    nb = int(inputs["num_blocks"])
+    mb = _blocks(L0 + int(div.max()), bs)
+    pool = BlockPool(nb, bs, pool_policy, free_order=inputs["free_order"].numpy())
+    S = P * B
+    tables = np.full((S, mb), -1, np.int32)
+    prefix_slots = np.empty(P * L0, np.int32)
+    for p in range(P):
+        root = p * B
+        _, sl, cow = pool.append(tables[root], 0, L0)
+        assert cow.size == 0
+        prefix_slots[p * L0:(p + 1) * L0] = sl
+        for b in range(1, B):
+            pool.fork(tables[root], L0, tables[root + b])
+    slots = np.empty(int(div.sum()), np.int32)
+    cows = []
+    ctx = np.empty(S, np.int32)
+    pos = 0
+    for p in range(P):
+        for b in range(B):
+            s = p * B + b
+            n = int(div[p, b])
+            nt, sl, cow = pool.append(tables[s], L0, n)
+            slots[pos:pos + n] = sl
+            pos += n
+            cows.append(cow)
+            ctx[s] = nt
+    cow_all = np.concatenate(cows).astype(np.int64) if cows else np.empty((0, 2), np.int64)
+    dev = torch.device(device)
+    NB, Hkv, D = nb, spec.num_kv_heads, spec.head_dim
+    dt = spec.torch_kv_dtype
+    max_ctx = int(ctx.max())
+    ws = None
+    if partition_size:
+        ws = torch.empty(pa_splitk_workspace_bytes(S, spec.num_heads, D, max_ctx, partition_size),
+                         dtype=torch.uint8, device=dev)
+    return SamplingBatch(
+        spec=spec, num_blocks=nb,
+        k_cache=torch.zeros((NB, Hkv, bs, D), dtype=dt, device=dev),
+        v_cache=torch.zeros((NB, Hkv, bs, D), dtype=dt, device=dev),
+        query=inputs["query"].to(dev),
+        out=torch.empty((S, spec.num_heads, D), dtype=spec.torch_out_dtype, device=dev),
+        block_tables=torch.from_numpy(tables).to(dev), context_lens=torch.from_numpy(ctx).to(dev),
+        new_key=inputs["divergent_key"].to(dev), new_value=inputs["divergent_value"].to(dev),
+        slot_mapping=torch.from_numpy(slots).to(dev), cow_pairs=torch.from_numpy(cow_all).to(dev),
+        max_context_len=max_ctx, partition_size=int(partition_size), workspace=ws,
+        host_tables=tables, host_slots=slots, host_cow=cow_all, host_context_lens=ctx,
+        prefix_key=inputs["prefix_key"].reshape(P * L0, Hkv, D).to(dev),
+        prefix_value=inputs["prefix_value"].reshape(P * L0, Hkv, D).to(dev),
+        prefix_slots=torch.from_numpy(prefix_slots).to(dev), host_prefix_slots=prefix_slots)
+
+
+def write_prefix(batch: SamplingBatch, stream=None) -> None:
+    """Writes every prompt's prefix into the pool (set-up, once)."""
+    pa_reshape_and_cache(batch.prefix_key, batch.prefix_value, batch.k_cache, batch.v_cache, batch.prefix_slots,
+                         stream=stream)
+
+
+def run_step(batch: DecodeBatch, stream=None) -> None:
+    """One pass of the hot path: copy-on-write block copies (if any), the slot
+    write of this step's tokens, then decode (split-K + reduce when the batch
+    has a partition size)."""
+    if batch.cow_pairs.shape[0]:
+        pa_copy_blocks(batch.k_cache, batch.v_cache, batch.cow_pairs, stream=stream)
+    pa_reshape_and_cache(batch.new_key, batch.new_value, batch.k_cache, batch.v_cache, batch.slot_mapping,
+                         stream=stream)
+    run_decode(batch, stream)
+
+
+def run_decode(batch: DecodeBatch, stream=None) -> None:
+    spec = batch.spec
+    if batch.partition_size:
+        pa_decode_splitk(batch.workspace, batch.query, batch.k_cache, batch.v_cache, batch.block_tables,
+                         batch.context_lens, spec.scale, batch.max_context_len, batch.partition_size, stream=stream)
+        pa_splitk_reduce(batch.out, batch.workspace, batch.context_lens, batch.max_context_len,
+                         batch.partition_size, stream=stream)
+    else:
+        pa_decode(batch.out, batch.query, batch.k_cache, batch.v_cache, batch.block_tables, batch.context_lens,
+                  spec.scale, stream=stream)

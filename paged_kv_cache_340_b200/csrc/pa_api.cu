@@ -1,0 +1,335 @@
+// C-ABI entry points of the device operations: host-side argument checks,
+// dispatch, the device error word and the split-K workspace layout.
+#include <atomic>
+#include <climits>
+#include <cmath>
+
+#include "pa_common.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+__device__ unsigned int g_device_errors = 0;
+
+static constexpr int kMaxDevices = 64;
+
+cudaError_t device_error_word(unsigned int **word) {
+    static std::atomic<unsigned int *> cache[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    unsigned int *w = cache[dev].load(std::memory_order_acquire);
+    if (w == nullptr) {
+        void *addr = nullptr;
+        e = cudaGetSymbolAddress(&addr, g_device_errors);
+        if (e != cudaSuccess) return e;
+        w = static_cast<unsigned int *>(addr);
+        cache[dev].store(w, std::memory_order_release);
+    }
+    *word = w;
+    return cudaSuccess;
+}
+
+int sm_count() {
+    static std::atomic<int> cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
+cudaError_t ensure_smem_attr(const void *func, int bytes, unsigned int *done_mask) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned int bit = 1u << (dev & 31);
+    std::atomic_ref<unsigned int> mask(*done_mask);
+    if (dev < 32 && (mask.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    if (dev < 32) mask.fetch_or(bit, std::memory_order_acq_rel);
+    return cudaSuccess;
+}
+
+static int elt_bytes(pa_dtype dt) {
+    switch (dt) {
+        case PA_F32: return 4;
+        case PA_F16: return 2;
+        case PA_BF16: return 2;
+    }
+    return 0;
+}
+
+static bool aligned(const void *p, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+// Checks shared by the decode entry points.
+static int check_decode_args(const void *query, const void *k_cache, const void *v_cache,
+                             const int32_t *block_tables, int max_blocks_per_seq,
+                             const int32_t *context_lens, int num_seqs, int num_heads,
+                             int num_kv_heads, int head_dim, float scale, int block_size,
+                             int num_blocks, pa_dtype kv_dtype) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks < 0 ||
+        max_blocks_per_seq < 0 || num_seqs > 65535 || num_kv_heads > 65535 || !std::isfinite(scale))
+        return PA_ERR_SHAPE;
+    if (elt_bytes(kv_dtype) == 0) return PA_ERR_DTYPE;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_HEAD_DIM;
+    if (block_size != 16 && block_size != 32) return PA_ERR_BLOCK_SIZE;
+    if (num_heads % num_kv_heads != 0) return PA_ERR_HEADS;
+    const int group = num_heads / num_kv_heads;
+    if (group != 1 && group != 2 && group != 4 && group != 8) return PA_ERR_HEADS;
+    if (max_blocks_per_seq > INT_MAX / block_size) return PA_ERR_SHAPE;
+    if (num_seqs == 0) return PA_OK;
+    if (!query || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_NULL;
+    if (!aligned(query, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4))
+        return PA_ERR_ALIGN;
+    return PA_OK;
+}
+
+static int max_parts_of(int max_context_len, int partition_size) {
+    return (max_context_len + partition_size - 1) / partition_size;
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static size_t ml_bytes(int num_seqs, int num_heads, int max_parts) {
+    return (size_t)num_seqs * num_heads * max_parts * 2 * sizeof(float);
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+const char *pa_status_string(int status) {
+    switch (status) {
+        case PA_OK: return "ok";
+        case PA_ERR_NULL: return "a required pointer is NULL";
+        case PA_ERR_DTYPE: return "unsupported element or output type";
+        case PA_ERR_SHAPE: return "a size is negative, too large or inconsistent";
+        case PA_ERR_HEADS: return "num_heads must be num_kv_heads times 1, 2, 4 or 8";
+        case PA_ERR_HEAD_DIM: return "head_dim must be 64 or 128";
+        case PA_ERR_BLOCK_SIZE: return "block_size must be 16 or 32";
+        case PA_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
+        case PA_ERR_PARTITION: return "partition_size must be a positive multiple of block_size";
+        case PA_ERR_WORKSPACE: return "workspace is missing or smaller than pa_splitk_workspace_bytes()";
+        case PA_ERR_CUDA: return "a CUDA call or kernel launch failed";
+        case PA_ERR_POOL_EXHAUSTED: return "block pool has no free block";
+        case PA_ERR_POOL_STATE: return "block id out of range or block already free";
+        case PA_ERR_CAPACITY: return "table row or output array too small";
+    }
+    return "unknown status";
+}
+
+int pa_read_device_errors(uint32_t *flags, cudaStream_t stream) {
+    if (!flags) return PA_ERR_NULL;
+    unsigned int *word = nullptr;
+    if (device_error_word(&word) != cudaSuccess) return PA_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return PA_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpy(&v, word, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return PA_ERR_CUDA;
+    if (cudaMemset(word, 0, sizeof(v)) != cudaSuccess) return PA_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
+    *flags = v;
+    return PA_OK;
+}
+
+int pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
+                         const int32_t *slot_mapping, int num_tokens, int num_blocks,
+                         int num_kv_heads, int head_dim, int block_size, pa_dtype kv_dtype,
+                         cudaStream_t stream) {
+    if (num_tokens < 0 || num_blocks < 0 || num_kv_heads <= 0) return PA_ERR_SHAPE;
+    const int eb = elt_bytes(kv_dtype);
+    if (eb == 0) return PA_ERR_DTYPE;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_HEAD_DIM;
+    if (block_size != 16 && block_size != 32) return PA_ERR_BLOCK_SIZE;
+    if ((long long)num_blocks * block_size > INT_MAX) return PA_ERR_SHAPE;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_NULL;
+    if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(slot_mapping, 4))
+        return PA_ERR_ALIGN;
+    unsigned int *err = nullptr;
+    if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    cudaError_t e = launch_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, num_tokens,
+                                             num_blocks, num_kv_heads, head_dim * eb, block_size,
+                                             err, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_decode(void *out, const void *query, const void *k_cache, const void *v_cache,
+              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+              int num_seqs, int num_heads, int num_kv_heads, int head_dim, float scale,
+              int block_size, int num_blocks, pa_dtype kv_dtype, pa_dtype out_dtype,
+              cudaStream_t stream) {
+    int rc = check_decode_args(query, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                               context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale,
+                               block_size, num_blocks, kv_dtype);
+    if (rc != PA_OK) return rc;
+    if (out_dtype != kv_dtype && out_dtype != PA_F32) return PA_ERR_DTYPE;
+    if (num_seqs == 0) return PA_OK;
+    if (!out) return PA_ERR_NULL;
+    if (!aligned(out, 16)) return PA_ERR_ALIGN;
+    unsigned int *err = nullptr;
+    if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    DecodeParams p{};
+    p.out = out;
+    p.query = query;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.num_blocks = num_blocks;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.partition_size = 0;
+    p.max_parts = 1;
+    p.max_context_len = INT_MAX;
+    p.out_dtype = out_dtype;
+    p.err = err;
+    cudaError_t e = launch_decode(p, kv_dtype, head_dim, block_size, num_heads / num_kv_heads, 1,
+                                  num_kv_heads, num_seqs, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+size_t pa_splitk_acc_offset(int num_seqs, int num_heads, int max_context_len, int partition_size) {
+    if (num_seqs < 0 || num_heads <= 0 || max_context_len < 0 || partition_size <= 0) return 0;
+    const int mp = max_parts_of(max_context_len, partition_size);
+    return align_up(ml_bytes(num_seqs, num_heads, mp), 256);
+}
+
+size_t pa_splitk_workspace_bytes(int num_seqs, int num_heads, int head_dim, int max_context_len,
+                                 int partition_size) {
+    if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
+        partition_size <= 0)
+        return 0;
+    const int mp = max_parts_of(max_context_len, partition_size);
+    return pa_splitk_acc_offset(num_seqs, num_heads, max_context_len, partition_size) +
+           (size_t)num_seqs * num_heads * mp * head_dim * sizeof(float);
+}
+
+int pa_decode_splitk(void *workspace, size_t workspace_bytes, const void *query,
+                     const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                     int max_blocks_per_seq, const int32_t *context_lens, int num_seqs,
+                     int num_heads, int num_kv_heads, int head_dim, float scale, int block_size,
+                     int num_blocks, int max_context_len, int partition_size, pa_dtype kv_dtype,
+                     cudaStream_t stream) {
+    int rc = check_decode_args(query, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                               context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale,
+                               block_size, num_blocks, kv_dtype);
+    if (rc != PA_OK) return rc;
+    if (max_context_len < 0) return PA_ERR_SHAPE;
+    if (partition_size <= 0 || partition_size % block_size != 0) return PA_ERR_PARTITION;
+    if (num_seqs == 0 || max_context_len == 0) return PA_OK;
+    const size_t need = pa_splitk_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len,
+                                                  partition_size);
+    if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return PA_ERR_ALIGN;
+    unsigned int *err = nullptr;
+    if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    const int mp = max_parts_of(max_context_len, partition_size);
+    DecodeParams p{};
+    p.ws_ml = static_cast<float *>(workspace);
+    p.ws_acc = reinterpret_cast<float *>(
+        static_cast<unsigned char *>(workspace) +
+        pa_splitk_acc_offset(num_seqs, num_heads, max_context_len, partition_size));
+    p.query = query;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.num_blocks = num_blocks;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.partition_size = partition_size;
+    p.max_parts = mp;
+    p.max_context_len = max_context_len;
+    p.out_dtype = PA_F32;
+    p.err = err;
+    cudaError_t e = launch_decode(p, kv_dtype, head_dim, block_size, num_heads / num_kv_heads, mp,
+                                  num_kv_heads, num_seqs, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_splitk_reduce(void *out, const void *workspace, size_t workspace_bytes,
+                     const int32_t *context_lens, int num_seqs, int num_heads, int head_dim,
+                     int max_context_len, int partition_size, pa_dtype out_dtype,
+                     cudaStream_t stream) {
+    if (num_seqs < 0 || num_heads <= 0 || max_context_len < 0 || num_seqs > 65535 ||
+        num_heads > INT_MAX / 2)
+        return PA_ERR_SHAPE;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_HEAD_DIM;
+    if (partition_size <= 0) return PA_ERR_PARTITION;
+    if (elt_bytes(out_dtype) == 0) return PA_ERR_DTYPE;
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !context_lens) return PA_ERR_NULL;
+    if (!aligned(out, 16) || !aligned(context_lens, 4)) return PA_ERR_ALIGN;
+    const int mp = max_parts_of(max_context_len, partition_size);
+    if ((size_t)mp * sizeof(float) > 200 * 1024) return PA_ERR_SHAPE;
+    const size_t need = pa_splitk_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len,
+                                                  partition_size);
+    if (mp > 0 && (!workspace || workspace_bytes < need)) return PA_ERR_WORKSPACE;
+    const float *ml = static_cast<const float *>(workspace);
+    const float *acc = workspace == nullptr
+                           ? nullptr
+                           : reinterpret_cast<const float *>(
+                                 static_cast<const unsigned char *>(workspace) +
+                                 pa_splitk_acc_offset(num_seqs, num_heads, max_context_len,
+                                                      partition_size));
+    cudaError_t e = launch_splitk_reduce(out, ml, acc, context_lens, num_seqs, num_heads, head_dim,
+                                         partition_size, mp > 0 ? mp : 1, max_context_len,
+                                         out_dtype, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_choose_partition(int num_seqs, int num_kv_heads, int max_context_len, int block_size,
+                        int head_dim, pa_dtype kv_dtype) {
+    (void)head_dim;
+    (void)kv_dtype;
+    if (num_seqs <= 0 || num_kv_heads <= 0 || max_context_len <= 0 || block_size <= 0) return 0;
+    const long long items = (long long)num_seqs * num_kv_heads;
+    const long long target = 4LL * sm_count();  // work items that keep every SM busy
+    if (items >= target) return 0;
+    // Enough partitions of the longest sequence to reach the target, in
+    // powers of two of at least 512 tokens.
+    long long want = (long long)max_context_len * items / target;
+    int P = 512;
+    while (P < want && P < (1 << 20)) P <<= 1;
+    P = (P + block_size - 1) / block_size * block_size;
+    return P >= max_context_len ? 0 : P;
+}
+
+int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pairs, int num_pairs,
+                   int num_blocks, int num_kv_heads, int head_dim, int block_size,
+                   pa_dtype kv_dtype, cudaStream_t stream) {
+    if (num_pairs < 0 || num_blocks < 0 || num_kv_heads <= 0) return PA_ERR_SHAPE;
+    const int eb = elt_bytes(kv_dtype);
+    if (eb == 0) return PA_ERR_DTYPE;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_HEAD_DIM;
+    if (block_size != 16 && block_size != 32) return PA_ERR_BLOCK_SIZE;
+    if (num_pairs == 0) return PA_OK;
+    if (!k_cache || !v_cache || !src_dst_pairs) return PA_ERR_NULL;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(src_dst_pairs, 8))
+        return PA_ERR_ALIGN;
+    unsigned int *err = nullptr;
+    if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    const size_t block_bytes = (size_t)num_kv_heads * block_size * head_dim * eb;
+    cudaError_t e = launch_copy_blocks(k_cache, v_cache, src_dst_pairs, num_pairs, num_blocks,
+                                       block_bytes, err, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // extern "C"

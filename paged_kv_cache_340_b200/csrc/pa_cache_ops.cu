@@ -1,0 +1,98 @@
+// Cache-side kernels: the slot write of new tokens and the copy-on-write
+// block copy. Both are bit copies moved in 16-byte vectors; HBM-bound.
+#include "pa_common.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+// Slot write ([P3 "Ascend C ... PagedAttention融合算子", §3.1 and §4.2:
+// block = slot / block_size, offset = slot % block_size]; [P4 "PagedAttention
+// 实现细节", §3.4: each new token's K/V goes into its block).
+// One thread moves one 16-byte vector of one (token, kv head) row of both key
+// and value; consecutive threads cover consecutive vectors of the source, so
+// loads and stores are coalesced per row.
+__global__ void __launch_bounds__(256)
+    reshape_and_cache_kernel(const uint4 *__restrict__ key, const uint4 *__restrict__ value,
+                             uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
+                             const int32_t *__restrict__ slot_mapping, int num_tokens,
+                             int num_blocks, int num_kv_heads, int vecs_per_row, int block_size,
+                             unsigned int *err) {
+    const long long per_token = (long long)num_kv_heads * vecs_per_row;
+    const long long total = per_token * num_tokens;
+    const long long slots = (long long)num_blocks * block_size;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int token = (int)(i / per_token);
+        const int rem = (int)(i - (long long)token * per_token);
+        const int h = rem / vecs_per_row;
+        const int v = rem - h * vecs_per_row;
+        const int slot = __ldg(slot_mapping + token);
+        if (slot < 0) continue;
+        if (slot >= slots) {
+            if (h == 0 && v == 0) record_error(err, PA_DEVERR_SLOT);
+            continue;
+        }
+        const int block = slot / block_size;
+        const int offset = slot - block * block_size;
+        const size_t dst = (((size_t)block * num_kv_heads + h) * block_size + offset) * vecs_per_row + v;
+        k_cache[dst] = __ldg(key + i);
+        v_cache[dst] = __ldg(value + i);
+    }
+}
+
+// Copy-on-write block copy ([P4 "PagedAttention 实现细节", §3.3]): grid.x walks
+// the pairs, grid.y picks K (0) or V (1), grid.z splits a block into chunks.
+__global__ void __launch_bounds__(256)
+    copy_blocks_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
+                       const int64_t *__restrict__ pairs, int num_blocks, long long vecs_per_block,
+                       unsigned int *err) {
+    const int64_t src = __ldg(pairs + 2 * blockIdx.x);
+    const int64_t dst = __ldg(pairs + 2 * blockIdx.x + 1);
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) record_error(err, PA_DEVERR_PAIR);
+        return;
+    }
+    uint4 *pool = blockIdx.y == 0 ? k_cache : v_cache;
+    const uint4 *s = pool + src * vecs_per_block;
+    uint4 *d = pool + dst * vecs_per_block;
+    const long long chunk = (vecs_per_block + gridDim.z - 1) / gridDim.z;
+    const long long begin = blockIdx.z * chunk;
+    const long long end = min(begin + chunk, vecs_per_block);
+    for (long long i = begin + threadIdx.x; i < end; i += blockDim.x) d[i] = s[i];
+}
+
+cudaError_t launch_reshape_and_cache(const void *key, const void *value, void *k_cache,
+                                     void *v_cache, const int32_t *slot_mapping, int num_tokens,
+                                     int num_blocks, int num_kv_heads, int row_bytes,
+                                     int block_size, unsigned int *err, cudaStream_t stream) {
+    if (num_tokens == 0) return cudaSuccess;
+    const int vecs_per_row = row_bytes / 16;
+    const long long total = (long long)num_tokens * num_kv_heads * vecs_per_row;
+    const int threads = 256;
+    long long blocks = (total + threads - 1) / threads;
+    const long long cap = (long long)sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    reshape_and_cache_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+        static_cast<const uint4 *>(key), static_cast<const uint4 *>(value),
+        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), slot_mapping, num_tokens,
+        num_blocks, num_kv_heads, vecs_per_row, block_size, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *pairs, int num_pairs,
+                               int num_blocks, size_t block_bytes, unsigned int *err,
+                               cudaStream_t stream) {
+    if (num_pairs == 0) return cudaSuccess;
+    const long long vecs = (long long)(block_bytes / 16);
+    // about 16 KiB per CTA
+    long long chunks = (vecs + 1023) / 1024;
+    if (chunks < 1) chunks = 1;
+    if (chunks > 65535) chunks = 65535;
+    dim3 grid((unsigned)num_pairs, 2, (unsigned)chunks);
+    copy_blocks_kernel<<<grid, 256, 0, stream>>>(static_cast<uint4 *>(k_cache),
+                                                 static_cast<uint4 *>(v_cache), pairs, num_blocks,
+                                                 vecs, err);
+    return cudaGetLastError();
+}
+
+}  // namespace pa

@@ -1,0 +1,60 @@
+// Internal interfaces between the C-ABI layer (pa_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+struct DecodeParams {
+    void *out;          // unpartitioned: [num_seqs, num_heads, head_dim] of out_dtype
+    float *ws_ml;       // split-K: [num_seqs, num_heads, max_parts, 2] (m, l)
+    float *ws_acc;      // split-K: [num_seqs, num_heads, max_parts, head_dim]
+    const void *query;  // [num_seqs, num_heads, head_dim]
+    const void *k_cache;
+    const void *v_cache;
+    const int32_t *block_tables;
+    const int32_t *context_lens;
+    int max_blocks_per_seq;
+    int num_heads;
+    int num_kv_heads;
+    int num_blocks;
+    float scale_log2;    // scale * log2(e)
+    int partition_size;  // 0: one CTA covers the whole sequence
+    int max_parts;
+    int max_context_len;
+    pa_dtype out_dtype;
+    unsigned int *err;   // device error word
+};
+
+cudaError_t launch_decode(const DecodeParams &p, pa_dtype kv_dtype, int head_dim, int block_size,
+                          int group, int grid_x, int num_kv_heads, int num_seqs,
+                          cudaStream_t stream);
+
+cudaError_t launch_splitk_reduce(void *out, const float *ws_ml, const float *ws_acc,
+                                 const int32_t *context_lens, int num_seqs, int num_heads,
+                                 int head_dim, int partition_size, int max_parts,
+                                 int max_context_len, pa_dtype out_dtype, cudaStream_t stream);
+
+cudaError_t launch_reshape_and_cache(const void *key, const void *value, void *k_cache,
+                                     void *v_cache, const int32_t *slot_mapping, int num_tokens,
+                                     int num_blocks, int num_kv_heads, int row_bytes,
+                                     int block_size, unsigned int *err, cudaStream_t stream);
+
+cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *pairs, int num_pairs,
+                               int num_blocks, size_t block_bytes, unsigned int *err,
+                               cudaStream_t stream);
+
+// Device address of the current device's error word (cached per device).
+cudaError_t device_error_word(unsigned int **word);
+
+// Number of SMs of the current device.
+int sm_count();
+
+// Sets the dynamic shared memory limit of `func` once per device.
+cudaError_t ensure_smem_attr(const void *func, int bytes, unsigned int *done_mask);
+
+}  // namespace pa

@@ -1,0 +1,179 @@
+"""Host-side checks that need no GPU: the shared library loads and exports
+every function include/pa.h declares; host argument checks return their
+status codes before touching the device; the library's C++ block pool makes
+exactly the decisions of the oracle's pool."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def pa():
+    from paged_kv_cache_340_b200 import _build
+    _build.build()
+    import paged_kv_cache_340_b200 as pa
+    return pa
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[a-z_ ]*?[\w\s\*]+?\b(pa_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_function(pa):
+    declared = _declared_functions()
+    assert len(declared) >= 20
+    lib = ctypes.CDLL(pa.LIB_PATH)
+    missing = [n for n in declared if not hasattr(lib, n)]
+    assert not missing, missing
+    assert sorted(pa.EXPORTED) == declared
+
+
+def test_status_strings(pa):
+    for code in range(0, -14, -1):
+        s = pa.status_string(code)
+        assert s and s != "unknown status"
+    assert pa.status_string(-99) == "unknown status"
+
+
+def test_workspace_layout(pa):
+    S, H, D, L, P = 3, 8, 128, 1000, 256
+    mp = 4
+    off = pa.pa_splitk_acc_offset(S, H, L, P)
+    assert off >= S * H * mp * 2 * 4 and off % 256 == 0
+    assert pa.pa_splitk_workspace_bytes(S, H, D, L, P) == off + S * H * mp * D * 4
+
+
+def test_choose_partition(pa):
+    import torch
+    # many (seq, kv head) items: no split
+    assert pa.pa_choose_partition(256, 8, 4096, 16, 128, torch.bfloat16) == 0
+    # few long sequences: split, multiple of the block size, shorter than the context
+    P = pa.pa_choose_partition(8, 8, 131072, 32, 128, torch.bfloat16)
+    assert P > 0 and P % 32 == 0 and P < 131072
+
+
+A16 = 1 << 20  # a fake 16-byte aligned address; never dereferenced by these calls
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=96), -5),
+    (dict(block_size=8), -6),
+    (dict(num_heads=12, num_kv_heads=8), -4),
+    (dict(num_heads=48, num_kv_heads=3), -4),
+    (dict(kv_dtype=7), -2),
+    (dict(out_dtype=1, kv_dtype=2), -2),
+    (dict(num_seqs=-1), -3),
+    (dict(query=A16 + 8), -7),
+    (dict(k_cache=0), -1),
+])
+def test_decode_host_checks(pa, kw, code):
+    args = dict(out=A16, query=A16, k_cache=A16, v_cache=A16, block_tables=A16, max_blocks=4, context_lens=A16,
+                num_seqs=2, num_heads=8, num_kv_heads=8, head_dim=128, scale=0.1, block_size=16, num_blocks=8,
+                kv_dtype=1, out_dtype=1)
+    args.update(kw)
+    rc = pa._lib.pa_decode(args["out"], args["query"], args["k_cache"], args["v_cache"], args["block_tables"],
+                           args["max_blocks"], args["context_lens"], args["num_seqs"], args["num_heads"],
+                           args["num_kv_heads"], args["head_dim"], args["scale"], args["block_size"],
+                           args["num_blocks"], args["kv_dtype"], args["out_dtype"], None)
+    assert rc == code
+
+
+def test_empty_batches_are_no_ops(pa):
+    assert pa._lib.pa_decode(None, None, None, None, None, 0, None, 0, 8, 8, 128, 0.1, 16, 0, 1, 1, None) == 0
+    assert pa._lib.pa_reshape_and_cache(None, None, None, None, None, 0, 4, 8, 128, 16, 1, None) == 0
+    assert pa._lib.pa_copy_blocks(None, None, None, 0, 4, 8, 128, 16, 1, None) == 0
+
+
+def test_splitk_host_checks(pa):
+    f = pa._lib.pa_decode_splitk
+    base = [A16, 1 << 30, A16, A16, A16, A16, 4, A16, 2, 8, 8, 128, 0.1, 16, 8, 64]
+    assert f(*(base + [24, 1, None])) == -8       # partition not a multiple of the block size
+    assert f(*(base + [0, 1, None])) == -8
+    small = list(base)
+    small[1] = 16
+    assert f(*(small + [32, 1, None])) == -9      # workspace too small
+    nows = list(base)
+    nows[0] = None
+    assert f(*(nows + [32, 1, None])) == -9
+
+
+# ------------------------------------------------------ pool vs oracle pool
+
+def _same_pool_state(pool, opool):
+    assert pool.num_free() == opool.num_free()
+    for b in range(opool.num_blocks):
+        assert pool.ref_count(b) == opool.ref_counts[b]
+
+
+@pytest.mark.parametrize("policy", ["fifo", "lifo"])
+def test_pool_matches_oracle_random_ops(pa, policy):
+    from oracle.block_pool import BlockPool as OPool, Sequence, append_tokens, fork, release
+    rng = np.random.default_rng(5 if policy == "fifo" else 6)
+    NB, bs, MB = 96, 16, 24
+    order = rng.permutation(NB)
+    pol = pa.PA_POOL_FIFO if policy == "fifo" else pa.PA_POOL_LIFO
+    pool = pa.BlockPool(NB, bs, pol, free_order=order)
+    opool = OPool(NB, bs, policy=policy, free_order=order.tolist())
+    seqs = []  # (table, num_tokens, oracle Sequence)
+    for step in range(400):
+        op = rng.integers(0, 10)
+        if op < 5 or not seqs:
+            if op < 5 and seqs:
+                i = int(rng.integers(len(seqs)))
+            else:
+                seqs.append([np.full(MB, -1, np.int32), 0, Sequence()])
+                i = len(seqs) - 1
+            tab, nt, oseq = seqs[i]
+            n = int(rng.integers(1, 40))
+            if opool.num_free() < n // bs + 2 or nt + n > MB * bs:
+                continue
+            nt2, slots, cow = pool.append(tab, nt, n)
+            oslots, ocow = append_tokens(opool, oseq, n)
+            assert nt2 == oseq.num_tokens
+            assert slots.tolist() == oslots
+            assert [tuple(x) for x in cow.tolist()] == ocow
+            assert tab[: len(oseq.block_table)].tolist() == oseq.block_table
+            seqs[i][1] = nt2
+        elif op < 8:
+            i = int(rng.integers(len(seqs)))
+            tab, nt, oseq = seqs[i]
+            dst = np.full(MB, -1, np.int32)
+            pool.fork(tab, nt, dst)
+            seqs.append([dst, nt, fork(opool, oseq)])
+        else:
+            i = int(rng.integers(len(seqs)))
+            tab, nt, oseq = seqs.pop(i)
+            pool.release(tab, nt)
+            release(opool, oseq)
+        _same_pool_state(pool, opool)
+
+
+def test_pool_errors(pa):
+    pool = pa.BlockPool(2, 4, pa.PA_POOL_FIFO)
+    tab = np.full(4, -1, np.int32)
+    nt, _, _ = pool.append(tab, 0, 8)
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pool.append(tab, nt, 1)
+    assert e.value.status == -11
+    with pytest.raises(pa.PagedAttentionError):
+        pool.free(5)
+    with pytest.raises(pa.PagedAttentionError):
+        pa.BlockPool(3, 4, pa.PA_POOL_FIFO, free_order=[0, 0, 1])
+    small = np.full(1, -1, np.int32)
+    pool2 = pa.BlockPool(4, 4, pa.PA_POOL_FIFO)
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pool2.append(small, 0, 5)
+    assert e.value.status == -13
