@@ -44,7 +44,9 @@ struct DecodeShape {
     static constexpr int kVec = 16 / kElt;             // elements per 16-byte lane vector
     static constexpr int kLpt = D / kVec;              // lanes per token row
     static constexpr int kRows = 32 / kLpt;            // token rows per warp instruction
-    static constexpr int kTpg = BS / kRows;            // tokens of one block per row group
+    static constexpr int kTS = 16;                     // tokens per pipeline stage
+    static constexpr int kSubs = BS / kTS;             // stages per physical block
+    static constexpr int kTpg = kTS / kRows;           // tokens of one stage per row group
     static constexpr int kTc = (G * kTpg <= 32) ? kTpg : (32 / G);  // tokens per softmax chunk
     static constexpr int kChunks = kTpg / kTc;
     static constexpr int kNv = G * kTc;                // scores per lane before the butterfly
@@ -53,19 +55,25 @@ struct DecodeShape {
     static constexpr int kLanesPerG = kLpt / G;        // lanes whose scores belong to one head
     static constexpr int kConsumerWarps = 4;
     static constexpr int kThreads = (kConsumerWarps + 1) * 32;
-    static constexpr int kTileBytes = BS * D * kElt;   // one (block, kv head) K or V tile
+    static constexpr int kTileBytes = kTS * D * kElt;  // 16 token rows of one kv head, K or V
     static constexpr int kStageBytes = 2 * kTileBytes;
-    static constexpr int kStages = kStageBytes <= 8192 ? 8 : (kStageBytes <= 16384 ? 6 : 5);
+    // Stage k is consumed by warp k % 4 and lives in buffer k % 8, so the
+    // previous use of a buffer always belongs to the same warp: a parity
+    // wait can never see a phase two behind.
+    static constexpr int kStages = 8;
     static constexpr int kRowGroups = kConsumerWarps * kRows;
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kMergeBytes = kRowGroups * G * (D + 2) * 4;
     static constexpr int kDataBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
     static constexpr int kSmemBytes = 128 + kDataBytes + kStages * 16 + kStages * 4;
 
+    static_assert(kStages % kConsumerWarps == 0, "buffer reuse must stay within one warp");
+    static_assert(BS % kTS == 0, "block size is a multiple of the stage");
     static_assert(kLpt >= 1 && kLpt <= 32 && (32 % kLpt) == 0, "row width");
-    static_assert(BS % kRows == 0 && kTpg % kTc == 0, "block split");
+    static_assert(kTS % kRows == 0 && kTpg % kTc == 0, "stage split");
     static_assert(G <= kLpt, "a lane's kept scores must belong to one query head");
     static_assert(kNvl <= kTc, "kept scores within one head");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
 // Butterfly over the lanes of a token row (xor masks MK, MK/2, .., 1): while a
@@ -124,7 +132,8 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads)
         if (t_begin >= ctx) return;  // empty partition: nothing written
         t_end = min(t_begin + p.partition_size, ctx);
     }
-    const int nblk = (t_end - t_begin + BS - 1) / BS;
+    const int nblk = (t_end - t_begin + BS - 1) / BS;           // table entries read
+    const int nstage = (t_end - t_begin + S::kTS - 1) / S::kTS;  // 16-token stages
     const size_t head0 = (size_t)s * p.num_heads + (size_t)kvh * G;  // first query head row
     if (nblk == 0) {  // unsplit, empty context: zeros
         for (int i = threadIdx.x; i < G * D; i += blockDim.x)
@@ -162,28 +171,33 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads)
             for (int j = 0; j < n; ++j) {
                 const int b = __shfl_sync(0xffffffffu, ids, j);
                 const bool v = __shfl_sync(0xffffffffu, valid ? 1 : 0, j) != 0;
-                if (lane == 0) {
-                    const int k = base + j;
-                    const int buf = k % S::kStages;
-                    if (k >= S::kStages && !mbar_wait(empty + buf, ((k / S::kStages) - 1) & 1)) {
-                        ok = false;
-                        record_error(p.err, PA_DEVERR_TIMEOUT);
-                    } else {
-                        if (v) {
-                            bad[buf] = 0;
-                            unsigned char *dst = ring + (size_t)buf * S::kStageBytes;
-                            mbar_arrive_expect_tx(full + buf, S::kStageBytes);
-                            bulk_load(dst, kc + (size_t)b * block_elems, S::kTileBytes, full + buf, pol);
-                            bulk_load(dst + S::kTileBytes, vc + (size_t)b * block_elems, S::kTileBytes,
-                                      full + buf, pol);
+#pragma unroll
+                for (int h = 0; h < S::kSubs; ++h) {
+                    const int k = (base + j) * S::kSubs + h;  // stage
+                    if (k >= nstage) break;
+                    if (lane == 0) {
+                        const int buf = k % S::kStages;
+                        if (k >= S::kStages && !mbar_wait(empty + buf, ((k / S::kStages) - 1) & 1)) {
+                            ok = false;
+                            record_error(p.err, PA_DEVERR_TIMEOUT);
                         } else {
-                            bad[buf] = 1;
-                            mbar_arrive(full + buf);
+                            if (v) {
+                                bad[buf] = 0;
+                                unsigned char *dst = ring + (size_t)buf * S::kStageBytes;
+                                const size_t src = (size_t)b * block_elems + (size_t)h * S::kTS * D;
+                                mbar_arrive_expect_tx(full + buf, S::kStageBytes);
+                                bulk_load(dst, kc + src, S::kTileBytes, full + buf, pol);
+                                bulk_load(dst + S::kTileBytes, vc + src, S::kTileBytes, full + buf, pol);
+                            } else {
+                                bad[buf] = 1;
+                                mbar_arrive(full + buf);
+                            }
+                            ++issued;
                         }
-                        ++issued;
                     }
+                    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                    if (!ok) break;
                 }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
             }
         }
@@ -223,7 +237,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads)
     }
     float l_lane = 0.f;
 
-    for (int k = warp; k < nblk; k += S::kConsumerWarps) {
+    for (int k = warp; k < nstage; k += S::kConsumerWarps) {
         const int buf = k % S::kStages;
         const bool got = mbar_wait(full + buf, (k / S::kStages) & 1);
         if (!__all_sync(0xffffffffu, got)) {
@@ -231,7 +245,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads)
             break;
         }
         if (!bad[buf]) {
-            const int nvalid = min(BS, t_end - (t_begin + k * BS));
+            const int nvalid = min(S::kTS, t_end - (t_begin + k * S::kTS));
             const unsigned char *Ks = ring + (size_t)buf * S::kStageBytes;
             const unsigned char *Vs = Ks + S::kTileBytes;
 #pragma unroll
