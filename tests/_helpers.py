@@ -19,11 +19,10 @@ def f64(t: torch.Tensor) -> np.ndarray:
 
 
 def raw(t: torch.Tensor) -> np.ndarray:
-    """Byte-exact numpy view of a CPU tensor (bf16 as int16)."""
+    """Bit-exact integer numpy view of a tensor's elements (shares memory for
+    a contiguous CPU tensor, so in-place oracle writes land in the tensor)."""
     t = t.detach().to("cpu").contiguous()
-    if t.dtype == torch.bfloat16:
-        return t.view(torch.int16).numpy()
-    return t.numpy()
+    return t.view({8: torch.int64, 4: torch.int32, 2: torch.int16, 1: torch.int8}[t.element_size()]).numpy()
 
 
 def assert_attention_close(out: torch.Tensor, ref: np.ndarray, kv_dtype: torch.dtype, what: str = "") -> None:

@@ -90,8 +90,8 @@ class Case:
         okp, ovp = raw(kp).copy(), raw(vp).copy()
         oracle.reshape_and_cache(okp, ovp, raw(self.new_k), raw(self.new_v), oslots)
         self.okp, self.ovp = okp, ovp
-        self.okp_t = torch.from_numpy(okp).view(dtype) if dtype == torch.bfloat16 else torch.from_numpy(okp)
-        self.ovp_t = torch.from_numpy(ovp).view(dtype) if dtype == torch.bfloat16 else torch.from_numpy(ovp)
+        self.okp_t = torch.from_numpy(okp).view(dtype)
+        self.ovp_t = torch.from_numpy(ovp).view(dtype)
         self.ref = oracle.paged_decode(f64(self.q), self.okp_t.double().numpy(), self.ovp_t.double().numpy(),
                                        tab, self.ctx, self.scale, BS)
 

@@ -99,7 +99,7 @@ def test_gqa_bf16(pa):
 
 def test_long_splitk_bf16(pa):
     b = _decode_workload(pa, "long_splitk_bf16", per_head=lambda s: [s % 8, (s * 5 + 3) % 8])
-    assert b.partition_size > 0 and b.num_blocks * 32 * 8 * 128 * 2 > 2 ** 31  # pool past 2 GiB
+    assert b.partition_size > 0 and 2 * b.num_blocks * 32 * 8 * 128 * 2 > 2 ** 31  # K+V pools past 2 GiB
 
 
 def test_parallel_sampling_fp16(pa):
