@@ -122,13 +122,30 @@ class ClockSampler:
             self.uuid = None
 
     def start(self):
+        """Starts sampling and returns once the first sample has arrived, so
+        that nvidia-smi's start-up does not fall inside the timed region."""
+        import threading
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
         if self.uuid:
             cmd += ["-i", self.uuid]
+        self.lines = []
+        first = threading.Event()
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return
+
+        def reader():
+            for ln in self.proc.stdout:
+                self.lines.append(ln)
+                first.set()
+            first.set()
+
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+        first.wait(timeout=20)
+        self.skip = len(self.lines)  # samples taken before the timed region
 
     def stop(self):
         if self.proc is None:
@@ -136,10 +153,11 @@ class ClockSampler:
         time.sleep(0.06)
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-            out, _ = self.proc.communicate()
+        self.thread.join(timeout=5)
+        out = "".join(self.lines[self.skip:])
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for row in csv.reader(io.StringIO(out)):
@@ -256,7 +274,6 @@ def time_steps(b, steps: int, warmup: int, world: int, sample_clocks=False, devi
     sampler = ClockSampler(device_index) if sample_clocks else None
     if sampler:
         sampler.start()
-        time.sleep(0.15)
     barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
