@@ -3,8 +3,7 @@
 Argument marshalling only: every operation runs in the CUDA kernels of
 ``lib/libpa_b200.so`` through its C ABI (``include/pa.h``); functions keep the
 C names. PyTorch supplies device memory and streams. There is no CPU or
-library fallback: if the shared library is missing, importing the binding
-raises.
+library fallback: if the shared library is missing, the first call raises.
 
 Layouts (contiguous): k_cache/v_cache [num_blocks, num_kv_heads, block_size,
 head_dim]; query/out [num_seqs, num_heads, head_dim]; key/value
@@ -86,7 +85,19 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-_lib = _load()
+class _Library:
+    """The shared library, loaded on first use (so that ``_build`` can be
+    imported, and run, before the library exists). Any call without the built
+    library raises ImportError: there is no fallback."""
+    _cdll = None
+
+    def __getattr__(self, name):
+        if _Library._cdll is None:
+            _Library._cdll = _load()
+        return getattr(_Library._cdll, name)
+
+
+_lib = _Library()
 
 
 def status_string(status: int) -> str:
