@@ -161,6 +161,40 @@ int pa_splitk_reduce(void *out, const void *workspace, size_t workspace_bytes,
                      cudaStream_t stream);
 
 /*
+ * pa_decode_splitk_static -- split-K decode plus reduce for callers that
+ * cannot allocate device memory. The source pages have no counterpart; this
+ * is an interface choice of this library.
+ *
+ * Same inputs and result as pa_decode_splitk followed by pa_splitk_reduce
+ * (out [num_seqs, num_heads, head_dim] of out_dtype), but the workspace is a
+ * fixed array inside the library (PA_STATIC_SCRATCH_BYTES of device memory on
+ * every GPU that loads the library, kept until the process exits), so the
+ * caller passes only inputs and the output. It suits code that must not
+ * allocate while it runs: a serving loop that gave nearly all of HBM to its
+ * KV pool up front, a plug-in whose host framework forbids allocation inside
+ * its execute callback, or a caller with no device allocator at all.
+ *   - Returns PA_ERR_WORKSPACE, with no device work, when
+ *     pa_splitk_workspace_bytes(num_seqs, num_heads, head_dim,
+ *     max_context_len, partition_size) exceeds PA_STATIC_SCRATCH_BYTES
+ *     (use a larger partition_size or fewer sequences per call).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls on a device share the array: calls whose kernels overlap on
+ *     the GPU (other streams, other host threads) race and must be
+ *     serialised. The array keeps the previous call's partials; none of it
+ *     needs to start at zero.
+ *   - Allocates nothing and calls no allocating routine.
+ */
+#define PA_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+int pa_decode_splitk_static(void *out, const void *query, const void *k_cache, const void *v_cache,
+                            const int32_t *block_tables, int max_blocks_per_seq,
+                            const int32_t *context_lens, int num_seqs, int num_heads,
+                            int num_kv_heads, int head_dim, float scale, int block_size,
+                            int num_blocks, int max_context_len, int partition_size,
+                            pa_dtype kv_dtype, pa_dtype out_dtype, cudaStream_t stream);
+
+/*
  * Partition size this library would pick for a batch: 0 when the
  * unpartitioned pa_decode already fills the GPU, else a multiple of
  * block_size. Host-only arithmetic on the sizes given (occupancy rule:

@@ -38,8 +38,10 @@ EXPORTED = (
     "pa_splitk_workspace_bytes", "pa_splitk_acc_offset", "pa_decode_splitk", "pa_splitk_reduce",
     "pa_choose_partition", "pa_copy_blocks", "pa_pool_create", "pa_pool_destroy", "pa_pool_num_free",
     "pa_pool_ref_count", "pa_pool_allocate", "pa_pool_share", "pa_pool_free", "pa_pool_append",
-    "pa_pool_fork", "pa_pool_release",
+    "pa_pool_fork", "pa_pool_release", "pa_decode_splitk_static",
 )
+
+PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class PagedAttentionError(RuntimeError):
@@ -77,6 +79,8 @@ def _load() -> ctypes.CDLL:
         "pa_pool_append": (i32, [vp, i32p, i32, i32p, i32, i32p, i64p, i32, ctypes.POINTER(ctypes.c_int)]),
         "pa_pool_fork": (i32, [vp, i32p, i32, i32p, i32]),
         "pa_pool_release": (i32, [vp, i32p, i32]),
+        "pa_decode_splitk_static": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32,
+                                          i32, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -176,6 +180,20 @@ def pa_splitk_reduce(out, workspace, context_lens, max_context_len, partition_si
                                _ptr(context_lens), S, Hq, D, int(max_context_len), int(partition_size),
                                _dtype(out), _stream(stream))
     _check(rc, "pa_splitk_reduce")
+
+
+def pa_decode_splitk_static(out, query, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
+                            partition_size, stream=None) -> None:
+    """Split-K decode plus reduce with the library's fixed scratch array
+    instead of a caller workspace (for callers that cannot allocate; calls on
+    one device must not overlap)."""
+    S, Hq, D = query.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    rc = _lib.pa_decode_splitk_static(_ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                      block_tables.shape[1], _ptr(context_lens), S, Hq, Hkv, D, float(scale), bs,
+                                      NB, int(max_context_len), int(partition_size), _dtype(k_cache), _dtype(out),
+                                      _stream(stream))
+    _check(rc, "pa_decode_splitk_static")
 
 
 def pa_choose_partition(num_seqs, num_kv_heads, max_context_len, block_size, head_dim, kv_dtype) -> int:
