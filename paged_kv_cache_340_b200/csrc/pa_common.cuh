@@ -137,6 +137,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     }
 }
 
+// Orders this thread's earlier generic-proxy shared-memory accesses before its
+// later async-proxy (bulk copy) accesses, e.g. reads of a buffer before a bulk
+// copy that overwrites it.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // L2 policy for data read once per step (the KV stream): evict first.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
     uint64_t pol;

@@ -9,26 +9,32 @@
 // back; §6: fp16 storage, fp32 arithmetic]).
 //
 // How (B200 design, not the pages'):
-//   * one CTA per (sequence, kv head[, partition]); all G query heads of the
-//     GQA group share every K/V tile, so each tile crosses HBM once;
-//   * warp 4 is the producer: it reads the table row 32 entries at a time
-//     (coalesced, prefetched one chunk ahead) and streams each (block, kv head)
-//     K tile and V tile -- contiguous block_size*head_dim runs in this layout --
-//     into a ring of shared-memory stages with one-dimensional bulk copies
-//     (cp.async.bulk, TMA engine) completing on per-stage mbarriers;
-//   * warps 0-3 are consumers; warp w takes stages w, w+4, ... Each 16-byte
-//     lane vector covers 8 (16-bit) or 4 (fp32) elements of a token row; a
-//     warp instruction covers 32 / (head_dim / vec) token rows ("row
-//     groups"). Scores are reduced across the lanes of a row with a
-//     transposing butterfly (each step halves the values a lane holds), so a
-//     lane ends with whole scores and runs one exp per score, not one per lane;
-//   * each row group keeps its own running max / sum / accumulator in fp32
-//     (log2 domain: q is pre-scaled by scale * log2 e); the CTA merges the
-//     row groups at the end, by the same log-sum-exp rule as the split-K
-//     reduce;
+//   * one CTA of four warps per (sequence, kv head[, partition]); all G query
+//     heads of the GQA group share every K/V tile, so each tile crosses HBM
+//     once;
+//   * the token range is cut into 16-token stages; stage k belongs to warp
+//     k % 4 and lives in shared-memory buffer k % 8 (two buffers per warp).
+//     The warp loads its own stages: lane 0 streams the stage's K and V tile
+//     (16 contiguous token rows of one kv head in this layout) with two
+//     one-dimensional bulk copies (cp.async.bulk, TMA engine) completing on
+//     the buffer's mbarrier, and right after consuming stage k it reloads the
+//     same buffer with stage k + 8. No other warp touches the buffer, so
+//     there are no empty barriers and a parity wait can never alias. Table
+//     entries are read 32 stages ahead, one per lane;
+//   * 16-bit GQA groups (G >= 2) compute QK^T and PV with tensor-core MMAs
+//     (mma.sync m16n8k16, the group's query heads padded to 16 rows); MHA
+//     and fp32 use CUDA cores, where each lane holds one 16-byte column
+//     vector of a token row and a transposing butterfly reduces the partial
+//     dot products across the row's lanes (each step halves what a lane
+//     holds, so a lane ends with whole scores and runs one exp per score);
+//   * running max / sum / accumulator in fp32 (log2 domain), per row group;
+//     the CTA merges its row groups at the end by the same log-sum-exp rule
+//     as the split-K reduce;
 //   * every wait is bounded (PA_DEVERR_TIMEOUT), bad table entries skip their
-//     block (PA_DEVERR_BLOCK_ID).
+//     stage (PA_DEVERR_BLOCK_ID).
 #include <math.h>
+
+#include <type_traits>
 
 #include "pa_common.cuh"
 #include "pa_internal.h"
@@ -53,21 +59,24 @@ struct DecodeShape {
     static constexpr int kNvl = kNv >= kLpt ? kNv / kLpt : 1;   // scores a lane keeps
     static constexpr int kDup = kNv >= kLpt ? 1 : kLpt / kNv;   // lanes keeping the same score
     static constexpr int kLanesPerG = kLpt / G;        // lanes whose scores belong to one head
-    static constexpr int kConsumerWarps = 4;
-    static constexpr int kThreads = (kConsumerWarps + 1) * 32;
+    // 16-bit GQA groups run QK^T and PV on the tensor cores; MHA and fp32 on
+    // the CUDA cores.
+    static constexpr bool kUseMma = (kElt == 2) && (G >= 2);
+    static constexpr int kWarps = 4;
+    static constexpr int kThreads = kWarps * 32;
     static constexpr int kTileBytes = kTS * D * kElt;  // 16 token rows of one kv head, K or V
     static constexpr int kStageBytes = 2 * kTileBytes;
-    // Stage k is consumed by warp k % 4 and lives in buffer k % 8, so the
-    // previous use of a buffer always belongs to the same warp: a parity
-    // wait can never see a phase two behind.
-    static constexpr int kStages = 8;
-    static constexpr int kRowGroups = kConsumerWarps * kRows;
+    static constexpr int kStages = 8;                  // two buffers per warp
+    static constexpr int kRowGroups = kUseMma ? kWarps : kWarps * kRows;
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kMergeBytes = kRowGroups * G * (D + 2) * 4;
     static constexpr int kDataBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
-    static constexpr int kSmemBytes = 128 + kDataBytes + kStages * 16 + kStages * 4;
+    static constexpr int kSmemBytes = 128 + kDataBytes + kStages * 8 + kStages * 4;
+    // Resident CTAs per SM the register budget is set for (a sub-partition
+    // holds one warp of each CTA, so 3 CTAs leave 170 registers a thread).
+    static constexpr int kMinBlocks = (kUseMma || G <= 4) ? 3 : 2;
 
-    static_assert(kStages % kConsumerWarps == 0, "buffer reuse must stay within one warp");
+    static_assert(kStages == 2 * kWarps, "stage k: warp k % 4, buffer k % 8");
     static_assert(BS % kTS == 0, "block size is a multiple of the stage");
     static_assert(kLpt >= 1 && kLpt <= 32 && (32 % kLpt) == 0, "row width");
     static_assert(kTS % kRows == 0 && kTpg % kTc == 0, "stage split");
@@ -101,16 +110,345 @@ struct RowReduce {
     }
 };
 
+// ------------------------------------------------------- CUDA-core consumer
+
+// One warp's share of the CTA on the CUDA cores. Lane = r * kLpt + c: row r of
+// a warp instruction (token), 16-byte column c of that row.
+template <typename T, int D, int G, typename S>
+struct FmaConsumer {
+    int r, c, rg, g_lane, v0;
+    bool counts_l;
+    float q[G][S::kVec];
+    float m_run[G];
+    float acc[G][S::kVec];
+    float l_lane;
+
+    __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int warp, int lane) {
+        r = lane / S::kLpt;
+        c = lane % S::kLpt;
+        rg = warp * S::kRows + r;
+        g_lane = c / S::kLanesPerG;     // query head of this lane's kept scores
+        v0 = (c * S::kNv) / S::kLpt;    // index of this lane's first kept score
+        counts_l = (c % S::kDup) == 0;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const T *>(p.query) +
+                                                             (head0 + g) * D + c * S::kVec);
+            Elt<T>::unpack(u, q[g]);
+#pragma unroll
+            for (int e = 0; e < S::kVec; ++e) q[g][e] *= p.scale_log2;
+            m_run[g] = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < S::kVec; ++e) acc[g][e] = 0.f;
+        }
+        l_lane = 0.f;
+    }
+
+    __device__ __forceinline__ void stage(const unsigned char *Ks, const unsigned char *Vs, int nvalid,
+                                          int lane, float) {
+#pragma unroll
+        for (int ci = 0; ci < S::kChunks; ++ci) {
+            // ---- scores: partial dots over this lane's columns
+            float sc[S::kNv];
+#pragma unroll
+            for (int i = 0; i < S::kTc; ++i) {
+                const int t = (ci * S::kTc + i) * S::kRows + r;
+                const uint4 u = *reinterpret_cast<const uint4 *>(Ks + ((size_t)t * D + c * S::kVec) * S::kElt);
+                float kf[S::kVec];
+                Elt<T>::unpack(u, kf);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    float d0 = 0.f;
+#pragma unroll
+                    for (int e = 0; e < S::kVec; ++e) d0 = fmaf(q[g][e], kf[e], d0);
+                    sc[g * S::kTc + i] = d0;
+                }
+            }
+            RowReduce<S::kNv, S::kLpt / 2>::run(sc, lane);
+            // ---- mask the tail and take the chunk max per head
+            float cmax = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < S::kNvl; ++j) {
+                const int i = (v0 + j) % S::kTc;
+                const int t = (ci * S::kTc + i) * S::kRows + r;
+                if (t >= nvalid) sc[j] = -INFINITY;
+                cmax = fmaxf(cmax, sc[j]);
+            }
+#pragma unroll
+            for (int mk = 1; mk < S::kLanesPerG; mk <<= 1)
+                cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, mk));
+            float my_m = 0.f, my_alpha = 1.f;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float cm =
+                    (G == 1) ? cmax : __shfl_sync(0xffffffffu, cmax, r * S::kLpt + g * S::kLanesPerG);
+                const float mn = fmaxf(m_run[g], cm);
+                const float alpha = (mn == -INFINITY) ? 1.f : fast_exp2(m_run[g] - mn);
+                m_run[g] = mn;
+#pragma unroll
+                for (int e = 0; e < S::kVec; ++e) acc[g][e] *= alpha;
+                if (g == g_lane) {
+                    my_m = mn;
+                    my_alpha = alpha;
+                }
+            }
+            // ---- probabilities of the kept scores
+            float pk[S::kNvl];
+            float psum = 0.f;
+#pragma unroll
+            for (int j = 0; j < S::kNvl; ++j) {
+                pk[j] = (sc[j] == -INFINITY) ? 0.f : fast_exp2(sc[j] - my_m);
+                psum += pk[j];
+            }
+            l_lane = l_lane * my_alpha + (counts_l ? psum : 0.f);
+            // ---- PV: broadcast each token's probability along its row
+#pragma unroll
+            for (int i = 0; i < S::kTc; ++i) {
+                const int t = (ci * S::kTc + i) * S::kRows + r;
+                const uint4 u = *reinterpret_cast<const uint4 *>(Vs + ((size_t)t * D + c * S::kVec) * S::kElt);
+                float vf[S::kVec];
+                Elt<T>::unpack(u, vf);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    constexpr int kNvl = S::kNvl;
+                    const int v = g * S::kTc + i;
+                    const int src_c = (v * S::kLpt) / S::kNv;
+                    const float pv = __shfl_sync(0xffffffffu, pk[v % kNvl], r * S::kLpt + src_c);
+                    if (t < nvalid) {
+#pragma unroll
+                        for (int e = 0; e < S::kVec; ++e) acc[g][e] = fmaf(pv, vf[e], acc[g][e]);
+                    }
+                }
+            }
+        }
+    }
+
+    // After the ring is drained: this row group's (m, l, acc) to shared memory.
+    __device__ __forceinline__ void store(float *mg, float *lg, float *ag, int, int) {
+#pragma unroll
+        for (int mk = 1; mk < S::kLanesPerG; mk <<= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, mk);
+        if (c % S::kLanesPerG == 0) {
+            float mine = 0.f;
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+                if (g == g_lane) mine = m_run[g];
+            mg[rg * G + g_lane] = mine;
+            lg[rg * G + g_lane] = l_lane;
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float4 *dst = reinterpret_cast<float4 *>(ag + ((size_t)rg * G + g) * D + c * S::kVec);
+#pragma unroll
+            for (int e = 0; e < S::kVec; e += 4)
+                dst[e / 4] = make_float4(acc[g][e], acc[g][e + 1], acc[g][e + 2], acc[g][e + 3]);
+        }
+    }
+};
+
+// ------------------------------------------------------ tensor-core consumer
+
+// m16n8k16 MMA with fp32 accumulation for one 16-bit type. A rows 8..15 are
+// always zero here (at most 8 query heads per group), so a1 = a3 = 0.
+template <typename T> struct Mma;
+
+template <> struct Mma<__nv_bfloat16> {
+    // bf16 keeps 8 mantissa bits: a probability rounded once would cost about
+    // 1e-3 relative error, so P goes in as hi + lo (two MMAs, ~2^-17).
+    static constexpr bool kSplitP = true;
+    static __device__ __forceinline__ void mma(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                               uint32_t b1) {
+        asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+            "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+    }
+    static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t *>(&v);
+    }
+    static __device__ __forceinline__ float2 unpack(uint32_t u) {
+        return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+    }
+};
+
+template <> struct Mma<__half> {
+    // fp16 keeps 11 bits: one rounding of P is ~3e-4 relative, inside the bound.
+    static constexpr bool kSplitP = false;
+    static __device__ __forceinline__ void mma(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                               uint32_t b1) {
+        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+            "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+    }
+    static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+        __half2 v = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t *>(&v);
+    }
+    static __device__ __forceinline__ float2 unpack(uint32_t u) {
+        return __half22float2(*reinterpret_cast<__half2 *>(&u));
+    }
+};
+
+__device__ __forceinline__ uint32_t word_of(const uint4 &v, int i) {
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// One warp's share on the tensor cores. Per 16-token stage, with
+// lane = 4 r + q (r: query head of the group, q: quad position):
+//   S = Q K^T: M = query heads (padded to 16), N = 8 tokens (two tiles),
+//     K = head_dim. The k -> d map of each MMA k-step is chosen so that one
+//     16-byte shared load of a K row (d = 8q + 32i .. +8) feeds two k-steps
+//     directly; Q's fragment (loaded once) uses the same map.
+//   O += P V: M = query heads, N = 8 columns of d per tile, K = 16 tokens.
+//     P comes straight from the S accumulators; the column -> d map
+//     d = 64 (nt / 8) + 8 n + nt % 8 lets each lane load 16 bytes of a V row
+//     and build 8 tiles' B fragments with byte permutes (no transposing load,
+//     no bank conflicts).
+// The running max / sum live per row (query head) and warp; tokens past the
+// context are masked to -inf, and their V rows are zeroed (they may hold NaN).
+template <typename T, int D, int G, typename S>
+struct MmaConsumer {
+    using M = Mma<T>;
+    static constexpr int kI = D / 32;   // 16-byte chunks of a K row per lane (2 k-steps each)
+    static constexpr int kNT = D / 8;   // PV n-tiles
+    static constexpr int kH = D / 64;   // 16-byte V chunks per token row per lane
+    int q4, r;
+    uint32_t qa[kI][4];
+    float o[kNT][4];
+    float m_run, l_lane;
+
+    __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int, int lane) {
+        q4 = lane & 3;
+        r = lane >> 2;
+#pragma unroll
+        for (int i = 0; i < kI; ++i) {
+            uint4 u = make_uint4(0u, 0u, 0u, 0u);
+            if (r < G)
+                u = *reinterpret_cast<const uint4 *>(static_cast<const T *>(p.query) + (head0 + r) * D +
+                                                     8 * q4 + 32 * i);
+            qa[i][0] = u.x;
+            qa[i][1] = u.y;
+            qa[i][2] = u.z;
+            qa[i][3] = u.w;
+        }
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+        m_run = -INFINITY;
+        l_lane = 0.f;
+    }
+
+    __device__ __forceinline__ void stage(const unsigned char *Kb, const unsigned char *Vb, int nvalid, int,
+                                          float scale_log2) {
+        const T *Ks = reinterpret_cast<const T *>(Kb);
+        const T *Vs = reinterpret_cast<const T *>(Vb);
+        // ---- S = Q K^T for tokens 8j + r (B columns), this lane's k-chunks
+        float sc[2][4];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+            const T *krow = Ks + (8 * j + r) * D + 8 * q4;
+#pragma unroll
+            for (int i = 0; i < kI; ++i) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(krow + 32 * i);
+                M::mma(sc[j], qa[i][0], qa[i][1], u.x, u.y);
+                M::mma(sc[j], qa[i][2], qa[i][3], u.z, u.w);
+            }
+        }
+        // ---- online softmax on row r: this lane holds tokens 2q, 2q+1, 8+2q, 9+2q
+        float x[4] = {sc[0][0], sc[0][1], sc[1][0], sc[1][1]};
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int t = 8 * (e >> 1) + 2 * q4 + (e & 1);
+            x[e] = t < nvalid ? x[e] * scale_log2 : -INFINITY;
+            mx = fmaxf(mx, x[e]);
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float mn = fmaxf(m_run, mx);
+        const float alpha = (mn == -INFINITY) ? 1.f : fast_exp2(m_run - mn);
+        m_run = mn;
+        float pr[4];
+        float psum = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            pr[e] = (x[e] == -INFINITY) ? 0.f : fast_exp2(x[e] - mn);
+            psum += pr[e];
+        }
+        l_lane = l_lane * alpha + psum;
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+            o[nt][0] *= alpha;
+            o[nt][1] *= alpha;
+        }
+        const uint32_t ph0 = M::pack(pr[0], pr[1]);
+        const uint32_t ph2 = M::pack(pr[2], pr[3]);
+        uint32_t pl0 = 0u, pl2 = 0u;
+        if constexpr (M::kSplitP) {
+            const float2 h0 = M::unpack(ph0);
+            const float2 h2 = M::unpack(ph2);
+            pl0 = M::pack(pr[0] - h0.x, pr[1] - h0.y);
+            pl2 = M::pack(pr[2] - h2.x, pr[3] - h2.y);
+        }
+        // ---- O += P V
+#pragma unroll
+        for (int hh = 0; hh < kH; ++hh) {
+            const T *vcol = Vs + 64 * hh + 8 * r;
+            uint4 va = *reinterpret_cast<const uint4 *>(vcol + (2 * q4) * D);
+            uint4 vb = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 1) * D);
+            uint4 vc = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 8) * D);
+            uint4 vd = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 9) * D);
+            if (nvalid < S::kTS) {  // rows past the context may hold anything
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                if (2 * q4 >= nvalid) va = z;
+                if (2 * q4 + 1 >= nvalid) vb = z;
+                if (2 * q4 + 8 >= nvalid) vc = z;
+                if (2 * q4 + 9 >= nvalid) vd = z;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const unsigned sel = (e & 1) ? 0x7632u : 0x5410u;
+                const uint32_t b0 = __byte_perm(word_of(va, e >> 1), word_of(vb, e >> 1), sel);
+                const uint32_t b1 = __byte_perm(word_of(vc, e >> 1), word_of(vd, e >> 1), sel);
+                M::mma(o[8 * hh + e], ph0, ph2, b0, b1);
+                if constexpr (M::kSplitP) M::mma(o[8 * hh + e], pl0, pl2, b0, b1);
+            }
+        }
+    }
+
+    // After the ring is drained: this warp's (m, l, O) rows to shared memory.
+    __device__ __forceinline__ void store(float *mg, float *lg, float *ag, int warp, int) {
+        l_lane += __shfl_xor_sync(0xffffffffu, l_lane, 1);
+        l_lane += __shfl_xor_sync(0xffffffffu, l_lane, 2);
+        if (r < G) {
+            if (q4 == 0) {
+                mg[warp * G + r] = m_run;
+                lg[warp * G + r] = l_lane;
+            }
+            float *row = ag + ((size_t)warp * G + r) * D;
+#pragma unroll
+            for (int nt = 0; nt < kNT; ++nt) {
+                const int d0 = 64 * (nt >> 3) + 16 * q4 + (nt & 7);  // C columns 2q and 2q + 1
+                row[d0] = o[nt][0];
+                row[d0 + 8] = o[nt][1];
+            }
+        }
+    }
+};
+
+// -------------------------------------------------------------------- kernel
+
 template <typename T, int D, int BS, int G>
-__global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads)
+__global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShape<T, D, BS, G>::kMinBlocks)
     decode_kernel(const DecodeParams p) {
     using S = DecodeShape<T, D, BS, G>;
+    using Consumer = std::conditional_t<S::kUseMma, MmaConsumer<T, D, G, S>, FmaConsumer<T, D, G, S>>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *ring = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     uint64_t *full = reinterpret_cast<uint64_t *>(ring + S::kDataBytes);
-    uint64_t *empty = full + S::kStages;
-    int *bad = reinterpret_cast<int *>(empty + S::kStages);
+    int *bad = reinterpret_cast<int *>(full + S::kStages);
 
     const int part = blockIdx.x;
     const int kvh = blockIdx.y;
@@ -132,236 +470,128 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads)
         if (t_begin >= ctx) return;  // empty partition: nothing written
         t_end = min(t_begin + p.partition_size, ctx);
     }
-    const int nblk = (t_end - t_begin + BS - 1) / BS;           // table entries read
     const int nstage = (t_end - t_begin + S::kTS - 1) / S::kTS;  // 16-token stages
     const size_t head0 = (size_t)s * p.num_heads + (size_t)kvh * G;  // first query head row
-    if (nblk == 0) {  // unsplit, empty context: zeros
-        for (int i = threadIdx.x; i < G * D; i += blockDim.x)
-            store_out(p.out, head0 * D + i, 0.f, p.out_dtype);
+    if (nstage == 0) {  // unsplit, empty context: zeros
+        for (int i = threadIdx.x; i < G * D; i += blockDim.x) store_out(p.out, head0 * D + i, 0.f, p.out_dtype);
         return;
     }
-    const int first_block = t_begin / BS;
-
     if (threadIdx.x == 0) {
-        for (int i = 0; i < S::kStages; ++i) {
-            mbar_init(full + i, 1);
-            mbar_init(empty + i, 1);
-        }
+        for (int i = 0; i < S::kStages; ++i) mbar_init(full + i, 1);
         fence_mbar_init();
     }
     __syncthreads();
 
-    if (warp == S::kConsumerWarps) {
-        // =========================== producer warp
-        const int32_t *row = p.block_tables + (size_t)s * p.max_blocks_per_seq + first_block;
-        const size_t block_elems = (size_t)p.num_kv_heads * BS * D;
-        const size_t head_off = (size_t)kvh * BS * D;
-        const T *kc = static_cast<const T *>(p.k_cache) + head_off;
-        const T *vc = static_cast<const T *>(p.v_cache) + head_off;
-        const uint64_t pol = l2_evict_first_policy();
-        bool ok = true;
-        int issued = 0;
-        int next = lane < nblk ? __ldg(row + lane) : 0;
-        for (int base = 0; base < nblk && ok; base += 32) {
-            const int ids = next;
-            if (base + 32 + lane < nblk) next = __ldg(row + base + 32 + lane);
-            const int n = min(32, nblk - base);
-            const bool valid = ids >= 0 && ids < p.num_blocks;
-            if (lane < n && !valid) record_error(p.err, PA_DEVERR_BLOCK_ID);
-            for (int j = 0; j < n; ++j) {
-                const int b = __shfl_sync(0xffffffffu, ids, j);
-                const bool v = __shfl_sync(0xffffffffu, valid ? 1 : 0, j) != 0;
-#pragma unroll
-                for (int h = 0; h < S::kSubs; ++h) {
-                    const int k = (base + j) * S::kSubs + h;  // stage
-                    if (k >= nstage) break;
-                    if (lane == 0) {
-                        const int buf = k % S::kStages;
-                        if (k >= S::kStages && !mbar_wait(empty + buf, ((k / S::kStages) - 1) & 1)) {
-                            ok = false;
-                            record_error(p.err, PA_DEVERR_TIMEOUT);
-                        } else {
-                            if (v) {
-                                bad[buf] = 0;
-                                unsigned char *dst = ring + (size_t)buf * S::kStageBytes;
-                                const size_t src = (size_t)b * block_elems + (size_t)h * S::kTS * D;
-                                mbar_arrive_expect_tx(full + buf, S::kStageBytes);
-                                bulk_load(dst, kc + src, S::kTileBytes, full + buf, pol);
-                                bulk_load(dst + S::kTileBytes, vc + src, S::kTileBytes, full + buf, pol);
-                            } else {
-                                bad[buf] = 1;
-                                mbar_arrive(full + buf);
-                            }
-                            ++issued;
-                        }
-                    }
-                    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                    if (!ok) break;
-                }
-                if (!ok) break;
+    // ---- this warp's stages k = warp + 4 m, m < nmine
+    const int nmine = nstage > warp ? (nstage - warp + S::kWarps - 1) / S::kWarps : 0;
+    const int32_t *row = p.block_tables + (size_t)s * p.max_blocks_per_seq + t_begin / BS;
+    const size_t block_elems = (size_t)p.num_kv_heads * BS * D;
+    const T *kc = static_cast<const T *>(p.k_cache) + (size_t)kvh * BS * D;
+    const T *vc = static_cast<const T *>(p.v_cache) + (size_t)kvh * BS * D;
+    const uint64_t pol = l2_evict_first_policy();
+
+    // Block id of local stage m0 + lane (-1: none, or a bad entry).
+    auto load_ids = [&](int m0) -> int {
+        const int m = m0 + lane;
+        int id = -1;
+        if (m < nmine) {
+            id = __ldg(row + ((warp + S::kWarps * m) * S::kTS) / BS);
+            if (id < 0 || id >= p.num_blocks) {
+                record_error(p.err, PA_DEVERR_BLOCK_ID);
+                id = -1;
             }
         }
-        // Before exiting, every copy this CTA started must have landed.
-        if (lane == 0) {
-            for (int k = max(0, issued - S::kStages); k < issued; ++k)
-                if (!mbar_wait(full + (k % S::kStages), (k / S::kStages) & 1))
-                    record_error(p.err, PA_DEVERR_TIMEOUT);
+        return id;
+    };
+    int m0 = 0;
+    int ids_cur = load_ids(0);
+    int ids_next = load_ids(32);
+    auto id_of = [&](int m) -> int {  // whole warp; m0 <= m < m0 + 64
+        const int a = __shfl_sync(0xffffffffu, ids_cur, (m - m0) & 31);
+        const int b = __shfl_sync(0xffffffffu, ids_next, (m - m0) & 31);
+        return (m - m0 < 32) ? a : b;
+    };
+    auto issue = [&](int m, int id) {  // lane 0
+        const int k = warp + S::kWarps * m;
+        const int buf = k % S::kStages;
+        if (id >= 0) {
+            bad[buf] = 0;
+            const size_t src = (size_t)id * block_elems + (size_t)(k % S::kSubs) * S::kTS * D;
+            unsigned char *dst = ring + (size_t)buf * S::kStageBytes;
+            mbar_arrive_expect_tx(full + buf, S::kStageBytes);
+            bulk_load(dst, kc + src, S::kTileBytes, full + buf, pol);
+            bulk_load(dst + S::kTileBytes, vc + src, S::kTileBytes, full + buf, pol);
+        } else {
+            bad[buf] = 1;
+            mbar_arrive(full + buf);
         }
-        return;
+    };
+    {
+        const int i0 = id_of(0);
+        const int i1 = id_of(1);
+        if (lane == 0) {
+            if (nmine > 0) issue(0, i0);
+            if (nmine > 1) issue(1, i1);
+        }
     }
 
-    // =============================== consumer warps
-    const int r = lane / S::kLpt;          // row within the warp instruction
-    const int c = lane % S::kLpt;          // 16-byte column of the row
-    const int rg = warp * S::kRows + r;    // row group
-    const int g_lane = c / S::kLanesPerG;  // query head of this lane's kept scores
-    const int v0 = (c * S::kNv) / S::kLpt; // index of this lane's first kept score
-    const bool counts_l = (c % S::kDup) == 0;
-
-    float q[G][S::kVec];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const T *>(p.query) +
-                                                         (head0 + g) * D + c * S::kVec);
-        Elt<T>::unpack(u, q[g]);
-#pragma unroll
-        for (int e = 0; e < S::kVec; ++e) q[g][e] *= p.scale_log2;
-    }
-    float m_run[G];
-    float acc[G][S::kVec];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        m_run[g] = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < S::kVec; ++e) acc[g][e] = 0.f;
-    }
-    float l_lane = 0.f;
-
-    for (int k = warp; k < nstage; k += S::kConsumerWarps) {
+    Consumer cons;
+    cons.init(p, head0, warp, lane);
+    int waited = 0;
+    bool ok = true;
+    for (int m = 0; m < nmine; ++m) {
+        if (m - m0 == 32) {
+            m0 = m;
+            ids_cur = ids_next;
+            ids_next = load_ids(m0 + 32);
+        }
+        const int k = warp + S::kWarps * m;
         const int buf = k % S::kStages;
         const bool got = mbar_wait(full + buf, (k / S::kStages) & 1);
         if (!__all_sync(0xffffffffu, got)) {
             if (lane == 0) record_error(p.err, PA_DEVERR_TIMEOUT);
+            ok = false;
             break;
         }
+        waited = m + 1;
         if (!bad[buf]) {
             const int nvalid = min(S::kTS, t_end - (t_begin + k * S::kTS));
-            const unsigned char *Ks = ring + (size_t)buf * S::kStageBytes;
-            const unsigned char *Vs = Ks + S::kTileBytes;
-#pragma unroll
-            for (int ci = 0; ci < S::kChunks; ++ci) {
-                // ---- scores: partial dots over this lane's columns
-                float sc[S::kNv];
-#pragma unroll
-                for (int i = 0; i < S::kTc; ++i) {
-                    const int t = (ci * S::kTc + i) * S::kRows + r;
-                    const uint4 u = *reinterpret_cast<const uint4 *>(
-                        Ks + ((size_t)t * D + c * S::kVec) * S::kElt);
-                    float kf[S::kVec];
-                    Elt<T>::unpack(u, kf);
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        float d0 = 0.f;
-#pragma unroll
-                        for (int e = 0; e < S::kVec; ++e) d0 = fmaf(q[g][e], kf[e], d0);
-                        sc[g * S::kTc + i] = d0;
-                    }
-                }
-                RowReduce<S::kNv, S::kLpt / 2>::run(sc, lane);
-                // ---- mask the tail and take the chunk max per head
-                float cmax = -INFINITY;
-#pragma unroll
-                for (int j = 0; j < S::kNvl; ++j) {
-                    const int i = (v0 + j) % S::kTc;
-                    const int t = (ci * S::kTc + i) * S::kRows + r;
-                    if (t >= nvalid) sc[j] = -INFINITY;
-                    cmax = fmaxf(cmax, sc[j]);
-                }
-#pragma unroll
-                for (int mk = 1; mk < S::kLanesPerG; mk <<= 1)
-                    cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, mk));
-                float my_m = 0.f, my_alpha = 1.f;
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float cm = (G == 1) ? cmax
-                                              : __shfl_sync(0xffffffffu, cmax,
-                                                            r * S::kLpt + g * S::kLanesPerG);
-                    const float mn = fmaxf(m_run[g], cm);
-                    const float alpha = (mn == -INFINITY) ? 1.f : fast_exp2(m_run[g] - mn);
-                    m_run[g] = mn;
-#pragma unroll
-                    for (int e = 0; e < S::kVec; ++e) acc[g][e] *= alpha;
-                    if (g == g_lane) { my_m = mn; my_alpha = alpha; }
-                }
-                // ---- probabilities of the kept scores
-                float pk[S::kNvl];
-                float psum = 0.f;
-#pragma unroll
-                for (int j = 0; j < S::kNvl; ++j) {
-                    pk[j] = (sc[j] == -INFINITY) ? 0.f : fast_exp2(sc[j] - my_m);
-                    psum += pk[j];
-                }
-                l_lane = l_lane * my_alpha + (counts_l ? psum : 0.f);
-                // ---- PV: broadcast each token's probability along its row
-#pragma unroll
-                for (int i = 0; i < S::kTc; ++i) {
-                    const int t = (ci * S::kTc + i) * S::kRows + r;
-                    const uint4 u = *reinterpret_cast<const uint4 *>(
-                        Vs + ((size_t)t * D + c * S::kVec) * S::kElt);
-                    float vf[S::kVec];
-                    Elt<T>::unpack(u, vf);
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        constexpr int kNvl = S::kNvl;
-                        const int v = g * S::kTc + i;
-                        const int src_c = (v * S::kLpt) / S::kNv;
-                        const float pv = __shfl_sync(0xffffffffu, pk[v % kNvl], r * S::kLpt + src_c);
-                        if (t < nvalid) {
-#pragma unroll
-                            for (int e = 0; e < S::kVec; ++e) acc[g][e] = fmaf(pv, vf[e], acc[g][e]);
-                        }
-                    }
-                }
-            }
+            const unsigned char *Kb = ring + (size_t)buf * S::kStageBytes;
+            cons.stage(Kb, Kb + S::kTileBytes, nvalid, lane, p.scale_log2);
         }
+        // Reload this buffer with this warp's stage m + 2.
+        const int idn = id_of(m + 2);
         __syncwarp();
-        if (lane == 0) mbar_arrive(empty + buf);
+        if (lane == 0 && m + 2 < nmine) {
+            fence_proxy_async_smem();
+            issue(m + 2, idn);
+        }
+    }
+    if (!ok && lane == 0) {  // after a timeout: let every copy this warp started land
+        for (int m = waited; m < min(nmine, waited + 2); ++m) {
+            const int k = warp + S::kWarps * m;
+            if (!mbar_wait(full + (k % S::kStages), (k / S::kStages) & 1)) record_error(p.err, PA_DEVERR_TIMEOUT);
+        }
     }
 
-    // ---- merge the row groups (log-sum-exp), reusing the ring
-#pragma unroll
-    for (int mk = 1; mk < S::kLanesPerG; mk <<= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, mk);
-    named_bar_sync(1, S::kConsumerWarps * 32);  // every consumer is done with the ring
-    float *mg = reinterpret_cast<float *>(ring);    // [row group][G]
-    float *lg = mg + S::kRowGroups * G;            // [row group][G]
-    float *ag = lg + S::kRowGroups * G;            // [row group][G][D]
-    if (c % S::kLanesPerG == 0) {
-        float mine = 0.f;
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-            if (g == g_lane) mine = m_run[g];
-        mg[rg * G + g_lane] = mine;
-        lg[rg * G + g_lane] = l_lane;
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        float4 *dst = reinterpret_cast<float4 *>(ag + ((size_t)rg * G + g) * D + c * S::kVec);
-#pragma unroll
-        for (int e = 0; e < S::kVec; e += 4)
-            dst[e / 4] = make_float4(acc[g][e], acc[g][e + 1], acc[g][e + 2], acc[g][e + 3]);
-    }
-    named_bar_sync(1, S::kConsumerWarps * 32);
-    for (int idx = threadIdx.x; idx < G * D; idx += S::kConsumerWarps * 32) {
+    // ---- merge the row groups (log-sum-exp), reusing the drained ring
+    float *mg = reinterpret_cast<float *>(ring);  // [row group][G]
+    float *lg = mg + S::kRowGroups * G;          // [row group][G]
+    float *ag = lg + S::kRowGroups * G;          // [row group][G][D]
+    __syncthreads();
+    cons.store(mg, lg, ag, warp, lane);
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < G * D; idx += S::kThreads) {
         const int g = idx / D;
         const int d = idx % D;
-        float M = -INFINITY;
+        float Mx = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < S::kRowGroups; ++i) M = fmaxf(M, mg[i * G + g]);
+        for (int i = 0; i < S::kRowGroups; ++i) Mx = fmaxf(Mx, mg[i * G + g]);
         float num = 0.f, den = 0.f;
-        if (M != -INFINITY) {
+        if (Mx != -INFINITY) {
 #pragma unroll
             for (int i = 0; i < S::kRowGroups; ++i) {
-                const float w = fast_exp2(mg[i * G + g] - M);
+                const float w = fast_exp2(mg[i * G + g] - Mx);
                 num = fmaf(w, ag[((size_t)i * G + g) * D + d], num);
                 den = fmaf(w, lg[i * G + g], den);
             }
@@ -371,7 +601,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads)
             const size_t slot = h * p.max_parts + part;
             p.ws_acc[slot * D + d] = num;
             if (d == 0) {
-                p.ws_ml[slot * 2] = M * kLn2;
+                p.ws_ml[slot * 2] = Mx * kLn2;
                 p.ws_ml[slot * 2 + 1] = den;
             }
         } else {
