@@ -69,7 +69,8 @@ struct DecodeShape {
     static constexpr int kStages = 8;                  // two buffers per warp
     static constexpr int kRowGroups = kUseMma ? kWarps : kWarps * kRows;
     static constexpr int kRingBytes = kStages * kStageBytes;
-    static constexpr int kMergeBytes = kRowGroups * G * (D + 2) * 4;
+    static constexpr int kAgStride = kUseMma ? D + 1 : D;  // floats per merged accumulator row
+    static constexpr int kMergeBytes = kRowGroups * G * (kAgStride + 2) * 4;
     static constexpr int kDataBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
     static constexpr int kSmemBytes = 128 + kDataBytes + kStages * 8 + kStages * 4;
     // Resident CTAs per SM the register budget is set for (a sub-partition
@@ -237,7 +238,7 @@ struct FmaConsumer {
         }
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            float4 *dst = reinterpret_cast<float4 *>(ag + ((size_t)rg * G + g) * D + c * S::kVec);
+            float4 *dst = reinterpret_cast<float4 *>(ag + ((size_t)rg * G + g) * S::kAgStride + c * S::kVec);
 #pragma unroll
             for (int e = 0; e < S::kVec; e += 4)
                 dst[e / 4] = make_float4(acc[g][e], acc[g][e + 1], acc[g][e + 2], acc[g][e + 3]);
@@ -247,20 +248,19 @@ struct FmaConsumer {
 
 // ------------------------------------------------------ tensor-core consumer
 
-// m16n8k16 MMA with fp32 accumulation for one 16-bit type. A rows 8..15 are
-// always zero here (at most 8 query heads per group), so a1 = a3 = 0.
+// m16n8k16 MMA, fp32 accumulation, for one 16-bit type.
 template <typename T> struct Mma;
 
 template <> struct Mma<__nv_bfloat16> {
     // bf16 keeps 8 mantissa bits: a probability rounded once would cost about
     // 1e-3 relative error, so P goes in as hi + lo (two MMAs, ~2^-17).
     static constexpr bool kSplitP = true;
-    static __device__ __forceinline__ void mma(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0,
-                                               uint32_t b1) {
+    static __device__ __forceinline__ void mma(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
         asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
             "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
             : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-            : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
     }
     static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
         __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -274,12 +274,12 @@ template <> struct Mma<__nv_bfloat16> {
 template <> struct Mma<__half> {
     // fp16 keeps 11 bits: one rounding of P is ~3e-4 relative, inside the bound.
     static constexpr bool kSplitP = false;
-    static __device__ __forceinline__ void mma(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0,
-                                               uint32_t b1) {
+    static __device__ __forceinline__ void mma(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
         asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
             "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
             : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-            : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
     }
     static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
         __half2 v = __floats2half2_rn(lo, hi);
@@ -290,33 +290,49 @@ template <> struct Mma<__half> {
     }
 };
 
+// Transpose of an 8x8 matrix of 16-bit pairs held one row pair per lane
+// (lane 4 r + q holds row r, columns 2q, 2q + 1).
+__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
+    uint32_t y;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-// One warp's share on the tensor cores. Per 16-token stage, with
-// lane = 4 r + q (r: query head of the group, q: quad position):
-//   S = Q K^T: M = query heads (padded to 16), N = 8 tokens (two tiles),
-//     K = head_dim. The k -> d map of each MMA k-step is chosen so that one
-//     16-byte shared load of a K row (d = 8q + 32i .. +8) feeds two k-steps
-//     directly; Q's fragment (loaded once) uses the same map.
-//   O += P V: M = query heads, N = 8 columns of d per tile, K = 16 tokens.
-//     P comes straight from the S accumulators; the column -> d map
-//     d = 64 (nt / 8) + 8 n + nt % 8 lets each lane load 16 bytes of a V row
-//     and build 8 tiles' B fragments with byte permutes (no transposing load,
-//     no bank conflicts).
-// The running max / sum live per row (query head) and warp; tokens past the
-// context are masked to -inf, and their V rows are zeroed (they may hold NaN).
+// One warp's share on the tensor cores, in transposed form so that the
+// 16-row M side of the MMA is filled by tokens and head dims instead of the
+// group's 2-8 query heads. Per 16-token stage, with lane = 4 r + q:
+//   S^T = K Q^T: M = the stage's 16 tokens, N = 8 query-head columns (the
+//     group, zero-padded), K = head_dim. The k -> d map of each k-step is
+//     chosen so that one 16-byte shared load of a K row (d = 8q + 32i .. +8)
+//     feeds two k-steps; Q's B fragment, loaded once, uses the same map.
+//     Lane holds S^T[t][g] for t in {r, r + 8}, g in {2q, 2q + 1}.
+//   O^T += V^T P^T: M = 16 head dims per tile, N = 8 query-head columns,
+//     K = 16 tokens. P^T's B fragment is the S^T accumulator, packed to 16
+//     bits and transposed in registers (movmatrix). V^T's A fragment is built
+//     with byte permutes from 16-byte loads of V rows (no transposing load,
+//     no bank conflicts): tile mt row m holds d = 8 (m % 8) + E % 8 +
+//     64 (E / 8) with E = mt for m < 8 and E = mt + D/16 for m >= 8.
+// Running max / sum per (query head, warp); tokens past the context are
+// masked to -inf and their V rows zeroed (they may hold NaN).
 template <typename T, int D, int G, typename S>
 struct MmaConsumer {
     using M = Mma<T>;
-    static constexpr int kI = D / 32;   // 16-byte chunks of a K row per lane (2 k-steps each)
-    static constexpr int kNT = D / 8;   // PV n-tiles
-    static constexpr int kH = D / 64;   // 16-byte V chunks per token row per lane
+    static constexpr int kI = D / 32;    // 16-byte chunks of a K row per lane (2 k-steps each)
+    static constexpr int kMT = D / 16;   // PV m-tiles
+    static constexpr int kCh = D / 64;   // 16-byte V chunks per token row per lane
     int q4, r;
-    uint32_t qa[kI][4];
-    float o[kNT][4];
-    float m_run, l_lane;
+    uint32_t qb[kI][4];
+    float o[kMT][4];
+    float m_run[2], l_lane[2];
+
+    static __device__ __forceinline__ int dim_of(int m, int mt) {  // head dim of m-tile mt, row m
+        const int E = m < 8 ? mt : mt + kMT;
+        return 8 * (m & 7) + (E & 7) + 64 * (E >> 3);
+    }
 
     __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int, int lane) {
         q4 = lane & 3;
@@ -327,74 +343,84 @@ struct MmaConsumer {
             if (r < G)
                 u = *reinterpret_cast<const uint4 *>(static_cast<const T *>(p.query) + (head0 + r) * D +
                                                      8 * q4 + 32 * i);
-            qa[i][0] = u.x;
-            qa[i][1] = u.y;
-            qa[i][2] = u.z;
-            qa[i][3] = u.w;
+            qb[i][0] = u.x;
+            qb[i][1] = u.y;
+            qb[i][2] = u.z;
+            qb[i][3] = u.w;
         }
 #pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-        m_run = -INFINITY;
-        l_lane = 0.f;
+        for (int mt = 0; mt < kMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+        m_run[0] = m_run[1] = -INFINITY;
+        l_lane[0] = l_lane[1] = 0.f;
     }
 
     __device__ __forceinline__ void stage(const unsigned char *Kb, const unsigned char *Vb, int nvalid, int,
                                           float scale_log2) {
         const T *Ks = reinterpret_cast<const T *>(Kb);
         const T *Vs = reinterpret_cast<const T *>(Vb);
-        // ---- S = Q K^T for tokens 8j + r (B columns), this lane's k-chunks
-        float sc[2][4];
+        // ---- S^T = K Q^T
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        const T *k0 = Ks + r * D + 8 * q4;
+        const T *k1 = k0 + 8 * D;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
-            const T *krow = Ks + (8 * j + r) * D + 8 * q4;
-#pragma unroll
-            for (int i = 0; i < kI; ++i) {
-                const uint4 u = *reinterpret_cast<const uint4 *>(krow + 32 * i);
-                M::mma(sc[j], qa[i][0], qa[i][1], u.x, u.y);
-                M::mma(sc[j], qa[i][2], qa[i][3], u.z, u.w);
-            }
+        for (int i = 0; i < kI; ++i) {
+            const uint4 u0 = *reinterpret_cast<const uint4 *>(k0 + 32 * i);
+            const uint4 u1 = *reinterpret_cast<const uint4 *>(k1 + 32 * i);
+            M::mma(sc, u0.x, u1.x, u0.y, u1.y, qb[i][0], qb[i][1]);
+            M::mma(sc, u0.z, u1.z, u0.w, u1.w, qb[i][2], qb[i][3]);
         }
-        // ---- online softmax on row r: this lane holds tokens 2q, 2q+1, 8+2q, 9+2q
-        float x[4] = {sc[0][0], sc[0][1], sc[1][0], sc[1][1]};
-        float mx = -INFINITY;
+        // ---- online softmax per query head g = 2q + h (h = 0, 1) over tokens r, r + 8
+        const bool v0 = r < nvalid;
+        const bool v1 = r + 8 < nvalid;
+        float x[4];
+        x[0] = v0 ? sc[0] * scale_log2 : -INFINITY;  // t = r,     g = 2q
+        x[1] = v0 ? sc[1] * scale_log2 : -INFINITY;  // t = r,     g = 2q + 1
+        x[2] = v1 ? sc[2] * scale_log2 : -INFINITY;  // t = r + 8, g = 2q
+        x[3] = v1 ? sc[3] * scale_log2 : -INFINITY;  // t = r + 8, g = 2q + 1
+        float mx0 = fmaxf(x[0], x[2]);
+        float mx1 = fmaxf(x[1], x[3]);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int t = 8 * (e >> 1) + 2 * q4 + (e & 1);
-            x[e] = t < nvalid ? x[e] * scale_log2 : -INFINITY;
-            mx = fmaxf(mx, x[e]);
+        for (int mk = 4; mk < 32; mk <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, mk));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, mk));
         }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float mn = fmaxf(m_run, mx);
-        const float alpha = (mn == -INFINITY) ? 1.f : fast_exp2(m_run - mn);
-        m_run = mn;
+        const float mn0 = fmaxf(m_run[0], mx0);
+        const float mn1 = fmaxf(m_run[1], mx1);
+        const float al0 = (mn0 == -INFINITY) ? 1.f : fast_exp2(m_run[0] - mn0);
+        const float al1 = (mn1 == -INFINITY) ? 1.f : fast_exp2(m_run[1] - mn1);
+        m_run[0] = mn0;
+        m_run[1] = mn1;
         float pr[4];
-        float psum = 0.f;
+        pr[0] = (x[0] == -INFINITY) ? 0.f : fast_exp2(x[0] - mn0);
+        pr[1] = (x[1] == -INFINITY) ? 0.f : fast_exp2(x[1] - mn1);
+        pr[2] = (x[2] == -INFINITY) ? 0.f : fast_exp2(x[2] - mn0);
+        pr[3] = (x[3] == -INFINITY) ? 0.f : fast_exp2(x[3] - mn1);
+        l_lane[0] = l_lane[0] * al0 + pr[0] + pr[2];
+        l_lane[1] = l_lane[1] * al1 + pr[1] + pr[3];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            pr[e] = (x[e] == -INFINITY) ? 0.f : fast_exp2(x[e] - mn);
-            psum += pr[e];
+        for (int mt = 0; mt < kMT; ++mt) {
+            o[mt][0] *= al0;
+            o[mt][1] *= al1;
+            o[mt][2] *= al0;
+            o[mt][3] *= al1;
         }
-        l_lane = l_lane * alpha + psum;
-#pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) {
-            o[nt][0] *= alpha;
-            o[nt][1] *= alpha;
-        }
-        const uint32_t ph0 = M::pack(pr[0], pr[1]);
-        const uint32_t ph2 = M::pack(pr[2], pr[3]);
-        uint32_t pl0 = 0u, pl2 = 0u;
+        // ---- P^T fragments -> PV's B fragments (tokens 0-7 and 8-15)
+        const uint32_t h01 = M::pack(pr[0], pr[1]);
+        const uint32_t h23 = M::pack(pr[2], pr[3]);
+        const uint32_t bh0 = transpose8x8(h01);
+        const uint32_t bh1 = transpose8x8(h23);
+        uint32_t bl0 = 0u, bl1 = 0u;
         if constexpr (M::kSplitP) {
-            const float2 h0 = M::unpack(ph0);
-            const float2 h2 = M::unpack(ph2);
-            pl0 = M::pack(pr[0] - h0.x, pr[1] - h0.y);
-            pl2 = M::pack(pr[2] - h2.x, pr[3] - h2.y);
+            const float2 f01 = M::unpack(h01);
+            const float2 f23 = M::unpack(h23);
+            bl0 = transpose8x8(M::pack(pr[0] - f01.x, pr[1] - f01.y));
+            bl1 = transpose8x8(M::pack(pr[2] - f23.x, pr[3] - f23.y));
         }
-        // ---- O += P V
+        // ---- O^T += V^T P^T
+        uint32_t a_lo[kMT][4];  // V^T A fragments of this stage
 #pragma unroll
-        for (int hh = 0; hh < kH; ++hh) {
-            const T *vcol = Vs + 64 * hh + 8 * r;
+        for (int ch = 0; ch < kCh; ++ch) {
+            const T *vcol = Vs + 64 * ch + 8 * r;
             uint4 va = *reinterpret_cast<const uint4 *>(vcol + (2 * q4) * D);
             uint4 vb = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 1) * D);
             uint4 vc = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 8) * D);
@@ -406,32 +432,50 @@ struct MmaConsumer {
                 if (2 * q4 + 8 >= nvalid) vc = z;
                 if (2 * q4 + 9 >= nvalid) vd = z;
             }
+            // element e of chunk ch is E = 8 ch + e: tile E (rows < 8) or tile E - kMT (rows >= 8)
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
+                const int E = 8 * ch + e;
                 const unsigned sel = (e & 1) ? 0x7632u : 0x5410u;
-                const uint32_t b0 = __byte_perm(word_of(va, e >> 1), word_of(vb, e >> 1), sel);
-                const uint32_t b1 = __byte_perm(word_of(vc, e >> 1), word_of(vd, e >> 1), sel);
-                M::mma(o[8 * hh + e], ph0, ph2, b0, b1);
-                if constexpr (M::kSplitP) M::mma(o[8 * hh + e], pl0, pl2, b0, b1);
+                const uint32_t lo_t = __byte_perm(word_of(va, e >> 1), word_of(vb, e >> 1), sel);  // t = 2q, 2q+1
+                const uint32_t hi_t = __byte_perm(word_of(vc, e >> 1), word_of(vd, e >> 1), sel);  // t = 2q+8, 2q+9
+                if (E < kMT) {
+                    a_lo[E][0] = lo_t;
+                    a_lo[E][2] = hi_t;
+                } else {
+                    a_lo[E - kMT][1] = lo_t;
+                    a_lo[E - kMT][3] = hi_t;
+                }
             }
         }
-    }
-
-    // After the ring is drained: this warp's (m, l, O) rows to shared memory.
-    __device__ __forceinline__ void store(float *mg, float *lg, float *ag, int warp, int) {
-        l_lane += __shfl_xor_sync(0xffffffffu, l_lane, 1);
-        l_lane += __shfl_xor_sync(0xffffffffu, l_lane, 2);
-        if (r < G) {
-            if (q4 == 0) {
-                mg[warp * G + r] = m_run;
-                lg[warp * G + r] = l_lane;
-            }
-            float *row = ag + ((size_t)warp * G + r) * D;
 #pragma unroll
-            for (int nt = 0; nt < kNT; ++nt) {
-                const int d0 = 64 * (nt >> 3) + 16 * q4 + (nt & 7);  // C columns 2q and 2q + 1
-                row[d0] = o[nt][0];
-                row[d0 + 8] = o[nt][1];
+        for (int mt = 0; mt < kMT; ++mt) {
+            M::mma(o[mt], a_lo[mt][0], a_lo[mt][1], a_lo[mt][2], a_lo[mt][3], bh0, bh1);
+            if constexpr (M::kSplitP) M::mma(o[mt], a_lo[mt][0], a_lo[mt][1], a_lo[mt][2], a_lo[mt][3], bl0, bl1);
+        }
+    }
+    // After the ring is drained: this warp's (m, l, O) to shared memory.
+    // Row stride D + 1 keeps the scattered stores off a single bank.
+    __device__ __forceinline__ void store(float *mg, float *lg, float *ag, int warp, int) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int mk = 4; mk < 32; mk <<= 1) l_lane[h] += __shfl_xor_sync(0xffffffffu, l_lane[h], mk);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int g = 2 * q4 + h;
+            if (g < G) {
+                if (r == 0) {
+                    mg[warp * G + g] = m_run[h];
+                    lg[warp * G + g] = l_lane[h];
+                }
+                float *row = ag + ((size_t)warp * G + g) * S::kAgStride;
+#pragma unroll
+                for (int mt = 0; mt < kMT; ++mt) {
+                    row[dim_of(r, mt)] = o[mt][h];
+                    row[dim_of(r + 8, mt)] = o[mt][2 + h];
+                }
             }
         }
     }
@@ -592,7 +636,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
 #pragma unroll
             for (int i = 0; i < S::kRowGroups; ++i) {
                 const float w = fast_exp2(mg[i * G + g] - Mx);
-                num = fmaf(w, ag[((size_t)i * G + g) * D + d], num);
+                num = fmaf(w, ag[((size_t)i * G + g) * S::kAgStride + d], num);
                 den = fmaf(w, lg[i * G + g], den);
             }
         }
