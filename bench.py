@@ -177,44 +177,27 @@ class ClockSampler:
 
 # ------------------------------------------------------------ distributed
 
+from paged_kv_cache_340_b200 import dist as pdist  # noqa: E402
+
+
 def dist_setup(n_gpus: int):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    elif torch.cuda.is_available():
-        torch.cuda.set_device(local)
-    return world, rank, local
+    return pdist.init("nccl")
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return pdist.max_over_ranks(x, world)
 
 
 def barrier(world: int):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    pdist.barrier(world)
 
 
 # ------------------------------------------------------------ measurement
 
 def build_batch(name: str, rank: int, partition=None):
     from paged_kv_cache_340_b200.batch import build_decode_batch, build_parallel_sampling_batch, write_prefix
-    from paged_kv_cache_340_b200.workloads import SPECS, make_decode_inputs, make_parallel_sampling_inputs, scaled
-    spec = SPECS[name]
-    if rank:
-        spec = scaled(spec, seed=spec.seed + 1000 * rank)
+    from paged_kv_cache_340_b200.workloads import SPECS, make_decode_inputs, make_parallel_sampling_inputs
+    spec = pdist.rank_spec(SPECS[name], rank)
     if spec.lengths[0] == "parallel":
         inp = make_parallel_sampling_inputs(spec)
         b = build_parallel_sampling_batch(spec, inp, partition_size=partition or 0)
@@ -334,30 +317,48 @@ def e2e_steps(b, steps: int, warmup: int, world: int):
 
 # ---------------------------------------------------------- CPU oracle legs
 
-def oracle_sample(spec, b, budget_s: float, start_seq: int = 0):
-    """Times the oracle (as it stands, single-threaded double C) on whole
-    sequences of the batch, from start_seq on, until budget_s of oracle time is
-    spent. Returns (bytes, seconds, sequences). The oracle reads the host
-    copies of the generated inputs; widening to float64 is outside the timed
-    calls."""
+class OracleBatch:
+    """The oracle's view of a decode workload, built on the host only: the
+    seeded inputs and the block tables from the oracle's own pool (same
+    free-block order as the library's), never from the CUDA path."""
+
+    def __init__(self, spec, inputs=None):
+        import oracle
+        from oracle.block_pool import BlockPool as OPool, Sequence, append_tokens
+        from paged_kv_cache_340_b200.workloads import make_decode_inputs
+        oracle.build()
+        self.spec = spec
+        self.inputs = inputs if inputs is not None else make_decode_inputs(spec)
+        ctx = self.inputs["context_lens"].numpy().astype(np.int32)
+        pool = OPool(int(self.inputs["num_blocks"]), spec.block_size, policy="fifo",
+                     free_order=self.inputs["free_order"].tolist())
+        self.tables = []
+        for L in ctx:
+            seq = Sequence()
+            append_tokens(pool, seq, int(L))
+            self.tables.append(np.array(seq.block_table, np.int64))
+        self.ctx = ctx
+
+
+def oracle_sample(ob: OracleBatch, budget_s: float, start_seq: int = 0):
+    """Times the oracle (as it stands, single-threaded float64 C) on whole
+    sequences of the batch, from start_seq on, until budget_s of oracle time
+    is spent. Returns (bytes, seconds, sequences). Widening the inputs to
+    float64 is outside the timed calls."""
     import oracle
-    oracle.build()
-    if "k_pool" not in b.host_inputs:
-        raise SystemExit("the CPU oracle legs time the decode-only workloads")
-    k = b.host_inputs["k_pool"]
-    v = b.host_inputs["v_pool"]
-    q = b.host_inputs["query"]
+    spec = ob.spec
+    k, v, q = ob.inputs["k_pool"], ob.inputs["v_pool"], ob.inputs["query"]
     tot_bytes, tot_s, n_seq = 0, 0.0, 0
-    S = len(b.host_context_lens)
+    S = len(ob.ctx)
     s = start_seq
     while tot_s < budget_s and n_seq < S:
-        L = int(b.host_context_lens[s % S])
-        nb = (L + spec.block_size - 1) // spec.block_size
-        ids = torch.from_numpy(b.host_tables[s % S, :nb].astype(np.int64))
+        i = s % S
+        L = int(ob.ctx[i])
+        ids = torch.from_numpy(ob.tables[i])
         kp = k.index_select(0, ids).double().numpy()
         vp = v.index_select(0, ids).double().numpy()
-        qs = q[s % S:s % S + 1].double().numpy()
-        tab = np.arange(max(nb, 1), dtype=np.int32)[None, :]
+        qs = q[i:i + 1].double().numpy()
+        tab = np.arange(max(len(ids), 1), dtype=np.int32)[None, :]
         t = time.perf_counter()
         oracle.paged_decode(qs, kp, vp, tab, np.array([L], np.int32), spec.scale, spec.block_size)
         tot_s += time.perf_counter() - t
@@ -369,16 +370,20 @@ def oracle_sample(spec, b, budget_s: float, start_seq: int = 0):
 
 def run_reference(args, world, rank):
     """Reference arm: the CPU oracle, timed on the host cores, on the same
-    workload, metric and unit. Rank 0 only."""
+    workload, metric and unit. Rank 0 only; no GPU is used."""
     if rank != 0:
         return
-    spec, b = build_batch(args.workload, 0)
+    from paged_kv_cache_340_b200.workloads import SPECS
+    spec = SPECS[args.workload]
+    if spec.lengths[0] == "parallel":
+        raise SystemExit("the reference arm times the decode-only workloads")
+    ob = OracleBatch(spec)
     budget = max(0.002, min(2.0, 90.0 / max(1, args.steps + args.warmup)))
-    for _ in range(args.warmup):
-        oracle_sample(spec, b, budget / 4)
+    for i in range(args.warmup):
+        oracle_sample(ob, budget / 4, start_seq=i)
     tot_b, tot_s, seqs = 0, 0.0, 0
     for i in range(args.steps):
-        nb_, ns_, nq_ = oracle_sample(spec, b, budget, start_seq=i)
+        nb_, ns_, nq_ = oracle_sample(ob, budget, start_seq=i)
         tot_b += nb_
         tot_s += ns_
         seqs += nq_
@@ -427,10 +432,12 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
-    world, rank, local = dist_setup(args.gpus)
     if args.impl == "reference":
+        # The reference arm runs on the host: rank 0 alone, no process group.
+        world, rank, _ = pdist.env_ranks()
         run_reference(args, world, rank)
         return
+    world, rank, local = dist_setup(args.gpus)
     import paged_kv_cache_340_b200 as pa  # noqa: F401  (fails loudly without the CUDA library)
 
     spec, b = build_batch(args.workload, rank, args.partition)
@@ -438,7 +445,7 @@ def main():
                                             device_index=local)
     by = step_bytes(spec, b)
     peak, peak_kind = peaks()
-    value = world * by["total"] / (ms * 1e-3) / 1e9
+    value = pdist.job_throughput(by["total"], ms, world)
     e2e_ms, h2d, d2h = e2e_steps(b, max(10, args.steps // 4), args.warmup, world)
     kernel = "pa_decode_splitk" if b.partition_size else "pa_decode"
     achieved = by["decode"] / (dec_ms * 1e-3) / 1e9
@@ -457,7 +464,7 @@ def main():
         "seq_tokens_per_s": round(world * spec.num_seqs / (ms * 1e-3), 1),
         "context_tokens_per_s": round(world * float(b.host_context_lens.sum()) / (ms * 1e-3), 1),
         "bytes_per_step": by,
-        "e2e": {"value": round(world * by["total"] / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(pdist.job_throughput(by["total"], e2e_ms, world), 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1), "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
@@ -468,8 +475,8 @@ def main():
     }
     if b.partition_size:
         line["roofline"]["reduce_kernel_ms"] = round(red_ms, 5)
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        nbytes, secs, nseq = oracle_sample(spec, b, 12.0)
+    if world == 1 and rank == 0 and not args.no_cpu_baseline and "k_pool" in b.host_inputs:
+        nbytes, secs, nseq = oracle_sample(OracleBatch(spec, b.host_inputs), 12.0)
         line["cpu_baseline"] = {"value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{nseq} of {spec.num_seqs} sequences (all heads), decode only; "
                                           f"float64 C oracle, one thread, {secs:.1f} s"}
@@ -480,9 +487,7 @@ def main():
                                    ("gqa_bf16", "long_splitk_bf16", "parallel_sampling_fp16")}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    pdist.finalize(world)
 
 
 if __name__ == "__main__":
