@@ -237,14 +237,14 @@ def time_steps(b, steps: int, warmup: int, world: int, sample_clocks=False, devi
             ev[0].record(stream)
         if b.partition_size:
             pa_decode_splitk(b.workspace, b.query, b.k_cache, b.v_cache, b.block_tables, b.context_lens, spec.scale,
-                             b.max_context_len, b.partition_size, stream=stream)
+                             b.max_context_len, b.partition_size, seq_order=b.seq_order, stream=stream)
             if ev is not None:
                 ev[1].record(stream)
             pa_splitk_reduce(b.out, b.workspace, b.context_lens, b.max_context_len, b.partition_size,
                              stream=stream)
         else:
             pa_decode(b.out, b.query, b.k_cache, b.v_cache, b.block_tables, b.context_lens, spec.scale,
-                      stream=stream)
+                      seq_order=b.seq_order, stream=stream)
             if ev is not None:
                 ev[1].record(stream)
         if ev is not None:
@@ -288,7 +288,7 @@ def e2e_steps(b, steps: int, warmup: int, world: int):
     from paged_kv_cache_340_b200.batch import run_step
     stream = torch.cuda.current_stream()
     host_in = [(t.cpu().pin_memory(), t) for t in (b.query, b.new_key, b.new_value, b.slot_mapping, b.block_tables,
-                                                    b.context_lens, b.cow_pairs) if t.numel()]
+                                                    b.context_lens, b.seq_order, b.cow_pairs) if t.numel()]
     host_out = torch.empty(b.out.shape, dtype=b.out.dtype, pin_memory=True)
     h2d = sum(h.numel() * h.element_size() for h, _ in host_in)
     d2h = host_out.numel() * host_out.element_size()

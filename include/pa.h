@@ -116,12 +116,19 @@ int pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void
  * [P4] §3.1 (index-based kernel over key_cache/value_cache
  * [num_blocks, num_kv_heads, block_size, head_dim]); [P5] §3.2 (inputs
  * query, key_cache, value_cache, block_tables, context_lens, scale).
+ *
+ * seq_order (nullable device int32 [num_seqs], a permutation of
+ * 0 .. num_seqs-1) is the order in which sequences are scheduled on the GPU;
+ * it changes no result. Work is handed to SMs roughly in this order, so
+ * listing sequences longest first keeps a long sequence from starting last
+ * and finishing alone. Entries outside [0, num_seqs) are skipped
+ * (PA_DEVERR_CONTEXT). NULL schedules 0, 1, 2, ...
  */
 int pa_decode(void *out, const void *query, const void *k_cache, const void *v_cache,
               const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
               int num_seqs, int num_heads, int num_kv_heads, int head_dim, float scale,
               int block_size, int num_blocks, pa_dtype kv_dtype, pa_dtype out_dtype,
-              cudaStream_t stream);
+              const int32_t *seq_order, cudaStream_t stream);
 
 /*
  * Split-K (partitioned) decode for few, long sequences ([P5] §2.3: the
@@ -142,7 +149,8 @@ int pa_decode(void *out, const void *query, const void *k_cache, const void *v_c
  * pa_splitk_reduce then merges them by log-sum-exp:
  *   M = max_p m_p,  out = sum_p e^(m_p - M) acc_p / sum_p e^(m_p - M) l_p
  * (the standard split of the softmax; the pages only name the partitioned
- * kernel). Both calls must get the same sizes.
+ * kernel). Both calls must get the same sizes. seq_order (nullable) is the
+ * scheduling order of sequences, as for pa_decode.
  */
 size_t pa_splitk_workspace_bytes(int num_seqs, int num_heads, int head_dim, int max_context_len,
                                  int partition_size);
@@ -153,7 +161,7 @@ int pa_decode_splitk(void *workspace, size_t workspace_bytes, const void *query,
                      int max_blocks_per_seq, const int32_t *context_lens, int num_seqs,
                      int num_heads, int num_kv_heads, int head_dim, float scale, int block_size,
                      int num_blocks, int max_context_len, int partition_size, pa_dtype kv_dtype,
-                     cudaStream_t stream);
+                     const int32_t *seq_order, cudaStream_t stream);
 
 int pa_splitk_reduce(void *out, const void *workspace, size_t workspace_bytes,
                      const int32_t *context_lens, int num_seqs, int num_heads, int head_dim,

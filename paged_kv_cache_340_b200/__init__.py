@@ -61,11 +61,11 @@ def _load() -> ctypes.CDLL:
         "pa_status_string": (ctypes.c_char_p, [i32]),
         "pa_read_device_errors": (i32, [ctypes.POINTER(ctypes.c_uint32), vp]),
         "pa_reshape_and_cache": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
-        "pa_decode": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32, vp]),
+        "pa_decode": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32, vp, vp]),
         "pa_splitk_workspace_bytes": (sz, [i32, i32, i32, i32, i32]),
         "pa_splitk_acc_offset": (sz, [i32, i32, i32, i32]),
         "pa_decode_splitk": (i32, [vp, sz, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32,
-                                   i32, vp]),
+                                   i32, vp, vp]),
         "pa_splitk_reduce": (i32, [vp, vp, sz, vp, i32, i32, i32, i32, i32, i32, vp]),
         "pa_choose_partition": (i32, [i32, i32, i32, i32, i32, i32]),
         "pa_copy_blocks": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
@@ -146,12 +146,13 @@ def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None
     _check(rc, "pa_reshape_and_cache")
 
 
-def pa_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale, stream=None) -> None:
+def pa_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale, seq_order=None,
+              stream=None) -> None:
     S, Hq, D = query.shape
     NB, Hkv, bs, _ = k_cache.shape
     rc = _lib.pa_decode(_ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                         block_tables.shape[1], _ptr(context_lens), S, Hq, Hkv, D, float(scale), bs, NB,
-                        _dtype(k_cache), _dtype(out), _stream(stream))
+                        _dtype(k_cache), _dtype(out), _ptr(seq_order), _stream(stream))
     _check(rc, "pa_decode")
 
 
@@ -164,13 +165,13 @@ def pa_splitk_acc_offset(num_seqs, num_heads, max_context_len, partition_size) -
 
 
 def pa_decode_splitk(workspace, query, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
-                     partition_size, stream=None) -> None:
+                     partition_size, seq_order=None, stream=None) -> None:
     S, Hq, D = query.shape
     NB, Hkv, bs, _ = k_cache.shape
     rc = _lib.pa_decode_splitk(_ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(query),
                                _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1],
                                _ptr(context_lens), S, Hq, Hkv, D, float(scale), bs, NB, int(max_context_len),
-                               int(partition_size), _dtype(k_cache), _stream(stream))
+                               int(partition_size), _dtype(k_cache), _ptr(seq_order), _stream(stream))
     _check(rc, "pa_decode_splitk")
 
 

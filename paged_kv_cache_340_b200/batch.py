@@ -34,6 +34,7 @@ class DecodeBatch:
     new_value: torch.Tensor
     slot_mapping: torch.Tensor  # device int32 [T]
     cow_pairs: torch.Tensor     # device int64 [n, 2] (n may be 0)
+    seq_order: torch.Tensor     # device int32 [S]: sequences longest first (scheduling order)
     max_context_len: int
     partition_size: int         # 0 = unpartitioned
     workspace: Optional[torch.Tensor]
@@ -45,6 +46,23 @@ class DecodeBatch:
 
 def _blocks(n: int, bs: int) -> int:
     return (n + bs - 1) // bs
+
+
+def longest_first(ctx: np.ndarray) -> np.ndarray:
+    """Sequence indices by decreasing context length (ties in index order):
+    the scheduling order that keeps a long sequence from starting last."""
+    return np.argsort(-ctx.astype(np.int64), kind="stable").astype(np.int32)
+
+
+def groups_longest_first(ctx: np.ndarray, group: int) -> np.ndarray:
+    """Like longest_first, but sequences that share a prefix (consecutive
+    groups of `group`) stay together, so the shared blocks are read while they
+    are still in L2: groups by their longest member, members longest first."""
+    g = ctx.reshape(-1, group).astype(np.int64)
+    order = []
+    for gi in np.argsort(-g.max(axis=1), kind="stable"):
+        order += [gi * group + j for j in np.argsort(-g[gi], kind="stable")]
+    return np.array(order, np.int32)
 
 
 def build_decode_batch(spec: Spec, inputs: dict, device="cuda", partition_size: Optional[int] = None,
@@ -83,6 +101,7 @@ def build_decode_batch(spec: Spec, inputs: dict, device="cuda", partition_size: 
         new_key=inputs["new_key"].to(dev), new_value=inputs["new_value"].to(dev),
         slot_mapping=torch.from_numpy(slots).to(dev),
         cow_pairs=torch.empty((0, 2), dtype=torch.int64, device=dev),
+        seq_order=torch.from_numpy(longest_first(ctx)).to(dev),
         max_context_len=max_ctx, partition_size=int(partition_size), workspace=ws,
         host_tables=tables, host_slots=slots, host_cow=np.empty((0, 2), np.int64), host_context_lens=ctx)
 
@@ -148,6 +167,7 @@ def build_parallel_sampling_batch(spec: Spec, inputs: dict, device="cuda", parti
         block_tables=torch.from_numpy(tables).to(dev), context_lens=torch.from_numpy(ctx).to(dev),
         new_key=inputs["divergent_key"].to(dev), new_value=inputs["divergent_value"].to(dev),
         slot_mapping=torch.from_numpy(slots).to(dev), cow_pairs=torch.from_numpy(cow_all).to(dev),
+        seq_order=torch.from_numpy(groups_longest_first(ctx, B)).to(dev),
         max_context_len=max_ctx, partition_size=int(partition_size), workspace=ws,
         host_tables=tables, host_slots=slots, host_cow=cow_all, host_context_lens=ctx,
         prefix_key=inputs["prefix_key"].reshape(P * L0, Hkv, D).to(dev),
@@ -176,9 +196,10 @@ def run_decode(batch: DecodeBatch, stream=None) -> None:
     spec = batch.spec
     if batch.partition_size:
         pa_decode_splitk(batch.workspace, batch.query, batch.k_cache, batch.v_cache, batch.block_tables,
-                         batch.context_lens, spec.scale, batch.max_context_len, batch.partition_size, stream=stream)
+                         batch.context_lens, spec.scale, batch.max_context_len, batch.partition_size,
+                         seq_order=batch.seq_order, stream=stream)
         pa_splitk_reduce(batch.out, batch.workspace, batch.context_lens, batch.max_context_len,
                          batch.partition_size, stream=stream)
     else:
         pa_decode(batch.out, batch.query, batch.k_cache, batch.v_cache, batch.block_tables, batch.context_lens,
-                  spec.scale, stream=stream)
+                  spec.scale, seq_order=batch.seq_order, stream=stream)

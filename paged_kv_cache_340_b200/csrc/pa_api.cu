@@ -170,13 +170,14 @@ int pa_decode(void *out, const void *query, const void *k_cache, const void *v_c
               const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
               int num_seqs, int num_heads, int num_kv_heads, int head_dim, float scale,
               int block_size, int num_blocks, pa_dtype kv_dtype, pa_dtype out_dtype,
-              cudaStream_t stream) {
+              const int32_t *seq_order, cudaStream_t stream) {
     int rc = check_decode_args(query, k_cache, v_cache, block_tables, max_blocks_per_seq,
                                context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale,
                                block_size, num_blocks, kv_dtype);
     if (rc != PA_OK) return rc;
     if (out_dtype != kv_dtype && out_dtype != PA_F32) return PA_ERR_DTYPE;
     if (num_seqs == 0) return PA_OK;
+    if (!aligned(seq_order, 4)) return PA_ERR_ALIGN;
     if (!out) return PA_ERR_NULL;
     if (!aligned(out, 16)) return PA_ERR_ALIGN;
     unsigned int *err = nullptr;
@@ -188,6 +189,7 @@ int pa_decode(void *out, const void *query, const void *k_cache, const void *v_c
     p.v_cache = v_cache;
     p.block_tables = block_tables;
     p.context_lens = context_lens;
+    p.seq_order = seq_order;
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.num_heads = num_heads;
     p.num_kv_heads = num_kv_heads;
@@ -224,7 +226,7 @@ int pa_decode_splitk(void *workspace, size_t workspace_bytes, const void *query,
                      int max_blocks_per_seq, const int32_t *context_lens, int num_seqs,
                      int num_heads, int num_kv_heads, int head_dim, float scale, int block_size,
                      int num_blocks, int max_context_len, int partition_size, pa_dtype kv_dtype,
-                     cudaStream_t stream) {
+                     const int32_t *seq_order, cudaStream_t stream) {
     int rc = check_decode_args(query, k_cache, v_cache, block_tables, max_blocks_per_seq,
                                context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale,
                                block_size, num_blocks, kv_dtype);
@@ -232,6 +234,7 @@ int pa_decode_splitk(void *workspace, size_t workspace_bytes, const void *query,
     if (max_context_len < 0) return PA_ERR_SHAPE;
     if (partition_size <= 0 || partition_size % block_size != 0) return PA_ERR_PARTITION;
     if (num_seqs == 0 || max_context_len == 0) return PA_OK;
+    if (!aligned(seq_order, 4)) return PA_ERR_ALIGN;
     const size_t need = pa_splitk_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len,
                                                   partition_size);
     if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE;
@@ -249,6 +252,7 @@ int pa_decode_splitk(void *workspace, size_t workspace_bytes, const void *query,
     p.v_cache = v_cache;
     p.block_tables = block_tables;
     p.context_lens = context_lens;
+    p.seq_order = seq_order;
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.num_heads = num_heads;
     p.num_kv_heads = num_kv_heads;

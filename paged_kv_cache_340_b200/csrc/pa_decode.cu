@@ -496,10 +496,14 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
 
     const int part = blockIdx.x;
     const int kvh = blockIdx.y;
-    const int s = blockIdx.z;
+    const int s = p.seq_order ? p.seq_order[blockIdx.z] : (int)blockIdx.z;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const bool split = p.partition_size > 0;
+    if (s < 0 || s >= (int)gridDim.z) {  // a bad schedule entry: nothing to do for it
+        if (threadIdx.x == 0 && part == 0 && kvh == 0) record_error(p.err, PA_DEVERR_CONTEXT);
+        return;
+    }
 
     // ---- token range of this CTA
     int ctx = p.context_lens[s];

@@ -18,6 +18,7 @@ struct DecodeParams {
     const void *v_cache;
     const int32_t *block_tables;
     const int32_t *context_lens;
+    const int32_t *seq_order;  // nullable: CTA row z serves sequence seq_order[z]
     int max_blocks_per_seq;
     int num_heads;
     int num_kv_heads;

@@ -73,7 +73,7 @@ extern "C" int pa_decode_splitk_static(void *out, const void *query, const void 
     int rc = pa_decode_splitk(scratch, (size_t)PA_STATIC_SCRATCH_BYTES, query, k_cache, v_cache,
                               block_tables, max_blocks_per_seq, context_lens, num_seqs, num_heads,
                               num_kv_heads, head_dim, scale, block_size, num_blocks,
-                              max_context_len, partition_size, kv_dtype, stream);
+                              max_context_len, partition_size, kv_dtype, nullptr, stream);
     if (rc != PA_OK) return rc;
     return pa_splitk_reduce(out, scratch, (size_t)PA_STATIC_SCRATCH_BYTES, context_lens, num_seqs,
                             num_heads, head_dim, max_context_len, partition_size, out_dtype,

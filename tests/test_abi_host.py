@@ -87,12 +87,12 @@ def test_decode_host_checks(pa, kw, code):
     rc = pa._lib.pa_decode(args["out"], args["query"], args["k_cache"], args["v_cache"], args["block_tables"],
                            args["max_blocks"], args["context_lens"], args["num_seqs"], args["num_heads"],
                            args["num_kv_heads"], args["head_dim"], args["scale"], args["block_size"],
-                           args["num_blocks"], args["kv_dtype"], args["out_dtype"], None)
+                           args["num_blocks"], args["kv_dtype"], args["out_dtype"], None, None)
     assert rc == code
 
 
 def test_empty_batches_are_no_ops(pa):
-    assert pa._lib.pa_decode(None, None, None, None, None, 0, None, 0, 8, 8, 128, 0.1, 16, 0, 1, 1, None) == 0
+    assert pa._lib.pa_decode(None, None, None, None, None, 0, None, 0, 8, 8, 128, 0.1, 16, 0, 1, 1, None, None) == 0
     assert pa._lib.pa_reshape_and_cache(None, None, None, None, None, 0, 4, 8, 128, 16, 1, None) == 0
     assert pa._lib.pa_copy_blocks(None, None, None, 0, 4, 8, 128, 16, 1, None) == 0
 
@@ -100,14 +100,15 @@ def test_empty_batches_are_no_ops(pa):
 def test_splitk_host_checks(pa):
     f = pa._lib.pa_decode_splitk
     base = [A16, 1 << 30, A16, A16, A16, A16, 4, A16, 2, 8, 8, 128, 0.1, 16, 8, 64]
-    assert f(*(base + [24, 1, None])) == -8       # partition not a multiple of the block size
-    assert f(*(base + [0, 1, None])) == -8
+    assert f(*(base + [24, 1, None, None])) == -8       # partition not a multiple of the block size
+    assert f(*(base + [0, 1, None, None])) == -8
     small = list(base)
     small[1] = 16
-    assert f(*(small + [32, 1, None])) == -9      # workspace too small
+    assert f(*(small + [32, 1, None, None])) == -9      # workspace too small
     nows = list(base)
     nows[0] = None
-    assert f(*(nows + [32, 1, None])) == -9
+    assert f(*(nows + [32, 1, None, None])) == -9
+    assert f(*(base + [32, 1, A16 + 2, None])) == -7    # misaligned schedule
 
 
 # ------------------------------------------------------ pool vs oracle pool

@@ -181,6 +181,36 @@ def test_permutation_of_physical_ids_is_bit_invariant(pa):
     assert torch.equal(out, out2)
 
 
+@pytest.mark.parametrize("partition", [0, 64])
+def test_schedule_order_changes_nothing(pa, partition):
+    """seq_order only reorders the work: any permutation gives bit-identical
+    outputs; an entry outside [0, num_seqs) is skipped and flagged."""
+    ctx = [40, 700, 3, 129, 0, 260]
+    c = Case(pa, torch.bfloat16, len(ctx), 8, 2, 128, 16, ctx, seed=21, out_dtype=torch.float32)
+    d, out = _run_write_and_decode(pa, c, partition)
+    for perm in ([5, 4, 3, 2, 1, 0], [1, 5, 3, 0, 2, 4]):
+        order = torch.tensor(perm, dtype=torch.int32, device="cuda")
+        out2 = torch.empty_like(out)
+        if partition:
+            mx = int(c.ctx.max())
+            ws = torch.empty(pa.pa_splitk_workspace_bytes(len(ctx), 8, 128, mx, partition), dtype=torch.uint8,
+                             device="cuda")
+            pa.pa_decode_splitk(ws, d["q"], d["k"], d["v"], d["bt"], d["cl"], c.scale, mx, partition,
+                                seq_order=order)
+            pa.pa_splitk_reduce(out2, ws, d["cl"], mx, partition)
+        else:
+            pa.pa_decode(out2, d["q"], d["k"], d["v"], d["bt"], d["cl"], c.scale, seq_order=order)
+        torch.cuda.synchronize()
+        assert pa.pa_read_device_errors() == 0
+        assert torch.equal(out, out2)
+    if not partition:
+        bad = torch.tensor([0, 1, 2, 3, 4, 9], dtype=torch.int32, device="cuda")
+        out3 = torch.full_like(out, 7.0)
+        pa.pa_decode(out3, d["q"], d["k"], d["v"], d["bt"], d["cl"], c.scale, seq_order=bad)
+        assert pa.pa_read_device_errors() & pa.PA_DEVERR_CONTEXT
+        assert torch.equal(out3[:5], out[:5]) and torch.all(out3[5] == 7.0)
+
+
 def test_splitk_partials_match_oracle(pa):
     ctx = [100, 1000, 31, 64]
     P = 128
