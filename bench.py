@@ -282,37 +282,30 @@ def time_steps(b, steps: int, warmup: int, world: int, sample_clocks=False, devi
 
 
 def e2e_steps(b, steps: int, warmup: int, world: int):
-    """The same step through the public API with host buffers: every step
-    copies its inputs from pinned host memory (query, new K/V, slots, block
-    tables, context lengths) and reads the output back to pinned memory."""
-    from paged_kv_cache_340_b200.batch import run_step
+    """The same step through the public host-buffer API (HostStepPipeline):
+    every step copies its inputs from pinned host memory (query, new K/V,
+    slots, block tables, context lengths, schedule) and reads its output back
+    into pinned memory; copies of neighbouring steps overlap the kernels."""
+    from paged_kv_cache_340_b200.batch import HostStepPipeline
     stream = torch.cuda.current_stream()
-    host_in = [(t.cpu().pin_memory(), t) for t in (b.query, b.new_key, b.new_value, b.slot_mapping, b.block_tables,
-                                                    b.context_lens, b.seq_order, b.cow_pairs) if t.numel()]
-    host_out = torch.empty(b.out.shape, dtype=b.out.dtype, pin_memory=True)
-    h2d = sum(h.numel() * h.element_size() for h, _ in host_in)
-    d2h = host_out.numel() * host_out.element_size()
-
-    def one():
-        for h, d in host_in:
-            d.copy_(h, non_blocking=True)
-        run_step(b, stream=stream)
-        host_out.copy_(b.out, non_blocking=True)
-
+    pipe = HostStepPipeline(b)
     for _ in range(warmup):
-        one()
+        pipe.step(stream)
+    pipe.drain(stream)
     torch.cuda.synchronize()
     barrier(world)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
+    pipe.start(stream)
     for _ in range(steps):
-        one()
+        pipe.step(stream)
+    pipe.drain(stream)
     t1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(t0.elapsed_time(t1), world) / steps
-    return ms, h2d, d2h
+    return ms, pipe.h2d_bytes, pipe.d2h_bytes
 
 
 # ---------------------------------------------------------- CPU oracle legs

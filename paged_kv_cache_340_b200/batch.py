@@ -203,3 +203,89 @@ def run_decode(batch: DecodeBatch, stream=None) -> None:
     else:
         pa_decode(batch.out, batch.query, batch.k_cache, batch.v_cache, batch.block_tables, batch.context_lens,
                   spec.scale, seq_order=batch.seq_order, stream=stream)
+
+
+class HostStepPipeline:
+    """Decode steps driven from pinned host buffers, with the copies of one
+    step overlapping the kernels of its neighbours.
+
+    Each step copies its inputs (query, new K/V, slots, block tables, context
+    lengths, schedule and copy-on-write pairs) host -> device, runs the hot
+    path (run_step) and copies the output back. Device inputs and outputs are
+    double-buffered: step i's host->device copies run on a copy stream while
+    step i-1 computes, and step i-1's output returns on a second copy stream
+    while step i computes. The KV pools stay resident on the device.
+    """
+
+    _IN = ("query", "new_key", "new_value", "slot_mapping", "block_tables", "context_lens", "seq_order",
+           "cow_pairs")
+
+    def __init__(self, batch: DecodeBatch):
+        import copy
+        self.batch = batch
+        self.names = [n for n in self._IN if getattr(batch, n).numel()]
+        self.host_in = {n: getattr(batch, n).cpu().pin_memory() for n in self.names}
+        self.host_out = [torch.empty(batch.out.shape, dtype=batch.out.dtype, pin_memory=True) for _ in range(2)]
+        self.views = []
+        for _ in range(2):
+            v = copy.copy(batch)
+            for n in self.names:
+                setattr(v, n, torch.empty_like(getattr(batch, n)))
+            v.out = torch.empty_like(batch.out)
+            if batch.workspace is not None:
+                v.workspace = torch.empty_like(batch.workspace)
+            self.views.append(v)
+        self.h2d = torch.cuda.Stream()
+        self.d2h = torch.cuda.Stream()
+        self.in_ready = [torch.cuda.Event() for _ in range(2)]
+        self.in_free = [torch.cuda.Event() for _ in range(2)]
+        self.out_ready = [torch.cuda.Event() for _ in range(2)]
+        self.out_free = [torch.cuda.Event() for _ in range(2)]
+        self.i = 0
+
+    @property
+    def h2d_bytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in self.host_in.values())
+
+    @property
+    def d2h_bytes(self) -> int:
+        return self.host_out[0].numel() * self.host_out[0].element_size()
+
+    def start(self, stream=None) -> None:
+        """Orders the copy streams after everything already on `stream` (e.g.
+        a timing event), so that no copy of the next step starts before it."""
+        comp = stream or torch.cuda.current_stream()
+        self.h2d.wait_stream(comp)
+        self.d2h.wait_stream(comp)
+
+    def step(self, stream=None) -> torch.Tensor:
+        """Enqueues one step; returns the pinned host tensor that will hold its
+        output once the stream work completes."""
+        comp = stream or torch.cuda.current_stream()
+        j = self.i & 1
+        v = self.views[j]
+        if self.i >= 2:
+            self.h2d.wait_event(self.in_free[j])
+        with torch.cuda.stream(self.h2d):
+            for n in self.names:
+                getattr(v, n).copy_(self.host_in[n], non_blocking=True)
+            self.in_ready[j].record(self.h2d)
+        comp.wait_event(self.in_ready[j])
+        if self.i >= 2:
+            comp.wait_event(self.out_free[j])
+        run_step(v, stream=comp)
+        self.in_free[j].record(comp)
+        self.out_ready[j].record(comp)
+        self.d2h.wait_event(self.out_ready[j])
+        with torch.cuda.stream(self.d2h):
+            self.host_out[j].copy_(v.out, non_blocking=True)
+            self.out_free[j].record(self.d2h)
+        self.i += 1
+        return self.host_out[j]
+
+    def drain(self, stream=None) -> None:
+        """Makes `stream` wait for every copy enqueued so far."""
+        comp = stream or torch.cuda.current_stream()
+        for j in range(2):
+            if self.i > j:
+                comp.wait_event(self.out_free[j])

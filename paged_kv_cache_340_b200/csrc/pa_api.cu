@@ -282,7 +282,6 @@ int pa_splitk_reduce(void *out, const void *workspace, size_t workspace_bytes,
     if (!out || !context_lens) return PA_ERR_NULL;
     if (!aligned(out, 16) || !aligned(context_lens, 4)) return PA_ERR_ALIGN;
     const int mp = max_parts_of(max_context_len, partition_size);
-    if ((size_t)mp * sizeof(float) > 200 * 1024) return PA_ERR_SHAPE;
     const size_t need = pa_splitk_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len,
                                                   partition_size);
     if (mp > 0 && (!workspace || workspace_bytes < need)) return PA_ERR_WORKSPACE;

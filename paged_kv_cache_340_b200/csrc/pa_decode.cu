@@ -595,6 +595,8 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
         }
         const int k = warp + S::kWarps * m;
         const int buf = k % S::kStages;
+        // Lane 0 polls the barrier (32 lanes polling would serialise on it);
+        // __syncwarp then orders the other lanes' reads after its acquire.
         const bool got = mbar_wait(full + buf, (k / S::kStages) & 1);
         if (!__all_sync(0xffffffffu, got)) {
             if (lane == 0) record_error(p.err, PA_DEVERR_TIMEOUT);
@@ -660,52 +662,76 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
 
 // -------------------------------------------------------------- split reduce
 
-__global__ void __launch_bounds__(128)
+// One CTA of 8 warps per (sequence, query head): warp w folds partitions
+// w, w + 8, ... (each lane holding 4 consecutive head dims as one float4, so
+// a partition row is one coalesced 512-byte read), then the warps combine
+// through shared memory.
+constexpr int kReduceWarps = 8;
+
+__global__ void __launch_bounds__(kReduceWarps * 32)
     splitk_reduce_kernel(void *out, const float *ws_ml, const float *ws_acc,
                          const int32_t *context_lens, int num_heads, int head_dim,
                          int partition_size, int max_parts, int max_context_len,
                          pa_dtype out_dtype) {
-    extern __shared__ float wsm[];  // [max_parts] weights
-    __shared__ float red[4];
-    __shared__ float bcast;
+    __shared__ float red_l[kReduceWarps];
+    __shared__ float4 red_acc[kReduceWarps][32];
     const int h = blockIdx.x;
     const int s = blockIdx.y;
-    const int tid = threadIdx.x;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
     int ctx = context_lens[s];
     ctx = max(0, min(ctx, max_context_len));
     const int n = (ctx + partition_size - 1) / partition_size;
     const size_t row = (size_t)s * num_heads + h;
+    const int vec = head_dim / 4;  // float4 per partition row (16 or 32)
     if (n == 0) {
-        for (int d = tid; d < head_dim; d += blockDim.x) store_out(out, row * head_dim + d, 0.f, out_dtype);
+        for (int d = threadIdx.x; d < head_dim; d += blockDim.x) store_out(out, row * head_dim + d, 0.f, out_dtype);
         return;
     }
     const float *ml = ws_ml + row * max_parts * 2;
-    const float *acc = ws_acc + row * max_parts * head_dim;
-    // M = max_p m_p
+    const float4 *acc = reinterpret_cast<const float4 *>(ws_acc + row * max_parts * head_dim);
+    // M = max_p m_p (every warp computes it; n is small)
     float M = -INFINITY;
-    for (int i = tid; i < n; i += blockDim.x) M = fmaxf(M, ml[2 * i]);
+    for (int i = lane; i < n; i += 32) M = fmaxf(M, ml[2 * i]);
+#pragma unroll
     for (int mk = 16; mk >= 1; mk >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, mk));
-    if ((tid & 31) == 0) red[tid >> 5] = M;
-    __syncthreads();
-    if (tid == 0) bcast = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    __syncthreads();
-    M = bcast;
-    // w_p = e^(m_p - M); den = sum_p w_p l_p
+    // this warp's partitions: weights e^(m_p - M), sum of w l, sum of w acc
     float den = 0.f;
-    for (int i = tid; i < n; i += blockDim.x) {
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = warp; i < n; i += kReduceWarps) {
         const float w = fast_exp2((ml[2 * i] - M) * kLog2e);
-        wsm[i] = w;
         den = fmaf(w, ml[2 * i + 1], den);
+        if (lane < vec) {
+            const float4 a = acc[(size_t)i * vec + lane];
+            num.x = fmaf(w, a.x, num.x);
+            num.y = fmaf(w, a.y, num.y);
+            num.z = fmaf(w, a.z, num.z);
+            num.w = fmaf(w, a.w, num.w);
+        }
     }
-    for (int mk = 16; mk >= 1; mk >>= 1) den += __shfl_xor_sync(0xffffffffu, den, mk);
-    __syncthreads();  // red[] reuse and wsm[] visibility
-    if ((tid & 31) == 0) red[tid >> 5] = den;
+    if (lane == 0) red_l[warp] = den;
+    red_acc[warp][lane] = num;
     __syncthreads();
-    den = red[0] + red[1] + red[2] + red[3];
-    for (int d = tid; d < head_dim; d += blockDim.x) {
-        float num = 0.f;
-        for (int i = 0; i < n; ++i) num = fmaf(wsm[i], acc[(size_t)i * head_dim + d], num);
-        store_out(out, row * head_dim + d, den > 0.f ? num / den : 0.f, out_dtype);
+    if (warp == 0) {
+        float dsum = 0.f;
+        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kReduceWarps; ++w) {
+            dsum += red_l[w];
+            const float4 a = red_acc[w][lane];
+            t.x += a.x;
+            t.y += a.y;
+            t.z += a.z;
+            t.w += a.w;
+        }
+        if (lane < vec) {
+            const float inv = dsum > 0.f ? 1.f / dsum : 0.f;
+            const size_t o = row * head_dim + 4 * lane;
+            store_out(out, o + 0, t.x * inv, out_dtype);
+            store_out(out, o + 1, t.y * inv, out_dtype);
+            store_out(out, o + 2, t.z * inv, out_dtype);
+            store_out(out, o + 3, t.w * inv, out_dtype);
+        }
     }
 }
 
@@ -761,17 +787,10 @@ cudaError_t launch_splitk_reduce(void *out, const float *ws_ml, const float *ws_
                                  const int32_t *context_lens, int num_seqs, int num_heads,
                                  int head_dim, int partition_size, int max_parts,
                                  int max_context_len, pa_dtype out_dtype, cudaStream_t stream) {
-    const size_t smem = (size_t)max_parts * sizeof(float);
-    if (smem > 48 * 1024) {
-        static unsigned int attr_done = 0;
-        cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(splitk_reduce_kernel),
-                                         227 * 1024, &attr_done);
-        if (e != cudaSuccess) return e;
-    }
     dim3 grid(num_heads, num_seqs);
-    splitk_reduce_kernel<<<grid, 128, smem, stream>>>(out, ws_ml, ws_acc, context_lens, num_heads,
-                                                      head_dim, partition_size, max_parts,
-                                                      max_context_len, out_dtype);
+    splitk_reduce_kernel<<<grid, kReduceWarps * 32, 0, stream>>>(out, ws_ml, ws_acc, context_lens,
+                                                                 num_heads, head_dim, partition_size,
+                                                                 max_parts, max_context_len, out_dtype);
     return cudaGetLastError();
 }
 

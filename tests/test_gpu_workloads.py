@@ -139,3 +139,23 @@ def test_parallel_sampling_fp16(pa):
     run_step(batch)
     torch.cuda.synchronize()
     assert torch.equal(out1, batch.out)
+
+
+def test_host_buffer_pipeline_matches_the_plain_step(pa):
+    """HostStepPipeline (inputs from pinned host memory, output back to host,
+    copies overlapping neighbouring steps) returns exactly what the plain
+    device-resident step computes."""
+    from paged_kv_cache_340_b200.batch import HostStepPipeline, build_decode_batch, run_step
+    from paged_kv_cache_340_b200.workloads import SPECS, make_decode_inputs, scaled
+    spec = scaled(SPECS["gqa_bf16"], num_seqs=32)
+    b = build_decode_batch(spec, make_decode_inputs(spec))
+    run_step(b)
+    torch.cuda.synchronize()
+    ref = b.out.cpu()
+    pipe = HostStepPipeline(b)
+    outs = [pipe.step() for _ in range(5)]
+    pipe.drain()
+    torch.cuda.synchronize()
+    for o in outs[-2:]:
+        assert torch.equal(o, ref)
+    assert pipe.h2d_bytes > 0 and pipe.d2h_bytes == ref.numel() * ref.element_size()
