@@ -222,38 +222,40 @@ def launches_per_step(b) -> int:
 
 
 def time_steps(b, steps: int, warmup: int, world: int, sample_clocks=False, device_index=0):
-    """Device time of `steps` steps (max over ranks), and the mean duration of
-    each kernel, from CUDA events on the launching stream."""
+    """Device time per step over `steps` steps (max over ranks), and the mean
+    duration of each kernel of the step (a second pass with CUDA events
+    around every launch, on the launching stream)."""
     from paged_kv_cache_340_b200 import pa_copy_blocks, pa_decode, pa_decode_splitk, pa_reshape_and_cache, \
         pa_splitk_reduce
     spec = b.spec
     stream = torch.cuda.current_stream()
 
+    def mark(ev, i):
+        if ev is not None:
+            ev[i].record(stream)
+
     def step(ev=None):
+        mark(ev, 0)
         if b.cow_pairs.shape[0]:
             pa_copy_blocks(b.k_cache, b.v_cache, b.cow_pairs, stream=stream)
+        mark(ev, 1)
         pa_reshape_and_cache(b.new_key, b.new_value, b.k_cache, b.v_cache, b.slot_mapping, stream=stream)
-        if ev is not None:
-            ev[0].record(stream)
+        mark(ev, 2)
         if b.partition_size:
             pa_decode_splitk(b.workspace, b.query, b.k_cache, b.v_cache, b.block_tables, b.context_lens, spec.scale,
                              b.max_context_len, b.partition_size, seq_order=b.seq_order, stream=stream)
-            if ev is not None:
-                ev[1].record(stream)
+            mark(ev, 3)
             pa_splitk_reduce(b.out, b.workspace, b.context_lens, b.max_context_len, b.partition_size,
                              stream=stream)
         else:
             pa_decode(b.out, b.query, b.k_cache, b.v_cache, b.block_tables, b.context_lens, spec.scale,
                       seq_order=b.seq_order, stream=stream)
-            if ev is not None:
-                ev[1].record(stream)
-        if ev is not None:
-            ev[2].record(stream)
+            mark(ev, 3)
+        mark(ev, 4)
 
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-    # whole-step timing (no per-kernel events inside)
     sampler = ClockSampler(device_index) if sample_clocks else None
     if sampler:
         sampler.start()
@@ -268,17 +270,22 @@ def time_steps(b, steps: int, warmup: int, world: int, sample_clocks=False, devi
     torch.cuda.synchronize()
     barrier(world)
     clocks = sampler.stop() if sampler else None
-    ms = t0.elapsed_time(t1)
-    ms = max_over_ranks(ms, world)
-    # per-kernel durations over a second pass of the same steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    ms = max_over_ranks(t0.elapsed_time(t1), world) / steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     torch.cuda.synchronize()
     for i in range(steps):
         step(evs[i])
     torch.cuda.synchronize()
-    dec = statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
-    red = statistics.fmean(e[1].elapsed_time(e[2]) for e in evs)
-    return ms / steps, dec, red, clocks
+
+    def mean(i, j):
+        return statistics.fmean(e[i].elapsed_time(e[j]) for e in evs)
+
+    kernels = {"reshape_and_cache": mean(1, 2), "decode": mean(2, 3)}
+    if b.cow_pairs.shape[0]:
+        kernels["copy_blocks"] = mean(0, 1)
+    if b.partition_size:
+        kernels["splitk_reduce"] = mean(3, 4)
+    return ms, kernels, clocks
 
 
 def e2e_steps(b, steps: int, warmup: int, world: int):
@@ -396,17 +403,27 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def kernel_lines(spec, b, kern: dict, by: dict) -> dict:
+    """Per kernel of the step: mean launch time and algorithmic GB/s."""
+    nbytes = {"decode": by["decode"], "reshape_and_cache": by["write"], "copy_blocks": by["copy"]}
+    if b.partition_size:
+        parts = ((b.host_context_lens.astype(np.int64) + b.partition_size - 1) // b.partition_size).sum()
+        nbytes["splitk_reduce"] = int(parts) * spec.num_heads * (spec.head_dim + 2) * 4 + \
+            len(b.host_context_lens) * spec.num_heads * spec.head_dim * elt(spec.torch_out_dtype)
+    return {k: {"ms": round(v, 5), "GBps": round(nbytes[k] / v / 1e6, 1)} for k, v in kern.items()}
+
+
 def measure_other(name: str, steps: int, warmup: int):
     spec, b = build_batch(name, 0)
-    ms, dec, red, _ = time_steps(b, steps, warmup, 1)
+    ms, kern, _ = time_steps(b, steps, warmup, 1)
     by = step_bytes(spec, b)
     peak, _ = peaks()
+    dec = kern["decode"]
     res = {"ms_per_step": round(ms, 4), "GBps": round(by["total"] / ms / 1e6, 1),
            "pct_of_hbm_peak": round(100 * by["total"] / ms / 1e6 / peak, 1),
            "decode_kernel_ms": round(dec, 4), "decode_kernel_GBps": round(by["decode"] / dec / 1e6, 1),
-           "partition_size": b.partition_size, "seq_tokens_per_s": round(spec.num_seqs / ms * 1e3, 1)}
-    if b.partition_size:
-        res["reduce_kernel_ms"] = round(red, 4)
+           "partition_size": b.partition_size, "seq_tokens_per_s": round(spec.num_seqs / ms * 1e3, 1),
+           "kernels": kernel_lines(spec, b, kern, by)}
     del b
     torch.cuda.empty_cache()
     return res
@@ -434,8 +451,9 @@ def main():
     import paged_kv_cache_340_b200 as pa  # noqa: F401  (fails loudly without the CUDA library)
 
     spec, b = build_batch(args.workload, rank, args.partition)
-    ms, dec_ms, red_ms, clocks = time_steps(b, args.steps, args.warmup, world, sample_clocks=(rank == 0),
-                                            device_index=local)
+    ms, kern, clocks = time_steps(b, args.steps, args.warmup, world, sample_clocks=(rank == 0),
+                                  device_index=local)
+    dec_ms = kern["decode"]
     by = step_bytes(spec, b)
     peak, peak_kind = peaks()
     value = pdist.job_throughput(by["total"], ms, world)
@@ -466,8 +484,7 @@ def main():
         "gpu_launches": launches_per_step(b) * args.steps,
         "clocks": clocks,
     }
-    if b.partition_size:
-        line["roofline"]["reduce_kernel_ms"] = round(red_ms, 5)
+    line["kernels"] = kernel_lines(spec, b, kern, by)
     if world == 1 and rank == 0 and not args.no_cpu_baseline and "k_pool" in b.host_inputs:
         nbytes, secs, nseq = oracle_sample(OracleBatch(spec, b.host_inputs), 12.0)
         line["cpu_baseline"] = {"value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
