@@ -50,6 +50,8 @@ def _load():
         lib.oracle_splitk_merge.argtypes = [f64p, f64p, f64p, f64p, i32p, ci, ci, ci, ci, ci]
         lib.oracle_reshape_and_cache.argtypes = [u8p, u8p, u8p, u8p, i32p, ci, ci, ci, ci, ci, ci]
         lib.oracle_copy_blocks.argtypes = [u8p, u8p, i64p, ci, ci, ctypes.c_int64]
+        lib.oracle_paged_prefill.argtypes = [f64p, f64p, i32p, f64p, f64p, i32p, ci, i32p, ci, ci, ci, ci, ci, ci,
+                                             cd]
         _lib = lib
     return _lib
 
@@ -151,3 +153,19 @@ def copy_blocks(k_cache: np.ndarray, v_cache: np.ndarray, src_dst_pairs) -> None
     rc = _load().oracle_copy_blocks(_bytes_view(k_cache), _bytes_view(v_cache), pairs, pairs.shape[0],
                                     NB, block_bytes)
     _check(rc, "copy_blocks")
+
+
+def paged_prefill(query, q_start, k_cache, v_cache, block_tables, context_lens, scale, block_size) -> np.ndarray:
+    """Causal attention of each sequence's new query tokens (rows q_start[s] ..
+    q_start[s+1]-1 of query [T, Hq, D]) over its cache; token i of sequence s
+    sits at position context_lens[s] - q_len + i."""
+    q, kc, vc = _f64(query), _f64(k_cache), _f64(v_cache)
+    qs, bt, cl = _i32(q_start), _i32(block_tables), _i32(context_lens)
+    T, Hq, D = q.shape
+    NB, Hkv, bs, _ = kc.shape
+    S = cl.shape[0]
+    assert qs.shape[0] == S + 1 and bs == block_size
+    out = np.zeros_like(q)
+    rc = _load().oracle_paged_prefill(out, q, qs, kc, vc, bt, bt.shape[1], cl, S, Hq, Hkv, D, bs, NB, float(scale))
+    _check(rc, "paged_prefill")
+    return out

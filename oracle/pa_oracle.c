@@ -368,3 +368,62 @@ int oracle_copy_blocks(unsigned char *k_cache, unsigned char *v_cache,
     }
     return OR_OK;
 }
+
+/* Paged prefill (chunked prefill) attention. Sequence s has
+ * q_len_s = q_start[s + 1] - q_start[s] new query tokens, rows q_start[s] ..
+ * of query/out, already written into its cache; query token i sits at
+ * position pos = context_lens[s] - q_len_s + i and attends to the cache
+ * tokens 0 .. pos (causal): out = softmax(scale q . K_t) V over t <= pos.
+ * Decode is the case q_len_s = 1. The pages place prefill beside decode in
+ * the serving step ([P4] §3.4, the model forward over the new tokens) and
+ * give the kernel a num_tokens axis of queries ([P3] §3.1, PagedAttnParams).
+ * Requires q_len_s <= context_lens[s]. */
+int oracle_paged_prefill(double *out, const double *query, const int32_t *q_start,
+                         const double *k_cache, const double *v_cache,
+                         const int32_t *block_tables, int max_blocks_per_seq,
+                         const int32_t *context_lens, int num_seqs, int num_heads,
+                         int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, double scale)
+{
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || num_heads % num_kv_heads != 0)
+        return OR_BAD_ARG;
+    int group = num_heads / num_kv_heads;
+    int max_len = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        int L = context_lens[s];
+        int ql = q_start[s + 1] - q_start[s];
+        if (L < 0 || ql < 0 || ql > L)
+            return OR_BAD_ARG;
+        int rc = check_table_row(block_tables + (size_t)s * max_blocks_per_seq, L,
+                                 block_size, max_blocks_per_seq, num_blocks);
+        if (rc != OR_OK)
+            return rc;
+        if (L > max_len)
+            max_len = L;
+    }
+    size_t n = (size_t)(max_len > 0 ? max_len : 1);
+    double *K = malloc(sizeof(double) * n * head_dim);
+    double *V = malloc(sizeof(double) * n * head_dim);
+    double *z = malloc(sizeof(double) * n);
+    if (!K || !V || !z) {
+        free(K); free(V); free(z);
+        return OR_NO_MEMORY;
+    }
+    for (int s = 0; s < num_seqs; ++s) {
+        const int32_t *row = block_tables + (size_t)s * max_blocks_per_seq;
+        int L = context_lens[s];
+        int ql = q_start[s + 1] - q_start[s];
+        for (int h = 0; h < num_heads; ++h) {
+            gather_tokens(K, V, k_cache, v_cache, row, L, h / group, num_kv_heads,
+                          head_dim, block_size);
+            for (int i = 0; i < ql; ++i) {
+                int pos = L - ql + i;
+                size_t qo = ((size_t)(q_start[s] + i) * num_heads + h) * head_dim;
+                dense_attention(out + qo, query + qo, K, V, z, pos + 1, head_dim, scale);
+            }
+        }
+    }
+    free(K); free(V); free(z);
+    return OR_OK;
+}

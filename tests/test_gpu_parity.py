@@ -309,3 +309,32 @@ def test_device_errors_are_recorded_not_faulted(pa):
     pa.pa_copy_blocks(d["k"], d["v"], torch.tensor([[0, c.NB]], dtype=torch.int64, device="cuda"))
     assert pa.pa_read_device_errors() & pa.PA_DEVERR_PAIR
     assert pa.pa_read_device_errors() == 0
+
+
+def test_largest_batch_grid(pa):
+    """65,535 sequences (the most one launch covers), contexts 0..40: every
+    sequence's output matches the oracle; a 65,536th is refused on the host."""
+    g = torch.Generator().manual_seed(31)
+    S, H, D, BS = 65535, 1, 64, 16
+    ctx = torch.randint(0, 41, (S,), generator=g).to(torch.int32)
+    nb = [(int(c) + BS - 1) // BS for c in ctx]
+    NB = sum(nb)
+    ids = torch.randperm(NB, generator=g).to(torch.int32)
+    tables = torch.full((S, 3), -1, dtype=torch.int32)
+    pos = 0
+    for s, n in enumerate(nb):
+        tables[s, :n] = ids[pos:pos + n]
+        pos += n
+    k = torch.randn((NB, H, BS, D), generator=g).to(torch.float16)
+    v = torch.randn((NB, H, BS, D), generator=g).to(torch.float16)
+    q = torch.randn((S, H, D), generator=g).to(torch.float16)
+    out = torch.empty((S, H, D), dtype=torch.float32, device="cuda")
+    pa.pa_decode(out, q.cuda(), k.cuda(), v.cuda(), tables.cuda(), ctx.cuda(), 0.125)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_errors() == 0
+    ref = oracle.paged_decode(f64(q), f64(k), f64(v), tables.numpy(), ctx.numpy(), 0.125, BS)
+    assert_attention_close(out, ref, torch.float16, "65535 sequences")
+    big = torch.empty((S + 1, H, D), dtype=torch.float32, device="cuda")
+    with pytest.raises(pa.PagedAttentionError):
+        pa.pa_decode(big, big.to(torch.float16), k.cuda(), v.cuda(), torch.cat([tables, tables[:1]]).cuda(),
+                     torch.cat([ctx, ctx[:1]]).cuda(), 0.125)

@@ -309,3 +309,50 @@ def test_copy_blocks(oracle_lib):
         assert np.array_equal(kc[b].view(np.uint16), k0[b].view(np.uint16))
     with pytest.raises(oracle.OracleError):
         oracle.copy_blocks(kc, vc, [(0, 8)])
+
+
+# ------------------------------------------------------------------ prefill
+
+def test_prefill_matches_causal_sdpa(oracle_lib):
+    """Each sequence's new tokens, attended causally over the paged cache,
+    equal torch SDPA in float64 with an explicit causal mask on the
+    contiguous K/V (query i sees positions <= L - q_len + i)."""
+    rng = np.random.default_rng(20)
+    ctx = [1, 17, 40, 33]
+    qlen = [1, 5, 40, 7]
+    Hq, Hkv, D, bs = 4, 2, 8, 16
+    q_, kp, vp, bt, cl, K, V = _paged_case(rng, len(ctx), Hq, Hkv, D, bs, ctx, 12)
+    qs = np.concatenate([[0], np.cumsum(qlen)]).astype(np.int32)
+    Q = rng.normal(size=(int(qs[-1]), Hq, D))
+    out = oracle.paged_prefill(Q, qs, kp, vp, bt, cl, 0.3, bs)
+    for s, (L, ql) in enumerate(zip(ctx, qlen)):
+        qt = torch.from_numpy(Q[qs[s]:qs[s + 1]]).permute(1, 0, 2)             # [Hq, ql, D]
+        kt = torch.from_numpy(K[s]).permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0)
+        vt = torch.from_numpy(V[s]).permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0)
+        pos = torch.arange(L - ql, L).unsqueeze(1)
+        mask = torch.arange(L).unsqueeze(0) <= pos                               # [ql, L]
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=0.3)
+        np.testing.assert_allclose(out[qs[s]:qs[s + 1]], ref.permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_of_one_token_is_decode(oracle_lib):
+    rng = np.random.default_rng(21)
+    ctx = [5, 64, 1]
+    q_, kp, vp, bt, cl, K, V = _paged_case(rng, 3, 4, 4, 8, 16, ctx, 10)
+    qs = np.arange(4, dtype=np.int32)
+    a = oracle.paged_prefill(q_, qs, kp, vp, bt, cl, 0.5, 16)
+    b = oracle.paged_decode(q_, kp, vp, bt, cl, 0.5, 16)
+    assert np.array_equal(a, b)
+
+
+def test_prefill_first_token_sees_only_itself(oracle_lib):
+    """A sequence prefilled from empty: its first token attends to itself
+    only (out = V[0]); its last token sees the whole context."""
+    rng = np.random.default_rng(22)
+    L = 20
+    q_, kp, vp, bt, cl, K, V = _paged_case(rng, 1, 2, 2, 8, 16, [L], 4)
+    Q = rng.normal(size=(L, 2, 8))
+    out = oracle.paged_prefill(Q, np.array([0, L], np.int32), kp, vp, bt, cl, 0.4, 16)
+    assert np.array_equal(out[0], V[0][0])
+    last = oracle.paged_decode(Q[L - 1:L], kp, vp, bt, cl, 0.4, 16)
+    np.testing.assert_allclose(out[L - 1], last[0], rtol=0, atol=0)
