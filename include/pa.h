@@ -203,6 +203,29 @@ int pa_decode_splitk_static(void *out, const void *query, const void *k_cache, c
                             pa_dtype kv_dtype, pa_dtype out_dtype, cudaStream_t stream);
 
 /*
+ * pa_prefill -- paged prefill (chunked prefill) attention on the tensor cores.
+ * Sequence s has q_len_s = q_start[s+1] - q_start[s] new query tokens, rows
+ * q_start[s] .. of query [num_tokens, num_heads, head_dim] (q_start is a device
+ * int32 [num_seqs + 1], non-decreasing, q_start[num_seqs] <= num_tokens),
+ * whose K/V are already in the cache (written by pa_reshape_and_cache). Query
+ * token i sits at position pos = context_lens[s] - q_len_s + i and attends
+ * causally to cache tokens 0 .. pos:
+ *   out[q_start[s] + i, h, :] = sum_{t <= pos} softmax_t(scale q . K_t) V_t.
+ * q_len_s = 1 is decode. max_q_len bounds every q_len_s. Requires
+ * q_len_s <= context_lens[s] (else PA_DEVERR_CONTEXT and that sequence is
+ * skipped). head_dim 128, kv_dtype PA_F16 or PA_BF16, out_dtype kv_dtype or
+ * PA_F32. ([P4] §3.4: the forward pass over the step's new tokens, each
+ * layer attending over the paged cache; [P3] §3.1: the num_tokens axis of
+ * queries.) QK^T and PV run as tcgen05 MMAs with accumulators in tensor
+ * memory; K/V tiles are gathered through the table by TMA.
+ */
+int pa_prefill(void *out, const void *query, const int32_t *q_start, int num_tokens, int max_q_len,
+               const void *k_cache, const void *v_cache, const int32_t *block_tables,
+               int max_blocks_per_seq, const int32_t *context_lens, int num_seqs, int num_heads,
+               int num_kv_heads, int head_dim, float scale, int block_size, int num_blocks,
+               pa_dtype kv_dtype, pa_dtype out_dtype, cudaStream_t stream);
+
+/*
  * Partition size this library would pick for a batch: 0 when the
  * unpartitioned pa_decode already fills the GPU, else a multiple of
  * block_size. Host-only arithmetic on the sizes given (occupancy rule:

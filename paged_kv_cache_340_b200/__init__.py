@@ -38,7 +38,7 @@ EXPORTED = (
     "pa_splitk_workspace_bytes", "pa_splitk_acc_offset", "pa_decode_splitk", "pa_splitk_reduce",
     "pa_choose_partition", "pa_copy_blocks", "pa_pool_create", "pa_pool_destroy", "pa_pool_num_free",
     "pa_pool_ref_count", "pa_pool_allocate", "pa_pool_share", "pa_pool_free", "pa_pool_append",
-    "pa_pool_fork", "pa_pool_release", "pa_decode_splitk_static",
+    "pa_pool_fork", "pa_pool_release", "pa_decode_splitk_static", "pa_prefill",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -81,6 +81,8 @@ def _load() -> ctypes.CDLL:
         "pa_pool_release": (i32, [vp, i32p, i32]),
         "pa_decode_splitk_static": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32,
                                           i32, i32, vp]),
+        "pa_prefill": (i32, [vp, vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32,
+                             vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -195,6 +197,19 @@ def pa_decode_splitk_static(out, query, k_cache, v_cache, block_tables, context_
                                       NB, int(max_context_len), int(partition_size), _dtype(k_cache), _dtype(out),
                                       _stream(stream))
     _check(rc, "pa_decode_splitk_static")
+
+
+def pa_prefill(out, query, q_start, max_q_len, k_cache, v_cache, block_tables, context_lens, scale,
+               stream=None) -> None:
+    """Causal attention of each sequence's new query tokens (rows q_start[s] ..
+    q_start[s+1]-1 of query [T, Hq, D]) over its paged cache."""
+    T, Hq, D = query.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    S = context_lens.shape[0]
+    rc = _lib.pa_prefill(_ptr(out), _ptr(query), _ptr(q_start), T, int(max_q_len), _ptr(k_cache), _ptr(v_cache),
+                         _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S, Hq, Hkv, D, float(scale),
+                         bs, NB, _dtype(k_cache), _dtype(out), _stream(stream))
+    _check(rc, "pa_prefill")
 
 
 def pa_choose_partition(num_seqs, num_kv_heads, max_context_len, block_size, head_dim, kv_dtype) -> int:

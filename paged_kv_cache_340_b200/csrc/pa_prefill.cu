@@ -1,0 +1,563 @@
+// Paged prefill (chunked prefill) attention for sm_100a on the 5th-generation
+// tensor cores.
+//
+// What is computed: sequence s has q_len new query tokens (rows q_start[s] ..
+// of query), already written into its paged cache; query token i sits at
+// position pos = context_len - q_len + i and attends causally to the cache
+// tokens 0 .. pos: out = softmax(scale q . K_t) V over t <= pos. Decode is
+// q_len = 1. ([P4 "PagedAttention 实现细节", §3.4: the model forward over the
+// step's new tokens, each layer's attention over the paged cache]; [P3 "Ascend
+// C ... PagedAttention融合算子", §3.1: a num_tokens axis of queries].)
+//
+// How (B200 design): one CTA per (sequence, kv head, 128-row query tile); the
+// rows are (token, query head of the GQA group) pairs, so every K/V tile is
+// loaded once for the whole group.
+//   * warp 4 lane 0 is the control thread. It loads the Q tile once and the
+//     K/V tiles (64 tokens, gathered block by block through the table) with
+//     2-D/3-D TMA tensor copies in the 128-byte swizzled layout, into two
+//     stages; it issues S = Q K^T (M 128, N 64, K = head_dim in 8 steps) and
+//     O += P V (M 128, N = head_dim, K 64 in 4 steps) as tcgen05.mma with the
+//     fp32 accumulators S and O in tensor memory, and tcgen05.commit signals
+//     each product's completion on an mbarrier;
+//   * warps 0-3 run the softmax: thread r owns row r (tensor-memory lane r),
+//     reads its S row with tcgen05.ld, masks positions past its token
+//     (causal) and past the context, keeps the running max and sum in fp32
+//     (log2 domain), rescales its O row in tensor memory when the max rises,
+//     and writes its probabilities as a 16-bit row of the P operand in shared
+//     memory (same swizzled K-major layout);
+//   * V rows past the context are zeroed in shared memory before P V (they
+//     may hold anything, and 0 * NaN is NaN on the tensor cores too).
+// Every wait is bounded (PA_DEVERR_TIMEOUT); tensor memory is always freed.
+#include <cuda.h>
+
+#include <mutex>
+#include <type_traits>
+
+#include "pa_common.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace prefill {
+
+constexpr int kM = 128;                 // query rows per CTA
+constexpr int kN = 64;                  // kv tokens per tile
+constexpr int kD = 128;                 // head dim
+constexpr int kHalfBytes = 128;         // one swizzled row: 64 16-bit elements
+constexpr int kQHalf = kM * kHalfBytes; // 16 KB: rows x d 0-63 (or 64-127)
+constexpr int kKVHalf = kN * kHalfBytes;  // 8 KB
+constexpr int kQBytes = 2 * kQHalf;
+constexpr int kKVBytes = 2 * kKVHalf;   // one K or V tile
+constexpr int kPBytes = kM * kHalfBytes;  // 128 rows x 64 tokens
+constexpr int kStages = 2;
+constexpr int kSoftmaxWarps = 4;
+constexpr int kThreads = (kSoftmaxWarps + 1) * 32;
+constexpr int kTmemCols = 256;          // O: columns 0-127, S: 128-191
+constexpr int kOCol = 0;
+constexpr int kSCol = 128;
+// shared memory (every operand region 1024-byte aligned for the swizzle)
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kQBytes;
+constexpr int kOffV = kOffK + kStages * kKVBytes;
+constexpr int kOffP = kOffV + kStages * kKVBytes;
+constexpr int kOffBar = kOffP + 2 * kPBytes;  // P (and, for bf16, its low part)
+constexpr int kSmemBytes = 1024 + kOffBar + 16 * 8;
+
+struct Params {
+    void *out;
+    const int32_t *q_start;
+    const int32_t *block_tables;
+    const int32_t *context_lens;
+    int max_blocks_per_seq;
+    int num_heads;
+    int num_kv_heads;
+    int num_blocks;
+    int block_size;
+    long long kv_rows;  // num_blocks * num_kv_heads * block_size (rows of the 2-D pool view)
+    float scale_log2;
+    pa_dtype out_dtype;
+    unsigned int *err;
+};
+
+// ---------------------------------------------------------------- helpers
+
+// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: start,
+// leading and stride byte offsets in 16-byte units, version 1).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16 with fp32 accumulation.
+__host__ __device__ constexpr uint32_t mma_idesc(bool bf16, int M, int N, bool b_mn_major) {
+    return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                     uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+                 :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+                 : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+        "[%2];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+template <typename T> struct Pack16;
+template <> struct Pack16<__nv_bfloat16> {
+    static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t *>(&v);
+    }
+};
+template <> struct Pack16<__half> {
+    static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+        __half2 v = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t *>(&v);
+    }
+};
+
+// ----------------------------------------------------------------- kernel
+
+template <typename T, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                   const __grid_constant__ CUtensorMap tmap_v, const Params p) {
+    constexpr bool kBf16 = std::is_same_v<T, __nv_bfloat16>;
+    constexpr int kTokPerTile = kM / G;
+    constexpr uint32_t kIdescQK = mma_idesc(kBf16, kM, kN, false);
+    constexpr uint32_t kIdescPV = mma_idesc(kBf16, kM, kD, true);
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char *Qs = sm + kOffQ;
+    unsigned char *Ks = sm + kOffK;
+    unsigned char *Vs = sm + kOffV;
+    unsigned char *Ps = sm + kOffP;
+    unsigned char *Pl = Ps + kPBytes;  // bf16 only: P - bf16(P)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBar);
+    uint64_t *q_full = bars + 0;
+    uint64_t *kv_full = bars + 1;  // [2]
+    uint64_t *s_full = bars + 3;
+    uint64_t *p_full = bars + 4;
+    uint64_t *o_done = bars + 5;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
+    int *abort_flag = reinterpret_cast<int *>(bars + 7);
+
+    const int qt = blockIdx.x;
+    const int kvh = blockIdx.y;
+    const int s = blockIdx.z;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const int q0 = p.q_start[s];
+    const int q_len = p.q_start[s + 1] - q0;
+    const int ctx = p.context_lens[s];
+    const int tok0 = qt * kTokPerTile;
+    if (tok0 >= q_len) return;
+    if (q_len > ctx || ctx > p.max_blocks_per_seq * p.block_size) {
+        if (threadIdx.x == 0) record_error(p.err, PA_DEVERR_CONTEXT);
+        return;
+    }
+    const int rows_valid = min(kM, (q_len - tok0) * G);
+    const int pos0 = ctx - q_len + tok0;                      // position of the tile's first token
+    const int pos_max = pos0 + rows_valid / G - 1;
+    const int ntiles = pos_max / kN + 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(kv_full + 0, 1);
+        mbar_init(kv_full + 1, 1);
+        mbar_init(s_full, 1);
+        mbar_init(p_full, kSoftmaxWarps * 32);
+        mbar_init(o_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kSoftmaxWarps) {
+        // ===================================================== control thread
+        if (lane == 0) {
+            const int32_t *trow = p.block_tables + (size_t)s * p.max_blocks_per_seq;
+            const int nblk = (ctx + p.block_size - 1) / p.block_size;
+            auto load_kv = [&](int j) {
+                const int b = j & 1;
+                unsigned char *kd = Ks + b * kKVBytes;
+                unsigned char *vd = Vs + b * kKVBytes;
+                mbar_arrive_expect_tx(kv_full + b, 2 * kKVBytes);
+#pragma unroll
+                for (int g = 0; g < kN / 16; ++g) {  // 16-row groups of the tile
+                    const int tok = j * kN + g * 16;
+                    const int lb = tok / p.block_size;
+                    long long row = p.kv_rows;  // past the end: the copy fills zeros
+                    if (lb < nblk) {
+                        const int id = __ldg(trow + lb);
+                        if (id >= 0 && id < p.num_blocks)
+                            row = ((long long)id * p.num_kv_heads + kvh) * p.block_size + (tok % p.block_size);
+                        else
+                            record_error(p.err, PA_DEVERR_BLOCK_ID);
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        tma_load_2d(kd + h * kKVHalf + g * 16 * kHalfBytes, &tmap_k, h * 64, (int)row, kv_full + b);
+                        tma_load_2d(vd + h * kKVHalf + g * 16 * kHalfBytes, &tmap_v, h * 64, (int)row, kv_full + b);
+                    }
+                }
+            };
+            mbar_arrive_expect_tx(q_full, kQBytes);
+            tma_load_3d(Qs, &tmap_q, 0, kvh * G, q0 + tok0, q_full);
+            tma_load_3d(Qs + kQHalf, &tmap_q, 64, kvh * G, q0 + tok0, q_full);
+            load_kv(0);
+            if (ntiles > 1) load_kv(1);
+            bool ok = true;
+            int waited_kv = 0;
+            for (int j = 0; j < ntiles && ok; ++j) {
+                const int b = j & 1;
+                if (!mbar_wait(kv_full + b, (j >> 1) & 1) || (j == 0 && !mbar_wait(q_full, 0))) {
+                    ok = false;
+                    break;
+                }
+                waited_kv = j + 1;
+                tc_fence_after();
+                const uint32_t qa = smem_addr(Qs), ka = smem_addr(Ks + b * kKVBytes);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
+                    umma(tmem + kSCol, sw128_desc(qa + (kk >> 2) * kQHalf + off, 16, 1024),
+                         sw128_desc(ka + (kk >> 2) * kKVHalf + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(s_full);
+                if (!mbar_wait(p_full, j & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t pa_ = smem_addr(Ps), pl_ = smem_addr(Pl), va = smem_addr(Vs + b * kKVBytes);
+#pragma unroll
+                for (int kk = 0; kk < kN / 16; ++kk) {
+                    const uint64_t vdesc = sw128_desc(va + kk * 16 * kHalfBytes, kKVHalf, 1024);
+                    umma(tmem + kOCol, sw128_desc(pa_ + kk * 32, 16, 1024), vdesc, kIdescPV,
+                         (j > 0 || kk > 0) ? 1u : 0u);
+                    if constexpr (kBf16) umma(tmem + kOCol, sw128_desc(pl_ + kk * 32, 16, 1024), vdesc, kIdescPV, 1u);
+                }
+                umma_commit(o_done);
+                if (j + 2 < ntiles) {
+                    if (!mbar_wait(o_done, j & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    load_kv(j + 2);
+                }
+            }
+            if (!ok) {
+                record_error(p.err, PA_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+                // let the copies this thread started land before the CTA leaves
+                for (int j = waited_kv; j < min(ntiles, waited_kv + 2); ++j) mbar_wait(kv_full + (j & 1), (j >> 1) & 1);
+                mbar_wait(q_full, 0);
+                // release the softmax warps from their waits
+                mbar_arrive(s_full);
+                mbar_arrive(o_done);
+            }
+        }
+        __syncwarp();  // reconverge the control warp before the block-wide barrier
+    } else {
+        // ======================================================= softmax warps
+        const int r = threadIdx.x;  // row = tensor-memory lane
+        const int tok = r / G;
+        const bool valid = r < rows_valid;
+        const int pos = valid ? pos0 + tok : -1;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        float m_run = -INFINITY, l_run = 0.f;
+        for (int j = 0; j < ntiles; ++j) {
+            if (!mbar_wait(s_full, j & 1) || *(volatile int *)abort_flag) break;
+            tc_fence_after();
+            uint32_t sr[2][32];
+            tmem_ld32(tmem + lane_base + kSCol, sr[0]);
+            tmem_ld32(tmem + lane_base + kSCol + 32, sr[1]);
+            tmem_wait_ld();
+            const int kv0 = j * kN;
+            float x[kN];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kN; ++c) {
+                const float sv = __uint_as_float(sr[c >> 5][c & 31]);
+                x[c] = (kv0 + c <= pos) ? sv * p.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, x[c]);
+            }
+            const float mn = fmaxf(m_run, mx);
+            const float alpha = (mn == -INFINITY) ? 1.f : fast_exp2(m_run - mn);
+            m_run = mn;
+            float psum = 0.f;
+#pragma unroll
+            for (int c = 0; c < kN; ++c) {
+                x[c] = (x[c] == -INFINITY) ? 0.f : fast_exp2(x[c] - mn);
+                psum += x[c];
+            }
+            l_run = l_run * alpha + psum;
+            if (j > 0) {
+                // O and P of tile j-1 are done with: rescale O, reuse P
+                if (!mbar_wait(o_done, (j - 1) & 1) || *(volatile int *)abort_flag) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                    for (int ch = 0; ch < kD / 32; ++ch) {
+                        uint32_t o[32];
+                        tmem_ld32(tmem + lane_base + kOCol + ch * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(tmem + lane_base + kOCol + ch * 32, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // this row of P: 64 probabilities as 16-bit pairs, 8 swizzled 16-byte chunks.
+            // bf16 keeps 8 mantissa bits, so P also goes in as its low part
+            // P - bf16(P) (a second P V pass), for ~2^-17 relative error.
+            unsigned char *prow = Ps + r * kHalfBytes;
+            unsigned char *plow = Pl + r * kHalfBytes;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) w[e] = Pack16<T>::pack(x[8 * ch + 2 * e], x[8 * ch + 2 * e + 1]);
+                *reinterpret_cast<uint4 *>(prow + ((ch ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                if constexpr (kBf16) {
+                    uint32_t lw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float hi0 = __uint_as_float(w[e] << 16), hi1 = __uint_as_float(w[e] & 0xffff0000u);
+                        lw[e] = Pack16<T>::pack(x[8 * ch + 2 * e] - hi0, x[8 * ch + 2 * e + 1] - hi1);
+                    }
+                    *reinterpret_cast<uint4 *>(plow + ((ch ^ (r & 7)) << 4)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+            }
+            // V rows past the context: zero (both halves) before P V reads them
+            const int zrow = max(0, ctx - kv0);
+            if (zrow < kN) {
+                unsigned char *vt = Vs + (j & 1) * kKVBytes;
+                const int nvec = (kN - zrow) * 2 * (kHalfBytes / 16);
+                for (int i = r; i < nvec; i += kSoftmaxWarps * 32) {
+                    const int row = zrow + i / 16;
+                    const int h = (i / 8) & 1;
+                    const int c = i & 7;
+                    *reinterpret_cast<uint4 *>(vt + h * kKVHalf + row * kHalfBytes + c * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(p_full);
+        }
+        // ---- output: O / l for valid rows
+        const bool done = mbar_wait(o_done, (ntiles - 1) & 1) && !*(volatile int *)abort_flag;
+        tc_fence_after();
+        if (!done) {
+            if (r == 0) record_error(p.err, PA_DEVERR_TIMEOUT);
+        } else {
+            const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+            const size_t orow = ((size_t)(q0 + tok0 + tok) * p.num_heads + (size_t)kvh * G + (r % G)) * kD;
+#pragma unroll
+            for (int ch = 0; ch < kD / 32; ++ch) {
+                uint32_t o[32];
+                tmem_ld32(tmem + lane_base + kOCol + ch * 32, o);
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) store_out(p.out, orow + ch * 32 + e, __uint_as_float(o[e]) * inv, p.out_dtype);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+}  // namespace prefill
+}  // namespace pa
+
+// ------------------------------------------------------------------ host side
+
+namespace pa {
+namespace prefill {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// A rank-2 or rank-3 tiled map over 16-bit elements, 128-byte swizzle, zero fill.
+static bool make_map(CUtensorMap *map, bool bf16, void *base, int rank, const cuuint64_t *dims,
+                     const cuuint64_t *strides_bytes, const cuuint32_t *box) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = f(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank, base, dims,
+                   strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename T, int G>
+static cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const Params &p,
+                            int q_tiles, int num_kv_heads, int num_seqs, cudaStream_t stream) {
+    auto kern = prefill_kernel<T, G>;
+    static unsigned int attr_done = 0;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), kSmemBytes, &attr_done);
+    if (e != cudaSuccess) return e;
+    kern<<<dim3(q_tiles, num_kv_heads, num_seqs), kThreads, kSmemBytes, stream>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace prefill
+}  // namespace pa
+
+extern "C" int pa_prefill(void *out, const void *query, const int32_t *q_start, int num_tokens,
+                          int max_q_len, const void *k_cache, const void *v_cache,
+                          const int32_t *block_tables, int max_blocks_per_seq,
+                          const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                          int head_dim, float scale, int block_size, int num_blocks, pa_dtype kv_dtype,
+                          pa_dtype out_dtype, cudaStream_t stream) {
+    using namespace pa::prefill;
+    if (num_seqs < 0 || num_tokens < 0 || max_q_len < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
+        num_blocks < 0 || max_blocks_per_seq < 0 || num_seqs > 65535 || num_kv_heads > 65535)
+        return PA_ERR_SHAPE;
+    if (kv_dtype != PA_F16 && kv_dtype != PA_BF16) return PA_ERR_DTYPE;
+    if (out_dtype != kv_dtype && out_dtype != PA_F32) return PA_ERR_DTYPE;
+    if (head_dim != 128) return PA_ERR_HEAD_DIM;
+    if (block_size != 16 && block_size != 32) return PA_ERR_BLOCK_SIZE;
+    if (num_heads % num_kv_heads != 0) return PA_ERR_HEADS;
+    const int group = num_heads / num_kv_heads;
+    if (group != 1 && group != 2 && group != 4 && group != 8) return PA_ERR_HEADS;
+    if (num_seqs == 0 || num_tokens == 0 || max_q_len == 0) return PA_OK;
+    if (!out || !query || !q_start || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_NULL;
+    auto al = [](const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) == 0; };
+    if (!al(out, 16) || !al(query, 16) || !al(k_cache, 16) || !al(v_cache, 16) || !al(q_start, 4) ||
+        !al(block_tables, 4) || !al(context_lens, 4))
+        return PA_ERR_ALIGN;
+    const long long kv_rows = (long long)num_blocks * num_kv_heads * block_size;
+    if (kv_rows >= INT32_MAX || (long long)num_tokens * num_heads >= INT32_MAX) return PA_ERR_SHAPE;
+    const bool bf16 = kv_dtype == PA_BF16;
+    CUtensorMap mq, mk, mv;
+    {
+        const cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_heads, (cuuint64_t)num_tokens};
+        const cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)num_heads * head_dim * 2};
+        const cuuint32_t box[3] = {64, (cuuint32_t)group, (cuuint32_t)(kM / group)};
+        if (!make_map(&mq, bf16, const_cast<void *>(query), 3, dims, strides, box)) return PA_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)(kv_rows > 0 ? kv_rows : 1)};
+        const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+        const cuuint32_t box[2] = {64, 16};
+        if (!make_map(&mk, bf16, const_cast<void *>(k_cache), 2, dims, strides, box)) return PA_ERR_CUDA;
+        if (!make_map(&mv, bf16, const_cast<void *>(v_cache), 2, dims, strides, box)) return PA_ERR_CUDA;
+    }
+    unsigned int *err = nullptr;
+    if (pa::device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    Params p{};
+    p.out = out;
+    p.q_start = q_start;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.num_blocks = num_blocks;
+    p.block_size = block_size;
+    p.kv_rows = kv_rows;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.out_dtype = out_dtype;
+    p.err = err;
+    const int q_tiles = (max_q_len * group + kM - 1) / kM;
+    cudaError_t e = cudaErrorInvalidValue;
+#define PA_PREFILL_CASE(T, GG) e = launch_t<T, GG>(mq, mk, mv, p, q_tiles, num_kv_heads, num_seqs, stream)
+    if (bf16) {
+        switch (group) {
+            case 1: PA_PREFILL_CASE(__nv_bfloat16, 1); break;
+            case 2: PA_PREFILL_CASE(__nv_bfloat16, 2); break;
+            case 4: PA_PREFILL_CASE(__nv_bfloat16, 4); break;
+            case 8: PA_PREFILL_CASE(__nv_bfloat16, 8); break;
+        }
+    } else {
+        switch (group) {
+            case 1: PA_PREFILL_CASE(__half, 1); break;
+            case 2: PA_PREFILL_CASE(__half, 2); break;
+            case 4: PA_PREFILL_CASE(__half, 4); break;
+            case 8: PA_PREFILL_CASE(__half, 8); break;
+        }
+    }
+#undef PA_PREFILL_CASE
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
