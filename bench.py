@@ -413,6 +413,57 @@ def kernel_lines(spec, b, kern: dict, by: dict) -> dict:
     return {k: {"ms": round(v, 5), "GBps": round(nbytes[k] / v / 1e6, 1)} for k, v in kern.items()}
 
 
+def tensor_peak():
+    """Measured dense bf16 tensor throughput (TFLOP/s), burst figure."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def measure_prefill(name: str, steps: int, warmup: int):
+    """Prefill step (slot write of the new tokens + causal paged attention):
+    TFLOP/s of the attention kernel against the bf16 tensor peak."""
+    from paged_kv_cache_340_b200 import pa_prefill, pa_reshape_and_cache
+    from paged_kv_cache_340_b200.batch import build_prefill_batch, prefill_flops
+    from paged_kv_cache_340_b200.workloads import SPECS, make_prefill_inputs
+    spec = SPECS[name]
+    b = build_prefill_batch(spec, make_prefill_inputs(spec))
+    stream = torch.cuda.current_stream()
+    flops = prefill_flops(spec, b.host_context_lens)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        pa_reshape_and_cache(b.new_key, b.new_value, b.k_cache, b.v_cache, b.slot_mapping, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        pa_prefill(b.out, b.query, b.q_start, b.max_q_len, b.k_cache, b.v_cache, b.block_tables, b.context_lens,
+                   spec.scale, stream=stream)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    att = statistics.fmean(e[1].elapsed_time(e[2]) for e in evs)
+    wr = statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
+    peak, kind = tensor_peak()
+    tf = flops / (att * 1e-3) / 1e12
+    res = {"prefill_kernel_ms": round(att, 4), "TFLOPs": round(tf, 1), "tensor_peak": peak, "peak_kind": kind,
+           "frac_of_tensor_peak": round(tf / peak, 3), "flops_per_step": flops,
+           "slot_write_ms": round(wr, 4), "new_tokens": int(b.host_slots.shape[0]),
+           "tokens_per_s": round(b.host_slots.shape[0] / ((att + wr) * 1e-3), 1)}
+    del b
+    torch.cuda.empty_cache()
+    return res
+
+
 def measure_other(name: str, steps: int, warmup: int):
     spec, b = build_batch(name, 0)
     ms, kern, _ = time_steps(b, steps, warmup, 1)
@@ -450,6 +501,13 @@ def main():
     world, rank, local = dist_setup(args.gpus)
     import paged_kv_cache_340_b200 as pa  # noqa: F401  (fails loudly without the CUDA library)
 
+    from paged_kv_cache_340_b200.workloads import SPECS as _SPECS
+    if _SPECS[args.workload].q_len:
+        if rank == 0:
+            print(json.dumps({"workload": args.workload, "prefill": measure_prefill(args.workload, args.steps,
+                                                                                    args.warmup)}), flush=True)
+        pdist.finalize(world)
+        return
     spec, b = build_batch(args.workload, rank, args.partition)
     ms, kern, clocks = time_steps(b, args.steps, args.warmup, world, sample_clocks=(rank == 0),
                                   device_index=local)
@@ -495,6 +553,8 @@ def main():
     if world == 1 and not args.no_others and args.workload == DEFAULT_WORKLOAD:
         line["other_workloads"] = {n: measure_other(n, 200, 10) for n in
                                    ("gqa_bf16", "long_splitk_bf16", "parallel_sampling_fp16")}
+        line["prefill_workloads"] = {n: measure_prefill(n, 20, 3) for n in
+                                     ("prefill_llama7b_mha_bf16", "chunked_prefill_gqa_bf16")}
     if rank == 0:
         print(json.dumps(line), flush=True)
     pdist.finalize(world)

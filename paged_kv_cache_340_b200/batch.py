@@ -16,7 +16,7 @@ import numpy as np
 import torch
 
 from . import (PA_POOL_FIFO, BlockPool, pa_choose_partition, pa_copy_blocks, pa_decode, pa_decode_splitk,
-               pa_reshape_and_cache, pa_splitk_reduce, pa_splitk_workspace_bytes)
+               pa_prefill, pa_reshape_and_cache, pa_splitk_reduce, pa_splitk_workspace_bytes)
 from .workloads import Spec
 
 
@@ -289,3 +289,71 @@ class HostStepPipeline:
         for j in range(2):
             if self.i > j:
                 comp.wait_event(self.out_free[j])
+
+
+@dataclass
+class PrefillBatch:
+    spec: Spec
+    num_blocks: int
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    query: torch.Tensor         # device [T, Hq, D], sequence-major
+    out: torch.Tensor           # device [T, Hq, D]
+    q_start: torch.Tensor       # device int32 [S + 1]
+    block_tables: torch.Tensor
+    context_lens: torch.Tensor
+    new_key: torch.Tensor       # device [T, Hkv, D]
+    new_value: torch.Tensor
+    slot_mapping: torch.Tensor  # device int32 [T]
+    max_q_len: int
+    host_tables: np.ndarray
+    host_slots: np.ndarray
+    host_context_lens: np.ndarray
+    host_q_start: np.ndarray
+
+
+def build_prefill_batch(spec: Spec, inputs: dict, device="cuda", pool_policy: int = PA_POOL_FIFO) -> PrefillBatch:
+    """Prefill step: every sequence holds context_lens - q_len tokens and
+    appends q_len new ones; their K/V go in through their slots, then their
+    queries attend causally over the cache."""
+    bs = spec.block_size
+    ctx = inputs["context_lens"].numpy().astype(np.int32)
+    S, ql = ctx.shape[0], spec.q_len
+    nb = int(inputs["num_blocks"])
+    pool = BlockPool(nb, bs, pool_policy, free_order=inputs["free_order"].numpy())
+    tables = np.full((S, max(1, _blocks(int(ctx.max()), bs))), -1, np.int32)
+    slots = np.empty(S * ql, np.int32)
+    for s in range(S):
+        nt, _, _ = pool.append(tables[s], 0, int(ctx[s]) - ql, want_slots=False)
+        _, sl, _ = pool.append(tables[s], nt, ql)
+        slots[s * ql:(s + 1) * ql] = sl
+    q_start = (np.arange(S + 1) * ql).astype(np.int32)
+    dev = torch.device(device)
+    return PrefillBatch(
+        spec=spec, num_blocks=nb, k_cache=inputs["k_pool"].to(dev), v_cache=inputs["v_pool"].to(dev),
+        query=inputs["query"].to(dev),
+        out=torch.empty((S * ql, spec.num_heads, spec.head_dim), dtype=spec.torch_out_dtype, device=dev),
+        q_start=torch.from_numpy(q_start).to(dev), block_tables=torch.from_numpy(tables).to(dev),
+        context_lens=torch.from_numpy(ctx).to(dev), new_key=inputs["new_key"].to(dev),
+        new_value=inputs["new_value"].to(dev), slot_mapping=torch.from_numpy(slots).to(dev), max_q_len=ql,
+        host_tables=tables, host_slots=slots, host_context_lens=ctx, host_q_start=q_start)
+
+
+def run_prefill_step(batch: PrefillBatch, stream=None) -> None:
+    """The new tokens' K/V through their slots, then causal attention."""
+    pa_reshape_and_cache(batch.new_key, batch.new_value, batch.k_cache, batch.v_cache, batch.slot_mapping,
+                         stream=stream)
+    pa_prefill(batch.out, batch.query, batch.q_start, batch.max_q_len, batch.k_cache, batch.v_cache,
+               batch.block_tables, batch.context_lens, batch.spec.scale, stream=stream)
+
+
+def prefill_flops(spec: Spec, ctx: np.ndarray) -> int:
+    """Causal attention FLOPs of a prefill step: query token i of a sequence
+    sees pos + 1 keys, 4 * head_dim FLOPs per key (QK^T and PV), per head."""
+    ql = spec.q_len
+    total = 0
+    for L in ctx.astype(np.int64):
+        first = int(L) - ql + 1                     # keys seen by the first new token
+        keys = ql * (2 * first + ql - 1) // 2       # sum over the q_len tokens
+        total += 4 * spec.head_dim * keys * spec.num_heads
+    return total

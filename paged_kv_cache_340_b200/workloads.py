@@ -22,6 +22,10 @@ Workloads (shapes follow LLaMA-style decode layers):
   parallel_sampling_fp16  16 prompts x 5 branches, 32 heads, head_dim 128, block 16,
                        1000-token shared prefix, each branch adds U{1..256} tokens;
                        q/k/v ~ N(0,1); fp16 out
+  prefill_llama7b_mha_bf16   8 prompts of 2048 tokens prefilled from empty, 32 heads,
+                       head_dim 128, block 16; q/k/v ~ N(0,1); fp32 out
+  chunked_prefill_gqa_bf16   16 sequences of 4096 tokens whose last 512 are new,
+                       32 query / 8 kv heads, head_dim 128, block 16; fp32 out
 """
 from __future__ import annotations
 
@@ -53,6 +57,7 @@ class Spec:
     kv_scale: float = 1.0
     v_uniform: bool = False
     partition_size: int = 0  # split-K partition (tokens) the workload is run with; 0 = unsplit
+    q_len: int = 0  # prefill workloads: new query tokens per sequence (0 = decode)
     # parallel sampling (copy-on-write) workload
     num_prompts: int = 0
     branches: int = 0
@@ -84,6 +89,11 @@ SPECS: Dict[str, Spec] = {
     "parallel_sampling_fp16": Spec("parallel_sampling_fp16", 80, 32, 32, 128, 16, "f16", "f16", 3404,
                                    ("parallel",), None, num_prompts=16, branches=5, prefix_len=1000,
                                    max_divergent=256),
+    # prefill: a prompt's tokens attend causally over the paged cache
+    "prefill_llama7b_mha_bf16": Spec("prefill_llama7b_mha_bf16", 8, 32, 32, 128, 16, "bf16", "f32", 3405,
+                                     ("fixed", (2048,) * 8), 1.0, q_len=2048),
+    "chunked_prefill_gqa_bf16": Spec("chunked_prefill_gqa_bf16", 16, 32, 8, 128, 16, "bf16", "f32", 3406,
+                                     ("fixed", (4096,) * 16), 1.0, q_len=512),
 }
 
 
@@ -188,3 +198,29 @@ def make_parallel_sampling_inputs(spec: Spec) -> dict:
     return dict(prefix_key=prefix_key, prefix_value=prefix_value, divergent_lens=div,
                 divergent_key=divergent_key, divergent_value=divergent_value, query=query,
                 free_order=free_order, num_blocks=nb)
+
+
+def make_prefill_inputs(spec: Spec) -> dict:
+    """Inputs for one prefill step: every sequence holds context_lens - q_len
+    cached tokens and appends q_len new ones (their K/V in new_key/new_value,
+    their queries in query, sequence-major).
+
+    Returns CPU tensors: context_lens [S]; free_order [NB]; k_pool/v_pool
+    [NB, Hkv, bs, D]; new_key/new_value [S * q_len, Hkv, D]; query
+    [S * q_len, Hq, D]; num_blocks."""
+    assert spec.q_len > 0
+    gen = torch.Generator().manual_seed(spec.seed)
+    dt = spec.torch_kv_dtype
+    ctx = context_lengths(spec, gen)
+    needed = int(sum((int(c) + spec.block_size - 1) // spec.block_size for c in ctx.tolist()))
+    nb = max(needed, int(math.ceil((spec.pool_factor or 1.0) * needed)))
+    free_order = torch.randperm(nb, generator=gen).to(torch.int32)
+    shape = (nb, spec.num_kv_heads, spec.block_size, spec.head_dim)
+    k_pool = _normal(gen, shape, spec.kv_scale, dt)
+    v_pool = _normal(gen, shape, spec.kv_scale, dt)
+    T = spec.num_seqs * spec.q_len
+    new_key = _normal(gen, (T, spec.num_kv_heads, spec.head_dim), spec.kv_scale, dt)
+    new_value = _normal(gen, (T, spec.num_kv_heads, spec.head_dim), spec.kv_scale, dt)
+    query = _normal(gen, (T, spec.num_heads, spec.head_dim), spec.q_scale, dt)
+    return dict(context_lens=ctx, free_order=free_order, k_pool=k_pool, v_pool=v_pool, new_key=new_key,
+                new_value=new_value, query=query, num_blocks=nb)

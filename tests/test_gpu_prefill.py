@@ -115,3 +115,50 @@ def test_prefill_rejects_queries_longer_than_context(pa):
                                c["tables"].numpy()[1:], np.array([50], np.int32), c["scale"], 16)
     assert_attention_close(out[ok:], ref, torch.float16, "valid sequence")
     assert torch.isnan(out[:ok]).all()                       # the skipped sequence is left untouched
+
+
+@pytest.mark.parametrize("name", ["prefill_llama7b_mha_bf16", "chunked_prefill_gqa_bf16"])
+def test_prefill_workloads_full_size(pa, name):
+    """The benchmark's prefill workloads at full size, in its launch
+    configuration (slot write of the new tokens, then prefill). Tables and
+    slots from the library pool match the oracle pool; sampled query rows
+    (tile edges, first and last tokens) match the oracle, each computed as the
+    last query of a context ending at that row's position."""
+    from oracle.block_pool import BlockPool as OPool, Sequence, append_tokens
+    from paged_kv_cache_340_b200.batch import build_prefill_batch, run_prefill_step
+    from paged_kv_cache_340_b200.workloads import SPECS, make_prefill_inputs
+    from _helpers import compact_for, raw
+    spec = SPECS[name]
+    inp = make_prefill_inputs(spec)
+    b = build_prefill_batch(spec, inp)
+    ctx = inp["context_lens"].numpy()
+    opool = OPool(int(inp["num_blocks"]), spec.block_size, policy="fifo", free_order=inp["free_order"].tolist())
+    oslots = []
+    for s, L in enumerate(ctx):
+        seq = Sequence()
+        append_tokens(opool, seq, int(L) - spec.q_len)
+        sl, _ = append_tokens(opool, seq, spec.q_len)
+        oslots += sl
+        assert list(b.host_tables[s, :len(seq.block_table)]) == seq.block_table
+    assert np.array_equal(b.host_slots, np.array(oslots, np.int32))
+    run_prefill_step(b)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_errors() == 0
+    k_host, v_host = inp["k_pool"], inp["v_pool"]
+    oracle.reshape_and_cache(raw(k_host), raw(v_host), raw(inp["new_key"]), raw(inp["new_value"]), np.array(oslots))
+    out = b.out.cpu()
+    q = inp["query"]
+    G = spec.num_heads // spec.num_kv_heads
+    rng = np.random.default_rng(5)
+    for s in (0, len(ctx) - 1):
+        L = int(ctx[s])
+        rows = sorted({0, 1, 63, 64, 127, 128, spec.q_len - 1, int(rng.integers(spec.q_len))})
+        for kvh in (0, spec.num_kv_heads - 1):
+            for i in rows:
+                pos = L - spec.q_len + i
+                kp, vp, tab = compact_for(k_host, v_host, b.host_tables[s], pos + 1, spec.block_size, kv_heads=[kvh])
+                qi = q[s * spec.q_len + i:s * spec.q_len + i + 1, kvh * G:(kvh + 1) * G]
+                ref = oracle.paged_prefill(f64(qi), np.array([0, 1], np.int32), kp, vp, tab,
+                                           np.array([pos + 1], np.int32), spec.scale, spec.block_size)
+                got = out[s * spec.q_len + i:s * spec.q_len + i + 1, kvh * G:(kvh + 1) * G]
+                assert_attention_close(got, ref, spec.torch_kv_dtype, f"{name} seq {s} kv {kvh} row {i}")
