@@ -48,7 +48,6 @@ constexpr int kKVHalf = kN * kHalfBytes;  // 8 KB
 constexpr int kQBytes = 2 * kQHalf;
 constexpr int kKVBytes = 2 * kKVHalf;   // one K or V tile
 constexpr int kPBytes = kM * kHalfBytes;  // 128 rows x 64 tokens
-constexpr int kStages = 2;
 constexpr int kSoftmaxWarps = 4;
 constexpr int kThreads = (kSoftmaxWarps + 1) * 32;
 constexpr int kTmemCols = 256;          // O: columns 0-127, S: 128-191
@@ -56,11 +55,14 @@ constexpr int kOCol = 0;
 constexpr int kSCol = 128;
 // shared memory (every operand region 1024-byte aligned for the swizzle)
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
-constexpr int kOffV = kOffK + kStages * kKVBytes;
-constexpr int kOffP = kOffV + kStages * kKVBytes;
+constexpr int kOffK = kOffQ + kQBytes;   // one K tile: reloaded as soon as S = Q K^T is done
+constexpr int kOffV = kOffK + kKVBytes;  // one V tile: reloaded as soon as O += P V is done
+constexpr int kOffP = kOffV + kKVBytes;
 constexpr int kOffBar = kOffP + 2 * kPBytes;  // P (and, for bf16, its low part)
-constexpr int kSmemBytes = 1024 + kOffBar + 16 * 8;
+constexpr int kSmemBytes = 1024 + kOffBar + 16 * 8;  // ~97 KB: two CTAs per SM
+// The running max is raised only when it grows by more than this (log2
+// units): probabilities then stay below 2^8 and O is rarely rescaled.
+constexpr float kRescaleThreshold = 8.f;
 
 struct Params {
     void *out;
@@ -163,7 +165,7 @@ template <> struct Pack16<__half> {
 // ----------------------------------------------------------------- kernel
 
 template <typename T, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const Params p) {
     constexpr bool kBf16 = std::is_same_v<T, __nv_bfloat16>;
@@ -181,7 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char *Pl = Ps + kPBytes;  // bf16 only: P - bf16(P)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBar);
     uint64_t *q_full = bars + 0;
-    uint64_t *kv_full = bars + 1;  // [2]
+    uint64_t *k_full = bars + 1;
+    uint64_t *v_full = bars + 2;
     uint64_t *s_full = bars + 3;
     uint64_t *p_full = bars + 4;
     uint64_t *o_done = bars + 5;
@@ -210,8 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        mbar_init(kv_full + 0, 1);
-        mbar_init(kv_full + 1, 1);
+        mbar_init(k_full, 1);
+        mbar_init(v_full, 1);
         mbar_init(s_full, 1);
         mbar_init(p_full, kSoftmaxWarps * 32);
         mbar_init(o_done, 1);
@@ -235,59 +238,58 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const int32_t *trow = p.block_tables + (size_t)s * p.max_blocks_per_seq;
             const int nblk = (ctx + p.block_size - 1) / p.block_size;
-            auto load_kv = [&](int j) {
-                const int b = j & 1;
-                unsigned char *kd = Ks + b * kKVBytes;
-                unsigned char *vd = Vs + b * kKVBytes;
-                mbar_arrive_expect_tx(kv_full + b, 2 * kKVBytes);
+            // Physical row of the 16-token group starting at token `tok` (past the
+            // pool's end when the sequence has no such block: the copy reads zeros).
+            auto group_row = [&](int tok) -> int {
+                const int lb = tok / p.block_size;
+                long long row = p.kv_rows;
+                if (lb < nblk) {
+                    const int id = __ldg(trow + lb);
+                    if (id >= 0 && id < p.num_blocks)
+                        row = ((long long)id * p.num_kv_heads + kvh) * p.block_size + (tok % p.block_size);
+                    else
+                        record_error(p.err, PA_DEVERR_BLOCK_ID);
+                }
+                return (int)row;
+            };
+            auto load_tile = [&](const CUtensorMap *map, unsigned char *dst, uint64_t *bar, int j) {
+                mbar_arrive_expect_tx(bar, kKVBytes);
 #pragma unroll
-                for (int g = 0; g < kN / 16; ++g) {  // 16-row groups of the tile
-                    const int tok = j * kN + g * 16;
-                    const int lb = tok / p.block_size;
-                    long long row = p.kv_rows;  // past the end: the copy fills zeros
-                    if (lb < nblk) {
-                        const int id = __ldg(trow + lb);
-                        if (id >= 0 && id < p.num_blocks)
-                            row = ((long long)id * p.num_kv_heads + kvh) * p.block_size + (tok % p.block_size);
-                        else
-                            record_error(p.err, PA_DEVERR_BLOCK_ID);
-                    }
+                for (int g = 0; g < kN / 16; ++g) {
+                    const int row = group_row(j * kN + g * 16);
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        tma_load_2d(kd + h * kKVHalf + g * 16 * kHalfBytes, &tmap_k, h * 64, (int)row, kv_full + b);
-                        tma_load_2d(vd + h * kKVHalf + g * 16 * kHalfBytes, &tmap_v, h * 64, (int)row, kv_full + b);
-                    }
+                    for (int h = 0; h < 2; ++h) tma_load_2d(dst + h * kKVHalf + g * 16 * kHalfBytes, map, h * 64, row, bar);
                 }
             };
             mbar_arrive_expect_tx(q_full, kQBytes);
             tma_load_3d(Qs, &tmap_q, 0, kvh * G, q0 + tok0, q_full);
             tma_load_3d(Qs + kQHalf, &tmap_q, 64, kvh * G, q0 + tok0, q_full);
-            load_kv(0);
-            if (ntiles > 1) load_kv(1);
+            load_tile(&tmap_k, Ks, k_full, 0);
+            load_tile(&tmap_v, Vs, v_full, 0);
+            const uint32_t qa = smem_addr(Qs), ka = smem_addr(Ks), va = smem_addr(Vs);
+            const uint32_t pa_ = smem_addr(Ps), pl_ = smem_addr(Pl);
             bool ok = true;
-            int waited_kv = 0;
+            int k_loaded = 1, k_waited = 0, v_loaded = 1, v_waited = 0;
             for (int j = 0; j < ntiles && ok; ++j) {
-                const int b = j & 1;
-                if (!mbar_wait(kv_full + b, (j >> 1) & 1) || (j == 0 && !mbar_wait(q_full, 0))) {
-                    ok = false;
-                    break;
-                }
-                waited_kv = j + 1;
+                const int par = j & 1;
+                if (!mbar_wait(k_full, par) || (j == 0 && !mbar_wait(q_full, 0))) { ok = false; break; }
+                k_waited = j + 1;
                 tc_fence_after();
-                const uint32_t qa = smem_addr(Qs), ka = smem_addr(Ks + b * kKVBytes);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
+                    const uint32_t off = (kk & 3) * 32;
                     umma(tmem + kSCol, sw128_desc(qa + (kk >> 2) * kQHalf + off, 16, 1024),
                          sw128_desc(ka + (kk >> 2) * kKVHalf + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(s_full);
-                if (!mbar_wait(p_full, j & 1)) {
-                    ok = false;
-                    break;
+                if (j + 1 < ntiles) {  // S done: the K buffer takes the next tile
+                    if (!mbar_wait(s_full, par)) { ok = false; break; }
+                    load_tile(&tmap_k, Ks, k_full, j + 1);
+                    k_loaded = j + 2;
                 }
+                if (!mbar_wait(p_full, par) || !mbar_wait(v_full, par)) { ok = false; break; }
+                v_waited = j + 1;
                 tc_fence_after();
-                const uint32_t pa_ = smem_addr(Ps), pl_ = smem_addr(Pl), va = smem_addr(Vs + b * kKVBytes);
 #pragma unroll
                 for (int kk = 0; kk < kN / 16; ++kk) {
                     const uint64_t vdesc = sw128_desc(va + kk * 16 * kHalfBytes, kKVHalf, 1024);
@@ -296,19 +298,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if constexpr (kBf16) umma(tmem + kOCol, sw128_desc(pl_ + kk * 32, 16, 1024), vdesc, kIdescPV, 1u);
                 }
                 umma_commit(o_done);
-                if (j + 2 < ntiles) {
-                    if (!mbar_wait(o_done, j & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    load_kv(j + 2);
+                if (j + 1 < ntiles) {  // O += P V done: the V buffer takes the next tile
+                    if (!mbar_wait(o_done, par)) { ok = false; break; }
+                    load_tile(&tmap_v, Vs, v_full, j + 1);
+                    v_loaded = j + 2;
                 }
             }
             if (!ok) {
                 record_error(p.err, PA_DEVERR_TIMEOUT);
                 *abort_flag = 1;
                 // let the copies this thread started land before the CTA leaves
-                for (int j = waited_kv; j < min(ntiles, waited_kv + 2); ++j) mbar_wait(kv_full + (j & 1), (j >> 1) & 1);
+                for (int j = k_waited; j < k_loaded; ++j) mbar_wait(k_full, j & 1);
+                for (int j = v_waited; j < v_loaded; ++j) mbar_wait(v_full, j & 1);
                 mbar_wait(q_full, 0);
                 // release the softmax warps from their waits
                 mbar_arrive(s_full);
@@ -340,8 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 x[c] = (kv0 + c <= pos) ? sv * p.scale_log2 : -INFINITY;
                 mx = fmaxf(mx, x[c]);
             }
-            const float mn = fmaxf(m_run, mx);
-            const float alpha = (mn == -INFINITY) ? 1.f : fast_exp2(m_run - mn);
+            // raise the running max only when it grows by more than the threshold
+            const bool raise = fmaxf(m_run, mx) - m_run > kRescaleThreshold;  // also the first finite max
+            const float mn = raise ? fmaxf(m_run, mx) : m_run;
+            const float alpha = raise ? fast_exp2(m_run - mn) : 1.f;  // 0 when m_run was -inf
             m_run = mn;
             float psum = 0.f;
 #pragma unroll
@@ -391,7 +394,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // V rows past the context: zero (both halves) before P V reads them
             const int zrow = max(0, ctx - kv0);
             if (zrow < kN) {
-                unsigned char *vt = Vs + (j & 1) * kKVBytes;
+                // V_j must have landed before its tail rows are overwritten
+                if (!mbar_wait(v_full, j & 1) || *(volatile int *)abort_flag) break;
+                unsigned char *vt = Vs;
                 const int nvec = (kN - zrow) * 2 * (kHalfBytes / 16);
                 for (int i = r; i < nvec; i += kSoftmaxWarps * 32) {
                     const int row = zrow + i / 16;
