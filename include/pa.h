@@ -298,6 +298,43 @@ int pa_pool_fork(pa_block_pool *pool, const int32_t *table, int num_tokens, int3
 /* Drops the sequence's reference to each of its blocks. */
 int pa_pool_release(pa_block_pool *pool, const int32_t *table, int num_tokens);
 
+/*
+ * Prefix cache over a host block pool ([P4] §3.2, Prefix Caching): a prompt
+ * prefix (e.g. a system prompt shared by many requests) gets its blocks, and
+ * its KV, once; later requests with the same prefix reuse them.
+ *   - pa_prefix_get_or_create: if this exact token list is cached, its use
+ *     count goes up by one and its block ids are written to block_ids
+ *     (*hit = 1). Otherwise ceil(num_tokens / block_size) blocks are taken
+ *     from the pool (PA_ERR_POOL_EXHAUSTED and nothing taken if the pool has
+ *     fewer free blocks), recorded with use count 1 and returned (*hit = 0);
+ *     the caller then writes the prefix's K/V into them. block_ids has room
+ *     for max_blocks ids (PA_ERR_CAPACITY, nothing changed, if too few);
+ *     *num_ids receives the count.
+ *   - pa_prefix_release: an unknown token list is ignored; otherwise the use
+ *     count drops by one and at zero every block of the entry is freed
+ *     (pa_pool_free) and the entry removed.
+ *   - The entry holds one pool reference per block. A sequence that maps the
+ *     prefix blocks into its own table row should take its own references
+ *     (pa_pool_fork over them) so that pa_pool_append copies a shared block
+ *     before writing into it.
+ * Entries are found by a 64-bit FNV-1a hash of the token ids, of which the
+ * low hash_bits bits are kept (0 = all 64; small values only make lookups
+ * slower), and a hit also needs equal token lists, so a hash collision never
+ * shares blocks. tokens: host int32 [num_tokens]. The cache keeps a pointer
+ * to the pool, which must outlive it; pa_prefix_cache_destroy frees no
+ * blocks. Not thread-safe.
+ */
+typedef struct pa_prefix_cache pa_prefix_cache;
+
+pa_prefix_cache *pa_prefix_cache_create(pa_block_pool *pool, int hash_bits);
+void pa_prefix_cache_destroy(pa_prefix_cache *cache);
+int pa_prefix_num_entries(const pa_prefix_cache *cache);
+int pa_prefix_get_or_create(pa_prefix_cache *cache, const int32_t *tokens, int num_tokens,
+                            int32_t *block_ids, int max_blocks, int *num_ids, int *hit);
+int pa_prefix_release(pa_prefix_cache *cache, const int32_t *tokens, int num_tokens);
+/* The use count of this token list (0 if it is not cached). */
+int pa_prefix_ref_count(pa_prefix_cache *cache, const int32_t *tokens, int num_tokens);
+
 #ifdef __cplusplus
 }
 #endif

@@ -39,6 +39,8 @@ EXPORTED = (
     "pa_choose_partition", "pa_copy_blocks", "pa_pool_create", "pa_pool_destroy", "pa_pool_num_free",
     "pa_pool_ref_count", "pa_pool_allocate", "pa_pool_share", "pa_pool_free", "pa_pool_append",
     "pa_pool_fork", "pa_pool_release", "pa_decode_splitk_static", "pa_prefill",
+    "pa_prefix_cache_create", "pa_prefix_cache_destroy", "pa_prefix_num_entries", "pa_prefix_get_or_create",
+    "pa_prefix_release", "pa_prefix_ref_count",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -83,6 +85,13 @@ def _load() -> ctypes.CDLL:
                                           i32, i32, vp]),
         "pa_prefill": (i32, [vp, vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32,
                              vp]),
+        "pa_prefix_cache_create": (vp, [vp, i32]),
+        "pa_prefix_cache_destroy": (None, [vp]),
+        "pa_prefix_num_entries": (i32, [vp]),
+        "pa_prefix_get_or_create": (i32, [vp, i32p, i32, i32p, i32, ctypes.POINTER(ctypes.c_int),
+                                          ctypes.POINTER(ctypes.c_int)]),
+        "pa_prefix_release": (i32, [vp, i32p, i32]),
+        "pa_prefix_ref_count": (i32, [vp, i32p, i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -311,3 +320,49 @@ class BlockPool:
 
     def release(self, table: np.ndarray, num_tokens: int) -> None:
         _check(_lib.pa_pool_release(self._h, _i32p(table), int(num_tokens)), "pa_pool_release")
+
+
+class PrefixCache:
+    """Prefix cache (pa_prefix_* calls) over a BlockPool: a token list's
+    blocks are taken once and reused while any request holds the prefix."""
+
+    def __init__(self, pool: BlockPool, hash_bits: int = 0):
+        self.pool = pool  # keeps the pool alive
+        h = _lib.pa_prefix_cache_create(pool._h, int(hash_bits))
+        if not h:
+            raise PagedAttentionError("pa_prefix_cache_create", -3)
+        self._h = ctypes.c_void_p(h)
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            _lib.pa_prefix_cache_destroy(h)
+            self._h = None
+
+    @staticmethod
+    def _tokens(tokens) -> np.ndarray:
+        return np.ascontiguousarray(np.asarray(tokens, dtype=np.int32).reshape(-1))
+
+    def get_or_create(self, tokens) -> Tuple[list, bool]:
+        """Returns (block ids, hit)."""
+        t = self._tokens(tokens)
+        cap = (t.shape[0] + self.pool.block_size - 1) // self.pool.block_size
+        ids = np.empty(max(1, cap), np.int32)
+        n, hit = ctypes.c_int(0), ctypes.c_int(0)
+        _check(_lib.pa_prefix_get_or_create(self._h, _i32p(t), t.shape[0], _i32p(ids), cap, ctypes.byref(n),
+                                            ctypes.byref(hit)), "pa_prefix_get_or_create")
+        return ids[: n.value].tolist(), bool(hit.value)
+
+    def release(self, tokens) -> None:
+        t = self._tokens(tokens)
+        _check(_lib.pa_prefix_release(self._h, _i32p(t), t.shape[0]), "pa_prefix_release")
+
+    def ref_count(self, tokens) -> int:
+        t = self._tokens(tokens)
+        rc = int(_lib.pa_prefix_ref_count(self._h, _i32p(t), t.shape[0]))
+        if rc < 0:
+            raise PagedAttentionError("pa_prefix_ref_count", rc)
+        return rc
+
+    def num_entries(self) -> int:
+        return int(_lib.pa_prefix_num_entries(self._h))

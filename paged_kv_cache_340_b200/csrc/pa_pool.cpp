@@ -11,9 +11,11 @@
 //   * before writing into a block whose count is above 1, take a new block,
 //     record (old, new) for the device copy, drop the old block's count and
 //     repoint the table; a block with count 1 is written in place.
+#include <algorithm>
 #include <cstdint>
 #include <deque>
 #include <new>
+#include <unordered_map>
 #include <vector>
 
 #include "pa.h"
@@ -167,6 +169,132 @@ int pa_pool_release(pa_block_pool *pool, const int32_t *table, int num_tokens) {
         if (!pool->valid(table[j]) || pool->ref[table[j]] <= 0) return PA_ERR_POOL_STATE;
     for (int j = 0; j < nb; ++j) pool->drop(table[j]);
     return PA_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------ prefix cache
+//
+// [P4 "PagedAttention 实现细节", §3.2]: a prompt prefix (a system prompt) is
+// computed once and its blocks are reused by every request that starts with
+// it. get_or_create: a cached prompt's use count goes up and its blocks are
+// returned; an unseen prompt gets ceil(len / bs) fresh blocks (all or none)
+// and use count 1. release: the count drops and at zero the blocks go back
+// to the pool and the entry is removed; an unknown prompt is ignored.
+//
+// Entries are bucketed by a 64-bit FNV-1a hash of the token ids (the
+// published FNV-1a definition: offset basis 14695981039346656037, prime
+// 1099511628211, over the ids' little-endian bytes), keeping the low
+// hash_bits bits, and a hit also requires equal token lists: two prompts
+// whose hashes agree never share blocks.
+
+struct pa_prefix_cache {
+    struct Entry {
+        std::vector<int32_t> tokens;
+        std::vector<int32_t> blocks;
+        int ref_count;
+    };
+    pa_block_pool *pool;
+    uint64_t mask;
+    std::unordered_map<uint64_t, std::vector<Entry>> buckets;
+    int entries = 0;
+
+    uint64_t key(const int32_t *t, int n) const {
+        uint64_t h = 14695981039346656037ull;
+        for (int i = 0; i < n; ++i) {
+            const uint32_t v = (uint32_t)t[i];
+            for (int b = 0; b < 4; ++b) {
+                h ^= (v >> (8 * b)) & 0xffu;
+                h *= 1099511628211ull;
+            }
+        }
+        return h & mask;
+    }
+
+    // The entry for this token list, or null; *bucket receives its bucket.
+    Entry *find(const int32_t *t, int n, std::vector<Entry> **bucket) {
+        auto it = buckets.find(key(t, n));
+        if (it == buckets.end()) {
+            *bucket = nullptr;
+            return nullptr;
+        }
+        *bucket = &it->second;
+        for (Entry &e : it->second)
+            if ((int)e.tokens.size() == n && std::equal(e.tokens.begin(), e.tokens.end(), t)) return &e;
+        return nullptr;
+    }
+};
+
+extern "C" {
+
+pa_prefix_cache *pa_prefix_cache_create(pa_block_pool *pool, int hash_bits) {
+    if (!pool || hash_bits < 0 || hash_bits > 64) return nullptr;
+    pa_prefix_cache *c = new (std::nothrow) pa_prefix_cache();
+    if (!c) return nullptr;
+    c->pool = pool;
+    c->mask = (hash_bits == 0 || hash_bits == 64) ? ~0ull : ((1ull << hash_bits) - 1);
+    return c;
+}
+
+void pa_prefix_cache_destroy(pa_prefix_cache *cache) { delete cache; }
+
+int pa_prefix_num_entries(const pa_prefix_cache *cache) { return cache ? cache->entries : PA_ERR_NULL; }
+
+int pa_prefix_get_or_create(pa_prefix_cache *cache, const int32_t *tokens, int num_tokens, int32_t *block_ids,
+                            int max_blocks, int *num_ids, int *hit) {
+    if (!cache || !num_ids || !hit || (num_tokens > 0 && !tokens)) return PA_ERR_NULL;
+    if (num_tokens < 0 || max_blocks < 0) return PA_ERR_SHAPE;
+    pa_block_pool *pool = cache->pool;
+    const int nb = (num_tokens + pool->block_size - 1) / pool->block_size;
+    if (nb > max_blocks) return PA_ERR_CAPACITY;
+    if (nb > 0 && !block_ids) return PA_ERR_NULL;
+    std::vector<pa_prefix_cache::Entry> *bucket = nullptr;
+    pa_prefix_cache::Entry *e = cache->find(tokens, num_tokens, &bucket);
+    if (e) {
+        ++e->ref_count;
+        std::copy(e->blocks.begin(), e->blocks.end(), block_ids);
+        *num_ids = nb;
+        *hit = 1;
+        return PA_OK;
+    }
+    if ((int)pool->free_list.size() < nb) return PA_ERR_POOL_EXHAUSTED;
+    pa_prefix_cache::Entry ne;
+    ne.tokens.assign(tokens, tokens + num_tokens);
+    ne.blocks.resize(nb);
+    for (int j = 0; j < nb; ++j) pool->take(&ne.blocks[j]);
+    ne.ref_count = 1;
+    std::copy(ne.blocks.begin(), ne.blocks.end(), block_ids);
+    if (!bucket) bucket = &cache->buckets[cache->key(tokens, num_tokens)];
+    bucket->push_back(std::move(ne));
+    ++cache->entries;
+    *num_ids = nb;
+    *hit = 0;
+    return PA_OK;
+}
+
+int pa_prefix_release(pa_prefix_cache *cache, const int32_t *tokens, int num_tokens) {
+    if (!cache || (num_tokens > 0 && !tokens)) return PA_ERR_NULL;
+    if (num_tokens < 0) return PA_ERR_SHAPE;
+    std::vector<pa_prefix_cache::Entry> *bucket = nullptr;
+    pa_prefix_cache::Entry *e = cache->find(tokens, num_tokens, &bucket);
+    if (!e) return PA_OK;
+    if (e->ref_count == 1)  // the blocks go back: each must still be held
+        for (int32_t b : e->blocks)
+            if (!cache->pool->valid(b) || cache->pool->ref[b] <= 0) return PA_ERR_POOL_STATE;
+    if (--e->ref_count > 0) return PA_OK;
+    for (int32_t b : e->blocks) cache->pool->drop(b);
+    bucket->erase(bucket->begin() + (e - bucket->data()));
+    if (bucket->empty()) cache->buckets.erase(cache->key(tokens, num_tokens));
+    --cache->entries;
+    return PA_OK;
+}
+
+int pa_prefix_ref_count(pa_prefix_cache *cache, const int32_t *tokens, int num_tokens) {
+    if (!cache || (num_tokens > 0 && !tokens)) return PA_ERR_NULL;
+    if (num_tokens < 0) return PA_ERR_SHAPE;
+    std::vector<pa_prefix_cache::Entry> *bucket = nullptr;
+    const pa_prefix_cache::Entry *e = cache->find(tokens, num_tokens, &bucket);
+    return e ? e->ref_count : 0;
 }
 
 }  // extern "C"
