@@ -115,3 +115,28 @@ def release(pool: BlockPool, seq: Sequence) -> None:
         pool.free(bid)
     seq.block_table.clear()
     seq.num_tokens = 0
+
+
+def beam_step(pool: BlockPool, beams: List[Sequence], parents: Sequence_[int]) -> Tuple[
+        List[Sequence], List[int], List[Tuple[int, int]]]:
+    """One beam-search step over the pool: new beam i continues old beam
+    parents[i] and writes one new token. In this order: every new beam forks
+    its parent (counts up), every old beam is released in beam order (blocks
+    reaching count 0 return to the free list), then the new beams write their
+    token in beam order, each by the copy-on-write rule. Returns (new beams,
+    slot of each new beam's token, copy-on-write pairs in the order taken).
+    [P2 "PagedAttention原理与KV Cache显存优化", §3.4 (beam search shares blocks
+    between beams, copy on write when one diverges)]; [P4 "PagedAttention
+    实现细节", §3.3 (the copy-on-write rule)]. The order of the three phases is
+    a reading: the pages give the rule, not a schedule; forking before
+    releasing keeps a parent's blocks alive for its children."""
+    children = [fork(pool, beams[p]) for p in parents]
+    for b in beams:
+        release(pool, b)
+    slots: List[int] = []
+    cow: List[Tuple[int, int]] = []
+    for c in children:
+        s, pairs = append_tokens(pool, c, 1)
+        slots += s
+        cow += pairs
+    return children, slots, cow
