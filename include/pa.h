@@ -77,6 +77,7 @@ typedef enum pa_status {
 #define PA_DEVERR_CONTEXT 0x4u   /* context_len < 0, or longer than its table row / max_context_len: clamped */
 #define PA_DEVERR_TIMEOUT 0x8u   /* an on-chip pipeline wait ran past its bound: output undefined */
 #define PA_DEVERR_PAIR 0x10u     /* copy pair with an id outside [0, num_blocks): skipped */
+#define PA_DEVERR_POOL 0x20u     /* device pool: exhausted, no table room, or state not initialised: step not applied */
 
 /* Text for a pa_status value (static storage, never NULL). */
 const char *pa_status_string(int status);
@@ -248,6 +249,13 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pairs, i
                    int num_blocks, int num_kv_heads, int head_dim, int block_size,
                    pa_dtype kv_dtype, cudaStream_t stream);
 
+/* As pa_copy_blocks, but the pair count is read on the device from
+ * *num_pairs (device int32, at most max_pairs): the form that follows
+ * pa_beam_step without a host round trip. */
+int pa_copy_blocks_counted(void *k_cache, void *v_cache, const int64_t *src_dst_pairs,
+                           const int32_t *num_pairs, int max_pairs, int num_blocks, int num_kv_heads,
+                           int head_dim, int block_size, pa_dtype kv_dtype, cudaStream_t stream);
+
 /*
  * Host block pool (no device memory): free list, reference counts and the
  * copy-on-write decision. These are plain host calls on host memory.
@@ -334,6 +342,61 @@ int pa_prefix_get_or_create(pa_prefix_cache *cache, const int32_t *tokens, int n
 int pa_prefix_release(pa_prefix_cache *cache, const int32_t *tokens, int num_tokens);
 /* The use count of this token list (0 if it is not cached). */
 int pa_prefix_ref_count(pa_prefix_cache *cache, const int32_t *tokens, int num_tokens);
+
+/*
+ * Device block pool and the beam-search step on the GPU.
+ *
+ * The pool's state lives in one caller-allocated DEVICE buffer of
+ * pa_dpool_state_bytes(num_blocks) bytes (16-byte aligned), int32 words:
+ *   [0] num_blocks  [1] block_size  [2] policy  [3] head  [4] count
+ *   [5] a marker set by pa_dpool_init  [6..7] reserved
+ *   ref   = words + PA_DPOOL_HEADER_WORDS          [num_blocks] reference counts
+ *   ring  = ref + num_blocks                       [num_blocks] free list: entries
+ *           ring[(head + k) % num_blocks], k < count, front first
+ *   then four scratch arrays of num_blocks words each (all zero / -1 between
+ *   calls). The library keeps no pointer to it.
+ * Same rules as the host pool: PA_POOL_FIFO takes the free list's front,
+ * PA_POOL_LIFO its back; freed blocks go to the back.
+ */
+#define PA_DPOOL_HEADER_WORDS 8
+#define PA_DPOOL_ARRAYS 6
+
+size_t pa_dpool_state_bytes(int num_blocks);
+
+/* Every block free, counts 0. free_order (device int32 [num_blocks],
+ * nullable) gives the initial free list, else 0 .. num_blocks-1; if it is
+ * not a permutation the state is left unusable and PA_DEVERR_POOL is set. */
+int pa_dpool_init(void *state, int num_blocks, int block_size, int policy, const int32_t *free_order,
+                  cudaStream_t stream);
+
+/*
+ * pa_beam_step -- one beam-search step on the device ([P2] §3.4: beams share
+ * blocks and copy one before writing into it; [P4] §3.3: the copy-on-write
+ * rule). New beam i (i < num_new) continues old beam parents[i] and writes
+ * one token. The result equals, run one after another: every new beam forks
+ * its parent (counts up); every old beam is released, beams in order and each
+ * table in order (a block reaching 0 goes to the back of the free list);
+ * every new beam writes its token in beam order: at a block boundary it
+ * takes a free block, else if its block's count is above 1 it takes a free
+ * block, appends (old, new) to cow_pairs and drops the old count, else it
+ * writes in place.
+ * Inputs (device): old_tables [num_old, max_blocks_per_seq] and
+ * old_context_lens [num_old] (entries past ceil(ctx / block_size) are not
+ * read), parents [num_new] in [0, num_old). Outputs (device):
+ * new_tables [num_new, max_blocks_per_seq] (-1 past the blocks in use; must
+ * not overlap old_tables), new_context_lens [num_new] = parent's + 1,
+ * slot_mapping [num_new] (the new tokens' slots, for pa_reshape_and_cache),
+ * cow_pairs int64 [num_new, 2] and *num_cow (for pa_copy_blocks_counted).
+ * A table row never lists a block twice (the pool never makes one).
+ * Any error (a bad parent, context or block id, a free list too short, no
+ * table room for the new token, an uninitialised state) applies nothing:
+ * the state is unchanged, every slot is -1, *num_cow = 0 and a PA_DEVERR_*
+ * bit is set. Runs as one CTA; calls on one state must not overlap.
+ */
+int pa_beam_step(void *state, int num_blocks, int block_size, const int32_t *old_tables,
+                 const int32_t *old_context_lens, int num_old, const int32_t *parents, int num_new,
+                 int32_t *new_tables, int32_t *new_context_lens, int max_blocks_per_seq,
+                 int32_t *slot_mapping, int64_t *cow_pairs, int32_t *num_cow, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -30,6 +30,8 @@ PA_DEVERR_SLOT = 0x2
 PA_DEVERR_CONTEXT = 0x4
 PA_DEVERR_TIMEOUT = 0x8
 PA_DEVERR_PAIR = 0x10
+PA_DEVERR_POOL = 0x20
+PA_DPOOL_HEADER_WORDS = 8
 
 PA_POOL_LIFO, PA_POOL_FIFO = 0, 1
 
@@ -40,7 +42,8 @@ EXPORTED = (
     "pa_pool_ref_count", "pa_pool_allocate", "pa_pool_share", "pa_pool_free", "pa_pool_append",
     "pa_pool_fork", "pa_pool_release", "pa_decode_splitk_static", "pa_prefill",
     "pa_prefix_cache_create", "pa_prefix_cache_destroy", "pa_prefix_num_entries", "pa_prefix_get_or_create",
-    "pa_prefix_release", "pa_prefix_ref_count",
+    "pa_prefix_release", "pa_prefix_ref_count", "pa_copy_blocks_counted", "pa_dpool_state_bytes", "pa_dpool_init",
+    "pa_beam_step",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -92,6 +95,10 @@ def _load() -> ctypes.CDLL:
                                           ctypes.POINTER(ctypes.c_int)]),
         "pa_prefix_release": (i32, [vp, i32p, i32]),
         "pa_prefix_ref_count": (i32, [vp, i32p, i32]),
+        "pa_copy_blocks_counted": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
+        "pa_dpool_state_bytes": (sz, [i32]),
+        "pa_dpool_init": (i32, [vp, i32, i32, i32, vp, vp]),
+        "pa_beam_step": (i32, [vp, i32, i32, vp, vp, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -232,6 +239,63 @@ def pa_copy_blocks(k_cache, v_cache, src_dst_pairs, stream=None) -> None:
     rc = _lib.pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(src_dst_pairs) if n else None, n, NB, Hkv, D,
                              bs, _dtype(k_cache), _stream(stream))
     _check(rc, "pa_copy_blocks")
+
+
+def pa_copy_blocks_counted(k_cache, v_cache, src_dst_pairs, num_pairs, stream=None) -> None:
+    """pa_copy_blocks over the first num_pairs[0] (a device int32, read by the
+    kernel) rows of src_dst_pairs [max_pairs, 2] int64."""
+    NB, Hkv, bs, D = k_cache.shape
+    m = src_dst_pairs.shape[0]
+    rc = _lib.pa_copy_blocks_counted(_ptr(k_cache), _ptr(v_cache), _ptr(src_dst_pairs) if m else None,
+                                     _ptr(num_pairs) if m else None, m, NB, Hkv, D, bs, _dtype(k_cache),
+                                     _stream(stream))
+    _check(rc, "pa_copy_blocks_counted")
+
+
+class DevicePool:
+    """Device block pool (pa_dpool_* calls): the state lives in a device int32
+    tensor; ``ref`` and ``ring`` are views of its reference counts and free-list
+    ring, ``header`` of [num_blocks, block_size, policy, head, count, marker]."""
+
+    def __init__(self, num_blocks: int, block_size: int, policy: int = PA_POOL_LIFO, free_order=None,
+                 device="cuda", stream=None):
+        self.num_blocks, self.block_size, self.policy = num_blocks, block_size, policy
+        nbytes = int(_lib.pa_dpool_state_bytes(num_blocks))
+        if nbytes == 0:
+            raise PagedAttentionError("pa_dpool_state_bytes", -3)
+        self.state = torch.empty(nbytes // 4, dtype=torch.int32, device=device)
+        fo = None
+        if free_order is not None:
+            fo = torch.as_tensor(np.asarray(free_order, dtype=np.int32)).to(device)
+        _check(_lib.pa_dpool_init(_ptr(self.state), num_blocks, block_size, policy, _ptr(fo), _stream(stream)),
+               "pa_dpool_init")
+        self._keep = fo
+        h = PA_DPOOL_HEADER_WORDS
+        self.header = self.state[:6]
+        self.ref = self.state[h:h + num_blocks]
+        self.ring = self.state[h + num_blocks:h + 2 * num_blocks]
+
+    def free_list(self) -> list:
+        """The free list, front first (synchronises)."""
+        hdr = self.header.cpu().tolist()
+        ring = self.ring.cpu().tolist()
+        return [ring[(hdr[3] + k) % self.num_blocks] for k in range(hdr[4])]
+
+
+def pa_beam_step(pool: DevicePool, old_tables, old_context_lens, parents, new_tables, new_context_lens,
+                 slot_mapping, cow_pairs, num_cow, stream=None) -> None:
+    """One beam-search step on the device: new beam i continues old beam
+    parents[i] and writes one token (all tensors on the device; see pa.h)."""
+    num_old = old_context_lens.shape[0]
+    num_new = parents.shape[0]
+    mb = new_tables.shape[1] if new_tables.dim() == 2 else old_tables.shape[1]
+    rc = _lib.pa_beam_step(_ptr(pool.state), pool.num_blocks, pool.block_size,
+                           _ptr(old_tables) if num_old else None, _ptr(old_context_lens) if num_old else None,
+                           num_old, _ptr(parents) if num_new else None, num_new,
+                           _ptr(new_tables) if num_new else None, _ptr(new_context_lens) if num_new else None, mb,
+                           _ptr(slot_mapping) if num_new else None, _ptr(cow_pairs) if num_new else None,
+                           _ptr(num_cow), _stream(stream))
+    _check(rc, "pa_beam_step")
 
 
 def pa_read_device_errors(stream=None) -> int:

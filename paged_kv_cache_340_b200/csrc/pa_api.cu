@@ -330,8 +330,71 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pairs, i
     unsigned int *err = nullptr;
     if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
     const size_t block_bytes = (size_t)num_kv_heads * block_size * head_dim * eb;
-    cudaError_t e = launch_copy_blocks(k_cache, v_cache, src_dst_pairs, num_pairs, num_blocks,
+    cudaError_t e = launch_copy_blocks(k_cache, v_cache, src_dst_pairs, num_pairs, nullptr, num_blocks,
                                        block_bytes, err, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_copy_blocks_counted(void *k_cache, void *v_cache, const int64_t *src_dst_pairs,
+                           const int32_t *num_pairs, int max_pairs, int num_blocks, int num_kv_heads,
+                           int head_dim, int block_size, pa_dtype kv_dtype, cudaStream_t stream) {
+    if (max_pairs < 0 || num_blocks < 0 || num_kv_heads <= 0) return PA_ERR_SHAPE;
+    const int eb = elt_bytes(kv_dtype);
+    if (eb == 0) return PA_ERR_DTYPE;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_HEAD_DIM;
+    if (block_size != 16 && block_size != 32) return PA_ERR_BLOCK_SIZE;
+    if (max_pairs == 0) return PA_OK;
+    if (!k_cache || !v_cache || !src_dst_pairs || !num_pairs) return PA_ERR_NULL;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(src_dst_pairs, 8) || !aligned(num_pairs, 4))
+        return PA_ERR_ALIGN;
+    unsigned int *err = nullptr;
+    if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    const size_t block_bytes = (size_t)num_kv_heads * block_size * head_dim * eb;
+    cudaError_t e = launch_copy_blocks(k_cache, v_cache, src_dst_pairs, max_pairs, num_pairs, num_blocks,
+                                       block_bytes, err, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+size_t pa_dpool_state_bytes(int num_blocks) {
+    if (num_blocks <= 0) return 0;
+    return (PA_DPOOL_HEADER_WORDS + (size_t)PA_DPOOL_ARRAYS * num_blocks) * sizeof(int32_t);
+}
+
+int pa_dpool_init(void *state, int num_blocks, int block_size, int policy, const int32_t *free_order,
+                  cudaStream_t stream) {
+    if (num_blocks <= 0 || block_size <= 0 || num_blocks > INT_MAX / PA_DPOOL_ARRAYS) return PA_ERR_SHAPE;
+    if (policy != PA_POOL_LIFO && policy != PA_POOL_FIFO) return PA_ERR_SHAPE;
+    if (!state) return PA_ERR_NULL;
+    if (!aligned(state, 16) || (free_order && !aligned(free_order, 4))) return PA_ERR_ALIGN;
+    unsigned int *err = nullptr;
+    if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    cudaError_t e = launch_dpool_init(static_cast<int32_t *>(state), num_blocks, block_size, policy, free_order,
+                                      err, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_beam_step(void *state, int num_blocks, int block_size, const int32_t *old_tables,
+                 const int32_t *old_context_lens, int num_old, const int32_t *parents, int num_new,
+                 int32_t *new_tables, int32_t *new_context_lens, int max_blocks_per_seq,
+                 int32_t *slot_mapping, int64_t *cow_pairs, int32_t *num_cow, cudaStream_t stream) {
+    if (num_blocks <= 0 || block_size <= 0 || num_old < 0 || num_new < 0 || max_blocks_per_seq <= 0)
+        return PA_ERR_SHAPE;
+    if ((long long)num_old * max_blocks_per_seq >= INT_MAX || (long long)num_new * max_blocks_per_seq >= INT_MAX ||
+        (long long)num_blocks * block_size >= INT_MAX)
+        return PA_ERR_SHAPE;
+    if (!state || !num_cow || (num_old > 0 && (!old_tables || !old_context_lens)) ||
+        (num_new > 0 && (!parents || !new_tables || !new_context_lens || !slot_mapping || !cow_pairs)))
+        return PA_ERR_NULL;
+    if (num_new > 0 && num_old > 0 && new_tables == old_tables) return PA_ERR_SHAPE;
+    if (!aligned(state, 16) || !aligned(num_cow, 4) || !aligned(old_tables, 4) || !aligned(old_context_lens, 4) ||
+        !aligned(parents, 4) || !aligned(new_tables, 4) || !aligned(new_context_lens, 4) ||
+        !aligned(slot_mapping, 4) || !aligned(cow_pairs, 8))
+        return PA_ERR_ALIGN;
+    unsigned int *err = nullptr;
+    if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    cudaError_t e = launch_beam_step(static_cast<int32_t *>(state), old_tables, old_context_lens, num_old, parents,
+                                     num_new, new_tables, new_context_lens, max_blocks_per_seq, slot_mapping,
+                                     cow_pairs, num_cow, num_blocks, block_size, err, stream);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

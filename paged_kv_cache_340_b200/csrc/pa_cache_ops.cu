@@ -44,8 +44,9 @@ __global__ void __launch_bounds__(256)
 // the pairs, grid.y picks K (0) or V (1), grid.z splits a block into chunks.
 __global__ void __launch_bounds__(256)
     copy_blocks_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
-                       const int64_t *__restrict__ pairs, int num_blocks, long long vecs_per_block,
-                       unsigned int *err) {
+                       const int64_t *__restrict__ pairs, const int32_t *__restrict__ pair_count,
+                       int num_blocks, long long vecs_per_block, unsigned int *err) {
+    if (pair_count && (int)blockIdx.x >= __ldg(pair_count)) return;  // past the device-side count
     const int64_t src = __ldg(pairs + 2 * blockIdx.x);
     const int64_t dst = __ldg(pairs + 2 * blockIdx.x + 1);
     if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
@@ -80,8 +81,8 @@ cudaError_t launch_reshape_and_cache(const void *key, const void *value, void *k
 }
 
 cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *pairs, int num_pairs,
-                               int num_blocks, size_t block_bytes, unsigned int *err,
-                               cudaStream_t stream) {
+                               const int32_t *pair_count, int num_blocks, size_t block_bytes,
+                               unsigned int *err, cudaStream_t stream) {
     if (num_pairs == 0) return cudaSuccess;
     const long long vecs = (long long)(block_bytes / 16);
     // about 16 KiB per CTA
@@ -90,8 +91,8 @@ cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *pair
     if (chunks > 65535) chunks = 65535;
     dim3 grid((unsigned)num_pairs, 2, (unsigned)chunks);
     copy_blocks_kernel<<<grid, 256, 0, stream>>>(static_cast<uint4 *>(k_cache),
-                                                 static_cast<uint4 *>(v_cache), pairs, num_blocks,
-                                                 vecs, err);
+                                                 static_cast<uint4 *>(v_cache), pairs, pair_count,
+                                                 num_blocks, vecs, err);
     return cudaGetLastError();
 }
 

@@ -45,9 +45,18 @@ cudaError_t launch_reshape_and_cache(const void *key, const void *value, void *k
                                      int num_blocks, int num_kv_heads, int row_bytes,
                                      int block_size, unsigned int *err, cudaStream_t stream);
 
+// pair_count (nullable, device): only the first *pair_count of num_pairs pairs are copied.
 cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *pairs, int num_pairs,
-                               int num_blocks, size_t block_bytes, unsigned int *err,
-                               cudaStream_t stream);
+                               const int32_t *pair_count, int num_blocks, size_t block_bytes,
+                               unsigned int *err, cudaStream_t stream);
+
+cudaError_t launch_dpool_init(int32_t *state, int num_blocks, int block_size, int policy,
+                              const int32_t *free_order, unsigned int *err, cudaStream_t stream);
+
+cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const int32_t *old_ctx, int num_old,
+                             const int32_t *parents, int num_new, int32_t *new_tables, int32_t *new_ctx,
+                             int max_blocks, int32_t *slots, int64_t *cow_pairs, int32_t *num_cow,
+                             int num_blocks, int block_size, unsigned int *err, cudaStream_t stream);
 
 // Device address of the current device's error word (cached per device).
 cudaError_t device_error_word(unsigned int **word);

@@ -178,3 +178,34 @@ def test_pool_errors(pa):
     with pytest.raises(pa.PagedAttentionError) as e:
         pool2.append(small, 0, 5)
     assert e.value.status == -13
+
+
+def test_device_pool_host_checks(pa):
+    """pa_dpool_* / pa_beam_step / pa_copy_blocks_counted argument checks
+    return before any device work (fake device addresses are never touched)."""
+    lib = pa._lib
+    assert lib.pa_dpool_state_bytes(10) == (pa.PA_DPOOL_HEADER_WORDS + 6 * 10) * 4
+    assert lib.pa_dpool_state_bytes(0) == 0
+    fake = 1 << 40                                       # 16-byte aligned, never dereferenced
+    assert lib.pa_dpool_init(None, 10, 16, 0, None, None) == -1
+    assert lib.pa_dpool_init(fake, 0, 16, 0, None, None) == -3
+    assert lib.pa_dpool_init(fake, 10, 16, 7, None, None) == -3
+    assert lib.pa_dpool_init(fake + 4, 10, 16, 0, None, None) == -7
+    args = dict(old_t=fake, old_c=fake, par=fake, new_t=fake + 4096, new_c=fake, slots=fake, cow=fake, ncow=fake)
+
+    def step(state=fake, nb=64, bs=16, num_old=2, num_new=2, mb=4, **kw):
+        a = dict(args, **kw)
+        return lib.pa_beam_step(state, nb, bs, a["old_t"], a["old_c"], num_old, a["par"], num_new, a["new_t"],
+                                a["new_c"], mb, a["slots"], a["cow"], a["ncow"], None)
+    assert step(state=None) == -1
+    assert step(ncow=None) == -1
+    assert step(par=None) == -1
+    assert step(nb=0) == -3
+    assert step(mb=0) == -3
+    assert step(num_old=-1) == -3
+    assert step(num_old=1 << 20, mb=1 << 12) == -3      # flattened table index past int32
+    assert step(new_t=fake) == -3                        # output tables alias the input tables
+    assert step(cow=fake + 4) == -7
+    assert lib.pa_copy_blocks_counted(fake, fake, fake, None, 4, 8, 2, 128, 16, 1, None) == -1
+    assert lib.pa_copy_blocks_counted(fake, fake, fake, fake, 4, 8, 2, 100, 16, 1, None) == -5
+    assert lib.pa_copy_blocks_counted(fake, fake, fake, fake, 0, 8, 2, 128, 16, 1, None) == 0
