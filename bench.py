@@ -464,6 +464,118 @@ def measure_prefill(name: str, steps: int, warmup: int):
     return res
 
 
+def measure_beam(name: str, steps: int, warmup: int, host_steps: int = 30):
+    """Beam-search decode steps with the beam step on the device (beam step,
+    counted copy, slot write, decode; no host round trip), each step replayed
+    as a CUDA graph; and for context the same steps through the host pool,
+    where each step must read the beams' parents back (a synchronisation) and
+    upload tables, slots and pairs."""
+    from paged_kv_cache_340_b200 import pa_copy_blocks, pa_decode, pa_reshape_and_cache
+    from paged_kv_cache_340_b200.batch import beam_decode_bytes, build_beam_batch, host_beam_step, run_beam_step
+    from paged_kv_cache_340_b200.workloads import SPECS, make_beam_inputs
+    spec = SPECS[name]
+    b = build_beam_batch(spec, make_beam_inputs(spec))
+    G = b.parents.shape[0]                               # distinct steps; graph k runs step k (mod G)
+    warmup = -(-warmup // G) * G
+    steps = min(steps, spec.max_divergent - warmup - host_steps - 3 * G - 12)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            run_beam_step(b, stream=stream)
+    torch.cuda.synchronize()
+    # one graph per distinct step, each with events between its launches
+    graphs, evs = [], []
+    with torch.cuda.stream(stream):
+        for k in range(G):
+            ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]  # recorded on replay
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                run_beam_step(b, stream=stream, events=ev)
+            graphs.append(g)
+            evs.append(ev)
+    b.steps_done -= G                                    # capturing ran nothing
+    first = b.steps_done
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(steps):
+            graphs[b.steps_done % G].replay()
+            b.steps_done += 1
+        t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    by = statistics.fmean(beam_decode_bytes(b, first + i) for i in range(steps))
+    # per-kernel times: replay each graph alone and read its own events
+    samples = []
+    with torch.cuda.stream(stream):
+        while b.steps_done % G:
+            graphs[b.steps_done % G].replay()
+            b.steps_done += 1
+        for _ in range(2):
+            for k in range(G):
+                graphs[k].replay()
+                b.steps_done += 1
+                torch.cuda.synchronize()
+                e = evs[k]
+                samples.append([e[i].elapsed_time(e[i + 1]) for i in range(4)])
+    kern = [statistics.fmean(x[i] for x in samples) for i in range(4)]
+    dec_by = statistics.fmean(beam_decode_bytes(b, b.steps_done - 1 - i) for i in range(len(samples)))
+    # the wall time of one step when the host waits for its result
+    wall = []
+    with torch.cuda.stream(stream):
+        for _ in range(12):
+            t = time.perf_counter()
+            graphs[b.steps_done % G].replay()
+            b.steps_done += 1
+            stream.synchronize()
+            wall.append(time.perf_counter() - t)
+    del graphs
+    # host-pool path over the same kind of steps, from the state the device has now
+    W = b.tables[0].shape[0]
+    cur = b.steps_done % 2
+    tables = b.tables[cur].cpu().numpy()
+    ctx = b.context_lens[cur].cpu().numpy()
+    from paged_kv_cache_340_b200 import BlockPool
+    ref, fl = b.pool.ref.cpu().numpy(), b.pool.free_list()
+    hp = BlockPool(b.num_blocks, spec.block_size, b.pool.policy, free_order=np.arange(b.num_blocks, dtype=np.int32))
+    for _ in range(b.num_blocks):
+        hp.allocate()
+    for blk in range(b.num_blocks):
+        for _ in range(int(ref[blk]) - 1):
+            hp.share(blk)
+    for blk in fl:
+        hp.free(int(blk))
+    dt_tab = torch.empty_like(b.tables[0])
+    dt_ctx = torch.empty_like(b.context_lens[0])
+    dt_slots = torch.empty_like(b.slot_mapping)
+    host = []
+    for i in range(host_steps):
+        t = time.perf_counter()
+        k = (b.steps_done + i) % G
+        parents = b.parents[k].cpu().numpy()             # read back: a synchronisation
+        tables, ctx, slots, cow = host_beam_step(hp, tables, ctx, parents)
+        dt_tab.copy_(torch.from_numpy(tables))
+        dt_ctx.copy_(torch.from_numpy(ctx))
+        dt_slots.copy_(torch.from_numpy(slots))
+        if cow.shape[0]:
+            pa_copy_blocks(b.k_cache, b.v_cache, torch.from_numpy(cow).cuda())
+        pa_reshape_and_cache(b.new_key[k], b.new_value[k], b.k_cache, b.v_cache, dt_slots)
+        pa_decode(b.out, b.query[k], b.k_cache, b.v_cache, dt_tab, dt_ctx, spec.scale)
+        torch.cuda.synchronize()
+        host.append(time.perf_counter() - t)
+    res = {"ms_per_step": round(ms, 4), "beams": W, "steps_timed": steps, "launch": "one CUDA graph per step",
+           "decode_kernel_ms": round(kern[3], 4), "decode_GBps_logical": round(dec_by / kern[3] / 1e6, 1),
+           "step_GBps_logical": round(by / ms / 1e6, 1),
+           "kernels_ms": {"beam_step": round(kern[0], 5), "copy_blocks_counted": round(kern[1], 5),
+                          "reshape_and_cache": round(kern[2], 5), "decode": round(kern[3], 5)},
+           "device_path_wall_ms_with_sync": round(1e3 * statistics.median(wall), 4),
+           "host_pool_path_wall_ms": round(1e3 * statistics.median(host), 4),
+           "note": "decode bytes are logical: beams of a prompt share their prefix blocks (read from L2)"}
+    del b
+    torch.cuda.empty_cache()
+    return res
+
+
 def measure_other(name: str, steps: int, warmup: int):
     spec, b = build_batch(name, 0)
     ms, kern, _ = time_steps(b, steps, warmup, 1)
@@ -502,6 +614,12 @@ def main():
     import paged_kv_cache_340_b200 as pa  # noqa: F401  (fails loudly without the CUDA library)
 
     from paged_kv_cache_340_b200.workloads import SPECS as _SPECS
+    if _SPECS[args.workload].branches and _SPECS[args.workload].num_prompts and args.workload.startswith("beam"):
+        if rank == 0:
+            print(json.dumps({"workload": args.workload, "beam": measure_beam(args.workload, args.steps,
+                                                                              args.warmup)}), flush=True)
+        pdist.finalize(world)
+        return
     if _SPECS[args.workload].q_len:
         if rank == 0:
             print(json.dumps({"workload": args.workload, "prefill": measure_prefill(args.workload, args.steps,
@@ -555,6 +673,7 @@ def main():
                                    ("gqa_bf16", "long_splitk_bf16", "parallel_sampling_fp16")}
         line["prefill_workloads"] = {n: measure_prefill(n, 20, 3) for n in
                                      ("prefill_llama7b_mha_bf16", "chunked_prefill_gqa_bf16")}
+        line["beam_search_fp16"] = measure_beam("beam_search_fp16", 200, 10)
     if rank == 0:
         print(json.dumps(line), flush=True)
     pdist.finalize(world)

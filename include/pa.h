@@ -306,6 +306,11 @@ int pa_pool_fork(pa_block_pool *pool, const int32_t *table, int num_tokens, int3
 /* Drops the sequence's reference to each of its blocks. */
 int pa_pool_release(pa_block_pool *pool, const int32_t *table, int num_tokens);
 
+/* Copies the pool's state out: ref_counts [num_blocks] and the free list
+ * front first (free_list has room for num_blocks; *num_free receives its
+ * length). With pa_dpool_load this hands a host pool over to the device. */
+int pa_pool_export(const pa_block_pool *pool, int32_t *ref_counts, int32_t *free_list, int *num_free);
+
 /*
  * Prefix cache over a host block pool ([P4] §3.2, Prefix Caching): a prompt
  * prefix (e.g. a system prompt shared by many requests) gets its blocks, and
@@ -369,6 +374,13 @@ size_t pa_dpool_state_bytes(int num_blocks);
 int pa_dpool_init(void *state, int num_blocks, int block_size, int policy, const int32_t *free_order,
                   cudaStream_t stream);
 
+/* Loads a pool state (e.g. from pa_pool_export): ref_counts [num_blocks]
+ * and free_list [num_free] (front first) are device int32 arrays. The free
+ * list must hold distinct ids of count 0, and every block of count 0 must be
+ * on it; otherwise the state is left unusable and PA_DEVERR_POOL is set. */
+int pa_dpool_load(void *state, int num_blocks, int block_size, int policy, const int32_t *ref_counts,
+                  const int32_t *free_list, int num_free, cudaStream_t stream);
+
 /*
  * pa_beam_step -- one beam-search step on the device ([P2] §3.4: beams share
  * blocks and copy one before writing into it; [P4] §3.3: the copy-on-write
@@ -392,7 +404,10 @@ int pa_dpool_init(void *state, int num_blocks, int block_size, int policy, const
  * table room for the new token, an uninitialised state) applies nothing:
  * the state is unchanged, every slot is -1, *num_cow = 0 and a PA_DEVERR_*
  * bit is set. Runs as one CTA; calls on one state must not overlap.
+ * Limits (else PA_ERR_SHAPE): 3 * num_old + num_new <= PA_BEAM_MAX_STAGED
+ * and (num_old + num_new) * max_blocks_per_seq < 2^30.
  */
+#define PA_BEAM_MAX_STAGED 24576
 int pa_beam_step(void *state, int num_blocks, int block_size, const int32_t *old_tables,
                  const int32_t *old_context_lens, int num_old, const int32_t *parents, int num_new,
                  int32_t *new_tables, int32_t *new_context_lens, int max_blocks_per_seq,

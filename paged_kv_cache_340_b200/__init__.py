@@ -43,7 +43,7 @@ EXPORTED = (
     "pa_pool_fork", "pa_pool_release", "pa_decode_splitk_static", "pa_prefill",
     "pa_prefix_cache_create", "pa_prefix_cache_destroy", "pa_prefix_num_entries", "pa_prefix_get_or_create",
     "pa_prefix_release", "pa_prefix_ref_count", "pa_copy_blocks_counted", "pa_dpool_state_bytes", "pa_dpool_init",
-    "pa_beam_step",
+    "pa_beam_step", "pa_pool_export", "pa_dpool_load",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -99,6 +99,8 @@ def _load() -> ctypes.CDLL:
         "pa_dpool_state_bytes": (sz, [i32]),
         "pa_dpool_init": (i32, [vp, i32, i32, i32, vp, vp]),
         "pa_beam_step": (i32, [vp, i32, i32, vp, vp, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp]),
+        "pa_pool_export": (i32, [vp, i32p, i32p, ctypes.POINTER(ctypes.c_int)]),
+        "pa_dpool_load": (i32, [vp, i32, i32, i32, vp, vp, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -258,18 +260,28 @@ class DevicePool:
     ring, ``header`` of [num_blocks, block_size, policy, head, count, marker]."""
 
     def __init__(self, num_blocks: int, block_size: int, policy: int = PA_POOL_LIFO, free_order=None,
-                 device="cuda", stream=None):
+                 device="cuda", stream=None, host_pool: "Optional[BlockPool]" = None):
+        """A fresh pool (free list free_order, else 0..num_blocks-1), or, with
+        host_pool, a copy of that host pool's counts and free list."""
         self.num_blocks, self.block_size, self.policy = num_blocks, block_size, policy
         nbytes = int(_lib.pa_dpool_state_bytes(num_blocks))
         if nbytes == 0:
             raise PagedAttentionError("pa_dpool_state_bytes", -3)
         self.state = torch.empty(nbytes // 4, dtype=torch.int32, device=device)
-        fo = None
-        if free_order is not None:
-            fo = torch.as_tensor(np.asarray(free_order, dtype=np.int32)).to(device)
-        _check(_lib.pa_dpool_init(_ptr(self.state), num_blocks, block_size, policy, _ptr(fo), _stream(stream)),
-               "pa_dpool_init")
-        self._keep = fo
+        if host_pool is not None:
+            assert host_pool.num_blocks == num_blocks and host_pool.block_size == block_size
+            ref, fl = host_pool.export()
+            self._keep = (torch.from_numpy(ref).to(device), torch.from_numpy(fl).to(device))
+            _check(_lib.pa_dpool_load(_ptr(self.state), num_blocks, block_size, policy, _ptr(self._keep[0]),
+                                      _ptr(self._keep[1]) if fl.shape[0] else None, fl.shape[0], _stream(stream)),
+                   "pa_dpool_load")
+        else:
+            fo = None
+            if free_order is not None:
+                fo = torch.as_tensor(np.asarray(free_order, dtype=np.int32)).to(device)
+            _check(_lib.pa_dpool_init(_ptr(self.state), num_blocks, block_size, policy, _ptr(fo), _stream(stream)),
+                   "pa_dpool_init")
+            self._keep = fo
         h = PA_DPOOL_HEADER_WORDS
         self.header = self.state[:6]
         self.ref = self.state[h:h + num_blocks]
@@ -384,6 +396,14 @@ class BlockPool:
 
     def release(self, table: np.ndarray, num_tokens: int) -> None:
         _check(_lib.pa_pool_release(self._h, _i32p(table), int(num_tokens)), "pa_pool_release")
+
+    def export(self) -> Tuple[np.ndarray, np.ndarray]:
+        """(reference counts [num_blocks], free list front first)."""
+        ref = np.empty(self.num_blocks, np.int32)
+        fl = np.empty(max(1, self.num_blocks), np.int32)
+        n = ctypes.c_int(0)
+        _check(_lib.pa_pool_export(self._h, _i32p(ref), _i32p(fl), ctypes.byref(n)), "pa_pool_export")
+        return ref, fl[: n.value].copy()
 
 
 class PrefixCache:

@@ -15,8 +15,9 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (PA_POOL_FIFO, BlockPool, pa_choose_partition, pa_copy_blocks, pa_decode, pa_decode_splitk,
-               pa_prefill, pa_reshape_and_cache, pa_splitk_reduce, pa_splitk_workspace_bytes)
+from . import (PA_POOL_FIFO, BlockPool, DevicePool, pa_beam_step, pa_choose_partition, pa_copy_blocks,
+               pa_copy_blocks_counted, pa_decode, pa_decode_splitk, pa_prefill, pa_reshape_and_cache,
+               pa_splitk_reduce, pa_splitk_workspace_bytes)
 from .workloads import Spec
 
 
@@ -357,3 +358,119 @@ def prefill_flops(spec: Spec, ctx: np.ndarray) -> int:
         keys = ql * (2 * first + ql - 1) // 2       # sum over the q_len tokens
         total += 4 * spec.head_dim * keys * spec.num_heads
     return total
+
+
+@dataclass
+class BeamBatch:
+    spec: Spec
+    num_blocks: int
+    pool: DevicePool
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    tables: list                # two device int32 [W, MB] buffers: step i reads [i % 2], writes [(i + 1) % 2]
+    context_lens: list          # two device int32 [W]
+    parents: torch.Tensor       # device int32 [steps, W]
+    query: torch.Tensor         # device [steps, W, Hq, D]
+    new_key: torch.Tensor       # device [steps, W, Hkv, D]
+    new_value: torch.Tensor
+    slot_mapping: torch.Tensor  # device int32 [W]
+    cow_pairs: torch.Tensor     # device int64 [W, 2]
+    num_cow: torch.Tensor       # device int32 [1]
+    out: torch.Tensor           # device [W, Hq, D]
+    host_prompt_lens: np.ndarray
+    host_pool: BlockPool        # the host pool the prompts were written with (state before step 0)
+    host_tables: np.ndarray     # [W, MB] before step 0
+    steps_done: int = 0
+
+
+def build_beam_batch(spec: Spec, inputs: dict, device="cuda", pool_policy: int = PA_POOL_FIFO) -> BeamBatch:
+    """Beam search start: each prompt's tokens go into blocks of the host pool
+    (a prefill), the prompt is forked into `branches` beams sharing them, and
+    the pool's state is loaded into a device pool for the device beam steps."""
+    bs, B, P = spec.block_size, spec.branches, spec.num_prompts
+    W = P * B
+    lens = inputs["prompt_lens"].numpy().astype(np.int32)
+    nb = int(inputs["num_blocks"])
+    mb = _blocks(int(lens.max()) + spec.max_divergent, bs) + 1
+    pool = BlockPool(nb, bs, pool_policy, free_order=inputs["free_order"].numpy())
+    tables = np.full((W, mb), -1, np.int32)
+    for p in range(P):
+        pool.append(tables[p * B], 0, int(lens[p]), want_slots=False)
+        for b in range(1, B):
+            pool.fork(tables[p * B], int(lens[p]), tables[p * B + b])
+    dev = torch.device(device)
+    ctx = np.repeat(lens, B).astype(np.int32)
+    dpool = DevicePool(nb, bs, pool_policy, device=dev, host_pool=pool)
+    tb = [torch.from_numpy(tables).to(dev), torch.empty((W, mb), dtype=torch.int32, device=dev)]
+    cl = [torch.from_numpy(ctx).to(dev), torch.empty(W, dtype=torch.int32, device=dev)]
+    return BeamBatch(
+        spec=spec, num_blocks=nb, pool=dpool, k_cache=inputs["k_pool"].to(dev), v_cache=inputs["v_pool"].to(dev),
+        tables=tb, context_lens=cl, parents=inputs["parents"].to(dev), query=inputs["query"].to(dev),
+        new_key=inputs["new_key"].to(dev), new_value=inputs["new_value"].to(dev),
+        slot_mapping=torch.empty(W, dtype=torch.int32, device=dev),
+        cow_pairs=torch.empty((W, 2), dtype=torch.int64, device=dev),
+        num_cow=torch.zeros(1, dtype=torch.int32, device=dev),
+        out=torch.empty((W, spec.num_heads, spec.head_dim), dtype=spec.torch_out_dtype, device=dev),
+        host_prompt_lens=lens, host_pool=pool, host_tables=tables)
+
+
+def run_beam_step(b: BeamBatch, stream=None, events=None) -> None:
+    """One beam-search decode step, all on the device: beam step (fork,
+    release, copy-on-write decisions), counted block copy, slot write of the
+    new tokens, decode over the new tables. events (optional, 5 CUDA events)
+    are recorded between the launches."""
+    i = b.steps_done
+    k = i % b.parents.shape[0]
+    src, dst = i % 2, (i + 1) % 2
+
+    def mark(j):
+        if events is not None:
+            events[j].record(stream if stream is not None else torch.cuda.current_stream())
+
+    mark(0)
+    pa_beam_step(b.pool, b.tables[src], b.context_lens[src], b.parents[k], b.tables[dst], b.context_lens[dst],
+                 b.slot_mapping, b.cow_pairs, b.num_cow, stream=stream)
+    mark(1)
+    pa_copy_blocks_counted(b.k_cache, b.v_cache, b.cow_pairs, b.num_cow, stream=stream)
+    mark(2)
+    pa_reshape_and_cache(b.new_key[k], b.new_value[k], b.k_cache, b.v_cache, b.slot_mapping, stream=stream)
+    mark(3)
+    pa_decode(b.out, b.query[k], b.k_cache, b.v_cache, b.tables[dst], b.context_lens[dst], b.spec.scale,
+              stream=stream)
+    mark(4)
+    b.steps_done = i + 1
+
+
+def beam_decode_bytes(b: BeamBatch, step: int) -> int:
+    """Algorithmic bytes of the decode of beam step `step` (0-based): every
+    beam of prompt p holds prompt_lens[p] + step + 1 tokens after it (beams of
+    one prompt grow together)."""
+    s = b.spec
+    elt = s.torch_kv_dtype.itemsize
+    ctx = (b.host_prompt_lens.astype(np.int64) + step + 1).repeat(s.branches)
+    nblk = (ctx + s.block_size - 1) // s.block_size
+    W = ctx.shape[0]
+    return int(ctx.sum() * 2 * s.num_kv_heads * s.head_dim * elt + W * s.num_heads * s.head_dim *
+               (elt + s.torch_out_dtype.itemsize) + 4 * nblk.sum() + 4 * W)
+
+
+def host_beam_step(pool: BlockPool, tables: np.ndarray, ctx: np.ndarray, parents: np.ndarray):
+    """The same step on the host pool (the path without the device pool):
+    fork every chosen parent, release the old beams, append one token to each
+    new beam. Returns (new tables, new context lengths, slots, copy pairs)."""
+    W_new, mb = parents.shape[0], tables.shape[1]
+    new_t = np.full((W_new, mb), -1, np.int32)
+    for i, p in enumerate(parents):
+        pool.fork(tables[p], int(ctx[p]), new_t[i])
+    for j in range(tables.shape[0]):
+        pool.release(tables[j], int(ctx[j]))
+    new_c = np.empty(W_new, np.int32)
+    slots = np.empty(W_new, np.int32)
+    pairs = []
+    for i, p in enumerate(parents):
+        nt, sl, cow = pool.append(new_t[i], int(ctx[p]), 1)
+        new_c[i] = nt
+        slots[i] = sl[0]
+        pairs.append(cow)
+    cow = np.concatenate(pairs).astype(np.int64) if pairs else np.empty((0, 2), np.int64)
+    return new_t, new_c, slots, cow

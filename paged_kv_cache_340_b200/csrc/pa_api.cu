@@ -373,14 +373,28 @@ int pa_dpool_init(void *state, int num_blocks, int block_size, int policy, const
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+int pa_dpool_load(void *state, int num_blocks, int block_size, int policy, const int32_t *ref_counts,
+                  const int32_t *free_list, int num_free, cudaStream_t stream) {
+    if (num_blocks <= 0 || block_size <= 0 || num_blocks > INT_MAX / PA_DPOOL_ARRAYS) return PA_ERR_SHAPE;
+    if (num_free < 0 || num_free > num_blocks) return PA_ERR_SHAPE;
+    if (policy != PA_POOL_LIFO && policy != PA_POOL_FIFO) return PA_ERR_SHAPE;
+    if (!state || !ref_counts || (num_free > 0 && !free_list)) return PA_ERR_NULL;
+    if (!aligned(state, 16) || !aligned(ref_counts, 4) || !aligned(free_list, 4)) return PA_ERR_ALIGN;
+    unsigned int *err = nullptr;
+    if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    cudaError_t e = launch_dpool_load(static_cast<int32_t *>(state), num_blocks, block_size, policy, ref_counts,
+                                      free_list, num_free, err, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 int pa_beam_step(void *state, int num_blocks, int block_size, const int32_t *old_tables,
                  const int32_t *old_context_lens, int num_old, const int32_t *parents, int num_new,
                  int32_t *new_tables, int32_t *new_context_lens, int max_blocks_per_seq,
                  int32_t *slot_mapping, int64_t *cow_pairs, int32_t *num_cow, cudaStream_t stream) {
     if (num_blocks <= 0 || block_size <= 0 || num_old < 0 || num_new < 0 || max_blocks_per_seq <= 0)
         return PA_ERR_SHAPE;
-    if ((long long)num_old * max_blocks_per_seq >= INT_MAX || (long long)num_new * max_blocks_per_seq >= INT_MAX ||
-        (long long)num_blocks * block_size >= INT_MAX)
+    if (((long long)num_old + num_new) * max_blocks_per_seq >= (1LL << 30) ||
+        (long long)num_blocks * block_size >= INT_MAX || 3LL * num_old + num_new > PA_BEAM_MAX_STAGED)
         return PA_ERR_SHAPE;
     if (!state || !num_cow || (num_old > 0 && (!old_tables || !old_context_lens)) ||
         (num_new > 0 && (!parents || !new_tables || !new_context_lens || !slot_mapping || !cow_pairs)))

@@ -37,7 +37,10 @@ namespace pa {
 namespace beam {
 
 constexpr int kThreads = 1024;
-constexpr int kItems = 8;          // table entries per thread per pass
+constexpr int kItems = 16;         // table entries per thread per pass
+constexpr int kScanItems = 8;      // the same in the scanned pass (four values per entry)
+// per-beam values staged in shared memory: 3 words per old beam, 1 per new beam
+constexpr int kMaxStageBytes = PA_BEAM_MAX_STAGED * 4;
 constexpr int32_t kMagic = 0x50414250;
 
 struct Pool {
@@ -132,6 +135,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// Loads counts and a free list, then checks them: free-list ids in range,
+// distinct and of count 0; counts not negative; as many blocks of count 0 as
+// free-list entries.
+__global__ void __launch_bounds__(kThreads, 1)
+    dpool_load_kernel(int32_t *state, int nb, int bs, int policy, const int32_t *ref_counts,
+                      const int32_t *free_list, int num_free, unsigned int *err) {
+    __shared__ int s_bad, s_zero;
+    const Pool p = views(state, nb);
+    if (threadIdx.x == 0) {
+        s_bad = 0;
+        s_zero = 0;
+    }
+    for (int i = threadIdx.x; i < nb; i += kThreads) {
+        const int r = ref_counts[i];
+        p.ref[i] = r;
+        p.ring[i] = i < num_free ? free_list[i] : -1;
+        p.delta[i] = 0;
+        p.last_old[i] = -1;
+        p.writers[i] = 0;
+        p.last_writer[i] = -1;
+    }
+    __syncthreads();
+    int zeros = 0;
+    for (int i = threadIdx.x; i < nb; i += kThreads) {
+        if (p.ref[i] < 0) s_bad = 1;
+        zeros += p.ref[i] == 0;
+        if (i < num_free) {
+            const int b = p.ring[i];
+            if (b < 0 || b >= nb || p.ref[b] != 0)
+                s_bad = 1;
+            else
+                atomicAdd(&p.delta[b], 1);
+        }
+    }
+    atomicAdd(&s_zero, zeros);
+    __syncthreads();
+    for (int i = threadIdx.x; i < nb; i += kThreads) {
+        if (p.delta[i] > 1) s_bad = 1;
+        p.delta[i] = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (s_zero != num_free) s_bad = 1;
+        p.hdr[0] = nb;
+        p.hdr[1] = bs;
+        p.hdr[2] = policy;
+        p.hdr[3] = 0;
+        p.hdr[4] = num_free;
+        p.hdr[5] = s_bad ? 0 : kMagic;
+        p.hdr[6] = 0;
+        p.hdr[7] = 0;
+        if (s_bad) record_error(err, PA_DEVERR_POOL);
+    }
+}
+
 struct StepParams {
     int32_t *state;
     const int32_t *old_tables;
@@ -152,14 +210,25 @@ struct StepParams {
 
 __device__ __forceinline__ int nblk(int ctx, int bs) { return (ctx + bs - 1) / bs; }
 
+// The kernel is latency-bound (one CTA, dependent loads), so every pass over
+// table entries first loads kItems entries per thread into registers, then
+// acts on them: one or two memory round trips per pass instead of one per
+// entry. Table, context and parent arrays are read-only here (__ldg).
 __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams q) {
+    extern __shared__ int dyn[];
     __shared__ int warp_sums[32];
     __shared__ int s_bad;
     const int tid = threadIdx.x;
     const int nb = q.num_blocks, bs = q.block_size, MB = q.max_blocks;
     const Pool p = views(q.state, nb);
-    const long long old_entries = (long long)q.num_old * MB;
-    const long long new_entries = (long long)q.num_new * MB;
+    const int n_old = q.num_old, n_new = q.num_new;
+    const int old_entries = n_old * MB;  // < 2^31 (host check)
+    const int new_entries = n_new * MB;
+    int *s_ctx = dyn;                    // [n_old] context length of old beam j
+    int *s_nb = dyn + n_old;             // [n_old] its block count
+    int *s_nch = dyn + 2 * n_old;        // [n_old] its number of children
+    int *s_par = dyn + 3 * n_old;        // [n_new] parent of new beam i
+    const int32_t *__restrict__ otab = q.old_tables;
 
     if (tid == 0) s_bad = 0;
     __syncthreads();
@@ -167,30 +236,51 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
     if (tid == 0 && (p.hdr[5] != kMagic || p.hdr[0] != nb || p.hdr[1] != bs || count < 0 || count > nb ||
                      head < 0 || head >= nb))
         atomicOr(&s_bad, PA_DEVERR_POOL);
-    // ---- phase 0: inputs (nothing is changed yet)
-    for (int j = tid; j < q.num_old; j += kThreads) {
-        const int c = q.old_ctx[j];
+    // ---- phase 0: stage and check the inputs (nothing is changed yet)
+    for (int j = tid; j < n_old; j += kThreads) {
+        const int c = __ldg(q.old_ctx + j);
+        s_ctx[j] = c;
+        s_nb[j] = c < 0 ? 0 : nblk(c, bs);
+        s_nch[j] = 0;
         if (c < 0 || nblk(c, bs) > MB) atomicOr(&s_bad, PA_DEVERR_CONTEXT);
     }
-    for (int i = tid; i < q.num_new; i += kThreads) {
-        const int par = q.parents[i];
-        if (par < 0 || par >= q.num_old) atomicOr(&s_bad, PA_DEVERR_CONTEXT);
+    __syncthreads();
+    for (int i = tid; i < n_new; i += kThreads) {
+        const int par = __ldg(q.parents + i);
+        s_par[i] = par;
+        if (par < 0 || par >= n_old)
+            atomicOr(&s_bad, PA_DEVERR_CONTEXT);
+        else
+            atomicAdd(&s_nch[par], 1);
     }
     __syncthreads();
     if (!s_bad) {
-        for (long long e = tid; e < old_entries; e += kThreads) {
-            const int j = (int)(e / MB), pos = (int)(e % MB);
-            if (pos < nblk(q.old_ctx[j], bs)) {
-                const int b = q.old_tables[e];
-                if (b < 0 || b >= nb || p.ref[b] <= 0) atomicOr(&s_bad, PA_DEVERR_BLOCK_ID);
+        for (int base = 0; base < old_entries; base += kThreads * kItems) {
+            int blk[kItems], in_use = 0;
+#pragma unroll
+            for (int k = 0; k < kItems; ++k) {
+                const int e = base + k * kThreads + tid;
+                blk[k] = 0;
+                if (e < old_entries) {
+                    const int j = e / MB;
+                    if (e - j * MB < s_nb[j]) {
+                        blk[k] = __ldg(otab + e);
+                        in_use |= 1 << k;
+                    }
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kItems; ++k) {
+                const int b = blk[k];
+                if ((in_use >> k & 1) && (b < 0 || b >= nb || p.ref[b] <= 0)) atomicOr(&s_bad, PA_DEVERR_BLOCK_ID);
             }
         }
-        for (int i = tid; i < q.num_new; i += kThreads)
-            if (q.old_ctx[q.parents[i]] / bs >= MB) atomicOr(&s_bad, PA_DEVERR_POOL);  // no room for the token
+        for (int i = tid; i < n_new; i += kThreads)
+            if (s_ctx[s_par[i]] / bs >= MB) atomicOr(&s_bad, PA_DEVERR_POOL);  // no room for the token
     }
     __syncthreads();
     if (s_bad) {
-        for (int i = tid; i < q.num_new; i += kThreads) q.slots[i] = -1;
+        for (int i = tid; i < n_new; i += kThreads) q.slots[i] = -1;
         if (tid == 0) {
             *q.num_cow = 0;
             record_error(q.err, (unsigned)s_bad);
@@ -198,74 +288,119 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
         return;
     }
 
-    // ---- phase 1: net count change, last releasing entry, writers
-    for (long long e = tid; e < new_entries; e += kThreads) {
-        const int i = (int)(e / MB), pos = (int)(e % MB);
-        const int par = q.parents[i];
-        if (pos < nblk(q.old_ctx[par], bs)) atomicAdd(&p.delta[q.old_tables[(long long)par * MB + pos]], 1);
-    }
-    for (long long e = tid; e < old_entries; e += kThreads) {
-        const int j = (int)(e / MB), pos = (int)(e % MB);
-        if (pos < nblk(q.old_ctx[j], bs)) {
-            const int b = q.old_tables[e];
-            atomicSub(&p.delta[b], 1);
-            atomicMax(&p.last_old[b], (int)e);
+    // ---- phase 1: net count change. A child's table is its parent's, so a
+    // block of old beam j gains (children of j) - 1 references: only beams
+    // with other than one child touch the counts. Then the writers.
+    for (int base = 0; base < old_entries; base += kThreads * kItems) {
+        int blk[kItems];
+#pragma unroll
+        for (int k = 0; k < kItems; ++k) {
+            const int e = base + k * kThreads + tid;
+            blk[k] = -1;
+            if (e < old_entries) {
+                const int j = e / MB;
+                if (e - j * MB < s_nb[j] && s_nch[j] != 1) blk[k] = __ldg(otab + e);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kItems; ++k) {
+            if (blk[k] >= 0) {
+                const int e = base + k * kThreads + tid;
+                atomicAdd(&p.delta[blk[k]], s_nch[e / MB] - 1);
+            }
         }
     }
-    for (int i = tid; i < q.num_new; i += kThreads) {
-        const int par = q.parents[i];
-        const int t = q.old_ctx[par];
+    for (int i = tid; i < n_new; i += kThreads) {
+        const int par = s_par[i];
+        const int t = s_ctx[par];
         if (t % bs) {
-            const int o = q.old_tables[(long long)par * MB + t / bs];
+            const int o = __ldg(otab + par * MB + t / bs);
             atomicAdd(&p.writers[o], 1);
             atomicMax(&p.last_writer[o], i);
+        }
+    }
+    __syncthreads();
+    // a block is freed only if every old beam holding it has no child; mark
+    // the last such entry (in release order) of each block reaching zero
+    for (int base = 0; base < old_entries; base += kThreads * kItems) {
+        int blk[kItems], r0[kItems];
+#pragma unroll
+        for (int k = 0; k < kItems; ++k) {
+            const int e = base + k * kThreads + tid;
+            blk[k] = -1;
+            if (e < old_entries) {
+                const int j = e / MB;
+                if (e - j * MB < s_nb[j] && s_nch[j] == 0) blk[k] = __ldg(otab + e);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kItems; ++k)
+            if (blk[k] >= 0) r0[k] = p.ref[blk[k]] + p.delta[blk[k]];
+#pragma unroll
+        for (int k = 0; k < kItems; ++k) {
+            if (blk[k] >= 0) {
+                if (r0[k] < 0) atomicOr(&s_bad, PA_DEVERR_POOL);  // a table holds a block more often than counted
+                if (r0[k] == 0) atomicMax(&p.last_old[blk[k]], base + k * kThreads + tid);
+            }
         }
     }
     __syncthreads();
 
     // ---- phase 2: freed blocks, pushed to the back of the free list in
     // order of their last release (written past the list's end: harmless
-    // until the count is updated)
+    // until the count is updated). Items are contiguous per thread so the
+    // scan runs in entry order.
     int freed = 0;
-    for (long long base = 0; base < old_entries; base += (long long)kThreads * kItems) {
-        int flag[kItems], blk[kItems], mine = 0;
+    for (int base = 0; base < old_entries; base += kThreads * kScanItems) {
+        int blk[kScanItems], r0[kScanItems], d0[kScanItems], l0[kScanItems];
 #pragma unroll
-        for (int k = 0; k < kItems; ++k) {
-            const long long e = base + (long long)tid * kItems + k;
-            flag[k] = 0;
+        for (int k = 0; k < kScanItems; ++k) {
+            const int e = base + tid * kScanItems + k;
             blk[k] = -1;
             if (e < old_entries) {
-                const int j = (int)(e / MB), pos = (int)(e % MB);
-                if (pos < nblk(q.old_ctx[j], bs)) {
-                    const int b = q.old_tables[e];
-                    const int r = p.ref[b] + p.delta[b];
-                    if (r < 0) atomicOr(&s_bad, PA_DEVERR_POOL);  // a table holds a block more often than counted
-                    flag[k] = (r == 0 && p.last_old[b] == (int)e);
-                    blk[k] = b;
+                const int j = e / MB;
+                if (e - j * MB < s_nb[j] && s_nch[j] == 0) blk[k] = __ldg(otab + e);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kScanItems; ++k) {
+            if (blk[k] >= 0) {
+                r0[k] = p.ref[blk[k]];
+                d0[k] = p.delta[blk[k]];
+                l0[k] = p.last_old[blk[k]];
+            }
+        }
+        int flag = 0, mine = 0;
+#pragma unroll
+        for (int k = 0; k < kScanItems; ++k) {
+            if (blk[k] >= 0) {
+                const int r = r0[k] + d0[k];
+                if (r == 0 && l0[k] == base + tid * kScanItems + k) {
+                    flag |= 1 << k;
+                    ++mine;
                 }
             }
-            mine += flag[k];
         }
         int tot;
         int r = cta_exclusive_scan(mine, warp_sums, &tot);
 #pragma unroll
-        for (int k = 0; k < kItems; ++k)
-            if (flag[k]) p.ring[(head + count + freed + r++) % nb] = blk[k];
+        for (int k = 0; k < kScanItems; ++k)
+            if (flag >> k & 1) p.ring[(head + count + freed + r++) % nb] = blk[k];
         freed += tot;
     }
 
     // ---- phase 3: blocks the new tokens take, and the copies
     int takes = 0, copies = 0;
-    for (int base = 0; base < q.num_new; base += kThreads) {
+    for (int base = 0; base < n_new; base += kThreads) {
         const int i = base + tid;
         int need = 0, copy = 0;
-        if (i < q.num_new) {
-            const int par = q.parents[i];
-            const int t = q.old_ctx[par];
+        if (i < n_new) {
+            const int par = s_par[i];
+            const int t = s_ctx[par];
             if (t % bs == 0) {
                 need = 1;
             } else {
-                const int o = q.old_tables[(long long)par * MB + t / bs];
+                const int o = __ldg(otab + par * MB + t / bs);
                 const int others = p.ref[o] + p.delta[o] - p.writers[o];
                 copy = (others > 0 || p.last_writer[o] != i);
                 need = copy;
@@ -282,48 +417,62 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
 
     // ---- phase 4: apply the net counts (each block once: whoever swaps its
     // delta out), reset the release marks
-    for (long long e = tid; e < new_entries + old_entries; e += kThreads) {
-        int b = -1;
-        if (e < new_entries) {
-            const int i = (int)(e / MB), pos = (int)(e % MB);
-            const int par = q.parents[i];
-            if (pos < nblk(q.old_ctx[par], bs)) b = q.old_tables[(long long)par * MB + pos];
-        } else {
-            const long long eo = e - new_entries;
-            const int j = (int)(eo / MB), pos = (int)(eo % MB);
-            if (pos < nblk(q.old_ctx[j], bs)) {
-                b = q.old_tables[eo];
-                p.last_old[b] = -1;
+    for (int base = 0; base < old_entries; base += kThreads * kItems) {
+        int blk[kItems];
+#pragma unroll
+        for (int k = 0; k < kItems; ++k) {
+            const int e = base + k * kThreads + tid;
+            blk[k] = -1;
+            if (e < old_entries) {
+                const int j = e / MB;
+                if (e - j * MB < s_nb[j] && s_nch[j] != 1) blk[k] = __ldg(otab + e);
             }
         }
-        if (b >= 0) {
-            const int d = atomicExch(&p.delta[b], 0);
-            if (ok && d) p.ref[b] += d;
+#pragma unroll
+        for (int k = 0; k < kItems; ++k) {
+            if (blk[k] >= 0) {
+                const int b = blk[k];
+                if (s_nch[(base + k * kThreads + tid) / MB] == 0) p.last_old[b] = -1;
+                const int d = atomicExch(&p.delta[b], 0);
+                if (ok && d) p.ref[b] += d;
+            }
         }
     }
     __syncthreads();
 
     if (ok) {
         // ---- phase 5: the new tables (parent rows, -1 past the blocks in use)
-        for (long long e = tid; e < new_entries; e += kThreads) {
-            const int i = (int)(e / MB), pos = (int)(e % MB);
-            const int par = q.parents[i];
-            const int t = q.old_ctx[par];
-            q.new_tables[e] = pos < nblk(t, bs) ? q.old_tables[(long long)par * MB + pos] : -1;
+        for (int base = 0; base < new_entries; base += kThreads * kItems) {
+            int v[kItems];
+#pragma unroll
+            for (int k = 0; k < kItems; ++k) {
+                const int e = base + k * kThreads + tid;
+                v[k] = -1;
+                if (e < new_entries) {
+                    const int i = e / MB, pos = e - i * MB;
+                    const int par = s_par[i];
+                    if (pos < s_nb[par]) v[k] = __ldg(otab + par * MB + pos);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kItems; ++k) {
+                const int e = base + k * kThreads + tid;
+                if (e < new_entries) q.new_tables[e] = v[k];
+            }
         }
         __syncthreads();
         // ---- phase 6: takes, copies, slots
         int tk = 0, cp = 0;
-        for (int base = 0; base < q.num_new; base += kThreads) {
+        for (int base = 0; base < n_new; base += kThreads) {
             const int i = base + tid;
-            int need = 0, copy = 0, o = -1, par = 0, t = 0;
-            if (i < q.num_new) {
-                par = q.parents[i];
-                t = q.old_ctx[par];
+            int need = 0, copy = 0, o = -1, t = 0;
+            if (i < n_new) {
+                const int par = s_par[i];
+                t = s_ctx[par];
                 if (t % bs == 0) {
                     need = 1;
                 } else {
-                    o = q.old_tables[(long long)par * MB + t / bs];
+                    o = __ldg(otab + par * MB + t / bs);
                     copy = (p.ref[o] - p.writers[o] > 0 || p.last_writer[o] != i);
                     need = copy;
                 }
@@ -333,12 +482,12 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
             const int c = cp + cta_exclusive_scan(copy, warp_sums, &tc);
             tk += tt;
             cp += tc;
-            if (i < q.num_new) {
+            if (i < n_new) {
                 int b = o;
                 if (need) {
                     b = policy == PA_POOL_FIFO ? p.ring[(head + k) % nb] : p.ring[(head + count + freed - 1 - k) % nb];
                     p.ref[b] = 1;
-                    q.new_tables[(long long)i * MB + t / bs] = b;
+                    q.new_tables[i * MB + t / bs] = b;
                 }
                 if (copy) {
                     q.cow_pairs[2 * c] = o;
@@ -350,22 +499,22 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
         }
         __syncthreads();
         // a copying writer gives up its reference to the old block
-        for (int i = tid; i < q.num_new; i += kThreads) {
-            const int par = q.parents[i];
-            const int t = q.old_ctx[par];
+        for (int i = tid; i < n_new; i += kThreads) {
+            const int par = s_par[i];
+            const int t = s_ctx[par];
             if (t % bs) {
-                const int o = q.old_tables[(long long)par * MB + t / bs];
-                if (q.new_tables[(long long)i * MB + t / bs] != o) atomicSub(&p.ref[o], 1);
+                const int o = __ldg(otab + par * MB + t / bs);
+                if (q.new_tables[i * MB + t / bs] != o) atomicSub(&p.ref[o], 1);
             }
         }
     }
     __syncthreads();
     // ---- reset the writer marks; header and outputs
-    for (int i = tid; i < q.num_new; i += kThreads) {
-        const int par = q.parents[i];
-        const int t = q.old_ctx[par];
+    for (int i = tid; i < n_new; i += kThreads) {
+        const int par = s_par[i];
+        const int t = s_ctx[par];
         if (t % bs) {
-            const int o = q.old_tables[(long long)par * MB + t / bs];
+            const int o = __ldg(otab + par * MB + t / bs);
             p.writers[o] = 0;
             p.last_writer[o] = -1;
         }
@@ -396,6 +545,13 @@ cudaError_t launch_dpool_init(int32_t *state, int num_blocks, int block_size, in
     return cudaGetLastError();
 }
 
+cudaError_t launch_dpool_load(int32_t *state, int num_blocks, int block_size, int policy, const int32_t *ref_counts,
+                              const int32_t *free_list, int num_free, unsigned int *err, cudaStream_t stream) {
+    beam::dpool_load_kernel<<<1, beam::kThreads, 0, stream>>>(state, num_blocks, block_size, policy, ref_counts,
+                                                              free_list, num_free, err);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const int32_t *old_ctx, int num_old,
                              const int32_t *parents, int num_new, int32_t *new_tables, int32_t *new_ctx,
                              int max_blocks, int32_t *slots, int64_t *cow_pairs, int32_t *num_cow,
@@ -416,7 +572,12 @@ cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const in
     q.num_blocks = num_blocks;
     q.block_size = block_size;
     q.err = err;
-    beam::beam_step_kernel<<<1, beam::kThreads, 0, stream>>>(q);
+    const int smem = (3 * num_old + num_new) * (int)sizeof(int);
+    static unsigned int attr_done = 0;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(beam::beam_step_kernel), beam::kMaxStageBytes,
+                                     &attr_done);
+    if (e != cudaSuccess) return e;
+    beam::beam_step_kernel<<<1, beam::kThreads, smem, stream>>>(q);
     return cudaGetLastError();
 }
 

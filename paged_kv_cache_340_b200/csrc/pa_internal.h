@@ -53,6 +53,9 @@ cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *pair
 cudaError_t launch_dpool_init(int32_t *state, int num_blocks, int block_size, int policy,
                               const int32_t *free_order, unsigned int *err, cudaStream_t stream);
 
+cudaError_t launch_dpool_load(int32_t *state, int num_blocks, int block_size, int policy, const int32_t *ref_counts,
+                              const int32_t *free_list, int num_free, unsigned int *err, cudaStream_t stream);
+
 cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const int32_t *old_ctx, int num_old,
                              const int32_t *parents, int num_new, int32_t *new_tables, int32_t *new_ctx,
                              int max_blocks, int32_t *slots, int64_t *cow_pairs, int32_t *num_cow,

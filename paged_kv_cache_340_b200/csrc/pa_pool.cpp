@@ -161,6 +161,14 @@ int pa_pool_fork(pa_block_pool *pool, const int32_t *table, int num_tokens, int3
     return PA_OK;
 }
 
+int pa_pool_export(const pa_block_pool *pool, int32_t *ref_counts, int32_t *free_list, int *num_free) {
+    if (!pool || !ref_counts || !free_list || !num_free) return PA_ERR_NULL;
+    std::copy(pool->ref.begin(), pool->ref.end(), ref_counts);
+    std::copy(pool->free_list.begin(), pool->free_list.end(), free_list);
+    *num_free = (int)pool->free_list.size();
+    return PA_OK;
+}
+
 int pa_pool_release(pa_block_pool *pool, const int32_t *table, int num_tokens) {
     if (!pool || !table) return PA_ERR_NULL;
     if (num_tokens < 0) return PA_ERR_SHAPE;

@@ -26,6 +26,10 @@ Workloads (shapes follow LLaMA-style decode layers):
                        head_dim 128, block 16; q/k/v ~ N(0,1); fp32 out
   chunked_prefill_gqa_bf16   16 sequences of 4096 tokens whose last 512 are new,
                        32 query / 8 kv heads, head_dim 128, block 16; fp32 out
+  beam_search_fp16     32 prompts of U{256..1024} tokens x beam width 4 (128 beams),
+                       32 heads, head_dim 128, block 16; every step each beam picks a
+                       parent among its prompt's 4 beams (uniform) and writes one token;
+                       q/k/v ~ N(0,1); fp16 out
 """
 from __future__ import annotations
 
@@ -94,6 +98,9 @@ SPECS: Dict[str, Spec] = {
                                      ("fixed", (2048,) * 8), 1.0, q_len=2048),
     "chunked_prefill_gqa_bf16": Spec("chunked_prefill_gqa_bf16", 16, 32, 8, 128, 16, "bf16", "f32", 3406,
                                      ("fixed", (4096,) * 16), 1.0, q_len=512),
+    # beam search: the beam step (fork, release, copy-on-write) on the device, then decode
+    "beam_search_fp16": Spec("beam_search_fp16", 128, 32, 32, 128, 16, "f16", "f16", 3407,
+                             ("uniform", 256, 1024), None, num_prompts=32, branches=4, max_divergent=512),
 }
 
 
@@ -224,3 +231,35 @@ def make_prefill_inputs(spec: Spec) -> dict:
     query = _normal(gen, (T, spec.num_heads, spec.head_dim), spec.q_scale, dt)
     return dict(context_lens=ctx, free_order=free_order, k_pool=k_pool, v_pool=v_pool, new_key=new_key,
                 new_value=new_value, query=query, num_blocks=nb)
+
+
+def make_beam_inputs(spec: Spec, distinct_steps: int = 16) -> dict:
+    """Inputs for the beam-search workload: num_prompts prompts (lengths by the
+    spec's law), each the root of `branches` beams; for `distinct_steps`
+    steps (cycled by longer runs) each beam's parent among its prompt's beams
+    and the new token's query, key and value. The pool has room for the
+    prompts plus max_divergent new tokens on every beam.
+
+    Returns CPU tensors: prompt_lens [P] int32; parents [steps, W] int32
+    (global beam indices); query [steps, W, Hq, D]; new_key/new_value
+    [steps, W, Hkv, D]; free_order [NB]; k_pool/v_pool [NB, Hkv, bs, D] (the
+    prompts' cached K/V are whatever their blocks hold); num_blocks."""
+    gen = torch.Generator().manual_seed(spec.seed)
+    dt = spec.torch_kv_dtype
+    P, B = spec.num_prompts, spec.branches
+    W = P * B
+    lens = context_lengths(replace(spec, num_seqs=P), gen)
+    bs = spec.block_size
+    needed = int(sum((int(c) + bs - 1) // bs for c in lens.tolist()))
+    nb = needed + W * ((spec.max_divergent + bs - 1) // bs + 2)
+    free_order = torch.randperm(nb, generator=gen).to(torch.int32)
+    choice = torch.randint(0, B, (distinct_steps, W), generator=gen, dtype=torch.int64)
+    parents = (choice + (torch.arange(W) // B * B)).to(torch.int32)
+    shape = (nb, spec.num_kv_heads, bs, spec.head_dim)
+    k_pool = _normal(gen, shape, 1.0, dt)
+    v_pool = _normal(gen, shape, 1.0, dt)
+    query = _normal(gen, (distinct_steps, W, spec.num_heads, spec.head_dim), 1.0, dt)
+    new_key = _normal(gen, (distinct_steps, W, spec.num_kv_heads, spec.head_dim), 1.0, dt)
+    new_value = _normal(gen, (distinct_steps, W, spec.num_kv_heads, spec.head_dim), 1.0, dt)
+    return dict(prompt_lens=lens, parents=parents, query=query, new_key=new_key, new_value=new_value,
+                free_order=free_order, k_pool=k_pool, v_pool=v_pool, num_blocks=nb)

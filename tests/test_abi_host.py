@@ -203,9 +203,63 @@ def test_device_pool_host_checks(pa):
     assert step(nb=0) == -3
     assert step(mb=0) == -3
     assert step(num_old=-1) == -3
-    assert step(num_old=1 << 20, mb=1 << 12) == -3      # flattened table index past int32
+    assert step(num_old=1 << 12, mb=1 << 18) == -3      # flattened table index past 2^30
+    assert step(num_old=20000, num_new=1) == -3           # per-beam values past the shared-memory stage
     assert step(new_t=fake) == -3                        # output tables alias the input tables
     assert step(cow=fake + 4) == -7
     assert lib.pa_copy_blocks_counted(fake, fake, fake, None, 4, 8, 2, 128, 16, 1, None) == -1
     assert lib.pa_copy_blocks_counted(fake, fake, fake, fake, 4, 8, 2, 100, 16, 1, None) == -5
     assert lib.pa_copy_blocks_counted(fake, fake, fake, fake, 0, 8, 2, 128, 16, 1, None) == 0
+
+
+def test_pool_export_matches_oracle(pa):
+    """pa_pool_export returns the counts and the free list (front first) that
+    the oracle pool holds after the same operations."""
+    from oracle.block_pool import BlockPool as OPool, Sequence, append_tokens, fork, release
+    order = np.random.default_rng(5).permutation(40).astype(np.int32)
+    for policy, name in ((pa.PA_POOL_FIFO, "fifo"), (pa.PA_POOL_LIFO, "lifo")):
+        lp = pa.BlockPool(40, 4, policy, free_order=order)
+        op = OPool(40, 4, policy=name, free_order=order.tolist())
+        tabs, seqs = [], []
+        for n in (9, 4, 13):
+            t = np.full(16, -1, np.int32)
+            lp.append(t, 0, n)
+            s = Sequence()
+            append_tokens(op, s, n)
+            tabs.append((t, n))
+            seqs.append(s)
+        child = np.full(16, -1, np.int32)
+        lp.fork(tabs[2][0], 13, child)
+        fork(op, seqs[2])
+        lp.release(tabs[0][0], 9)
+        release(op, seqs[0])
+        ref, fl = lp.export()
+        assert ref.tolist() == op.ref_counts and fl.tolist() == op.free_blocks
+
+
+def test_host_beam_step_matches_oracle(pa):
+    """batch.host_beam_step (the host-pool path the bench compares against)
+    makes the oracle's beam_step decisions."""
+    from oracle.block_pool import BlockPool as OPool, Sequence, append_tokens, beam_step
+    from paged_kv_cache_340_b200.batch import host_beam_step
+    rng = np.random.default_rng(8)
+    nb, bs, mb = 300, 4, 40
+    order = rng.permutation(nb).astype(np.int32)
+    lp = pa.BlockPool(nb, bs, pa.PA_POOL_FIFO, free_order=order)
+    op = OPool(nb, bs, policy="fifo", free_order=order.tolist())
+    beams, tables, ctx = [], np.full((5, mb), -1, np.int32), np.zeros(5, np.int32)
+    for i, n in enumerate((7, 12, 1, 30, 9)):
+        s = Sequence()
+        append_tokens(op, s, n)
+        beams.append(s)
+        ctx[i], _, _ = lp.append(tables[i], 0, n)
+    for _ in range(25):
+        parents = rng.integers(0, len(beams), size=int(rng.integers(1, 8))).astype(np.int32)
+        beams, slots, cow = beam_step(op, beams, parents.tolist())
+        tables, ctx, lslots, lcow = host_beam_step(lp, tables, ctx, parents)
+        assert lslots.tolist() == slots and [tuple(x) for x in lcow.tolist()] == cow
+        assert ctx.tolist() == [b.num_tokens for b in beams]
+        for t, b in zip(tables, beams):
+            assert t[:len(b.block_table)].tolist() == b.block_table
+    ref, fl = lp.export()
+    assert ref.tolist() == op.ref_counts and fl.tolist() == op.free_blocks

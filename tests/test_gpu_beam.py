@@ -38,24 +38,20 @@ def _policy(pa, name):
 
 def _start(pa, nb, bs, policy, lengths, seed):
     """Oracle pool and device pool from one seeded free order, with beams of
-    the given lengths appended through the oracle pool (the device pool is
-    brought to the same state by the same appends as identity beam steps)."""
+    the given lengths: appended through the oracle pool and through the
+    library's host pool, whose state is then loaded into the device pool."""
     order = np.random.default_rng(seed).permutation(nb).astype(np.int32)
     opool = OPool(nb, bs, policy=policy, free_order=order.tolist())
-    dpool = pa.DevicePool(nb, bs, _policy(pa, policy), free_order=order)
+    hpool = pa.BlockPool(nb, bs, _policy(pa, policy), free_order=order)
     beams = []
     for n in lengths:
         s = Sequence()
         append_tokens(opool, s, n)
         beams.append(s)
-    # the device pool reaches the same state by writing the same counts and free list
-    dpool.ref.copy_(torch.tensor(opool.ref_counts, dtype=torch.int32))
-    fl = opool.free_blocks
-    ring = np.full(nb, -1, np.int32)
-    ring[:len(fl)] = fl
-    dpool.ring.copy_(torch.from_numpy(ring))
-    dpool.header[3] = 0
-    dpool.header[4] = len(fl)
+        tab = np.full(nb, -1, np.int32)
+        hpool.append(tab, 0, n)
+        assert tab[:len(s.block_table)].tolist() == s.block_table
+    dpool = pa.DevicePool(nb, bs, _policy(pa, policy), host_pool=hpool)
     return opool, dpool, beams
 
 
@@ -73,6 +69,24 @@ def _device_step(pa, dpool, beams, parents, mb):
     pa.pa_beam_step(dpool, old_t, old_c, par, new_t, new_c, slots, cow, ncow)
     torch.cuda.synchronize()
     return new_t.cpu().numpy(), new_c.cpu().numpy(), slots.cpu().numpy(), cow.cpu().numpy(), int(ncow.item())
+
+
+def _host_copy(pa, opool):
+    """A library host pool in the oracle pool's state (same counts and free
+    list), built by the pool's own calls: allocate everything in free-list
+    order, then free back to the oracle's state."""
+    nb = opool.num_blocks
+    hp = pa.BlockPool(nb, opool.block_size, pa.PA_POOL_FIFO, free_order=np.arange(nb, dtype=np.int32))
+    for _ in range(nb):
+        hp.allocate()
+    for b in range(nb):                                  # counts: share up to the oracle's count
+        for _ in range(opool.ref_counts[b] - 1):
+            hp.share(b)
+    for b in opool.free_blocks:                          # free in free-list order
+        hp.free(b)
+    ref, fl = hp.export()
+    assert ref.tolist() == opool.ref_counts and fl.tolist() == opool.free_blocks
+    return hp
 
 
 def _assert_same_state(dpool, opool):
@@ -98,6 +112,28 @@ def test_dpool_init(pa):
     t, c, slots, cow, ncow = _device_step(pa, d3, [Sequence([1], 3)], [0], 4)
     assert pa.pa_read_device_errors() & pa.PA_DEVERR_POOL
     assert (slots == -1).all() and ncow == 0
+
+
+def test_dpool_load_checks_consistency(pa):
+    """A free list naming a block still in use, or a block of count 0 left off
+    the list, is refused (PA_DEVERR_POOL) and the state is unusable."""
+    nb = 16
+    ref = torch.zeros(nb, dtype=torch.int32, device="cuda")
+    ref[:4] = 1
+    good = torch.arange(4, nb, dtype=torch.int32, device="cuda")
+    for fl in (torch.arange(3, nb, dtype=torch.int32, device="cuda"),     # block 3 has count 1
+               torch.arange(5, nb, dtype=torch.int32, device="cuda"),     # block 4 (count 0) missing
+               torch.cat([good[:-1], good[:1]])):                         # a repeat
+        st = torch.empty(int(pa._lib.pa_dpool_state_bytes(nb)) // 4, dtype=torch.int32, device="cuda")
+        assert pa._lib.pa_dpool_load(st.data_ptr(), nb, 4, 0, ref.data_ptr(), fl.data_ptr(), fl.shape[0],
+                                     None) == 0
+        torch.cuda.synchronize()
+        assert pa.pa_read_device_errors() & pa.PA_DEVERR_POOL
+        assert st[5].item() == 0
+    st = torch.empty(int(pa._lib.pa_dpool_state_bytes(nb)) // 4, dtype=torch.int32, device="cuda")
+    assert pa._lib.pa_dpool_load(st.data_ptr(), nb, 4, 0, ref.data_ptr(), good.data_ptr(), good.shape[0], None) == 0
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_errors() == 0 and st[5].item() != 0
 
 
 def test_worked_example_on_device(pa):
@@ -178,7 +214,7 @@ def _beam_data_case(pa, seed, dtype):
     ob = []
     for r in roots:                                      # 4 beams per prompt share its blocks
         ob += [r] + [fork(opool, r) for _ in range(3)]
-    dpool.ref.copy_(torch.tensor(opool.ref_counts, dtype=torch.int32))
+    dpool = pa.DevicePool(NB, bs, pa.PA_POOL_LIFO, host_pool=_host_copy(pa, opool))
     W = len(ob)
     k = torch.randn((NB, Hkv, bs, D), generator=g).to(dtype)
     v = torch.randn((NB, Hkv, bs, D), generator=g).to(dtype)
@@ -234,20 +270,13 @@ def test_beam_step_in_cuda_graph(pa):
     a CUDA graph and replayed: same results as eager calls on a twin state."""
     nb, bs, mb, W = 256, 16, 16, 8
     order = np.random.default_rng(4).permutation(nb).astype(np.int32)
-    pools = [pa.DevicePool(nb, bs, pa.PA_POOL_FIFO, free_order=order) for _ in range(2)]
     opool = OPool(nb, bs, policy="fifo", free_order=order.tolist())
     beams = []
     for n in [40, 33, 16, 70, 5, 90, 64, 17]:
         s = Sequence()
         append_tokens(opool, s, n)
         beams.append(s)
-    for d in pools:
-        d.ref.copy_(torch.tensor(opool.ref_counts, dtype=torch.int32))
-        ring = np.full(nb, -1, np.int32)
-        ring[:len(opool.free_blocks)] = opool.free_blocks
-        d.ring.copy_(torch.from_numpy(ring))
-        d.header[3] = 0
-        d.header[4] = len(opool.free_blocks)
+    pools = [pa.DevicePool(nb, bs, pa.PA_POOL_FIFO, host_pool=_host_copy(pa, opool)) for _ in range(2)]
     Hkv, Hq, D = 4, 16, 128
     g = torch.Generator().manual_seed(9)
     caches = [[torch.randn((nb, Hkv, bs, D), generator=g).half().cuda() for _ in range(2)]]
@@ -292,3 +321,47 @@ def test_beam_step_in_cuda_graph(pa):
     assert torch.equal(pools[0].state, pools[1].state)
     assert all(torch.equal(a.view(torch.int16), b.view(torch.int16)) for a, b in zip(caches[0], caches[1]))
     assert pa.pa_read_device_errors() == 0
+
+
+def test_beam_search_workload_full_size(pa):
+    """The benchmark's beam-search workload at full size, in its launch
+    configuration (run_beam_step): the library host pool's prompt tables
+    equal the oracle pool's; over 6 device steps the tables, slots and pairs
+    equal the oracle's beam_step; the caches equal the oracle's byte copies;
+    the last step's decode (all 128 beams, all heads) matches the oracle."""
+    from oracle.block_pool import fork
+    from paged_kv_cache_340_b200.batch import build_beam_batch, run_beam_step
+    from paged_kv_cache_340_b200.workloads import SPECS, make_beam_inputs
+    spec = SPECS["beam_search_fp16"]
+    inp = make_beam_inputs(spec)
+    b = build_beam_batch(spec, inp)
+    P, B, bs = spec.num_prompts, spec.branches, spec.block_size
+    mb = b.tables[0].shape[1]
+    opool = OPool(b.num_blocks, bs, policy="fifo", free_order=inp["free_order"].tolist())
+    ob = []
+    for p in range(P):
+        root = Sequence()
+        append_tokens(opool, root, int(inp["prompt_lens"][p]))
+        ob += [root] + [fork(opool, root) for _ in range(B - 1)]
+    assert b.host_tables.tolist() == _tables(ob, mb).tolist()
+    _assert_same_state(b.pool, opool)
+    k_or, v_or = raw(inp["k_pool"]).copy(), raw(inp["v_pool"]).copy()
+    for i in range(6):
+        run_beam_step(b)
+        torch.cuda.synchronize()
+        k = i % inp["parents"].shape[0]
+        ob, oslots, ocow = beam_step(opool, ob, inp["parents"][k].tolist())
+        if ocow:
+            oracle.copy_blocks(k_or, v_or, np.array(ocow, np.int64))
+        oracle.reshape_and_cache(k_or, v_or, raw(inp["new_key"][k]), raw(inp["new_value"][k]), np.array(oslots))
+        dst = (i + 1) % 2
+        assert b.tables[dst].cpu().numpy().tolist() == _tables(ob, mb).tolist(), i
+        assert b.slot_mapping.cpu().tolist() == oslots
+        n = int(b.num_cow.item())
+        assert n == len(ocow) and [tuple(x) for x in b.cow_pairs[:n].cpu().tolist()] == ocow
+    assert pa.pa_read_device_errors() == 0
+    _assert_same_state(b.pool, opool)
+    assert np.array_equal(raw(b.k_cache), k_or) and np.array_equal(raw(b.v_cache), v_or)
+    ref = oracle.paged_decode(f64(inp["query"][5]), _f64_of(k_or, torch.float16), _f64_of(v_or, torch.float16),
+                              _tables(ob, mb), np.array([s.num_tokens for s in ob], np.int32), spec.scale, bs)
+    assert_attention_close(b.out, ref, torch.float16, "beam workload decode")
