@@ -52,6 +52,10 @@ def _load():
         lib.oracle_copy_blocks.argtypes = [u8p, u8p, i64p, ci, ci, ctypes.c_int64]
         lib.oracle_paged_prefill.argtypes = [f64p, f64p, i32p, f64p, f64p, i32p, ci, i32p, ci, ci, ci, ci, ci, ci,
                                              cd]
+        f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
+        i8p = np.ctypeslib.ndpointer(np.int8, flags="C_CONTIGUOUS")
+        lib.oracle_quantize_rows.argtypes = [f32p, ci, ci, i8p, f32p]
+        lib.oracle_reshape_and_cache_q8.argtypes = [i8p, i8p, f32p, f32p, f32p, f32p, i32p, ci, ci, ci, ci, ci]
         _lib = lib
     return _lib
 
@@ -169,3 +173,46 @@ def paged_prefill(query, q_start, k_cache, v_cache, block_tables, context_lens, 
     rc = _load().oracle_paged_prefill(out, q, qs, kc, vc, bt, bt.shape[1], cl, S, Hq, Hkv, D, bs, NB, float(scale))
     _check(rc, "paged_prefill")
     return out
+
+
+# ------------------------------------------------------------ int8 KV cache
+
+def quantize_rows(x):
+    """Symmetric int8 codes and fp32 scales of each row (last axis) of x,
+    computed in fp32 as pa_oracle.c states: returns (codes int8, scales f32)."""
+    x32 = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    n = x32.shape[-1]
+    rows = x32.size // n
+    q = np.empty(x32.shape, np.int8)
+    s = np.empty(x32.shape[:-1], np.float32)
+    _check(_load().oracle_quantize_rows(x32.reshape(-1), rows, n, q.reshape(-1), s.reshape(-1)), "quantize_rows")
+    return q, s
+
+
+def reshape_and_cache_q8(k_cache, v_cache, k_scale, v_scale, key, value, slot_mapping) -> None:
+    """In place: quantizes key/value [T, Hkv, D] (fp32 values) row by row into
+    the int8 pools [NB, Hkv, bs, D] and scale pools [NB, Hkv, bs]."""
+    NB, Hkv, bs, D = k_cache.shape
+    assert k_cache.dtype == v_cache.dtype == np.int8 and k_scale.dtype == v_scale.dtype == np.float32
+    for a in (k_cache, v_cache, k_scale, v_scale):
+        assert a.flags["C_CONTIGUOUS"]
+    sm = _i32(slot_mapping)
+    T = sm.shape[0]
+    kf = np.ascontiguousarray(np.asarray(key, dtype=np.float32))
+    vf = np.ascontiguousarray(np.asarray(value, dtype=np.float32))
+    assert kf.shape == (T, Hkv, D) and vf.shape == (T, Hkv, D)
+    rc = _load().oracle_reshape_and_cache_q8(k_cache.reshape(-1), v_cache.reshape(-1), k_scale.reshape(-1),
+                                             v_scale.reshape(-1), kf.reshape(-1), vf.reshape(-1), sm, T, NB, Hkv, D,
+                                             bs)
+    _check(rc, "reshape_and_cache_q8")
+
+
+def dequantize(codes, scales) -> np.ndarray:
+    """K = q * scale in double (exact: an 8-bit code times an fp32 scale)."""
+    return np.asarray(codes, dtype=np.float64) * np.asarray(scales, dtype=np.float64)[..., None]
+
+
+def paged_decode_q8(query, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, block_size):
+    """Paged decode over an int8 cache: attention over the dequantized K/V."""
+    return paged_decode(query, dequantize(k_cache, k_scale), dequantize(v_cache, v_scale), block_tables,
+                        context_lens, scale, block_size)

@@ -347,9 +347,9 @@ int oracle_reshape_and_cache(unsigned char *k_cache, unsigned char *v_cache,
 }
 
 /* Copy-on-write block copy: for each pair (src, dst), the whole physical
- * block dst of both pools becomes a byte copy of block src ([P4] §3.3:
- * "copy the original block's full contents to the new block", done with a
- * device-to-device copy). Pairs are applied in order. */
+ * block dst of both pools becomes a byte copy of block src ([P4] §3.3: the
+ * new block receives all of the old block's contents by a device-to-device
+ * copy). Pairs are applied in order. */
 int oracle_copy_blocks(unsigned char *k_cache, unsigned char *v_cache,
                        const int64_t *src_dst_pairs, int num_pairs,
                        int num_blocks, int64_t block_bytes)
@@ -425,5 +425,87 @@ int oracle_paged_prefill(double *out, const double *query, const int32_t *q_star
         }
     }
     free(K); free(V); free(z);
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------ int8 KV cache
+ *
+ * The pages list int8 among the paged backend's storage types ([P4] §3.4,
+ * attention backends) and name KV quantization as a way to cut cache memory
+ * at some cost in precision ([P2] §2.3, §6.3); they give no scheme. Reading
+ * taken here: symmetric int8 per (token, kv head) row of head_dim values,
+ * one fp32 scale per row, decided when the row is written:
+ *     amax = max_d |x_d|,  inv = 127 / amax,  q_d = round_half_even(x_d * inv)
+ *     clamped to [-127, 127],  scale = amax / 127;  amax = 0 gives q = 0, scale 0.
+ * Every step is one IEEE fp32 operation (x is the stored 16- or 32-bit value,
+ * exact in fp32), so the integer codes are the same wherever this is run in
+ * fp32 with round-to-nearest. The cache then holds K_t = q_t * scale_t.
+ * Scale pools: [num_blocks, num_kv_heads, block_size] fp32. */
+
+static void quantize_row(const float *x, int n, int8_t *q, float *scale)
+{
+    float amax = 0.0f;
+    for (int d = 0; d < n; ++d) {
+        float a = fabsf(x[d]);
+        if (a > amax)
+            amax = a;
+    }
+    if (amax == 0.0f) {
+        for (int d = 0; d < n; ++d)
+            q[d] = 0;
+        *scale = 0.0f;
+        return;
+    }
+    float inv = 127.0f / amax;
+    for (int d = 0; d < n; ++d) {
+        float y = x[d] * inv;
+        long r = lrintf(y);
+        if (r > 127)
+            r = 127;
+        if (r < -127)
+            r = -127;
+        q[d] = (int8_t)r;
+    }
+    *scale = amax / 127.0f;
+}
+
+/* rows x n values -> rows x n codes and rows scales. */
+int oracle_quantize_rows(const float *x, int rows, int n, int8_t *q, float *scale)
+{
+    if (rows < 0 || n <= 0)
+        return OR_BAD_ARG;
+    for (int r = 0; r < rows; ++r)
+        quantize_row(x + (size_t)r * n, n, q + (size_t)r * n, scale + r);
+    return OR_OK;
+}
+
+/* Slot write into an int8 cache: token i's row for kv head h is quantized
+ * and lands at (slot / block_size, h, slot % block_size) of the code pools,
+ * its scale at the same (block, h, offset) of the scale pools. slot < 0 is
+ * skipped. key/value: [num_tokens, num_kv_heads, head_dim] fp32 (the stored
+ * values, widened). */
+int oracle_reshape_and_cache_q8(int8_t *k_cache, int8_t *v_cache, float *k_scale, float *v_scale,
+                                const float *key, const float *value, const int32_t *slot_mapping,
+                                int num_tokens, int num_blocks, int num_kv_heads, int head_dim,
+                                int block_size)
+{
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
+        return OR_BAD_ARG;
+    for (int i = 0; i < num_tokens; ++i) {
+        int64_t slot = slot_mapping[i];
+        if (slot < 0)
+            continue;
+        if (slot >= (int64_t)num_blocks * block_size)
+            return OR_BAD_SLOT;
+        int block = (int)(slot / block_size);
+        int offset = (int)(slot % block_size);
+        for (int h = 0; h < num_kv_heads; ++h) {
+            size_t row = pool_row(block, h, offset, num_kv_heads, block_size, head_dim);
+            size_t srow = ((size_t)block * num_kv_heads + h) * block_size + offset;
+            size_t src = ((size_t)i * num_kv_heads + h) * head_dim;
+            quantize_row(key + src, head_dim, k_cache + row, k_scale + srow);
+            quantize_row(value + src, head_dim, v_cache + row, v_scale + srow);
+        }
+    }
     return OR_OK;
 }

@@ -356,3 +356,98 @@ def test_prefill_first_token_sees_only_itself(oracle_lib):
     assert np.array_equal(out[0], V[0][0])
     last = oracle.paged_decode(Q[L - 1:L], kp, vp, bt, cl, 0.4, 16)
     np.testing.assert_allclose(out[L - 1], last[0], rtol=0, atol=0)
+
+
+# ------------------------------------------------------------ int8 KV cache
+
+def test_quantize_worked_rows(oracle_lib):
+    """Hand-worked rows. [254, 1, -1, 3]: amax 254, inv = 127/254 = 0.5
+    exactly, codes rint(127, 0.5, -0.5, 1.5) = 127, 0, 0, 2 (halves go to
+    even), scale 2. [1, -3, 0.5, 2.5]: inv = 127/3, codes 42.33 -> 42,
+    -127, 21.17 -> 21, 105.83 -> 106. A zero row: codes 0, scale 0. A row
+    with amax 127 and integer values: scale 1, codes equal to the values."""
+    x = np.array([[254, 1, -1, 3], [1, -3, 0.5, 2.5], [0, 0, 0, 0], [127, -5, 64, -127]], np.float32)
+    q, s = oracle.quantize_rows(x)
+    assert q.tolist() == [[127, 0, 0, 2], [42, -127, 21, 106], [0, 0, 0, 0], [127, -5, 64, -127]]
+    assert s[0] == 2.0 and s[2] == 0.0 and s[3] == 1.0
+    assert s[1] == np.float32(3.0) / np.float32(127.0)
+
+
+def test_quantize_error_bound_and_range(oracle_lib):
+    """Every nonzero row uses the full code range (max |q| = 127, at the
+    row's largest magnitude), keeps each sign, and dequantizes within half a
+    step: |x - q s| <= s / 2 (plus fp32 rounding of the step)."""
+    rng = np.random.default_rng(21)
+    x = (rng.normal(size=(500, 128)) * rng.uniform(1e-3, 1e3, size=(500, 1))).astype(np.float32)
+    x[7] = 0.0
+    x[8, :5] = [1e-30, -2e-30, 0, 0, 0]
+    x[8, 5:] = 0
+    q, s = oracle.quantize_rows(x)
+    nz = np.abs(x).max(axis=1) > 0
+    assert np.all(np.abs(q[nz].astype(int)).max(axis=1) == 127)
+    assert np.all(q[~nz] == 0) and np.all(s[~nz] == 0)
+    assert np.all((q == 0) | (np.sign(q) == np.sign(x)))
+    err = np.abs(x.astype(np.float64) - q.astype(np.float64) * s[:, None].astype(np.float64))
+    assert np.all(err <= s[:, None].astype(np.float64) * (0.5 + 1e-5))
+    am = np.abs(x).max(axis=1)
+    assert np.allclose(s[nz], am[nz] / 127.0, rtol=1e-6)
+
+
+def test_reshape_and_cache_q8_lands_on_slot_rows(oracle_lib):
+    """Per kv head, code row s and scale s of the reshaped pools are token i's
+    quantized row (slot s = slots[i]); negative slots write nothing."""
+    rng = np.random.default_rng(12)
+    NB, Hkv, bs, D, T = 5, 2, 4, 16, 6
+    kc = rng.integers(-127, 128, size=(NB, Hkv, bs, D)).astype(np.int8)
+    vc = kc.copy()
+    ks = rng.uniform(size=(NB, Hkv, bs)).astype(np.float32)
+    vs = ks.copy()
+    k0, ks0 = kc.copy(), ks.copy()
+    key = rng.normal(size=(T, Hkv, D)).astype(np.float32)
+    val = rng.normal(size=(T, Hkv, D)).astype(np.float32)
+    slots = np.array([3, 19, -1, 0, 10, 7], np.int32)
+    oracle.reshape_and_cache_q8(kc, vc, ks, vs, key, val, slots)
+    krows = kc.transpose(1, 0, 2, 3).reshape(Hkv, NB * bs, D)
+    vrows = vc.transpose(1, 0, 2, 3).reshape(Hkv, NB * bs, D)
+    kscl = ks.transpose(1, 0, 2).reshape(Hkv, NB * bs)
+    vscl = vs.transpose(1, 0, 2).reshape(Hkv, NB * bs)
+    k0rows = k0.transpose(1, 0, 2, 3).reshape(Hkv, NB * bs, D)
+    ks0r = ks0.transpose(1, 0, 2).reshape(Hkv, NB * bs)
+    qk, sk = oracle.quantize_rows(key)
+    qv, sv = oracle.quantize_rows(val)
+    for i, s in enumerate(slots):
+        if s < 0:
+            continue
+        assert np.array_equal(krows[:, s], qk[i]) and np.array_equal(vrows[:, s], qv[i])
+        assert np.array_equal(kscl[:, s], sk[i]) and np.array_equal(vscl[:, s], sv[i])
+    for s in set(range(NB * bs)) - {int(x) for x in slots if x >= 0}:
+        assert np.array_equal(krows[:, s], k0rows[:, s]) and np.array_equal(kscl[:, s], ks0r[:, s])
+
+
+def test_decode_q8_closed_forms_and_precision(oracle_lib):
+    """ctx = 1 gives the dequantized V[0] exactly; over random N(0, 1) data
+    the int8 cache's attention stays within 2% (relative L2) of the same
+    attention over the unquantized values, the precision the pages warn
+    quantization costs."""
+    rng = np.random.default_rng(13)
+    S, Hq, Hkv, D, bs = 3, 8, 2, 64, 16
+    ctx = np.array([1, 200, 77], np.int32)
+    NB = 40
+    tables = np.full((S, 13), -1, np.int32)
+    perm = rng.permutation(NB)
+    pos = 0
+    for s_, L in enumerate(ctx):
+        n = -(-int(L) // bs)
+        tables[s_, :n] = perm[pos:pos + n]
+        pos += n
+    kf = rng.normal(size=(NB, Hkv, bs, D)).astype(np.float32)
+    vf = rng.normal(size=(NB, Hkv, bs, D)).astype(np.float32)
+    kq, ks = oracle.quantize_rows(kf)
+    vq, vs = oracle.quantize_rows(vf)
+    q = rng.normal(size=(S, Hq, D))
+    out = oracle.paged_decode_q8(q, kq, vq, ks, vs, tables, ctx, 1 / 8, bs)
+    v0 = vq[tables[0, 0], :, 0].astype(np.float64) * vs[tables[0, 0], :, 0, None]
+    assert np.array_equal(out[0], np.repeat(v0, Hq // Hkv, axis=0))
+    ref = oracle.paged_decode(q, kf, vf, tables, ctx, 1 / 8, bs)
+    rel = np.linalg.norm(out[1:] - ref[1:]) / np.linalg.norm(ref[1:])
+    assert 1e-4 < rel < 2e-2
