@@ -47,12 +47,17 @@ def elt(dtype: torch.dtype) -> int:
     return torch.tensor([], dtype=dtype).element_size()
 
 
+def kv_row_bytes(spec) -> int:
+    """Bytes of one (token, kv head) row of K or V in the cache (int8: codes
+    plus the fp32 row scale)."""
+    return spec.head_dim * elt(spec.torch_kv_dtype) + (4 if spec.kv_dtype == "i8" else 0)
+
+
 def decode_bytes(spec, ctx: np.ndarray) -> int:
     """Algorithmic bytes of one decode over the batch (K/V read once, q read,
     out written, the used table entries and the context lengths read)."""
-    e = elt(spec.torch_kv_dtype)
-    kv = int(ctx.astype(np.int64).sum()) * 2 * spec.num_kv_heads * spec.head_dim * e
-    qo = len(ctx) * spec.num_heads * spec.head_dim * (e + elt(spec.torch_out_dtype))
+    kv = int(ctx.astype(np.int64).sum()) * 2 * spec.num_kv_heads * kv_row_bytes(spec)
+    qo = len(ctx) * spec.num_heads * spec.head_dim * (elt(spec.torch_q_dtype) + elt(spec.torch_out_dtype))
     tables = 4 * int(((ctx.astype(np.int64) + spec.block_size - 1) // spec.block_size).sum()) + 4 * len(ctx)
     return kv + qo + tables
 
@@ -63,12 +68,13 @@ def kv_bytes_per_token(num_layers: int, num_kv_heads: int, head_dim: int, elt_by
 
 
 def write_bytes(spec, num_tokens: int) -> int:
-    row = spec.num_kv_heads * spec.head_dim * elt(spec.torch_kv_dtype)
-    return 2 * 2 * num_tokens * row + 4 * num_tokens
+    src = spec.num_kv_heads * spec.head_dim * elt(spec.torch_q_dtype)   # the new rows read
+    dst = spec.num_kv_heads * kv_row_bytes(spec)                         # and written (int8: + scale)
+    return 2 * num_tokens * (src + dst) + 4 * num_tokens
 
 
 def copy_bytes(spec, num_pairs: int) -> int:
-    blk = spec.num_kv_heads * spec.block_size * spec.head_dim * elt(spec.torch_kv_dtype)
+    blk = spec.num_kv_heads * spec.block_size * kv_row_bytes(spec)
     return 2 * 2 * num_pairs * blk + 16 * num_pairs
 
 
@@ -225,8 +231,8 @@ def time_steps(b, steps: int, warmup: int, world: int, sample_clocks=False, devi
     """Device time per step over `steps` steps (max over ranks), and the mean
     duration of each kernel of the step (a second pass with CUDA events
     around every launch, on the launching stream)."""
-    from paged_kv_cache_340_b200 import pa_copy_blocks, pa_decode, pa_decode_splitk, pa_reshape_and_cache, \
-        pa_splitk_reduce
+    from paged_kv_cache_340_b200 import pa_copy_blocks, pa_copy_blocks_q8, pa_decode, pa_decode_q8, \
+        pa_decode_splitk, pa_decode_splitk_q8, pa_reshape_and_cache, pa_reshape_and_cache_q8, pa_splitk_reduce
     spec = b.spec
     stream = torch.cuda.current_stream()
 
@@ -236,6 +242,26 @@ def time_steps(b, steps: int, warmup: int, world: int, sample_clocks=False, devi
 
     def step(ev=None):
         mark(ev, 0)
+        if b.k_scale is not None:  # int8 cache
+            if b.cow_pairs.shape[0]:
+                pa_copy_blocks_q8(b.k_cache, b.v_cache, b.k_scale, b.v_scale, b.cow_pairs, stream=stream)
+            mark(ev, 1)
+            pa_reshape_and_cache_q8(b.new_key, b.new_value, b.k_cache, b.v_cache, b.k_scale, b.v_scale,
+                                    b.slot_mapping, stream=stream)
+            mark(ev, 2)
+            if b.partition_size:
+                pa_decode_splitk_q8(b.workspace, b.query, b.k_cache, b.v_cache, b.k_scale, b.v_scale, b.block_tables,
+                                    b.context_lens, spec.scale, b.max_context_len, b.partition_size,
+                                    seq_order=b.seq_order, stream=stream)
+                mark(ev, 3)
+                pa_splitk_reduce(b.out, b.workspace, b.context_lens, b.max_context_len, b.partition_size,
+                                 stream=stream)
+            else:
+                pa_decode_q8(b.out, b.query, b.k_cache, b.v_cache, b.k_scale, b.v_scale, b.block_tables,
+                             b.context_lens, spec.scale, seq_order=b.seq_order, stream=stream)
+                mark(ev, 3)
+            mark(ev, 4)
+            return
         if b.cow_pairs.shape[0]:
             pa_copy_blocks(b.k_cache, b.v_cache, b.cow_pairs, stream=stream)
         mark(ev, 1)
@@ -586,6 +612,7 @@ def measure_other(name: str, steps: int, warmup: int):
            "pct_of_hbm_peak": round(100 * by["total"] / ms / 1e6 / peak, 1),
            "decode_kernel_ms": round(dec, 4), "decode_kernel_GBps": round(by["decode"] / dec / 1e6, 1),
            "partition_size": b.partition_size, "seq_tokens_per_s": round(spec.num_seqs / ms * 1e3, 1),
+           "context_tokens_per_s": round(float(b.host_context_lens.sum()) / ms * 1e3, 1),
            "kernels": kernel_lines(spec, b, kern, by)}
     del b
     torch.cuda.empty_cache()
@@ -670,7 +697,8 @@ def main():
     torch.cuda.empty_cache()
     if world == 1 and not args.no_others and args.workload == DEFAULT_WORKLOAD:
         line["other_workloads"] = {n: measure_other(n, 200, 10) for n in
-                                   ("gqa_bf16", "long_splitk_bf16", "parallel_sampling_fp16")}
+                                   ("gqa_bf16", "long_splitk_bf16", "parallel_sampling_fp16", "llama7b_mha_int8",
+                                    "gqa_int8")}
         line["prefill_workloads"] = {n: measure_prefill(n, 20, 3) for n in
                                      ("prefill_llama7b_mha_bf16", "chunked_prefill_gqa_bf16")}
         line["beam_search_fp16"] = measure_beam("beam_search_fp16", 200, 10)

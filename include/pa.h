@@ -257,6 +257,53 @@ int pa_copy_blocks_counted(void *k_cache, void *v_cache, const int64_t *src_dst_
                            int head_dim, int block_size, pa_dtype kv_dtype, cudaStream_t stream);
 
 /*
+ * int8 KV caches. The pages list int8 among the paged backend's storage
+ * types ([P4] §3.4, attention backends) and name KV quantization as a memory
+ * saving with a precision cost ([P2] §2.3, §6.3), without a scheme. This
+ * library's scheme: symmetric int8 per (token, kv head) row with one fp32
+ * scale, decided at the slot write:
+ *   amax = max_d |x_d|; q_d = round_half_even(x_d * (127 / amax)) clamped to
+ *   [-127, 127]; scale = amax / 127 (a zero row: codes 0, scale 0);
+ * every step one IEEE fp32 operation. The cache holds K_t = q_t * scale_t.
+ * Layouts: k_cache/v_cache int8 [num_blocks, num_kv_heads, block_size,
+ * head_dim]; k_scale/v_scale fp32 [num_blocks, num_kv_heads, block_size];
+ * all device pointers 16-byte aligned. Half the bytes of an fp16 cache plus
+ * 4 bytes per row.
+ */
+
+/* Quantizing slot write: key/value [num_tokens, num_kv_heads, head_dim] of
+ * src_dtype (PA_F32, PA_F16 or PA_BF16) -> codes and scales at each token's
+ * slot (slot < 0 skipped, out of range PA_DEVERR_SLOT). */
+int pa_reshape_and_cache_q8(const void *key, const void *value, pa_dtype src_dtype, int8_t *k_cache,
+                            int8_t *v_cache, float *k_scale, float *v_scale, const int32_t *slot_mapping,
+                            int num_tokens, int num_blocks, int num_kv_heads, int head_dim, int block_size,
+                            cudaStream_t stream);
+
+/* pa_decode over an int8 cache: out = softmax(scale q . K_t) V_t with
+ * K_t = kq_t * k_scale_t, V_t = vq_t * v_scale_t. query is q_dtype (PA_F16
+ * or PA_BF16; a bf16 query is converted to fp16 for the tensor cores, exact
+ * for magnitudes in [2^-14, 65504]); out_dtype q_dtype or PA_F32. Other
+ * arguments, checks and device errors as pa_decode. */
+int pa_decode_q8(void *out, const void *query, pa_dtype q_dtype, const int8_t *k_cache, const int8_t *v_cache,
+                 const float *k_scale, const float *v_scale, const int32_t *block_tables, int max_blocks_per_seq,
+                 const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                 float scale, int block_size, int num_blocks, pa_dtype out_dtype, const int32_t *seq_order,
+                 cudaStream_t stream);
+
+/* pa_decode_splitk over an int8 cache (then pa_splitk_reduce as usual). */
+int pa_decode_splitk_q8(void *workspace, size_t workspace_bytes, const void *query, pa_dtype q_dtype,
+                        const int8_t *k_cache, const int8_t *v_cache, const float *k_scale, const float *v_scale,
+                        const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                        int num_seqs, int num_heads, int num_kv_heads, int head_dim, float scale, int block_size,
+                        int num_blocks, int max_context_len, int partition_size, const int32_t *seq_order,
+                        cudaStream_t stream);
+
+/* pa_copy_blocks for an int8 cache: codes and scales of each pair. */
+int pa_copy_blocks_q8(int8_t *k_cache, int8_t *v_cache, float *k_scale, float *v_scale,
+                      const int64_t *src_dst_pairs, int num_pairs, int num_blocks, int num_kv_heads, int head_dim,
+                      int block_size, cudaStream_t stream);
+
+/*
  * Host block pool (no device memory): free list, reference counts and the
  * copy-on-write decision. These are plain host calls on host memory.
  * [P2] §3.3-§3.4 and §4.2 (PhysicalBlockPool: allocate sets the count to 1,

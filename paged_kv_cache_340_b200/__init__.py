@@ -43,7 +43,8 @@ EXPORTED = (
     "pa_pool_fork", "pa_pool_release", "pa_decode_splitk_static", "pa_prefill",
     "pa_prefix_cache_create", "pa_prefix_cache_destroy", "pa_prefix_num_entries", "pa_prefix_get_or_create",
     "pa_prefix_release", "pa_prefix_ref_count", "pa_copy_blocks_counted", "pa_dpool_state_bytes", "pa_dpool_init",
-    "pa_beam_step", "pa_pool_export", "pa_dpool_load",
+    "pa_beam_step", "pa_pool_export", "pa_dpool_load", "pa_reshape_and_cache_q8", "pa_decode_q8",
+    "pa_decode_splitk_q8", "pa_copy_blocks_q8",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -101,6 +102,12 @@ def _load() -> ctypes.CDLL:
         "pa_beam_step": (i32, [vp, i32, i32, vp, vp, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp]),
         "pa_pool_export": (i32, [vp, i32p, i32p, ctypes.POINTER(ctypes.c_int)]),
         "pa_dpool_load": (i32, [vp, i32, i32, i32, vp, vp, i32, vp]),
+        "pa_reshape_and_cache_q8": (i32, [vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]),
+        "pa_decode_q8": (i32, [vp, vp, i32, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, vp,
+                               vp]),
+        "pa_decode_splitk_q8": (i32, [vp, sz, vp, i32, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32,
+                                      i32, i32, vp, vp]),
+        "pa_copy_blocks_q8": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -193,6 +200,50 @@ def pa_decode_splitk(workspace, query, k_cache, v_cache, block_tables, context_l
                                _ptr(context_lens), S, Hq, Hkv, D, float(scale), bs, NB, int(max_context_len),
                                int(partition_size), _dtype(k_cache), _ptr(seq_order), _stream(stream))
     _check(rc, "pa_decode_splitk")
+
+
+# ------------------------------------------------------------ int8 caches
+# k_cache/v_cache int8 [NB, Hkv, bs, D]; k_scale/v_scale float32 [NB, Hkv, bs].
+
+def pa_reshape_and_cache_q8(key, value, k_cache, v_cache, k_scale, v_scale, slot_mapping, stream=None) -> None:
+    NB, Hkv, bs, D = k_cache.shape
+    assert k_cache.dtype == torch.int8 and k_scale.dtype == torch.float32
+    rc = _lib.pa_reshape_and_cache_q8(_ptr(key), _ptr(value), _dtype(key), _ptr(k_cache), _ptr(v_cache),
+                                      _ptr(k_scale), _ptr(v_scale), _ptr(slot_mapping), slot_mapping.shape[0], NB,
+                                      Hkv, D, bs, _stream(stream))
+    _check(rc, "pa_reshape_and_cache_q8")
+
+
+def pa_decode_q8(out, query, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, seq_order=None,
+                 stream=None) -> None:
+    S, Hq, D = query.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    assert k_cache.dtype == torch.int8 and k_scale.dtype == torch.float32
+    rc = _lib.pa_decode_q8(_ptr(out), _ptr(query), _dtype(query), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale),
+                           _ptr(v_scale), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S, Hq, Hkv,
+                           D, float(scale), bs, NB, _dtype(out), _ptr(seq_order), _stream(stream))
+    _check(rc, "pa_decode_q8")
+
+
+def pa_decode_splitk_q8(workspace, query, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale,
+                        max_context_len, partition_size, seq_order=None, stream=None) -> None:
+    S, Hq, D = query.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    assert k_cache.dtype == torch.int8 and k_scale.dtype == torch.float32
+    rc = _lib.pa_decode_splitk_q8(_ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(query),
+                                  _dtype(query), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+                                  _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S, Hq, Hkv, D,
+                                  float(scale), bs, NB, int(max_context_len), int(partition_size), _ptr(seq_order),
+                                  _stream(stream))
+    _check(rc, "pa_decode_splitk_q8")
+
+
+def pa_copy_blocks_q8(k_cache, v_cache, k_scale, v_scale, src_dst_pairs, stream=None) -> None:
+    NB, Hkv, bs, D = k_cache.shape
+    n = src_dst_pairs.shape[0] if src_dst_pairs is not None else 0
+    rc = _lib.pa_copy_blocks_q8(_ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+                                _ptr(src_dst_pairs) if n else None, n, NB, Hkv, D, bs, _stream(stream))
+    _check(rc, "pa_copy_blocks_q8")
 
 
 def pa_splitk_reduce(out, workspace, context_lens, max_context_len, partition_size, stream=None) -> None:

@@ -16,8 +16,9 @@ import numpy as np
 import torch
 
 from . import (PA_POOL_FIFO, BlockPool, DevicePool, pa_beam_step, pa_choose_partition, pa_copy_blocks,
-               pa_copy_blocks_counted, pa_decode, pa_decode_splitk, pa_prefill, pa_reshape_and_cache,
-               pa_splitk_reduce, pa_splitk_workspace_bytes)
+               pa_copy_blocks_counted, pa_copy_blocks_q8, pa_decode, pa_decode_q8, pa_decode_splitk,
+               pa_decode_splitk_q8, pa_prefill, pa_reshape_and_cache, pa_reshape_and_cache_q8, pa_splitk_reduce,
+               pa_splitk_workspace_bytes)
 from .workloads import Spec
 
 
@@ -43,6 +44,8 @@ class DecodeBatch:
     host_slots: np.ndarray
     host_cow: np.ndarray
     host_context_lens: np.ndarray
+    k_scale: Optional[torch.Tensor] = None  # int8 caches: device float32 [NB, Hkv, bs] row scales
+    v_scale: Optional[torch.Tensor] = None
 
 
 def _blocks(n: int, bs: int) -> int:
@@ -88,14 +91,17 @@ def build_decode_batch(spec: Spec, inputs: dict, device="cuda", partition_size: 
     max_ctx = int(ctx.max())
     if partition_size is None:
         partition_size = spec.partition_size or pa_choose_partition(S, spec.num_kv_heads, max_ctx, bs, spec.head_dim,
-                                                                    spec.torch_kv_dtype)
+                                                                    spec.torch_q_dtype)
     ws = None
     if partition_size:
         nbytes = pa_splitk_workspace_bytes(S, spec.num_heads, spec.head_dim, max_ctx, partition_size)
         ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    if spec.kv_dtype == "i8":
+        kc, vc, ks, vs = quantized_pool(inputs["k_pool"], inputs["v_pool"], dev)
+    else:
+        kc, vc, ks, vs = inputs["k_pool"].to(dev), inputs["v_pool"].to(dev), None, None
     return DecodeBatch(
-        spec=spec, num_blocks=nb,
-        k_cache=inputs["k_pool"].to(dev), v_cache=inputs["v_pool"].to(dev),
+        spec=spec, num_blocks=nb, k_cache=kc, v_cache=vc, k_scale=ks, v_scale=vs,
         query=inputs["query"].to(dev),
         out=torch.empty((S, spec.num_heads, spec.head_dim), dtype=spec.torch_out_dtype, device=dev),
         block_tables=torch.from_numpy(tables).to(dev), context_lens=torch.from_numpy(ctx).to(dev),
@@ -182,19 +188,58 @@ def write_prefix(batch: SamplingBatch, stream=None) -> None:
                          stream=stream)
 
 
+def quantized_pool(k_pool: torch.Tensor, v_pool: torch.Tensor, device, chunk_blocks: int = 4096):
+    """int8 codes and row scales of whole K/V pools [NB, Hkv, bs, D] (values of
+    a 16- or 32-bit type), made by the library's quantizing slot write with
+    every slot written once (slot b * bs + o <- pool row (b, :, o))."""
+    NB, Hkv, bs, D = k_pool.shape
+    dev = torch.device(device)
+    kc = torch.empty((NB, Hkv, bs, D), dtype=torch.int8, device=dev)
+    vc = torch.empty_like(kc)
+    ks = torch.empty((NB, Hkv, bs), dtype=torch.float32, device=dev)
+    vs = torch.empty_like(ks)
+    for b0 in range(0, NB, chunk_blocks):
+        b1 = min(NB, b0 + chunk_blocks)
+        kk = k_pool[b0:b1].to(dev).permute(0, 2, 1, 3).reshape(-1, Hkv, D).contiguous()
+        vv = v_pool[b0:b1].to(dev).permute(0, 2, 1, 3).reshape(-1, Hkv, D).contiguous()
+        slots = torch.arange(b0 * bs, b1 * bs, dtype=torch.int32, device=dev)
+        pa_reshape_and_cache_q8(kk, vv, kc, vc, ks, vs, slots)
+    return kc, vc, ks, vs
+
+
 def run_step(batch: DecodeBatch, stream=None) -> None:
     """One pass of the hot path: copy-on-write block copies (if any), the slot
     write of this step's tokens, then decode (split-K + reduce when the batch
-    has a partition size)."""
+    has a partition size). int8 caches quantize at the slot write."""
+    q8 = batch.k_scale is not None
     if batch.cow_pairs.shape[0]:
-        pa_copy_blocks(batch.k_cache, batch.v_cache, batch.cow_pairs, stream=stream)
-    pa_reshape_and_cache(batch.new_key, batch.new_value, batch.k_cache, batch.v_cache, batch.slot_mapping,
-                         stream=stream)
+        if q8:
+            pa_copy_blocks_q8(batch.k_cache, batch.v_cache, batch.k_scale, batch.v_scale, batch.cow_pairs,
+                              stream=stream)
+        else:
+            pa_copy_blocks(batch.k_cache, batch.v_cache, batch.cow_pairs, stream=stream)
+    if q8:
+        pa_reshape_and_cache_q8(batch.new_key, batch.new_value, batch.k_cache, batch.v_cache, batch.k_scale,
+                                batch.v_scale, batch.slot_mapping, stream=stream)
+    else:
+        pa_reshape_and_cache(batch.new_key, batch.new_value, batch.k_cache, batch.v_cache, batch.slot_mapping,
+                             stream=stream)
     run_decode(batch, stream)
 
 
 def run_decode(batch: DecodeBatch, stream=None) -> None:
     spec = batch.spec
+    if batch.k_scale is not None:
+        if batch.partition_size:
+            pa_decode_splitk_q8(batch.workspace, batch.query, batch.k_cache, batch.v_cache, batch.k_scale,
+                                batch.v_scale, batch.block_tables, batch.context_lens, spec.scale,
+                                batch.max_context_len, batch.partition_size, seq_order=batch.seq_order, stream=stream)
+            pa_splitk_reduce(batch.out, batch.workspace, batch.context_lens, batch.max_context_len,
+                             batch.partition_size, stream=stream)
+        else:
+            pa_decode_q8(batch.out, batch.query, batch.k_cache, batch.v_cache, batch.k_scale, batch.v_scale,
+                         batch.block_tables, batch.context_lens, spec.scale, seq_order=batch.seq_order, stream=stream)
+        return
     if batch.partition_size:
         pa_decode_splitk(batch.workspace, batch.query, batch.k_cache, batch.v_cache, batch.block_tables,
                          batch.context_lens, spec.scale, batch.max_context_len, batch.partition_size,

@@ -355,6 +355,151 @@ int pa_copy_blocks_counted(void *k_cache, void *v_cache, const int64_t *src_dst_
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------ int8 caches
+
+int pa_reshape_and_cache_q8(const void *key, const void *value, pa_dtype src_dtype, int8_t *k_cache,
+                            int8_t *v_cache, float *k_scale, float *v_scale, const int32_t *slot_mapping,
+                            int num_tokens, int num_blocks, int num_kv_heads, int head_dim, int block_size,
+                            cudaStream_t stream) {
+    if (num_tokens < 0 || num_blocks < 0 || num_kv_heads <= 0) return PA_ERR_SHAPE;
+    if (elt_bytes(src_dtype) == 0) return PA_ERR_DTYPE;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_HEAD_DIM;
+    if (block_size != 16 && block_size != 32) return PA_ERR_BLOCK_SIZE;
+    if ((long long)num_blocks * block_size > INT_MAX) return PA_ERR_SHAPE;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !k_cache || !v_cache || !k_scale || !v_scale || !slot_mapping) return PA_ERR_NULL;
+    if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(k_scale, 16) || !aligned(v_scale, 16) || !aligned(slot_mapping, 4))
+        return PA_ERR_ALIGN;
+    unsigned int *err = nullptr;
+    if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    cudaError_t e = launch_reshape_and_cache_q8(key, value, src_dtype, k_cache, v_cache, k_scale, v_scale,
+                                                slot_mapping, num_tokens, num_blocks, num_kv_heads, head_dim,
+                                                block_size, err, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// Shared by the int8 decode entries: query type, scale pools, then the common checks.
+static int check_q8_args(const void *query, pa_dtype q_dtype, const int8_t *k_cache, const int8_t *v_cache,
+                         const float *k_scale, const float *v_scale, const int32_t *block_tables,
+                         int max_blocks_per_seq, const int32_t *context_lens, int num_seqs, int num_heads,
+                         int num_kv_heads, int head_dim, float scale, int block_size, int num_blocks) {
+    if (q_dtype != PA_F16 && q_dtype != PA_BF16) return PA_ERR_DTYPE;
+    int rc = check_decode_args(query, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                               num_heads, num_kv_heads, head_dim, scale, block_size, num_blocks, q_dtype);
+    if (rc != PA_OK || num_seqs == 0) return rc;
+    if (!k_scale || !v_scale) return PA_ERR_NULL;
+    if (!aligned(k_scale, 16) || !aligned(v_scale, 16)) return PA_ERR_ALIGN;
+    return PA_OK;
+}
+
+int pa_decode_q8(void *out, const void *query, pa_dtype q_dtype, const int8_t *k_cache, const int8_t *v_cache,
+                 const float *k_scale, const float *v_scale, const int32_t *block_tables, int max_blocks_per_seq,
+                 const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                 float scale, int block_size, int num_blocks, pa_dtype out_dtype, const int32_t *seq_order,
+                 cudaStream_t stream) {
+    int rc = check_q8_args(query, q_dtype, k_cache, v_cache, k_scale, v_scale, block_tables, max_blocks_per_seq,
+                           context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale, block_size, num_blocks);
+    if (rc != PA_OK) return rc;
+    if (out_dtype != q_dtype && out_dtype != PA_F32) return PA_ERR_DTYPE;
+    if (num_seqs == 0) return PA_OK;
+    if (!aligned(seq_order, 4)) return PA_ERR_ALIGN;
+    if (!out) return PA_ERR_NULL;
+    if (!aligned(out, 16)) return PA_ERR_ALIGN;
+    unsigned int *err = nullptr;
+    if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    DecodeParams p{};
+    p.out = out;
+    p.query = query;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.seq_order = seq_order;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.num_blocks = num_blocks;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.partition_size = 0;
+    p.max_parts = 1;
+    p.max_context_len = INT_MAX;
+    p.out_dtype = out_dtype;
+    p.err = err;
+    cudaError_t e = launch_decode_q8(p, q_dtype, head_dim, block_size, num_heads / num_kv_heads, 1, num_kv_heads,
+                                     num_seqs, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_decode_splitk_q8(void *workspace, size_t workspace_bytes, const void *query, pa_dtype q_dtype,
+                        const int8_t *k_cache, const int8_t *v_cache, const float *k_scale, const float *v_scale,
+                        const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                        int num_seqs, int num_heads, int num_kv_heads, int head_dim, float scale, int block_size,
+                        int num_blocks, int max_context_len, int partition_size, const int32_t *seq_order,
+                        cudaStream_t stream) {
+    int rc = check_q8_args(query, q_dtype, k_cache, v_cache, k_scale, v_scale, block_tables, max_blocks_per_seq,
+                           context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale, block_size, num_blocks);
+    if (rc != PA_OK) return rc;
+    if (max_context_len < 0) return PA_ERR_SHAPE;
+    if (partition_size <= 0 || partition_size % block_size != 0) return PA_ERR_PARTITION;
+    if (num_seqs == 0 || max_context_len == 0) return PA_OK;
+    if (!aligned(seq_order, 4)) return PA_ERR_ALIGN;
+    const size_t need = pa_splitk_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, partition_size);
+    if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return PA_ERR_ALIGN;
+    unsigned int *err = nullptr;
+    if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    const int mp = max_parts_of(max_context_len, partition_size);
+    DecodeParams p{};
+    p.ws_ml = static_cast<float *>(workspace);
+    p.ws_acc = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) +
+                                         pa_splitk_acc_offset(num_seqs, num_heads, max_context_len, partition_size));
+    p.query = query;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.seq_order = seq_order;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.num_blocks = num_blocks;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.partition_size = partition_size;
+    p.max_parts = mp;
+    p.max_context_len = max_context_len;
+    p.out_dtype = PA_F32;
+    p.err = err;
+    cudaError_t e = launch_decode_q8(p, q_dtype, head_dim, block_size, num_heads / num_kv_heads, mp, num_kv_heads,
+                                     num_seqs, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_copy_blocks_q8(int8_t *k_cache, int8_t *v_cache, float *k_scale, float *v_scale,
+                      const int64_t *src_dst_pairs, int num_pairs, int num_blocks, int num_kv_heads, int head_dim,
+                      int block_size, cudaStream_t stream) {
+    if (num_pairs < 0 || num_blocks < 0 || num_kv_heads <= 0) return PA_ERR_SHAPE;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_HEAD_DIM;
+    if (block_size != 16 && block_size != 32) return PA_ERR_BLOCK_SIZE;
+    if (num_pairs == 0) return PA_OK;
+    if (!k_cache || !v_cache || !k_scale || !v_scale || !src_dst_pairs) return PA_ERR_NULL;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(k_scale, 16) || !aligned(v_scale, 16) ||
+        !aligned(src_dst_pairs, 8))
+        return PA_ERR_ALIGN;
+    unsigned int *err = nullptr;
+    if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    cudaError_t e = launch_copy_blocks(k_cache, v_cache, src_dst_pairs, num_pairs, nullptr, num_blocks,
+                                       (size_t)num_kv_heads * block_size * head_dim, err, stream);
+    if (e == cudaSuccess)
+        e = launch_copy_blocks(k_scale, v_scale, src_dst_pairs, num_pairs, nullptr, num_blocks,
+                               (size_t)num_kv_heads * block_size * sizeof(float), err, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 size_t pa_dpool_state_bytes(int num_blocks) {
     if (num_blocks <= 0) return 0;
     return (PA_DPOOL_HEADER_WORDS + (size_t)PA_DPOOL_ARRAYS * num_blocks) * sizeof(int32_t);

@@ -97,3 +97,100 @@ cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *pair
 }
 
 }  // namespace pa
+
+namespace pa {
+
+// Slot write into an int8 cache: one warp per (token, kv head) row. The row's
+// largest magnitude sets the scale; codes are round-half-even(x * (127 /
+// amax)), clamped to +-127, every step one IEEE fp32 operation (the same
+// arithmetic wherever it runs); scale = amax / 127; a zero row gives codes 0
+// and scale 0. The pages name int8 KV storage without a scheme; this is the
+// library's (symmetric, per token and kv head).
+template <typename TS, int D>
+__global__ void __launch_bounds__(256)
+    reshape_and_cache_q8_kernel(const TS *__restrict__ key, const TS *__restrict__ value, int8_t *__restrict__ k_cache,
+                                int8_t *__restrict__ v_cache, float *__restrict__ k_scale, float *__restrict__ v_scale,
+                                const int32_t *__restrict__ slot_mapping, int num_tokens, int num_blocks,
+                                int num_kv_heads, int block_size, unsigned int *err) {
+    constexpr int kPer = D / 32;  // values per lane
+    const int lane = threadIdx.x & 31;
+    const long long rows = (long long)num_tokens * num_kv_heads;
+    const long long slots = (long long)num_blocks * block_size;
+    for (long long row = (blockIdx.x * (long long)blockDim.x + threadIdx.x) / 32; row < rows;
+         row += (long long)gridDim.x * blockDim.x / 32) {
+        const int token = (int)(row / num_kv_heads);
+        const int h = (int)(row - (long long)token * num_kv_heads);
+        const int slot = __ldg(slot_mapping + token);
+        if (slot < 0) continue;
+        if (slot >= slots) {
+            if (h == 0 && lane == 0) record_error(err, PA_DEVERR_SLOT);
+            continue;
+        }
+        const int block = slot / block_size;
+        const int offset = slot - block * block_size;
+        const size_t srow = ((size_t)block * num_kv_heads + h) * block_size + offset;
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv) {
+            const TS *src = (kv == 0 ? key : value) + row * D + lane * kPer;
+            float x[kPer];
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) x[e] = static_cast<float>(src[e]);
+            float amax = 0.f;
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) amax = fmaxf(amax, fabsf(x[e]));
+#pragma unroll
+            for (int mk = 16; mk >= 1; mk >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, mk));
+            uint32_t packed = 0;
+            if (amax > 0.f) {
+                const float inv = __fdiv_rn(127.f, amax);
+#pragma unroll
+                for (int e = 0; e < kPer; ++e) {
+                    int qv = __float2int_rn(__fmul_rn(x[e], inv));
+                    qv = max(-127, min(127, qv));
+                    packed |= (uint32_t)(qv & 0xff) << (8 * e);
+                }
+            }
+            int8_t *dst = (kv == 0 ? k_cache : v_cache) + srow * D + lane * kPer;
+            if constexpr (kPer == 4)
+                *reinterpret_cast<uint32_t *>(dst) = packed;
+            else
+                *reinterpret_cast<uint16_t *>(dst) = (uint16_t)packed;
+            if (lane == 0) (kv == 0 ? k_scale : v_scale)[srow] = amax > 0.f ? __fdiv_rn(amax, 127.f) : 0.f;
+        }
+    }
+}
+
+template <typename TS>
+static cudaError_t launch_q8_t(const void *key, const void *value, int8_t *k_cache, int8_t *v_cache, float *k_scale,
+                               float *v_scale, const int32_t *slot_mapping, int num_tokens, int num_blocks,
+                               int num_kv_heads, int head_dim, int block_size, unsigned int *err, cudaStream_t stream) {
+    const long long rows = (long long)num_tokens * num_kv_heads;
+    long long blocks = (rows * 32 + 255) / 256;
+    const long long cap = (long long)sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    if (head_dim == 128)
+        reshape_and_cache_q8_kernel<TS, 128><<<(unsigned)blocks, 256, 0, stream>>>(
+            static_cast<const TS *>(key), static_cast<const TS *>(value), k_cache, v_cache, k_scale, v_scale,
+            slot_mapping, num_tokens, num_blocks, num_kv_heads, block_size, err);
+    else
+        reshape_and_cache_q8_kernel<TS, 64><<<(unsigned)blocks, 256, 0, stream>>>(
+            static_cast<const TS *>(key), static_cast<const TS *>(value), k_cache, v_cache, k_scale, v_scale,
+            slot_mapping, num_tokens, num_blocks, num_kv_heads, block_size, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reshape_and_cache_q8(const void *key, const void *value, pa_dtype src_dtype, int8_t *k_cache,
+                                        int8_t *v_cache, float *k_scale, float *v_scale,
+                                        const int32_t *slot_mapping, int num_tokens, int num_blocks,
+                                        int num_kv_heads, int head_dim, int block_size, unsigned int *err,
+                                        cudaStream_t stream) {
+    if (num_tokens == 0) return cudaSuccess;
+    switch (src_dtype) {
+        case PA_F32: return launch_q8_t<float>(key, value, k_cache, v_cache, k_scale, v_scale, slot_mapping, num_tokens, num_blocks, num_kv_heads, head_dim, block_size, err, stream);
+        case PA_F16: return launch_q8_t<__half>(key, value, k_cache, v_cache, k_scale, v_scale, slot_mapping, num_tokens, num_blocks, num_kv_heads, head_dim, block_size, err, stream);
+        case PA_BF16: return launch_q8_t<__nv_bfloat16>(key, value, k_cache, v_cache, k_scale, v_scale, slot_mapping, num_tokens, num_blocks, num_kv_heads, head_dim, block_size, err, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pa

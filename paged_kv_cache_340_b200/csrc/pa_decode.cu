@@ -59,13 +59,15 @@ struct DecodeShape {
     static constexpr int kNvl = kNv >= kLpt ? kNv / kLpt : 1;   // scores a lane keeps
     static constexpr int kDup = kNv >= kLpt ? 1 : kLpt / kNv;   // lanes keeping the same score
     static constexpr int kLanesPerG = kLpt / G;        // lanes whose scores belong to one head
-    // 16-bit GQA groups run QK^T and PV on the tensor cores; MHA and fp32 on
-    // the CUDA cores.
-    static constexpr bool kUseMma = (kElt == 2) && (G >= 2);
+    // 16-bit GQA groups and every int8 cache run QK^T and PV on the tensor
+    // cores; 16-bit MHA and fp32 on the CUDA cores.
+    static constexpr bool kInt8 = (kElt == 1);
+    static constexpr bool kUseMma = kInt8 || ((kElt == 2) && (G >= 2));
     static constexpr int kWarps = 4;
     static constexpr int kThreads = kWarps * 32;
     static constexpr int kTileBytes = kTS * D * kElt;  // 16 token rows of one kv head, K or V
-    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kScaleBytes = kInt8 ? kTS * 4 : 0;  // int8: the 16 rows' fp32 scales, K or V
+    static constexpr int kStageBytes = 2 * kTileBytes + 2 * kScaleBytes;
     static constexpr int kStages = 8;                  // two buffers per warp
     static constexpr int kRowGroups = kUseMma ? kWarps : kWarps * kRows;
     static constexpr int kRingBytes = kStages * kStageBytes;
@@ -79,10 +81,11 @@ struct DecodeShape {
 
     static_assert(kStages == 2 * kWarps, "stage k: warp k % 4, buffer k % 8");
     static_assert(BS % kTS == 0, "block size is a multiple of the stage");
-    static_assert(kLpt >= 1 && kLpt <= 32 && (32 % kLpt) == 0, "row width");
-    static_assert(kTS % kRows == 0 && kTpg % kTc == 0, "stage split");
-    static_assert(G <= kLpt, "a lane's kept scores must belong to one query head");
-    static_assert(kNvl <= kTc, "kept scores within one head");
+    // the CUDA-core consumer's lane layout
+    static_assert(kUseMma || (kLpt >= 1 && kLpt <= 32 && (32 % kLpt) == 0), "row width");
+    static_assert(kUseMma || (kTS % kRows == 0 && kTpg % kTc == 0), "stage split");
+    static_assert(kUseMma || G <= kLpt, "a lane's kept scores must belong to one query head");
+    static_assert(kUseMma || kNvl <= kTc, "kept scores within one head");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -302,6 +305,11 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+    Mma<__half>::mma(c, a0, a1, a2, a3, b0, b1);
+}
+
 // One warp's share on the tensor cores, in transposed form so that the
 // 16-row M side of the MMA is filled by tokens and head dims instead of the
 // group's 2-8 query heads. Per 16-token stage, with lane = 4 r + q:
@@ -481,13 +489,222 @@ struct MmaConsumer {
     }
 };
 
+// ------------------------------------------------- int8 tensor-core consumer
+
+// int8 codes -> exact fp16: x + 128 as an unsigned byte becomes the mantissa
+// of 1024 + (x + 128) (fp16 0x64xx), then 1152 is subtracted (0x6480).
+__device__ __forceinline__ uint32_t i8pair_to_h2(uint32_t biased, unsigned sel) {
+    const uint32_t m = __byte_perm(biased, 0x64646464u, sel);
+    __half2 h = *reinterpret_cast<const __half2 *>(&m);
+    const uint32_t k1152 = 0x64806480u;
+    h = __hsub2(h, *reinterpret_cast<const __half2 *>(&k1152));
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// As MmaConsumer, for int8 caches with per-row scales. The MMAs run in fp16
+// (int8 codes are exact in fp16; a bf16 query is converted to fp16 once, exact
+// for magnitudes in [2^-14, 65504]). Per 16-token stage, lane = 4 r + q:
+//   S^T = Kq Q^T: lane loads 16-byte chunks q + 4 j of token rows r and r + 8
+//     (16 dims each); word w of a chunk feeds one k-step (dims 4w .. 4w+3 as
+//     k columns 2q, 2q+1, 2q+8, 2q+9), so one load feeds four k-steps; Q's B
+//     fragment uses the same map. The score of token t is scaled by its K
+//     row scale after the MMA.
+//   O^T += Vq^T P'^T with P'_t = p_t * sv_t / svmax (sv_t the V row scale,
+//     svmax the stage's largest), so P' is in [0, 1] in fp16; the stage's
+//     product is added to O times svmax (fp32). Lane loads W = D/8 dims
+//     (W r .. W r + W - 1) of token rows 2q, 2q+1, 2q+8, 2q+9; byte permutes
+//     pair two tokens' codes of one dim before the fp16 conversion. m-tile
+//     mt row m holds dim W (m % 8) + mt + (m >= 8 ? W/2 : 0).
+// Tokens past the context have p = 0 and P' = 0 (their scales may hold
+// anything; int8 codes are always finite).
+template <typename TQ, int D, int G, typename S>
+struct MmaConsumerQ8 {
+    static constexpr int kJ = D / 64;    // 16-byte K chunks per lane per row
+    static constexpr int kMT = D / 16;   // PV m-tiles
+    static constexpr int kW = D / 8;     // V dims per lane
+    int q4, r;
+    uint32_t qb[kJ][8];
+    float o[kMT][4];
+    float m_run[2], l_lane[2];
+
+    static __device__ __forceinline__ int dim_of(int m, int mt) {
+        return kW * (m & 7) + mt + (m >= 8 ? kW / 2 : 0);
+    }
+
+    __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int, int lane) {
+        q4 = lane & 3;
+        r = lane >> 2;
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint4 u = make_uint4(0u, 0u, 0u, 0u);
+                if (r < G)
+                    u = *reinterpret_cast<const uint4 *>(static_cast<const TQ *>(p.query) + (head0 + r) * D +
+                                                         16 * (q4 + 4 * j) + 8 * h);
+                float f[8];
+                Elt<TQ>::unpack(u, f);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    __half2 v = __floats2half2_rn(f[2 * e], f[2 * e + 1]);
+                    qb[j][4 * h + e] = *reinterpret_cast<uint32_t *>(&v);
+                }
+            }
+        }
+#pragma unroll
+        for (int mt = 0; mt < kMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+        m_run[0] = m_run[1] = -INFINITY;
+        l_lane[0] = l_lane[1] = 0.f;
+    }
+
+    __device__ __forceinline__ void stage(const unsigned char *Kb, const unsigned char *Vb, int nvalid, int,
+                                          float scale_log2) {
+        const float *ksc = reinterpret_cast<const float *>(Kb + 2 * S::kTileBytes);
+        const float *vsc = ksc + S::kTS;
+        // ---- S^T = Kq Q^T
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+            const uint4 u0 = *reinterpret_cast<const uint4 *>(Kb + r * D + 16 * (q4 + 4 * j));
+            const uint4 u1 = *reinterpret_cast<const uint4 *>(Kb + (r + 8) * D + 16 * (q4 + 4 * j));
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const uint32_t x0 = word_of(u0, w) ^ 0x80808080u;
+                const uint32_t x1 = word_of(u1, w) ^ 0x80808080u;
+                mma_f16(sc, i8pair_to_h2(x0, 0x4140u), i8pair_to_h2(x1, 0x4140u), i8pair_to_h2(x0, 0x4342u),
+                        i8pair_to_h2(x1, 0x4342u), qb[j][2 * w], qb[j][2 * w + 1]);
+            }
+        }
+        // ---- online softmax per query head g = 2q + h over tokens r, r + 8
+        const bool v0 = r < nvalid;
+        const bool v1 = r + 8 < nvalid;
+        const float s0 = v0 ? ksc[r] * scale_log2 : 0.f;
+        const float s1 = v1 ? ksc[r + 8] * scale_log2 : 0.f;
+        float x[4];
+        x[0] = v0 ? sc[0] * s0 : -INFINITY;
+        x[1] = v0 ? sc[1] * s0 : -INFINITY;
+        x[2] = v1 ? sc[2] * s1 : -INFINITY;
+        x[3] = v1 ? sc[3] * s1 : -INFINITY;
+        float mx0 = fmaxf(x[0], x[2]);
+        float mx1 = fmaxf(x[1], x[3]);
+#pragma unroll
+        for (int mk = 4; mk < 32; mk <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, mk));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, mk));
+        }
+        const float mn0 = fmaxf(m_run[0], mx0);
+        const float mn1 = fmaxf(m_run[1], mx1);
+        const float al0 = (mn0 == -INFINITY) ? 1.f : fast_exp2(m_run[0] - mn0);
+        const float al1 = (mn1 == -INFINITY) ? 1.f : fast_exp2(m_run[1] - mn1);
+        m_run[0] = mn0;
+        m_run[1] = mn1;
+        float pr[4];
+        pr[0] = (x[0] == -INFINITY) ? 0.f : fast_exp2(x[0] - mn0);
+        pr[1] = (x[1] == -INFINITY) ? 0.f : fast_exp2(x[1] - mn1);
+        pr[2] = (x[2] == -INFINITY) ? 0.f : fast_exp2(x[2] - mn0);
+        pr[3] = (x[3] == -INFINITY) ? 0.f : fast_exp2(x[3] - mn1);
+        l_lane[0] = l_lane[0] * al0 + pr[0] + pr[2];
+        l_lane[1] = l_lane[1] * al1 + pr[1] + pr[3];
+        // ---- V scales: P' = p * sv / svmax
+        const float sv0 = v0 ? vsc[r] : 0.f;
+        const float sv1 = v1 ? vsc[r + 8] : 0.f;
+        float svmax = fmaxf(sv0, sv1);
+#pragma unroll
+        for (int mk = 4; mk < 32; mk <<= 1) svmax = fmaxf(svmax, __shfl_xor_sync(0xffffffffu, svmax, mk));
+        const float inv = svmax > 0.f ? 1.f / svmax : 0.f;
+        const float w0 = sv0 * inv, w1 = sv1 * inv;
+        const uint32_t bh0 = transpose8x8(Mma<__half>::pack(pr[0] * w0, pr[1] * w0));
+        const uint32_t bh1 = transpose8x8(Mma<__half>::pack(pr[2] * w1, pr[3] * w1));
+        // ---- O^T = O^T alpha + svmax (Vq^T P'^T)
+        uint32_t wa[kW / 4], wb[kW / 4], wc[kW / 4], wd[kW / 4];  // token rows 2q, 2q+1, 2q+8, 2q+9
+        const unsigned char *vcol = Vb + kW * r;
+        if constexpr (kW == 16) {
+            const uint4 a = *reinterpret_cast<const uint4 *>(vcol + (2 * q4) * D);
+            const uint4 b = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 1) * D);
+            const uint4 c = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 8) * D);
+            const uint4 d = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 9) * D);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                wa[w] = word_of(a, w);
+                wb[w] = word_of(b, w);
+                wc[w] = word_of(c, w);
+                wd[w] = word_of(d, w);
+            }
+        } else {
+            const uint2 a = *reinterpret_cast<const uint2 *>(vcol + (2 * q4) * D);
+            const uint2 b = *reinterpret_cast<const uint2 *>(vcol + (2 * q4 + 1) * D);
+            const uint2 c = *reinterpret_cast<const uint2 *>(vcol + (2 * q4 + 8) * D);
+            const uint2 d = *reinterpret_cast<const uint2 *>(vcol + (2 * q4 + 9) * D);
+            wa[0] = a.x; wa[1] = a.y;
+            wb[0] = b.x; wb[1] = b.y;
+            wc[0] = c.x; wc[1] = c.y;
+            wd[0] = d.x; wd[1] = d.y;
+        }
+        // pairs (token lo, token hi) of one dim e: lo tokens (2q, 2q+1) -> cols 2q, 2q+1; hi -> 2q+8, 2q+9
+        uint32_t plo[kW], phi[kW];
+#pragma unroll
+        for (int w = 0; w < kW / 4; ++w) {
+            const uint32_t l01 = __byte_perm(wa[w], wb[w], 0x5140u) ^ 0x80808080u;  // dims 4w, 4w+1
+            const uint32_t l23 = __byte_perm(wa[w], wb[w], 0x7362u) ^ 0x80808080u;  // dims 4w+2, 4w+3
+            const uint32_t h01 = __byte_perm(wc[w], wd[w], 0x5140u) ^ 0x80808080u;
+            const uint32_t h23 = __byte_perm(wc[w], wd[w], 0x7362u) ^ 0x80808080u;
+            plo[4 * w + 0] = i8pair_to_h2(l01, 0x4140u);
+            plo[4 * w + 1] = i8pair_to_h2(l01, 0x4342u);
+            plo[4 * w + 2] = i8pair_to_h2(l23, 0x4140u);
+            plo[4 * w + 3] = i8pair_to_h2(l23, 0x4342u);
+            phi[4 * w + 0] = i8pair_to_h2(h01, 0x4140u);
+            phi[4 * w + 1] = i8pair_to_h2(h01, 0x4342u);
+            phi[4 * w + 2] = i8pair_to_h2(h23, 0x4140u);
+            phi[4 * w + 3] = i8pair_to_h2(h23, 0x4342u);
+        }
+#pragma unroll
+        for (int mt = 0; mt < kMT; ++mt) {
+            float t[4] = {0.f, 0.f, 0.f, 0.f};
+            // row r: dim mt; row r + 8: dim kW/2 + mt (of this lane's W dims)
+            mma_f16(t, plo[mt], plo[kW / 2 + mt], phi[mt], phi[kW / 2 + mt], bh0, bh1);
+            o[mt][0] = fmaf(svmax, t[0], o[mt][0] * al0);
+            o[mt][1] = fmaf(svmax, t[1], o[mt][1] * al1);
+            o[mt][2] = fmaf(svmax, t[2], o[mt][2] * al0);
+            o[mt][3] = fmaf(svmax, t[3], o[mt][3] * al1);
+        }
+    }
+
+    __device__ __forceinline__ void store(float *mg, float *lg, float *ag, int warp, int) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int mk = 4; mk < 32; mk <<= 1) l_lane[h] += __shfl_xor_sync(0xffffffffu, l_lane[h], mk);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int g = 2 * q4 + h;
+            if (g < G) {
+                if (r == 0) {
+                    mg[warp * G + g] = m_run[h];
+                    lg[warp * G + g] = l_lane[h];
+                }
+                float *row = ag + ((size_t)warp * G + g) * S::kAgStride;
+#pragma unroll
+                for (int mt = 0; mt < kMT; ++mt) {
+                    row[dim_of(r, mt)] = o[mt][h];
+                    row[dim_of(r + 8, mt)] = o[mt][2 + h];
+                }
+            }
+        }
+    }
+};
+
 // -------------------------------------------------------------------- kernel
 
-template <typename T, int D, int BS, int G>
+// T: the cache's element type (int8_t: codes with per-row scales); TQ: the
+// query's type (T for 16- and 32-bit caches).
+template <typename T, int D, int BS, int G, typename TQ = T>
 __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShape<T, D, BS, G>::kMinBlocks)
     decode_kernel(const DecodeParams p) {
     using S = DecodeShape<T, D, BS, G>;
-    using Consumer = std::conditional_t<S::kUseMma, MmaConsumer<T, D, G, S>, FmaConsumer<T, D, G, S>>;
+    using Consumer = std::conditional_t<
+        S::kInt8, MmaConsumerQ8<TQ, D, G, S>,
+        std::conditional_t<S::kUseMma, MmaConsumer<T, D, G, S>, FmaConsumer<T, D, G, S>>>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *ring = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -536,6 +753,8 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     const size_t block_elems = (size_t)p.num_kv_heads * BS * D;
     const T *kc = static_cast<const T *>(p.k_cache) + (size_t)kvh * BS * D;
     const T *vc = static_cast<const T *>(p.v_cache) + (size_t)kvh * BS * D;
+    const float *ksc = S::kInt8 ? p.k_scale + (size_t)kvh * BS : nullptr;
+    const float *vsc = S::kInt8 ? p.v_scale + (size_t)kvh * BS : nullptr;
     const uint64_t pol = l2_evict_first_policy();
 
     // Block id of local stage m0 + lane (-1: none, or a bad entry).
@@ -569,6 +788,11 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
             mbar_arrive_expect_tx(full + buf, S::kStageBytes);
             bulk_load(dst, kc + src, S::kTileBytes, full + buf, pol);
             bulk_load(dst + S::kTileBytes, vc + src, S::kTileBytes, full + buf, pol);
+            if constexpr (S::kInt8) {  // the 16 rows' scales: 64 contiguous bytes each
+                const size_t ssrc = (size_t)id * p.num_kv_heads * BS + (size_t)(k % S::kSubs) * S::kTS;
+                bulk_load(dst + 2 * S::kTileBytes, ksc + ssrc, S::kScaleBytes, full + buf, pol);
+                bulk_load(dst + 2 * S::kTileBytes + S::kScaleBytes, vsc + ssrc, S::kScaleBytes, full + buf, pol);
+            }
         } else {
             bad[buf] = 1;
             mbar_arrive(full + buf);
@@ -737,11 +961,11 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
 
 // ------------------------------------------------------------------ launchers
 
-template <typename T, int D, int BS, int G>
+template <typename T, int D, int BS, int G, typename TQ = T>
 static cudaError_t launch_decode_t(const DecodeParams &p, int grid_x, int num_kv_heads, int num_seqs,
                                    cudaStream_t stream) {
     using S = DecodeShape<T, D, BS, G>;
-    auto kern = decode_kernel<T, D, BS, G>;
+    auto kern = decode_kernel<T, D, BS, G, TQ>;
     static unsigned int attr_done = 0;  // one bit per device
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), S::kSmemBytes, &attr_done);
     if (e != cudaSuccess) return e;
@@ -750,25 +974,25 @@ static cudaError_t launch_decode_t(const DecodeParams &p, int grid_x, int num_kv
     return cudaGetLastError();
 }
 
-template <typename T, int D, int BS>
+template <typename T, int D, int BS, typename TQ = T>
 static cudaError_t dispatch_group(const DecodeParams &p, int group, int grid_x, int num_kv_heads,
                                   int num_seqs, cudaStream_t stream) {
     switch (group) {
-        case 1: return launch_decode_t<T, D, BS, 1>(p, grid_x, num_kv_heads, num_seqs, stream);
-        case 2: return launch_decode_t<T, D, BS, 2>(p, grid_x, num_kv_heads, num_seqs, stream);
-        case 4: return launch_decode_t<T, D, BS, 4>(p, grid_x, num_kv_heads, num_seqs, stream);
-        case 8: return launch_decode_t<T, D, BS, 8>(p, grid_x, num_kv_heads, num_seqs, stream);
+        case 1: return launch_decode_t<T, D, BS, 1, TQ>(p, grid_x, num_kv_heads, num_seqs, stream);
+        case 2: return launch_decode_t<T, D, BS, 2, TQ>(p, grid_x, num_kv_heads, num_seqs, stream);
+        case 4: return launch_decode_t<T, D, BS, 4, TQ>(p, grid_x, num_kv_heads, num_seqs, stream);
+        case 8: return launch_decode_t<T, D, BS, 8, TQ>(p, grid_x, num_kv_heads, num_seqs, stream);
         default: return cudaErrorInvalidValue;
     }
 }
 
-template <typename T>
+template <typename T, typename TQ = T>
 static cudaError_t dispatch_shape(const DecodeParams &p, int head_dim, int block_size, int group,
                                   int grid_x, int num_kv_heads, int num_seqs, cudaStream_t stream) {
-    if (head_dim == 64 && block_size == 16) return dispatch_group<T, 64, 16>(p, group, grid_x, num_kv_heads, num_seqs, stream);
-    if (head_dim == 64 && block_size == 32) return dispatch_group<T, 64, 32>(p, group, grid_x, num_kv_heads, num_seqs, stream);
-    if (head_dim == 128 && block_size == 16) return dispatch_group<T, 128, 16>(p, group, grid_x, num_kv_heads, num_seqs, stream);
-    if (head_dim == 128 && block_size == 32) return dispatch_group<T, 128, 32>(p, group, grid_x, num_kv_heads, num_seqs, stream);
+    if (head_dim == 64 && block_size == 16) return dispatch_group<T, 64, 16, TQ>(p, group, grid_x, num_kv_heads, num_seqs, stream);
+    if (head_dim == 64 && block_size == 32) return dispatch_group<T, 64, 32, TQ>(p, group, grid_x, num_kv_heads, num_seqs, stream);
+    if (head_dim == 128 && block_size == 16) return dispatch_group<T, 128, 16, TQ>(p, group, grid_x, num_kv_heads, num_seqs, stream);
+    if (head_dim == 128 && block_size == 32) return dispatch_group<T, 128, 32, TQ>(p, group, grid_x, num_kv_heads, num_seqs, stream);
     return cudaErrorInvalidValue;
 }
 
@@ -781,6 +1005,15 @@ cudaError_t launch_decode(const DecodeParams &p, pa_dtype kv_dtype, int head_dim
         case PA_BF16: return dispatch_shape<__nv_bfloat16>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream);
     }
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_q8(const DecodeParams &p, pa_dtype q_dtype, int head_dim, int block_size, int group,
+                             int grid_x, int num_kv_heads, int num_seqs, cudaStream_t stream) {
+    switch (q_dtype) {
+        case PA_F16: return dispatch_shape<int8_t, __half>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream);
+        case PA_BF16: return dispatch_shape<int8_t, __nv_bfloat16>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_splitk_reduce(void *out, const float *ws_ml, const float *ws_acc,

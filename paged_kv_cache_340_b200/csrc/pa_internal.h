@@ -16,6 +16,8 @@ struct DecodeParams {
     const void *query;  // [num_seqs, num_heads, head_dim]
     const void *k_cache;
     const void *v_cache;
+    const float *k_scale;  // int8 caches: [num_blocks, num_kv_heads, block_size] per-row scales
+    const float *v_scale;
     const int32_t *block_tables;
     const int32_t *context_lens;
     const int32_t *seq_order;  // nullable: CTA row z serves sequence seq_order[z]
@@ -34,6 +36,17 @@ struct DecodeParams {
 cudaError_t launch_decode(const DecodeParams &p, pa_dtype kv_dtype, int head_dim, int block_size,
                           int group, int grid_x, int num_kv_heads, int num_seqs,
                           cudaStream_t stream);
+
+// int8 caches (codes plus per-row scales in p.k_scale / p.v_scale); q_dtype is
+// the query's type (PA_F16 or PA_BF16).
+cudaError_t launch_decode_q8(const DecodeParams &p, pa_dtype q_dtype, int head_dim, int block_size, int group,
+                             int grid_x, int num_kv_heads, int num_seqs, cudaStream_t stream);
+
+cudaError_t launch_reshape_and_cache_q8(const void *key, const void *value, pa_dtype src_dtype, int8_t *k_cache,
+                                        int8_t *v_cache, float *k_scale, float *v_scale,
+                                        const int32_t *slot_mapping, int num_tokens, int num_blocks,
+                                        int num_kv_heads, int head_dim, int block_size, unsigned int *err,
+                                        cudaStream_t stream);
 
 cudaError_t launch_splitk_reduce(void *out, const float *ws_ml, const float *ws_acc,
                                  const int32_t *context_lens, int num_seqs, int num_heads,

@@ -26,6 +26,9 @@ Workloads (shapes follow LLaMA-style decode layers):
                        head_dim 128, block 16; q/k/v ~ N(0,1); fp32 out
   chunked_prefill_gqa_bf16   16 sequences of 4096 tokens whose last 512 are new,
                        32 query / 8 kv heads, head_dim 128, block 16; fp32 out
+  llama7b_mha_int8     llama7b_mha_fp16's shapes and values with an int8 cache (the fp16
+                       values quantized at the slot write); fp16 query and out
+  gqa_int8             gqa_bf16's shapes and values with an int8 cache; bf16 query, fp32 out
   beam_search_fp16     32 prompts of U{256..1024} tokens x beam width 4 (128 beams),
                        32 heads, head_dim 128, block 16; every step each beam picks a
                        parent among its prompt's 4 beams (uniform) and writes one token;
@@ -39,7 +42,7 @@ from typing import Dict, Optional
 
 import torch
 
-DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16, "i8": torch.int8}
 
 
 @dataclass(frozen=True)
@@ -62,6 +65,7 @@ class Spec:
     v_uniform: bool = False
     partition_size: int = 0  # split-K partition (tokens) the workload is run with; 0 = unsplit
     q_len: int = 0  # prefill workloads: new query tokens per sequence (0 = decode)
+    q_dtype: str = ""  # query (and source K/V) type when it differs from the cache's (int8 caches)
     # parallel sampling (copy-on-write) workload
     num_prompts: int = 0
     branches: int = 0
@@ -79,6 +83,12 @@ class Spec:
     @property
     def torch_out_dtype(self) -> torch.dtype:
         return DTYPES[self.out_dtype]
+
+    @property
+    def torch_q_dtype(self) -> torch.dtype:
+        """The query's type; also the type of the K/V values before an int8
+        cache quantizes them."""
+        return DTYPES[self.q_dtype or self.kv_dtype]
 
 
 SPECS: Dict[str, Spec] = {
@@ -98,6 +108,11 @@ SPECS: Dict[str, Spec] = {
                                      ("fixed", (2048,) * 8), 1.0, q_len=2048),
     "chunked_prefill_gqa_bf16": Spec("chunked_prefill_gqa_bf16", 16, 32, 8, 128, 16, "bf16", "f32", 3406,
                                      ("fixed", (4096,) * 16), 1.0, q_len=512),
+    # int8 caches: the K/V values (fp16 / bf16) are quantized by the slot write
+    "llama7b_mha_int8": Spec("llama7b_mha_int8", 64, 32, 32, 128, 16, "i8", "f16", 3408,
+                             ("uniform", 256, 2048), 1.1, q_scale=0.5, kv_scale=0.5, q_dtype="f16"),
+    "gqa_int8": Spec("gqa_int8", 256, 32, 8, 128, 16, "i8", "f32", 3409,
+                     ("lognormal", 1024, 0.5, 128, 4096), 1.1, q_dtype="bf16"),
     # beam search: the beam step (fork, release, copy-on-write) on the device, then decode
     "beam_search_fp16": Spec("beam_search_fp16", 128, 32, 32, 128, 16, "f16", "f16", 3407,
                              ("uniform", 256, 1024), None, num_prompts=32, branches=4, max_divergent=512),
@@ -159,7 +174,7 @@ def make_decode_inputs(spec: Spec) -> dict:
     """
     assert spec.lengths[0] != "parallel"
     gen = torch.Generator().manual_seed(spec.seed)
-    dt = spec.torch_kv_dtype
+    dt = spec.torch_q_dtype  # int8 caches: the values before quantization
     ctx = context_lengths(spec, gen)
     needed = int(sum((int(c) + spec.block_size - 1) // spec.block_size for c in ctx.tolist()))
     nb = spec.pool_blocks if spec.pool_factor is None else int(math.ceil(spec.pool_factor * needed))
