@@ -13,12 +13,13 @@
 //     heads of the GQA group share every K/V tile, so each tile crosses HBM
 //     once;
 //   * the token range is cut into 16-token stages; stage k belongs to warp
-//     k % 4 and lives in shared-memory buffer k % 8 (two buffers per warp).
+//     k % 4 and lives in shared-memory buffer k % R, the ring of R = 8
+//     buffers (two per warp).
 //     The warp loads its own stages: lane 0 streams the stage's K and V tile
 //     (16 contiguous token rows of one kv head in this layout) with two
 //     one-dimensional bulk copies (cp.async.bulk, TMA engine) completing on
 //     the buffer's mbarrier, and right after consuming stage k it reloads the
-//     same buffer with stage k + 8. No other warp touches the buffer, so
+//     same buffer with stage k + R. No other warp touches the buffer, so
 //     there are no empty barriers and a parity wait can never alias. Table
 //     entries are read 32 stages ahead, one per lane;
 //   * 16-bit GQA groups (G >= 2) compute QK^T and PV with tensor-core MMAs
@@ -68,7 +69,11 @@ struct DecodeShape {
     static constexpr int kTileBytes = kTS * D * kElt;  // 16 token rows of one kv head, K or V
     static constexpr int kScaleBytes = kInt8 ? kTS * 4 : 0;  // int8: the 16 rows' fp32 scales, K or V
     static constexpr int kStageBytes = 2 * kTileBytes + 2 * kScaleBytes;
-    static constexpr int kStages = 8;                  // two buffers per warp
+    // Buffers per warp (a ring of kWarps * kBufPerWarp stages). int8 stages
+    // are half the bytes; measured, a deeper int8 ring did not help, five
+    // CTAs per SM did.
+    static constexpr int kBufPerWarp = 2;
+    static constexpr int kStages = kWarps * kBufPerWarp;
     static constexpr int kRowGroups = kUseMma ? kWarps : kWarps * kRows;
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kAgStride = kUseMma ? D + 1 : D;  // floats per merged accumulator row
@@ -77,9 +82,9 @@ struct DecodeShape {
     static constexpr int kSmemBytes = 128 + kDataBytes + kStages * 8 + kStages * 4;
     // Resident CTAs per SM the register budget is set for (a sub-partition
     // holds one warp of each CTA, so 3 CTAs leave 170 registers a thread).
-    static constexpr int kMinBlocks = (kUseMma || G <= 4) ? 3 : 2;
+    static constexpr int kMinBlocks = kInt8 ? 5 : ((kUseMma || G <= 4) ? 3 : 2);
 
-    static_assert(kStages == 2 * kWarps, "stage k: warp k % 4, buffer k % 8");
+    static_assert(kStages == kBufPerWarp * kWarps, "stage k: warp k % 4, buffer k % kStages");
     static_assert(BS % kTS == 0, "block size is a multiple of the stage");
     // the CUDA-core consumer's lane layout
     static_assert(kUseMma || (kLpt >= 1 && kLpt <= 32 && (32 % kLpt) == 0), "row width");
@@ -798,13 +803,10 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
             mbar_arrive(full + buf);
         }
     };
-    {
-        const int i0 = id_of(0);
-        const int i1 = id_of(1);
-        if (lane == 0) {
-            if (nmine > 0) issue(0, i0);
-            if (nmine > 1) issue(1, i1);
-        }
+#pragma unroll
+    for (int m = 0; m < S::kBufPerWarp; ++m) {
+        const int id = id_of(m);
+        if (lane == 0 && m < nmine) issue(m, id);
     }
 
     Consumer cons;
@@ -833,16 +835,16 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
             const unsigned char *Kb = ring + (size_t)buf * S::kStageBytes;
             cons.stage(Kb, Kb + S::kTileBytes, nvalid, lane, p.scale_log2);
         }
-        // Reload this buffer with this warp's stage m + 2.
-        const int idn = id_of(m + 2);
+        // Reload this buffer with this warp's stage m + kBufPerWarp.
+        const int idn = id_of(m + S::kBufPerWarp);
         __syncwarp();
-        if (lane == 0 && m + 2 < nmine) {
+        if (lane == 0 && m + S::kBufPerWarp < nmine) {
             fence_proxy_async_smem();
-            issue(m + 2, idn);
+            issue(m + S::kBufPerWarp, idn);
         }
     }
     if (!ok && lane == 0) {  // after a timeout: let every copy this warp started land
-        for (int m = waited; m < min(nmine, waited + 2); ++m) {
+        for (int m = waited; m < min(nmine, waited + S::kBufPerWarp); ++m) {
             const int k = warp + S::kWarps * m;
             if (!mbar_wait(full + (k % S::kStages), (k / S::kStages) & 1)) record_error(p.err, PA_DEVERR_TIMEOUT);
         }

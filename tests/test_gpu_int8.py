@@ -133,7 +133,7 @@ def test_decode_q8_16bit_output_and_ctx1(pa):
                         torch.from_numpy(c.ctx).cuda(), c.scale)
         torch.cuda.synchronize()
         assert_attention_close(out, c.ref(qdt), qdt, f"q8 {qdt} out")
-    # one token: the dequantized V row (fp32 product), whatever the query
+    # one token: the dequantized V row (one fp32 product), whatever the query
     out = torch.empty((4, 8, 128), device="cuda")
     pa.pa_decode_q8(out, c.q.half().cuda(), kq, vq, ks, vs, torch.from_numpy(c.tables).cuda(),
                     torch.from_numpy(c.ctx).cuda(), c.scale)
