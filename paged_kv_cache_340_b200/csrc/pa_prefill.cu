@@ -47,18 +47,23 @@ constexpr int kQHalf = kM * kHalfBytes; // 16 KB: rows x d 0-63 (or 64-127)
 constexpr int kKVHalf = kN * kHalfBytes;  // 8 KB
 constexpr int kQBytes = 2 * kQHalf;
 constexpr int kKVBytes = 2 * kKVHalf;   // one K or V tile
-constexpr int kPBytes = kM * kHalfBytes;  // 128 rows x 64 tokens
 constexpr int kSoftmaxWarps = 4;
 constexpr int kThreads = (kSoftmaxWarps + 1) * 32;
-constexpr int kTmemCols = 256;          // O: columns 0-127, S: 128-191
-constexpr int kOCol = 0;
-constexpr int kSCol = 128;
-// shared memory (every operand region 1024-byte aligned for the swizzle)
+// tensor memory (256 columns x 128 lanes, lane = query row): O, S, and P as
+// the A operand of O += P V (16-bit pairs per 32-bit column; bf16 also its
+// low part P - bf16(P))
+constexpr int kTmemCols = 256;
+constexpr int kOCol = 0;     // O: 128 fp32 columns
+constexpr int kSCol = 128;   // S: 64 fp32 columns
+constexpr int kPCol = 192;   // P: 32 columns of pairs
+constexpr int kPlCol = 224;  // bf16: P's low part
+// shared memory (every operand region 1024-byte aligned for the swizzle):
+// Q, and two stages each of K and V, each reloaded as soon as the product
+// that reads it has finished
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;   // one K tile: reloaded as soon as S = Q K^T is done
-constexpr int kOffV = kOffK + kKVBytes;  // one V tile: reloaded as soon as O += P V is done
-constexpr int kOffP = kOffV + kKVBytes;
-constexpr int kOffBar = kOffP + 2 * kPBytes;  // P (and, for bf16, its low part)
+constexpr int kOffK = kOffQ + kQBytes;         // K stages 0, 1
+constexpr int kOffV = kOffK + 2 * kKVBytes;    // V stages 0, 1
+constexpr int kOffBar = kOffV + 2 * kKVBytes;
 constexpr int kSmemBytes = 1024 + kOffBar + 16 * 8;  // ~97 KB: two CTAs per SM
 // The running max is raised only when it grows by more than this (log2
 // units): probabilities then stay below 2^8 and O is rarely rescaled.
@@ -164,6 +169,44 @@ template <> struct Pack16<__half> {
 
 // ----------------------------------------------------------------- kernel
 
+// A operand in tensor memory: O += A B with A read from TMEM columns.
+__device__ __forceinline__ void umma_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 consecutive outputs of one row, as 16-byte stores.
+__device__ __forceinline__ void store_row32(void *base, size_t idx, const float (&v)[32], pa_dtype dt) {
+    if (dt == PA_F32) {
+        float4 *d = reinterpret_cast<float4 *>(static_cast<float *>(base) + idx);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) d[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+    } else if (dt == PA_BF16) {
+        uint4 *d = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(base) + idx);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) w[i] = Pack16<__nv_bfloat16>::pack(v[8 * e + 2 * i], v[8 * e + 2 * i + 1]);
+            d[e] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    } else {
+        uint4 *d = reinterpret_cast<uint4 *>(static_cast<__half *>(base) + idx);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) w[i] = Pack16<__half>::pack(v[8 * e + 2 * i], v[8 * e + 2 * i + 1]);
+            d[e] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
 template <typename T, int G>
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -177,19 +220,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     unsigned char *Qs = sm + kOffQ;
-    unsigned char *Ks = sm + kOffK;
+    unsigned char *Ks = sm + kOffK;  // stage b at Ks + b * kKVBytes
     unsigned char *Vs = sm + kOffV;
-    unsigned char *Ps = sm + kOffP;
-    unsigned char *Pl = Ps + kPBytes;  // bf16 only: P - bf16(P)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBar);
     uint64_t *q_full = bars + 0;
-    uint64_t *k_full = bars + 1;
-    uint64_t *v_full = bars + 2;
-    uint64_t *s_full = bars + 3;
-    uint64_t *p_full = bars + 4;
-    uint64_t *o_done = bars + 5;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
-    int *abort_flag = reinterpret_cast<int *>(bars + 7);
+    uint64_t *k_full = bars + 1;  // [2]
+    uint64_t *v_full = bars + 3;  // [2]
+    uint64_t *s_full = bars + 5;
+    uint64_t *p_full = bars + 6;
+    uint64_t *o_done = bars + 7;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
+    int *abort_flag = reinterpret_cast<int *>(bars + 9);
 
     const int qt = blockIdx.x;
     const int kvh = blockIdx.y;
@@ -214,7 +255,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         mbar_init(k_full, 1);
+        mbar_init(k_full + 1, 1);
         mbar_init(v_full, 1);
+        mbar_init(v_full + 1, 1);
         mbar_init(s_full, 1);
         mbar_init(p_full, kSoftmaxWarps * 32);
         mbar_init(o_done, 1);
@@ -235,6 +278,11 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (warp == kSoftmaxWarps) {
         // ===================================================== control thread
+        // Tile j uses K/V stage j & 1 (its use j >> 1 of that stage). Order
+        // per tile: S_j = Q K_j^T; once PV_{j-1} is done, V_{j+1} goes into
+        // the stage PV_{j-1} read; once the softmax of tile j is done (S_j
+        // read, P_j written), K_{j+2} goes into K_j's stage; then
+        // O += P_j V_j.
         if (lane == 0) {
             const int32_t *trow = p.block_tables + (size_t)s * p.max_blocks_per_seq;
             const int nblk = (ctx + p.block_size - 1) / p.block_size;
@@ -264,17 +312,22 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_arrive_expect_tx(q_full, kQBytes);
             tma_load_3d(Qs, &tmap_q, 0, kvh * G, q0 + tok0, q_full);
             tma_load_3d(Qs + kQHalf, &tmap_q, 64, kvh * G, q0 + tok0, q_full);
-            load_tile(&tmap_k, Ks, k_full, 0);
-            load_tile(&tmap_v, Vs, v_full, 0);
-            const uint32_t qa = smem_addr(Qs), ka = smem_addr(Ks), va = smem_addr(Vs);
-            const uint32_t pa_ = smem_addr(Ps), pl_ = smem_addr(Pl);
+            const int pre = min(2, ntiles);
+            for (int j = 0; j < pre; ++j) {
+                load_tile(&tmap_k, Ks + j * kKVBytes, k_full + j, j);
+                load_tile(&tmap_v, Vs + j * kKVBytes, v_full + j, j);
+            }
+            const uint32_t qa = smem_addr(Qs);
             bool ok = true;
-            int k_loaded = 1, k_waited = 0, v_loaded = 1, v_waited = 0;
+            // copies started / waited per stage, for the drain after an abort
+            int k_started = pre, k_waited = 0, v_started = pre, v_waited = 0;
             for (int j = 0; j < ntiles && ok; ++j) {
-                const int par = j & 1;
-                if (!mbar_wait(k_full, par) || (j == 0 && !mbar_wait(q_full, 0))) { ok = false; break; }
+                const int b = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                if (!mbar_wait(k_full + b, ph) || (j == 0 && !mbar_wait(q_full, 0))) { ok = false; break; }
                 k_waited = j + 1;
                 tc_fence_after();
+                const uint32_t ka = smem_addr(Ks + b * kKVBytes);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
                     const uint32_t off = (kk & 3) * 32;
@@ -282,34 +335,34 @@ __global__ void __launch_bounds__(kThreads, 2)
                          sw128_desc(ka + (kk >> 2) * kKVHalf + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(s_full);
-                if (j + 1 < ntiles) {  // S done: the K buffer takes the next tile
-                    if (!mbar_wait(s_full, par)) { ok = false; break; }
-                    load_tile(&tmap_k, Ks, k_full, j + 1);
-                    k_loaded = j + 2;
+                if (j >= 1 && j + 1 < ntiles) {  // PV_{j-1} done: its V stage takes V_{j+1}
+                    if (!mbar_wait(o_done, (j - 1) & 1)) { ok = false; break; }
+                    load_tile(&tmap_v, Vs + ((j + 1) & 1) * kKVBytes, v_full + ((j + 1) & 1), j + 1);
+                    ++v_started;
                 }
-                if (!mbar_wait(p_full, par) || !mbar_wait(v_full, par)) { ok = false; break; }
+                if (!mbar_wait(p_full, j & 1)) { ok = false; break; }
+                if (j + 2 < ntiles) {  // S_j read and P_j written: K_j's stage takes K_{j+2}
+                    load_tile(&tmap_k, Ks + b * kKVBytes, k_full + b, j + 2);
+                    ++k_started;
+                }
+                if (!mbar_wait(v_full + b, ph)) { ok = false; break; }
                 v_waited = j + 1;
                 tc_fence_after();
+                const uint32_t va = smem_addr(Vs + b * kKVBytes);
 #pragma unroll
                 for (int kk = 0; kk < kN / 16; ++kk) {
                     const uint64_t vdesc = sw128_desc(va + kk * 16 * kHalfBytes, kKVHalf, 1024);
-                    umma(tmem + kOCol, sw128_desc(pa_ + kk * 32, 16, 1024), vdesc, kIdescPV,
-                         (j > 0 || kk > 0) ? 1u : 0u);
-                    if constexpr (kBf16) umma(tmem + kOCol, sw128_desc(pl_ + kk * 32, 16, 1024), vdesc, kIdescPV, 1u);
+                    umma_ta(tmem + kOCol, tmem + kPCol + kk * 8, vdesc, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                    if constexpr (kBf16) umma_ta(tmem + kOCol, tmem + kPlCol + kk * 8, vdesc, kIdescPV, 1u);
                 }
                 umma_commit(o_done);
-                if (j + 1 < ntiles) {  // O += P V done: the V buffer takes the next tile
-                    if (!mbar_wait(o_done, par)) { ok = false; break; }
-                    load_tile(&tmap_v, Vs, v_full, j + 1);
-                    v_loaded = j + 2;
-                }
             }
             if (!ok) {
                 record_error(p.err, PA_DEVERR_TIMEOUT);
                 *abort_flag = 1;
                 // let the copies this thread started land before the CTA leaves
-                for (int j = k_waited; j < k_loaded; ++j) mbar_wait(k_full, j & 1);
-                for (int j = v_waited; j < v_loaded; ++j) mbar_wait(v_full, j & 1);
+                for (int j = k_waited; j < k_started; ++j) mbar_wait(k_full + (j & 1), (j >> 1) & 1);
+                for (int j = v_waited; j < v_started; ++j) mbar_wait(v_full + (j & 1), (j >> 1) & 1);
                 mbar_wait(q_full, 0);
                 // release the softmax warps from their waits
                 mbar_arrive(s_full);
@@ -324,6 +377,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const bool valid = r < rows_valid;
         const int pos = valid ? pos0 + tok : -1;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const float sl2 = p.scale_log2;
         float m_run = -INFINITY, l_run = 0.f;
         for (int j = 0; j < ntiles; ++j) {
             if (!mbar_wait(s_full, j & 1) || *(volatile int *)abort_flag) break;
@@ -335,11 +389,21 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int kv0 = j * kN;
             float x[kN];
             float mx = -INFINITY;
+            const bool full = kv0 + kN - 1 <= pos;  // no position of this tile is masked for this row
+            if (full) {
 #pragma unroll
-            for (int c = 0; c < kN; ++c) {
-                const float sv = __uint_as_float(sr[c >> 5][c & 31]);
-                x[c] = (kv0 + c <= pos) ? sv * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, x[c]);
+                for (int c = 0; c < kN; ++c) {
+                    x[c] = __uint_as_float(sr[c >> 5][c & 31]);
+                    mx = fmaxf(mx, x[c]);
+                }
+                mx *= sl2;
+            } else {
+#pragma unroll
+                for (int c = 0; c < kN; ++c) {
+                    x[c] = (kv0 + c <= pos) ? __uint_as_float(sr[c >> 5][c & 31]) : -INFINITY;
+                    mx = fmaxf(mx, x[c]);
+                }
+                mx *= sl2;  // -inf stays -inf (the scale is positive)
             }
             // raise the running max only when it grows by more than the threshold
             const bool raise = fmaxf(m_run, mx) - m_run > kRescaleThreshold;  // also the first finite max
@@ -347,14 +411,33 @@ __global__ void __launch_bounds__(kThreads, 2)
             const float alpha = raise ? fast_exp2(m_run - mn) : 1.f;  // 0 when m_run was -inf
             m_run = mn;
             float psum = 0.f;
+            if (full) {
 #pragma unroll
-            for (int c = 0; c < kN; ++c) {
-                x[c] = (x[c] == -INFINITY) ? 0.f : fast_exp2(x[c] - mn);
-                psum += x[c];
+                for (int c = 0; c < kN; ++c) {
+                    x[c] = fast_exp2(fmaf(x[c], sl2, -mn));
+                    psum += x[c];
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < kN; ++c) {
+                    x[c] = (x[c] == -INFINITY) ? 0.f : fast_exp2(fmaf(x[c], sl2, -mn));
+                    psum += x[c];
+                }
             }
             l_run = l_run * alpha + psum;
+            // P as 16-bit pairs (bf16 also its low part P - bf16(P), for ~2^-17
+            // relative error through a second P V pass)
+            uint32_t ph_[32], pl_[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                ph_[c] = Pack16<T>::pack(x[2 * c], x[2 * c + 1]);
+                if constexpr (kBf16) {
+                    const float hi0 = __uint_as_float(ph_[c] << 16), hi1 = __uint_as_float(ph_[c] & 0xffff0000u);
+                    pl_[c] = Pack16<T>::pack(x[2 * c] - hi0, x[2 * c + 1] - hi1);
+                }
+            }
             if (j > 0) {
-                // O and P of tile j-1 are done with: rescale O, reuse P
+                // O += P_{j-1} V_{j-1} done: O may be rescaled and P overwritten
                 if (!mbar_wait(o_done, (j - 1) & 1) || *(volatile int *)abort_flag) break;
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -367,36 +450,17 @@ __global__ void __launch_bounds__(kThreads, 2)
                         for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
                         tmem_st32(tmem + lane_base + kOCol + ch * 32, o);
                     }
-                    tmem_wait_st();
                 }
             }
-            // this row of P: 64 probabilities as 16-bit pairs, 8 swizzled 16-byte chunks.
-            // bf16 keeps 8 mantissa bits, so P also goes in as its low part
-            // P - bf16(P) (a second P V pass), for ~2^-17 relative error.
-            unsigned char *prow = Ps + r * kHalfBytes;
-            unsigned char *plow = Pl + r * kHalfBytes;
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) w[e] = Pack16<T>::pack(x[8 * ch + 2 * e], x[8 * ch + 2 * e + 1]);
-                *reinterpret_cast<uint4 *>(prow + ((ch ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-                if constexpr (kBf16) {
-                    uint32_t lw[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float hi0 = __uint_as_float(w[e] << 16), hi1 = __uint_as_float(w[e] & 0xffff0000u);
-                        lw[e] = Pack16<T>::pack(x[8 * ch + 2 * e] - hi0, x[8 * ch + 2 * e + 1] - hi1);
-                    }
-                    *reinterpret_cast<uint4 *>(plow + ((ch ^ (r & 7)) << 4)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-                }
-            }
+            tmem_st32(tmem + lane_base + kPCol, ph_);
+            if constexpr (kBf16) tmem_st32(tmem + lane_base + kPlCol, pl_);
+            tmem_wait_st();
             // V rows past the context: zero (both halves) before P V reads them
             const int zrow = max(0, ctx - kv0);
             if (zrow < kN) {
                 // V_j must have landed before its tail rows are overwritten
-                if (!mbar_wait(v_full, j & 1) || *(volatile int *)abort_flag) break;
-                unsigned char *vt = Vs;
+                if (!mbar_wait(v_full + (j & 1), (j >> 1) & 1) || *(volatile int *)abort_flag) break;
+                unsigned char *vt = Vs + (j & 1) * kKVBytes;
                 const int nvec = (kN - zrow) * 2 * (kHalfBytes / 16);
                 for (int i = r; i < nvec; i += kSoftmaxWarps * 32) {
                     const int row = zrow + i / 16;
@@ -405,8 +469,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                     *reinterpret_cast<uint4 *>(vt + h * kKVHalf + row * kHalfBytes + c * 16) =
                         make_uint4(0u, 0u, 0u, 0u);
                 }
+                fence_proxy_async_smem();
             }
-            fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(p_full);
         }
@@ -424,8 +488,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tmem_ld32(tmem + lane_base + kOCol + ch * 32, o);
                 tmem_wait_ld();
                 if (valid) {
+                    float v[32];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) store_out(p.out, orow + ch * 32 + e, __uint_as_float(o[e]) * inv, p.out_dtype);
+                    for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * inv;
+                    store_row32(p.out, orow + ch * 32, v, p.out_dtype);
                 }
             }
         }
