@@ -48,23 +48,24 @@ constexpr int kKVHalf = kN * kHalfBytes;  // 8 KB
 constexpr int kQBytes = 2 * kQHalf;
 constexpr int kKVBytes = 2 * kKVHalf;   // one K or V tile
 constexpr int kSoftmaxWarps = 4;
-constexpr int kThreads = (kSoftmaxWarps + 1) * 32;
-// tensor memory (256 columns x 128 lanes, lane = query row): O, S, and P as
-// the A operand of O += P V (16-bit pairs per 32-bit column; bf16 also its
-// low part P - bf16(P))
+constexpr int kMmaWarp = kSoftmaxWarps;       // warp 4: issues the tensor-core MMAs
+constexpr int kLoadWarp = kSoftmaxWarps + 1;  // warp 5: table lookups and TMA copies
+constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
+// tensor memory (256 columns x 128 lanes, lane = query row): O and two S
+// buffers. The softmax of tile j writes P_j (16-bit pairs; bf16 also its low
+// part P - bf16(P)) over its own S_j, and O += P_j V_j reads it from there:
+// S_{j+1} is computed while the softmax of tile j runs.
 constexpr int kTmemCols = 256;
-constexpr int kOCol = 0;     // O: 128 fp32 columns
-constexpr int kSCol = 128;   // S: 64 fp32 columns
-constexpr int kPCol = 192;   // P: 32 columns of pairs
-constexpr int kPlCol = 224;  // bf16: P's low part
+constexpr int kOCol = 0;      // O: 128 fp32 columns
+constexpr int kSCol = 128;    // S buffers 0, 1: 64 fp32 columns each
+constexpr int kPlOff = 32;    // within an S buffer: P at +0, P's low part at +32
 // shared memory (every operand region 1024-byte aligned for the swizzle):
-// Q, and two stages each of K and V, each reloaded as soon as the product
-// that reads it has finished
+// Q, and two stages each of K and V
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQBytes;         // K stages 0, 1
 constexpr int kOffV = kOffK + 2 * kKVBytes;    // V stages 0, 1
 constexpr int kOffBar = kOffV + 2 * kKVBytes;
-constexpr int kSmemBytes = 1024 + kOffBar + 16 * 8;  // ~97 KB: two CTAs per SM
+constexpr int kSmemBytes = 1024 + kOffBar + 24 * 8;  // ~97 KB: two CTAs per SM
 // The running max is raised only when it grows by more than this (log2
 // units): probabilities then stay below 2^8 and O is rarely rescaled.
 constexpr float kRescaleThreshold = 8.f;
@@ -224,13 +225,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     unsigned char *Vs = sm + kOffV;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBar);
     uint64_t *q_full = bars + 0;
-    uint64_t *k_full = bars + 1;  // [2]
-    uint64_t *v_full = bars + 3;  // [2]
-    uint64_t *s_full = bars + 5;
-    uint64_t *p_full = bars + 6;
-    uint64_t *o_done = bars + 7;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
-    int *abort_flag = reinterpret_cast<int *>(bars + 9);
+    uint64_t *k_full = bars + 1;    // [2] stage loaded
+    uint64_t *v_full = bars + 3;    // [2]
+    uint64_t *k_empty = bars + 5;   // [2] S that read the stage is done
+    uint64_t *v_empty = bars + 7;   // [2] PV that read the stage is done
+    uint64_t *s_full = bars + 9;    // [2] S buffer computed
+    uint64_t *p_full = bars + 11;   // softmax of the tile done (P written)
+    uint64_t *o_done = bars + 12;   // PV of the tile done
+    uint64_t *mma_idle = bars + 13; // every MMA issued has finished (end of kernel)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
+    int *abort_flag = reinterpret_cast<int *>(bars + 15);
 
     const int qt = blockIdx.x;
     const int kvh = blockIdx.y;
@@ -254,13 +258,16 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        mbar_init(k_full, 1);
-        mbar_init(k_full + 1, 1);
-        mbar_init(v_full, 1);
-        mbar_init(v_full + 1, 1);
-        mbar_init(s_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(k_full + i, 1);
+            mbar_init(v_full + i, 1);
+            mbar_init(k_empty + i, 1);
+            mbar_init(v_empty + i, 1);
+            mbar_init(s_full + i, 1);
+        }
         mbar_init(p_full, kSoftmaxWarps * 32);
         mbar_init(o_done, 1);
+        mbar_init(mma_idle, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -276,100 +283,144 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kSoftmaxWarps) {
-        // ===================================================== control thread
-        // Tile j uses K/V stage j & 1 (its use j >> 1 of that stage). Order
-        // per tile: S_j = Q K_j^T; once PV_{j-1} is done, V_{j+1} goes into
-        // the stage PV_{j-1} read; once the softmax of tile j is done (S_j
-        // read, P_j written), K_{j+2} goes into K_j's stage; then
-        // O += P_j V_j.
+    if (warp == kLoadWarp) {
+        // ========================================================= load warp
+        // Tile j goes into K/V stage j & 1 (its use j >> 1 of the stage); a
+        // stage is refilled once the S (K) or PV (V) product that read it is
+        // done. Block ids of 32 16-token groups are looked up at a time, one
+        // per lane.
+        const int32_t *trow = p.block_tables + (size_t)s * p.max_blocks_per_seq;
+        const int nblk = (ctx + p.block_size - 1) / p.block_size;
+        // Pool row of group g (16 tokens from g * 16), past the pool's end when
+        // the sequence has no such block (the copy then reads zeros).
+        auto rows_from = [&](int g0) -> int {
+            const int g = g0 + lane;
+            const int tok = g * 16;
+            const int lb = tok / p.block_size;
+            long long row = p.kv_rows;
+            if (lb < nblk) {
+                const int id = __ldg(trow + lb);
+                if (id >= 0 && id < p.num_blocks)
+                    row = ((long long)id * p.num_kv_heads + kvh) * p.block_size + (tok % p.block_size);
+                else
+                    record_error(p.err, PA_DEVERR_BLOCK_ID);
+            }
+            return (int)row;
+        };
         if (lane == 0) {
-            const int32_t *trow = p.block_tables + (size_t)s * p.max_blocks_per_seq;
-            const int nblk = (ctx + p.block_size - 1) / p.block_size;
-            // Physical row of the 16-token group starting at token `tok` (past the
-            // pool's end when the sequence has no such block: the copy reads zeros).
-            auto group_row = [&](int tok) -> int {
-                const int lb = tok / p.block_size;
-                long long row = p.kv_rows;
-                if (lb < nblk) {
-                    const int id = __ldg(trow + lb);
-                    if (id >= 0 && id < p.num_blocks)
-                        row = ((long long)id * p.num_kv_heads + kvh) * p.block_size + (tok % p.block_size);
-                    else
-                        record_error(p.err, PA_DEVERR_BLOCK_ID);
-                }
-                return (int)row;
-            };
-            auto load_tile = [&](const CUtensorMap *map, unsigned char *dst, uint64_t *bar, int j) {
-                mbar_arrive_expect_tx(bar, kKVBytes);
-#pragma unroll
-                for (int g = 0; g < kN / 16; ++g) {
-                    const int row = group_row(j * kN + g * 16);
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) tma_load_2d(dst + h * kKVHalf + g * 16 * kHalfBytes, map, h * 64, row, bar);
-                }
-            };
             mbar_arrive_expect_tx(q_full, kQBytes);
             tma_load_3d(Qs, &tmap_q, 0, kvh * G, q0 + tok0, q_full);
             tma_load_3d(Qs + kQHalf, &tmap_q, 64, kvh * G, q0 + tok0, q_full);
-            const int pre = min(2, ntiles);
-            for (int j = 0; j < pre; ++j) {
-                load_tile(&tmap_k, Ks + j * kKVBytes, k_full + j, j);
-                load_tile(&tmap_v, Vs + j * kKVBytes, v_full + j, j);
+        }
+        constexpr int kGroups = kN / 16;  // 16-token groups per tile
+        int rows = rows_from(0);
+        int k_issued = 0, v_issued = 0;
+        bool ok = true;
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int b = j & 1;
+            const int g0 = j * kGroups;
+            if (g0 % 32 == 0 && j > 0) rows = rows_from(g0);
+            int r4[kGroups];
+#pragma unroll
+            for (int g = 0; g < kGroups; ++g) r4[g] = __shfl_sync(0xffffffffu, rows, (g0 + g) % 32);
+            for (int kv = 0; kv < 2; ++kv) {
+                uint64_t *empty = (kv == 0 ? k_empty : v_empty) + b;
+                if (j >= 2) {  // every lane waits; the outcome is made warp-uniform
+                    const bool got = mbar_wait(empty, ((j >> 1) - 1) & 1) && !*(volatile int *)abort_flag;
+                    if (!__all_sync(0xffffffffu, got)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (lane == 0) {
+                    uint64_t *full = (kv == 0 ? k_full : v_full) + b;
+                    unsigned char *dst = (kv == 0 ? Ks : Vs) + b * kKVBytes;
+                    const CUtensorMap *map = kv == 0 ? &tmap_k : &tmap_v;
+                    mbar_arrive_expect_tx(full, kKVBytes);
+#pragma unroll
+                    for (int g = 0; g < kGroups; ++g)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_2d(dst + h * kKVHalf + g * 16 * kHalfBytes, map, h * 64, r4[g], full);
+                }
+                if (kv == 0) ++k_issued; else ++v_issued;
             }
+        }
+        if (!ok) {
+            if (lane == 0) {
+                record_error(p.err, PA_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+        }
+        // let the copies this warp started land before the CTA leaves
+        // (normally the MMA warp has consumed them all: these waits return at once)
+        if (lane == 0) {
+            mbar_wait(q_full, 0);
+            for (int j = max(0, k_issued - 2); j < k_issued; ++j) mbar_wait(k_full + (j & 1), (j >> 1) & 1);
+            for (int j = max(0, v_issued - 2); j < v_issued; ++j) mbar_wait(v_full + (j & 1), (j >> 1) & 1);
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ========================================================== MMA warp
+        // S_0, S_1; then per tile j: (softmax j done) O += P_j V_j; (that
+        // product done, so P_j's buffer is free) S_{j+2} into the same buffer.
+        if (lane == 0) {
             const uint32_t qa = smem_addr(Qs);
-            bool ok = true;
-            // copies started / waited per stage, for the drain after an abort
-            int k_started = pre, k_waited = 0, v_started = pre, v_waited = 0;
-            for (int j = 0; j < ntiles && ok; ++j) {
+            bool ok = mbar_wait(q_full, 0);
+            bool issued = false;
+            auto issue_s = [&](int j) -> bool {
                 const int b = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
-                if (!mbar_wait(k_full + b, ph) || (j == 0 && !mbar_wait(q_full, 0))) { ok = false; break; }
-                k_waited = j + 1;
+                if (!mbar_wait(k_full + b, (j >> 1) & 1) || *(volatile int *)abort_flag) return false;
                 tc_fence_after();
                 const uint32_t ka = smem_addr(Ks + b * kKVBytes);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
                     const uint32_t off = (kk & 3) * 32;
-                    umma(tmem + kSCol, sw128_desc(qa + (kk >> 2) * kQHalf + off, 16, 1024),
+                    umma(tmem + kSCol + b * kN, sw128_desc(qa + (kk >> 2) * kQHalf + off, 16, 1024),
                          sw128_desc(ka + (kk >> 2) * kKVHalf + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(s_full);
-                if (j >= 1 && j + 1 < ntiles) {  // PV_{j-1} done: its V stage takes V_{j+1}
-                    if (!mbar_wait(o_done, (j - 1) & 1)) { ok = false; break; }
-                    load_tile(&tmap_v, Vs + ((j + 1) & 1) * kKVBytes, v_full + ((j + 1) & 1), j + 1);
-                    ++v_started;
+                umma_commit(s_full + b);
+                umma_commit(k_empty + b);
+                issued = true;
+                return true;
+            };
+            for (int j = 0; ok && j < min(2, ntiles); ++j) ok = issue_s(j);
+            for (int j = 0; ok && j < ntiles; ++j) {
+                const int b = j & 1;
+                if (!mbar_wait(p_full, j & 1) || !mbar_wait(v_full + b, (j >> 1) & 1) ||
+                    *(volatile int *)abort_flag) {
+                    ok = false;
+                    break;
                 }
-                if (!mbar_wait(p_full, j & 1)) { ok = false; break; }
-                if (j + 2 < ntiles) {  // S_j read and P_j written: K_j's stage takes K_{j+2}
-                    load_tile(&tmap_k, Ks + b * kKVBytes, k_full + b, j + 2);
-                    ++k_started;
-                }
-                if (!mbar_wait(v_full + b, ph)) { ok = false; break; }
-                v_waited = j + 1;
                 tc_fence_after();
                 const uint32_t va = smem_addr(Vs + b * kKVBytes);
+                const uint32_t pcol = tmem + kSCol + b * kN;
 #pragma unroll
                 for (int kk = 0; kk < kN / 16; ++kk) {
                     const uint64_t vdesc = sw128_desc(va + kk * 16 * kHalfBytes, kKVHalf, 1024);
-                    umma_ta(tmem + kOCol, tmem + kPCol + kk * 8, vdesc, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-                    if constexpr (kBf16) umma_ta(tmem + kOCol, tmem + kPlCol + kk * 8, vdesc, kIdescPV, 1u);
+                    umma_ta(tmem + kOCol, pcol + kk * 8, vdesc, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                    if constexpr (kBf16) umma_ta(tmem + kOCol, pcol + kPlOff + kk * 8, vdesc, kIdescPV, 1u);
                 }
                 umma_commit(o_done);
+                umma_commit(v_empty + b);
+                if (j + 2 < ntiles) {
+                    if (!mbar_wait(o_done, j & 1)) { ok = false; break; }
+                    ok = issue_s(j + 2);
+                }
             }
             if (!ok) {
                 record_error(p.err, PA_DEVERR_TIMEOUT);
                 *abort_flag = 1;
-                // let the copies this thread started land before the CTA leaves
-                for (int j = k_waited; j < k_started; ++j) mbar_wait(k_full + (j & 1), (j >> 1) & 1);
-                for (int j = v_waited; j < v_started; ++j) mbar_wait(v_full + (j & 1), (j >> 1) & 1);
-                mbar_wait(q_full, 0);
-                // release the softmax warps from their waits
-                mbar_arrive(s_full);
+                mbar_arrive(s_full);      // release the softmax warps from their waits
+                mbar_arrive(s_full + 1);
                 mbar_arrive(o_done);
             }
+            if (issued) {  // tensor memory is freed below: every MMA must have finished
+                umma_commit(mma_idle);
+                if (!mbar_wait(mma_idle, 0)) record_error(p.err, PA_DEVERR_TIMEOUT);
+            }
         }
-        __syncwarp();  // reconverge the control warp before the block-wide barrier
+        __syncwarp();
     } else {
         // ======================================================= softmax warps
         const int r = threadIdx.x;  // row = tensor-memory lane
@@ -380,11 +431,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         const float sl2 = p.scale_log2;
         float m_run = -INFINITY, l_run = 0.f;
         for (int j = 0; j < ntiles; ++j) {
-            if (!mbar_wait(s_full, j & 1) || *(volatile int *)abort_flag) break;
+            const int b = j & 1;
+            if (!mbar_wait(s_full + b, (j >> 1) & 1) || *(volatile int *)abort_flag) break;
             tc_fence_after();
+            const uint32_t sbuf = tmem + lane_base + kSCol + b * kN;
             uint32_t sr[2][32];
-            tmem_ld32(tmem + lane_base + kSCol, sr[0]);
-            tmem_ld32(tmem + lane_base + kSCol + 32, sr[1]);
+            tmem_ld32(sbuf, sr[0]);
+            tmem_ld32(sbuf + 32, sr[1]);
             tmem_wait_ld();
             const int kv0 = j * kN;
             float x[kN];
@@ -396,15 +449,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                     x[c] = __uint_as_float(sr[c >> 5][c & 31]);
                     mx = fmaxf(mx, x[c]);
                 }
-                mx *= sl2;
             } else {
 #pragma unroll
                 for (int c = 0; c < kN; ++c) {
                     x[c] = (kv0 + c <= pos) ? __uint_as_float(sr[c >> 5][c & 31]) : -INFINITY;
                     mx = fmaxf(mx, x[c]);
                 }
-                mx *= sl2;  // -inf stays -inf (the scale is positive)
             }
+            mx *= sl2;  // -inf stays -inf (the scale is positive)
             // raise the running max only when it grows by more than the threshold
             const bool raise = fmaxf(m_run, mx) - m_run > kRescaleThreshold;  // also the first finite max
             const float mn = raise ? fmaxf(m_run, mx) : m_run;
@@ -437,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
             }
             if (j > 0) {
-                // O += P_{j-1} V_{j-1} done: O may be rescaled and P overwritten
+                // O += P_{j-1} V_{j-1} done (waited every tile, so the phases stay in step): O may be rescaled
                 if (!mbar_wait(o_done, (j - 1) & 1) || *(volatile int *)abort_flag) break;
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -452,15 +504,15 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 }
             }
-            tmem_st32(tmem + lane_base + kPCol, ph_);
-            if constexpr (kBf16) tmem_st32(tmem + lane_base + kPlCol, pl_);
+            tmem_st32(sbuf, ph_);  // over this row of S_j, already read
+            if constexpr (kBf16) tmem_st32(sbuf + kPlOff, pl_);
             tmem_wait_st();
             // V rows past the context: zero (both halves) before P V reads them
             const int zrow = max(0, ctx - kv0);
             if (zrow < kN) {
                 // V_j must have landed before its tail rows are overwritten
-                if (!mbar_wait(v_full + (j & 1), (j >> 1) & 1) || *(volatile int *)abort_flag) break;
-                unsigned char *vt = Vs + (j & 1) * kKVBytes;
+                if (!mbar_wait(v_full + b, (j >> 1) & 1) || *(volatile int *)abort_flag) break;
+                unsigned char *vt = Vs + b * kKVBytes;
                 const int nvec = (kN - zrow) * 2 * (kHalfBytes / 16);
                 for (int i = r; i < nvec; i += kSoftmaxWarps * 32) {
                     const int row = zrow + i / 16;
