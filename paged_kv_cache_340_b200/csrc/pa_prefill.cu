@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
     int *abort_flag = reinterpret_cast<int *>(bars + 15);
 
-    const int qt = blockIdx.x;
+    const int qt = gridDim.x - 1 - blockIdx.x;  // longest query tile of each (head, sequence) first
     const int kvh = blockIdx.y;
     const int s = blockIdx.z;
     const int warp = threadIdx.x >> 5;
