@@ -688,7 +688,8 @@ def main():
         "clocks": clocks,
     }
     line["kernels"] = kernel_lines(spec, b, kern, by)
-    if world == 1 and rank == 0 and not args.no_cpu_baseline and "k_pool" in b.host_inputs:
+    if world == 1 and rank == 0 and not args.no_cpu_baseline and "k_pool" in b.host_inputs and \
+            spec.kv_dtype != "i8":  # the sampled oracle leg is the 16/32-bit decode
         nbytes, secs, nseq = oracle_sample(OracleBatch(spec, b.host_inputs), 12.0)
         line["cpu_baseline"] = {"value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{nseq} of {spec.num_seqs} sequences (all heads), decode only; "
