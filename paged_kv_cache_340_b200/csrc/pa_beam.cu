@@ -41,6 +41,8 @@ constexpr int kItems = 16;         // table entries per thread per pass
 constexpr int kScanItems = 8;      // the same in the scanned pass (four values per entry)
 // per-beam values staged in shared memory: 3 words per old beam, 1 per new beam
 constexpr int kMaxStageBytes = PA_BEAM_MAX_STAGED * 4;
+// per-beam values plus the old tables, when they fit in this much
+constexpr int kMaxDynBytes = 200 * 1024;
 constexpr int32_t kMagic = 0x50414250;
 
 struct Pool {
@@ -214,6 +216,9 @@ __device__ __forceinline__ int nblk(int ctx, int bs) { return (ctx + bs - 1) / b
 // table entries first loads kItems entries per thread into registers, then
 // acts on them: one or two memory round trips per pass instead of one per
 // entry. Table, context and parent arrays are read-only here (__ldg).
+// kStaged: the old tables are first copied to shared memory (when they fit),
+// so the passes below read them there instead of from L2.
+template <bool kStaged>
 __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams q) {
     extern __shared__ int dyn[];
     __shared__ int warp_sums[32];
@@ -228,7 +233,14 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
     int *s_nb = dyn + n_old;             // [n_old] its block count
     int *s_nch = dyn + 2 * n_old;        // [n_old] its number of children
     int *s_par = dyn + 3 * n_old;        // [n_new] parent of new beam i
+    int *s_tab = dyn + 3 * n_old + n_new;  // kStaged: [n_old * MB] the old tables
     const int32_t *__restrict__ otab = q.old_tables;
+    auto tab = [&](int e) -> int {
+        if constexpr (kStaged)
+            return s_tab[e];
+        else
+            return __ldg(otab + e);
+    };
 
     if (tid == 0) s_bad = 0;
     __syncthreads();
@@ -243,6 +255,21 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
         s_nb[j] = c < 0 ? 0 : nblk(c, bs);
         s_nch[j] = 0;
         if (c < 0 || nblk(c, bs) > MB) atomicOr(&s_bad, PA_DEVERR_CONTEXT);
+    }
+    if constexpr (kStaged) {
+        for (int base = 0; base < old_entries; base += kThreads * kItems) {
+            int v[kItems];
+#pragma unroll
+            for (int k = 0; k < kItems; ++k) {
+                const int e = base + k * kThreads + tid;
+                v[k] = e < old_entries ? __ldg(otab + e) : 0;
+            }
+#pragma unroll
+            for (int k = 0; k < kItems; ++k) {
+                const int e = base + k * kThreads + tid;
+                if (e < old_entries) s_tab[e] = v[k];
+            }
+        }
     }
     __syncthreads();
     for (int i = tid; i < n_new; i += kThreads) {
@@ -264,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
                 if (e < old_entries) {
                     const int j = e / MB;
                     if (e - j * MB < s_nb[j]) {
-                        blk[k] = __ldg(otab + e);
+                        blk[k] = tab(e);
                         in_use |= 1 << k;
                     }
                 }
@@ -299,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
             blk[k] = -1;
             if (e < old_entries) {
                 const int j = e / MB;
-                if (e - j * MB < s_nb[j] && s_nch[j] != 1) blk[k] = __ldg(otab + e);
+                if (e - j * MB < s_nb[j] && s_nch[j] != 1) blk[k] = tab(e);
             }
         }
 #pragma unroll
@@ -314,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
         const int par = s_par[i];
         const int t = s_ctx[par];
         if (t % bs) {
-            const int o = __ldg(otab + par * MB + t / bs);
+            const int o = tab(par * MB + t / bs);
             atomicAdd(&p.writers[o], 1);
             atomicMax(&p.last_writer[o], i);
         }
@@ -330,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
             blk[k] = -1;
             if (e < old_entries) {
                 const int j = e / MB;
-                if (e - j * MB < s_nb[j] && s_nch[j] == 0) blk[k] = __ldg(otab + e);
+                if (e - j * MB < s_nb[j] && s_nch[j] == 0) blk[k] = tab(e);
             }
         }
 #pragma unroll
@@ -359,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
             blk[k] = -1;
             if (e < old_entries) {
                 const int j = e / MB;
-                if (e - j * MB < s_nb[j] && s_nch[j] == 0) blk[k] = __ldg(otab + e);
+                if (e - j * MB < s_nb[j] && s_nch[j] == 0) blk[k] = tab(e);
             }
         }
 #pragma unroll
@@ -400,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
             if (t % bs == 0) {
                 need = 1;
             } else {
-                const int o = __ldg(otab + par * MB + t / bs);
+                const int o = tab(par * MB + t / bs);
                 const int others = p.ref[o] + p.delta[o] - p.writers[o];
                 copy = (others > 0 || p.last_writer[o] != i);
                 need = copy;
@@ -425,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
             blk[k] = -1;
             if (e < old_entries) {
                 const int j = e / MB;
-                if (e - j * MB < s_nb[j] && s_nch[j] != 1) blk[k] = __ldg(otab + e);
+                if (e - j * MB < s_nb[j] && s_nch[j] != 1) blk[k] = tab(e);
             }
         }
 #pragma unroll
@@ -451,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
                 if (e < new_entries) {
                     const int i = e / MB, pos = e - i * MB;
                     const int par = s_par[i];
-                    if (pos < s_nb[par]) v[k] = __ldg(otab + par * MB + pos);
+                    if (pos < s_nb[par]) v[k] = tab(par * MB + pos);
                 }
             }
 #pragma unroll
@@ -472,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
                 if (t % bs == 0) {
                     need = 1;
                 } else {
-                    o = __ldg(otab + par * MB + t / bs);
+                    o = tab(par * MB + t / bs);
                     copy = (p.ref[o] - p.writers[o] > 0 || p.last_writer[o] != i);
                     need = copy;
                 }
@@ -503,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
             const int par = s_par[i];
             const int t = s_ctx[par];
             if (t % bs) {
-                const int o = __ldg(otab + par * MB + t / bs);
+                const int o = tab(par * MB + t / bs);
                 if (q.new_tables[i * MB + t / bs] != o) atomicSub(&p.ref[o], 1);
             }
         }
@@ -514,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
         const int par = s_par[i];
         const int t = s_ctx[par];
         if (t % bs) {
-            const int o = __ldg(otab + par * MB + t / bs);
+            const int o = tab(par * MB + t / bs);
             p.writers[o] = 0;
             p.last_writer[o] = -1;
         }
@@ -572,12 +599,21 @@ cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const in
     q.num_blocks = num_blocks;
     q.block_size = block_size;
     q.err = err;
-    const int smem = (3 * num_old + num_new) * (int)sizeof(int);
-    static unsigned int attr_done = 0;
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(beam::beam_step_kernel), beam::kMaxStageBytes,
-                                     &attr_done);
-    if (e != cudaSuccess) return e;
-    beam::beam_step_kernel<<<1, beam::kThreads, smem, stream>>>(q);
+    const long long base = (3LL * num_old + num_new) * (long long)sizeof(int);
+    const long long with_tables = base + (long long)num_old * max_blocks * (long long)sizeof(int);
+    static unsigned int attr_done[2] = {0, 0};
+    cudaError_t e;
+    if (with_tables <= beam::kMaxDynBytes) {
+        e = ensure_smem_attr(reinterpret_cast<const void *>(beam::beam_step_kernel<true>), beam::kMaxDynBytes,
+                             &attr_done[1]);
+        if (e != cudaSuccess) return e;
+        beam::beam_step_kernel<true><<<1, beam::kThreads, (int)with_tables, stream>>>(q);
+    } else {
+        e = ensure_smem_attr(reinterpret_cast<const void *>(beam::beam_step_kernel<false>), beam::kMaxStageBytes,
+                             &attr_done[0]);
+        if (e != cudaSuccess) return e;
+        beam::beam_step_kernel<false><<<1, beam::kThreads, (int)base, stream>>>(q);
+    }
     return cudaGetLastError();
 }
 
