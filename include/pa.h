@@ -281,9 +281,10 @@ int pa_reshape_and_cache_q8(const void *key, const void *value, pa_dtype src_dty
 
 /* pa_decode over an int8 cache: out = softmax(scale q . K_t) V_t with
  * K_t = kq_t * k_scale_t, V_t = vq_t * v_scale_t. query is q_dtype (PA_F16
- * or PA_BF16; a bf16 query is converted to fp16 for the tensor cores, exact
- * for magnitudes in [2^-14, 65504]); out_dtype q_dtype or PA_F32. Other
- * arguments, checks and device errors as pa_decode. */
+ * or PA_BF16); out_dtype q_dtype or PA_F32. On the tensor cores q . kq_t is
+ * an exact integer product of kq_t and the query held as 16-bit fixed point
+ * per head (each q_d within 2^-16 of the head's largest |q_d|); P enters
+ * P V in fp16. Other arguments, checks and device errors as pa_decode. */
 int pa_decode_q8(void *out, const void *query, pa_dtype q_dtype, const int8_t *k_cache, const int8_t *v_cache,
                  const float *k_scale, const float *v_scale, const int32_t *block_tables, int max_blocks_per_seq,
                  const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,

@@ -506,14 +506,15 @@ __device__ __forceinline__ uint32_t i8pair_to_h2(uint32_t biased, unsigned sel) 
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// As MmaConsumer, for int8 caches with per-row scales. The MMAs run in fp16
-// (int8 codes are exact in fp16; a bf16 query is converted to fp16 once, exact
-// for magnitudes in [2^-14, 65504]). Per 16-token stage, lane = 4 r + q:
-//   S^T = Kq Q^T: lane loads 16-byte chunks q + 4 j of token rows r and r + 8
-//     (16 dims each); word w of a chunk feeds one k-step (dims 4w .. 4w+3 as
-//     k columns 2q, 2q+1, 2q+8, 2q+9), so one load feeds four k-steps; Q's B
-//     fragment uses the same map. The score of token t is scaled by its K
-//     row scale after the MMA.
+// As MmaConsumer, for int8 caches with per-row scales. Per 16-token stage,
+// lane = 4 r + q:
+//   S^T = Kq Q^T on the int8 tensor cores (mma.sync m16n8k32, int32
+//     accumulation): the query of each head is held as 16-bit fixed point
+//     (step = its largest |q_d| / 32767, split into a signed high byte and an
+//     unsigned low byte: two exact integer products); lane loads 16-byte
+//     chunks q + 4 j of token rows r and r + 8 and feeds their words to the
+//     MMAs' A fragments directly (no conversion). The score of token t is the
+//     integer product times the step and its K row scale.
 //   O^T += Vq^T P'^T with P'_t = p_t * sv_t / svmax (sv_t the V row scale,
 //     svmax the stage's largest), so P' is in [0, 1] in fp16; the stage's
 //     product is added to O times svmax (fp32). Lane loads W = D/8 dims
@@ -528,7 +529,8 @@ struct MmaConsumerQ8 {
     static constexpr int kMT = D / 16;   // PV m-tiles
     static constexpr int kW = D / 8;     // V dims per lane
     int q4, r;
-    uint32_t qb[kJ][8];
+    uint32_t qhi[kJ][4], qlo[kJ][4];     // query as 16-bit fixed point: signed high bytes, unsigned low bytes
+    float qs[2];                         // fixed-point step of heads 2q, 2q + 1
     float o[kMT][4];
     float m_run[2], l_lane[2];
 
@@ -536,9 +538,32 @@ struct MmaConsumerQ8 {
         return kW * (m & 7) + mt + (m >= 8 ? kW / 2 : 0);
     }
 
+    // mma.sync m16n8k32, int8 x int8 -> int32 (B signed or unsigned)
+    static __device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                  uint32_t b0, uint32_t b1) {
+        asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+    static __device__ __forceinline__ void mma_u8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                  uint32_t b0, uint32_t b1) {
+        asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+
+    // The query of head r (this lane's B column) as Q = rint(q / step) with
+    // step = max_d |q_d| / 32767 (|Q| <= 32767), split Q = 256 hi + lo (hi
+    // signed, lo in [0, 255]): q . k = step (256 hi.k + lo.k), both products
+    // exact in int32 on the int8 tensor cores. |q - step Q| <= step / 2, i.e.
+    // 2^-16 of the head's largest component.
     __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int, int lane) {
         q4 = lane & 3;
         r = lane >> 2;
+        float f[kJ][16];
+        float amax = 0.f;
 #pragma unroll
         for (int j = 0; j < kJ; ++j) {
 #pragma unroll
@@ -547,15 +572,32 @@ struct MmaConsumerQ8 {
                 if (r < G)
                     u = *reinterpret_cast<const uint4 *>(static_cast<const TQ *>(p.query) + (head0 + r) * D +
                                                          16 * (q4 + 4 * j) + 8 * h);
-                float f[8];
-                Elt<TQ>::unpack(u, f);
+                Elt<TQ>::unpack(u, f[j] + 8 * h);
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[j][e]));
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const float inv = amax > 0.f ? __fdiv_rn(32767.f, amax) : 0.f;
+        const float step = amax > 0.f ? __fdiv_rn(amax, 32767.f) : 0.f;
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {  // word w: dims 4w .. 4w + 3 of the chunk
+                uint32_t hi = 0, lo = 0;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    __half2 v = __floats2half2_rn(f[2 * e], f[2 * e + 1]);
-                    qb[j][4 * h + e] = *reinterpret_cast<uint32_t *>(&v);
+                    const int Q = max(-32767, min(32767, __float2int_rn(f[j][4 * w + e] * inv)));
+                    hi |= (uint32_t)((Q >> 8) & 0xff) << (8 * e);
+                    lo |= (uint32_t)(Q & 0xff) << (8 * e);
                 }
+                qhi[j][w] = hi;
+                qlo[j][w] = lo;
             }
         }
+        qs[0] = __shfl_sync(0xffffffffu, step, (2 * q4) * 4);
+        qs[1] = __shfl_sync(0xffffffffu, step, (2 * q4 + 1) * 4);
 #pragma unroll
         for (int mt = 0; mt < kMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
         m_run[0] = m_run[1] = -INFINITY;
@@ -566,20 +608,24 @@ struct MmaConsumerQ8 {
                                           float scale_log2) {
         const float *ksc = reinterpret_cast<const float *>(Kb + 2 * S::kTileBytes);
         const float *vsc = ksc + S::kTS;
-        // ---- S^T = Kq Q^T
-        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- S^T = Kq Q^T on the int8 tensor cores: MMA (j, m) takes dims
+        // 16 (q + 4 j) + 8 m + 0..3 as k columns 4q..4q+3 and + 4..7 as 16 + 4q..
+        int chi[4] = {0, 0, 0, 0}, clo[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int j = 0; j < kJ; ++j) {
             const uint4 u0 = *reinterpret_cast<const uint4 *>(Kb + r * D + 16 * (q4 + 4 * j));
             const uint4 u1 = *reinterpret_cast<const uint4 *>(Kb + (r + 8) * D + 16 * (q4 + 4 * j));
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const uint32_t x0 = word_of(u0, w) ^ 0x80808080u;
-                const uint32_t x1 = word_of(u1, w) ^ 0x80808080u;
-                mma_f16(sc, i8pair_to_h2(x0, 0x4140u), i8pair_to_h2(x1, 0x4140u), i8pair_to_h2(x0, 0x4342u),
-                        i8pair_to_h2(x1, 0x4342u), qb[j][2 * w], qb[j][2 * w + 1]);
+            for (int m = 0; m < 2; ++m) {
+                const uint32_t a0 = word_of(u0, 2 * m), a2 = word_of(u0, 2 * m + 1);
+                const uint32_t a1 = word_of(u1, 2 * m), a3 = word_of(u1, 2 * m + 1);
+                mma_s8(chi, a0, a1, a2, a3, qhi[j][2 * m], qhi[j][2 * m + 1]);
+                mma_u8(clo, a0, a1, a2, a3, qlo[j][2 * m], qlo[j][2 * m + 1]);
             }
         }
+        float sc[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sc[i] = (float)((chi[i] << 8) + clo[i]) * qs[i & 1];
         // ---- online softmax per query head g = 2q + h over tokens r, r + 8
         const bool v0 = r < nvalid;
         const bool v1 = r + 8 < nvalid;

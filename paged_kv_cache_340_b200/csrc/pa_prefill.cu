@@ -632,6 +632,7 @@ extern "C" int pa_prefill(void *out, const void *query, const int32_t *q_start, 
         return PA_ERR_ALIGN;
     const long long kv_rows = (long long)num_blocks * num_kv_heads * block_size;
     if (kv_rows >= INT32_MAX || (long long)num_tokens * num_heads >= INT32_MAX) return PA_ERR_SHAPE;
+    if ((long long)max_q_len * group >= INT32_MAX) return PA_ERR_SHAPE;
     const bool bf16 = kv_dtype == PA_BF16;
     CUtensorMap mq, mk, mv;
     {

@@ -365,3 +365,33 @@ def test_beam_search_workload_full_size(pa):
     ref = oracle.paged_decode(f64(inp["query"][5]), _f64_of(k_or, torch.float16), _f64_of(v_or, torch.float16),
                               _tables(ob, mb), np.array([s.num_tokens for s in ob], np.int32), spec.scale, bs)
     assert_attention_close(b.out, ref, torch.float16, "beam workload decode")
+
+
+@pytest.mark.parametrize("policy", ["fifo", "lifo"])
+def test_beam_step_release_all_and_empty_beams(pa, policy):
+    """No new beams (every old beam released: all their blocks return to the
+    free list in release order), then new beams from an empty parent (context
+    0: the token takes a fresh block)."""
+    opool, dpool, beams = _start(pa, 64, 4, policy, [9, 4, 13, 1], seed=5)
+    ob = [Sequence(list(b.block_table), b.num_tokens) for b in beams]
+    new, slots, cow = beam_step(opool, ob, [])
+    dev = "cuda"
+    old_t = torch.from_numpy(_tables(beams, 8)).to(dev)
+    old_c = torch.tensor([b.num_tokens for b in beams], dtype=torch.int32, device=dev)
+    empty_i = torch.empty(0, dtype=torch.int32, device=dev)
+    ncow = torch.full((1,), -5, dtype=torch.int32, device=dev)
+    pa.pa_beam_step(dpool, old_t, old_c, empty_i, torch.empty((0, 8), dtype=torch.int32, device=dev), empty_i,
+                    empty_i, torch.empty((0, 2), dtype=torch.int64, device=dev), ncow)
+    torch.cuda.synchronize()
+    assert new == [] and int(ncow.item()) == 0
+    _assert_same_state(dpool, opool)
+    assert dpool.ref.cpu().tolist() == [0] * 64
+    # a context-0 beam forked twice: both take a fresh block for position 0
+    zero = [Sequence([], 0)]
+    ob = [Sequence([], 0)]
+    new, slots, cow = beam_step(opool, ob, [0, 0])
+    t, c, s_, cw, n = _device_step(pa, dpool, zero, [0, 0], 8)
+    assert t.tolist() == _tables(new, 8).tolist() and s_.tolist() == slots and n == 0 == len(cow)
+    assert c.tolist() == [1, 1]
+    _assert_same_state(dpool, opool)
+    assert pa.pa_read_device_errors() == 0

@@ -228,3 +228,22 @@ def test_int8_workloads_full_size(pa, name):
         ref = oracle.paged_decode_q8(f64(q[s:s + 1]), kq[ids], vq[ids], ks[ids], vs[ids], tab,
                                      np.array([L], np.int32), spec.scale, spec.block_size)
         assert_attention_close(out[s:s + 1], ref, torch.float16, f"{name} seq {s}")
+
+
+def test_decode_splitk_q8_head_dim_64_with_schedule(pa):
+    """Split-K over an int8 cache with head_dim 64 and a GQA group of 8, with a
+    longest-first schedule: same result as the oracle."""
+    S, Hq, Hkv, D, bs, ctx = 4, 16, 2, 64, 32, [900, 1, 300, 64]
+    c = Q8Case(S, Hq, Hkv, D, bs, ctx, seed=81)
+    kq, vq, ks, vs = c.device()
+    L, P = 900, 128
+    ws = torch.empty(pa.pa_splitk_workspace_bytes(S, Hq, D, L, P), dtype=torch.uint8, device="cuda")
+    out = torch.empty((S, Hq, D), device="cuda")
+    tab, cl = torch.from_numpy(c.tables).cuda(), torch.from_numpy(c.ctx).cuda()
+    order = torch.tensor([0, 2, 3, 1], dtype=torch.int32, device="cuda")
+    pa.pa_decode_splitk_q8(ws, c.q.to(torch.bfloat16).cuda(), kq, vq, ks, vs, tab, cl, c.scale, L, P,
+                           seq_order=order)
+    pa.pa_splitk_reduce(out, ws, cl, L, P)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_errors() == 0
+    assert_attention_close(out, c.ref(torch.bfloat16), torch.float16, "q8 split D=64")

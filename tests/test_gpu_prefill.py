@@ -71,6 +71,7 @@ CASES = [
     ([200, 129, 40], [130, 129, 3], 8, 8, 32),                # crossing the 128-row tile, bs 32
     ([96, 513, 17], [96, 100, 17], 16, 4, 16),                # GQA G = 4
     ([250, 64], [250, 33], 16, 2, 32),                        # GQA G = 8
+    ([700, 300, 1], [640, 300, 1], 16, 8, 16),                # GQA G = 2, several query tiles per sequence
 ]
 
 
@@ -162,3 +163,4 @@ def test_prefill_workloads_full_size(pa, name):
                                            np.array([pos + 1], np.int32), spec.scale, spec.block_size)
                 got = out[s * spec.q_len + i:s * spec.q_len + i + 1, kvh * G:(kvh + 1) * G]
                 assert_attention_close(got, ref, spec.torch_kv_dtype, f"{name} seq {s} kv {kvh} row {i}")
+
