@@ -379,6 +379,20 @@ int pa_reshape_and_cache_q8(const void *key, const void *value, pa_dtype src_dty
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// The V pool of an int8 cache with head_dim 128 as 2-D rows for the decode
+// kernel's swizzled TMA loads (see DecodeParams::v_map).
+static int q8_v_map(DecodeParams &p, const int8_t *v_cache, int num_blocks, int num_kv_heads, int head_dim,
+                    int block_size) {
+    if (head_dim != 128) return PA_OK;
+    const long long rows = (long long)num_blocks * num_kv_heads * block_size;
+    if (rows <= 0) return PA_OK;
+    if (rows >= INT_MAX) return PA_ERR_SHAPE;  // TMA row coordinates are 32-bit
+    return encode_rows_2d(&p.v_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, v_cache, 128, (unsigned long long)rows, 128, 128,
+                          16, CU_TENSOR_MAP_SWIZZLE_128B)
+               ? PA_OK
+               : PA_ERR_CUDA;
+}
+
 // Shared by the int8 decode entries: query type, scale pools, then the common checks.
 static int check_q8_args(const void *query, pa_dtype q_dtype, const int8_t *k_cache, const int8_t *v_cache,
                          const float *k_scale, const float *v_scale, const int32_t *block_tables,
@@ -428,6 +442,8 @@ int pa_decode_q8(void *out, const void *query, pa_dtype q_dtype, const int8_t *k
     p.max_context_len = INT_MAX;
     p.out_dtype = out_dtype;
     p.err = err;
+    rc = q8_v_map(p, v_cache, num_blocks, num_kv_heads, head_dim, block_size);
+    if (rc != PA_OK) return rc;
     cudaError_t e = launch_decode_q8(p, q_dtype, head_dim, block_size, num_heads / num_kv_heads, 1, num_kv_heads,
                                      num_seqs, stream);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
@@ -474,6 +490,8 @@ int pa_decode_splitk_q8(void *workspace, size_t workspace_bytes, const void *que
     p.max_context_len = max_context_len;
     p.out_dtype = PA_F32;
     p.err = err;
+    rc = q8_v_map(p, v_cache, num_blocks, num_kv_heads, head_dim, block_size);
+    if (rc != PA_OK) return rc;
     cudaError_t e = launch_decode_q8(p, q_dtype, head_dim, block_size, num_heads / num_kv_heads, mp, num_kv_heads,
                                      num_seqs, stream);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;

@@ -68,18 +68,25 @@ struct DecodeShape {
     static constexpr int kThreads = kWarps * 32;
     static constexpr int kTileBytes = kTS * D * kElt;  // 16 token rows of one kv head, K or V
     static constexpr int kScaleBytes = kInt8 ? kTS * 4 : 0;  // int8: the 16 rows' fp32 scales, K or V
-    static constexpr int kStageBytes = 2 * kTileBytes + 2 * kScaleBytes;
+    // int8 with 128-byte rows: V tiles come by 2-D TMA in the 128-byte
+    // swizzled layout, in their own 1024-byte-aligned region; each stage
+    // buffer then holds K and the scales only.
+    static constexpr bool kVSwizzle = kInt8 && D == 128;
+    static constexpr int kStageBytes = (kVSwizzle ? 1 : 2) * kTileBytes + 2 * kScaleBytes;
+    static constexpr int kScaleOff = (kVSwizzle ? 1 : 2) * kTileBytes;  // scales within a stage buffer
     // Buffers per warp (a ring of kWarps * kBufPerWarp stages). int8 stages
     // are half the bytes; measured, a deeper int8 ring did not help, five
     // CTAs per SM did.
     static constexpr int kBufPerWarp = 2;
     static constexpr int kStages = kWarps * kBufPerWarp;
     static constexpr int kRowGroups = kUseMma ? kWarps : kWarps * kRows;
-    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kVRegion = kVSwizzle ? kStages * kTileBytes : 0;
+    static constexpr int kRingBytes = kVRegion + kStages * kStageBytes;
+    static constexpr int kAlign = kVSwizzle ? 1024 : 128;  // ring base alignment
     static constexpr int kAgStride = kUseMma ? D + 1 : D;  // floats per merged accumulator row
     static constexpr int kMergeBytes = kRowGroups * G * (kAgStride + 2) * 4;
     static constexpr int kDataBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
-    static constexpr int kSmemBytes = 128 + kDataBytes + kStages * 8 + kStages * 4;
+    static constexpr int kSmemBytes = kAlign + kDataBytes + kStages * 8 + kStages * 4;
     // Resident CTAs per SM the register budget is set for (a sub-partition
     // holds one warp of each CTA, so 3 CTAs leave 170 registers a thread).
     static constexpr int kMinBlocks = kInt8 ? 5 : ((kUseMma || G <= 4) ? 3 : 2);
@@ -606,7 +613,7 @@ struct MmaConsumerQ8 {
 
     __device__ __forceinline__ void stage(const unsigned char *Kb, const unsigned char *Vb, int nvalid, int,
                                           float scale_log2) {
-        const float *ksc = reinterpret_cast<const float *>(Kb + 2 * S::kTileBytes);
+        const float *ksc = reinterpret_cast<const float *>(Kb + S::kScaleOff);
         const float *vsc = ksc + S::kTS;
         // ---- S^T = Kq Q^T on the int8 tensor cores: MMA (j, m) takes dims
         // 16 (q + 4 j) + 8 m + 0..3 as k columns 4q..4q+3 and + 4..7 as 16 + 4q..
@@ -669,7 +676,22 @@ struct MmaConsumerQ8 {
         // ---- O^T = O^T alpha + svmax (Vq^T P'^T)
         uint32_t wa[kW / 4], wb[kW / 4], wc[kW / 4], wd[kW / 4];  // token rows 2q, 2q+1, 2q+8, 2q+9
         const unsigned char *vcol = Vb + kW * r;
-        if constexpr (kW == 16) {
+        if constexpr (S::kVSwizzle) {
+            // swizzled tile: 16-byte chunk c of row t sits at chunk c ^ (t % 8), so the
+            // four lanes reading dims W r .. of rows 2q, .. hit four different chunks
+            const int c0 = r ^ (2 * q4), c1 = r ^ (2 * q4 + 1);
+            const uint4 a = *reinterpret_cast<const uint4 *>(Vb + (2 * q4) * D + 16 * c0);
+            const uint4 b = *reinterpret_cast<const uint4 *>(Vb + (2 * q4 + 1) * D + 16 * c1);
+            const uint4 c = *reinterpret_cast<const uint4 *>(Vb + (2 * q4 + 8) * D + 16 * c0);
+            const uint4 d = *reinterpret_cast<const uint4 *>(Vb + (2 * q4 + 9) * D + 16 * c1);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                wa[w] = word_of(a, w);
+                wb[w] = word_of(b, w);
+                wc[w] = word_of(c, w);
+                wd[w] = word_of(d, w);
+            }
+        } else if constexpr (kW == 16) {
             const uint4 a = *reinterpret_cast<const uint4 *>(vcol + (2 * q4) * D);
             const uint4 b = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 1) * D);
             const uint4 c = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 8) * D);
@@ -751,14 +773,14 @@ struct MmaConsumerQ8 {
 // query's type (T for 16- and 32-bit caches).
 template <typename T, int D, int BS, int G, typename TQ = T>
 __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShape<T, D, BS, G>::kMinBlocks)
-    decode_kernel(const DecodeParams p) {
+    decode_kernel(const __grid_constant__ DecodeParams p) {
     using S = DecodeShape<T, D, BS, G>;
     using Consumer = std::conditional_t<
         S::kInt8, MmaConsumerQ8<TQ, D, G, S>,
         std::conditional_t<S::kUseMma, MmaConsumer<T, D, G, S>, FmaConsumer<T, D, G, S>>>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *ring = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+        (reinterpret_cast<uintptr_t>(smem_raw) + S::kAlign - 1) & ~uintptr_t(S::kAlign - 1));
     uint64_t *full = reinterpret_cast<uint64_t *>(ring + S::kDataBytes);
     int *bad = reinterpret_cast<int *>(full + S::kStages);
 
@@ -835,14 +857,19 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
         if (id >= 0) {
             bad[buf] = 0;
             const size_t src = (size_t)id * block_elems + (size_t)(k % S::kSubs) * S::kTS * D;
-            unsigned char *dst = ring + (size_t)buf * S::kStageBytes;
-            mbar_arrive_expect_tx(full + buf, S::kStageBytes);
+            unsigned char *dst = ring + S::kVRegion + (size_t)buf * S::kStageBytes;
+            mbar_arrive_expect_tx(full + buf, 2 * S::kTileBytes + 2 * S::kScaleBytes);
             bulk_load(dst, kc + src, S::kTileBytes, full + buf, pol);
-            bulk_load(dst + S::kTileBytes, vc + src, S::kTileBytes, full + buf, pol);
+            if constexpr (S::kVSwizzle) {  // V: pool row (block, kv head, token) as a 2-D box
+                const int vrow = (int)(((long long)id * p.num_kv_heads + kvh) * BS + (k % S::kSubs) * S::kTS);
+                tma_load_2d(ring + (size_t)buf * S::kTileBytes, &p.v_map, 0, vrow, full + buf);
+            } else {
+                bulk_load(dst + S::kTileBytes, vc + src, S::kTileBytes, full + buf, pol);
+            }
             if constexpr (S::kInt8) {  // the 16 rows' scales: 64 contiguous bytes each
                 const size_t ssrc = (size_t)id * p.num_kv_heads * BS + (size_t)(k % S::kSubs) * S::kTS;
-                bulk_load(dst + 2 * S::kTileBytes, ksc + ssrc, S::kScaleBytes, full + buf, pol);
-                bulk_load(dst + 2 * S::kTileBytes + S::kScaleBytes, vsc + ssrc, S::kScaleBytes, full + buf, pol);
+                bulk_load(dst + S::kScaleOff, ksc + ssrc, S::kScaleBytes, full + buf, pol);
+                bulk_load(dst + S::kScaleOff + S::kScaleBytes, vsc + ssrc, S::kScaleBytes, full + buf, pol);
             }
         } else {
             bad[buf] = 1;
@@ -878,8 +905,9 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
         waited = m + 1;
         if (!bad[buf]) {
             const int nvalid = min(S::kTS, t_end - (t_begin + k * S::kTS));
-            const unsigned char *Kb = ring + (size_t)buf * S::kStageBytes;
-            cons.stage(Kb, Kb + S::kTileBytes, nvalid, lane, p.scale_log2);
+            const unsigned char *Kb = ring + S::kVRegion + (size_t)buf * S::kStageBytes;
+            const unsigned char *Vb = S::kVSwizzle ? ring + (size_t)buf * S::kTileBytes : Kb + S::kTileBytes;
+            cons.stage(Kb, Vb, nvalid, lane, p.scale_log2);
         }
         // Reload this buffer with this warp's stage m + kBufPerWarp.
         const int idn = id_of(m + S::kBufPerWarp);

@@ -1,6 +1,7 @@
 // Internal interfaces between the C-ABI layer (pa_api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -31,6 +32,10 @@ struct DecodeParams {
     int max_context_len;
     pa_dtype out_dtype;
     unsigned int *err;   // device error word
+    // int8 caches with head_dim 128: the V pool as rows of 128 bytes, 16-row
+    // boxes in the 128-byte swizzled layout (the kernel's V fragment loads are
+    // then free of shared-memory bank conflicts)
+    alignas(64) CUtensorMap v_map;
 };
 
 cudaError_t launch_decode(const DecodeParams &p, pa_dtype kv_dtype, int head_dim, int block_size,
@@ -73,6 +78,13 @@ cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const in
                              const int32_t *parents, int num_new, int32_t *new_tables, int32_t *new_ctx,
                              int max_blocks, int32_t *slots, int64_t *cow_pairs, int32_t *num_cow,
                              int num_blocks, int block_size, unsigned int *err, cudaStream_t stream);
+
+// A rank-2 TMA tensor map over `rows` rows of `inner` elements (row stride in
+// bytes), box box_inner x box_rows, zero fill. False if the encoder is
+// unavailable or refuses the shape.
+bool encode_rows_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, unsigned long long inner,
+                    unsigned long long rows, unsigned long long row_stride_bytes, unsigned box_inner,
+                    unsigned box_rows, CUtensorMapSwizzle swizzle);
 
 // Device address of the current device's error word (cached per device).
 cudaError_t device_error_word(unsigned int **word);
