@@ -1,5 +1,8 @@
 /*
- * pa.h -- C ABI of the paged KV-cache decode library for NVIDIA B200 (sm_100a).
+ * pa.h -- C ABI of the paged KV-cache library for NVIDIA B200 (sm_100a):
+ * decode, split-K decode, prefill, slot writes and block copies (16-bit, fp32
+ * and int8 caches), the host block pool with its prefix cache, and a device
+ * block pool with a beam-search step.
  *
  * A sequence's keys and values live in fixed-size blocks of a shared pool; a
  * per-sequence block table maps logical block i (tokens i*bs .. i*bs+bs-1) to

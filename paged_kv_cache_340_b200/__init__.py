@@ -1,15 +1,24 @@
-"""Python binding of the paged KV-cache decode library for B200 (sm_100a).
+"""Python binding of the paged KV-cache library for B200 (sm_100a).
 
 Argument marshalling only: every operation runs in the CUDA kernels of
-``lib/libpa_b200.so`` through its C ABI (``include/pa.h``); functions keep the
-C names. PyTorch supplies device memory and streams. There is no CPU or
-library fallback: if the shared library is missing, the first call raises.
+``lib/libpa_b200.so`` (or, for the pools, its C++ host code) through its C ABI
+(``include/pa.h``); functions keep the C names. PyTorch supplies device memory
+and streams. There is no CPU or library fallback: if the shared library is
+missing, the first call raises.
+
+Calls: slot write (pa_reshape_and_cache), decode (pa_decode), split-K decode
+and reduce (pa_decode_splitk, pa_splitk_reduce, pa_decode_splitk_static),
+copy-on-write block copy (pa_copy_blocks, pa_copy_blocks_counted), paged
+prefill (pa_prefill), the int8 cache (pa_*_q8), the host block pool and
+prefix cache (BlockPool, PrefixCache), and the device pool with its beam step
+(DevicePool, pa_beam_step).
 
 Layouts (contiguous): k_cache/v_cache [num_blocks, num_kv_heads, block_size,
 head_dim]; query/out [num_seqs, num_heads, head_dim]; key/value
 [num_tokens, num_kv_heads, head_dim]; block_tables [num_seqs,
 max_blocks_per_seq] int32; context_lens [num_seqs] int32; slot_mapping
-[num_tokens] int32; src_dst_pairs [n, 2] int64.
+[num_tokens] int32; src_dst_pairs [n, 2] int64; int8 caches add
+k_scale/v_scale [num_blocks, num_kv_heads, block_size] float32.
 """
 from __future__ import annotations
 
