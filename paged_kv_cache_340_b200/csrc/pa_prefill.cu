@@ -408,9 +408,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mbar_arrive(s_full + 1);
                 mbar_arrive(o_done);
             }
-            if (issued) {  // tensor memory is freed below: every MMA must have finished
+            // tensor memory is freed below, and the softmax warps read O: every MMA
+            // must have finished (with none issued, release the waiters at once)
+            if (issued) {
                 umma_commit(mma_idle);
                 if (!mbar_wait(mma_idle, 0)) record_error(p.err, PA_DEVERR_TIMEOUT);
+            } else {
+                mbar_arrive(mma_idle);
             }
         }
         __syncwarp();
@@ -425,7 +429,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         float m_run = -INFINITY, l_run = 0.f;
         for (int j = 0; j < ntiles; ++j) {
             const int b = j & 1;
-            if (!mbar_wait(s_full + b, (j >> 1) & 1) || *(volatile int *)abort_flag) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(s_full + b, (j >> 1) & 1) && !*(volatile int *)abort_flag))
+                break;
             tc_fence_after();
             const uint32_t sbuf = tmem + lane_base + kSCol + b * kN;
             uint32_t sr[2][32];
@@ -481,20 +486,20 @@ __global__ void __launch_bounds__(kThreads, 2)
                     pl_[c] = Pack16<T>::pack(x[2 * c] - hi0, x[2 * c + 1] - hi1);
                 }
             }
-            if (j > 0) {
-                // O += P_{j-1} V_{j-1} done (waited every tile, so the phases stay in step): O may be rescaled
-                if (!mbar_wait(o_done, (j - 1) & 1) || *(volatile int *)abort_flag) break;
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                // O is rescaled: O += P_{j-1} V_{j-1} must be done. (O += P_{j-2} V_{j-2}
+                // is: S_j was issued after it, so this parity wait cannot alias.)
+                const bool got = mbar_wait(o_done, (j - 1) & 1) && !*(volatile int *)abort_flag;
+                if (!__all_sync(0xffffffffu, got)) break;
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                    for (int ch = 0; ch < kD / 32; ++ch) {
-                        uint32_t o[32];
-                        tmem_ld32(tmem + lane_base + kOCol + ch * 32, o);
-                        tmem_wait_ld();
+                for (int ch = 0; ch < kD / 32; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_base + kOCol + ch * 32, o);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(tmem + lane_base + kOCol + ch * 32, o);
-                    }
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(tmem + lane_base + kOCol + ch * 32, o);
                 }
             }
             tmem_st32(sbuf, ph_);  // over this row of S_j, already read
@@ -504,7 +509,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int zrow = max(0, ctx - kv0);
             if (zrow < kN) {
                 // V_j must have landed before its tail rows are overwritten
-                if (!mbar_wait(v_full + b, (j >> 1) & 1) || *(volatile int *)abort_flag) break;
+                if (!__all_sync(0xffffffffu, mbar_wait(v_full + b, (j >> 1) & 1) && !*(volatile int *)abort_flag))
+                    break;
                 unsigned char *vt = Vs + b * kKVBytes;
                 const int nvec = (kN - zrow) * 2 * (kHalfBytes / 16);
                 for (int i = r; i < nvec; i += kSoftmaxWarps * 32) {
@@ -520,7 +526,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_arrive(p_full);
         }
         // ---- output: O / l for valid rows
-        const bool done = mbar_wait(o_done, (ntiles - 1) & 1) && !*(volatile int *)abort_flag;
+        // every product done (the MMA warp's single-use end-of-kernel commit)
+        const bool done = __all_sync(0xffffffffu, mbar_wait(mma_idle, 0) && !*(volatile int *)abort_flag);
         tc_fence_after();
         if (!done) {
             if (r == 0) record_error(p.err, PA_DEVERR_TIMEOUT);
