@@ -12,19 +12,21 @@
 // How (B200 design): one CTA per (sequence, kv head, 128-row query tile); the
 // rows are (token, query head of the GQA group) pairs, so every K/V tile is
 // loaded once for the whole group.
-//   * warp 4 lane 0 is the control thread. It loads the Q tile once and the
-//     K/V tiles (64 tokens, gathered block by block through the table) with
-//     2-D/3-D TMA tensor copies in the 128-byte swizzled layout, into two
-//     stages; it issues S = Q K^T (M 128, N 64, K = head_dim in 8 steps) and
-//     O += P V (M 128, N = head_dim, K 64 in 4 steps) as tcgen05.mma with the
-//     fp32 accumulators S and O in tensor memory, and tcgen05.commit signals
-//     each product's completion on an mbarrier;
+//   * warp 5 loads: the Q tile once and the K/V tiles (64 tokens, gathered
+//     block by block through the table, 32 lookups at a time, one per lane)
+//     with 2-D/3-D TMA tensor copies in the 128-byte swizzled layout, into
+//     two stages each, refilling a stage once the product that read it is done;
+//   * warp 4 lane 0 issues S = Q K^T (M 128, N 64, K = head_dim in 8 steps)
+//     into one of two S buffers and O += P V (M 128, N = head_dim, K 64 in 4
+//     steps) as tcgen05.mma with the fp32 accumulators S and O in tensor
+//     memory; tcgen05.commit signals each product's completion on an mbarrier;
 //   * warps 0-3 run the softmax: thread r owns row r (tensor-memory lane r),
 //     reads its S row with tcgen05.ld, masks positions past its token
 //     (causal) and past the context, keeps the running max and sum in fp32
-//     (log2 domain), rescales its O row in tensor memory when the max rises,
-//     and writes its probabilities as a 16-bit row of the P operand in shared
-//     memory (same swizzled K-major layout);
+//     (log2 domain), rescales its O row in tensor memory when the max rises
+//     by more than 2^8, and writes its probabilities with tcgen05.st as a
+//     16-bit row over its own S row, where O += P V reads them (the A operand
+//     from tensor memory); the four warps do not wait for each other;
 //   * V rows past the context are zeroed in shared memory before P V (they
 //     may hold anything, and 0 * NaN is NaN on the tensor cores too).
 // Every wait is bounded (PA_DEVERR_TIMEOUT); tensor memory is always freed.
@@ -223,11 +225,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t *k_empty = bars + 5;   // [2] S that read the stage is done
     uint64_t *v_empty = bars + 7;   // [2] PV that read the stage is done
     uint64_t *s_full = bars + 9;    // [2] S buffer computed
-    uint64_t *p_full = bars + 11;   // softmax of the tile done (P written)
-    uint64_t *o_done = bars + 12;   // PV of the tile done
-    uint64_t *mma_idle = bars + 13; // every MMA issued has finished (end of kernel)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
-    int *abort_flag = reinterpret_cast<int *>(bars + 15);
+    // [2] softmax of tile j done (P_j written), on p_full[j & 1]: the softmax
+    // warps do not wait for each other, and one may reach tile j + 1 before
+    // another has finished tile j (never tile j + 2, whose S needs P_j V_j),
+    // so the arrivals of neighbouring tiles go to different barriers
+    uint64_t *p_full = bars + 11;
+    uint64_t *o_done = bars + 13;   // PV of the tile done
+    uint64_t *mma_idle = bars + 14; // every MMA issued has finished (end of kernel)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 15);
+    int *abort_flag = reinterpret_cast<int *>(bars + 16);
 
     const int qt = gridDim.x - 1 - blockIdx.x;  // longest query tile of each (head, sequence) first
     const int kvh = blockIdx.y;
@@ -257,8 +263,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_init(k_empty + i, 1);
             mbar_init(v_empty + i, 1);
             mbar_init(s_full + i, 1);
+            mbar_init(p_full + i, kSoftmaxWarps * 32);
         }
-        mbar_init(p_full, kSoftmaxWarps * 32);
         mbar_init(o_done, 1);
         mbar_init(mma_idle, 1);
         *abort_flag = 0;
@@ -380,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int j = 0; ok && j < min(2, ntiles); ++j) ok = issue_s(j);
             for (int j = 0; ok && j < ntiles; ++j) {
                 const int b = j & 1;
-                if (!mbar_wait(p_full, j & 1) || !mbar_wait(v_full + b, (j >> 1) & 1) ||
+                if (!mbar_wait(p_full + b, (j >> 1) & 1) || !mbar_wait(v_full + b, (j >> 1) & 1) ||
                     *(volatile int *)abort_flag) {
                     ok = false;
                     break;
@@ -523,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 fence_proxy_async_smem();
             }
             tc_fence_before();
-            mbar_arrive(p_full);
+            mbar_arrive(p_full + b);
         }
         // ---- output: O / l for valid rows
         // every product done (the MMA warp's single-use end-of-kernel commit)

@@ -106,6 +106,23 @@ def test_prefill_of_single_tokens_equals_decode(pa):
     assert_attention_close(out, _ref(c), torch.bfloat16, "prefill vs oracle")
 
 
+@pytest.mark.parametrize("G", [1, 2, 4])
+def test_prefill_repeated_runs_are_bitwise_identical(pa, G):
+    """The kernel's arithmetic order is fixed (same MMAs, same per-row softmax),
+    so every run on the same input gives the same bits. A hand-off between the
+    load, MMA and softmax warps that lets one warp's tile overtake another's
+    shows up here as a run that differs, or as NaN from the poisoned slots."""
+    c = _case(11 + G, [1500, 700, 300], [1400, 640, 300], 8 * G, 8, 16, torch.bfloat16)
+    pa.pa_read_device_errors()  # clear what earlier tests left
+    first = _run(pa, c, torch.float32)
+    assert torch.isfinite(first).all()
+    for _ in range(8):
+        again = _run(pa, c, torch.float32)
+        assert torch.equal(again, first)
+    assert pa.pa_read_device_errors() == 0
+    assert_attention_close(first, _ref(c), torch.bfloat16, f"G = {G}")
+
+
 def test_prefill_rejects_queries_longer_than_context(pa):
     c = _case(10, [30, 50], [30, 10], 8, 8, 16, torch.float16, poison=False)
     c["ctx"] = torch.tensor([20, 50], dtype=torch.int32)   # sequence 0: 30 queries over 20 tokens
