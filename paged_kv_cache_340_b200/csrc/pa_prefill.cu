@@ -176,14 +176,15 @@ __device__ __forceinline__ void umma_ta(uint32_t d_tmem, uint32_t a_tmem, uint64
         : "memory");
 }
 
-// 32 consecutive outputs of one row, as 16-byte stores.
-__device__ __forceinline__ void store_row32(void *base, size_t idx, const float (&v)[32], pa_dtype dt) {
+// 32 consecutive outputs of one row in the output type, as 16-byte stores at
+// `dst` (global or shared memory, 16-byte aligned).
+__device__ __forceinline__ void store_row32(unsigned char *dst, const float (&v)[32], pa_dtype dt) {
     if (dt == PA_F32) {
-        float4 *d = reinterpret_cast<float4 *>(static_cast<float *>(base) + idx);
+        float4 *d = reinterpret_cast<float4 *>(dst);
 #pragma unroll
         for (int e = 0; e < 8; ++e) d[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
     } else if (dt == PA_BF16) {
-        uint4 *d = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(base) + idx);
+        uint4 *d = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             uint32_t w[4];
@@ -192,7 +193,7 @@ __device__ __forceinline__ void store_row32(void *base, size_t idx, const float 
             d[e] = make_uint4(w[0], w[1], w[2], w[3]);
         }
     } else {
-        uint4 *d = reinterpret_cast<uint4 *>(static_cast<__half *>(base) + idx);
+        uint4 *d = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             uint32_t w[4];
@@ -201,6 +202,21 @@ __device__ __forceinline__ void store_row32(void *base, size_t idx, const float 
             d[e] = make_uint4(w[0], w[1], w[2], w[3]);
         }
     }
+}
+
+// Barrier over the softmax warps only (named barrier 1): true when `v` holds
+// in every one of their threads.
+__device__ __forceinline__ bool softmax_sync_and(bool v) {
+    uint32_t all;
+    asm volatile(
+        "{\n\t.reg .pred pv, pa;\n\t"
+        "setp.ne.u32 pv, %1, 0;\n\t"
+        "barrier.cta.red.and.pred pa, 1, %2, pv;\n\t"
+        "selp.u32 %0, 1, 0, pa;\n\t}"
+        : "=r"(all)
+        : "r"((uint32_t)v), "n"(kSoftmaxWarps * 32)
+        : "memory");
+    return all != 0;
 }
 
 template <typename T, int G>
@@ -255,20 +271,51 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int pos_max = pos0 + rows_valid / G - 1;
     const int ntiles = pos_max / kN + 1;
 
-    if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(k_full + i, 1);
-            mbar_init(v_full + i, 1);
-            mbar_init(k_empty + i, 1);
-            mbar_init(v_empty + i, 1);
-            mbar_init(s_full + i, 1);
-            mbar_init(p_full + i, kSoftmaxWarps * 32);
+    // Pool row of the load warp's 16-token group g0 + lane (16 tokens from
+    // (g0 + lane) * 16), past the pool's end when the sequence has no such
+    // block (the copy then reads zeros).
+    const int32_t *trow = p.block_tables + (size_t)s * p.max_blocks_per_seq;
+    const int nblk = (ctx + p.block_size - 1) / p.block_size;
+    auto rows_from = [&](int g0) -> int {
+        const int g = g0 + lane;
+        const int tok = g * 16;
+        const int lb = tok / p.block_size;
+        long long row = p.kv_rows;
+        if (lb < nblk) {
+            const int id = __ldg(trow + lb);
+            if (id >= 0 && id < p.num_blocks)
+                row = ((long long)id * p.num_kv_heads + kvh) * p.block_size + (tok % p.block_size);
+            else
+                record_error(p.err, PA_DEVERR_BLOCK_ID);
         }
-        mbar_init(o_done, 1);
-        mbar_init(mma_idle, 1);
-        *abort_flag = 0;
-        fence_mbar_init();
+        return (int)row;
+    };
+    // The load warp starts its first table lookups and the Q copy before the
+    // tensor-memory allocation and the CTA barrier, so their latency overlaps
+    // the setup.
+    int rows = 0, rows_next = 0;  // pool rows of groups g0 .. g0 + 31 and of the next 32
+    if (warp == kLoadWarp) {
+        rows = rows_from(0);
+        rows_next = rows_from(32);
+        if (lane == 0) {
+            mbar_init(q_full, 1);
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(k_full + i, 1);
+                mbar_init(v_full + i, 1);
+                mbar_init(k_empty + i, 1);
+                mbar_init(v_empty + i, 1);
+                mbar_init(s_full + i, 1);
+                mbar_init(p_full + i, kSoftmaxWarps * 32);
+            }
+            mbar_init(o_done, 1);
+            mbar_init(mma_idle, 1);
+            *abort_flag = 0;
+            fence_mbar_init();
+            fence_proxy_async_smem();  // the initialised barriers, before the copy that signals one
+            mbar_arrive_expect_tx(q_full, kQBytes);
+            tma_load_3d(Qs, &tmap_q, 0, kvh * G, q0 + tok0, q_full);
+            tma_load_3d(Qs + kQHalf, &tmap_q, 64, kvh * G, q0 + tok0, q_full);
+        }
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -288,37 +335,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         // stage is refilled once the S (K) or PV (V) product that read it is
         // done. Block ids of 32 16-token groups are looked up at a time, one
         // per lane.
-        const int32_t *trow = p.block_tables + (size_t)s * p.max_blocks_per_seq;
-        const int nblk = (ctx + p.block_size - 1) / p.block_size;
-        // Pool row of group g (16 tokens from g * 16), past the pool's end when
-        // the sequence has no such block (the copy then reads zeros).
-        auto rows_from = [&](int g0) -> int {
-            const int g = g0 + lane;
-            const int tok = g * 16;
-            const int lb = tok / p.block_size;
-            long long row = p.kv_rows;
-            if (lb < nblk) {
-                const int id = __ldg(trow + lb);
-                if (id >= 0 && id < p.num_blocks)
-                    row = ((long long)id * p.num_kv_heads + kvh) * p.block_size + (tok % p.block_size);
-                else
-                    record_error(p.err, PA_DEVERR_BLOCK_ID);
-            }
-            return (int)row;
-        };
-        if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, kQBytes);
-            tma_load_3d(Qs, &tmap_q, 0, kvh * G, q0 + tok0, q_full);
-            tma_load_3d(Qs + kQHalf, &tmap_q, 64, kvh * G, q0 + tok0, q_full);
-        }
         constexpr int kGroups = kN / 16;  // 16-token groups per tile
-        int rows = rows_from(0);
         int k_issued = 0, v_issued = 0;
         bool ok = true;
         for (int j = 0; j < ntiles && ok; ++j) {
             const int b = j & 1;
             const int g0 = j * kGroups;
-            if (g0 % 32 == 0 && j > 0) rows = rows_from(g0);
+            if (g0 % 32 == 0 && j > 0) {  // the lookups for the next 32 groups start a batch ahead
+                rows = rows_next;
+                rows_next = rows_from(g0 + 32);
+            }
             int r4[kGroups];
 #pragma unroll
             for (int g = 0; g < kGroups; ++g) r4[g] = __shfl_sync(0xffffffffu, rows, (g0 + g) % 32);
@@ -535,21 +561,63 @@ __global__ void __launch_bounds__(kThreads, 2)
         // every product done (the MMA warp's single-use end-of-kernel commit)
         const bool done = __all_sync(0xffffffffu, mbar_wait(mma_idle, 0) && !*(volatile int *)abort_flag);
         tc_fence_after();
-        if (!done) {
-            if (r == 0) record_error(p.err, PA_DEVERR_TIMEOUT);
-        } else {
-            const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-            const size_t orow = ((size_t)(q0 + tok0 + tok) * p.num_heads + (size_t)kvh * G + (r % G)) * kD;
+        // Each thread holds O of its row in tensor-memory lane r. For G <= 2 it
+        // writes O / l in the output type into shared memory (the Q, K and V
+        // tiles are dead once every product is done; the row pitch is padded by
+        // 16 bytes so the 32 rows of a warp's store fall in different banks),
+        // then the four softmax warps copy whole rows out, so consecutive lanes
+        // store consecutive 16 bytes of one output row; rows from rows_valid on
+        // belong to no query and are not written. For G >= 4 each thread stores
+        // its own row directly, which measured faster there (the staged form
+        // measured 2 % slower on the 4-head-group chunked-prefill workload and
+        // 4 % faster on the MHA prompt workload).
+        const int ebytes = p.out_dtype == PA_F32 ? 4 : 2;
+        const int row_bytes = kD * ebytes;
+        const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+        if constexpr (G <= 2) {
+            if (done) {
+                unsigned char *srow = Qs + r * (row_bytes + 16);
 #pragma unroll
-            for (int ch = 0; ch < kD / 32; ++ch) {
-                uint32_t o[32];
-                tmem_ld32(tmem + lane_base + kOCol + ch * 32, o);
-                tmem_wait_ld();
-                if (valid) {
+                for (int ch = 0; ch < kD / 32; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_base + kOCol + ch * 32, o);
+                    tmem_wait_ld();
                     float v[32];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * inv;
-                    store_row32(p.out, orow + ch * 32, v, p.out_dtype);
+                    store_row32(srow + ch * 32 * ebytes, v, p.out_dtype);
+                }
+            }
+            // all four softmax warps arrive here whatever their outcome
+            if (!softmax_sync_and(done)) {
+                if (r == 0) record_error(p.err, PA_DEVERR_TIMEOUT);
+            } else {
+                const int cpr = row_bytes / 16;  // 16-byte pieces per row
+                unsigned char *out = static_cast<unsigned char *>(p.out);
+                for (int i = r; i < rows_valid * cpr; i += kSoftmaxWarps * 32) {
+                    const int row = i / cpr, c = i % cpr;
+                    const size_t orow = (size_t)(q0 + tok0 + row / G) * p.num_heads + (size_t)kvh * G + (row % G);
+                    *reinterpret_cast<uint4 *>(out + orow * row_bytes + c * 16) =
+                        *reinterpret_cast<const uint4 *>(Qs + row * (row_bytes + 16) + c * 16);
+                }
+            }
+        } else {
+            if (!done) {
+                if (r == 0) record_error(p.err, PA_DEVERR_TIMEOUT);
+            } else {
+                const size_t orow = (size_t)(q0 + tok0 + tok) * p.num_heads + (size_t)kvh * G + (r % G);
+                unsigned char *dst = static_cast<unsigned char *>(p.out) + orow * row_bytes;
+#pragma unroll
+                for (int ch = 0; ch < kD / 32; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_base + kOCol + ch * 32, o);
+                    tmem_wait_ld();
+                    if (valid) {
+                        float v[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * inv;
+                        store_row32(dst + ch * 32 * ebytes, v, p.out_dtype);
+                    }
                 }
             }
         }
