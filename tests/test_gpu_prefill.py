@@ -85,11 +85,12 @@ def test_prefill_matches_oracle(pa, dtype, case):
     assert_attention_close(out, _ref(c), dtype, f"prefill case {case} {dtype}")
 
 
-def test_prefill_16bit_output(pa):
-    c = _case(7, [150, 60], [150, 10], 8, 2, 16, torch.bfloat16)
+@pytest.mark.parametrize("Hkv", [8, 4, 2])  # head groups 1, 2 (rows staged in shared memory), 4 (rows stored directly)
+def test_prefill_16bit_output(pa, Hkv):
+    c = _case(7, [150, 60], [150, 10], 8, Hkv, 16, torch.bfloat16)
     out = _run(pa, c, torch.bfloat16)
     assert_attention_close(out, _ref(c), torch.bfloat16, "bf16 out")
-    c = _case(8, [150, 60], [150, 10], 8, 2, 16, torch.float16)
+    c = _case(8, [150, 60], [150, 10], 8, Hkv, 16, torch.float16)
     out = _run(pa, c, torch.float16)
     assert_attention_close(out, _ref(c), torch.float16, "fp16 out")
 
@@ -133,6 +134,23 @@ def test_prefill_rejects_queries_longer_than_context(pa):
                                c["tables"].numpy()[1:], np.array([50], np.int32), c["scale"], 16)
     assert_attention_close(out[ok:], ref, torch.float16, "valid sequence")
     assert torch.isnan(out[:ok]).all()                       # the skipped sequence is left untouched
+
+
+@pytest.mark.parametrize("Hkv", [8, 4, 2])  # head groups 1, 2 (staged rows), 4 (direct rows)
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_prefill_writes_no_row_past_a_partial_tile(pa, Hkv, out_dtype):
+    """Sequence 0 ends inside its query tile; the rows after it belong to
+    sequence 1, which the kernel skips (more queries than context). They must
+    keep the NaN they were filled with."""
+    c = _case(12, [40, 50], [10, 30], 8, Hkv, 16, torch.bfloat16, poison=False)
+    c["ctx"] = torch.tensor([40, 20], dtype=torch.int32)     # sequence 1: 30 queries over 20 tokens
+    pa.pa_read_device_errors()
+    out = _run(pa, c, out_dtype)
+    assert pa.pa_read_device_errors() & pa.PA_DEVERR_CONTEXT
+    ref = oracle.paged_prefill(f64(c["q"][:10]), np.array([0, 10], np.int32), f64(c["k"]), f64(c["v"]),
+                               c["tables"].numpy()[:1], np.array([40], np.int32), c["scale"], 16)
+    assert_attention_close(out[:10], ref, torch.bfloat16, "sequence 0")
+    assert torch.isnan(out[10:].float()).all()
 
 
 @pytest.mark.parametrize("name", ["prefill_llama7b_mha_bf16", "chunked_prefill_gqa_bf16"])
