@@ -212,6 +212,23 @@ struct StepParams {
 
 __device__ __forceinline__ int nblk(int ctx, int bs) { return (ctx + bs - 1) / bs; }
 
+// Beam j and table position pos of the flattened entries e0, e0 + stride, ...
+// of [beams][mb] tables: one division, then per step one add and at most one
+// carry (the step's remainder is below mb). The passes below visit 16 entries
+// per thread; a division per entry cost more than the memory traffic.
+struct EntryWalk {
+    int j, pos;
+    __device__ __forceinline__ EntryWalk(int e0, int mb) : j(e0 / mb), pos(e0 % mb) {}
+    __device__ __forceinline__ void step(int dj, int dpos, int mb) {
+        j += dj;
+        pos += dpos;
+        if (pos >= mb) {
+            pos -= mb;
+            ++j;
+        }
+    }
+};
+
 // The kernel is latency-bound (one CTA, dependent loads), so every pass over
 // table entries first loads kItems entries per thread into registers, then
 // acts on them: one or two memory round trips per pass instead of one per
@@ -229,6 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
     const int n_old = q.num_old, n_new = q.num_new;
     const int old_entries = n_old * MB;  // < 2^31 (host check)
     const int new_entries = n_new * MB;
+    const int sdj = kThreads / MB, sdp = kThreads % MB;  // a step of kThreads entries
     int *s_ctx = dyn;                    // [n_old] context length of old beam j
     int *s_nb = dyn + n_old;             // [n_old] its block count
     int *s_nch = dyn + 2 * n_old;        // [n_old] its number of children
@@ -284,17 +302,16 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
     if (!s_bad) {
         for (int base = 0; base < old_entries; base += kThreads * kItems) {
             int blk[kItems], in_use = 0;
+            EntryWalk w(base + tid, MB);
 #pragma unroll
             for (int k = 0; k < kItems; ++k) {
                 const int e = base + k * kThreads + tid;
                 blk[k] = 0;
-                if (e < old_entries) {
-                    const int j = e / MB;
-                    if (e - j * MB < s_nb[j]) {
-                        blk[k] = tab(e);
-                        in_use |= 1 << k;
-                    }
+                if (e < old_entries && w.pos < s_nb[w.j]) {
+                    blk[k] = tab(e);
+                    in_use |= 1 << k;
                 }
+                w.step(sdj, sdp, MB);
             }
 #pragma unroll
             for (int k = 0; k < kItems; ++k) {
@@ -320,21 +337,19 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
     // with other than one child touch the counts. Then the writers.
     for (int base = 0; base < old_entries; base += kThreads * kItems) {
         int blk[kItems];
+        EntryWalk w(base + tid, MB);
 #pragma unroll
         for (int k = 0; k < kItems; ++k) {
             const int e = base + k * kThreads + tid;
             blk[k] = -1;
-            if (e < old_entries) {
-                const int j = e / MB;
-                if (e - j * MB < s_nb[j] && s_nch[j] != 1) blk[k] = tab(e);
-            }
+            if (e < old_entries && w.pos < s_nb[w.j] && s_nch[w.j] != 1) blk[k] = tab(e);
+            w.step(sdj, sdp, MB);
         }
+        EntryWalk w2(base + tid, MB);
 #pragma unroll
         for (int k = 0; k < kItems; ++k) {
-            if (blk[k] >= 0) {
-                const int e = base + k * kThreads + tid;
-                atomicAdd(&p.delta[blk[k]], s_nch[e / MB] - 1);
-            }
+            if (blk[k] >= 0) atomicAdd(&p.delta[blk[k]], s_nch[w2.j] - 1);
+            w2.step(sdj, sdp, MB);
         }
     }
     for (int i = tid; i < n_new; i += kThreads) {
@@ -351,14 +366,13 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
     // the last such entry (in release order) of each block reaching zero
     for (int base = 0; base < old_entries; base += kThreads * kItems) {
         int blk[kItems], r0[kItems];
+        EntryWalk w(base + tid, MB);
 #pragma unroll
         for (int k = 0; k < kItems; ++k) {
             const int e = base + k * kThreads + tid;
             blk[k] = -1;
-            if (e < old_entries) {
-                const int j = e / MB;
-                if (e - j * MB < s_nb[j] && s_nch[j] == 0) blk[k] = tab(e);
-            }
+            if (e < old_entries && w.pos < s_nb[w.j] && s_nch[w.j] == 0) blk[k] = tab(e);
+            w.step(sdj, sdp, MB);
         }
 #pragma unroll
         for (int k = 0; k < kItems; ++k)
@@ -380,14 +394,13 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
     int freed = 0;
     for (int base = 0; base < old_entries; base += kThreads * kScanItems) {
         int blk[kScanItems], r0[kScanItems], d0[kScanItems], l0[kScanItems];
+        EntryWalk w(base + tid * kScanItems, MB);
 #pragma unroll
         for (int k = 0; k < kScanItems; ++k) {
             const int e = base + tid * kScanItems + k;
             blk[k] = -1;
-            if (e < old_entries) {
-                const int j = e / MB;
-                if (e - j * MB < s_nb[j] && s_nch[j] == 0) blk[k] = tab(e);
-            }
+            if (e < old_entries && w.pos < s_nb[w.j] && s_nch[w.j] == 0) blk[k] = tab(e);
+            w.step(MB == 1 ? 1 : 0, MB == 1 ? 0 : 1, MB);
         }
 #pragma unroll
         for (int k = 0; k < kScanItems; ++k) {
@@ -446,20 +459,22 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
     // delta out), reset the release marks
     for (int base = 0; base < old_entries; base += kThreads * kItems) {
         int blk[kItems];
+        EntryWalk w(base + tid, MB);
 #pragma unroll
         for (int k = 0; k < kItems; ++k) {
             const int e = base + k * kThreads + tid;
             blk[k] = -1;
-            if (e < old_entries) {
-                const int j = e / MB;
-                if (e - j * MB < s_nb[j] && s_nch[j] != 1) blk[k] = tab(e);
-            }
+            if (e < old_entries && w.pos < s_nb[w.j] && s_nch[w.j] != 1) blk[k] = tab(e);
+            w.step(sdj, sdp, MB);
         }
+        EntryWalk w2(base + tid, MB);
 #pragma unroll
         for (int k = 0; k < kItems; ++k) {
+            const int jk = w2.j;
+            w2.step(sdj, sdp, MB);
             if (blk[k] >= 0) {
                 const int b = blk[k];
-                if (s_nch[(base + k * kThreads + tid) / MB] == 0) p.last_old[b] = -1;
+                if (s_nch[jk] == 0) p.last_old[b] = -1;
                 const int d = atomicExch(&p.delta[b], 0);
                 if (ok && d) p.ref[b] += d;
             }
@@ -471,15 +486,16 @@ __global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams
         // ---- phase 5: the new tables (parent rows, -1 past the blocks in use)
         for (int base = 0; base < new_entries; base += kThreads * kItems) {
             int v[kItems];
+            EntryWalk w(base + tid, MB);
 #pragma unroll
             for (int k = 0; k < kItems; ++k) {
                 const int e = base + k * kThreads + tid;
                 v[k] = -1;
                 if (e < new_entries) {
-                    const int i = e / MB, pos = e - i * MB;
-                    const int par = s_par[i];
-                    if (pos < s_nb[par]) v[k] = tab(par * MB + pos);
+                    const int par = s_par[w.j];
+                    if (w.pos < s_nb[par]) v[k] = tab(par * MB + w.pos);
                 }
+                w.step(sdj, sdp, MB);
             }
 #pragma unroll
             for (int k = 0; k < kItems; ++k) {
