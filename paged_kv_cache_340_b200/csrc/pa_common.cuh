@@ -163,7 +163,7 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
 
 // One-dimensional bulk copy global -> this CTA's shared memory (TMA engine),
 // completing `bytes` on the mbarrier. dst, src and bytes are multiples of 16.
-// No multicast.
+// The copy lands in this CTA alone.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
                                           uint64_t *bar, uint64_t policy) {
     asm volatile(

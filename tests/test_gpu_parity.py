@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from _helpers import (assert_attention_close, compact_for, f64, oracle_decode_tables, oracle_sampling_flow, raw)
+from _helpers import assert_attention_close, f64, oracle_decode_tables, raw
 
 pytestmark = pytest.mark.gpu
 
