@@ -3,7 +3,10 @@
 A step is one pass of the hot path over one synthetic batch: the copy-on-write
 block copies the batch needs (none for the decode-only workloads), the slot
 write of the step's new tokens, and decode (split-K plus its reduce when the
-partition rule splits the batch). The default workload is the LLaMA-7B-shaped
+partition rule splits the batch). When the step writes only each sequence's
+newest token and decodes unsplit from a 16- or 32-bit cache, the slot write
+and decode run as one launch (pa_decode_append); the bytes counted are the
+same. The default workload is the LLaMA-7B-shaped
 fp16 decode layer (64 sequences, 32 heads, head_dim 128, block 16, context
 lengths U{256..2048}).
 
@@ -223,6 +226,8 @@ def step_bytes(spec, b) -> dict:
 
 
 def launches_per_step(b) -> int:
+    if b.fused_append:
+        return (1 if b.cow_pairs.shape[0] else 0) + 1
     return (1 if b.cow_pairs.shape[0] else 0) + 1 + (2 if b.partition_size else 1)
 
 
@@ -230,8 +235,9 @@ def time_steps(b, steps: int, warmup: int, world: int, sample_clocks=False, devi
     """Device time per step over `steps` steps (max over ranks), and the mean
     duration of each kernel of the step (a second pass with CUDA events
     around every launch, on the launching stream)."""
-    from paged_kv_cache_340_b200 import pa_copy_blocks, pa_copy_blocks_q8, pa_decode, pa_decode_q8, \
-        pa_decode_splitk, pa_decode_splitk_q8, pa_reshape_and_cache, pa_reshape_and_cache_q8, pa_splitk_reduce
+    from paged_kv_cache_340_b200 import pa_copy_blocks, pa_copy_blocks_q8, pa_decode, pa_decode_append, \
+        pa_decode_q8, pa_decode_splitk, pa_decode_splitk_q8, pa_reshape_and_cache, pa_reshape_and_cache_q8, \
+        pa_splitk_reduce
     spec = b.spec
     stream = torch.cuda.current_stream()
 
@@ -264,6 +270,13 @@ def time_steps(b, steps: int, warmup: int, world: int, sample_clocks=False, devi
         if b.cow_pairs.shape[0]:
             pa_copy_blocks(b.k_cache, b.v_cache, b.cow_pairs, stream=stream)
         mark(ev, 1)
+        if b.fused_append:  # slot write and decode in one launch
+            mark(ev, 2)
+            pa_decode_append(b.out, b.query, b.new_key, b.new_value, b.k_cache, b.v_cache, b.block_tables,
+                             b.context_lens, spec.scale, seq_order=b.seq_order, stream=stream)
+            mark(ev, 3)
+            mark(ev, 4)
+            return
         pa_reshape_and_cache(b.new_key, b.new_value, b.k_cache, b.v_cache, b.slot_mapping, stream=stream)
         mark(ev, 2)
         if b.partition_size:
@@ -305,7 +318,10 @@ def time_steps(b, steps: int, warmup: int, world: int, sample_clocks=False, devi
     def mean(i, j):
         return statistics.fmean(e[i].elapsed_time(e[j]) for e in evs)
 
-    kernels = {"reshape_and_cache": mean(1, 2), "decode": mean(2, 3)}
+    if b.fused_append:
+        kernels = {"decode_append": mean(2, 3)}
+    else:
+        kernels = {"reshape_and_cache": mean(1, 2), "decode": mean(2, 3)}
     if b.cow_pairs.shape[0]:
         kernels["copy_blocks"] = mean(0, 1)
     if b.partition_size:
@@ -430,7 +446,8 @@ def run_reference(args, world, rank):
 
 def kernel_lines(spec, b, kern: dict, by: dict) -> dict:
     """Per kernel of the step: mean launch time and algorithmic GB/s."""
-    nbytes = {"decode": by["decode"], "reshape_and_cache": by["write"], "copy_blocks": by["copy"]}
+    nbytes = {"decode": by["decode"], "reshape_and_cache": by["write"], "copy_blocks": by["copy"],
+              "decode_append": by["decode"] + by["write"]}
     if b.partition_size:
         parts = ((b.host_context_lens.astype(np.int64) + b.partition_size - 1) // b.partition_size).sum()
         nbytes["splitk_reduce"] = int(parts) * spec.num_heads * (spec.head_dim + 2) * 4 + \
@@ -601,15 +618,24 @@ def measure_beam(name: str, steps: int, warmup: int, host_steps: int = 30):
     return res
 
 
+def decode_kernel_of(b, by: dict):
+    """The step's decode kernel: its name in the kernel timings and the
+    algorithmic bytes it moves (the fused form also does the slot write)."""
+    if b.fused_append:
+        return "decode_append", by["decode"] + by["write"]
+    return "decode", by["decode"]
+
+
 def measure_other(name: str, steps: int, warmup: int):
     spec, b = build_batch(name, 0)
     ms, kern, _ = time_steps(b, steps, warmup, 1)
     by = step_bytes(spec, b)
     peak, _ = peaks()
-    dec = kern["decode"]
+    dname, dbytes = decode_kernel_of(b, by)
+    dec = kern[dname]
     res = {"ms_per_step": round(ms, 4), "GBps": round(by["total"] / ms / 1e6, 1),
            "pct_of_hbm_peak": round(100 * by["total"] / ms / 1e6 / peak, 1),
-           "decode_kernel_ms": round(dec, 4), "decode_kernel_GBps": round(by["decode"] / dec / 1e6, 1),
+           "decode_kernel_ms": round(dec, 4), "decode_kernel_GBps": round(dbytes / dec / 1e6, 1),
            "partition_size": b.partition_size, "seq_tokens_per_s": round(spec.num_seqs / ms * 1e3, 1),
            "context_tokens_per_s": round(float(b.host_context_lens.sum()) / ms * 1e3, 1),
            "kernels": kernel_lines(spec, b, kern, by)}
@@ -655,13 +681,14 @@ def main():
     spec, b = build_batch(args.workload, rank, args.partition)
     ms, kern, clocks = time_steps(b, args.steps, args.warmup, world, sample_clocks=(rank == 0),
                                   device_index=local)
-    dec_ms = kern["decode"]
     by = step_bytes(spec, b)
+    dname, dbytes = decode_kernel_of(b, by)
+    dec_ms = kern[dname]
     peak, peak_kind = peaks()
     value = pdist.job_throughput(by["total"], ms, world)
     e2e_ms, h2d, d2h = e2e_steps(b, max(10, args.steps // 4), args.warmup, world)
-    kernel = "pa_decode_splitk" if b.partition_size else "pa_decode"
-    achieved = by["decode"] / (dec_ms * 1e-3) / 1e9
+    kernel = "pa_decode_splitk" if b.partition_size else ("pa_decode_append" if b.fused_append else "pa_decode")
+    achieved = dbytes / (dec_ms * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
@@ -672,7 +699,9 @@ def main():
                    "kv_dtype": spec.kv_dtype, "out_dtype": spec.out_dtype, "partition_size": b.partition_size,
                    "parallelism": f"dp{world} (sequences shard, no exchange)",
                    "l2": "inputs larger than L2 (K/V >= 1.2 GB per step), no flush",
-                   "step": "copy_blocks (if any) + reshape_and_cache + decode"},
+                   "step": ("copy_blocks (if any) + decode_append (slot write of each sequence's newest token "
+                            "and decode, one launch)" if b.fused_append else
+                            "copy_blocks (if any) + reshape_and_cache + decode")},
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "seq_tokens_per_s": round(world * spec.num_seqs / (ms * 1e-3), 1),
         "context_tokens_per_s": round(world * float(b.host_context_lens.sum()) / (ms * 1e-3), 1),

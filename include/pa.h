@@ -135,6 +135,29 @@ int pa_decode(void *out, const void *query, const void *k_cache, const void *v_c
               const int32_t *seq_order, cudaStream_t stream);
 
 /*
+ * pa_decode_append -- pa_reshape_and_cache of each sequence's newest token
+ * followed by pa_decode, in one launch. The newest token of sequence s is at
+ * position L - 1 (L = context_lens[s] >= 1, the new token counted): its rows
+ * new_key[s, :, :] and new_value[s, :, :] ([num_seqs, num_kv_heads,
+ * head_dim], dtype kv_dtype, device, 16-byte aligned) are written into the
+ * slot block_tables[s][(L - 1) / block_size] * block_size + (L - 1) %
+ * block_size of k_cache / v_cache, and the attention uses them for t = L - 1.
+ * The result (pools and out) is that of the two calls in sequence, provided no
+ * other sequence of the call reads that block (true once copy-on-write has
+ * given each sequence its own last block). L == 0 writes nothing and outputs
+ * zeros; a table entry out of range skips the block (PA_DEVERR_BLOCK_ID) and
+ * writes nothing for it. Arguments otherwise as pa_decode. [P4] §3.4 (the
+ * runner writes each new token's K/V into its block, then attention reads the
+ * cache); the fusion is this library's: the warp whose 16-token stage holds
+ * position L - 1 puts the new row over its landed tile before using it.
+ */
+int pa_decode_append(void *out, const void *query, const void *new_key, const void *new_value, void *k_cache,
+                     void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                     const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                     float scale, int block_size, int num_blocks, pa_dtype kv_dtype, pa_dtype out_dtype,
+                     const int32_t *seq_order, cudaStream_t stream);
+
+/*
  * Split-K (partitioned) decode for few, long sequences ([P5] §2.3: the
  * partitioned kernel of the pair). Tokens of sequence s are cut into
  * partitions of `partition_size` tokens (a multiple of block_size); partition

@@ -53,7 +53,7 @@ EXPORTED = (
     "pa_prefix_cache_create", "pa_prefix_cache_destroy", "pa_prefix_num_entries", "pa_prefix_get_or_create",
     "pa_prefix_release", "pa_prefix_ref_count", "pa_copy_blocks_counted", "pa_dpool_state_bytes", "pa_dpool_init",
     "pa_beam_step", "pa_pool_export", "pa_dpool_load", "pa_reshape_and_cache_q8", "pa_decode_q8",
-    "pa_decode_splitk_q8", "pa_copy_blocks_q8",
+    "pa_decode_splitk_q8", "pa_copy_blocks_q8", "pa_decode_append",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -77,6 +77,8 @@ def _load() -> ctypes.CDLL:
         "pa_read_device_errors": (i32, [ctypes.POINTER(ctypes.c_uint32), vp]),
         "pa_reshape_and_cache": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
         "pa_decode": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32, vp, vp]),
+        "pa_decode_append": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32,
+                                   vp, vp]),
         "pa_splitk_workspace_bytes": (sz, [i32, i32, i32, i32, i32]),
         "pa_splitk_acc_offset": (sz, [i32, i32, i32, i32]),
         "pa_decode_splitk": (i32, [vp, sz, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32,
@@ -190,6 +192,19 @@ def pa_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale, s
                         block_tables.shape[1], _ptr(context_lens), S, Hq, Hkv, D, float(scale), bs, NB,
                         _dtype(k_cache), _dtype(out), _ptr(seq_order), _stream(stream))
     _check(rc, "pa_decode")
+
+
+def pa_decode_append(out, query, new_key, new_value, k_cache, v_cache, block_tables, context_lens, scale,
+                     seq_order=None, stream=None) -> None:
+    """Writes new_key / new_value [S, Hkv, D] as token context_lens[s] - 1 of
+    each sequence (into the slot its table gives), then decodes: one launch."""
+    S, Hq, D = query.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    rc = _lib.pa_decode_append(_ptr(out), _ptr(query), _ptr(new_key), _ptr(new_value), _ptr(k_cache),
+                               _ptr(v_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S, Hq,
+                               Hkv, D, float(scale), bs, NB, _dtype(k_cache), _dtype(out), _ptr(seq_order),
+                               _stream(stream))
+    _check(rc, "pa_decode_append")
 
 
 def pa_splitk_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, partition_size) -> int:

@@ -16,7 +16,7 @@ import numpy as np
 import torch
 
 from . import (PA_POOL_FIFO, BlockPool, DevicePool, pa_beam_step, pa_choose_partition, pa_copy_blocks,
-               pa_copy_blocks_counted, pa_copy_blocks_q8, pa_decode, pa_decode_q8, pa_decode_splitk,
+               pa_copy_blocks_counted, pa_copy_blocks_q8, pa_decode, pa_decode_append, pa_decode_q8, pa_decode_splitk,
                pa_decode_splitk_q8, pa_prefill, pa_reshape_and_cache, pa_reshape_and_cache_q8, pa_splitk_reduce,
                pa_splitk_workspace_bytes)
 from .workloads import Spec
@@ -46,6 +46,10 @@ class DecodeBatch:
     host_context_lens: np.ndarray
     k_scale: Optional[torch.Tensor] = None  # int8 caches: device float32 [NB, Hkv, bs] row scales
     v_scale: Optional[torch.Tensor] = None
+    # the step writes exactly each sequence's newest token, into the slot its
+    # table gives, and decodes unpartitioned from a 16- or 32-bit cache: the
+    # slot write and decode then run as one launch (pa_decode_append)
+    fused_append: bool = False
 
 
 def _blocks(n: int, bs: int) -> int:
@@ -110,7 +114,18 @@ def build_decode_batch(spec: Spec, inputs: dict, device="cuda", partition_size: 
         cow_pairs=torch.empty((0, 2), dtype=torch.int64, device=dev),
         seq_order=torch.from_numpy(longest_first(ctx)).to(dev),
         max_context_len=max_ctx, partition_size=int(partition_size), workspace=ws,
-        host_tables=tables, host_slots=slots, host_cow=np.empty((0, 2), np.int64), host_context_lens=ctx)
+        host_tables=tables, host_slots=slots, host_cow=np.empty((0, 2), np.int64), host_context_lens=ctx,
+        fused_append=bool(partition_size == 0 and spec.kv_dtype != "i8" and newest_token_slots(tables, ctx, bs, slots)))
+
+
+def newest_token_slots(tables: np.ndarray, ctx: np.ndarray, bs: int, slots: np.ndarray) -> bool:
+    """Whether slots[s] is the slot of token ctx[s] - 1 of every sequence (as
+    its table gives it), the case pa_decode_append covers."""
+    if slots.shape[0] != ctx.shape[0] or (ctx < 1).any():
+        return False
+    pos = ctx.astype(np.int64) - 1
+    blk = tables[np.arange(ctx.shape[0]), pos // bs].astype(np.int64)
+    return bool(np.array_equal(blk * bs + pos % bs, slots.astype(np.int64)))
 
 
 @dataclass
@@ -210,7 +225,9 @@ def quantized_pool(k_pool: torch.Tensor, v_pool: torch.Tensor, device, chunk_blo
 def run_step(batch: DecodeBatch, stream=None) -> None:
     """One pass of the hot path: copy-on-write block copies (if any), the slot
     write of this step's tokens, then decode (split-K + reduce when the batch
-    has a partition size). int8 caches quantize at the slot write."""
+    has a partition size). int8 caches quantize at the slot write. When the
+    step writes only each sequence's newest token (fused_append), the slot
+    write and decode are one launch."""
     q8 = batch.k_scale is not None
     if batch.cow_pairs.shape[0]:
         if q8:
@@ -218,6 +235,11 @@ def run_step(batch: DecodeBatch, stream=None) -> None:
                               stream=stream)
         else:
             pa_copy_blocks(batch.k_cache, batch.v_cache, batch.cow_pairs, stream=stream)
+    if batch.fused_append:
+        pa_decode_append(batch.out, batch.query, batch.new_key, batch.new_value, batch.k_cache, batch.v_cache,
+                         batch.block_tables, batch.context_lens, batch.spec.scale, seq_order=batch.seq_order,
+                         stream=stream)
+        return
     if q8:
         pa_reshape_and_cache_q8(batch.new_key, batch.new_value, batch.k_cache, batch.v_cache, batch.k_scale,
                                 batch.v_scale, batch.slot_mapping, stream=stream)

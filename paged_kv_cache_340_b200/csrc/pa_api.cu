@@ -166,11 +166,11 @@ int pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-int pa_decode(void *out, const void *query, const void *k_cache, const void *v_cache,
-              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
-              int num_seqs, int num_heads, int num_kv_heads, int head_dim, float scale,
-              int block_size, int num_blocks, pa_dtype kv_dtype, pa_dtype out_dtype,
-              const int32_t *seq_order, cudaStream_t stream) {
+static int decode_unsplit(void *out, const void *query, const void *new_key, const void *new_value,
+                          const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                          int max_blocks_per_seq, const int32_t *context_lens, int num_seqs, int num_heads,
+                          int num_kv_heads, int head_dim, float scale, int block_size, int num_blocks,
+                          pa_dtype kv_dtype, pa_dtype out_dtype, const int32_t *seq_order, cudaStream_t stream) {
     int rc = check_decode_args(query, k_cache, v_cache, block_tables, max_blocks_per_seq,
                                context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale,
                                block_size, num_blocks, kv_dtype);
@@ -179,7 +179,7 @@ int pa_decode(void *out, const void *query, const void *k_cache, const void *v_c
     if (num_seqs == 0) return PA_OK;
     if (!aligned(seq_order, 4)) return PA_ERR_ALIGN;
     if (!out) return PA_ERR_NULL;
-    if (!aligned(out, 16)) return PA_ERR_ALIGN;
+    if (!aligned(out, 16) || !aligned(new_key, 16) || !aligned(new_value, 16)) return PA_ERR_ALIGN;
     unsigned int *err = nullptr;
     if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
     DecodeParams p{};
@@ -200,9 +200,32 @@ int pa_decode(void *out, const void *query, const void *k_cache, const void *v_c
     p.max_context_len = INT_MAX;
     p.out_dtype = out_dtype;
     p.err = err;
+    p.new_key = new_key;
+    p.new_value = new_value;
     cudaError_t e = launch_decode(p, kv_dtype, head_dim, block_size, num_heads / num_kv_heads, 1,
                                   num_kv_heads, num_seqs, stream);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_decode(void *out, const void *query, const void *k_cache, const void *v_cache,
+              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+              int num_seqs, int num_heads, int num_kv_heads, int head_dim, float scale,
+              int block_size, int num_blocks, pa_dtype kv_dtype, pa_dtype out_dtype,
+              const int32_t *seq_order, cudaStream_t stream) {
+    return decode_unsplit(out, query, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                          context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale, block_size,
+                          num_blocks, kv_dtype, out_dtype, seq_order, stream);
+}
+
+int pa_decode_append(void *out, const void *query, const void *new_key, const void *new_value, void *k_cache,
+                     void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                     const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                     float scale, int block_size, int num_blocks, pa_dtype kv_dtype, pa_dtype out_dtype,
+                     const int32_t *seq_order, cudaStream_t stream) {
+    if (num_seqs > 0 && (!new_key || !new_value)) return PA_ERR_NULL;
+    return decode_unsplit(out, query, new_key, new_value, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                          context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale, block_size,
+                          num_blocks, kv_dtype, out_dtype, seq_order, stream);
 }
 
 size_t pa_splitk_acc_offset(int num_seqs, int num_heads, int max_context_len, int partition_size) {

@@ -770,8 +770,10 @@ struct MmaConsumerQ8 {
 // -------------------------------------------------------------------- kernel
 
 // T: the cache's element type (int8_t: codes with per-row scales); TQ: the
-// query's type (T for 16- and 32-bit caches).
-template <typename T, int D, int BS, int G, typename TQ = T>
+// query's type (T for 16- and 32-bit caches); kAppend: each sequence's newest
+// token comes from p.new_key / p.new_value (pa_decode_append; 16- and 32-bit
+// caches).
+template <typename T, int D, int BS, int G, typename TQ = T, bool kAppend = false>
 __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShape<T, D, BS, G>::kMinBlocks)
     decode_kernel(const __grid_constant__ DecodeParams p) {
     using S = DecodeShape<T, D, BS, G>;
@@ -882,6 +884,32 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
         if (lane == 0 && m < nmine) issue(m, id);
     }
 
+    // pa_decode_append: the sequence's newest token (position ctx - 1) comes
+    // from new_key / new_value. The warp whose stage k_new holds it loads the
+    // two rows now; once that stage has landed it puts them over the tile
+    // rows (the pool's copy may be stale) and writes them into the pool.
+    static_assert(!(kAppend && S::kInt8), "the append form is for 16- and 32-bit caches");
+    constexpr int kRowChunks = D * S::kElt / 16;  // 16-byte pieces of one K or V row
+    constexpr int kNewPerLane = kAppend ? (2 * kRowChunks + 31) / 32 : 1;
+    int k_new = -1;
+    uint4 nrow[kNewPerLane];
+    if constexpr (kAppend) {
+        if (ctx > 0 && ctx - 1 >= t_begin && ctx - 1 < t_end)
+            k_new = (ctx - 1 - t_begin) / S::kTS;
+        if (k_new >= 0 && k_new % S::kWarps == warp) {
+            const size_t row0 = ((size_t)s * p.num_kv_heads + kvh) * D * S::kElt;  // bytes
+#pragma unroll
+            for (int i = 0; i < kNewPerLane; ++i) {
+                const int c = lane + 32 * i;
+                nrow[i] = make_uint4(0u, 0u, 0u, 0u);
+                if (c < 2 * kRowChunks) {
+                    const unsigned char *src = static_cast<const unsigned char *>(c < kRowChunks ? p.new_key : p.new_value);
+                    nrow[i] = __ldg(reinterpret_cast<const uint4 *>(src + row0) + (c % kRowChunks));
+                }
+            }
+        }
+    }
+
     Consumer cons;
     cons.init(p, head0, warp, lane);
     int waited = 0;
@@ -903,6 +931,28 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
             break;
         }
         waited = m + 1;
+        if constexpr (kAppend) {
+            if (k == k_new) {
+                const int id = id_of(m);  // the stage's block (whole warp)
+                if (!bad[buf]) {
+                    const int r = (ctx - 1 - t_begin) % S::kTS;  // row in the stage
+                    unsigned char *Kw = ring + S::kVRegion + (size_t)buf * S::kStageBytes;
+                    const size_t prow = ((size_t)id * block_elems + (size_t)((ctx - 1) % BS) * D) * S::kElt;
+#pragma unroll
+                    for (int i = 0; i < kNewPerLane; ++i) {
+                        const int c = lane + 32 * i;
+                        if (c < 2 * kRowChunks) {
+                            const bool isv = c >= kRowChunks;
+                            const int cc = c % kRowChunks;
+                            reinterpret_cast<uint4 *>(Kw + (isv ? S::kTileBytes : 0) + (size_t)r * D * S::kElt)[cc] = nrow[i];
+                            const unsigned char *pool = reinterpret_cast<const unsigned char *>(isv ? vc : kc);
+                            reinterpret_cast<uint4 *>(const_cast<unsigned char *>(pool) + prow)[cc] = nrow[i];
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+        }
         if (!bad[buf]) {
             const int nvalid = min(S::kTS, t_end - (t_begin + k * S::kTS));
             const unsigned char *Kb = ring + S::kVRegion + (size_t)buf * S::kStageBytes;
@@ -1037,11 +1087,11 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
 
 // ------------------------------------------------------------------ launchers
 
-template <typename T, int D, int BS, int G, typename TQ = T>
+template <typename T, int D, int BS, int G, typename TQ = T, bool kAppend = false>
 static cudaError_t launch_decode_t(const DecodeParams &p, int grid_x, int num_kv_heads, int num_seqs,
                                    cudaStream_t stream) {
     using S = DecodeShape<T, D, BS, G>;
-    auto kern = decode_kernel<T, D, BS, G, TQ>;
+    auto kern = decode_kernel<T, D, BS, G, TQ, kAppend>;
     static unsigned int attr_done = 0;  // one bit per device
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), S::kSmemBytes, &attr_done);
     if (e != cudaSuccess) return e;
@@ -1050,35 +1100,42 @@ static cudaError_t launch_decode_t(const DecodeParams &p, int grid_x, int num_kv
     return cudaGetLastError();
 }
 
-template <typename T, int D, int BS, typename TQ = T>
+template <typename T, int D, int BS, typename TQ = T, bool kAppend = false>
 static cudaError_t dispatch_group(const DecodeParams &p, int group, int grid_x, int num_kv_heads,
                                   int num_seqs, cudaStream_t stream) {
     switch (group) {
-        case 1: return launch_decode_t<T, D, BS, 1, TQ>(p, grid_x, num_kv_heads, num_seqs, stream);
-        case 2: return launch_decode_t<T, D, BS, 2, TQ>(p, grid_x, num_kv_heads, num_seqs, stream);
-        case 4: return launch_decode_t<T, D, BS, 4, TQ>(p, grid_x, num_kv_heads, num_seqs, stream);
-        case 8: return launch_decode_t<T, D, BS, 8, TQ>(p, grid_x, num_kv_heads, num_seqs, stream);
+        case 1: return launch_decode_t<T, D, BS, 1, TQ, kAppend>(p, grid_x, num_kv_heads, num_seqs, stream);
+        case 2: return launch_decode_t<T, D, BS, 2, TQ, kAppend>(p, grid_x, num_kv_heads, num_seqs, stream);
+        case 4: return launch_decode_t<T, D, BS, 4, TQ, kAppend>(p, grid_x, num_kv_heads, num_seqs, stream);
+        case 8: return launch_decode_t<T, D, BS, 8, TQ, kAppend>(p, grid_x, num_kv_heads, num_seqs, stream);
         default: return cudaErrorInvalidValue;
     }
 }
 
-template <typename T, typename TQ = T>
+template <typename T, typename TQ = T, bool kAppend = false>
 static cudaError_t dispatch_shape(const DecodeParams &p, int head_dim, int block_size, int group,
                                   int grid_x, int num_kv_heads, int num_seqs, cudaStream_t stream) {
-    if (head_dim == 64 && block_size == 16) return dispatch_group<T, 64, 16, TQ>(p, group, grid_x, num_kv_heads, num_seqs, stream);
-    if (head_dim == 64 && block_size == 32) return dispatch_group<T, 64, 32, TQ>(p, group, grid_x, num_kv_heads, num_seqs, stream);
-    if (head_dim == 128 && block_size == 16) return dispatch_group<T, 128, 16, TQ>(p, group, grid_x, num_kv_heads, num_seqs, stream);
-    if (head_dim == 128 && block_size == 32) return dispatch_group<T, 128, 32, TQ>(p, group, grid_x, num_kv_heads, num_seqs, stream);
+    if (head_dim == 64 && block_size == 16) return dispatch_group<T, 64, 16, TQ, kAppend>(p, group, grid_x, num_kv_heads, num_seqs, stream);
+    if (head_dim == 64 && block_size == 32) return dispatch_group<T, 64, 32, TQ, kAppend>(p, group, grid_x, num_kv_heads, num_seqs, stream);
+    if (head_dim == 128 && block_size == 16) return dispatch_group<T, 128, 16, TQ, kAppend>(p, group, grid_x, num_kv_heads, num_seqs, stream);
+    if (head_dim == 128 && block_size == 32) return dispatch_group<T, 128, 32, TQ, kAppend>(p, group, grid_x, num_kv_heads, num_seqs, stream);
     return cudaErrorInvalidValue;
+}
+
+template <typename T>
+static cudaError_t dispatch_append(const DecodeParams &p, int head_dim, int block_size, int group, int grid_x,
+                                   int num_kv_heads, int num_seqs, cudaStream_t stream) {
+    return p.new_key ? dispatch_shape<T, T, true>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream)
+                     : dispatch_shape<T, T, false>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream);
 }
 
 cudaError_t launch_decode(const DecodeParams &p, pa_dtype kv_dtype, int head_dim, int block_size,
                           int group, int grid_x, int num_kv_heads, int num_seqs,
                           cudaStream_t stream) {
     switch (kv_dtype) {
-        case PA_F32: return dispatch_shape<float>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream);
-        case PA_F16: return dispatch_shape<__half>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream);
-        case PA_BF16: return dispatch_shape<__nv_bfloat16>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream);
+        case PA_F32: return dispatch_append<float>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream);
+        case PA_F16: return dispatch_append<__half>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream);
+        case PA_BF16: return dispatch_append<__nv_bfloat16>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream);
     }
     return cudaErrorInvalidValue;
 }

@@ -32,6 +32,12 @@ struct DecodeParams {
     int max_context_len;
     pa_dtype out_dtype;
     unsigned int *err;   // device error word
+    // nullable (16-bit and fp32 caches): the newest token of every sequence
+    // (position context_len - 1), [num_seqs, num_kv_heads, head_dim] each,
+    // written into the slot its table gives and used in place of the pool's
+    // copy (pa_decode_append)
+    const void *new_key;
+    const void *new_value;
     // int8 caches with head_dim 128: the V pool as rows of 128 bytes, 16-row
     // boxes in the 128-byte swizzled layout (the kernel's V fragment loads are
     // then free of shared-memory bank conflicts)

@@ -91,6 +91,24 @@ def test_decode_host_checks(pa, kw, code):
     assert rc == code
 
 
+@pytest.mark.parametrize("new_key,new_value,code", [
+    (0, A16, -1),            # no new key rows
+    (A16, 0, -1),
+    (A16 + 8, A16, -7),      # rows not 16-byte aligned
+    (A16, A16 + 4, -7),
+])
+def test_decode_append_host_checks(pa, new_key, new_value, code):
+    rc = pa._lib.pa_decode_append(A16, A16, new_key, new_value, A16, A16, A16, 4, A16, 2, 8, 8, 128, 0.1, 16, 8,
+                                  1, 1, None, None)
+    assert rc == code
+    # the checks of pa_decode apply as well
+    assert pa._lib.pa_decode_append(A16, A16, A16, A16, A16, A16, A16, 4, A16, 2, 8, 8, 96, 0.1, 16, 8,
+                                    1, 1, None, None) == -5
+    # an empty batch needs no rows
+    assert pa._lib.pa_decode_append(None, None, None, None, None, None, None, 0, None, 0, 8, 8, 128, 0.1, 16, 0,
+                                    1, 1, None, None) == 0
+
+
 def test_empty_batches_are_no_ops(pa):
     assert pa._lib.pa_decode(None, None, None, None, None, 0, None, 0, 8, 8, 128, 0.1, 16, 0, 1, 1, None, None) == 0
     assert pa._lib.pa_reshape_and_cache(None, None, None, None, None, 0, 4, 8, 128, 16, 1, None) == 0

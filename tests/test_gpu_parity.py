@@ -281,6 +281,56 @@ def test_copy_blocks_bitwise(pa):
     assert pa.pa_read_device_errors() == 0
 
 
+def _bits(t):
+    return t.view(torch.int32 if t.element_size() == 4 else torch.int16)
+
+
+@pytest.mark.parametrize("dt,D,BS,Hq,Hkv", SHAPES)
+def test_decode_append_equals_write_then_decode(pa, dt, D, BS, Hq, Hkv):
+    """pa_decode_append gives, bit for bit, the pools and the output of
+    pa_reshape_and_cache of the newest tokens followed by pa_decode. Its side
+    starts with NaN in the newest tokens' slots, so attention that read the
+    pool's copy of a newest row instead of the new one would show NaN."""
+    ctx = [1, 17, 45, 100, 16, 33, 0, 64]
+    c = Case(pa, DT[dt], len(ctx), Hq, Hkv, D, BS, ctx, seed=41 + D + BS + Hq)
+    d1, out1 = _run_write_and_decode(pa, c)
+    d2 = c.device()
+    for s, L in enumerate(ctx):
+        if L:
+            b, o = divmod(int(c.slots[s]), BS)
+            d2["k"][b, :, o, :] = float("nan")
+            d2["v"][b, :, o, :] = float("nan")
+    from paged_kv_cache_340_b200.batch import longest_first
+    order = torch.from_numpy(longest_first(c.ctx)).cuda()
+    out2 = torch.empty_like(out1)
+    pa.pa_decode_append(out2, d2["q"], d2["nk"], d2["nv"], d2["k"], d2["v"], d2["bt"], d2["cl"], c.scale,
+                        seq_order=order)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_errors() == 0
+    assert torch.equal(_bits(d2["k"]), _bits(d1["k"])) and torch.equal(_bits(d2["v"]), _bits(d1["v"]))
+    assert torch.isfinite(out2.float()).all()
+    assert torch.equal(out2, out1)
+    assert_attention_close(out2, c.ref, DT[dt], "decode_append")
+
+
+def test_decode_append_skips_a_bad_block(pa):
+    """A table entry out of range at a sequence's newest token: that block is
+    skipped (nothing written, error flagged); the other sequences match."""
+    c = Case(pa, torch.bfloat16, 3, 8, 2, 128, 16, [40, 40, 40], seed=43, poison=False)
+    d = c.device()
+    bt = d["bt"].clone()
+    bt[1, 2] = c.NB + 7                                      # holds token 39 of sequence 1
+    k0 = d["k"].clone()
+    pa.pa_read_device_errors()
+    out = torch.empty((3, 8, 128), dtype=torch.bfloat16, device="cuda")
+    pa.pa_decode_append(out, d["q"], d["nk"], d["nv"], d["k"], d["v"], bt, d["cl"], c.scale)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_errors() & pa.PA_DEVERR_BLOCK_ID
+    b1, o1 = divmod(int(c.slots[1]), 16)
+    assert torch.equal(_bits(d["k"][b1, :, o1]), _bits(k0[b1, :, o1]))   # sequence 1's newest row not written
+    assert_attention_close(out[[0, 2]], c.ref[[0, 2]], torch.bfloat16, "unaffected sequences")
+
+
 def test_device_errors_are_recorded_not_faulted(pa):
     c = Case(pa, torch.float16, 3, 4, 4, 128, 16, [40, 40, 40], seed=12, poison=False)
     d = c.device()
