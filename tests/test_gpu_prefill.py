@@ -72,6 +72,7 @@ CASES = [
     ([96, 513, 17], [96, 100, 17], 16, 4, 16),                # GQA G = 4
     ([250, 64], [250, 33], 16, 2, 32),                        # GQA G = 8
     ([700, 300, 1], [640, 300, 1], 16, 8, 16),                # GQA G = 2, several query tiles per sequence
+    ([64, 30, 100], [10, 0, 50], 8, 4, 16),                   # a sequence with no new tokens in the middle
 ]
 
 
