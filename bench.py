@@ -512,7 +512,7 @@ def measure_beam(name: str, steps: int, warmup: int, host_steps: int = 30):
     as a CUDA graph; and for context the same steps through the host pool,
     where each step must read the beams' parents back (a synchronisation) and
     upload tables, slots and pairs."""
-    from paged_kv_cache_340_b200 import pa_copy_blocks, pa_decode, pa_reshape_and_cache
+    from paged_kv_cache_340_b200 import pa_copy_blocks, pa_decode_append
     from paged_kv_cache_340_b200.batch import beam_decode_bytes, build_beam_batch, host_beam_step, run_beam_step
     from paged_kv_cache_340_b200.workloads import SPECS, make_beam_inputs
     spec = SPECS[name]
@@ -601,15 +601,15 @@ def measure_beam(name: str, steps: int, warmup: int, host_steps: int = 30):
         dt_slots.copy_(torch.from_numpy(slots))
         if cow.shape[0]:
             pa_copy_blocks(b.k_cache, b.v_cache, torch.from_numpy(cow).cuda())
-        pa_reshape_and_cache(b.new_key[k], b.new_value[k], b.k_cache, b.v_cache, dt_slots)
-        pa_decode(b.out, b.query[k], b.k_cache, b.v_cache, dt_tab, dt_ctx, spec.scale)
+        pa_decode_append(b.out, b.query[k], b.new_key[k], b.new_value[k], b.k_cache, b.v_cache, dt_tab, dt_ctx,
+                         spec.scale)
         torch.cuda.synchronize()
         host.append(time.perf_counter() - t)
     res = {"ms_per_step": round(ms, 4), "beams": W, "steps_timed": steps, "launch": "one CUDA graph per step",
            "decode_kernel_ms": round(kern[3], 4), "decode_GBps_logical": round(dec_by / kern[3] / 1e6, 1),
            "step_GBps_logical": round(by / ms / 1e6, 1),
            "kernels_ms": {"beam_step": round(kern[0], 5), "copy_blocks_counted": round(kern[1], 5),
-                          "reshape_and_cache": round(kern[2], 5), "decode": round(kern[3], 5)},
+                          "decode_append": round(kern[3], 5)},
            "device_path_wall_ms_with_sync": round(1e3 * statistics.median(wall), 4),
            "host_pool_path_wall_ms": round(1e3 * statistics.median(host), 4),
            "note": "decode bytes are logical: beams of a prompt share their prefix blocks (read from L2)"}

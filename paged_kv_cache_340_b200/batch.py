@@ -483,9 +483,11 @@ def build_beam_batch(spec: Spec, inputs: dict, device="cuda", pool_policy: int =
 
 def run_beam_step(b: BeamBatch, stream=None, events=None) -> None:
     """One beam-search decode step, all on the device: beam step (fork,
-    release, copy-on-write decisions), counted block copy, slot write of the
-    new tokens, decode over the new tables. events (optional, 5 CUDA events)
-    are recorded between the launches."""
+    release, copy-on-write decisions), counted block copy, then the slot
+    write of the new tokens and decode over the new tables as one launch
+    (each new token is its beam's newest, in a block that beam alone holds
+    after the copy-on-write). events (optional, 5 CUDA events) are recorded
+    between the launches (the fourth right after the third)."""
     i = b.steps_done
     k = i % b.parents.shape[0]
     src, dst = i % 2, (i + 1) % 2
@@ -500,10 +502,9 @@ def run_beam_step(b: BeamBatch, stream=None, events=None) -> None:
     mark(1)
     pa_copy_blocks_counted(b.k_cache, b.v_cache, b.cow_pairs, b.num_cow, stream=stream)
     mark(2)
-    pa_reshape_and_cache(b.new_key[k], b.new_value[k], b.k_cache, b.v_cache, b.slot_mapping, stream=stream)
     mark(3)
-    pa_decode(b.out, b.query[k], b.k_cache, b.v_cache, b.tables[dst], b.context_lens[dst], b.spec.scale,
-              stream=stream)
+    pa_decode_append(b.out, b.query[k], b.new_key[k], b.new_value[k], b.k_cache, b.v_cache, b.tables[dst],
+                     b.context_lens[dst], b.spec.scale, stream=stream)
     mark(4)
     b.steps_done = i + 1
 
