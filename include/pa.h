@@ -1,8 +1,8 @@
 /*
  * pa.h -- C ABI of the paged KV-cache library for NVIDIA B200 (sm_100a):
- * decode, split-K decode, prefill, slot writes and block copies (16-bit, fp32
- * and int8 caches), the host block pool with its prefix cache, and a device
- * block pool with a beam-search step.
+ * decode, split-K decode, slot write fused with decode, prefill, slot writes
+ * and block copies (16-bit, fp32 and int8 caches), the host block pool with
+ * its prefix cache, and a device block pool with a beam-search step.
  *
  * A sequence's keys and values live in fixed-size blocks of a shared pool; a
  * per-sequence block table maps logical block i (tokens i*bs .. i*bs+bs-1) to
@@ -16,8 +16,8 @@
  *   [P5] "Ascend平台下的PageAttention优化实践" (jsqmd.com)
  *
  * Conventions for every device entry point:
- *   - Pointers named *_cache, query, out, key, value, block_tables,
- *     context_lens, slot_mapping, src_dst_pairs and workspace are DEVICE
+ *   - Pointers named *_cache, query, out, key, value, new_key, new_value,
+ *     block_tables, context_lens, slot_mapping, src_dst_pairs and workspace are DEVICE
  *     pointers owned by the caller. The library never allocates, frees or
  *     keeps them.
  *   - Layouts (row-major, contiguous):
