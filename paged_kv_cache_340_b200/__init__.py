@@ -6,8 +6,10 @@ Argument marshalling only: every operation runs in the CUDA kernels of
 and streams. There is no CPU or library fallback: if the shared library is
 missing, the first call raises.
 
-Calls: slot write (pa_reshape_and_cache), decode (pa_decode), split-K decode
-and reduce (pa_decode_splitk, pa_splitk_reduce, pa_decode_splitk_static),
+Calls: slot write (pa_reshape_and_cache), decode (pa_decode), the slot write
+of each sequence's newest token with decode in one launch (pa_decode_append),
+split-K decode and reduce (pa_decode_splitk, pa_splitk_reduce,
+pa_decode_splitk_static),
 copy-on-write block copy (pa_copy_blocks, pa_copy_blocks_counted), paged
 prefill (pa_prefill), the int8 cache (pa_*_q8), the host block pool and
 prefix cache (BlockPool, PrefixCache), and the device pool with its beam step
