@@ -109,6 +109,53 @@ def test_decode_append_host_checks(pa, new_key, new_value, code):
                                     1, 1, None, None) == 0
 
 
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=64), -5),                       # the tensor-core prefill is built for head_dim 128
+    (dict(kv_dtype=0, out_dtype=0), -2),           # fp32 caches: decode only
+    (dict(out_dtype=1, kv_dtype=2), -2),
+    (dict(block_size=8), -6),
+    (dict(num_heads=12, num_kv_heads=8), -4),
+    (dict(num_heads=48, num_kv_heads=3), -4),      # head group 16
+    (dict(num_seqs=-1), -3),
+    (dict(query=0), -1),
+    (dict(q_start=A16 + 2), -7),
+    (dict(out=A16 + 8), -7),
+    (dict(num_blocks=1 << 27, num_kv_heads=8, num_heads=8), -3),   # pool rows past int32
+    (dict(max_q_len=1 << 29, num_heads=32, num_kv_heads=4), -3),   # query tile index past int32
+    (dict(num_tokens=0), 0),                       # nothing to do
+])
+def test_prefill_host_checks(pa, kw, code):
+    a = dict(out=A16, query=A16, q_start=A16, num_tokens=40, max_q_len=20, k_cache=A16, v_cache=A16,
+             block_tables=A16, max_blocks=4, context_lens=A16, num_seqs=2, num_heads=8, num_kv_heads=8,
+             head_dim=128, scale=0.1, block_size=16, num_blocks=8, kv_dtype=2, out_dtype=0)
+    a.update(kw)
+    rc = pa._lib.pa_prefill(a["out"], a["query"], a["q_start"], a["num_tokens"], a["max_q_len"], a["k_cache"],
+                            a["v_cache"], a["block_tables"], a["max_blocks"], a["context_lens"], a["num_seqs"],
+                            a["num_heads"], a["num_kv_heads"], a["head_dim"], a["scale"], a["block_size"],
+                            a["num_blocks"], a["kv_dtype"], a["out_dtype"], None)
+    assert rc == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q_dtype=0), -2),                         # the query is 16-bit
+    (dict(k_scale=0), -1),
+    (dict(v_scale=A16 + 4), -7),
+    (dict(out_dtype=2), -2),                       # fp16 query, bf16 output
+    (dict(head_dim=96), -5),
+    (dict(num_seqs=0), 0),
+])
+def test_decode_q8_host_checks(pa, kw, code):
+    a = dict(out=A16, query=A16, q_dtype=1, k_cache=A16, v_cache=A16, k_scale=A16, v_scale=A16, block_tables=A16,
+             max_blocks=4, context_lens=A16, num_seqs=2, num_heads=8, num_kv_heads=2, head_dim=128, scale=0.1,
+             block_size=16, num_blocks=8, out_dtype=1)
+    a.update(kw)
+    rc = pa._lib.pa_decode_q8(a["out"], a["query"], a["q_dtype"], a["k_cache"], a["v_cache"], a["k_scale"],
+                              a["v_scale"], a["block_tables"], a["max_blocks"], a["context_lens"], a["num_seqs"],
+                              a["num_heads"], a["num_kv_heads"], a["head_dim"], a["scale"], a["block_size"],
+                              a["num_blocks"], a["out_dtype"], None, None)
+    assert rc == code
+
+
 def test_empty_batches_are_no_ops(pa):
     assert pa._lib.pa_decode(None, None, None, None, None, 0, None, 0, 8, 8, 128, 0.1, 16, 0, 1, 1, None, None) == 0
     assert pa._lib.pa_reshape_and_cache(None, None, None, None, None, 0, 4, 8, 128, 16, 1, None) == 0
