@@ -156,6 +156,41 @@ def test_decode_q8_host_checks(pa, kw, code):
     assert rc == code
 
 
+def test_slot_write_and_copy_host_checks(pa):
+    lib = pa._lib
+    # pa_reshape_and_cache(key, value, k_cache, v_cache, slots, T, NB, Hkv, D, bs, dtype, stream)
+    w = [A16, A16, A16, A16, A16, 4, 8, 2, 128, 16, 1, None]
+
+    def w_(**kw):
+        a = list(w)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return lib.pa_reshape_and_cache(*a)
+    assert w_(a8=96) == -5 and w_(a9=8) == -6 and w_(a10=7) == -2 and w_(a5=-1) == -3
+    assert w_(a4=0) == -1 and w_(a4=A16 + 2) == -7 and w_(a0=A16 + 8) == -7
+    assert w_(a6=1 << 27, a9=32) == -3                     # slots past int32
+    # pa_reshape_and_cache_q8(key, value, src_dtype, kq, vq, ks, vs, slots, T, NB, Hkv, D, bs, stream)
+    q = [A16, A16, 1, A16, A16, A16, A16, A16, 4, 8, 2, 128, 16, None]
+
+    def q_(**kw):
+        a = list(q)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return lib.pa_reshape_and_cache_q8(*a)
+    assert q_(a2=9) == -2 and q_(a11=32) == -5 and q_(a12=64) == -6
+    assert q_(a5=0) == -1 and q_(a6=A16 + 4) == -7 and q_(a8=0) == 0
+    # pa_copy_blocks(k_cache, v_cache, pairs, n, NB, Hkv, D, bs, dtype, stream)
+    c = [A16, A16, A16, 3, 8, 2, 128, 16, 1, None]
+
+    def c_(**kw):
+        a = list(c)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return lib.pa_copy_blocks(*a)
+    assert c_(a6=80) == -5 and c_(a7=48) == -6 and c_(a8=5) == -2 and c_(a3=-2) == -3
+    assert c_(a2=0) == -1 and c_(a2=A16 + 4) == -7 and c_(a3=0) == 0
+
+
 def test_empty_batches_are_no_ops(pa):
     assert pa._lib.pa_decode(None, None, None, None, None, 0, None, 0, 8, 8, 128, 0.1, 16, 0, 1, 1, None, None) == 0
     assert pa._lib.pa_reshape_and_cache(None, None, None, None, None, 0, 4, 8, 128, 16, 1, None) == 0
