@@ -1,7 +1,8 @@
 """CPU oracle for paged KV-cache decode attention.
 
 TEST INFRASTRUCTURE. Only the test suite, ``__graft_entry__.smoke()`` and the
-CPU-baseline leg of ``bench.py`` may import this package. The CUDA library and
+CPU-baseline leg and reference arm (``--impl reference``) of ``bench.py`` may
+import this package. The CUDA library and
 its Python binding never import it, and the two share no code: this package
 wraps ``pa_oracle.c`` (plain single-threaded C in double precision) through
 ctypes, plus the host block pool in ``block_pool.py``.

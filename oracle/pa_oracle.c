@@ -2,7 +2,7 @@
  * pa_oracle.c -- plain CPU oracle for paged KV-cache decode attention.
  *
  * TEST INFRASTRUCTURE. Only the test suite, the smoke check and the
- * benchmark's CPU-baseline leg call this file. The CUDA library never links,
+ * benchmark's CPU-baseline leg and reference arm call this file. The CUDA library never links,
  * loads or calls it, and it shares no code, header or table with that library.
  *
  * Everything here is single-threaded, in double precision, and written in the
