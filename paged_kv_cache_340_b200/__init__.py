@@ -425,11 +425,12 @@ class BlockPool:
         if not h:
             raise PagedAttentionError("pa_pool_create", -3)
         self._h = ctypes.c_void_p(h)
+        self._destroy = _lib.pa_pool_destroy  # still callable at interpreter exit, when _lib may be gone
 
     def __del__(self):
-        h = getattr(self, "_h", None)
-        if h is not None and h.value:
-            _lib.pa_pool_destroy(h)
+        h, destroy = getattr(self, "_h", None), getattr(self, "_destroy", None)
+        if h is not None and h.value and destroy is not None:
+            destroy(h)
             self._h = None
 
     def num_free(self) -> int:
@@ -493,11 +494,12 @@ class PrefixCache:
         if not h:
             raise PagedAttentionError("pa_prefix_cache_create", -3)
         self._h = ctypes.c_void_p(h)
+        self._destroy = _lib.pa_prefix_cache_destroy  # still callable at interpreter exit
 
     def __del__(self):
-        h = getattr(self, "_h", None)
-        if h is not None and h.value:
-            _lib.pa_prefix_cache_destroy(h)
+        h, destroy = getattr(self, "_h", None), getattr(self, "_destroy", None)
+        if h is not None and h.value and destroy is not None:
+            destroy(h)
             self._h = None
 
     @staticmethod
