@@ -15,11 +15,14 @@ step, with
   decode bytes = sum_s ctx_s * 2 * Hkv * D * elt + S * Hq * D * (elt_q + elt_out)
                  + 4 * sum_s ceil(ctx_s / bs) + 4 * S
   slot-write bytes = 2 * T * Hkv * D * elt (read) + the same (write) + 4 * T
-Inputs (>= 1.2 GB of K/V) are larger than L2, so no flush between steps.
+Inputs (>= 1.1 GB of K/V per step) are larger than L2 (126 MB), so no flush between steps.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-For N > 1, launch under torchrun: each rank runs its own batch (sequences
-shard across GPUs with no exchange), value = all ranks' bytes / max time.
+For N > 1 each rank runs its own batch on its own GPU (sequences shard across
+GPUs with no exchange); value = all ranks' bytes / the slowest rank's time.
+Under torchrun the ranks come from the launcher (WORLD_SIZE must equal N);
+without one, bench.py starts N local ranks itself under torch.distributed.run.
+--dry-run --backend gloo runs that launch and the timing plumbing on CPU only.
 """
 from __future__ import annotations
 
@@ -188,8 +191,39 @@ class ClockSampler:
 from paged_kv_cache_340_b200 import dist as pdist  # noqa: E402
 
 
-def dist_setup(n_gpus: int):
-    return pdist.init("nccl")
+def dist_setup(n_gpus: int, backend: str = "nccl"):
+    world, rank, local = pdist.init(backend)
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but {world} rank(s) were started")
+    return world, rank, local
+
+
+def launch_ranks(args) -> None:
+    """--gpus N > 1 with no launcher around this process: start N local ranks
+    (one process per GPU) under torch.distributed.run with this script and
+    these arguments, wait for them and exit with their status. With a
+    launcher, check that it started N ranks; with N = 1, return."""
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is not None:
+        if int(env_world) != args.gpus:
+            raise SystemExit(f"--gpus {args.gpus} but the launcher started {env_world} rank(s)")
+        return
+    if args.gpus <= 1:
+        return
+    if not args.dry_run and torch.cuda.device_count() < args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but {torch.cuda.device_count()} GPU(s) are visible")
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    bound = 3600
+    import shutil
+    if shutil.which("timeout"):
+        cmd = ["timeout", "-k", "60", str(bound)] + cmd
+    r = subprocess.run(cmd, env=dict(os.environ, MASTER_ADDR="127.0.0.1"))
+    raise SystemExit(r.returncode)
 
 
 def max_over_ranks(x: float, world: int) -> float:
@@ -410,6 +444,39 @@ def oracle_sample(ob: OracleBatch, budget_s: float, start_seq: int = 0):
     return tot_bytes, tot_s, n_seq
 
 
+def host_cores() -> int:
+    """Cores this process may run on (nproc)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_parallel(ob: OracleBatch, budget_s: float, threads: int):
+    """The same oracle, as it stands, on `threads` host threads at once, each
+    over its own whole sequences of the batch (the C call runs without the
+    Python lock, so the threads run in parallel), until each thread has spent
+    budget_s of oracle time. Returns (bytes per second summed over the
+    threads, sequences, wall seconds)."""
+    import threading
+    res = [None] * threads
+    prev = torch.get_num_threads()
+    torch.set_num_threads(1)  # the per-sequence widening stays on its own thread
+
+    def work(i):
+        res[i] = oracle_sample(ob, budget_s, start_seq=(i * 13) % len(ob.ctx))
+
+    t = time.perf_counter()
+    ths = [threading.Thread(target=work, args=(i,)) for i in range(threads)]
+    for th in ths:
+        th.start()
+    for th in ths:
+        th.join()
+    wall = time.perf_counter() - t
+    torch.set_num_threads(prev)
+    return sum(b / sec for b, sec, _ in res), sum(n for _, _, n in res), wall
+
+
 def run_reference(args, world, rank):
     """Reference arm: the CPU oracle, timed on the host cores, on the same
     workload, metric and unit. Rank 0 only; no GPU is used."""
@@ -439,7 +506,8 @@ def run_reference(args, world, rank):
         "config": {"workload": spec.name, "num_seqs": spec.num_seqs, "num_heads": spec.num_heads,
                    "num_kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim, "block_size": spec.block_size,
                    "kv_dtype": spec.kv_dtype},
-        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "host_cores": host_cores(),
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -645,6 +713,32 @@ def measure_other(name: str, steps: int, warmup: int):
     return res
 
 
+def run_dry(args, world: int, rank: int) -> None:
+    """The multi-rank plumbing with no GPU work: each rank takes its own
+    workload seed, warms up and times K empty steps between barriers, and the
+    job's time is the slowest rank's. Rank 0 prints one line listing every
+    rank it heard from (a CPU test of the --gpus N launch)."""
+    from paged_kv_cache_340_b200.workloads import SPECS
+    spec = pdist.rank_spec(SPECS[args.workload], rank)
+    for _ in range(args.warmup):
+        barrier(world)
+    barrier(world)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        barrier(world)
+    ms = max_over_ranks(1e3 * (time.perf_counter() - t), world) / max(1, args.steps)
+    ranks = [None] * world
+    if world > 1:
+        torch.distributed.all_gather_object(ranks, {"rank": rank, "seed": spec.seed, "pid": os.getpid()})
+    else:
+        ranks = [{"rank": rank, "seed": spec.seed, "pid": os.getpid()}]
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": round(ms, 5), "backend": args.backend, "ranks": ranks,
+                          "config": {"workload": spec.name}}), flush=True)
+    pdist.finalize(world)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -655,13 +749,24 @@ def main():
     ap.add_argument("--partition", type=int, default=None, help="force a split-K partition size (0 = unsplit)")
     ap.add_argument("--no-others", action="store_true", help="skip the other workloads' lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backend", default="nccl", choices=["nccl", "gloo"],
+                    help="process-group backend (gloo only with --dry-run)")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="start the ranks and run the barriers and max-over-ranks timing, no GPU work")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
+    if args.backend == "gloo" and not args.dry_run:
+        raise SystemExit("--backend gloo is for --dry-run (the GPU path uses nccl)")
     if args.impl == "reference":
         # The reference arm runs on the host: rank 0 alone, no process group.
         world, rank, _ = pdist.env_ranks()
         run_reference(args, world, rank)
+        return
+    launch_ranks(args)  # --gpus N > 1 without a launcher: starts N ranks and exits
+    if args.dry_run:
+        world, rank, _ = dist_setup(args.gpus, args.backend)
+        run_dry(args, world, rank)
         return
     world, rank, local = dist_setup(args.gpus)
     import paged_kv_cache_340_b200 as pa  # noqa: F401  (fails loudly without the CUDA library)
@@ -699,7 +804,7 @@ def main():
                    "context_lens": "U{256..2048}" if spec.name == DEFAULT_WORKLOAD else str(spec.lengths),
                    "kv_dtype": spec.kv_dtype, "out_dtype": spec.out_dtype, "partition_size": b.partition_size,
                    "parallelism": f"dp{world} (sequences shard, no exchange)",
-                   "l2": "inputs larger than L2 (K/V >= 1.2 GB per step), no flush",
+                   "l2": f"inputs larger than L2 (decode reads {by['decode'] / 1e9:.3f} GB per step, L2 126 MB), no flush",
                    "step": ("copy_blocks (if any) + decode_append (slot write of each sequence's newest token "
                             "and decode, one launch)" if b.fused_append else
                             "copy_blocks (if any) + reshape_and_cache + decode")},
@@ -719,11 +824,21 @@ def main():
     line["kernels"] = kernel_lines(spec, b, kern, by)
     if world == 1 and rank == 0 and not args.no_cpu_baseline and "k_pool" in b.host_inputs and \
             spec.kv_dtype != "i8":  # the sampled oracle leg is the 16/32-bit decode
-        nbytes, secs, nseq = oracle_sample(OracleBatch(spec, b.host_inputs), 12.0)
-        line["cpu_baseline"] = {"value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+        ob = OracleBatch(spec, b.host_inputs)
+        nbytes, secs, nseq = oracle_sample(ob, 12.0)
+        ncores = host_cores()
+        line["cpu_baseline"] = {"value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": 1,
+                                "host_cores": ncores, "kind": "oracle",
                                 "sample": f"{nseq} sequences (all heads; {nseq / spec.num_seqs:.1f} passes over the "
                                           f"{spec.num_seqs}-sequence batch), decode only; float64 C oracle, "
-                                          f"one thread, {secs:.1f} s"}
+                                          f"one thread of {ncores} host cores, {secs:.1f} s"}
+        nth = min(ncores, 128)
+        rate, nseq_p, wall = oracle_sample_parallel(ob, 4.0, nth)
+        line["cpu_baseline_all_cores"] = {
+            "value": round(rate / 1e9, 4), "unit": "GB/s", "cores": nth, "host_cores": ncores, "kind": "oracle",
+            "sample": f"{nseq_p} whole sequences of the same batch on {nth} threads at once (each over its own "
+                      f"sequences, 4 s of oracle time per thread, {wall:.1f} s wall); value = sum of the "
+                      f"threads' rates; the same float64 C oracle, unchanged"}
     del b
     torch.cuda.empty_cache()
     if world == 1 and not args.no_others and args.workload == DEFAULT_WORKLOAD:

@@ -203,7 +203,7 @@ int pa_splitk_reduce(void *out, const void *workspace, size_t workspace_bytes,
  * Same inputs and result as pa_decode_splitk followed by pa_splitk_reduce
  * (out [num_seqs, num_heads, head_dim] of out_dtype), but the workspace is a
  * fixed array inside the library (PA_STATIC_SCRATCH_BYTES of device memory on
- * every GPU that loads the library, kept until the process exits), so the
+ * every GPU where it has been called, kept until the process exits), so the
  * caller passes only inputs and the output. It suits code that must not
  * allocate while it runs: a serving loop that gave nearly all of HBM to its
  * KV pool up front, a plug-in whose host framework forbids allocation inside
@@ -212,13 +212,21 @@ int pa_splitk_reduce(void *out, const void *workspace, size_t workspace_bytes,
  *     pa_splitk_workspace_bytes(num_seqs, num_heads, head_dim,
  *     max_context_len, partition_size) exceeds PA_STATIC_SCRATCH_BYTES
  *     (use a larger partition_size or fewer sequences per call).
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every other argument the split-K decode or the reduce would refuse
+ *     (NULL or misaligned out, an out_dtype other than PA_F32, PA_F16 or
+ *     PA_BF16, ...) is also refused before any device work.
+ *   - The array belongs to a module that CUDA loads lazily: the first call on
+ *     each device (and again after a cudaDeviceReset) loads it, which takes
+ *     the PA_STATIC_SCRATCH_BYTES of device memory then, and looks up its
+ *     device address (cudaGetSymbolAddress). A caller that gives nearly all
+ *     of HBM to its KV pool therefore makes one call first -- an empty one,
+ *     num_seqs == 0 with valid sizes, does only this -- before sizing the
+ *     pool, and before any stream capture. Later calls allocate nothing and
+ *     call no allocating routine.
  *   - All calls on a device share the array: calls whose kernels overlap on
  *     the GPU (other streams, other host threads) race and must be
  *     serialised. The array keeps the previous call's partials; none of it
  *     needs to start at zero.
- *   - Allocates nothing and calls no allocating routine.
  */
 #define PA_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
 

@@ -3,6 +3,7 @@
 #include <atomic>
 #include <climits>
 #include <cmath>
+#include <mutex>
 
 #include "pa_common.cuh"
 #include "pa_internal.h"
@@ -13,22 +14,50 @@ __device__ unsigned int g_device_errors = 0;
 
 static constexpr int kMaxDevices = 64;
 
-cudaError_t device_error_word(unsigned int **word) {
-    static std::atomic<unsigned int *> cache[kMaxDevices];
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+void *current_context() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(f);
+    });
+    CUcontext c = nullptr;
+    if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+cudaError_t symbol_address(const void *symbol, SymbolCache *cache, void **addr) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    unsigned int *w = cache[dev].load(std::memory_order_acquire);
-    if (w == nullptr) {
-        void *addr = nullptr;
-        e = cudaGetSymbolAddress(&addr, g_device_errors);
-        if (e != cudaSuccess) return e;
-        w = static_cast<unsigned int *>(addr);
-        cache[dev].store(w, std::memory_order_release);
+    void *ctx = current_context();
+    if (ctx != nullptr && cache->ctx[dev].load(std::memory_order_acquire) == ctx) {
+        *addr = cache->addr[dev].load(std::memory_order_relaxed);
+        return cudaSuccess;
     }
-    *word = w;
+    void *a = nullptr;
+    e = cudaGetSymbolAddress(&a, symbol);  // loads the module on its first use in this context
+    if (e != cudaSuccess) return e;
+    ctx = current_context();
+    // address first, then the context it belongs to (readers check the context)
+    cache->addr[dev].store(a, std::memory_order_relaxed);
+    cache->ctx[dev].store(ctx, std::memory_order_release);
+    *addr = a;
     return cudaSuccess;
+}
+
+cudaError_t device_error_word(unsigned int **word) {
+    static SymbolCache cache;
+    void *a = nullptr;
+    cudaError_t e = symbol_address(&g_device_errors, &cache, &a);
+    if (e == cudaSuccess) *word = static_cast<unsigned int *>(a);
+    return e;
 }
 
 int sm_count() {
@@ -44,16 +73,16 @@ int sm_count() {
     return n;
 }
 
-cudaError_t ensure_smem_attr(const void *func, int bytes, unsigned int *done_mask) {
+cudaError_t ensure_smem_attr(const void *func, int bytes, AttrCache *done) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const unsigned int bit = 1u << (dev & 31);
-    std::atomic_ref<unsigned int> mask(*done_mask);
-    if (dev < 32 && (mask.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    void *ctx = current_context();
+    if (ctx != nullptr && done->ctx[dev].load(std::memory_order_acquire) == ctx) return cudaSuccess;
     e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    if (dev < 32) mask.fetch_or(bit, std::memory_order_acq_rel);
+    done->ctx[dev].store(current_context(), std::memory_order_release);
     return cudaSuccess;
 }
 

@@ -617,7 +617,7 @@ cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const in
     q.err = err;
     const long long base = (3LL * num_old + num_new) * (long long)sizeof(int);
     const long long with_tables = base + (long long)num_old * max_blocks * (long long)sizeof(int);
-    static unsigned int attr_done[2] = {0, 0};
+    static AttrCache attr_done[2];
     cudaError_t e;
     if (with_tables <= beam::kMaxDynBytes) {
         e = ensure_smem_attr(reinterpret_cast<const void *>(beam::beam_step_kernel<true>), beam::kMaxDynBytes,

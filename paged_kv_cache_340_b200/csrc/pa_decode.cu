@@ -1092,7 +1092,7 @@ static cudaError_t launch_decode_t(const DecodeParams &p, int grid_x, int num_kv
                                    cudaStream_t stream) {
     using S = DecodeShape<T, D, BS, G>;
     auto kern = decode_kernel<T, D, BS, G, TQ, kAppend>;
-    static unsigned int attr_done = 0;  // one bit per device
+    static AttrCache attr_done;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), S::kSmemBytes, &attr_done);
     if (e != cudaSuccess) return e;
     dim3 grid(grid_x, num_kv_heads, num_seqs);

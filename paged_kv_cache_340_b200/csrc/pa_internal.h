@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "pa.h"
 
 namespace pa {
@@ -92,13 +94,34 @@ bool encode_rows_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *bas
                     unsigned long long rows, unsigned long long row_stride_bytes, unsigned box_inner,
                     unsigned box_rows, CUtensorMapSwizzle swizzle);
 
-// Device address of the current device's error word (cached per device).
+// Per-device caches of the host side (symbol addresses, kernel attributes)
+// are keyed by the device's current CUDA context, so that a context torn down
+// and made again (cudaDeviceReset) is noticed and the entry refreshed.
+constexpr int kCacheDevices = 64;
+
+struct SymbolCache {
+    std::atomic<void *> ctx[kCacheDevices];
+    std::atomic<void *> addr[kCacheDevices];
+};
+
+struct AttrCache {
+    std::atomic<void *> ctx[kCacheDevices];
+};
+
+// The calling thread's current CUDA context (driver handle), or nullptr.
+void *current_context();
+
+// Device address of a __device__ variable (its host-side stand-in `symbol`)
+// on the current device, looked up once per context.
+cudaError_t symbol_address(const void *symbol, SymbolCache *cache, void **addr);
+
+// Device address of the current device's error word.
 cudaError_t device_error_word(unsigned int **word);
 
 // Number of SMs of the current device.
 int sm_count();
 
-// Sets the dynamic shared memory limit of `func` once per device.
-cudaError_t ensure_smem_attr(const void *func, int bytes, unsigned int *done_mask);
+// Sets the dynamic shared memory limit of `func` once per device context.
+cudaError_t ensure_smem_attr(const void *func, int bytes, AttrCache *done);
 
 }  // namespace pa

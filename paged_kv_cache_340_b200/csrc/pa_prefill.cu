@@ -671,7 +671,7 @@ template <typename T, int G>
 static cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const Params &p,
                             int q_tiles, int num_kv_heads, int num_seqs, cudaStream_t stream) {
     auto kern = prefill_kernel<T, G>;
-    static unsigned int attr_done = 0;
+    static AttrCache attr_done;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), kSmemBytes, &attr_done);
     if (e != cudaSuccess) return e;
     kern<<<dim3(q_tiles, num_kv_heads, num_seqs), kThreads, kSmemBytes, stream>>>(mq, mk, mv, p);
