@@ -237,10 +237,16 @@ def barrier(world: int):
 # ------------------------------------------------------------ measurement
 
 def build_batch(name: str, rank: int, partition=None):
-    from paged_kv_cache_340_b200.batch import build_decode_batch, build_parallel_sampling_batch, write_prefix
-    from paged_kv_cache_340_b200.workloads import SPECS, make_decode_inputs, make_parallel_sampling_inputs
+    from paged_kv_cache_340_b200.batch import build_decode_batch, build_parallel_sampling_batch, \
+        build_prefix_cache_batch, write_prefix
+    from paged_kv_cache_340_b200.workloads import SPECS, make_decode_inputs, make_parallel_sampling_inputs, \
+        make_prefix_cache_inputs
     spec = pdist.rank_spec(SPECS[name], rank)
-    if spec.lengths[0] == "parallel":
+    if spec.lengths[0] == "prefix":
+        inp = make_prefix_cache_inputs(spec)
+        b = build_prefix_cache_batch(spec, inp)
+        write_prefix(b)
+    elif spec.lengths[0] == "parallel":
         inp = make_parallel_sampling_inputs(spec)
         b = build_parallel_sampling_batch(spec, inp, partition_size=partition or 0)
         write_prefix(b)
@@ -250,6 +256,19 @@ def build_batch(name: str, rank: int, partition=None):
     torch.cuda.synchronize()
     b.host_inputs = inp
     return spec, b
+
+
+def unique_kv_bytes(spec, tables: np.ndarray, ctx: np.ndarray) -> int:
+    """K/V bytes of the distinct cache rows one decode reads: a block that
+    several sequences share (a prefix) counts once, with the most tokens any
+    of them reads from it."""
+    used = {}
+    bs = spec.block_size
+    for row, L in zip(tables, ctx.astype(np.int64)):
+        for j in range(int((L + bs - 1) // bs)):
+            b = int(row[j])
+            used[b] = max(used.get(b, 0), int(min(bs, L - j * bs)))
+    return sum(used.values()) * 2 * spec.num_kv_heads * kv_row_bytes(spec)
 
 
 def step_bytes(spec, b) -> dict:
@@ -708,6 +727,13 @@ def measure_other(name: str, steps: int, warmup: int):
            "partition_size": b.partition_size, "seq_tokens_per_s": round(spec.num_seqs / ms * 1e3, 1),
            "context_tokens_per_s": round(float(b.host_context_lens.sum()) / ms * 1e3, 1),
            "kernels": kernel_lines(spec, b, kern, by)}
+    if spec.lengths[0] in ("parallel", "prefix"):  # shared prefix blocks: logical and distinct bytes
+        uniq = unique_kv_bytes(spec, b.host_tables, b.host_context_lens)
+        logical = int(b.host_context_lens.astype(np.int64).sum()) * 2 * spec.num_kv_heads * kv_row_bytes(spec)
+        res["kv_bytes_logical"] = logical
+        res["kv_bytes_unique"] = uniq
+        res["decode_kernel_GBps_unique_kv"] = round(uniq / dec / 1e6, 1)
+        res["note"] = "GBps counts logical bytes: sequences sharing a prefix each read its blocks (L2 hits)"
     del b
     torch.cuda.empty_cache()
     return res
@@ -843,8 +869,8 @@ def main():
     torch.cuda.empty_cache()
     if world == 1 and not args.no_others and args.workload == DEFAULT_WORKLOAD:
         line["other_workloads"] = {n: measure_other(n, 200, 10) for n in
-                                   ("gqa_bf16", "long_splitk_bf16", "parallel_sampling_fp16", "llama7b_mha_int8",
-                                    "gqa_int8")}
+                                   ("gqa_bf16", "long_splitk_bf16", "parallel_sampling_fp16", "prefix_cache_fp16",
+                                    "llama7b_mha_int8", "gqa_int8")}
         line["prefill_workloads"] = {n: measure_prefill(n, 20, 3) for n in
                                      ("prefill_llama7b_mha_bf16", "chunked_prefill_gqa_bf16")}
         line["beam_search_fp16"] = measure_beam("beam_search_fp16", 200, 10)

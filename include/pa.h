@@ -158,6 +158,29 @@ int pa_decode_append(void *out, const void *query, const void *new_key, const vo
                      const int32_t *seq_order, cudaStream_t stream);
 
 /*
+ * pa_decode_withhold_stage -- pa_decode with a fault planted on the host, for
+ * testing the bounded waits; not for production use. The CTA of sequence
+ * `seq` (its index in the call), kv head `kv_head` never issues the copy of
+ * its 16-token stage `stage` (tokens 16 * stage .. 16 * stage + 15), so the
+ * warp that owns the stage waits for data that never comes. After
+ * wait_limit_ns (between 1e5 and 1e9; the library's own bound is 1 s) it
+ * records PA_DEVERR_TIMEOUT, waits with the same bound for the copies it
+ * still has in flight, and leaves its loop; the launch ends normally. That
+ * (sequence, kv head)'s output is undefined, every other output is
+ * pa_decode's. A stage past the sequence's end withholds nothing. Nothing
+ * faults and nothing hangs: this runs the path that a copy which never lands
+ * would take, so a test can check that it returns and reports. Other
+ * arguments as pa_decode; seq and kv_head out of range, stage < 0 or the
+ * limit out of range give PA_ERR_SHAPE.
+ */
+int pa_decode_withhold_stage(void *out, const void *query, const void *k_cache, const void *v_cache,
+                             const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                             int num_seqs, int num_heads, int num_kv_heads, int head_dim, float scale,
+                             int block_size, int num_blocks, pa_dtype kv_dtype, pa_dtype out_dtype,
+                             const int32_t *seq_order, int seq, int kv_head, int stage,
+                             unsigned long long wait_limit_ns, cudaStream_t stream);
+
+/*
  * Split-K (partitioned) decode for few, long sequences ([P5] §2.3: the
  * partitioned kernel of the pair). Tokens of sequence s are cut into
  * partitions of `partition_size` tokens (a multiple of block_size); partition

@@ -24,7 +24,9 @@ from __future__ import annotations
 from dataclasses import dataclass
 from typing import Dict, List, Sequence as Sequence_, Tuple
 
-from .block_pool import BlockPool, PoolExhausted
+import numpy as np
+
+from .block_pool import BlockPool, PoolExhausted, Sequence, append_tokens, fork, release
 
 
 @dataclass
@@ -71,3 +73,51 @@ class PrefixCacheManager:
 
     def num_entries(self) -> int:
         return len(self.cache)
+
+
+def request_flow(system_lens, system_tokens, choice, user_lens, num_blocks: int, free_order, block_size: int,
+                 max_blocks: int, finish_after=None):
+    """Requests that share system prompts through the cache, on a FIFO pool
+    handing out free_order: for request r in order, get_or_create its system
+    prompt's blocks (a miss is followed by the write of the prompt's K/V, token
+    t at slot block * block_size + t % block_size of the block holding t,
+    [P3 "Ascend C ... PagedAttention融合算子" §3.1]); fork them into the
+    request's own sequence; append its user tokens by the copy-on-write rule
+    ([P4] §3.3); then every request in finish_after[r] releases its prompt and
+    its blocks. Returns (ops as (kind, index, slots or pairs) in order, tables
+    int32 [R, max_blocks] (-1 where unused or finished), context lengths [R],
+    live [R])."""
+    R = len(choice)
+    pool = BlockPool(num_blocks, block_size, policy="fifo", free_order=[int(b) for b in free_order])
+    mgr = PrefixCacheManager(pool)
+    seqs = [None] * R
+    ops = []
+
+    def prompt_of(r):
+        p = int(choice[r])
+        return p, [int(t) for t in system_tokens[p][:int(system_lens[p])]]
+
+    for r in range(R):
+        p, prompt = prompt_of(r)
+        ids, hit = mgr.get_or_create(prompt)
+        if not hit:
+            ops.append(("prefix", p, [ids[t // block_size] * block_size + t % block_size
+                                      for t in range(len(prompt))]))
+        seqs[r] = fork(pool, Sequence(block_table=list(ids), num_tokens=len(prompt)))
+        slots, cow = append_tokens(pool, seqs[r], int(user_lens[r]))
+        if cow:
+            ops.append(("copy", r, [list(c) for c in cow]))
+        ops.append(("user", r, slots))
+        for j in (finish_after or {}).get(r, ()):
+            mgr.release(prompt_of(j)[1])
+            release(pool, seqs[j])
+            seqs[j] = None
+            ops.append(("finish", j, []))
+    tables = np.full((R, max_blocks), -1, np.int32)
+    ctx = np.zeros(R, np.int32)
+    live = np.array([sq is not None for sq in seqs])
+    for r, sq in enumerate(seqs):
+        if sq is not None:
+            tables[r, :len(sq.block_table)] = sq.block_table
+            ctx[r] = sq.num_tokens
+    return ops, tables, ctx, live

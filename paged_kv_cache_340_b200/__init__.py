@@ -6,7 +6,8 @@ Argument marshalling only: every operation runs in the CUDA kernels of
 and streams. There is no CPU or library fallback: if the shared library is
 missing, the first call raises.
 
-Calls: slot write (pa_reshape_and_cache), decode (pa_decode), the slot write
+Calls: slot write (pa_reshape_and_cache), decode (pa_decode; and
+pa_decode_withhold_stage, which tests its bounded waits), the slot write
 of each sequence's newest token with decode in one launch (pa_decode_append),
 split-K decode and reduce (pa_decode_splitk, pa_splitk_reduce,
 pa_decode_splitk_static),
@@ -55,7 +56,7 @@ EXPORTED = (
     "pa_prefix_cache_create", "pa_prefix_cache_destroy", "pa_prefix_num_entries", "pa_prefix_get_or_create",
     "pa_prefix_release", "pa_prefix_ref_count", "pa_copy_blocks_counted", "pa_dpool_state_bytes", "pa_dpool_init",
     "pa_beam_step", "pa_pool_export", "pa_dpool_load", "pa_reshape_and_cache_q8", "pa_decode_q8",
-    "pa_decode_splitk_q8", "pa_copy_blocks_q8", "pa_decode_append",
+    "pa_decode_splitk_q8", "pa_copy_blocks_q8", "pa_decode_append", "pa_decode_withhold_stage",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -81,6 +82,8 @@ def _load() -> ctypes.CDLL:
         "pa_decode": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32, vp, vp]),
         "pa_decode_append": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32,
                                    vp, vp]),
+        "pa_decode_withhold_stage": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32,
+                                           vp, i32, i32, i32, ctypes.c_ulonglong, vp]),
         "pa_splitk_workspace_bytes": (sz, [i32, i32, i32, i32, i32]),
         "pa_splitk_acc_offset": (sz, [i32, i32, i32, i32]),
         "pa_decode_splitk": (i32, [vp, sz, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32,
@@ -194,6 +197,20 @@ def pa_decode(out, query, k_cache, v_cache, block_tables, context_lens, scale, s
                         block_tables.shape[1], _ptr(context_lens), S, Hq, Hkv, D, float(scale), bs, NB,
                         _dtype(k_cache), _dtype(out), _ptr(seq_order), _stream(stream))
     _check(rc, "pa_decode")
+
+
+def pa_decode_withhold_stage(out, query, k_cache, v_cache, block_tables, context_lens, scale, seq, kv_head, stage,
+                             wait_limit_ns, seq_order=None, stream=None) -> None:
+    """pa_decode with the copy of one 16-token stage of one (sequence, kv
+    head) withheld, so that its bounded wait runs out (a test of the timeout
+    path; that head group's output is undefined)."""
+    S, Hq, D = query.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    rc = _lib.pa_decode_withhold_stage(_ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                       block_tables.shape[1], _ptr(context_lens), S, Hq, Hkv, D, float(scale), bs, NB,
+                                       _dtype(k_cache), _dtype(out), _ptr(seq_order), int(seq), int(kv_head),
+                                       int(stage), int(wait_limit_ns), _stream(stream))
+    _check(rc, "pa_decode_withhold_stage")
 
 
 def pa_decode_append(out, query, new_key, new_value, k_cache, v_cache, block_tables, context_lens, scale,

@@ -15,7 +15,7 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (PA_POOL_FIFO, BlockPool, DevicePool, pa_beam_step, pa_choose_partition, pa_copy_blocks,
+from . import (PA_POOL_FIFO, BlockPool, DevicePool, PrefixCache, pa_beam_step, pa_choose_partition, pa_copy_blocks,
                pa_copy_blocks_counted, pa_copy_blocks_q8, pa_decode, pa_decode_append, pa_decode_q8, pa_decode_splitk,
                pa_decode_splitk_q8, pa_prefill, pa_reshape_and_cache, pa_reshape_and_cache_q8, pa_splitk_reduce,
                pa_splitk_workspace_bytes)
@@ -194,6 +194,117 @@ def build_parallel_sampling_batch(spec: Spec, inputs: dict, device="cuda", parti
         host_tables=tables, host_slots=slots, host_cow=cow_all, host_context_lens=ctx,
         prefix_key=inputs["prefix_key"].reshape(P * L0, Hkv, D).to(dev),
         prefix_value=inputs["prefix_value"].reshape(P * L0, Hkv, D).to(dev),
+        prefix_slots=torch.from_numpy(prefix_slots).to(dev), host_prefix_slots=prefix_slots)
+
+
+def shared_prefix_order(ctx: np.ndarray, group_of: np.ndarray) -> np.ndarray:
+    """Scheduling order for sequences that share prefixes: sequences of one
+    group (same prefix) stay together, so the shared blocks are read while
+    they are still in L2; groups by their longest member, members longest
+    first."""
+    ctx = ctx.astype(np.int64)
+    groups = np.unique(group_of)
+    longest = np.array([ctx[group_of == g].max() for g in groups])
+    order = []
+    for gi in np.argsort(-longest, kind="stable"):
+        members = np.nonzero(group_of == groups[gi])[0]
+        order += members[np.argsort(-ctx[members], kind="stable")].tolist()
+    return np.array(order, np.int32)
+
+
+@dataclass
+class PrefixOp:
+    """One device step of the prefix-cache flow, in the order the host took it."""
+    kind: str          # "prefix": write system prompt `index`'s K/V; "copy": copy-on-write pairs;
+                       # "user": request `index`'s own tokens; "finish": request `index` is done
+    index: int
+    slots: np.ndarray  # int32 slots ("prefix", "user") or int64 [n, 2] pairs ("copy"); empty for "finish"
+
+
+def prefix_cache_flow(spec: Spec, inputs: dict, finish_after: Optional[dict] = None,
+                      pool_policy: int = PA_POOL_FIFO):
+    """Host side of requests that share system prompts through the prefix
+    cache ([P4] "PagedAttention 实现细节" §3.2, with the copy-on-write rule of
+    §3.3). For request r in order: get_or_create its system prompt's blocks
+    (a miss is followed by the write of the prompt's K/V into them); fork them
+    into the request's own table row (its own reference to each block); append
+    its user tokens (the first write into the shared partial last block
+    copies it). finish_after maps r to requests that finish once r is set up:
+    the cache releases their prompt and the pool their blocks, which later
+    requests may then be handed. Returns (ops in order, tables [R, MB], ctx
+    [R], live [R] bool)."""
+    bs = spec.block_size
+    lens = inputs["system_lens"].numpy().astype(np.int64)
+    toks = inputs["system_tokens"].numpy()
+    choice = inputs["choice"].numpy().astype(np.int64)
+    ulens = inputs["user_lens"].numpy().astype(np.int64)
+    R = choice.shape[0]
+    mb = _blocks(spec.prefix_len + spec.max_divergent, bs)
+    pool = BlockPool(int(inputs["num_blocks"]), bs, pool_policy, free_order=inputs["free_order"].numpy())
+    cache = PrefixCache(pool)
+    tables = np.full((R, mb), -1, np.int32)
+    ctx = np.zeros(R, np.int32)
+    live = np.zeros(R, bool)
+    ops = []
+    for r in range(R):
+        p = int(choice[r])
+        L0 = int(lens[p])
+        ids, hit = cache.get_or_create(toks[p, :L0])
+        ids = np.array(ids, np.int32)
+        if not hit:  # the prompt's K/V go into the blocks the cache just took
+            t = np.arange(L0, dtype=np.int64)
+            ops.append(PrefixOp("prefix", p, (ids[t // bs].astype(np.int64) * bs + t % bs).astype(np.int32)))
+        pool.fork(ids, L0, tables[r])
+        nt, sl, cow = pool.append(tables[r], L0, int(ulens[r]), cow_capacity=4)
+        if cow.shape[0]:
+            ops.append(PrefixOp("copy", r, cow))
+        ops.append(PrefixOp("user", r, sl))
+        ctx[r] = nt
+        live[r] = True
+        for j in (finish_after or {}).get(r, ()):
+            assert live[j]
+            cache.release(toks[int(choice[j]), :int(lens[int(choice[j])])])
+            pool.release(tables[j], int(ctx[j]))
+            tables[j] = -1
+            ctx[j] = 0
+            live[j] = False
+            ops.append(PrefixOp("finish", j, np.empty(0, np.int32)))
+    return ops, tables, ctx, live
+
+
+def build_prefix_cache_batch(spec: Spec, inputs: dict, device="cuda", pool_policy: int = PA_POOL_FIFO
+                             ) -> SamplingBatch:
+    """The prefix-cache workload as a decode step: every system prompt the
+    requests use is written once (set-up, write_prefix); a step copies the
+    shared partial blocks each request writes into, writes the requests' own
+    tokens and decodes every request."""
+    ops, tables, ctx, _ = prefix_cache_flow(spec, inputs, pool_policy=pool_policy)
+    dev = torch.device(device)
+    Hkv, D, bs = spec.num_kv_heads, spec.head_dim, spec.block_size
+    R = ctx.shape[0]
+    pre = [o for o in ops if o.kind == "prefix"]
+    lens = inputs["system_lens"].numpy()
+    prefix_key = torch.cat([inputs["prefix_key"][o.index, :int(lens[o.index])] for o in pre])
+    prefix_value = torch.cat([inputs["prefix_value"][o.index, :int(lens[o.index])] for o in pre])
+    prefix_slots = np.concatenate([o.slots for o in pre]).astype(np.int32)
+    cows = [o.slots for o in ops if o.kind == "copy"]
+    cow_all = np.concatenate(cows).astype(np.int64) if cows else np.empty((0, 2), np.int64)
+    slots = np.concatenate([o.slots for o in ops if o.kind == "user"]).astype(np.int32)
+    nb = int(inputs["num_blocks"])
+    dt = spec.torch_kv_dtype
+    return SamplingBatch(
+        spec=spec, num_blocks=nb,
+        k_cache=torch.zeros((nb, Hkv, bs, D), dtype=dt, device=dev),
+        v_cache=torch.zeros((nb, Hkv, bs, D), dtype=dt, device=dev),
+        query=inputs["query"].to(dev),
+        out=torch.empty((R, spec.num_heads, D), dtype=spec.torch_out_dtype, device=dev),
+        block_tables=torch.from_numpy(tables).to(dev), context_lens=torch.from_numpy(ctx).to(dev),
+        new_key=inputs["user_key"].to(dev), new_value=inputs["user_value"].to(dev),
+        slot_mapping=torch.from_numpy(slots).to(dev), cow_pairs=torch.from_numpy(cow_all).to(dev),
+        seq_order=torch.from_numpy(shared_prefix_order(ctx, inputs["choice"].numpy())).to(dev),
+        max_context_len=int(ctx.max()), partition_size=0, workspace=None,
+        host_tables=tables, host_slots=slots, host_cow=cow_all, host_context_lens=ctx,
+        prefix_key=prefix_key.to(dev), prefix_value=prefix_value.to(dev),
         prefix_slots=torch.from_numpy(prefix_slots).to(dev), host_prefix_slots=prefix_slots)
 
 

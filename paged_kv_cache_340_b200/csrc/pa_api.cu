@@ -195,11 +195,18 @@ int pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// The test hook of pa_decode_withhold_stage (none by default).
+struct WithholdHook {
+    int seq = -1, kv_head = -1, stage = -1;
+    unsigned long long wait_limit_ns = 0;
+};
+
 static int decode_unsplit(void *out, const void *query, const void *new_key, const void *new_value,
                           const void *k_cache, const void *v_cache, const int32_t *block_tables,
                           int max_blocks_per_seq, const int32_t *context_lens, int num_seqs, int num_heads,
                           int num_kv_heads, int head_dim, float scale, int block_size, int num_blocks,
-                          pa_dtype kv_dtype, pa_dtype out_dtype, const int32_t *seq_order, cudaStream_t stream) {
+                          pa_dtype kv_dtype, pa_dtype out_dtype, const int32_t *seq_order, cudaStream_t stream,
+                          const WithholdHook &hook = WithholdHook()) {
     int rc = check_decode_args(query, k_cache, v_cache, block_tables, max_blocks_per_seq,
                                context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale,
                                block_size, num_blocks, kv_dtype);
@@ -231,6 +238,10 @@ static int decode_unsplit(void *out, const void *query, const void *new_key, con
     p.err = err;
     p.new_key = new_key;
     p.new_value = new_value;
+    p.withhold_seq = hook.seq;
+    p.withhold_kvh = hook.kv_head;
+    p.withhold_stage = hook.stage;
+    p.wait_limit_ns = hook.wait_limit_ns;
     cudaError_t e = launch_decode(p, kv_dtype, head_dim, block_size, num_heads / num_kv_heads, 1,
                                   num_kv_heads, num_seqs, stream);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
@@ -255,6 +266,24 @@ int pa_decode_append(void *out, const void *query, const void *new_key, const vo
     return decode_unsplit(out, query, new_key, new_value, k_cache, v_cache, block_tables, max_blocks_per_seq,
                           context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale, block_size,
                           num_blocks, kv_dtype, out_dtype, seq_order, stream);
+}
+
+int pa_decode_withhold_stage(void *out, const void *query, const void *k_cache, const void *v_cache,
+                             const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                             int num_seqs, int num_heads, int num_kv_heads, int head_dim, float scale,
+                             int block_size, int num_blocks, pa_dtype kv_dtype, pa_dtype out_dtype,
+                             const int32_t *seq_order, int seq, int kv_head, int stage,
+                             unsigned long long wait_limit_ns, cudaStream_t stream) {
+    if (seq < 0 || seq >= num_seqs || kv_head < 0 || kv_head >= num_kv_heads || stage < 0) return PA_ERR_SHAPE;
+    if (wait_limit_ns < 100000ull || wait_limit_ns > 1000000000ull) return PA_ERR_SHAPE;
+    WithholdHook hook;
+    hook.seq = seq;
+    hook.kv_head = kv_head;
+    hook.stage = stage;
+    hook.wait_limit_ns = wait_limit_ns;
+    return decode_unsplit(out, query, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                          context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale, block_size,
+                          num_blocks, kv_dtype, out_dtype, seq_order, stream, hook);
 }
 
 size_t pa_splitk_acc_offset(int num_seqs, int num_heads, int max_context_len, int partition_size) {

@@ -811,6 +811,8 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
         t_end = min(t_begin + p.partition_size, ctx);
     }
     const int nstage = (t_end - t_begin + S::kTS - 1) / S::kTS;  // 16-token stages
+    const uint64_t wait_limit = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
+    const int withheld = (p.withhold_seq == s && p.withhold_kvh == kvh && part == 0) ? p.withhold_stage : -1;
     const size_t head0 = (size_t)s * p.num_heads + (size_t)kvh * G;  // first query head row
     if (nstage == 0) {  // unsplit, empty context: zeros
         for (int i = threadIdx.x; i < G * D; i += blockDim.x) store_out(p.out, head0 * D + i, 0.f, p.out_dtype);
@@ -856,7 +858,9 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     auto issue = [&](int m, int id) {  // lane 0
         const int k = warp + S::kWarps * m;
         const int buf = k % S::kStages;
-        if (id >= 0) {
+        if (k == withheld) {  // test hook: no copy and no arrival, so this stage's wait runs out
+            bad[buf] = 1;
+        } else if (id >= 0) {
             bad[buf] = 0;
             const size_t src = (size_t)id * block_elems + (size_t)(k % S::kSubs) * S::kTS * D;
             unsigned char *dst = ring + S::kVRegion + (size_t)buf * S::kStageBytes;
@@ -924,7 +928,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
         const int buf = k % S::kStages;
         // Lane 0 polls the barrier (32 lanes polling would serialise on it);
         // __syncwarp then orders the other lanes' reads after its acquire.
-        const bool got = mbar_wait(full + buf, (k / S::kStages) & 1);
+        const bool got = mbar_wait(full + buf, (k / S::kStages) & 1, wait_limit);
         if (!__all_sync(0xffffffffu, got)) {
             if (lane == 0) record_error(p.err, PA_DEVERR_TIMEOUT);
             ok = false;
@@ -970,7 +974,8 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     if (!ok && lane == 0) {  // after a timeout: let every copy this warp started land
         for (int m = waited; m < min(nmine, waited + S::kBufPerWarp); ++m) {
             const int k = warp + S::kWarps * m;
-            if (!mbar_wait(full + (k % S::kStages), (k / S::kStages) & 1)) record_error(p.err, PA_DEVERR_TIMEOUT);
+            if (!mbar_wait(full + (k % S::kStages), (k / S::kStages) & 1, wait_limit))
+                record_error(p.err, PA_DEVERR_TIMEOUT);
         }
     }
 

@@ -40,6 +40,15 @@ struct DecodeParams {
     // copy (pa_decode_append)
     const void *new_key;
     const void *new_value;
+    // Test hook of the bounded waits (pa_decode_withhold_stage): the CTA of
+    // sequence withhold_seq, kv head withhold_kvh (partition 0) never issues
+    // the copy of its 16-token stage withhold_stage, so that stage's wait runs
+    // out; every wait of the launch gives up after wait_limit_ns (0: the
+    // default bound). withhold_seq = -1 withholds nothing.
+    int withhold_seq = -1;
+    int withhold_kvh = -1;
+    int withhold_stage = -1;
+    unsigned long long wait_limit_ns = 0;
     // int8 caches with head_dim 128: the V pool as rows of 128 bytes, 16-row
     // boxes in the 128-byte swizzled layout (the kernel's V fragment loads are
     // then free of shared-memory bank conflicts)

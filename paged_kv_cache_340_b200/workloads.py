@@ -29,6 +29,11 @@ Workloads (shapes follow LLaMA-style decode layers):
   llama7b_mha_int8     llama7b_mha_fp16's shapes and values with an int8 cache (the fp16
                        values quantized at the slot write); fp16 query and out
   gqa_int8             gqa_bf16's shapes and values with an int8 cache; bf16 query, fp32 out
+  prefix_cache_fp16    96 requests, each a system prompt (one of 4, lengths U{500..2000},
+                       chosen uniformly) followed by U{1..256} user tokens; 32 heads,
+                       head_dim 128, block 16; the prompts' blocks come from the prefix
+                       cache (written once, shared by every request that uses them);
+                       q/k/v ~ N(0,1); fp16 out
   beam_search_fp16     32 prompts of U{256..1024} tokens x beam width 4 (128 beams),
                        32 heads, head_dim 128, block 16; every step each beam picks a
                        parent among its prompt's 4 beams (uniform) and writes one token;
@@ -113,6 +118,9 @@ SPECS: Dict[str, Spec] = {
                              ("uniform", 256, 2048), 1.1, q_scale=0.5, kv_scale=0.5, q_dtype="f16"),
     "gqa_int8": Spec("gqa_int8", 256, 32, 8, 128, 16, "i8", "f32", 3409,
                      ("lognormal", 1024, 0.5, 128, 4096), 1.1, q_dtype="bf16"),
+    # prefix cache: requests share a few system prompts' blocks through the prefix cache
+    "prefix_cache_fp16": Spec("prefix_cache_fp16", 96, 32, 32, 128, 16, "f16", "f16", 3410,
+                              ("prefix", 500, 2000), None, num_prompts=4, prefix_len=2000, max_divergent=256),
     # beam search: the beam step (fork, release, copy-on-write) on the device, then decode
     "beam_search_fp16": Spec("beam_search_fp16", 128, 32, 32, 128, 16, "f16", "f16", 3407,
                              ("uniform", 256, 1024), None, num_prompts=32, branches=4, max_divergent=512),
@@ -220,6 +228,41 @@ def make_parallel_sampling_inputs(spec: Spec) -> dict:
     return dict(prefix_key=prefix_key, prefix_value=prefix_value, divergent_lens=div,
                 divergent_key=divergent_key, divergent_value=divergent_value, query=query,
                 free_order=free_order, num_blocks=nb)
+
+
+def make_prefix_cache_inputs(spec: Spec) -> dict:
+    """Inputs for the prefix-cache workload: num_prompts system prompts
+    (lengths U{lo..hi} of the spec's law, random token ids), and num_seqs
+    requests, each one system prompt (chosen uniformly) followed by
+    U{1..max_divergent} user tokens.
+
+    Returns CPU tensors: system_lens [P] int32; system_tokens [P, prefix_len]
+    int32 (the first system_lens[p] are prompt p's tokens); choice [R] int32;
+    user_lens [R] int32; prefix_key/prefix_value [P, prefix_len, Hkv, D];
+    user_key/user_value [sum(user_lens), Hkv, D] in request order; query
+    [R, Hq, D]; free_order [NB] int32; num_blocks (room for every prompt and
+    request, with no block ever freed)."""
+    assert spec.lengths[0] == "prefix"
+    lo, hi = spec.lengths[1], spec.lengths[2]
+    gen = torch.Generator().manual_seed(spec.seed)
+    dt = spec.torch_kv_dtype
+    P, R, bs = spec.num_prompts, spec.num_seqs, spec.block_size
+    system_lens = torch.randint(lo, hi + 1, (P,), generator=gen, dtype=torch.int64).to(torch.int32)
+    system_tokens = torch.randint(0, 1 << 30, (P, spec.prefix_len), generator=gen, dtype=torch.int64).to(torch.int32)
+    choice = torch.randint(0, P, (R,), generator=gen, dtype=torch.int64).to(torch.int32)
+    user_lens = torch.randint(1, spec.max_divergent + 1, (R,), generator=gen, dtype=torch.int64).to(torch.int32)
+    nb = P * ((spec.prefix_len + bs - 1) // bs) + R * ((spec.max_divergent + bs - 1) // bs + 2)
+    free_order = torch.randperm(nb, generator=gen).to(torch.int32)
+    kv = (spec.num_kv_heads, spec.head_dim)
+    prefix_key = _normal(gen, (P, spec.prefix_len) + kv, spec.kv_scale, dt)
+    prefix_value = _normal(gen, (P, spec.prefix_len) + kv, spec.kv_scale, dt)
+    total = int(user_lens.sum())
+    user_key = _normal(gen, (total,) + kv, spec.kv_scale, dt)
+    user_value = _normal(gen, (total,) + kv, spec.kv_scale, dt)
+    query = _normal(gen, (R, spec.num_heads, spec.head_dim), spec.q_scale, dt)
+    return dict(system_lens=system_lens, system_tokens=system_tokens, choice=choice, user_lens=user_lens,
+                prefix_key=prefix_key, prefix_value=prefix_value, user_key=user_key, user_value=user_value,
+                query=query, free_order=free_order, num_blocks=nb)
 
 
 def make_prefill_inputs(spec: Spec) -> dict:

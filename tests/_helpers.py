@@ -103,3 +103,12 @@ def compact_for(k_pool: torch.Tensor, v_pool: torch.Tensor, table_row: np.ndarra
         h = torch.as_tensor(kv_heads, dtype=torch.int64)
         kp, vp = kp.index_select(1, h), vp.index_select(1, h)
     return kp.double().numpy(), vp.double().numpy(), np.arange(max(nb, 1), dtype=np.int32)[None, :]
+
+
+
+def oracle_prefix_cache_flow(inputs: dict, block_size: int, prefix_len: int, max_user: int, finish_after=None):
+    """The oracle's prefix-cache request flow on a workload's inputs."""
+    from oracle.prefix_cache import request_flow
+    return request_flow(inputs["system_lens"].numpy(), inputs["system_tokens"].numpy(), inputs["choice"].numpy(),
+                        inputs["user_lens"].numpy(), int(inputs["num_blocks"]), inputs["free_order"].numpy(),
+                        block_size, oracle.blocks_needed(prefix_len + max_user, block_size), finish_after)

@@ -197,3 +197,57 @@ def test_library_prefix_errors(pa):
     assert rc == -13
     assert pa._lib.pa_prefix_cache_create(None, 0) is None
     assert pa._lib.pa_prefix_cache_create(lp._h, 65) is None
+
+
+def test_oracle_request_flow_hand_worked():
+    """Requests over the cache, worked by hand (pool of 8 blocks of 4 tokens,
+    FIFO from 0): prompt A = 6 tokens (blocks 0, 1; block 1 partial), B = 3.
+    r0 (A + 3): miss, writes A at slots 0..5, copies block 1 -> 2 before its
+    first token (slot 10), then 11 and a new block 3 (12). r1 (A + 1): hit,
+    copies 1 -> 4 (slot 18). r0 finishes: blocks 2 and 3 return to the free
+    list's end (5, 6, 7, 2, 3); block 0 stays (cache and r1). r2 (A + 2): hit,
+    copies 1 -> 5 (slots 22, 23). r3 (B + 1): miss, block 6 (slots 24..26),
+    copied to 7 before its own token (slot 31)."""
+    from oracle.prefix_cache import request_flow
+    A = [11, 12, 13, 14, 15, 16]
+    B = [21, 22, 23]
+    toks = np.zeros((2, 6), np.int32)
+    toks[0, :6], toks[1, :3] = A, B
+    ops, tables, ctx, live = request_flow([6, 3], toks, [0, 0, 0, 1], [3, 1, 2, 1], 8, list(range(8)), 4, 3,
+                                          finish_after={1: [0]})
+    assert ops == [("prefix", 0, [0, 1, 2, 3, 4, 5]), ("copy", 0, [[1, 2]]), ("user", 0, [10, 11, 12]),
+                   ("copy", 1, [[1, 4]]), ("user", 1, [18]), ("finish", 0, []),
+                   ("copy", 2, [[1, 5]]), ("user", 2, [22, 23]),
+                   ("prefix", 1, [24, 25, 26]), ("copy", 3, [[6, 7]]), ("user", 3, [31])]
+    assert tables.tolist() == [[-1, -1, -1], [0, 4, -1], [0, 5, -1], [7, -1, -1]]
+    assert ctx.tolist() == [0, 7, 8, 4] and live.tolist() == [False, True, True, True]
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_library_request_flow_matches_oracle(pa, seed):
+    """The library's host flow (its pool and prefix cache) makes the oracle's
+    decisions: the same prefix writes, copy pairs, slots, tables and lengths,
+    with requests finishing (and prompts released and re-created) mid-flow."""
+    from paged_kv_cache_340_b200.batch import prefix_cache_flow
+    from paged_kv_cache_340_b200.workloads import SPECS, make_prefix_cache_inputs, scaled
+    from oracle.prefix_cache import request_flow
+    spec = scaled(SPECS["prefix_cache_fp16"], seed=100 + seed, num_seqs=40, num_heads=2, num_kv_heads=2,
+                  head_dim=64, lengths=("prefix", 1, 120), num_prompts=4, prefix_len=120, max_divergent=50)
+    inp = make_prefix_cache_inputs(spec)
+    rng = np.random.default_rng(seed)
+    finish_after, alive = {}, []
+    for r in range(40):
+        alive.append(r)
+        if rng.random() < 0.4 and len(alive) > 1:
+            done = [int(x) for x in rng.choice(alive, size=int(rng.integers(1, len(alive))), replace=False)]
+            finish_after[r] = done
+            alive = [a for a in alive if a not in done]
+    ops, tables, ctx, live = prefix_cache_flow(spec, inp, finish_after=finish_after)
+    want = request_flow(inp["system_lens"].numpy(), inp["system_tokens"].numpy(), inp["choice"].numpy(),
+                        inp["user_lens"].numpy(), int(inp["num_blocks"]), inp["free_order"].numpy(),
+                        spec.block_size, tables.shape[1], finish_after)
+    assert [(o.kind, o.index) for o in ops] == [(k, i) for k, i, _ in want[0]]
+    for o, (_, _, w) in zip(ops, want[0]):
+        assert np.array_equal(o.slots.reshape(-1), np.asarray(w, np.int64).reshape(-1))
+    assert np.array_equal(tables, want[1]) and np.array_equal(ctx, want[2]) and np.array_equal(live, want[3])
+    assert sum(o.kind == "prefix" for o in ops) > spec.num_prompts   # some prompt was released and written again
