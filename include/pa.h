@@ -29,11 +29,10 @@
  *       slot_mapping      [num_tokens] int32
  *     Token t of sequence s is row (block_tables[s][t / block_size], kv head,
  *     t % block_size) of the pools ([P2] §3.1; [P4] §3.1 index-based kernel).
- *   - Supported: head_dim 64 or 128; block_size 16 or 32; num_heads a
- *     multiple of num_kv_heads with num_heads / num_kv_heads in {1, 2, 4, 8}
- *     (query head h reads kv head h / (num_heads / num_kv_heads)); element
- *     types PA_F32, PA_F16, PA_BF16. Every device pointer must be 16-byte
- *     aligned.
+ *   - Supported: head_dim 64 or 128; block_size 16 or 32; num_heads any
+ *     multiple of num_kv_heads (query head h reads kv head
+ *     h / (num_heads / num_kv_heads)); element types PA_F32, PA_F16,
+ *     PA_BF16. Every device pointer must be 16-byte aligned.
  *   - Calls are asynchronous on `stream` (NULL = the legacy default stream)
  *     and return PA_OK once the work is enqueued. Arguments are checked on
  *     the host first; a violation returns a negative pa_status and enqueues
@@ -62,7 +61,7 @@ typedef enum pa_status {
     PA_ERR_NULL = -1,            /* a required pointer is NULL */
     PA_ERR_DTYPE = -2,           /* unsupported element type or output type */
     PA_ERR_SHAPE = -3,           /* a size is negative or inconsistent */
-    PA_ERR_HEADS = -4,           /* num_heads % num_kv_heads != 0 or group not in {1,2,4,8} */
+    PA_ERR_HEADS = -4,           /* num_heads % num_kv_heads != 0 */
     PA_ERR_HEAD_DIM = -5,        /* head_dim not in {64, 128} */
     PA_ERR_BLOCK_SIZE = -6,      /* block_size not in {16, 32} */
     PA_ERR_ALIGN = -7,           /* a device pointer is not 16-byte aligned */
@@ -464,12 +463,14 @@ int pa_prefix_ref_count(pa_prefix_cache *cache, const int32_t *tokens, int num_t
  *   ring  = ref + num_blocks                       [num_blocks] free list: entries
  *           ring[(head + k) % num_blocks], k < count, front first
  *   then four scratch arrays of num_blocks words each (all zero / -1 between
- *   calls). The library keeps no pointer to it.
+ *   calls), then PA_DPOOL_TAIL_WORDS words of step scratch (a status word and
+ *   per-chunk totals; zero between calls). The library keeps no pointer to it.
  * Same rules as the host pool: PA_POOL_FIFO takes the free list's front,
  * PA_POOL_LIFO its back; freed blocks go to the back.
  */
 #define PA_DPOOL_HEADER_WORDS 8
 #define PA_DPOOL_ARRAYS 6
+#define PA_DPOOL_TAIL_WORDS 1024
 
 size_t pa_dpool_state_bytes(int num_blocks);
 
@@ -508,7 +509,8 @@ int pa_dpool_load(void *state, int num_blocks, int block_size, int policy, const
  * Any error (a bad parent, context or block id, a free list too short, no
  * table room for the new token, an uninitialised state) applies nothing:
  * the state is unchanged, every slot is -1, *num_cow = 0 and a PA_DEVERR_*
- * bit is set. Runs as one CTA; calls on one state must not overlap.
+ * bit is set. Runs as four launches over chunks of the old tables (spread
+ * over the SMs); calls on one state must not overlap.
  * Limits (else PA_ERR_SHAPE): 3 * num_old + num_new <= PA_BEAM_MAX_STAGED
  * and (num_old + num_new) * max_blocks_per_seq < 2^30.
  */

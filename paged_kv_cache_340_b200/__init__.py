@@ -44,6 +44,7 @@ PA_DEVERR_TIMEOUT = 0x8
 PA_DEVERR_PAIR = 0x10
 PA_DEVERR_POOL = 0x20
 PA_DPOOL_HEADER_WORDS = 8
+PA_DPOOL_TAIL_WORDS = 1024
 
 PA_POOL_LIFO, PA_POOL_FIFO = 0, 1
 

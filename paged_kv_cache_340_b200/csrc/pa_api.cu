@@ -113,7 +113,8 @@ static int check_decode_args(const void *query, const void *k_cache, const void 
     if (block_size != 16 && block_size != 32) return PA_ERR_BLOCK_SIZE;
     if (num_heads % num_kv_heads != 0) return PA_ERR_HEADS;
     const int group = num_heads / num_kv_heads;
-    if (group != 1 && group != 2 && group != 4 && group != 8) return PA_ERR_HEADS;
+    // a group above 8 runs as sub-groups of 8 query heads, one CTA each along gridDim.y
+    if ((long long)num_kv_heads * ((group + 7) / 8) > 65535) return PA_ERR_SHAPE;
     if (max_blocks_per_seq > INT_MAX / block_size) return PA_ERR_SHAPE;
     if (num_seqs == 0) return PA_OK;
     if (!query || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_NULL;
@@ -145,7 +146,7 @@ const char *pa_status_string(int status) {
         case PA_ERR_NULL: return "a required pointer is NULL";
         case PA_ERR_DTYPE: return "unsupported element or output type";
         case PA_ERR_SHAPE: return "a size is negative, too large or inconsistent";
-        case PA_ERR_HEADS: return "num_heads must be num_kv_heads times 1, 2, 4 or 8";
+        case PA_ERR_HEADS: return "num_heads must be a multiple of num_kv_heads";
         case PA_ERR_HEAD_DIM: return "head_dim must be 64 or 128";
         case PA_ERR_BLOCK_SIZE: return "block_size must be 16 or 32";
         case PA_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
@@ -267,6 +268,52 @@ int pa_decode_append(void *out, const void *query, const void *new_key, const vo
                           context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale, block_size,
                           num_blocks, kv_dtype, out_dtype, seq_order, stream);
 }
+
+}  // extern "C"
+
+namespace pa {
+
+int prefill_cuda_cores(void *out, const void *query, const int32_t *q_start, int num_tokens, const void *k_cache,
+                       const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                       const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                       float scale, int block_size, int num_blocks, cudaStream_t stream) {
+    int rc = check_decode_args(query, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                               num_heads, num_kv_heads, head_dim, scale, block_size, num_blocks, PA_F32);
+    if (rc != PA_OK) return rc;
+    if (num_tokens < 0) return PA_ERR_SHAPE;
+    if (num_seqs == 0 || num_tokens == 0) return PA_OK;
+    if (!out || !q_start) return PA_ERR_NULL;
+    if (!aligned(out, 16) || !aligned(q_start, 4)) return PA_ERR_ALIGN;
+    if ((long long)num_tokens * num_heads >= INT_MAX) return PA_ERR_SHAPE;
+    unsigned int *err = nullptr;
+    if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
+    DecodeParams p{};
+    p.out = out;
+    p.query = query;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.q_start = q_start;
+    p.num_seqs = num_seqs;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.num_blocks = num_blocks;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.partition_size = 0;
+    p.max_parts = 1;
+    p.max_context_len = INT_MAX;
+    p.out_dtype = PA_F32;
+    p.err = err;
+    cudaError_t e = launch_decode(p, PA_F32, head_dim, block_size, num_heads / num_kv_heads, num_tokens,
+                                  num_kv_heads, 1, stream);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace pa
+
+extern "C" {
 
 int pa_decode_withhold_stage(void *out, const void *query, const void *k_cache, const void *v_cache,
                              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
@@ -601,7 +648,7 @@ int pa_copy_blocks_q8(int8_t *k_cache, int8_t *v_cache, float *k_scale, float *v
 
 size_t pa_dpool_state_bytes(int num_blocks) {
     if (num_blocks <= 0) return 0;
-    return (PA_DPOOL_HEADER_WORDS + (size_t)PA_DPOOL_ARRAYS * num_blocks) * sizeof(int32_t);
+    return (PA_DPOOL_HEADER_WORDS + (size_t)PA_DPOOL_ARRAYS * num_blocks + PA_DPOOL_TAIL_WORDS) * sizeof(int32_t);
 }
 
 int pa_dpool_init(void *state, int num_blocks, int block_size, int policy, const int32_t *free_order,

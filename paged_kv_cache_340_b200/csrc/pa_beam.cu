@@ -17,36 +17,35 @@
 //      takes a free block; otherwise, if its block's count is above 1, it
 //      takes a free block, records (old, new) for the copy and drops the old
 //      block's count; else it writes in place.
-// The kernel reaches that sequential result in parallel with one CTA:
+// The launches below reach that sequential result in parallel:
 //   * counts: net change per block accumulated with atomics in a scratch
 //     array, applied once;
 //   * free-list order: a block is freed at its last decrement, the largest
-//     flattened (beam, table position) index holding it; a block-wide scan
-//     over those indices gives each freed block its place;
+//     flattened (beam, table position) index holding it; per-chunk totals and
+//     a scan within each chunk give each freed block its place;
 //   * copy-on-write: writer i into block b finds count > 1 unless it is the
 //     last writer into b (largest i) and no other new beam holds b, so
 //     copies = (not last writer) or (other holders > 0);
-//   * takes: a block-wide scan of "needs a block" in beam order gives each
-//     writer its position in the free list (front for FIFO, back for LIFO).
+//   * takes: a scan of "needs a block" in beam order gives each writer its
+//     position in the free list (front for FIFO, back for LIFO).
 // Everything is checked before anything changes: on an error the state is
 // unchanged, every slot is -1 and the copy count is 0.
+#include <algorithm>
+
 #include "pa_common.cuh"
 #include "pa_internal.h"
 
 namespace pa {
 namespace beam {
 
-constexpr int kThreads = 1024;
-constexpr int kItems = 16;         // table entries per thread per pass
-constexpr int kScanItems = 8;      // the same in the scanned pass (four values per entry)
-// per-beam values staged in shared memory: 3 words per old beam, 1 per new beam
+constexpr int kThreads = 1024;     // pool set-up kernels
+// per-beam values staged in shared memory by each CTA of the step: 3 words
+// per old beam, 1 per new beam
 constexpr int kMaxStageBytes = PA_BEAM_MAX_STAGED * 4;
-// per-beam values plus the old tables, when they fit in this much
-constexpr int kMaxDynBytes = 200 * 1024;
 constexpr int32_t kMagic = 0x50414250;
 
 struct Pool {
-    int32_t *hdr, *ref, *ring, *delta, *last_old, *writers, *last_writer;
+    int32_t *hdr, *ref, *ring, *delta, *last_old, *writers, *last_writer, *tail;
 };
 
 __device__ __forceinline__ Pool views(int32_t *state, int nb) {
@@ -58,35 +57,8 @@ __device__ __forceinline__ Pool views(int32_t *state, int nb) {
     p.last_old = p.delta + nb;
     p.writers = p.last_old + nb;
     p.last_writer = p.writers + nb;
+    p.tail = p.last_writer + nb;
     return p;
-}
-
-// Exclusive scan of v over the CTA (all kThreads threads call it); *total
-// receives the sum. Ends with a barrier, so warp_sums can be reused.
-__device__ __forceinline__ int cta_exclusive_scan(int v, int *warp_sums, int *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, d);
-        if (lane >= d) x += y;
-    }
-    if (lane == 31) warp_sums[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int w = warp_sums[lane];
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, w, d);
-            if (lane >= d) w += y;
-        }
-        warp_sums[lane] = w;
-    }
-    __syncthreads();
-    const int excl = x - v + (warp ? warp_sums[warp - 1] : 0);
-    *total = warp_sums[31];
-    __syncthreads();
-    return excl;
 }
 
 __global__ void __launch_bounds__(256) dpool_fill_kernel(int32_t *state, int nb, const int32_t *free_order) {
@@ -99,6 +71,8 @@ __global__ void __launch_bounds__(256) dpool_fill_kernel(int32_t *state, int nb,
         p.writers[i] = 0;
         p.last_writer[i] = -1;
     }
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < PA_DPOOL_TAIL_WORDS; i += gridDim.x * blockDim.x)
+        p.tail[i] = 0;
 }
 
 // Checks that the free list is a permutation (using delta as a counter and
@@ -158,6 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.writers[i] = 0;
         p.last_writer[i] = -1;
     }
+    for (int i = threadIdx.x; i < PA_DPOOL_TAIL_WORDS; i += kThreads) p.tail[i] = 0;
     __syncthreads();
     int zeros = 0;
     for (int i = threadIdx.x; i < nb; i += kThreads) {
@@ -207,370 +182,402 @@ struct StepParams {
     int max_blocks;
     int num_blocks;
     int block_size;
+    int chunk;       // old-table entries per CTA
+    int num_chunks;  // CTAs of each launch
     unsigned int *err;
+};
+
+// ------------------------------------------------------------------ beam step
+//
+// Four launches over chunks of the old tables' entries (flattened (beam,
+// position) index e = j * max_blocks + pos), so that the passes over the
+// tables and their atomics spread over the SMs; a kernel boundary is the
+// only grid-wide ordering used. Every CTA first stages the per-beam values
+// (context length, block count, number of children, parent) in shared
+// memory and makes the same argument checks, so all CTAs agree on them
+// without a global exchange. Between launches the step keeps a status word
+// and per-chunk totals in the state's tail.
+//   1. count:  validate each entry in use (block id in range, count > 0);
+//              delta[b] += children - 1 for beams without exactly one
+//              child; last_old[b] = max e over beams with no child; count
+//              the writers into each block (writers, last_writer).
+//   2. flags:  an entry frees its block if the block's count reaches 0 and
+//              it is the block's last release (last_old[b] == e); per-chunk
+//              totals of such entries; blocks whose count stays above 0 get
+//              last_old = -2 so that later tests need no count. CTA 0 also
+//              totals the blocks the new tokens take.
+//   3. apply:  freed blocks go to the back of the free list in entry order
+//              (chunk prefix + rank within the chunk); counts take their net
+//              change; the new tables get their parents' rows (except the
+//              entry each new beam writes into).
+//   4. finish: CTA 0 decides, in beam order, the block each new token takes
+//              and the copies (scans over the new beams), writes slots,
+//              context lengths and pairs, updates the header and clears the
+//              status; every CTA clears the release marks of its chunk.
+// Everything that changes the pool happens in launch 3 and 4, and only if
+// launches 1 and 2 found nothing wrong (status 0) and the free list is long
+// enough; otherwise the pool is left as it was, every slot is -1 and the
+// copy count is 0.
+
+constexpr int kStepThreads = 256;
+constexpr int kMaxChunks = PA_DPOOL_TAIL_WORDS - 4;
+// tail words: [0] status bits of this step, [1] blocks taken, [2] copies,
+// [4 + c] freed blocks in chunk c
+
+struct Staged {
+    int *ctx, *nblk, *nch, *par;
+    int bad;  // PA_DEVERR_* bits of the checks every CTA makes alike
 };
 
 __device__ __forceinline__ int nblk(int ctx, int bs) { return (ctx + bs - 1) / bs; }
 
-// Beam j and table position pos of the flattened entries e0, e0 + stride, ...
-// of [beams][mb] tables: one division, then per step one add and at most one
-// carry (the step's remainder is below mb). The passes below visit 16 entries
-// per thread; a division per entry cost more than the memory traffic.
-struct EntryWalk {
-    int j, pos;
-    __device__ __forceinline__ EntryWalk(int e0, int mb) : j(e0 / mb), pos(e0 % mb) {}
-    __device__ __forceinline__ void step(int dj, int dpos, int mb) {
-        j += dj;
-        pos += dpos;
-        if (pos >= mb) {
-            pos -= mb;
-            ++j;
-        }
+// Stages the per-beam values and checks the header, contexts and parents.
+__device__ Staged stage_beams(const StepParams &q, const Pool &p, int *dyn, int *s_bad) {
+    Staged st;
+    const int n_old = q.num_old, n_new = q.num_new, bs = q.block_size, MB = q.max_blocks;
+    st.ctx = dyn;
+    st.nblk = dyn + n_old;
+    st.nch = dyn + 2 * n_old;
+    st.par = dyn + 3 * n_old;
+    if (threadIdx.x == 0) {
+        *s_bad = 0;
+        const int count = p.hdr[4], head = p.hdr[3];
+        if (p.hdr[5] != kMagic || p.hdr[0] != q.num_blocks || p.hdr[1] != bs || count < 0 ||
+            count > q.num_blocks || head < 0 || head >= q.num_blocks)
+            *s_bad = PA_DEVERR_POOL;
     }
-};
-
-// The kernel is latency-bound (one CTA, dependent loads), so every pass over
-// table entries first loads kItems entries per thread into registers, then
-// acts on them: one or two memory round trips per pass instead of one per
-// entry. Table, context and parent arrays are read-only here (__ldg).
-// kStaged: the old tables are first copied to shared memory (when they fit),
-// so the passes below read them there instead of from L2.
-template <bool kStaged>
-__global__ void __launch_bounds__(kThreads, 1) beam_step_kernel(const StepParams q) {
-    extern __shared__ int dyn[];
-    __shared__ int warp_sums[32];
-    __shared__ int s_bad;
-    const int tid = threadIdx.x;
-    const int nb = q.num_blocks, bs = q.block_size, MB = q.max_blocks;
-    const Pool p = views(q.state, nb);
-    const int n_old = q.num_old, n_new = q.num_new;
-    const int old_entries = n_old * MB;  // < 2^31 (host check)
-    const int new_entries = n_new * MB;
-    const int sdj = kThreads / MB, sdp = kThreads % MB;  // a step of kThreads entries
-    int *s_ctx = dyn;                    // [n_old] context length of old beam j
-    int *s_nb = dyn + n_old;             // [n_old] its block count
-    int *s_nch = dyn + 2 * n_old;        // [n_old] its number of children
-    int *s_par = dyn + 3 * n_old;        // [n_new] parent of new beam i
-    int *s_tab = dyn + 3 * n_old + n_new;  // kStaged: [n_old * MB] the old tables
-    const int32_t *__restrict__ otab = q.old_tables;
-    auto tab = [&](int e) -> int {
-        if constexpr (kStaged)
-            return s_tab[e];
-        else
-            return __ldg(otab + e);
-    };
-
-    if (tid == 0) s_bad = 0;
-    __syncthreads();
-    const int policy = p.hdr[2], head = p.hdr[3], count = p.hdr[4];
-    if (tid == 0 && (p.hdr[5] != kMagic || p.hdr[0] != nb || p.hdr[1] != bs || count < 0 || count > nb ||
-                     head < 0 || head >= nb))
-        atomicOr(&s_bad, PA_DEVERR_POOL);
-    // ---- phase 0: stage and check the inputs (nothing is changed yet)
-    for (int j = tid; j < n_old; j += kThreads) {
+    for (int j = threadIdx.x; j < n_old; j += kStepThreads) {
         const int c = __ldg(q.old_ctx + j);
-        s_ctx[j] = c;
-        s_nb[j] = c < 0 ? 0 : nblk(c, bs);
-        s_nch[j] = 0;
-        if (c < 0 || nblk(c, bs) > MB) atomicOr(&s_bad, PA_DEVERR_CONTEXT);
-    }
-    if constexpr (kStaged) {
-        for (int base = 0; base < old_entries; base += kThreads * kItems) {
-            int v[kItems];
-#pragma unroll
-            for (int k = 0; k < kItems; ++k) {
-                const int e = base + k * kThreads + tid;
-                v[k] = e < old_entries ? __ldg(otab + e) : 0;
-            }
-#pragma unroll
-            for (int k = 0; k < kItems; ++k) {
-                const int e = base + k * kThreads + tid;
-                if (e < old_entries) s_tab[e] = v[k];
-            }
-        }
+        st.ctx[j] = c;
+        st.nblk[j] = c < 0 ? 0 : nblk(c, bs);
+        st.nch[j] = 0;
     }
     __syncthreads();
-    for (int i = tid; i < n_new; i += kThreads) {
+    for (int j = threadIdx.x; j < n_old; j += kStepThreads)
+        if (st.ctx[j] < 0 || st.nblk[j] > MB) atomicOr(s_bad, PA_DEVERR_CONTEXT);
+    for (int i = threadIdx.x; i < n_new; i += kStepThreads) {
         const int par = __ldg(q.parents + i);
-        s_par[i] = par;
-        if (par < 0 || par >= n_old)
-            atomicOr(&s_bad, PA_DEVERR_CONTEXT);
-        else
-            atomicAdd(&s_nch[par], 1);
+        st.par[i] = par;
+        if (par < 0 || par >= n_old) {
+            atomicOr(s_bad, PA_DEVERR_CONTEXT);
+        } else {
+            atomicAdd(&st.nch[par], 1);
+            if (st.ctx[par] >= 0 && st.ctx[par] / bs >= MB) atomicOr(s_bad, PA_DEVERR_POOL);  // no room
+        }
     }
     __syncthreads();
-    if (!s_bad) {
-        for (int base = 0; base < old_entries; base += kThreads * kItems) {
-            int blk[kItems], in_use = 0;
-            EntryWalk w(base + tid, MB);
-#pragma unroll
-            for (int k = 0; k < kItems; ++k) {
-                const int e = base + k * kThreads + tid;
-                blk[k] = 0;
-                if (e < old_entries && w.pos < s_nb[w.j]) {
-                    blk[k] = tab(e);
-                    in_use |= 1 << k;
-                }
-                w.step(sdj, sdp, MB);
-            }
-#pragma unroll
-            for (int k = 0; k < kItems; ++k) {
-                const int b = blk[k];
-                if ((in_use >> k & 1) && (b < 0 || b >= nb || p.ref[b] <= 0)) atomicOr(&s_bad, PA_DEVERR_BLOCK_ID);
-            }
-        }
-        for (int i = tid; i < n_new; i += kThreads)
-            if (s_ctx[s_par[i]] / bs >= MB) atomicOr(&s_bad, PA_DEVERR_POOL);  // no room for the token
-    }
-    __syncthreads();
-    if (s_bad) {
-        for (int i = tid; i < n_new; i += kThreads) q.slots[i] = -1;
-        if (tid == 0) {
-            *q.num_cow = 0;
-            record_error(q.err, (unsigned)s_bad);
-        }
+    st.bad = *s_bad;
+    return st;
+}
+
+// This CTA's chunk of old-table entries: [e0, e1).
+__device__ __forceinline__ void chunk_of(const StepParams &q, int *e0, int *e1) {
+    const long long entries = (long long)q.num_old * q.max_blocks;
+    const long long b = (long long)blockIdx.x * q.chunk;
+    *e0 = (int)min(b, entries);
+    *e1 = (int)min(b + q.chunk, entries);
+}
+
+__device__ __forceinline__ volatile int *status_word(const Pool &p) { return p.tail; }
+
+__global__ void __launch_bounds__(kStepThreads) beam_count_kernel(const StepParams q) {
+    extern __shared__ int dyn[];
+    __shared__ int s_bad;
+    const Pool p = views(q.state, q.num_blocks);
+    const Staged st = stage_beams(q, p, dyn, &s_bad);
+    if (st.bad) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.tail, st.bad);
         return;
     }
-
-    // ---- phase 1: net count change. A child's table is its parent's, so a
-    // block of old beam j gains (children of j) - 1 references: only beams
-    // with other than one child touch the counts. Then the writers.
-    for (int base = 0; base < old_entries; base += kThreads * kItems) {
-        int blk[kItems];
-        EntryWalk w(base + tid, MB);
-#pragma unroll
-        for (int k = 0; k < kItems; ++k) {
-            const int e = base + k * kThreads + tid;
-            blk[k] = -1;
-            if (e < old_entries && w.pos < s_nb[w.j] && s_nch[w.j] != 1) blk[k] = tab(e);
-            w.step(sdj, sdp, MB);
+    const int MB = q.max_blocks, nb = q.num_blocks, bs = q.block_size;
+    int e0, e1;
+    chunk_of(q, &e0, &e1);
+    for (int e = e0 + threadIdx.x; e < e1; e += kStepThreads) {
+        const int j = e / MB, pos = e - j * MB;
+        if (pos >= st.nblk[j]) continue;
+        const int b = __ldg(q.old_tables + e);
+        if (b < 0 || b >= nb || p.ref[b] <= 0) {
+            atomicOr(p.tail, PA_DEVERR_BLOCK_ID);
+            continue;
         }
-        EntryWalk w2(base + tid, MB);
-#pragma unroll
-        for (int k = 0; k < kItems; ++k) {
-            if (blk[k] >= 0) atomicAdd(&p.delta[blk[k]], s_nch[w2.j] - 1);
-            w2.step(sdj, sdp, MB);
-        }
+        const int n = st.nch[j];
+        if (n != 1) atomicAdd(&p.delta[b], n - 1);
+        if (n == 0) atomicMax(&p.last_old[b], e);
     }
-    for (int i = tid; i < n_new; i += kThreads) {
-        const int par = s_par[i];
-        const int t = s_ctx[par];
+    for (int i = blockIdx.x * kStepThreads + threadIdx.x; i < q.num_new; i += gridDim.x * kStepThreads) {
+        const int par = st.par[i];
+        const int t = st.ctx[par];
         if (t % bs) {
-            const int o = tab(par * MB + t / bs);
-            atomicAdd(&p.writers[o], 1);
-            atomicMax(&p.last_writer[o], i);
-        }
-    }
-    __syncthreads();
-    // a block is freed only if every old beam holding it has no child; mark
-    // the last such entry (in release order) of each block reaching zero
-    for (int base = 0; base < old_entries; base += kThreads * kItems) {
-        int blk[kItems], r0[kItems];
-        EntryWalk w(base + tid, MB);
-#pragma unroll
-        for (int k = 0; k < kItems; ++k) {
-            const int e = base + k * kThreads + tid;
-            blk[k] = -1;
-            if (e < old_entries && w.pos < s_nb[w.j] && s_nch[w.j] == 0) blk[k] = tab(e);
-            w.step(sdj, sdp, MB);
-        }
-#pragma unroll
-        for (int k = 0; k < kItems; ++k)
-            if (blk[k] >= 0) r0[k] = p.ref[blk[k]] + p.delta[blk[k]];
-#pragma unroll
-        for (int k = 0; k < kItems; ++k) {
-            if (blk[k] >= 0) {
-                if (r0[k] < 0) atomicOr(&s_bad, PA_DEVERR_POOL);  // a table holds a block more often than counted
-                if (r0[k] == 0) atomicMax(&p.last_old[blk[k]], base + k * kThreads + tid);
+            const int o = __ldg(q.old_tables + par * MB + t / bs);
+            if (o >= 0 && o < nb) {
+                atomicAdd(&p.writers[o], 1);
+                atomicMax(&p.last_writer[o], i);
             }
         }
     }
-    __syncthreads();
+}
 
-    // ---- phase 2: freed blocks, pushed to the back of the free list in
-    // order of their last release (written past the list's end: harmless
-    // until the count is updated). Items are contiguous per thread so the
-    // scan runs in entry order.
-    int freed = 0;
-    for (int base = 0; base < old_entries; base += kThreads * kScanItems) {
-        int blk[kScanItems], r0[kScanItems], d0[kScanItems], l0[kScanItems];
-        EntryWalk w(base + tid * kScanItems, MB);
+// Block-wide sum over kStepThreads threads (ends with a barrier).
+__device__ __forceinline__ int cta_sum(int v, int *warp_sums) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-        for (int k = 0; k < kScanItems; ++k) {
-            const int e = base + tid * kScanItems + k;
-            blk[k] = -1;
-            if (e < old_entries && w.pos < s_nb[w.j] && s_nch[w.j] == 0) blk[k] = tab(e);
-            w.step(MB == 1 ? 1 : 0, MB == 1 ? 0 : 1, MB);
-        }
+    for (int d = 16; d >= 1; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+    if (lane == 0) warp_sums[warp] = v;
+    __syncthreads();
+    int t = 0;
 #pragma unroll
-        for (int k = 0; k < kScanItems; ++k) {
-            if (blk[k] >= 0) {
-                r0[k] = p.ref[blk[k]];
-                d0[k] = p.delta[blk[k]];
-                l0[k] = p.last_old[blk[k]];
+    for (int w = 0; w < kStepThreads / 32; ++w) t += warp_sums[w];
+    __syncthreads();
+    return t;
+}
+
+// Exclusive scan over kStepThreads threads; *total receives the sum (ends with a barrier).
+__device__ __forceinline__ int cta_scan(int v, int *warp_sums, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, d);
+        if (lane >= d) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    int before = 0, t = 0;
+#pragma unroll
+    for (int w = 0; w < kStepThreads / 32; ++w) {
+        if (w < warp) before += warp_sums[w];
+        t += warp_sums[w];
+    }
+    __syncthreads();
+    *total = t;
+    return x - v + before;
+}
+
+// Whether new beam i needs a block and whether it copies (counts as the
+// sequential order sees them when the new tokens are written: after every
+// fork and release). `applied`: the net changes are already in ref.
+__device__ __forceinline__ void take_and_copy(const StepParams &q, const Pool &p, const Staged &st, int i,
+                                              bool applied, int *need, int *copy, int *o, int *t) {
+    const int par = st.par[i];
+    *t = st.ctx[par];
+    *need = 0;
+    *copy = 0;
+    *o = -1;
+    if (*t % q.block_size == 0) {
+        *need = 1;
+    } else {
+        *o = __ldg(q.old_tables + par * q.max_blocks + *t / q.block_size);
+        const int r = applied ? p.ref[*o] : p.ref[*o] + p.delta[*o];
+        *copy = (r - p.writers[*o] > 0 || p.last_writer[*o] != i);
+        *need = *copy;
+    }
+}
+
+__global__ void __launch_bounds__(kStepThreads) beam_flags_kernel(const StepParams q) {
+    extern __shared__ int dyn[];
+    __shared__ int s_bad;
+    __shared__ int warp_sums[kStepThreads / 32];
+    const Pool p = views(q.state, q.num_blocks);
+    const Staged st = stage_beams(q, p, dyn, &s_bad);
+    const bool bad = st.bad || *status_word(p) != 0;
+    const int MB = q.max_blocks;
+    int e0, e1;
+    chunk_of(q, &e0, &e1);
+    int cnt = 0;
+    if (!bad) {
+        for (int e = e0 + threadIdx.x; e < e1; e += kStepThreads) {
+            const int j = e / MB, pos = e - j * MB;
+            if (pos >= st.nblk[j] || st.nch[j] != 0) continue;
+            const int b = __ldg(q.old_tables + e);
+            const int r = p.ref[b] + p.delta[b];
+            if (r < 0) {
+                atomicOr(p.tail, PA_DEVERR_POOL);  // a table holds a block more often than counted
+            } else if (r > 0) {
+                p.last_old[b] = -2;  // not freed (every entry of b sees the same r)
+            } else if (p.last_old[b] == e) {
+                ++cnt;
             }
         }
-        int flag = 0, mine = 0;
-#pragma unroll
-        for (int k = 0; k < kScanItems; ++k) {
-            if (blk[k] >= 0) {
-                const int r = r0[k] + d0[k];
-                if (r == 0 && l0[k] == base + tid * kScanItems + k) {
-                    flag |= 1 << k;
-                    ++mine;
-                }
+    }
+    cnt = cta_sum(cnt, warp_sums);
+    if (threadIdx.x == 0) p.tail[4 + blockIdx.x] = cnt;
+    if (blockIdx.x == 0) {
+        int takes = 0, copies = 0;
+        if (!bad) {
+            for (int base = 0; base < q.num_new; base += kStepThreads) {
+                const int i = base + threadIdx.x;
+                int need = 0, copy = 0, o, t;
+                if (i < q.num_new) take_and_copy(q, p, st, i, false, &need, &copy, &o, &t);
+                takes += need;
+                copies += copy;
             }
+        }
+        takes = cta_sum(takes, warp_sums);
+        copies = cta_sum(copies, warp_sums);
+        if (threadIdx.x == 0) {
+            p.tail[1] = takes;
+            p.tail[2] = copies;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kStepThreads) beam_apply_kernel(const StepParams q) {
+    extern __shared__ int dyn[];
+    __shared__ int s_bad;
+    __shared__ int warp_sums[kStepThreads / 32];
+    const Pool p = views(q.state, q.num_blocks);
+    const Staged st = stage_beams(q, p, dyn, &s_bad);
+    const int MB = q.max_blocks, nb = q.num_blocks, bs = q.block_size;
+    const int head = p.hdr[3], count = p.hdr[4];
+    // freed blocks in all chunks and in the chunks before this one
+    int before = 0, freed = 0;
+    for (int c = threadIdx.x; c < (int)gridDim.x; c += kStepThreads) {
+        const int v = p.tail[4 + c];
+        freed += v;
+        if (c < (int)blockIdx.x) before += v;
+    }
+    freed = cta_sum(freed, warp_sums);
+    before = cta_sum(before, warp_sums);
+    const int status = *status_word(p);  // final: launches 1 and 2 are done, this one adds nothing
+    const bool ok = !st.bad && status == 0 && p.tail[1] <= count + freed;
+    int e0, e1;
+    chunk_of(q, &e0, &e1);
+    if (!st.bad && status == 0) {  // every entry in use holds a valid block id
+        // freed blocks, in entry order: each thread takes a contiguous run of the chunk
+        const int per = (q.chunk + kStepThreads - 1) / kStepThreads;
+        const int a0 = min(e1, e0 + threadIdx.x * per), a1 = min(e1, a0 + per);
+        int mine = 0;
+        for (int e = a0; e < a1; ++e) {
+            const int j = e / MB, pos = e - j * MB;
+            if (pos < st.nblk[j] && st.nch[j] == 0 && p.last_old[__ldg(q.old_tables + e)] == e) ++mine;
         }
         int tot;
-        int r = cta_exclusive_scan(mine, warp_sums, &tot);
-#pragma unroll
-        for (int k = 0; k < kScanItems; ++k)
-            if (flag >> k & 1) p.ring[(head + count + freed + r++) % nb] = blk[k];
-        freed += tot;
+        int r = cta_scan(mine, warp_sums, &tot);
+        if (ok && mine) {
+            for (int e = a0; e < a1; ++e) {
+                const int j = e / MB, pos = e - j * MB;
+                if (pos >= st.nblk[j] || st.nch[j] != 0) continue;
+                const int b = __ldg(q.old_tables + e);
+                if (p.last_old[b] == e) p.ring[(head + count + before + r++) % nb] = b;
+            }
+        }
     }
+    if (!st.bad) {  // (with st.bad set, launch 1 changed nothing)
+        // net count changes (each block once: whoever swaps its delta out);
+        // every delta goes back to 0 whatever the outcome
+        for (int e = e0 + threadIdx.x; e < e1; e += kStepThreads) {
+            const int j = e / MB, pos = e - j * MB;
+            if (pos >= st.nblk[j] || st.nch[j] == 1) continue;
+            const int b = __ldg(q.old_tables + e);
+            if (b < 0 || b >= nb) continue;
+            const int d = atomicExch(&p.delta[b], 0);
+            if (ok && d) p.ref[b] += d;
+        }
+    }
+    if (ok) {  // the new tables: parents' rows, -1 past them; each beam's write entry is left to launch 4
+        const long long new_entries = (long long)q.num_new * MB;
+        for (long long e = (long long)blockIdx.x * kStepThreads + threadIdx.x; e < new_entries;
+             e += (long long)gridDim.x * kStepThreads) {
+            const int i = (int)(e / MB), pos = (int)(e - (long long)i * MB);
+            const int par = st.par[i];
+            if (pos == st.ctx[par] / bs) continue;
+            q.new_tables[e] = pos < st.nblk[par] ? __ldg(q.old_tables + par * MB + pos) : -1;
+        }
+    }
+}
 
-    // ---- phase 3: blocks the new tokens take, and the copies
-    int takes = 0, copies = 0;
-    for (int base = 0; base < n_new; base += kThreads) {
-        const int i = base + tid;
-        int need = 0, copy = 0;
-        if (i < n_new) {
-            const int par = s_par[i];
-            const int t = s_ctx[par];
-            if (t % bs == 0) {
-                need = 1;
-            } else {
-                const int o = tab(par * MB + t / bs);
-                const int others = p.ref[o] + p.delta[o] - p.writers[o];
-                copy = (others > 0 || p.last_writer[o] != i);
-                need = copy;
-            }
-        }
-        int tt, tc;
-        cta_exclusive_scan(need, warp_sums, &tt);
-        cta_exclusive_scan(copy, warp_sums, &tc);
-        takes += tt;
-        copies += tc;
-    }
-    __syncthreads();
-    const bool ok = !s_bad && takes <= count + freed;
-
-    // ---- phase 4: apply the net counts (each block once: whoever swaps its
-    // delta out), reset the release marks
-    for (int base = 0; base < old_entries; base += kThreads * kItems) {
-        int blk[kItems];
-        EntryWalk w(base + tid, MB);
-#pragma unroll
-        for (int k = 0; k < kItems; ++k) {
-            const int e = base + k * kThreads + tid;
-            blk[k] = -1;
-            if (e < old_entries && w.pos < s_nb[w.j] && s_nch[w.j] != 1) blk[k] = tab(e);
-            w.step(sdj, sdp, MB);
-        }
-        EntryWalk w2(base + tid, MB);
-#pragma unroll
-        for (int k = 0; k < kItems; ++k) {
-            const int jk = w2.j;
-            w2.step(sdj, sdp, MB);
-            if (blk[k] >= 0) {
-                const int b = blk[k];
-                if (s_nch[jk] == 0) p.last_old[b] = -1;
-                const int d = atomicExch(&p.delta[b], 0);
-                if (ok && d) p.ref[b] += d;
-            }
-        }
-    }
-    __syncthreads();
-
-    if (ok) {
-        // ---- phase 5: the new tables (parent rows, -1 past the blocks in use)
-        for (int base = 0; base < new_entries; base += kThreads * kItems) {
-            int v[kItems];
-            EntryWalk w(base + tid, MB);
-#pragma unroll
-            for (int k = 0; k < kItems; ++k) {
-                const int e = base + k * kThreads + tid;
-                v[k] = -1;
-                if (e < new_entries) {
-                    const int par = s_par[w.j];
-                    if (w.pos < s_nb[par]) v[k] = tab(par * MB + w.pos);
-                }
-                w.step(sdj, sdp, MB);
-            }
-#pragma unroll
-            for (int k = 0; k < kItems; ++k) {
-                const int e = base + k * kThreads + tid;
-                if (e < new_entries) q.new_tables[e] = v[k];
-            }
-        }
-        __syncthreads();
-        // ---- phase 6: takes, copies, slots
-        int tk = 0, cp = 0;
-        for (int base = 0; base < n_new; base += kThreads) {
-            const int i = base + tid;
-            int need = 0, copy = 0, o = -1, t = 0;
-            if (i < n_new) {
-                const int par = s_par[i];
-                t = s_ctx[par];
-                if (t % bs == 0) {
-                    need = 1;
-                } else {
-                    o = tab(par * MB + t / bs);
-                    copy = (p.ref[o] - p.writers[o] > 0 || p.last_writer[o] != i);
-                    need = copy;
-                }
-            }
-            int tt, tc;
-            const int k = tk + cta_exclusive_scan(need, warp_sums, &tt);
-            const int c = cp + cta_exclusive_scan(copy, warp_sums, &tc);
-            tk += tt;
-            cp += tc;
-            if (i < n_new) {
-                int b = o;
-                if (need) {
-                    b = policy == PA_POOL_FIFO ? p.ring[(head + k) % nb] : p.ring[(head + count + freed - 1 - k) % nb];
-                    p.ref[b] = 1;
-                    q.new_tables[i * MB + t / bs] = b;
-                }
-                if (copy) {
-                    q.cow_pairs[2 * c] = o;
-                    q.cow_pairs[2 * c + 1] = b;
-                }
-                q.slots[i] = b * bs + t % bs;
-                q.new_ctx[i] = t + 1;
-            }
-        }
-        __syncthreads();
-        // a copying writer gives up its reference to the old block
-        for (int i = tid; i < n_new; i += kThreads) {
-            const int par = s_par[i];
-            const int t = s_ctx[par];
-            if (t % bs) {
-                const int o = tab(par * MB + t / bs);
-                if (q.new_tables[i * MB + t / bs] != o) atomicSub(&p.ref[o], 1);
-            }
-        }
-    }
-    __syncthreads();
-    // ---- reset the writer marks; header and outputs
-    for (int i = tid; i < n_new; i += kThreads) {
-        const int par = s_par[i];
-        const int t = s_ctx[par];
-        if (t % bs) {
-            const int o = tab(par * MB + t / bs);
-            p.writers[o] = 0;
-            p.last_writer[o] = -1;
-        }
-        if (!ok) q.slots[i] = -1;
-    }
-    if (tid == 0) {
+__global__ void __launch_bounds__(kStepThreads) beam_finish_kernel(const StepParams q) {
+    extern __shared__ int dyn[];
+    __shared__ int s_bad;
+    __shared__ int warp_sums[kStepThreads / 32];
+    const Pool p = views(q.state, q.num_blocks);
+    const Staged st = stage_beams(q, p, dyn, &s_bad);
+    const int MB = q.max_blocks, nb = q.num_blocks, bs = q.block_size;
+    if (blockIdx.x == 0) {
+        const int policy = p.hdr[2], head = p.hdr[3], count = p.hdr[4];
+        int freed = 0;
+        for (int c = threadIdx.x; c < q.num_chunks; c += kStepThreads) freed += p.tail[4 + c];
+        freed = cta_sum(freed, warp_sums);
+        const int status = *status_word(p);
+        const int takes = p.tail[1];
+        const bool ok = !st.bad && status == 0 && takes <= count + freed;
         if (ok) {
-            p.hdr[3] = policy == PA_POOL_FIFO ? (head + takes) % nb : head;
-            p.hdr[4] = count + freed - takes;
-            *q.num_cow = copies;
-        } else {
-            *q.num_cow = 0;
-            record_error(q.err, s_bad ? (unsigned)s_bad : PA_DEVERR_POOL);
+            int tk = 0, cp = 0;
+            for (int base = 0; base < q.num_new; base += kStepThreads) {
+                const int i = base + threadIdx.x;
+                int need = 0, copy = 0, o = -1, t = 0;
+                if (i < q.num_new) take_and_copy(q, p, st, i, true, &need, &copy, &o, &t);
+                int tt, tc;
+                const int k = tk + cta_scan(need, warp_sums, &tt);
+                const int c = cp + cta_scan(copy, warp_sums, &tc);
+                tk += tt;
+                cp += tc;
+                if (i < q.num_new) {
+                    int b = o;
+                    if (need) {
+                        b = policy == PA_POOL_FIFO ? p.ring[(head + k) % nb] : p.ring[(head + count + freed - 1 - k) % nb];
+                        p.ref[b] = 1;
+                    }
+                    q.new_tables[(long long)i * MB + t / bs] = b;
+                    if (copy) {
+                        q.cow_pairs[2 * c] = o;
+                        q.cow_pairs[2 * c + 1] = b;
+                    }
+                    q.slots[i] = b * bs + t % bs;
+                    q.new_ctx[i] = t + 1;
+                }
+            }
+            __syncthreads();
+            // a copying writer gives up its reference to the old block
+            for (int i = threadIdx.x; i < q.num_new; i += kStepThreads) {
+                const int par = st.par[i];
+                const int t = st.ctx[par];
+                if (t % bs) {
+                    const int o = __ldg(q.old_tables + par * MB + t / bs);
+                    if (q.new_tables[(long long)i * MB + t / bs] != o) atomicSub(&p.ref[o], 1);
+                }
+            }
+        }
+        __syncthreads();
+        // reset the writer marks; outputs of a failed step
+        if (!st.bad) {
+            for (int i = threadIdx.x; i < q.num_new; i += kStepThreads) {
+                const int par = st.par[i];
+                const int t = st.ctx[par];
+                if (t % bs) {
+                    const int o = __ldg(q.old_tables + par * MB + t / bs);
+                    if (o >= 0 && o < nb) {
+                        p.writers[o] = 0;
+                        p.last_writer[o] = -1;
+                    }
+                }
+            }
+        }
+        if (!ok)
+            for (int i = threadIdx.x; i < q.num_new; i += kStepThreads) q.slots[i] = -1;
+        if (threadIdx.x == 0) {
+            if (ok) {
+                p.hdr[3] = policy == PA_POOL_FIFO ? (head + takes) % nb : head;
+                p.hdr[4] = count + freed - takes;
+                *q.num_cow = p.tail[2];
+            } else {
+                *q.num_cow = 0;
+                const int bits = st.bad | status;
+                record_error(q.err, bits ? (unsigned)bits : PA_DEVERR_POOL);
+            }
+        }
+        __syncthreads();  // every thread has read the totals: the step scratch goes back to zero
+        for (int i = threadIdx.x; i < 4 + q.num_chunks; i += kStepThreads) p.tail[i] = 0;
+    }
+    // every CTA: clear the release marks of its chunk
+    if (!st.bad) {
+        int e0, e1;
+        chunk_of(q, &e0, &e1);
+        for (int e = e0 + threadIdx.x; e < e1; e += kStepThreads) {
+            const int j = e / MB, pos = e - j * MB;
+            if (pos >= st.nblk[j] || st.nch[j] != 0) continue;
+            const int b = __ldg(q.old_tables + e);
+            if (b >= 0 && b < nb) p.last_old[b] = -1;
         }
     }
 }
@@ -615,21 +622,27 @@ cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const in
     q.num_blocks = num_blocks;
     q.block_size = block_size;
     q.err = err;
-    const long long base = (3LL * num_old + num_new) * (long long)sizeof(int);
-    const long long with_tables = base + (long long)num_old * max_blocks * (long long)sizeof(int);
-    static AttrCache attr_done[2];
-    cudaError_t e;
-    if (with_tables <= beam::kMaxDynBytes) {
-        e = ensure_smem_attr(reinterpret_cast<const void *>(beam::beam_step_kernel<true>), beam::kMaxDynBytes,
-                             &attr_done[1]);
+    // chunks of at least one entry per thread, at most kMaxChunks of them
+    const long long entries = (long long)num_old * max_blocks;
+    long long chunk = beam::kStepThreads;
+    while ((entries + chunk - 1) / chunk > beam::kMaxChunks) chunk += beam::kStepThreads;
+    q.chunk = (int)chunk;
+    q.num_chunks = (int)std::max(1LL, (entries + chunk - 1) / chunk);
+    const int smem = (3 * num_old + num_new) * (int)sizeof(int);
+    static AttrCache attr_done[4];
+    const void *kernels[4] = {reinterpret_cast<const void *>(beam::beam_count_kernel),
+                              reinterpret_cast<const void *>(beam::beam_flags_kernel),
+                              reinterpret_cast<const void *>(beam::beam_apply_kernel),
+                              reinterpret_cast<const void *>(beam::beam_finish_kernel)};
+    for (int k = 0; k < 4; ++k) {
+        cudaError_t e = ensure_smem_attr(kernels[k], beam::kMaxStageBytes, &attr_done[k]);
         if (e != cudaSuccess) return e;
-        beam::beam_step_kernel<true><<<1, beam::kThreads, (int)with_tables, stream>>>(q);
-    } else {
-        e = ensure_smem_attr(reinterpret_cast<const void *>(beam::beam_step_kernel<false>), beam::kMaxStageBytes,
-                             &attr_done[0]);
-        if (e != cudaSuccess) return e;
-        beam::beam_step_kernel<false><<<1, beam::kThreads, (int)base, stream>>>(q);
     }
+    const dim3 grid(q.num_chunks), block(beam::kStepThreads);
+    beam::beam_count_kernel<<<grid, block, smem, stream>>>(q);
+    beam::beam_flags_kernel<<<grid, block, smem, stream>>>(q);
+    beam::beam_apply_kernel<<<grid, block, smem, stream>>>(q);
+    beam::beam_finish_kernel<<<grid, block, smem, stream>>>(q);
     return cudaGetLastError();
 }
 

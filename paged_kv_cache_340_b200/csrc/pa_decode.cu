@@ -139,7 +139,7 @@ struct FmaConsumer {
     float acc[G][S::kVec];
     float l_lane;
 
-    __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int warp, int lane) {
+    __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int g_valid, int warp, int lane) {
         r = lane / S::kLpt;
         c = lane % S::kLpt;
         rg = warp * S::kRows + r;
@@ -148,8 +148,9 @@ struct FmaConsumer {
         counts_l = (c % S::kDup) == 0;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const T *>(p.query) +
-                                                             (head0 + g) * D + c * S::kVec);
+            uint4 u = make_uint4(0u, 0u, 0u, 0u);  // padding heads: zero queries
+            if (g < g_valid)
+                u = *reinterpret_cast<const uint4 *>(static_cast<const T *>(p.query) + (head0 + g) * D + c * S::kVec);
             Elt<T>::unpack(u, q[g]);
 #pragma unroll
             for (int e = 0; e < S::kVec; ++e) q[g][e] *= p.scale_log2;
@@ -354,13 +355,13 @@ struct MmaConsumer {
         return 8 * (m & 7) + (E & 7) + 64 * (E >> 3);
     }
 
-    __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int, int lane) {
+    __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int g_valid, int, int lane) {
         q4 = lane & 3;
         r = lane >> 2;
 #pragma unroll
         for (int i = 0; i < kI; ++i) {
             uint4 u = make_uint4(0u, 0u, 0u, 0u);
-            if (r < G)
+            if (r < g_valid)
                 u = *reinterpret_cast<const uint4 *>(static_cast<const T *>(p.query) + (head0 + r) * D +
                                                      8 * q4 + 32 * i);
             qb[i][0] = u.x;
@@ -566,7 +567,7 @@ struct MmaConsumerQ8 {
     // signed, lo in [0, 255]): q . k = step (256 hi.k + lo.k), both products
     // exact in int32 on the int8 tensor cores. |q - step Q| <= step / 2, i.e.
     // 2^-16 of the head's largest component.
-    __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int, int lane) {
+    __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int g_valid, int, int lane) {
         q4 = lane & 3;
         r = lane >> 2;
         float f[kJ][16];
@@ -576,7 +577,7 @@ struct MmaConsumerQ8 {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint4 u = make_uint4(0u, 0u, 0u, 0u);
-                if (r < G)
+                if (r < g_valid)
                     u = *reinterpret_cast<const uint4 *>(static_cast<const TQ *>(p.query) + (head0 + r) * D +
                                                          16 * (q4 + 4 * j) + 8 * h);
                 Elt<TQ>::unpack(u, f[j] + 8 * h);
@@ -786,20 +787,48 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     uint64_t *full = reinterpret_cast<uint64_t *>(ring + S::kDataBytes);
     int *bad = reinterpret_cast<int *>(full + S::kStages);
 
-    const int part = blockIdx.x;
-    const int kvh = blockIdx.y;
-    const int s = p.seq_order ? p.seq_order[blockIdx.z] : (int)blockIdx.z;
+    // prefill through this kernel is for fp32 caches only (the other types
+    // prefill on the tensor cores); one CTA column per query token
+    constexpr bool kPrefillMode = std::is_same_v<T, float>;
+    const bool prefill = kPrefillMode && p.q_start != nullptr;
+    const int part = prefill ? 0 : (int)blockIdx.x;
+    // groups of 1 and 2 run unpadded; only the compiled size 8 has sub-groups
+    const int kvh = (G == 8 && p.sub_groups > 1) ? (int)blockIdx.y / p.sub_groups : (int)blockIdx.y;
+    const int sub = (G == 8 && p.sub_groups > 1) ? (int)blockIdx.y % p.sub_groups : 0;
+    const int g_valid = G <= 2 ? G : min(G, p.group - sub * G);  // real query heads of this CTA
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const bool split = p.partition_size > 0;
-    if (s < 0 || s >= (int)gridDim.z) {  // a bad schedule entry: nothing to do for it
-        if (threadIdx.x == 0 && part == 0 && kvh == 0) record_error(p.err, PA_DEVERR_CONTEXT);
-        return;
+    int s, qrow;  // sequence (table row, context) and query / output row
+    int ctx;
+    bool ctx_bad = false;
+    if (kPrefillMode && prefill) {
+        qrow = blockIdx.x;
+        if (qrow < p.q_start[0] || qrow >= p.q_start[p.num_seqs]) return;  // a token of no sequence
+        int lo = 0, hi = p.num_seqs;  // q_start[lo] <= qrow < q_start[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (p.q_start[mid] <= qrow) lo = mid; else hi = mid;
+        }
+        s = lo;
+        const int q_len = p.q_start[s + 1] - p.q_start[s];
+        const int ctx_s = p.context_lens[s];
+        if (q_len > ctx_s) {  // more new tokens than cached ones: the sequence is skipped
+            if (threadIdx.x == 0 && kvh == 0) record_error(p.err, PA_DEVERR_CONTEXT);
+            return;
+        }
+        ctx = ctx_s - q_len + (qrow - p.q_start[s]) + 1;  // causal: up to this token's own position
+    } else {
+        s = p.seq_order ? p.seq_order[blockIdx.z] : (int)blockIdx.z;
+        if (s < 0 || s >= (int)gridDim.z) {  // a bad schedule entry: nothing to do for it
+            if (threadIdx.x == 0 && part == 0 && kvh == 0) record_error(p.err, PA_DEVERR_CONTEXT);
+            return;
+        }
+        qrow = s;
+        ctx = p.context_lens[s];
     }
 
     // ---- token range of this CTA
-    int ctx = p.context_lens[s];
-    bool ctx_bad = false;
     if (ctx < 0) { ctx = 0; ctx_bad = true; }
     if (ctx > p.max_blocks_per_seq * BS) { ctx = p.max_blocks_per_seq * BS; ctx_bad = true; }
     if (split && ctx > p.max_context_len) { ctx = p.max_context_len; ctx_bad = true; }
@@ -811,11 +840,10 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
         t_end = min(t_begin + p.partition_size, ctx);
     }
     const int nstage = (t_end - t_begin + S::kTS - 1) / S::kTS;  // 16-token stages
-    const uint64_t wait_limit = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
-    const int withheld = (p.withhold_seq == s && p.withhold_kvh == kvh && part == 0) ? p.withhold_stage : -1;
-    const size_t head0 = (size_t)s * p.num_heads + (size_t)kvh * G;  // first query head row
+
+    const size_t head0 = (size_t)qrow * p.num_heads + (size_t)kvh * (G <= 2 ? G : p.group) + (size_t)sub * G;
     if (nstage == 0) {  // unsplit, empty context: zeros
-        for (int i = threadIdx.x; i < G * D; i += blockDim.x) store_out(p.out, head0 * D + i, 0.f, p.out_dtype);
+        for (int i = threadIdx.x; i < g_valid * D; i += blockDim.x) store_out(p.out, head0 * D + i, 0.f, p.out_dtype);
         return;
     }
     if (threadIdx.x == 0) {
@@ -858,7 +886,8 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     auto issue = [&](int m, int id) {  // lane 0
         const int k = warp + S::kWarps * m;
         const int buf = k % S::kStages;
-        if (k == withheld) {  // test hook: no copy and no arrival, so this stage's wait runs out
+        if (k == p.withhold_stage && s == p.withhold_seq && kvh == p.withhold_kvh && part == 0) {
+            // test hook: no copy and no arrival, so this stage's wait runs out
             bad[buf] = 1;
         } else if (id >= 0) {
             bad[buf] = 0;
@@ -915,7 +944,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     }
 
     Consumer cons;
-    cons.init(p, head0, warp, lane);
+    cons.init(p, head0, g_valid, warp, lane);
     int waited = 0;
     bool ok = true;
     for (int m = 0; m < nmine; ++m) {
@@ -928,7 +957,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
         const int buf = k % S::kStages;
         // Lane 0 polls the barrier (32 lanes polling would serialise on it);
         // __syncwarp then orders the other lanes' reads after its acquire.
-        const bool got = mbar_wait(full + buf, (k / S::kStages) & 1, wait_limit);
+        const bool got = mbar_wait(full + buf, (k / S::kStages) & 1, p.wait_limit_ns);
         if (!__all_sync(0xffffffffu, got)) {
             if (lane == 0) record_error(p.err, PA_DEVERR_TIMEOUT);
             ok = false;
@@ -949,8 +978,10 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
                             const bool isv = c >= kRowChunks;
                             const int cc = c % kRowChunks;
                             reinterpret_cast<uint4 *>(Kw + (isv ? S::kTileBytes : 0) + (size_t)r * D * S::kElt)[cc] = nrow[i];
-                            const unsigned char *pool = reinterpret_cast<const unsigned char *>(isv ? vc : kc);
-                            reinterpret_cast<uint4 *>(const_cast<unsigned char *>(pool) + prow)[cc] = nrow[i];
+                            if (sub == 0) {  // one CTA of the kv head writes the pool
+                                const unsigned char *pool = reinterpret_cast<const unsigned char *>(isv ? vc : kc);
+                                reinterpret_cast<uint4 *>(const_cast<unsigned char *>(pool) + prow)[cc] = nrow[i];
+                            }
                         }
                     }
                 }
@@ -974,7 +1005,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     if (!ok && lane == 0) {  // after a timeout: let every copy this warp started land
         for (int m = waited; m < min(nmine, waited + S::kBufPerWarp); ++m) {
             const int k = warp + S::kWarps * m;
-            if (!mbar_wait(full + (k % S::kStages), (k / S::kStages) & 1, wait_limit))
+            if (!mbar_wait(full + (k % S::kStages), (k / S::kStages) & 1, p.wait_limit_ns))
                 record_error(p.err, PA_DEVERR_TIMEOUT);
         }
     }
@@ -986,7 +1017,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     __syncthreads();
     cons.store(mg, lg, ag, warp, lane);
     __syncthreads();
-    for (int idx = threadIdx.x; idx < G * D; idx += S::kThreads) {
+    for (int idx = threadIdx.x; idx < g_valid * D; idx += S::kThreads) {
         const int g = idx / D;
         const int d = idx % D;
         float Mx = -INFINITY;
@@ -1100,20 +1131,28 @@ static cudaError_t launch_decode_t(const DecodeParams &p, int grid_x, int num_kv
     static AttrCache attr_done;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), S::kSmemBytes, &attr_done);
     if (e != cudaSuccess) return e;
-    dim3 grid(grid_x, num_kv_heads, num_seqs);
+    dim3 grid(grid_x, num_kv_heads * p.sub_groups, num_seqs);
     kern<<<grid, S::kThreads, S::kSmemBytes, stream>>>(p);
     return cudaGetLastError();
 }
 
+// The compiled group size serving a head group of `group` query heads: the
+// next power of two up to 8 (larger groups run as sub-groups of 8).
+static int padded_group(int group) { return group <= 1 ? 1 : group <= 2 ? 2 : group <= 4 ? 4 : 8; }
+
 template <typename T, int D, int BS, typename TQ = T, bool kAppend = false>
-static cudaError_t dispatch_group(const DecodeParams &p, int group, int grid_x, int num_kv_heads,
+static cudaError_t dispatch_group(const DecodeParams &p0, int group, int grid_x, int num_kv_heads,
                                   int num_seqs, cudaStream_t stream) {
-    switch (group) {
+    if (group < 1) return cudaErrorInvalidValue;
+    DecodeParams p = p0;
+    const int gt = padded_group(group);
+    p.group = group;
+    p.sub_groups = (group + gt - 1) / gt;
+    switch (gt) {
         case 1: return launch_decode_t<T, D, BS, 1, TQ, kAppend>(p, grid_x, num_kv_heads, num_seqs, stream);
         case 2: return launch_decode_t<T, D, BS, 2, TQ, kAppend>(p, grid_x, num_kv_heads, num_seqs, stream);
         case 4: return launch_decode_t<T, D, BS, 4, TQ, kAppend>(p, grid_x, num_kv_heads, num_seqs, stream);
-        case 8: return launch_decode_t<T, D, BS, 8, TQ, kAppend>(p, grid_x, num_kv_heads, num_seqs, stream);
-        default: return cudaErrorInvalidValue;
+        default: return launch_decode_t<T, D, BS, 8, TQ, kAppend>(p, grid_x, num_kv_heads, num_seqs, stream);
     }
 }
 

@@ -28,6 +28,13 @@ struct DecodeParams {
     int num_heads;
     int num_kv_heads;
     int num_blocks;
+    // head group: query heads per kv head (num_heads / num_kv_heads). A CTA
+    // serves up to the kernel's compiled group size G of them (a power of two
+    // >= the group, padded with zero queries whose outputs are not written);
+    // a group larger than G is served by sub_groups CTAs of G heads each,
+    // adjacent along gridDim.y (kv head = blockIdx.y / sub_groups).
+    int group = 1;
+    int sub_groups = 1;
     float scale_log2;    // scale * log2(e)
     int partition_size;  // 0: one CTA covers the whole sequence
     int max_parts;
@@ -40,6 +47,14 @@ struct DecodeParams {
     // copy (pa_decode_append)
     const void *new_key;
     const void *new_value;
+    // Prefill on the CUDA cores (pa_prefill over an fp32 cache): when q_start
+    // (device int32 [num_seqs + 1]) is set, blockIdx.x is a query token t
+    // (the grid has one CTA column per token and no partitions); its sequence
+    // s has q_start[s] <= t < q_start[s + 1], and it attends to cache tokens
+    // 0 .. context_lens[s] - q_len_s + (t - q_start[s]). query and out rows
+    // are tokens; the table row and context are the sequence's.
+    const int32_t *q_start = nullptr;
+    int num_seqs = 0;
     // Test hook of the bounded waits (pa_decode_withhold_stage): the CTA of
     // sequence withhold_seq, kv head withhold_kvh (partition 0) never issues
     // the copy of its 16-token stage withhold_stage, so that stage's wait runs
@@ -126,6 +141,13 @@ cudaError_t symbol_address(const void *symbol, SymbolCache *cache, void **addr);
 
 // Device address of the current device's error word.
 cudaError_t device_error_word(unsigned int **word);
+
+// pa_prefill over an fp32 cache: the decode kernel with one CTA column per
+// query token (see DecodeParams::q_start). Arguments as pa_prefill.
+int prefill_cuda_cores(void *out, const void *query, const int32_t *q_start, int num_tokens, const void *k_cache,
+                       const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                       const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                       float scale, int block_size, int num_blocks, cudaStream_t stream);
 
 // Number of SMs of the current device.
 int sm_count();

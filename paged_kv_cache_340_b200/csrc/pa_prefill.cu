@@ -43,12 +43,9 @@ namespace prefill {
 
 constexpr int kM = 128;                 // query rows per CTA
 constexpr int kN = 64;                  // kv tokens per tile
-constexpr int kD = 128;                 // head dim
 constexpr int kHalfBytes = 128;         // one swizzled row: 64 16-bit elements
 constexpr int kQHalf = kM * kHalfBytes; // 16 KB: rows x d 0-63 (or 64-127)
 constexpr int kKVHalf = kN * kHalfBytes;  // 8 KB
-constexpr int kQBytes = 2 * kQHalf;
-constexpr int kKVBytes = 2 * kKVHalf;   // one K or V tile
 constexpr int kSoftmaxWarps = 4;
 constexpr int kMmaWarp = kSoftmaxWarps;       // warp 4: issues the tensor-core MMAs
 constexpr int kLoadWarp = kSoftmaxWarps + 1;  // warp 5: table lookups and TMA copies
@@ -58,16 +55,25 @@ constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 // part P - bf16(P)) over its own S_j, and O += P_j V_j reads it from there:
 // S_{j+1} is computed while the softmax of tile j runs.
 constexpr int kTmemCols = 256;
-constexpr int kOCol = 0;      // O: 128 fp32 columns
+constexpr int kOCol = 0;      // O: head_dim (64 or 128) fp32 columns
 constexpr int kSCol = 128;    // S buffers 0, 1: 64 fp32 columns each
 constexpr int kPlOff = 32;    // within an S buffer: P at +0, P's low part at +32
-// shared memory (every operand region 1024-byte aligned for the swizzle):
-// Q, and two stages each of K and V
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;         // K stages 0, 1
-constexpr int kOffV = kOffK + 2 * kKVBytes;    // V stages 0, 1
-constexpr int kOffBar = kOffV + 2 * kKVBytes;
-constexpr int kSmemBytes = 1024 + kOffBar + 24 * 8;  // ~97 KB: two CTAs per SM
+
+// Shared-memory layout for head_dim D (64 or 128; every operand region
+// 1024-byte aligned for the swizzle): Q, and two stages each of K and V, each
+// stored as D / 64 swizzled halves of 64 columns.
+template <int D>
+struct Layout {
+    static_assert(D == 64 || D == 128, "head_dim");
+    static constexpr int kHalves = D / 64;
+    static constexpr int kQBytes = kHalves * kQHalf;
+    static constexpr int kKVBytes = kHalves * kKVHalf;  // one K or V tile
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQBytes;       // K stages 0, 1
+    static constexpr int kOffV = kOffK + 2 * kKVBytes;  // V stages 0, 1
+    static constexpr int kOffBar = kOffV + 2 * kKVBytes;
+    static constexpr int kSmemBytes = 1024 + kOffBar + 24 * 8;  // ~97 KB at D 128: two CTAs per SM
+};
 // The running max is raised only when it grows by more than this (log2
 // units): probabilities then stay below 2^8 and O is rarely rescaled.
 constexpr float kRescaleThreshold = 8.f;
@@ -75,6 +81,14 @@ constexpr float kRescaleThreshold = 8.f;
 struct Params {
     void *out;
     const int32_t *q_start;
+    // rows of a CTA are (token, head slot) pairs: 2^gshift head slots per
+    // token (the head group rounded up to a power of two, at most 128); slots
+    // past the group are padding, computed but never written. A group above
+    // 128 runs as sub_groups CTAs along gridDim.y (kv head = blockIdx.y /
+    // sub_groups), each over 128 of its query heads.
+    int group;
+    int gshift;
+    int sub_groups;
     const int32_t *block_tables;
     const int32_t *context_lens;
     int max_blocks_per_seq;
@@ -219,14 +233,20 @@ __device__ __forceinline__ bool softmax_sync_and(bool v) {
     return all != 0;
 }
 
-template <typename T, int G>
+// kStagedOut: the output rows go through shared memory (head groups of 1-2
+// slots per token); otherwise each softmax thread stores its own row.
+template <typename T, int kD, bool kStagedOut>
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const Params p) {
+    using L = Layout<kD>;
+    constexpr int kQBytes = L::kQBytes, kKVBytes = L::kKVBytes, kOffQ = L::kOffQ, kOffK = L::kOffK,
+                  kOffV = L::kOffV, kOffBar = L::kOffBar, kHalves = L::kHalves;
     constexpr bool kBf16 = std::is_same_v<T, __nv_bfloat16>;
-    constexpr int kTokPerTile = kM / G;
     constexpr uint32_t kIdescQK = mma_idesc(kBf16, kM, kN, false);
     constexpr uint32_t kIdescPV = mma_idesc(kBf16, kM, kD, true);
+    const int G = 1 << p.gshift;                       // head slots per token
+    const int kTokPerTile = kM >> p.gshift;
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -252,7 +272,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     int *abort_flag = reinterpret_cast<int *>(bars + 16);
 
     const int qt = gridDim.x - 1 - blockIdx.x;  // longest query tile of each (head, sequence) first
-    const int kvh = blockIdx.y;
+    const int kvh = p.sub_groups > 1 ? (int)blockIdx.y / p.sub_groups : (int)blockIdx.y;
+    const int sub = p.sub_groups > 1 ? (int)blockIdx.y % p.sub_groups : 0;
+    const int head_base = kvh * p.group + sub * G;     // query head of slot 0
+    const int g_valid = min(G, p.group - sub * G);     // slots holding a real query head
     const int s = blockIdx.z;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -268,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     const int rows_valid = min(kM, (q_len - tok0) * G);
     const int pos0 = ctx - q_len + tok0;                      // position of the tile's first token
-    const int pos_max = pos0 + rows_valid / G - 1;
+    const int pos_max = pos0 + (rows_valid >> p.gshift) - 1;
     const int ntiles = pos_max / kN + 1;
 
     // Pool row of the load warp's 16-token group g0 + lane (16 tokens from
@@ -313,8 +336,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             fence_mbar_init();
             fence_proxy_async_smem();  // the initialised barriers, before the copy that signals one
             mbar_arrive_expect_tx(q_full, kQBytes);
-            tma_load_3d(Qs, &tmap_q, 0, kvh * G, q0 + tok0, q_full);
-            tma_load_3d(Qs + kQHalf, &tmap_q, 64, kvh * G, q0 + tok0, q_full);
+#pragma unroll
+            for (int h = 0; h < kHalves; ++h) tma_load_3d(Qs + h * kQHalf, &tmap_q, 64 * h, head_base, q0 + tok0, q_full);
         }
     }
     if (warp == 0) {
@@ -365,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                     for (int g = 0; g < kGroups; ++g)
 #pragma unroll
-                        for (int h = 0; h < 2; ++h)
+                        for (int h = 0; h < kHalves; ++h)
                             tma_load_2d(dst + h * kKVHalf + g * 16 * kHalfBytes, map, h * 64, r4[g], full);
                 }
                 if (kv == 0) ++k_issued; else ++v_issued;
@@ -453,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     } else {
         // ======================================================= softmax warps
         const int r = threadIdx.x;  // row = tensor-memory lane
-        const int tok = r / G;
+        const int tok = r >> p.gshift;
         const bool valid = r < rows_valid;
         const int pos = valid ? pos0 + tok : -1;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -544,10 +567,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (!__all_sync(0xffffffffu, mbar_wait(v_full + b, (j >> 1) & 1) && !*(volatile int *)abort_flag))
                     break;
                 unsigned char *vt = Vs + b * kKVBytes;
-                const int nvec = (kN - zrow) * 2 * (kHalfBytes / 16);
+                const int nvec = (kN - zrow) * kHalves * (kHalfBytes / 16);
                 for (int i = r; i < nvec; i += kSoftmaxWarps * 32) {
-                    const int row = zrow + i / 16;
-                    const int h = (i / 8) & 1;
+                    const int row = zrow + i / (8 * kHalves);
+                    const int h = (i / 8) % kHalves;
                     const int c = i & 7;
                     *reinterpret_cast<uint4 *>(vt + h * kKVHalf + row * kHalfBytes + c * 16) =
                         make_uint4(0u, 0u, 0u, 0u);
@@ -574,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int ebytes = p.out_dtype == PA_F32 ? 4 : 2;
         const int row_bytes = kD * ebytes;
         const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-        if constexpr (G <= 2) {
+        if constexpr (kStagedOut) {
             if (done) {
                 unsigned char *srow = Qs + r * (row_bytes + 16);
 #pragma unroll
@@ -596,7 +619,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                 unsigned char *out = static_cast<unsigned char *>(p.out);
                 for (int i = r; i < rows_valid * cpr; i += kSoftmaxWarps * 32) {
                     const int row = i / cpr, c = i % cpr;
-                    const size_t orow = (size_t)(q0 + tok0 + row / G) * p.num_heads + (size_t)kvh * G + (row % G);
+                    if ((row & (G - 1)) >= g_valid) continue;  // a padding slot
+                    const size_t orow =
+                        (size_t)(q0 + tok0 + (row >> p.gshift)) * p.num_heads + (size_t)head_base + (row & (G - 1));
                     *reinterpret_cast<uint4 *>(out + orow * row_bytes + c * 16) =
                         *reinterpret_cast<const uint4 *>(Qs + row * (row_bytes + 16) + c * 16);
                 }
@@ -605,14 +630,15 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (!done) {
                 if (r == 0) record_error(p.err, PA_DEVERR_TIMEOUT);
             } else {
-                const size_t orow = (size_t)(q0 + tok0 + tok) * p.num_heads + (size_t)kvh * G + (r % G);
+                const size_t orow = (size_t)(q0 + tok0 + tok) * p.num_heads + (size_t)head_base + (r & (G - 1));
                 unsigned char *dst = static_cast<unsigned char *>(p.out) + orow * row_bytes;
+                const bool write = valid && (r & (G - 1)) < g_valid;
 #pragma unroll
                 for (int ch = 0; ch < kD / 32; ++ch) {
                     uint32_t o[32];
                     tmem_ld32(tmem + lane_base + kOCol + ch * 32, o);
                     tmem_wait_ld();
-                    if (valid) {
+                    if (write) {
                         float v[32];
 #pragma unroll
                         for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * inv;
@@ -667,14 +693,15 @@ static bool make_map(CUtensorMap *map, bool bf16, void *base, int rank, const cu
     return r == CUDA_SUCCESS;
 }
 
-template <typename T, int G>
+template <typename T, int D, bool kStagedOut>
 static cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const Params &p,
                             int q_tiles, int num_kv_heads, int num_seqs, cudaStream_t stream) {
-    auto kern = prefill_kernel<T, G>;
+    auto kern = prefill_kernel<T, D, kStagedOut>;
     static AttrCache attr_done;
-    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), kSmemBytes, &attr_done);
+    constexpr int kSmem = Layout<D>::kSmemBytes;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), kSmem, &attr_done);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(q_tiles, num_kv_heads, num_seqs), kThreads, kSmemBytes, stream>>>(mq, mk, mv, p);
+    kern<<<dim3(q_tiles, num_kv_heads * p.sub_groups, num_seqs), kThreads, kSmem, stream>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
 
@@ -691,13 +718,23 @@ extern "C" int pa_prefill(void *out, const void *query, const int32_t *q_start, 
     if (num_seqs < 0 || num_tokens < 0 || max_q_len < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
         num_blocks < 0 || max_blocks_per_seq < 0 || num_seqs > 65535 || num_kv_heads > 65535)
         return PA_ERR_SHAPE;
+    if (kv_dtype == PA_F32) {  // fp32 caches: exact fp32 arithmetic on the CUDA cores
+        if (out_dtype != PA_F32) return PA_ERR_DTYPE;
+        return pa::prefill_cuda_cores(out, query, q_start, num_tokens, k_cache, v_cache, block_tables,
+                                      max_blocks_per_seq, context_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                                      scale, block_size, num_blocks, stream);
+    }
     if (kv_dtype != PA_F16 && kv_dtype != PA_BF16) return PA_ERR_DTYPE;
     if (out_dtype != kv_dtype && out_dtype != PA_F32) return PA_ERR_DTYPE;
-    if (head_dim != 128) return PA_ERR_HEAD_DIM;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_HEAD_DIM;
     if (block_size != 16 && block_size != 32) return PA_ERR_BLOCK_SIZE;
     if (num_heads % num_kv_heads != 0) return PA_ERR_HEADS;
     const int group = num_heads / num_kv_heads;
-    if (group != 1 && group != 2 && group != 4 && group != 8) return PA_ERR_HEADS;
+    int gshift = 0;  // head slots per token: the group rounded up to a power of two, at most 128
+    while ((1 << gshift) < group && gshift < 7) ++gshift;
+    const int gslots = 1 << gshift;
+    const int sub_groups = (group + gslots - 1) / gslots;
+    if ((long long)num_kv_heads * sub_groups > 65535) return PA_ERR_SHAPE;
     if (num_seqs == 0 || num_tokens == 0 || max_q_len == 0) return PA_OK;
     if (!out || !query || !q_start || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_NULL;
     auto al = [](const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) == 0; };
@@ -706,13 +743,13 @@ extern "C" int pa_prefill(void *out, const void *query, const int32_t *q_start, 
         return PA_ERR_ALIGN;
     const long long kv_rows = (long long)num_blocks * num_kv_heads * block_size;
     if (kv_rows >= INT32_MAX || (long long)num_tokens * num_heads >= INT32_MAX) return PA_ERR_SHAPE;
-    if ((long long)max_q_len * group >= INT32_MAX) return PA_ERR_SHAPE;
+    if ((long long)max_q_len * gslots >= INT32_MAX) return PA_ERR_SHAPE;
     const bool bf16 = kv_dtype == PA_BF16;
     CUtensorMap mq, mk, mv;
     {
         const cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_heads, (cuuint64_t)num_tokens};
         const cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)num_heads * head_dim * 2};
-        const cuuint32_t box[3] = {64, (cuuint32_t)group, (cuuint32_t)(kM / group)};
+        const cuuint32_t box[3] = {64, (cuuint32_t)gslots, (cuuint32_t)(kM / gslots)};
         if (!make_map(&mq, bf16, const_cast<void *>(query), 3, dims, strides, box)) return PA_ERR_CUDA;
     }
     {
@@ -738,23 +775,20 @@ extern "C" int pa_prefill(void *out, const void *query, const int32_t *q_start, 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.out_dtype = out_dtype;
     p.err = err;
-    const int q_tiles = (max_q_len * group + kM - 1) / kM;
+    p.group = group;
+    p.gshift = gshift;
+    p.sub_groups = sub_groups;
+    const int q_tiles = (max_q_len * gslots + kM - 1) / kM;
     cudaError_t e = cudaErrorInvalidValue;
-#define PA_PREFILL_CASE(T, GG) e = launch_t<T, GG>(mq, mk, mv, p, q_tiles, num_kv_heads, num_seqs, stream)
+#define PA_PREFILL_CASE(T, DD)                                                                   \
+    e = gslots <= 2 ? launch_t<T, DD, true>(mq, mk, mv, p, q_tiles, num_kv_heads, num_seqs, stream) \
+                    : launch_t<T, DD, false>(mq, mk, mv, p, q_tiles, num_kv_heads, num_seqs, stream)
     if (bf16) {
-        switch (group) {
-            case 1: PA_PREFILL_CASE(__nv_bfloat16, 1); break;
-            case 2: PA_PREFILL_CASE(__nv_bfloat16, 2); break;
-            case 4: PA_PREFILL_CASE(__nv_bfloat16, 4); break;
-            case 8: PA_PREFILL_CASE(__nv_bfloat16, 8); break;
-        }
+        if (head_dim == 128) PA_PREFILL_CASE(__nv_bfloat16, 128);
+        else PA_PREFILL_CASE(__nv_bfloat16, 64);
     } else {
-        switch (group) {
-            case 1: PA_PREFILL_CASE(__half, 1); break;
-            case 2: PA_PREFILL_CASE(__half, 2); break;
-            case 4: PA_PREFILL_CASE(__half, 4); break;
-            case 8: PA_PREFILL_CASE(__half, 8); break;
-        }
+        if (head_dim == 128) PA_PREFILL_CASE(__half, 128);
+        else PA_PREFILL_CASE(__half, 64);
     }
 #undef PA_PREFILL_CASE
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;

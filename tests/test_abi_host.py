@@ -72,7 +72,7 @@ A16 = 1 << 20  # a fake 16-byte aligned address; never dereferenced by these cal
     (dict(head_dim=96), -5),
     (dict(block_size=8), -6),
     (dict(num_heads=12, num_kv_heads=8), -4),
-    (dict(num_heads=48, num_kv_heads=3), -4),
+    (dict(num_heads=16 * 65535, num_kv_heads=65535), -3),   # head group 16: two CTAs per kv head, past gridDim.y
     (dict(kv_dtype=7), -2),
     (dict(out_dtype=1, kv_dtype=2), -2),
     (dict(num_seqs=-1), -3),
@@ -110,12 +110,14 @@ def test_decode_append_host_checks(pa, new_key, new_value, code):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(head_dim=64), -5),                       # the tensor-core prefill is built for head_dim 128
-    (dict(kv_dtype=0, out_dtype=0), -2),           # fp32 caches: decode only
+    (dict(head_dim=96), -5),
+    (dict(kv_dtype=0, out_dtype=1), -2),           # fp32 caches prefill into fp32 outputs
+    (dict(kv_dtype=0, out_dtype=0, head_dim=96), -5),
+    (dict(kv_dtype=0, out_dtype=0, query=A16 + 4), -7),
     (dict(out_dtype=1, kv_dtype=2), -2),
     (dict(block_size=8), -6),
     (dict(num_heads=12, num_kv_heads=8), -4),
-    (dict(num_heads=48, num_kv_heads=3), -4),      # head group 16
+    (dict(num_heads=256 * 65535, num_kv_heads=65535), -3),   # two sub-groups of 128 per kv head, past gridDim.y
     (dict(num_seqs=-1), -3),
     (dict(query=0), -1),
     (dict(q_start=A16 + 2), -7),
@@ -284,7 +286,7 @@ def test_device_pool_host_checks(pa):
     """pa_dpool_* / pa_beam_step / pa_copy_blocks_counted argument checks
     return before any device work (fake device addresses are never touched)."""
     lib = pa._lib
-    assert lib.pa_dpool_state_bytes(10) == (pa.PA_DPOOL_HEADER_WORDS + 6 * 10) * 4
+    assert lib.pa_dpool_state_bytes(10) == (pa.PA_DPOOL_HEADER_WORDS + 6 * 10 + pa.PA_DPOOL_TAIL_WORDS) * 4
     assert lib.pa_dpool_state_bytes(0) == 0
     fake = 1 << 40                                       # 16-byte aligned, never dereferenced
     assert lib.pa_dpool_init(None, 10, 16, 0, None, None) == -1
