@@ -502,7 +502,8 @@ int pa_dpool_load(void *state, int num_blocks, int block_size, int policy, const
  * old_context_lens [num_old] (entries past ceil(ctx / block_size) are not
  * read), parents [num_new] in [0, num_old). Outputs (device):
  * new_tables [num_new, max_blocks_per_seq] (-1 past the blocks in use; must
- * not overlap old_tables), new_context_lens [num_new] = parent's + 1,
+ * not overlap old_tables), new_context_lens [num_new] = parent's + 1 (must
+ * not overlap old_context_lens),
  * slot_mapping [num_new] (the new tokens' slots, for pa_reshape_and_cache),
  * cow_pairs int64 [num_new, 2] and *num_cow (for pa_copy_blocks_counted).
  * A table row never lists a block twice (the pool never makes one).

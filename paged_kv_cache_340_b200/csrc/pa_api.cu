@@ -690,7 +690,8 @@ int pa_beam_step(void *state, int num_blocks, int block_size, const int32_t *old
     if (!state || !num_cow || (num_old > 0 && (!old_tables || !old_context_lens)) ||
         (num_new > 0 && (!parents || !new_tables || !new_context_lens || !slot_mapping || !cow_pairs)))
         return PA_ERR_NULL;
-    if (num_new > 0 && num_old > 0 && new_tables == old_tables) return PA_ERR_SHAPE;
+    if (num_new > 0 && num_old > 0 && (new_tables == old_tables || new_context_lens == old_context_lens))
+        return PA_ERR_SHAPE;
     if (!aligned(state, 16) || !aligned(num_cow, 4) || !aligned(old_tables, 4) || !aligned(old_context_lens, 4) ||
         !aligned(parents, 4) || !aligned(new_tables, 4) || !aligned(new_context_lens, 4) ||
         !aligned(slot_mapping, 4) || !aligned(cow_pairs, 8))

@@ -280,9 +280,17 @@ __device__ __forceinline__ void chunk_of(const StepParams &q, int *e0, int *e1) 
 
 __device__ __forceinline__ volatile int *status_word(const Pool &p) { return p.tail; }
 
+// Programmatic dependent launch: launches 2-4 start while the previous one
+// runs (each stages the per-beam values, which no launch writes) and wait
+// for it to finish, its writes visible, before they read its results. Both
+// are no-ops for a launch made without the attribute.
+__device__ __forceinline__ void allow_next_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void wait_previous_launch() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __global__ void __launch_bounds__(kStepThreads) beam_count_kernel(const StepParams q) {
     extern __shared__ int dyn[];
     __shared__ int s_bad;
+    allow_next_launch();
     const Pool p = views(q.state, q.num_blocks);
     const Staged st = stage_beams(q, p, dyn, &s_bad);
     if (st.bad) {
@@ -377,8 +385,10 @@ __global__ void __launch_bounds__(kStepThreads) beam_flags_kernel(const StepPara
     extern __shared__ int dyn[];
     __shared__ int s_bad;
     __shared__ int warp_sums[kStepThreads / 32];
+    allow_next_launch();
     const Pool p = views(q.state, q.num_blocks);
     const Staged st = stage_beams(q, p, dyn, &s_bad);
+    wait_previous_launch();  // from here on: the previous launch's results
     const bool bad = st.bad || *status_word(p) != 0;
     const int MB = q.max_blocks;
     int e0, e1;
@@ -425,8 +435,10 @@ __global__ void __launch_bounds__(kStepThreads) beam_apply_kernel(const StepPara
     extern __shared__ int dyn[];
     __shared__ int s_bad;
     __shared__ int warp_sums[kStepThreads / 32];
+    allow_next_launch();
     const Pool p = views(q.state, q.num_blocks);
     const Staged st = stage_beams(q, p, dyn, &s_bad);
+    wait_previous_launch();  // from here on: the previous launch's results
     const int MB = q.max_blocks, nb = q.num_blocks, bs = q.block_size;
     const int head = p.hdr[3], count = p.hdr[4];
     // freed blocks in all chunks and in the chunks before this one
@@ -492,6 +504,7 @@ __global__ void __launch_bounds__(kStepThreads) beam_finish_kernel(const StepPar
     __shared__ int warp_sums[kStepThreads / 32];
     const Pool p = views(q.state, q.num_blocks);
     const Staged st = stage_beams(q, p, dyn, &s_bad);
+    wait_previous_launch();  // from here on: the previous launch's results
     const int MB = q.max_blocks, nb = q.num_blocks, bs = q.block_size;
     if (blockIdx.x == 0) {
         const int policy = p.hdr[2], head = p.hdr[3], count = p.hdr[4];
@@ -639,11 +652,23 @@ cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const in
         if (e != cudaSuccess) return e;
     }
     const dim3 grid(q.num_chunks), block(beam::kStepThreads);
-    beam::beam_count_kernel<<<grid, block, smem, stream>>>(q);
-    beam::beam_flags_kernel<<<grid, block, smem, stream>>>(q);
-    beam::beam_apply_kernel<<<grid, block, smem, stream>>>(q);
-    beam::beam_finish_kernel<<<grid, block, smem, stream>>>(q);
-    return cudaGetLastError();
+    beam::beam_count_kernel<<<grid, block, smem, stream>>>(q);  // after all earlier work on the stream
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, beam::beam_flags_kernel, q);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, beam::beam_apply_kernel, q);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, beam::beam_finish_kernel, q);
+    return e;
 }
 
 }  // namespace pa

@@ -129,13 +129,14 @@ __device__ __forceinline__ uint64_t global_ns() {
 // PA_DEVERR_TIMEOUT and leaves its loop instead of spinning forever.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
 
-// limit_ns: a bound other than kWaitLimitNs (0: kWaitLimitNs).
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns = 0) {
+// limit_ns (nullable, shared memory): a bound other than kWaitLimitNs, read
+// only once the wait has started to spin.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const uint64_t *limit_ns = nullptr) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0u && global_ns() - t0 > (limit_ns ? limit_ns : kWaitLimitNs)) return false;
+        if ((it & 63u) == 0u && global_ns() - t0 > (limit_ns ? *limit_ns : kWaitLimitNs)) return false;
     }
 }
 

@@ -86,7 +86,9 @@ struct DecodeShape {
     static constexpr int kAgStride = kUseMma ? D + 1 : D;  // floats per merged accumulator row
     static constexpr int kMergeBytes = kRowGroups * G * (kAgStride + 2) * 4;
     static constexpr int kDataBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
-    static constexpr int kSmemBytes = kAlign + kDataBytes + kStages * 8 + kStages * 4;
+    // ring (or merge area), full barriers, per-buffer "skipped" flags, and
+    // the test hook (the withheld stage and the wait bound, 16 bytes)
+    static constexpr int kSmemBytes = kAlign + kDataBytes + kStages * 8 + kStages * 4 + 16;
     // Resident CTAs per SM the register budget is set for (a sub-partition
     // holds one warp of each CTA, so 3 CTAs leave 170 registers a thread).
     static constexpr int kMinBlocks = kInt8 ? 5 : ((kUseMma || G <= 4) ? 3 : 2);
@@ -786,6 +788,10 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
         (reinterpret_cast<uintptr_t>(smem_raw) + S::kAlign - 1) & ~uintptr_t(S::kAlign - 1));
     uint64_t *full = reinterpret_cast<uint64_t *>(ring + S::kDataBytes);
     int *bad = reinterpret_cast<int *>(full + S::kStages);
+    // test hook, staged by thread 0 and read only where used: [0] this CTA's
+    // withheld stage (-1: none); [2..3] the wait bound in ns
+    int *hook = bad + S::kStages;
+    const uint64_t *wait_limit = reinterpret_cast<const uint64_t *>(hook + 2);
 
     // prefill through this kernel is for fp32 caches only (the other types
     // prefill on the tensor cores); one CTA column per query token
@@ -849,6 +855,8 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     if (threadIdx.x == 0) {
         for (int i = 0; i < S::kStages; ++i) mbar_init(full + i, 1);
         fence_mbar_init();
+        hook[0] = (s == p.withhold_seq && kvh == p.withhold_kvh && part == 0) ? p.withhold_stage : -1;
+        *reinterpret_cast<uint64_t *>(hook + 2) = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
     }
     __syncthreads();
 
@@ -886,7 +894,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     auto issue = [&](int m, int id) {  // lane 0
         const int k = warp + S::kWarps * m;
         const int buf = k % S::kStages;
-        if (k == p.withhold_stage && s == p.withhold_seq && kvh == p.withhold_kvh && part == 0) {
+        if (k == hook[0]) {
             // test hook: no copy and no arrival, so this stage's wait runs out
             bad[buf] = 1;
         } else if (id >= 0) {
@@ -957,7 +965,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
         const int buf = k % S::kStages;
         // Lane 0 polls the barrier (32 lanes polling would serialise on it);
         // __syncwarp then orders the other lanes' reads after its acquire.
-        const bool got = mbar_wait(full + buf, (k / S::kStages) & 1, p.wait_limit_ns);
+        const bool got = mbar_wait(full + buf, (k / S::kStages) & 1, wait_limit);
         if (!__all_sync(0xffffffffu, got)) {
             if (lane == 0) record_error(p.err, PA_DEVERR_TIMEOUT);
             ok = false;
@@ -1005,7 +1013,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     if (!ok && lane == 0) {  // after a timeout: let every copy this warp started land
         for (int m = waited; m < min(nmine, waited + S::kBufPerWarp); ++m) {
             const int k = warp + S::kWarps * m;
-            if (!mbar_wait(full + (k % S::kStages), (k / S::kStages) & 1, p.wait_limit_ns))
+            if (!mbar_wait(full + (k % S::kStages), (k / S::kStages) & 1, wait_limit))
                 record_error(p.err, PA_DEVERR_TIMEOUT);
         }
     }

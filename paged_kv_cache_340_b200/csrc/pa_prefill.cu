@@ -233,9 +233,11 @@ __device__ __forceinline__ bool softmax_sync_and(bool v) {
     return all != 0;
 }
 
-// kStagedOut: the output rows go through shared memory (head groups of 1-2
-// slots per token); otherwise each softmax thread stores its own row.
-template <typename T, int kD, bool kStagedOut>
+// kGS: log2 of the head slots per token when the head group is exactly 1, 2,
+// 4 or 8 (no padding, no sub-groups; compiled for that size), or -1 for any
+// other group (slots and sub-groups from Params). Groups of 1-2 stage their
+// output rows in shared memory; larger ones store one row per thread.
+template <typename T, int kD, int kGS>
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const Params p) {
@@ -245,8 +247,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     constexpr bool kBf16 = std::is_same_v<T, __nv_bfloat16>;
     constexpr uint32_t kIdescQK = mma_idesc(kBf16, kM, kN, false);
     constexpr uint32_t kIdescPV = mma_idesc(kBf16, kM, kD, true);
-    const int G = 1 << p.gshift;                       // head slots per token
-    const int kTokPerTile = kM >> p.gshift;
+    constexpr bool kExact = kGS >= 0;
+    constexpr bool kStagedOut = kGS == 0 || kGS == 1;
+    const int gshift = kExact ? kGS : p.gshift;
+    const int G = 1 << gshift;                         // head slots per token
+    const int kTokPerTile = kM >> gshift;
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -272,10 +277,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     int *abort_flag = reinterpret_cast<int *>(bars + 16);
 
     const int qt = gridDim.x - 1 - blockIdx.x;  // longest query tile of each (head, sequence) first
-    const int kvh = p.sub_groups > 1 ? (int)blockIdx.y / p.sub_groups : (int)blockIdx.y;
-    const int sub = p.sub_groups > 1 ? (int)blockIdx.y % p.sub_groups : 0;
-    const int head_base = kvh * p.group + sub * G;     // query head of slot 0
-    const int g_valid = min(G, p.group - sub * G);     // slots holding a real query head
+    const int kvh = (!kExact && p.sub_groups > 1) ? (int)blockIdx.y / p.sub_groups : (int)blockIdx.y;
+    const int sub = (!kExact && p.sub_groups > 1) ? (int)blockIdx.y % p.sub_groups : 0;
+    const int head_base = kExact ? kvh * G : kvh * p.group + sub * G;  // query head of slot 0
+    const int g_valid = kExact ? G : min(G, p.group - sub * G);         // slots holding a real query head
     const int s = blockIdx.z;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -291,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     const int rows_valid = min(kM, (q_len - tok0) * G);
     const int pos0 = ctx - q_len + tok0;                      // position of the tile's first token
-    const int pos_max = pos0 + (rows_valid >> p.gshift) - 1;
+    const int pos_max = pos0 + (rows_valid >> gshift) - 1;
     const int ntiles = pos_max / kN + 1;
 
     // Pool row of the load warp's 16-token group g0 + lane (16 tokens from
@@ -476,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     } else {
         // ======================================================= softmax warps
         const int r = threadIdx.x;  // row = tensor-memory lane
-        const int tok = r >> p.gshift;
+        const int tok = r >> gshift;
         const bool valid = r < rows_valid;
         const int pos = valid ? pos0 + tok : -1;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -621,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     const int row = i / cpr, c = i % cpr;
                     if ((row & (G - 1)) >= g_valid) continue;  // a padding slot
                     const size_t orow =
-                        (size_t)(q0 + tok0 + (row >> p.gshift)) * p.num_heads + (size_t)head_base + (row & (G - 1));
+                        (size_t)(q0 + tok0 + (row >> gshift)) * p.num_heads + (size_t)head_base + (row & (G - 1));
                     *reinterpret_cast<uint4 *>(out + orow * row_bytes + c * 16) =
                         *reinterpret_cast<const uint4 *>(Qs + row * (row_bytes + 16) + c * 16);
                 }
@@ -693,10 +698,10 @@ static bool make_map(CUtensorMap *map, bool bf16, void *base, int rank, const cu
     return r == CUDA_SUCCESS;
 }
 
-template <typename T, int D, bool kStagedOut>
+template <typename T, int D, int kGS>
 static cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const Params &p,
                             int q_tiles, int num_kv_heads, int num_seqs, cudaStream_t stream) {
-    auto kern = prefill_kernel<T, D, kStagedOut>;
+    auto kern = prefill_kernel<T, D, kGS>;
     static AttrCache attr_done;
     constexpr int kSmem = Layout<D>::kSmemBytes;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), kSmem, &attr_done);
@@ -780,9 +785,11 @@ extern "C" int pa_prefill(void *out, const void *query, const int32_t *q_start, 
     p.sub_groups = sub_groups;
     const int q_tiles = (max_q_len * gslots + kM - 1) / kM;
     cudaError_t e = cudaErrorInvalidValue;
-#define PA_PREFILL_CASE(T, DD)                                                                   \
-    e = gslots <= 2 ? launch_t<T, DD, true>(mq, mk, mv, p, q_tiles, num_kv_heads, num_seqs, stream) \
-                    : launch_t<T, DD, false>(mq, mk, mv, p, q_tiles, num_kv_heads, num_seqs, stream)
+#define PA_PREFILL_GS(T, DD, GS) launch_t<T, DD, GS>(mq, mk, mv, p, q_tiles, num_kv_heads, num_seqs, stream)
+#define PA_PREFILL_CASE(T, DD)                                                                  \
+    e = group == 1 ? PA_PREFILL_GS(T, DD, 0) : group == 2 ? PA_PREFILL_GS(T, DD, 1)             \
+      : group == 4 ? PA_PREFILL_GS(T, DD, 2) : group == 8 ? PA_PREFILL_GS(T, DD, 3)             \
+                   : PA_PREFILL_GS(T, DD, -1)
     if (bf16) {
         if (head_dim == 128) PA_PREFILL_CASE(__nv_bfloat16, 128);
         else PA_PREFILL_CASE(__nv_bfloat16, 64);
@@ -791,5 +798,6 @@ extern "C" int pa_prefill(void *out, const void *query, const int32_t *q_start, 
         else PA_PREFILL_CASE(__half, 64);
     }
 #undef PA_PREFILL_CASE
+#undef PA_PREFILL_GS
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -293,7 +293,8 @@ def test_device_pool_host_checks(pa):
     assert lib.pa_dpool_init(fake, 0, 16, 0, None, None) == -3
     assert lib.pa_dpool_init(fake, 10, 16, 7, None, None) == -3
     assert lib.pa_dpool_init(fake + 4, 10, 16, 0, None, None) == -7
-    args = dict(old_t=fake, old_c=fake, par=fake, new_t=fake + 4096, new_c=fake, slots=fake, cow=fake, ncow=fake)
+    args = dict(old_t=fake, old_c=fake, par=fake, new_t=fake + 4096, new_c=fake + 8192, slots=fake, cow=fake,
+                ncow=fake)
 
     def step(state=fake, nb=64, bs=16, num_old=2, num_new=2, mb=4, **kw):
         a = dict(args, **kw)
@@ -308,6 +309,7 @@ def test_device_pool_host_checks(pa):
     assert step(num_old=1 << 12, mb=1 << 18) == -3      # flattened table index past 2^30
     assert step(num_old=20000, num_new=1) == -3           # per-beam values past the shared-memory stage
     assert step(new_t=fake) == -3                        # output tables alias the input tables
+    assert step(new_c=fake) == -3                        # output context lengths alias the input ones
     assert step(cow=fake + 4) == -7
     assert lib.pa_copy_blocks_counted(fake, fake, fake, None, 4, 8, 2, 128, 16, 1, None) == -1
     assert lib.pa_copy_blocks_counted(fake, fake, fake, fake, 4, 8, 2, 100, 16, 1, None) == -5
