@@ -458,13 +458,16 @@ int pa_prefix_ref_count(pa_prefix_cache *cache, const int32_t *tokens, int num_t
  * The pool's state lives in one caller-allocated DEVICE buffer of
  * pa_dpool_state_bytes(num_blocks) bytes (16-byte aligned), int32 words:
  *   [0] num_blocks  [1] block_size  [2] policy  [3] head  [4] count
- *   [5] a marker set by pa_dpool_init  [6..7] reserved
+ *   [5] a marker set by pa_dpool_init  [6..7] the beam step's own
+ *   bookkeeping (a step count and a grid-barrier base; every step advances
+ *   them, also a step that applies nothing)
  *   ref   = words + PA_DPOOL_HEADER_WORDS          [num_blocks] reference counts
  *   ring  = ref + num_blocks                       [num_blocks] free list: entries
  *           ring[(head + k) % num_blocks], k < count, front first
  *   then four scratch arrays of num_blocks words each (all zero / -1 between
- *   calls), then PA_DPOOL_TAIL_WORDS words of step scratch (a status word and
- *   per-chunk totals; zero between calls). The library keeps no pointer to it.
+ *   calls), then PA_DPOOL_TAIL_WORDS words of beam-step scratch (status
+ *   words, per-chunk totals, a grid-barrier count). The library keeps no
+ *   pointer to it.
  * Same rules as the host pool: PA_POOL_FIFO takes the free list's front,
  * PA_POOL_LIFO its back; freed blocks go to the back.
  */
@@ -509,9 +512,12 @@ int pa_dpool_load(void *state, int num_blocks, int block_size, int policy, const
  * A table row never lists a block twice (the pool never makes one).
  * Any error (a bad parent, context or block id, a free list too short, no
  * table room for the new token, an uninitialised state) applies nothing:
- * the state is unchanged, every slot is -1, *num_cow = 0 and a PA_DEVERR_*
- * bit is set. Runs as four launches over chunks of the old tables (spread
- * over the SMs); calls on one state must not overlap.
+ * counts, free list and header words 0-5 are unchanged, every slot is -1,
+ * *num_cow = 0 and a PA_DEVERR_* bit is set. Runs over chunks of the old
+ * tables spread over the SMs: one cooperative launch (up to 1024 new beams
+ * and 1024 table entries per SM; its grid barriers wait at most 200 ms, and a
+ * wait that gives up marks the state unusable), else four launches. Calls on
+ * one state must not overlap.
  * Limits (else PA_ERR_SHAPE): 3 * num_old + num_new <= PA_BEAM_MAX_STAGED
  * and (num_old + num_new) * max_blocks_per_seq < 2^30.
  */

@@ -189,10 +189,12 @@ struct StepParams {
 
 // ------------------------------------------------------------------ beam step
 //
-// Four launches over chunks of the old tables' entries (flattened (beam,
+// Four phases over chunks of the old tables' entries (flattened (beam,
 // position) index e = j * max_blocks + pos), so that the passes over the
-// tables and their atomics spread over the SMs; a kernel boundary is the
-// only grid-wide ordering used. Every CTA first stages the per-beam values
+// tables and their atomics spread over the SMs. They run as one cooperative
+// launch with a grid barrier between phases (at most one CTA per SM, all
+// resident at once), or, where a cooperative launch is refused, as four
+// launches whose boundaries order them. Every CTA first stages the per-beam values
 // (context length, block count, number of children, parent) in shared
 // memory and makes the same argument checks, so all CTAs agree on them
 // without a global exchange. Between launches the step keeps a status word
@@ -220,7 +222,7 @@ struct StepParams {
 // copy count is 0.
 
 constexpr int kStepThreads = 256;
-constexpr int kMaxChunks = PA_DPOOL_TAIL_WORDS - 4;
+constexpr int kMaxChunks = PA_DPOOL_TAIL_WORDS - 10;  // tail: 4 words, chunk totals, the one-launch words
 // tail words: [0] status bits of this step, [1] blocks taken, [2] copies,
 // [4 + c] freed blocks in chunk c
 
@@ -246,18 +248,19 @@ __device__ Staged stage_beams(const StepParams &q, const Pool &p, int *dyn, int 
             count > q.num_blocks || head < 0 || head >= q.num_blocks)
             *s_bad = PA_DEVERR_POOL;
     }
+    // contexts and parents are independent loads: one round trip for both
     for (int j = threadIdx.x; j < n_old; j += kStepThreads) {
         const int c = __ldg(q.old_ctx + j);
         st.ctx[j] = c;
         st.nblk[j] = c < 0 ? 0 : nblk(c, bs);
         st.nch[j] = 0;
     }
+    for (int i = threadIdx.x; i < n_new; i += kStepThreads) st.par[i] = __ldg(q.parents + i);
     __syncthreads();
     for (int j = threadIdx.x; j < n_old; j += kStepThreads)
         if (st.ctx[j] < 0 || st.nblk[j] > MB) atomicOr(s_bad, PA_DEVERR_CONTEXT);
     for (int i = threadIdx.x; i < n_new; i += kStepThreads) {
-        const int par = __ldg(q.parents + i);
-        st.par[i] = par;
+        const int par = st.par[i];
         if (par < 0 || par >= n_old) {
             atomicOr(s_bad, PA_DEVERR_CONTEXT);
         } else {
@@ -287,12 +290,8 @@ __device__ __forceinline__ volatile int *status_word(const Pool &p) { return p.t
 __device__ __forceinline__ void allow_next_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void wait_previous_launch() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-__global__ void __launch_bounds__(kStepThreads) beam_count_kernel(const StepParams q) {
-    extern __shared__ int dyn[];
-    __shared__ int s_bad;
-    allow_next_launch();
-    const Pool p = views(q.state, q.num_blocks);
-    const Staged st = stage_beams(q, p, dyn, &s_bad);
+// ---- phase 1 (count)
+__device__ void phase_count(const StepParams &q, const Pool &p, const Staged &st) {
     if (st.bad) {
         if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.tail, st.bad);
         return;
@@ -381,14 +380,8 @@ __device__ __forceinline__ void take_and_copy(const StepParams &q, const Pool &p
     }
 }
 
-__global__ void __launch_bounds__(kStepThreads) beam_flags_kernel(const StepParams q) {
-    extern __shared__ int dyn[];
-    __shared__ int s_bad;
-    __shared__ int warp_sums[kStepThreads / 32];
-    allow_next_launch();
-    const Pool p = views(q.state, q.num_blocks);
-    const Staged st = stage_beams(q, p, dyn, &s_bad);
-    wait_previous_launch();  // from here on: the previous launch's results
+// ---- phase 2 (flags)
+__device__ void phase_flags(const StepParams &q, const Pool &p, const Staged &st, int *warp_sums) {
     const bool bad = st.bad || *status_word(p) != 0;
     const int MB = q.max_blocks;
     int e0, e1;
@@ -431,19 +424,13 @@ __global__ void __launch_bounds__(kStepThreads) beam_flags_kernel(const StepPara
     }
 }
 
-__global__ void __launch_bounds__(kStepThreads) beam_apply_kernel(const StepParams q) {
-    extern __shared__ int dyn[];
-    __shared__ int s_bad;
-    __shared__ int warp_sums[kStepThreads / 32];
-    allow_next_launch();
-    const Pool p = views(q.state, q.num_blocks);
-    const Staged st = stage_beams(q, p, dyn, &s_bad);
-    wait_previous_launch();  // from here on: the previous launch's results
+// ---- phase 3 (apply)
+__device__ void phase_apply(const StepParams &q, const Pool &p, const Staged &st, int *warp_sums) {
     const int MB = q.max_blocks, nb = q.num_blocks, bs = q.block_size;
     const int head = p.hdr[3], count = p.hdr[4];
     // freed blocks in all chunks and in the chunks before this one
     int before = 0, freed = 0;
-    for (int c = threadIdx.x; c < (int)gridDim.x; c += kStepThreads) {
+    for (int c = threadIdx.x; c < q.num_chunks; c += kStepThreads) {
         const int v = p.tail[4 + c];
         freed += v;
         if (c < (int)blockIdx.x) before += v;
@@ -498,13 +485,8 @@ __global__ void __launch_bounds__(kStepThreads) beam_apply_kernel(const StepPara
     }
 }
 
-__global__ void __launch_bounds__(kStepThreads) beam_finish_kernel(const StepParams q) {
-    extern __shared__ int dyn[];
-    __shared__ int s_bad;
-    __shared__ int warp_sums[kStepThreads / 32];
-    const Pool p = views(q.state, q.num_blocks);
-    const Staged st = stage_beams(q, p, dyn, &s_bad);
-    wait_previous_launch();  // from here on: the previous launch's results
+// ---- phase 4 (finish)
+__device__ void phase_finish(const StepParams &q, const Pool &p, const Staged &st, int *warp_sums) {
     const int MB = q.max_blocks, nb = q.num_blocks, bs = q.block_size;
     if (blockIdx.x == 0) {
         const int policy = p.hdr[2], head = p.hdr[3], count = p.hdr[4];
@@ -595,6 +577,339 @@ __global__ void __launch_bounds__(kStepThreads) beam_finish_kernel(const StepPar
     }
 }
 
+
+// ---- the four phases as four launches (launches 2-4 by programmatic
+// dependent launch)
+
+__global__ void __launch_bounds__(kStepThreads) beam_count_kernel(const StepParams q) {
+    extern __shared__ int dyn[];
+    __shared__ int s_bad;
+    allow_next_launch();
+    const Pool p = views(q.state, q.num_blocks);
+    const Staged st = stage_beams(q, p, dyn, &s_bad);
+    phase_count(q, p, st);
+}
+
+#define PA_BEAM_PHASE_KERNEL(NAME, PHASE, ALLOW_NEXT)                                    \
+    __global__ void __launch_bounds__(kStepThreads) NAME(const StepParams q) {           \
+        extern __shared__ int dyn[];                                                     \
+        __shared__ int s_bad;                                                            \
+        __shared__ int warp_sums[kStepThreads / 32];                                     \
+        if (ALLOW_NEXT) allow_next_launch();                                             \
+        const Pool p = views(q.state, q.num_blocks);                                     \
+        const Staged st = stage_beams(q, p, dyn, &s_bad);                                \
+        wait_previous_launch(); /* from here on: the previous launch's results */        \
+        PHASE(q, p, st, warp_sums);                                                      \
+    }
+PA_BEAM_PHASE_KERNEL(beam_flags_kernel, phase_flags, true)
+PA_BEAM_PHASE_KERNEL(beam_apply_kernel, phase_apply, true)
+PA_BEAM_PHASE_KERNEL(beam_finish_kernel, phase_finish, false)
+#undef PA_BEAM_PHASE_KERNEL
+
+// ---- the four phases in one cooperative launch: every CTA is resident at
+// once (the launch guarantees it, or fails), so a CTA may wait for the others
+// at a grid barrier between phases. Barrier and exit counters live in the
+// pool's tail; each wait is bounded (a CTA that gives up records
+// PA_DEVERR_TIMEOUT and the step stops; with every CTA resident that does
+// not happen).
+
+// Words of the one-launch form: a status word per epoch parity (the step's
+// PA_DEVERR bits; each step clears the next step's), the grid barrier's
+// arrival count (it only grows: barrier k of a step waits for base + k * CTAs
+// arrivals, base kept in header word 7), and the epoch + 1 of a step whose
+// barrier wait gave up. Header word 6 counts the steps (the epoch).
+constexpr int kFusedStatus = PA_DPOOL_TAIL_WORDS - 6;  // and - 5
+constexpr int kBarArrive = PA_DPOOL_TAIL_WORDS - 3;
+constexpr int kBarAbort = PA_DPOOL_TAIL_WORDS - 2;
+constexpr uint64_t kBarrierLimitNs = 200ull * 1000ull * 1000ull;  // 200 ms
+
+__device__ __forceinline__ int ld_acquire(const int *a) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+    return v;
+}
+
+// Grid barrier: true once `target` arrivals are counted. A wait that gives
+// up (or sees that another CTA gave up) leaves the pool unusable: the step
+// stopped part way, and later steps refuse the state (PA_DEVERR_POOL).
+__device__ bool grid_barrier(const Pool &p, unsigned target, int epoch, unsigned int *err, int *s_go) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();  // this CTA's writes, before its arrival
+        atomicAdd(reinterpret_cast<unsigned *>(&p.tail[kBarArrive]), 1u);
+        bool ok = true;
+        uint64_t t0 = 0;
+        for (uint32_t it = 0; (int)((unsigned)ld_acquire(&p.tail[kBarArrive]) - target) < 0; ++it) {
+            if ((it & 63u) != 63u) continue;
+            if (ld_acquire(&p.tail[kBarAbort]) == epoch + 1) { ok = false; break; }
+            const uint64_t t = global_ns();
+            if (t0 == 0) t0 = t;
+            else if (t - t0 > kBarrierLimitNs) {
+                atomicExch(&p.tail[kBarAbort], epoch + 1);
+                p.hdr[5] = 0;
+                record_error(err, PA_DEVERR_TIMEOUT);
+                ok = false;
+                break;
+            }
+        }
+        __threadfence();
+        *s_go = ok;
+    }
+    __syncthreads();
+    return *s_go != 0;
+}
+
+// Entries of the old tables (contiguous, per thread) and new beams (one per
+// thread per round) the fused kernel keeps in registers across its phases.
+constexpr int kFusedEntries = 4;
+constexpr int kFusedBeams = 4;
+
+__global__ void __launch_bounds__(kStepThreads) beam_step_kernel(const StepParams q) {
+    extern __shared__ int dyn[];
+    __shared__ int s_bad, s_go;
+    __shared__ int warp_sums[kStepThreads / 32];
+    const Pool p = views(q.state, q.num_blocks);
+    const int MB = q.max_blocks, nb = q.num_blocks, bs = q.block_size;
+    const int tid = threadIdx.x;
+    const unsigned G = gridDim.x;
+    // the header as it stands before the step (only CTA 0 changes it, after
+    // every CTA has passed the first barrier)
+    const int policy = p.hdr[2], head = p.hdr[3], count = p.hdr[4];
+    const int epoch = p.hdr[6];
+    const unsigned base = (unsigned)p.hdr[7];
+    int *status = p.tail + kFusedStatus + (epoch & 1);
+    if (blockIdx.x == 0 && tid == 0) p.tail[kFusedStatus + ((epoch + 1) & 1)] = 0;  // the next step's
+    const Staged st = stage_beams(q, p, dyn, &s_bad);
+
+    // ---- phase 1: this thread's entries (contiguous run of the chunk):
+    // validate, net count change, last release; writers per block
+    int e0, e1;
+    chunk_of(q, &e0, &e1);
+    const int per = q.chunk / kStepThreads;  // <= kFusedEntries (host check)
+    const int ea = e0 + tid * per;
+    // eb: block id of entry k; ev: in use and valid (only such entries are
+    // ever acted on); ench: children of its beam; eref: its count before the step
+    int eb[kFusedEntries], eref[kFusedEntries], ench[kFusedEntries];
+    bool euse[kFusedEntries], ev[kFusedEntries], efree[kFusedEntries];
+#pragma unroll
+    for (int k = 0; k < kFusedEntries; ++k) {
+        eb[k] = -1;
+        ench[k] = 1;
+        euse[k] = ev[k] = efree[k] = false;
+        const int e = ea + k;
+        if (!st.bad && k < per && e < e1) {
+            const int j = e / MB, pos = e - j * MB;
+            if (pos < st.nblk[j]) {
+                eb[k] = __ldg(q.old_tables + e);
+                ench[k] = st.nch[j];
+                euse[k] = true;
+            }
+        }
+    }
+    // new beam i = round * 256 + tid: CTA 0 keeps its old block (-1 at a block
+    // boundary) and context for phases 2-3
+    int bo[kFusedBeams], bt[kFusedBeams];
+#pragma unroll
+    for (int r = 0; r < kFusedBeams; ++r) {
+        bo[r] = -1;
+        bt[r] = 0;
+        const int i = r * kStepThreads + tid;
+        if (blockIdx.x == 0 && !st.bad && i < q.num_new) {
+            bt[r] = st.ctx[st.par[i]];
+            if (bt[r] % bs) bo[r] = __ldg(q.old_tables + st.par[i] * MB + bt[r] / bs);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < kFusedEntries; ++k)
+        if (euse[k] && eb[k] >= 0 && eb[k] < nb) eref[k] = p.ref[eb[k]];
+#pragma unroll
+    for (int k = 0; k < kFusedEntries; ++k) {
+        if (!euse[k]) continue;
+        const int b = eb[k];
+        if (b < 0 || b >= nb || eref[k] <= 0) {
+            atomicOr(status, PA_DEVERR_BLOCK_ID);
+            continue;
+        }
+        ev[k] = true;
+        if (ench[k] != 1) atomicAdd(&p.delta[b], ench[k] - 1);
+        if (ench[k] == 0) atomicMax(&p.last_old[b], ea + k);
+    }
+    if (blockIdx.x == 0) {
+#pragma unroll
+        for (int r = 0; r < kFusedBeams; ++r) {
+            const int o = bo[r];
+            if (o >= 0 && o < nb) {
+                atomicAdd(&p.writers[o], 1);
+                atomicMax(&p.last_writer[o], r * kStepThreads + tid);
+            }
+        }
+        if (tid == 0 && st.bad) atomicOr(status, st.bad);
+    }
+
+    bool go = grid_barrier(p, base + G, epoch, q.err, &s_go);
+    // ---- phase 2: which entries free their block (count reaches 0 at its last
+    // release); per-chunk totals; CTA 0 decides each new beam's take and copy.
+    // Every load of the phase is issued before the status is tested.
+    int bk[kFusedBeams], bc[kFusedBeams];  // CTA 0: take index, copy index (-1: none)
+    int takes = 0, copies = 0;
+    {
+        int dl[kFusedEntries], lo[kFusedEntries];
+#pragma unroll
+        for (int k = 0; k < kFusedEntries; ++k)
+            if (ev[k] && ench[k] == 0) {
+                dl[k] = p.delta[eb[k]];
+                lo[k] = p.last_old[eb[k]];
+            }
+        int rr[kFusedBeams], wr[kFusedBeams], lw[kFusedBeams];
+        if (blockIdx.x == 0) {
+#pragma unroll
+            for (int r = 0; r < kFusedBeams; ++r)
+                if (bo[r] >= 0 && bo[r] < nb) {
+                    rr[r] = p.ref[bo[r]] + p.delta[bo[r]];
+                    wr[r] = p.writers[bo[r]];
+                    lw[r] = p.last_writer[bo[r]];
+                }
+        }
+        const bool bad2 = !go || st.bad || ld_acquire(status) != 0;
+        int cnt = 0;
+#pragma unroll
+        for (int k = 0; k < kFusedEntries; ++k)
+            if (!bad2 && ev[k] && ench[k] == 0) {
+                const int r = eref[k] + dl[k];
+                if (r < 0) atomicOr(status, PA_DEVERR_POOL);  // a table holds a block more often than counted
+                efree[k] = r == 0 && lo[k] == ea + k;
+                cnt += efree[k];
+            }
+        cnt = cta_sum(cnt, warp_sums);
+        if (tid == 0) p.tail[4 + blockIdx.x] = cnt;
+        if (blockIdx.x == 0) {
+#pragma unroll
+            for (int r = 0; r < kFusedBeams; ++r) {
+                const int i = r * kStepThreads + tid;
+                int need = 0, copy = 0;
+                if (!bad2 && i < q.num_new) {
+                    if (bo[r] < 0) {
+                        need = 1;
+                    } else {
+                        copy = rr[r] - wr[r] > 0 || lw[r] != i;
+                        need = copy;
+                    }
+                }
+                int tt, tc;
+                const int k = takes + cta_scan(need, warp_sums, &tt);
+                const int c = copies + cta_scan(copy, warp_sums, &tc);
+                bk[r] = need ? k : -1;
+                bc[r] = copy ? c : -1;
+                takes += tt;
+                copies += tc;
+            }
+            if (tid == 0) {
+                p.tail[1] = takes;
+                p.tail[2] = copies;
+            }
+        }
+    }
+
+    go = grid_barrier(p, base + 2 * G, epoch, q.err, &s_go) && go;
+    // ---- phase 3: apply. Deltas are swapped out first (their values are
+    // needed only once the outcome is known), then freed blocks go to the
+    // back of the free list in entry order, counts take their net change, the
+    // new tables get their parents' rows; CTA 0 the takes (from the free
+    // list's front: FIFO with enough free blocks) or, otherwise, after one
+    // more barrier
+    int dx[kFusedEntries];
+#pragma unroll
+    for (int k = 0; k < kFusedEntries; ++k) {
+        dx[k] = 0;
+        if (ev[k] && ench[k] != 1) dx[k] = atomicExch(&p.delta[eb[k]], 0);
+    }
+    int freed = 0, before = 0;
+    for (int c = tid; c < q.num_chunks; c += kStepThreads) {
+        const int v = p.tail[4 + c];
+        freed += v;
+        if (c < (int)blockIdx.x) before += v;
+    }
+    takes = p.tail[1];
+    copies = p.tail[2];
+    const int bits = ld_acquire(status);
+    freed = cta_sum(freed, warp_sums);
+    before = cta_sum(before, warp_sums);
+    const bool ok = go && !st.bad && bits == 0 && takes <= count + freed;
+    {
+        int mine = 0;
+#pragma unroll
+        for (int k = 0; k < kFusedEntries; ++k) mine += efree[k];
+        int tot;
+        int r = before + cta_scan(mine, warp_sums, &tot);
+#pragma unroll
+        for (int k = 0; k < kFusedEntries; ++k)
+            if (ok && efree[k]) p.ring[(head + count + r++) % nb] = eb[k];
+    }
+#pragma unroll
+    for (int k = 0; k < kFusedEntries; ++k) {
+        if (ok && dx[k]) atomicAdd(&p.ref[eb[k]], dx[k]);
+        if (ev[k] && ench[k] == 0) p.last_old[eb[k]] = -1;
+    }
+    if (ok) {  // the new tables: parents' rows, -1 past them; each beam's write entry is CTA 0's
+        const long long new_entries = (long long)q.num_new * MB;
+        for (long long e = (long long)blockIdx.x * kStepThreads + tid; e < new_entries;
+             e += (long long)G * kStepThreads) {
+            const int i = (int)(e / MB), pos = (int)(e - (long long)i * MB);
+            const int par = st.par[i];
+            if (pos == st.ctx[par] / bs) continue;
+            q.new_tables[e] = pos < st.nblk[par] ? __ldg(q.old_tables + par * MB + pos) : -1;
+        }
+    }
+    const bool early = policy == PA_POOL_FIFO && takes <= count;  // the same in every CTA
+    if (!early) go = grid_barrier(p, base + 3 * G, epoch, q.err, &s_go) && go;  // the freed blocks are listed
+    if (blockIdx.x == 0) {
+        const bool ok4 = ok && go;
+#pragma unroll
+        for (int r = 0; r < kFusedBeams; ++r) {
+            const int i = r * kStepThreads + tid;
+            if (!ok4 || i >= q.num_new) continue;
+            const int o = bo[r], t = bt[r];
+            int b = o;
+            if (bk[r] >= 0) {
+                const int k = bk[r];
+                b = policy == PA_POOL_FIFO ? p.ring[(head + k) % nb] : p.ring[(head + count + freed - 1 - k) % nb];
+                p.ref[b] = 1;
+            }
+            q.new_tables[(long long)i * MB + t / bs] = b;
+            if (bc[r] >= 0) {
+                q.cow_pairs[2 * bc[r]] = o;
+                q.cow_pairs[2 * bc[r] + 1] = b;
+                atomicSub(&p.ref[o], 1);  // a copying writer gives up its reference to the old block
+            }
+            q.slots[i] = b * bs + t % bs;
+            q.new_ctx[i] = t + 1;
+        }
+#pragma unroll
+        for (int r = 0; r < kFusedBeams; ++r) {  // writer marks back, failed outputs
+            const int i = r * kStepThreads + tid;
+            if (bo[r] >= 0 && bo[r] < nb) {
+                p.writers[bo[r]] = 0;
+                p.last_writer[bo[r]] = -1;
+            }
+            if (!ok4 && i < q.num_new) q.slots[i] = -1;
+        }
+        if (tid == 0) {
+            if (ok4) {
+                p.hdr[3] = policy == PA_POOL_FIFO ? (head + takes) % nb : head;
+                p.hdr[4] = count + freed - takes;
+                *q.num_cow = copies;
+            } else {
+                *q.num_cow = 0;
+                const int why = st.bad | bits;
+                record_error(q.err, why ? (unsigned)why : (go ? PA_DEVERR_POOL : PA_DEVERR_TIMEOUT));
+            }
+            // the next step's epoch and barrier base (every CTA read them before barrier 1)
+            p.hdr[7] = (int)(base + (early ? 2u : 3u) * G);
+            p.hdr[6] = epoch + 1;
+        }
+    }
+}
+
 }  // namespace beam
 
 cudaError_t launch_dpool_init(int32_t *state, int num_blocks, int block_size, int policy,
@@ -635,13 +950,48 @@ cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const in
     q.num_blocks = num_blocks;
     q.block_size = block_size;
     q.err = err;
-    // chunks of at least one entry per thread, at most kMaxChunks of them
     const long long entries = (long long)num_old * max_blocks;
-    long long chunk = beam::kStepThreads;
-    while ((entries + chunk - 1) / chunk > beam::kMaxChunks) chunk += beam::kStepThreads;
+    const int smem = (3 * num_old + num_new) * (int)sizeof(int);
+    const dim3 block(beam::kStepThreads);
+    // chunk: a multiple of the CTA size, so that there are at most max_ctas chunks
+    auto chunk_for = [&](long long max_ctas) {
+        long long c = (entries + max_ctas - 1) / max_ctas;
+        c = (c + beam::kStepThreads - 1) / beam::kStepThreads * beam::kStepThreads;
+        return std::max<long long>(c, beam::kStepThreads);
+    };
+    // One cooperative launch, one CTA per chunk and at most one chunk per SM
+    // (one such CTA fits on any SM: 256 threads, < 100 KB of shared memory,
+    // few registers, so the whole grid can be resident at once).
+    const long long fused_chunk = chunk_for(std::min<long long>(sm_count(), beam::kMaxChunks));
+    if (fused_chunk <= (long long)beam::kStepThreads * beam::kFusedEntries &&
+        num_new <= beam::kStepThreads * beam::kFusedBeams) {
+        const long long chunk = fused_chunk;
+        q.chunk = (int)chunk;
+        q.num_chunks = (int)std::max(1LL, (entries + chunk - 1) / chunk);
+        static AttrCache fused_attr;
+        cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(beam::beam_step_kernel),
+                                         beam::kMaxStageBytes, &fused_attr);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(q.num_chunks);
+        cfg.blockDim = block;
+        cfg.dynamicSmemBytes = (size_t)smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, beam::beam_step_kernel, q);
+        if (e == cudaSuccess) return cudaSuccess;
+        if (e != cudaErrorCooperativeLaunchTooLarge && e != cudaErrorNotSupported) return e;
+        (void)cudaGetLastError();  // not launched: the four launches below instead
+    }
+    // Four launches (launches 2-4 by programmatic dependent launch), chunks
+    // of at least one entry per thread, at most kMaxChunks of them.
+    const long long chunk = chunk_for(beam::kMaxChunks);
     q.chunk = (int)chunk;
     q.num_chunks = (int)std::max(1LL, (entries + chunk - 1) / chunk);
-    const int smem = (3 * num_old + num_new) * (int)sizeof(int);
     static AttrCache attr_done[4];
     const void *kernels[4] = {reinterpret_cast<const void *>(beam::beam_count_kernel),
                               reinterpret_cast<const void *>(beam::beam_flags_kernel),
@@ -651,7 +1001,7 @@ cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const in
         cudaError_t e = ensure_smem_attr(kernels[k], beam::kMaxStageBytes, &attr_done[k]);
         if (e != cudaSuccess) return e;
     }
-    const dim3 grid(q.num_chunks), block(beam::kStepThreads);
+    const dim3 grid(q.num_chunks);
     beam::beam_count_kernel<<<grid, block, smem, stream>>>(q);  // after all earlier work on the stream
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -152,13 +152,14 @@ def test_worked_example_on_device(pa):
 
 @pytest.mark.parametrize("policy", ["fifo", "lifo"])
 @pytest.mark.parametrize("bs", [4, 16])
-@pytest.mark.parametrize("extra", [8, 1600])
+@pytest.mark.parametrize("extra", [8, 1600, 5000])
 def test_random_beam_search_matches_oracle(pa, policy, bs, extra):
     """60 steps of random beam choices (widths 1-40, some parents chosen many
     times, some beams dropped) from 12 prompts: after every step the device
-    state, tables, slots and pairs equal the oracle's. With 1600 spare table
-    columns, steps from 30 or more beams have old tables too large to stage
-    in shared memory (over 200 KB), so both forms of the kernel run."""
+    state, tables, slots and pairs equal the oracle's. With 5000 spare table
+    columns, steps from 30 or more beams have more old-table entries than the
+    one-launch form keeps in registers (1024 per SM), so the four-launch form
+    runs for those steps and the one-launch form for the others."""
     rng = np.random.default_rng(3 + bs)
     mb = 400 // bs + extra
     lengths = [int(x) for x in rng.integers(1, 300, size=12)]
@@ -179,28 +180,36 @@ def test_random_beam_search_matches_oracle(pa, policy, bs, extra):
     assert pa.pa_read_device_errors() == 0
 
 
+def _pool_words(pa, dpool):
+    """The pool proper: header words 0-5, counts, free-list ring and the
+    per-block scratch arrays (words 6-7 and the tail are the device step's
+    own bookkeeping, which every step advances)."""
+    h, nb = pa.PA_DPOOL_HEADER_WORDS, dpool.num_blocks
+    return torch.cat([dpool.state[:6], dpool.state[h:h + 6 * nb]]).clone()
+
+
 def test_exhausted_pool_applies_nothing(pa):
     """Fewer free blocks than the step needs: state unchanged, slots -1, no pairs."""
     opool, dpool, beams = _start(pa, 12, 4, "fifo", [4, 8], seed=1)   # 3 blocks used, 9 free
-    before = dpool.state.clone()
+    before = _pool_words(pa, dpool)
     # 10 children all at a block boundary (4 and 8 tokens): 10 new blocks wanted, 9 free (+0 freed)
     t, c, s, cw, n = _device_step(pa, dpool, beams, [0] * 5 + [1] * 5, 4)
     assert pa.pa_read_device_errors() & pa.PA_DEVERR_POOL
     assert (s == -1).all() and n == 0
-    assert torch.equal(dpool.state, before)
+    assert torch.equal(_pool_words(pa, dpool), before)
     # bad parent index
     t, c, s, cw, n = _device_step(pa, dpool, beams, [0, 2], 4)
     assert pa.pa_read_device_errors() & pa.PA_DEVERR_CONTEXT
-    assert torch.equal(dpool.state, before)
+    assert torch.equal(_pool_words(pa, dpool), before)
     # a table entry that the pool says is free
     bad = [Sequence([beams[0].block_table[0]], 4), Sequence([opool.free_blocks[0]], 2)]
     t, c, s, cw, n = _device_step(pa, dpool, bad, [0, 1], 4)
     assert pa.pa_read_device_errors() & pa.PA_DEVERR_BLOCK_ID
-    assert torch.equal(dpool.state, before)
+    assert torch.equal(_pool_words(pa, dpool), before)
     # no table room for the new token
     t, c, s, cw, n = _device_step(pa, dpool, beams, [1], 2)
     assert pa.pa_read_device_errors() & pa.PA_DEVERR_POOL
-    assert torch.equal(dpool.state, before)
+    assert torch.equal(_pool_words(pa, dpool), before)
 
 
 def _beam_data_case(pa, seed, dtype):
@@ -397,4 +406,27 @@ def test_beam_step_release_all_and_empty_beams(pa, policy):
     assert t.tolist() == _tables(new, 8).tolist() and s_.tolist() == slots and n == 0 == len(cow)
     assert c.tolist() == [1, 1]
     _assert_same_state(dpool, opool)
+    assert pa.pa_read_device_errors() == 0
+
+
+@pytest.mark.parametrize("policy", ["fifo", "lifo"])
+def test_many_beams_matches_oracle(pa, policy):
+    """Steps with more new beams (1100-1300) than the one-launch form serves
+    (1024): the four-launch form, against the oracle, and a step after it
+    with few beams (the one-launch form) on the state it left."""
+    rng = np.random.default_rng(17)
+    bs, mb = 16, 24
+    lengths = [int(x) for x in rng.integers(1, 200, size=40)]
+    opool, dpool, beams = _start(pa, 6000, bs, policy, lengths, seed=5)
+    for step, w in enumerate((1100, 1300, 12, 1200)):
+        parents = [int(rng.integers(len(beams))) for _ in range(w)]
+        ob = [Sequence(list(b.block_table), b.num_tokens) for b in beams]
+        new, slots, cow = beam_step(opool, ob, parents)
+        t, c, s, cw, n = _device_step(pa, dpool, beams, parents, mb)
+        assert t.tolist() == _tables(new, mb).tolist(), step
+        assert c.tolist() == [b.num_tokens for b in new]
+        assert s.tolist() == slots
+        assert n == len(cow) and [tuple(x) for x in cw[:n].tolist()] == cow
+        _assert_same_state(dpool, opool)
+        beams = new
     assert pa.pa_read_device_errors() == 0
