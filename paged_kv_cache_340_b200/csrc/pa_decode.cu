@@ -91,7 +91,7 @@ struct DecodeShape {
     static constexpr int kSmemBytes = kAlign + kDataBytes + kStages * 8 + kStages * 4 + 16;
     // Resident CTAs per SM the register budget is set for (a sub-partition
     // holds one warp of each CTA, so 3 CTAs leave 170 registers a thread).
-    static constexpr int kMinBlocks = kInt8 ? 5 : ((kUseMma || G <= 4) ? 3 : 2);
+    static constexpr int kMinBlocks = kInt8 ? (G >= 4 ? 4 : 5) : ((kUseMma || G <= 4) ? 3 : 2);
 
     static_assert(kStages == kBufPerWarp * kWarps, "stage k: warp k % 4, buffer k % kStages");
     static_assert(BS % kTS == 0, "block size is a multiple of the stage");
