@@ -86,12 +86,18 @@ struct DecodeShape {
     static constexpr int kAgStride = kUseMma ? D + 1 : D;  // floats per merged accumulator row
     static constexpr int kMergeBytes = kRowGroups * G * (kAgStride + 2) * 4;
     static constexpr int kDataBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
-    // ring (or merge area), full barriers, per-buffer "skipped" flags, and
-    // the test hook (the withheld stage and the wait bound, 16 bytes)
-    static constexpr int kSmemBytes = kAlign + kDataBytes + kStages * 8 + kStages * 4 + 16;
+    // int8 groups of two or more heads keep the query's fixed-point MMA
+    // fragments (2 D/64 16-byte words per lane) in shared memory and read
+    // them once per stage: every O column is live there, and the registers
+    // this frees let five CTAs share an SM without spilling.
+    static constexpr bool kQShared = kInt8 && G >= 2;
+    static constexpr int kQBytes = kQShared ? 2 * (D / 64) * 32 * 16 : 0;
+    // ring (or merge area), full barriers, per-buffer "skipped" flags, the
+    // test hook and head range (32 bytes) and the shared query fragments
+    static constexpr int kSmemBytes = kAlign + kDataBytes + kStages * 8 + kStages * 4 + 32 + kQBytes;
     // Resident CTAs per SM the register budget is set for (a sub-partition
     // holds one warp of each CTA, so 3 CTAs leave 170 registers a thread).
-    static constexpr int kMinBlocks = kInt8 ? (G >= 4 ? 4 : 5) : ((kUseMma || G <= 4) ? 3 : 2);
+    static constexpr int kMinBlocks = kInt8 ? 5 : ((kUseMma || G <= 4) ? 3 : 2);
 
     static_assert(kStages == kBufPerWarp * kWarps, "stage k: warp k % 4, buffer k % kStages");
     static_assert(BS % kTS == 0, "block size is a multiple of the stage");
@@ -100,6 +106,7 @@ struct DecodeShape {
     static_assert(kUseMma || (kTS % kRows == 0 && kTpg % kTc == 0), "stage split");
     static_assert(kUseMma || G <= kLpt, "a lane's kept scores must belong to one query head");
     static_assert(kUseMma || kNvl <= kTc, "kept scores within one head");
+    static_assert(kDataBytes % 16 == 0, "barriers, flags, hook and query fragments stay 16-byte aligned");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -538,8 +545,12 @@ struct MmaConsumerQ8 {
     static constexpr int kJ = D / 64;    // 16-byte K chunks per lane per row
     static constexpr int kMT = D / 16;   // PV m-tiles
     static constexpr int kW = D / 8;     // V dims per lane
+    static constexpr bool kQShared = S::kQShared;
     int q4, r;
-    uint32_t qhi[kJ][4], qlo[kJ][4];     // query as 16-bit fixed point: signed high bytes, unsigned low bytes
+    // query as 16-bit fixed point: signed high bytes, unsigned low bytes; in
+    // registers (kQShared false) or as words [2 j + 0/1][lane] of qsm
+    uint32_t qhi[kQShared ? 1 : kJ][4], qlo[kQShared ? 1 : kJ][4];
+    const uint4 *qsm;                    // this lane's word 0 of the shared fragments
     float qs[2];                         // fixed-point step of heads 2q, 2q + 1
     float o[kMT][4];
     float m_run[2], l_lane[2];
@@ -569,7 +580,10 @@ struct MmaConsumerQ8 {
     // signed, lo in [0, 255]): q . k = step (256 hi.k + lo.k), both products
     // exact in int32 on the int8 tensor cores. |q - step Q| <= step / 2, i.e.
     // 2^-16 of the head's largest component.
-    __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int g_valid, int, int lane) {
+    // qarea: the CTA's shared query fragments (kQShared), written by warp 0;
+    // every thread of the CTA calls init.
+    __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int g_valid, int warp, int lane,
+                                         uint4 *qarea) {
         q4 = lane & 3;
         r = lane >> 2;
         float f[kJ][16];
@@ -593,6 +607,7 @@ struct MmaConsumerQ8 {
         const float step = amax > 0.f ? __fdiv_rn(amax, 32767.f) : 0.f;
 #pragma unroll
         for (int j = 0; j < kJ; ++j) {
+            uint32_t hw[4], lw[4];
 #pragma unroll
             for (int w = 0; w < 4; ++w) {  // word w: dims 4w .. 4w + 3 of the chunk
                 uint32_t hi = 0, lo = 0;
@@ -602,10 +617,24 @@ struct MmaConsumerQ8 {
                     hi |= (uint32_t)((Q >> 8) & 0xff) << (8 * e);
                     lo |= (uint32_t)(Q & 0xff) << (8 * e);
                 }
-                qhi[j][w] = hi;
-                qlo[j][w] = lo;
+                hw[w] = hi;
+                lw[w] = lo;
+            }
+            if constexpr (kQShared) {
+                if (warp == 0) {
+                    qarea[(2 * j) * 32 + lane] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    qarea[(2 * j + 1) * 32 + lane] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+            } else {
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    qhi[j][w] = hw[w];
+                    qlo[j][w] = lw[w];
+                }
             }
         }
+        qsm = qarea + lane;
+        if constexpr (kQShared) __syncthreads();
         qs[0] = __shfl_sync(0xffffffffu, step, (2 * q4) * 4);
         qs[1] = __shfl_sync(0xffffffffu, step, (2 * q4 + 1) * 4);
 #pragma unroll
@@ -625,12 +654,24 @@ struct MmaConsumerQ8 {
         for (int j = 0; j < kJ; ++j) {
             const uint4 u0 = *reinterpret_cast<const uint4 *>(Kb + r * D + 16 * (q4 + 4 * j));
             const uint4 u1 = *reinterpret_cast<const uint4 *>(Kb + (r + 8) * D + 16 * (q4 + 4 * j));
+            uint32_t bh[4], bl[4];
+            if constexpr (kQShared) {
+                const uint4 h = qsm[(2 * j) * 32], l = qsm[(2 * j + 1) * 32];
+                bh[0] = h.x; bh[1] = h.y; bh[2] = h.z; bh[3] = h.w;
+                bl[0] = l.x; bl[1] = l.y; bl[2] = l.z; bl[3] = l.w;
+            } else {
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    bh[w] = qhi[j][w];
+                    bl[w] = qlo[j][w];
+                }
+            }
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
                 const uint32_t a0 = word_of(u0, 2 * m), a2 = word_of(u0, 2 * m + 1);
                 const uint32_t a1 = word_of(u1, 2 * m), a3 = word_of(u1, 2 * m + 1);
-                mma_s8(chi, a0, a1, a2, a3, qhi[j][2 * m], qhi[j][2 * m + 1]);
-                mma_u8(clo, a0, a1, a2, a3, qlo[j][2 * m], qlo[j][2 * m + 1]);
+                mma_s8(chi, a0, a1, a2, a3, bh[2 * m], bh[2 * m + 1]);
+                mma_u8(clo, a0, a1, a2, a3, bl[2 * m], bl[2 * m + 1]);
             }
         }
         float sc[4];
@@ -789,7 +830,9 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     uint64_t *full = reinterpret_cast<uint64_t *>(ring + S::kDataBytes);
     int *bad = reinterpret_cast<int *>(full + S::kStages);
     // test hook, staged by thread 0 and read only where used: [0] this CTA's
-    // withheld stage (-1: none); [2..3] the wait bound in ns
+    // withheld stage (-1: none); [2..3] the wait bound in ns. [4..5] the
+    // CTA's first query head and [6] its head count, kept here across the
+    // stage loop instead of in registers.
     int *hook = bad + S::kStages;
     const uint64_t *wait_limit = reinterpret_cast<const uint64_t *>(hook + 2);
 
@@ -857,6 +900,8 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
         fence_mbar_init();
         hook[0] = (s == p.withhold_seq && kvh == p.withhold_kvh && part == 0) ? p.withhold_stage : -1;
         *reinterpret_cast<uint64_t *>(hook + 2) = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
+        *reinterpret_cast<uint64_t *>(hook + 4) = head0;
+        hook[6] = g_valid;
     }
     __syncthreads();
 
@@ -952,7 +997,11 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     }
 
     Consumer cons;
-    cons.init(p, head0, g_valid, warp, lane);
+    if constexpr (S::kInt8) {
+        cons.init(p, head0, g_valid, warp, lane, reinterpret_cast<uint4 *>(hook + 8));
+    } else {
+        cons.init(p, head0, g_valid, warp, lane);
+    }
     int waited = 0;
     bool ok = true;
     for (int m = 0; m < nmine; ++m) {
@@ -1025,7 +1074,11 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
     __syncthreads();
     cons.store(mg, lg, ag, warp, lane);
     __syncthreads();
-    for (int idx = threadIdx.x; idx < g_valid * D; idx += S::kThreads) {
+    // the head range, read back from shared memory (nothing keeps it live
+    // through the loop)
+    const size_t head_first = *reinterpret_cast<volatile uint64_t *>(hook + 4);
+    const int heads = *reinterpret_cast<volatile int *>(hook + 6);
+    for (int idx = threadIdx.x; idx < heads * D; idx += S::kThreads) {
         const int g = idx / D;
         const int d = idx % D;
         float Mx = -INFINITY;
@@ -1040,7 +1093,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
                 den = fmaf(w, lg[i * G + g], den);
             }
         }
-        const size_t h = head0 + g;
+        const size_t h = head_first + g;
         if (split) {
             const size_t slot = h * p.max_parts + part;
             p.ws_acc[slot * D + d] = num;
