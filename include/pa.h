@@ -270,17 +270,51 @@ int pa_decode_splitk_static(void *out, const void *query, const void *k_cache, c
  *   out[q_start[s] + i, h, :] = sum_{t <= pos} softmax_t(scale q . K_t) V_t.
  * q_len_s = 1 is decode. max_q_len bounds every q_len_s. Requires
  * q_len_s <= context_lens[s] (else PA_DEVERR_CONTEXT and that sequence is
- * skipped). head_dim 128, kv_dtype PA_F16 or PA_BF16, out_dtype kv_dtype or
- * PA_F32. ([P4] §3.4: the forward pass over the step's new tokens, each
- * layer attending over the paged cache; [P3] §3.1: the num_tokens axis of
- * queries.) QK^T and PV run as tcgen05 MMAs with accumulators in tensor
- * memory; K/V tiles are gathered through the table by TMA.
+ * skipped). head_dim 64 or 128, block_size 16 or 32, any head group
+ * (num_heads a multiple of num_kv_heads). kv_dtype PA_F16 or PA_BF16
+ * (out_dtype kv_dtype or PA_F32): QK^T and PV run as tcgen05 MMAs with
+ * accumulators in tensor memory, K/V tiles gathered through the table by
+ * TMA. kv_dtype PA_F32 (out_dtype PA_F32): exact fp32 arithmetic on the CUDA
+ * cores, each query token a decode over its causal prefix (the tensor cores
+ * take fp32 only as tf32). ([P4] §3.4: the forward pass over the step's new
+ * tokens, each layer attending over the paged cache; [P3] §3.1: the
+ * num_tokens axis of queries.)
  */
 int pa_prefill(void *out, const void *query, const int32_t *q_start, int num_tokens, int max_q_len,
                const void *k_cache, const void *v_cache, const int32_t *block_tables,
                int max_blocks_per_seq, const int32_t *context_lens, int num_seqs, int num_heads,
                int num_kv_heads, int head_dim, float scale, int block_size, int num_blocks,
                pa_dtype kv_dtype, pa_dtype out_dtype, cudaStream_t stream);
+
+/*
+ * pa_prefill_withhold_tile -- pa_prefill (16-bit caches, the tensor-core
+ * kernel) with a fault planted on the host, for testing the bounded waits;
+ * not for production use. The CTA of sequence `seq`, kv head `kv_head` and
+ * query tile `query_tile` (its 128 rows of (token, query head) pairs: tokens
+ * query_tile * 128 / G' .. of the sequence's new tokens, G' the head group
+ * rounded up to a power of two; a group above 128 withholds in its first
+ * sub-group only) never issues the copy of its 64-token K tile `tile`
+ * (cache tokens 64 * tile ..), so the MMA thread that needs it waits for data
+ * that never comes. After wait_limit_ns (between 1e5 and 1e9; the library's
+ * own bound is 1 s) it records PA_DEVERR_TIMEOUT and releases the CTA's other
+ * warps, which leave their loops; the load warp waits, with the same bound,
+ * for the copies it still has in flight; every product issued finishes
+ * before tensor memory is freed, and the launch ends normally. That CTA's
+ * output rows are undefined, every other output is pa_prefill's. A tile or
+ * query tile past the CTA's work withholds nothing. Other arguments as
+ * pa_prefill; PA_F32 caches give PA_ERR_DTYPE, head_dim other than 128
+ * PA_ERR_HEAD_DIM (the hook is compiled into separate head_dim-128 instances
+ * of the kernel, so pa_prefill's own carry none of it), and seq or kv_head
+ * out of range, query_tile or tile < 0, or the limit out of range
+ * PA_ERR_SHAPE.
+ */
+int pa_prefill_withhold_tile(void *out, const void *query, const int32_t *q_start, int num_tokens,
+                             int max_q_len, const void *k_cache, const void *v_cache,
+                             const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                             int num_seqs, int num_heads, int num_kv_heads, int head_dim, float scale,
+                             int block_size, int num_blocks, pa_dtype kv_dtype, pa_dtype out_dtype, int seq,
+                             int kv_head, int query_tile, int tile, unsigned long long wait_limit_ns,
+                             cudaStream_t stream);
 
 /*
  * Partition size this library would pick for a batch: 0 when the

@@ -58,6 +58,7 @@ EXPORTED = (
     "pa_prefix_release", "pa_prefix_ref_count", "pa_copy_blocks_counted", "pa_dpool_state_bytes", "pa_dpool_init",
     "pa_beam_step", "pa_pool_export", "pa_dpool_load", "pa_reshape_and_cache_q8", "pa_decode_q8",
     "pa_decode_splitk_q8", "pa_copy_blocks_q8", "pa_decode_append", "pa_decode_withhold_stage",
+    "pa_prefill_withhold_tile",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -104,6 +105,8 @@ def _load() -> ctypes.CDLL:
         "pa_pool_release": (i32, [vp, i32p, i32]),
         "pa_decode_splitk_static": (i32, [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32,
                                           i32, i32, vp]),
+        "pa_prefill_withhold_tile": (i32, [vp, vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32,
+                                           i32, i32, i32, i32, i32, i32, ctypes.c_ulonglong, vp]),
         "pa_prefill": (i32, [vp, vp, vp, i32, i32, vp, vp, vp, i32, vp, i32, i32, i32, i32, f32, i32, i32, i32, i32,
                              vp]),
         "pa_prefix_cache_create": (vp, [vp, i32]),
@@ -323,6 +326,21 @@ def pa_prefill(out, query, q_start, max_q_len, k_cache, v_cache, block_tables, c
                          _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S, Hq, Hkv, D, float(scale),
                          bs, NB, _dtype(k_cache), _dtype(out), _stream(stream))
     _check(rc, "pa_prefill")
+
+
+def pa_prefill_withhold_tile(out, query, q_start, max_q_len, k_cache, v_cache, block_tables, context_lens, scale,
+                             seq, kv_head, query_tile, tile, wait_limit_ns, stream=None) -> None:
+    """pa_prefill with the copy of one 64-token K tile of one (sequence, kv
+    head, query tile) withheld, so that its bounded wait runs out (a test of
+    the timeout path; that CTA's output rows are undefined)."""
+    T, Hq, D = query.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    S = context_lens.shape[0]
+    rc = _lib.pa_prefill_withhold_tile(_ptr(out), _ptr(query), _ptr(q_start), T, int(max_q_len), _ptr(k_cache),
+                                       _ptr(v_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S,
+                                       Hq, Hkv, D, float(scale), bs, NB, _dtype(k_cache), _dtype(out), int(seq),
+                                       int(kv_head), int(query_tile), int(tile), int(wait_limit_ns), _stream(stream))
+    _check(rc, "pa_prefill_withhold_tile")
 
 
 def pa_choose_partition(num_seqs, num_kv_heads, max_context_len, block_size, head_dim, kv_dtype) -> int:

@@ -100,6 +100,11 @@ struct Params {
     float scale_log2;
     pa_dtype out_dtype;
     unsigned int *err;
+    // test hook (pa_prefill_withhold_tile): the CTA of (sequence, kv head,
+    // query tile) never issues the copy of its K tile withhold_tile (-1:
+    // none), and every wait gives up after wait_limit_ns (0: kWaitLimitNs)
+    int withhold_seq = -1, withhold_kvh = -1, withhold_qt = -1, withhold_tile = -1;
+    unsigned long long wait_limit_ns = 0;
 };
 
 // ---------------------------------------------------------------- helpers
@@ -237,7 +242,7 @@ __device__ __forceinline__ bool softmax_sync_and(bool v) {
 // 4 or 8 (no padding, no sub-groups; compiled for that size), or -1 for any
 // other group (slots and sub-groups from Params). Groups of 1-2 stage their
 // output rows in shared memory; larger ones store one row per thread.
-template <typename T, int kD, int kGS>
+template <typename T, int kD, int kGS, bool kHook = false>
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const Params p) {
@@ -275,6 +280,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t *mma_idle = bars + 14; // every MMA issued has finished (end of kernel)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 15);
     int *abort_flag = reinterpret_cast<int *>(bars + 16);
+    // test hook (kHook instances only): the wait bound and this CTA's
+    // withheld K tile, set with the barriers; other instances wait with the
+    // library's bound and withhold nothing
+    uint64_t *const wl = kHook ? bars + 17 : nullptr;
+    int *const withheld = reinterpret_cast<int *>(bars + 18);
 
     const int qt = gridDim.x - 1 - blockIdx.x;  // longest query tile of each (head, sequence) first
     const int kvh = (!kExact && p.sub_groups > 1) ? (int)blockIdx.y / p.sub_groups : (int)blockIdx.y;
@@ -338,6 +348,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_init(o_done, 1);
             mbar_init(mma_idle, 1);
             *abort_flag = 0;
+            if constexpr (kHook) {
+                *wl = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
+                *withheld = (s == p.withhold_seq && kvh == p.withhold_kvh && sub == 0 && qt == p.withhold_qt)
+                                ? p.withhold_tile : -1;
+            }
             fence_mbar_init();
             fence_proxy_async_smem();  // the initialised barriers, before the copy that signals one
             mbar_arrive_expect_tx(q_full, kQBytes);
@@ -379,13 +394,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int kv = 0; kv < 2; ++kv) {
                 uint64_t *empty = (kv == 0 ? k_empty : v_empty) + b;
                 if (j >= 2) {  // every lane waits; the outcome is made warp-uniform
-                    const bool got = mbar_wait(empty, ((j >> 1) - 1) & 1) && !*(volatile int *)abort_flag;
+                    const bool got = mbar_wait(empty, ((j >> 1) - 1) & 1, wl) && !*(volatile int *)abort_flag;
                     if (!__all_sync(0xffffffffu, got)) {
                         ok = false;
                         break;
                     }
                 }
-                if (lane == 0) {
+                if (lane == 0 && !(kHook && kv == 0 && j == *withheld)) {  // (test hook: never issued)
                     uint64_t *full = (kv == 0 ? k_full : v_full) + b;
                     unsigned char *dst = (kv == 0 ? Ks : Vs) + b * kKVBytes;
                     const CUtensorMap *map = kv == 0 ? &tmap_k : &tmap_v;
@@ -408,9 +423,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         // let the copies this warp started land before the CTA leaves
         // (normally the MMA warp has consumed them all: these waits return at once)
         if (lane == 0) {
-            mbar_wait(q_full, 0);
-            for (int j = max(0, k_issued - 2); j < k_issued; ++j) mbar_wait(k_full + (j & 1), (j >> 1) & 1);
-            for (int j = max(0, v_issued - 2); j < v_issued; ++j) mbar_wait(v_full + (j & 1), (j >> 1) & 1);
+            mbar_wait(q_full, 0, wl);
+            for (int j = max(0, k_issued - 2); j < k_issued; ++j) mbar_wait(k_full + (j & 1), (j >> 1) & 1, wl);
+            for (int j = max(0, v_issued - 2); j < v_issued; ++j) mbar_wait(v_full + (j & 1), (j >> 1) & 1, wl);
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -419,11 +434,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         // product done, so P_j's buffer is free) S_{j+2} into the same buffer.
         if (lane == 0) {
             const uint32_t qa = smem_addr(Qs);
-            bool ok = mbar_wait(q_full, 0);
+            bool ok = mbar_wait(q_full, 0, wl);
             bool issued = false;
             auto issue_s = [&](int j) -> bool {
                 const int b = j & 1;
-                if (!mbar_wait(k_full + b, (j >> 1) & 1) || *(volatile int *)abort_flag) return false;
+                if (!mbar_wait(k_full + b, (j >> 1) & 1, wl) || *(volatile int *)abort_flag) return false;
                 tc_fence_after();
                 const uint32_t ka = smem_addr(Ks + b * kKVBytes);
 #pragma unroll
@@ -440,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int j = 0; ok && j < min(2, ntiles); ++j) ok = issue_s(j);
             for (int j = 0; ok && j < ntiles; ++j) {
                 const int b = j & 1;
-                if (!mbar_wait(p_full + b, (j >> 1) & 1) || !mbar_wait(v_full + b, (j >> 1) & 1) ||
+                if (!mbar_wait(p_full + b, (j >> 1) & 1, wl) || !mbar_wait(v_full + b, (j >> 1) & 1, wl) ||
                     *(volatile int *)abort_flag) {
                     ok = false;
                     break;
@@ -457,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 umma_commit(o_done);
                 umma_commit(v_empty + b);
                 if (j + 2 < ntiles) {
-                    if (!mbar_wait(o_done, j & 1)) { ok = false; break; }
+                    if (!mbar_wait(o_done, j & 1, wl)) { ok = false; break; }
                     ok = issue_s(j + 2);
                 }
             }
@@ -472,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             // must have finished (with none issued, release the waiters at once)
             if (issued) {
                 umma_commit(mma_idle);
-                if (!mbar_wait(mma_idle, 0)) record_error(p.err, PA_DEVERR_TIMEOUT);
+                if (!mbar_wait(mma_idle, 0, wl)) record_error(p.err, PA_DEVERR_TIMEOUT);
             } else {
                 mbar_arrive(mma_idle);
             }
@@ -489,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         float m_run = -INFINITY, l_run = 0.f;
         for (int j = 0; j < ntiles; ++j) {
             const int b = j & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(s_full + b, (j >> 1) & 1) && !*(volatile int *)abort_flag))
+            if (!__all_sync(0xffffffffu, mbar_wait(s_full + b, (j >> 1) & 1, wl) && !*(volatile int *)abort_flag))
                 break;
             tc_fence_after();
             const uint32_t sbuf = tmem + lane_base + kSCol + b * kN;
@@ -549,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                 // O is rescaled: O += P_{j-1} V_{j-1} must be done. (O += P_{j-2} V_{j-2}
                 // is: S_j was issued after it, so this parity wait cannot alias.)
-                const bool got = mbar_wait(o_done, (j - 1) & 1) && !*(volatile int *)abort_flag;
+                const bool got = mbar_wait(o_done, (j - 1) & 1, wl) && !*(volatile int *)abort_flag;
                 if (!__all_sync(0xffffffffu, got)) break;
                 tc_fence_after();
 #pragma unroll
@@ -569,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int zrow = max(0, ctx - kv0);
             if (zrow < kN) {
                 // V_j must have landed before its tail rows are overwritten
-                if (!__all_sync(0xffffffffu, mbar_wait(v_full + b, (j >> 1) & 1) && !*(volatile int *)abort_flag))
+                if (!__all_sync(0xffffffffu, mbar_wait(v_full + b, (j >> 1) & 1, wl) && !*(volatile int *)abort_flag))
                     break;
                 unsigned char *vt = Vs + b * kKVBytes;
                 const int nvec = (kN - zrow) * kHalves * (kHalfBytes / 16);
@@ -587,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         // ---- output: O / l for valid rows
         // every product done (the MMA warp's single-use end-of-kernel commit)
-        const bool done = __all_sync(0xffffffffu, mbar_wait(mma_idle, 0) && !*(volatile int *)abort_flag);
+        const bool done = __all_sync(0xffffffffu, mbar_wait(mma_idle, 0, wl) && !*(volatile int *)abort_flag);
         tc_fence_after();
         // Each thread holds O of its row in tensor-memory lane r. For G <= 2 it
         // writes O / l in the output type into shared memory (the Q, K and V
@@ -698,10 +713,10 @@ static bool make_map(CUtensorMap *map, bool bf16, void *base, int rank, const cu
     return r == CUDA_SUCCESS;
 }
 
-template <typename T, int D, int kGS>
+template <typename T, int D, int kGS, bool kHook>
 static cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const Params &p,
                             int q_tiles, int num_kv_heads, int num_seqs, cudaStream_t stream) {
-    auto kern = prefill_kernel<T, D, kGS>;
+    auto kern = prefill_kernel<T, D, kGS, kHook>;
     static AttrCache attr_done;
     constexpr int kSmem = Layout<D>::kSmemBytes;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(kern), kSmem, &attr_done);
@@ -713,12 +728,15 @@ static cudaError_t launch_t(const CUtensorMap &mq, const CUtensorMap &mk, const 
 }  // namespace prefill
 }  // namespace pa
 
-extern "C" int pa_prefill(void *out, const void *query, const int32_t *q_start, int num_tokens,
-                          int max_q_len, const void *k_cache, const void *v_cache,
-                          const int32_t *block_tables, int max_blocks_per_seq,
-                          const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads,
-                          int head_dim, float scale, int block_size, int num_blocks, pa_dtype kv_dtype,
-                          pa_dtype out_dtype, cudaStream_t stream) {
+namespace {
+
+// pa_prefill, with the test hook's fields of Params (hook.withhold_* -1 and
+// hook.wait_limit_ns 0 for a normal call).
+int prefill_call(void *out, const void *query, const int32_t *q_start, int num_tokens, int max_q_len,
+                 const void *k_cache, const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                 const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                 float scale, int block_size, int num_blocks, pa_dtype kv_dtype, pa_dtype out_dtype,
+                 const pa::prefill::Params &hook, cudaStream_t stream) {
     using namespace pa::prefill;
     if (num_seqs < 0 || num_tokens < 0 || max_q_len < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
         num_blocks < 0 || max_blocks_per_seq < 0 || num_seqs > 65535 || num_kv_heads > 65535)
@@ -766,7 +784,7 @@ extern "C" int pa_prefill(void *out, const void *query, const int32_t *q_start, 
     }
     unsigned int *err = nullptr;
     if (pa::device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
-    Params p{};
+    Params p = hook;
     p.out = out;
     p.q_start = q_start;
     p.block_tables = block_tables;
@@ -785,19 +803,68 @@ extern "C" int pa_prefill(void *out, const void *query, const int32_t *q_start, 
     p.sub_groups = sub_groups;
     const int q_tiles = (max_q_len * gslots + kM - 1) / kM;
     cudaError_t e = cudaErrorInvalidValue;
-#define PA_PREFILL_GS(T, DD, GS) launch_t<T, DD, GS>(mq, mk, mv, p, q_tiles, num_kv_heads, num_seqs, stream)
-#define PA_PREFILL_CASE(T, DD)                                                                  \
-    e = group == 1 ? PA_PREFILL_GS(T, DD, 0) : group == 2 ? PA_PREFILL_GS(T, DD, 1)             \
-      : group == 4 ? PA_PREFILL_GS(T, DD, 2) : group == 8 ? PA_PREFILL_GS(T, DD, 3)             \
-                   : PA_PREFILL_GS(T, DD, -1)
+    // the test hook's instances (head_dim 128 only) are separate, so the
+    // production instances carry none of it
+    const bool with_hook = p.withhold_seq >= 0;
+#define PA_PREFILL_GS(T, DD, GS, H) launch_t<T, DD, GS, H>(mq, mk, mv, p, q_tiles, num_kv_heads, num_seqs, stream)
+#define PA_PREFILL_CASE(T, DD, H)                                                               \
+    e = group == 1 ? PA_PREFILL_GS(T, DD, 0, H) : group == 2 ? PA_PREFILL_GS(T, DD, 1, H)       \
+      : group == 4 ? PA_PREFILL_GS(T, DD, 2, H) : group == 8 ? PA_PREFILL_GS(T, DD, 3, H)       \
+                   : PA_PREFILL_GS(T, DD, -1, H)
     if (bf16) {
-        if (head_dim == 128) PA_PREFILL_CASE(__nv_bfloat16, 128);
-        else PA_PREFILL_CASE(__nv_bfloat16, 64);
+        if (head_dim == 128) {
+            if (with_hook) PA_PREFILL_CASE(__nv_bfloat16, 128, true);
+            else PA_PREFILL_CASE(__nv_bfloat16, 128, false);
+        } else {
+            PA_PREFILL_CASE(__nv_bfloat16, 64, false);
+        }
     } else {
-        if (head_dim == 128) PA_PREFILL_CASE(__half, 128);
-        else PA_PREFILL_CASE(__half, 64);
+        if (head_dim == 128) {
+            if (with_hook) PA_PREFILL_CASE(__half, 128, true);
+            else PA_PREFILL_CASE(__half, 128, false);
+        } else {
+            PA_PREFILL_CASE(__half, 64, false);
+        }
     }
 #undef PA_PREFILL_CASE
 #undef PA_PREFILL_GS
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int pa_prefill(void *out, const void *query, const int32_t *q_start, int num_tokens,
+                          int max_q_len, const void *k_cache, const void *v_cache,
+                          const int32_t *block_tables, int max_blocks_per_seq,
+                          const int32_t *context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                          int head_dim, float scale, int block_size, int num_blocks, pa_dtype kv_dtype,
+                          pa_dtype out_dtype, cudaStream_t stream) {
+    const pa::prefill::Params hook{};
+    return prefill_call(out, query, q_start, num_tokens, max_q_len, k_cache, v_cache, block_tables,
+                        max_blocks_per_seq, context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale,
+                        block_size, num_blocks, kv_dtype, out_dtype, hook, stream);
+}
+
+extern "C" int pa_prefill_withhold_tile(void *out, const void *query, const int32_t *q_start, int num_tokens,
+                                        int max_q_len, const void *k_cache, const void *v_cache,
+                                        const int32_t *block_tables, int max_blocks_per_seq,
+                                        const int32_t *context_lens, int num_seqs, int num_heads,
+                                        int num_kv_heads, int head_dim, float scale, int block_size,
+                                        int num_blocks, pa_dtype kv_dtype, pa_dtype out_dtype, int seq,
+                                        int kv_head, int query_tile, int tile, unsigned long long wait_limit_ns,
+                                        cudaStream_t stream) {
+    if (kv_dtype != PA_F16 && kv_dtype != PA_BF16) return PA_ERR_DTYPE;  // the tensor-core kernel only
+    if (head_dim != 128) return PA_ERR_HEAD_DIM;                          // its hook instances
+    if (seq < 0 || seq >= num_seqs || kv_head < 0 || kv_head >= num_kv_heads || query_tile < 0 || tile < 0 ||
+        wait_limit_ns < 100000ull || wait_limit_ns > 1000000000ull)
+        return PA_ERR_SHAPE;
+    pa::prefill::Params hook{};
+    hook.withhold_seq = seq;
+    hook.withhold_kvh = kv_head;
+    hook.withhold_qt = query_tile;
+    hook.withhold_tile = tile;
+    hook.wait_limit_ns = wait_limit_ns;
+    return prefill_call(out, query, q_start, num_tokens, max_q_len, k_cache, v_cache, block_tables,
+                        max_blocks_per_seq, context_lens, num_seqs, num_heads, num_kv_heads, head_dim, scale,
+                        block_size, num_blocks, kv_dtype, out_dtype, hook, stream);
 }

@@ -1,13 +1,14 @@
 """The bounded pipeline waits on the GPU. A copy that never lands must not
 hang the GPU: the waiting warp gives up after its bound, records
 PA_DEVERR_TIMEOUT, waits (again bounded) for the copies it still has in flight
-and leaves, and the launch ends. pa_decode_withhold_stage plants that fault
-from the host (one stage's copy is never issued) with a bound of a few
-milliseconds, so the test makes the wait run out and checks what the host
-reads back; nothing faults or traps.
+and leaves, and the launch ends. pa_decode_withhold_stage (decode: one 16-token
+stage) and pa_prefill_withhold_tile (prefill: one 64-token K tile) plant that
+fault from the host, with a bound of a few milliseconds, so the test makes the
+wait run out and checks what the host reads back; nothing faults or traps.
 
-After such a launch, every (sequence, kv head) other than the one with the
-withheld stage still matches the oracle, and the next normal call is clean."""
+After such a launch, every other (sequence, kv head) of a decode, and every
+other CTA's rows of a prefill, still match the oracle, and the next normal
+call is clean."""
 import math
 import time
 
@@ -95,3 +96,109 @@ def test_hook_arguments_are_checked(pa):
         with pytest.raises(pa.PagedAttentionError) as e:
             pa.pa_decode_withhold_stage(out, p["q"], p["k"], p["v"], p["bt"], p["cl"], 0.1, seq, kvh, stage, lim)
         assert e.value.status == -3
+
+
+# ---- prefill (the tcgen05 kernel): a withheld K tile
+
+def _prefill_problem(dtype, ctx, qlen, Hq, Hkv, BS, seed, D=128):
+    g = torch.Generator().manual_seed(seed)
+    S = len(ctx)
+    nb = [oracle.blocks_needed(int(c), BS) for c in ctx]
+    NB = sum(nb) + 3
+    ids = torch.randperm(NB, generator=g).numpy().astype(np.int32)
+    tables = np.full((S, max(nb)), -1, np.int32)
+    pos = 0
+    for s, n in enumerate(nb):
+        tables[s, :n] = ids[pos:pos + n]
+        pos += n
+    k = torch.randn((NB, Hkv, BS, D), generator=g).to(dtype)
+    v = torch.randn((NB, Hkv, BS, D), generator=g).to(dtype)
+    qs = np.concatenate([[0], np.cumsum(qlen)]).astype(np.int32)
+    q = torch.randn((int(qs[-1]), Hq, D), generator=g).to(dtype)
+    ctx = np.array(ctx, np.int32)
+    scale = 1.0 / math.sqrt(D)
+    ref = oracle.paged_prefill(f64(q), qs, f64(k), f64(v), tables, ctx, scale, BS)
+    dev = dict(q=q.cuda(), k=k.cuda(), v=v.cuda(), qs=torch.from_numpy(qs).cuda(), bt=torch.from_numpy(tables).cuda(),
+               cl=torch.from_numpy(ctx).cuda(), max_q=int(max(qlen)), scale=scale, qs_host=qs)
+    return dev, ref
+
+
+def _cta_rows(qs, seq, kvh, qt, Hq, Hkv):
+    """(token rows, heads) of the prefill CTA (sequence, kv head, query tile):
+    128 (token, head slot) rows, the head group rounded up to a power of two."""
+    G = Hq // Hkv
+    slots = 1 << (G - 1).bit_length()
+    tok_per_tile = 128 // slots
+    t0 = int(qs[seq]) + qt * tok_per_tile
+    t1 = min(int(qs[seq + 1]), t0 + tok_per_tile)
+    return slice(t0, t1), slice(kvh * G, (kvh + 1) * G)
+
+
+# query tile qt of sequence 0 (300 new tokens from an empty cache) sees four
+# 64-key tiles: tokens 128..255 at head group 1, tokens 192..223 at group 4
+@pytest.mark.parametrize("dtype,Hq,Hkv,BS,qt", [(torch.bfloat16, 4, 4, 16, 1),   # group 1: rows staged in shared memory
+                                                (torch.float16, 16, 4, 32, 6)])  # group 4: rows stored directly
+def test_prefill_withheld_tile_times_out_and_reports(pa, dtype, Hq, Hkv, BS, qt):
+    ctx, qlen = [300, 200, 90], [300, 64, 90]
+    p, ref = _prefill_problem(dtype, ctx, qlen, Hq, Hkv, BS, seed=11)
+    T = int(p["qs_host"][-1])
+    assert pa.pa_read_device_errors() == 0
+    seq, kvh = 0, Hkv - 1
+    for tile in (0, 3):  # a tile of the prologue (S_0), and one loaded in the loop
+        out = torch.full((T, Hq, 128), float("nan"), dtype=torch.float32, device="cuda")
+        t = time.perf_counter()
+        pa.pa_prefill_withhold_tile(out, p["q"], p["qs"], p["max_q"], p["k"], p["v"], p["bt"], p["cl"], p["scale"],
+                                    seq, kvh, qt, tile, LIMIT_NS)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t
+        assert pa.pa_read_device_errors() == pa.PA_DEVERR_TIMEOUT
+        assert wall < 2.0  # a few bounded waits of 5 ms, not the default 1 s bound, and never a hang
+        rows, heads = _cta_rows(p["qs_host"], seq, kvh, qt, Hq, Hkv)
+        mask = np.ones((T, Hq), bool)
+        mask[rows, heads] = False
+        o = out.cpu().numpy()
+        assert_attention_close(torch.from_numpy(o[mask]), ref[mask], dtype, f"tile {tile}")
+    # the next normal call: clean and correct
+    out = torch.empty((T, Hq, 128), dtype=torch.float32, device="cuda")
+    pa.pa_prefill(out, p["q"], p["qs"], p["max_q"], p["k"], p["v"], p["bt"], p["cl"], p["scale"])
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_errors() == 0
+    assert_attention_close(out, ref, dtype, "prefill after the timeouts")
+
+
+def test_prefill_tile_past_the_work_withholds_nothing(pa):
+    p, _ = _prefill_problem(torch.bfloat16, [300, 64], [300, 64], 8, 4, 16, seed=12)
+    T = int(p["qs_host"][-1])
+    out = torch.empty((T, 8, 128), dtype=torch.float32, device="cuda")
+    out2 = torch.empty_like(out)
+    # sequence 1's single query tile covers 64 keys: its tile 1 and a query tile 3 do not exist
+    for seq, qt, tile in ((1, 0, 1), (1, 3, 0)):
+        pa.pa_prefill_withhold_tile(out, p["q"], p["qs"], p["max_q"], p["k"], p["v"], p["bt"], p["cl"], p["scale"],
+                                    seq, 0, qt, tile, LIMIT_NS)
+        pa.pa_prefill(out2, p["q"], p["qs"], p["max_q"], p["k"], p["v"], p["bt"], p["cl"], p["scale"])
+        torch.cuda.synchronize()
+        assert pa.pa_read_device_errors() == 0
+        assert torch.equal(out, out2)
+
+
+def test_prefill_hook_arguments_are_checked(pa):
+    p, _ = _prefill_problem(torch.float16, [40, 17], [40, 17], 4, 2, 16, seed=13)
+    out = torch.empty((57, 4, 128), dtype=torch.float32, device="cuda")
+    for seq, kvh, qt, tile, lim in ((2, 0, 0, 0, LIMIT_NS), (0, 2, 0, 0, LIMIT_NS), (0, 0, -1, 0, LIMIT_NS),
+                                    (0, 0, 0, -1, LIMIT_NS), (0, 0, 0, 0, 10), (0, 0, 0, 0, 2_000_000_000)):
+        with pytest.raises(pa.PagedAttentionError) as e:
+            pa.pa_prefill_withhold_tile(out, p["q"], p["qs"], p["max_q"], p["k"], p["v"], p["bt"], p["cl"],
+                                        p["scale"], seq, kvh, qt, tile, lim)
+        assert e.value.status == -3
+    k32, v32 = p["k"].float(), p["v"].float()
+    q32 = p["q"].float()
+    with pytest.raises(pa.PagedAttentionError) as e:  # fp32 caches run on the CUDA cores: no hook there
+        pa.pa_prefill_withhold_tile(out, q32, p["qs"], p["max_q"], k32, v32, p["bt"], p["cl"], p["scale"],
+                                    0, 0, 0, 0, LIMIT_NS)
+    assert e.value.status == -2
+    p64, _ = _prefill_problem(torch.float16, [40, 17], [40, 17], 4, 2, 16, seed=14, D=64)
+    out64 = torch.empty((57, 4, 64), dtype=torch.float32, device="cuda")
+    with pytest.raises(pa.PagedAttentionError) as e:  # the hook's instances are head_dim 128 only
+        pa.pa_prefill_withhold_tile(out64, p64["q"], p64["qs"], p64["max_q"], p64["k"], p64["v"], p64["bt"], p64["cl"],
+                                    p64["scale"], 0, 0, 0, 0, LIMIT_NS)
+    assert e.value.status == -5
