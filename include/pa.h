@@ -561,6 +561,27 @@ int pa_beam_step(void *state, int num_blocks, int block_size, const int32_t *old
                  int32_t *new_tables, int32_t *new_context_lens, int max_blocks_per_seq,
                  int32_t *slot_mapping, int64_t *cow_pairs, int32_t *num_cow, cudaStream_t stream);
 
+/*
+ * pa_beam_step_withhold_arrival -- pa_beam_step (its one-launch form) with a
+ * fault planted on the host, for testing the bounded grid barrier; not for
+ * production use. CTA `cta` of the cooperative launch (CTA c takes old-table
+ * entries c * chunk ..) never counts itself at the first grid barrier, so
+ * every CTA's wait there runs out after wait_limit_ns (between 1e5 and 1e9;
+ * the library's own bound is 200 ms). The step then applies nothing, sets
+ * PA_DEVERR_TIMEOUT, every slot is -1 and *num_cow = 0, and the state is
+ * marked unusable (header word 5 cleared): later steps on it report
+ * PA_DEVERR_POOL until pa_dpool_init or pa_dpool_load. A CTA index past the
+ * launch withholds nothing. The hook is compiled into a separate instance of
+ * the kernel, so pa_beam_step's own carries none of it. Other arguments as
+ * pa_beam_step; a step too large for the one-launch form, cta < 0 or the
+ * limit out of range give PA_ERR_SHAPE.
+ */
+int pa_beam_step_withhold_arrival(void *state, int num_blocks, int block_size, const int32_t *old_tables,
+                                  const int32_t *old_context_lens, int num_old, const int32_t *parents, int num_new,
+                                  int32_t *new_tables, int32_t *new_context_lens, int max_blocks_per_seq,
+                                  int32_t *slot_mapping, int64_t *cow_pairs, int32_t *num_cow, int cta,
+                                  unsigned long long wait_limit_ns, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -58,7 +58,7 @@ EXPORTED = (
     "pa_prefix_release", "pa_prefix_ref_count", "pa_copy_blocks_counted", "pa_dpool_state_bytes", "pa_dpool_init",
     "pa_beam_step", "pa_pool_export", "pa_dpool_load", "pa_reshape_and_cache_q8", "pa_decode_q8",
     "pa_decode_splitk_q8", "pa_copy_blocks_q8", "pa_decode_append", "pa_decode_withhold_stage",
-    "pa_prefill_withhold_tile",
+    "pa_prefill_withhold_tile", "pa_beam_step_withhold_arrival",
 )
 
 PA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -120,6 +120,8 @@ def _load() -> ctypes.CDLL:
         "pa_dpool_state_bytes": (sz, [i32]),
         "pa_dpool_init": (i32, [vp, i32, i32, i32, vp, vp]),
         "pa_beam_step": (i32, [vp, i32, i32, vp, vp, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp]),
+        "pa_beam_step_withhold_arrival": (i32, [vp, i32, i32, vp, vp, i32, vp, i32, vp, vp, i32, vp, vp, vp, i32,
+                                                ctypes.c_ulonglong, vp]),
         "pa_pool_export": (i32, [vp, i32p, i32p, ctypes.POINTER(ctypes.c_int)]),
         "pa_dpool_load": (i32, [vp, i32, i32, i32, vp, vp, i32, vp]),
         "pa_reshape_and_cache_q8": (i32, [vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]),
@@ -421,6 +423,24 @@ def pa_beam_step(pool: DevicePool, old_tables, old_context_lens, parents, new_ta
                            _ptr(slot_mapping) if num_new else None, _ptr(cow_pairs) if num_new else None,
                            _ptr(num_cow), _stream(stream))
     _check(rc, "pa_beam_step")
+
+
+def pa_beam_step_withhold_arrival(pool: DevicePool, old_tables, old_context_lens, parents, new_tables,
+                                  new_context_lens, slot_mapping, cow_pairs, num_cow, cta, wait_limit_ns,
+                                  stream=None) -> None:
+    """pa_beam_step with one CTA's arrival at the first grid barrier withheld,
+    so that the barrier's bounded wait runs out (a test of the timeout path:
+    the step applies nothing and the state is marked unusable)."""
+    num_old = old_context_lens.shape[0]
+    num_new = parents.shape[0]
+    mb = new_tables.shape[1] if new_tables.dim() == 2 else old_tables.shape[1]
+    rc = _lib.pa_beam_step_withhold_arrival(
+        _ptr(pool.state), pool.num_blocks, pool.block_size, _ptr(old_tables) if num_old else None,
+        _ptr(old_context_lens) if num_old else None, num_old, _ptr(parents) if num_new else None, num_new,
+        _ptr(new_tables) if num_new else None, _ptr(new_context_lens) if num_new else None, mb,
+        _ptr(slot_mapping) if num_new else None, _ptr(cow_pairs) if num_new else None, _ptr(num_cow), int(cta),
+        int(wait_limit_ns), _stream(stream))
+    _check(rc, "pa_beam_step_withhold_arrival")
 
 
 def pa_read_device_errors(stream=None) -> int:

@@ -678,10 +678,16 @@ int pa_dpool_load(void *state, int num_blocks, int block_size, int policy, const
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-int pa_beam_step(void *state, int num_blocks, int block_size, const int32_t *old_tables,
-                 const int32_t *old_context_lens, int num_old, const int32_t *parents, int num_new,
-                 int32_t *new_tables, int32_t *new_context_lens, int max_blocks_per_seq,
-                 int32_t *slot_mapping, int64_t *cow_pairs, int32_t *num_cow, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// pa_beam_step, with the test hook's arguments (withhold_cta -1 for a normal call).
+int beam_step_call(void *state, int num_blocks, int block_size, const int32_t *old_tables,
+                   const int32_t *old_context_lens, int num_old, const int32_t *parents, int num_new,
+                   int32_t *new_tables, int32_t *new_context_lens, int max_blocks_per_seq, int32_t *slot_mapping,
+                   int64_t *cow_pairs, int32_t *num_cow, int withhold_cta, unsigned long long limit_ns,
+                   cudaStream_t stream) {
     if (num_blocks <= 0 || block_size <= 0 || num_old < 0 || num_new < 0 || max_blocks_per_seq <= 0)
         return PA_ERR_SHAPE;
     if (((long long)num_old + num_new) * max_blocks_per_seq >= (1LL << 30) ||
@@ -700,8 +706,36 @@ int pa_beam_step(void *state, int num_blocks, int block_size, const int32_t *old
     if (device_error_word(&err) != cudaSuccess) return PA_ERR_CUDA;
     cudaError_t e = launch_beam_step(static_cast<int32_t *>(state), old_tables, old_context_lens, num_old, parents,
                                      num_new, new_tables, new_context_lens, max_blocks_per_seq, slot_mapping,
-                                     cow_pairs, num_cow, num_blocks, block_size, err, stream);
+                                     cow_pairs, num_cow, num_blocks, block_size, err, stream, withhold_cta, limit_ns);
+    if (withhold_cta >= 0 && e == cudaErrorNotSupported) {  // no one-launch form for this step
+        (void)cudaGetLastError();
+        return PA_ERR_SHAPE;
+    }
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_beam_step(void *state, int num_blocks, int block_size, const int32_t *old_tables,
+                 const int32_t *old_context_lens, int num_old, const int32_t *parents, int num_new,
+                 int32_t *new_tables, int32_t *new_context_lens, int max_blocks_per_seq,
+                 int32_t *slot_mapping, int64_t *cow_pairs, int32_t *num_cow, cudaStream_t stream) {
+    return beam_step_call(state, num_blocks, block_size, old_tables, old_context_lens, num_old, parents, num_new,
+                          new_tables, new_context_lens, max_blocks_per_seq, slot_mapping, cow_pairs, num_cow, -1, 0,
+                          stream);
+}
+
+int pa_beam_step_withhold_arrival(void *state, int num_blocks, int block_size, const int32_t *old_tables,
+                                  const int32_t *old_context_lens, int num_old, const int32_t *parents, int num_new,
+                                  int32_t *new_tables, int32_t *new_context_lens, int max_blocks_per_seq,
+                                  int32_t *slot_mapping, int64_t *cow_pairs, int32_t *num_cow, int cta,
+                                  unsigned long long wait_limit_ns, cudaStream_t stream) {
+    if (cta < 0 || wait_limit_ns < 100000ull || wait_limit_ns > 1000000000ull) return PA_ERR_SHAPE;
+    return beam_step_call(state, num_blocks, block_size, old_tables, old_context_lens, num_old, parents, num_new,
+                          new_tables, new_context_lens, max_blocks_per_seq, slot_mapping, cow_pairs, num_cow, cta,
+                          wait_limit_ns, stream);
 }
 
 }  // extern "C"

@@ -185,6 +185,11 @@ struct StepParams {
     int chunk;       // old-table entries per CTA
     int num_chunks;  // CTAs of each launch
     unsigned int *err;
+    // test hook (pa_beam_step_withhold_arrival; the one-launch form's hook
+    // instance only): CTA withhold_cta never arrives at the first grid
+    // barrier, and barrier waits give up after barrier_limit_ns
+    int withhold_cta = -1;
+    unsigned long long barrier_limit_ns = 0;
 };
 
 // ------------------------------------------------------------------ beam step
@@ -632,11 +637,14 @@ __device__ __forceinline__ int ld_acquire(const int *a) {
 // Grid barrier: true once `target` arrivals are counted. A wait that gives
 // up (or sees that another CTA gave up) leaves the pool unusable: the step
 // stopped part way, and later steps refuse the state (PA_DEVERR_POOL).
-__device__ bool grid_barrier(const Pool &p, unsigned target, int epoch, unsigned int *err, int *s_go) {
+// limit_ns: the wait bound; arrive false (test hook only): this CTA does not
+// count itself.
+__device__ bool grid_barrier(const Pool &p, unsigned target, int epoch, unsigned int *err, int *s_go,
+                             uint64_t limit_ns = kBarrierLimitNs, bool arrive = true) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();  // this CTA's writes, before its arrival
-        atomicAdd(reinterpret_cast<unsigned *>(&p.tail[kBarArrive]), 1u);
+        if (arrive) atomicAdd(reinterpret_cast<unsigned *>(&p.tail[kBarArrive]), 1u);
         bool ok = true;
         uint64_t t0 = 0;
         for (uint32_t it = 0; (int)((unsigned)ld_acquire(&p.tail[kBarArrive]) - target) < 0; ++it) {
@@ -644,7 +652,7 @@ __device__ bool grid_barrier(const Pool &p, unsigned target, int epoch, unsigned
             if (ld_acquire(&p.tail[kBarAbort]) == epoch + 1) { ok = false; break; }
             const uint64_t t = global_ns();
             if (t0 == 0) t0 = t;
-            else if (t - t0 > kBarrierLimitNs) {
+            else if (t - t0 > limit_ns) {
                 atomicExch(&p.tail[kBarAbort], epoch + 1);
                 p.hdr[5] = 0;
                 record_error(err, PA_DEVERR_TIMEOUT);
@@ -664,6 +672,7 @@ __device__ bool grid_barrier(const Pool &p, unsigned target, int epoch, unsigned
 constexpr int kFusedEntries = 4;
 constexpr int kFusedBeams = 4;
 
+template <bool kHook>
 __global__ void __launch_bounds__(kStepThreads) beam_step_kernel(const StepParams q) {
     extern __shared__ int dyn[];
     __shared__ int s_bad, s_go;
@@ -746,7 +755,9 @@ __global__ void __launch_bounds__(kStepThreads) beam_step_kernel(const StepParam
         if (tid == 0 && st.bad) atomicOr(status, st.bad);
     }
 
-    bool go = grid_barrier(p, base + G, epoch, q.err, &s_go);
+    // (hook instance: the bound given, and one CTA that never arrives here)
+    const uint64_t blim = kHook && q.barrier_limit_ns ? q.barrier_limit_ns : kBarrierLimitNs;
+    bool go = grid_barrier(p, base + G, epoch, q.err, &s_go, blim, !(kHook && (int)blockIdx.x == q.withhold_cta));
     // ---- phase 2: which entries free their block (count reaches 0 at its last
     // release); per-chunk totals; CTA 0 decides each new beam's take and copy.
     // Every load of the phase is issued before the status is tested.
@@ -810,7 +821,7 @@ __global__ void __launch_bounds__(kStepThreads) beam_step_kernel(const StepParam
         }
     }
 
-    go = grid_barrier(p, base + 2 * G, epoch, q.err, &s_go) && go;
+    go = grid_barrier(p, base + 2 * G, epoch, q.err, &s_go, blim) && go;
     // ---- phase 3: apply. Deltas are swapped out first (their values are
     // needed only once the outcome is known), then freed blocks go to the
     // back of the free list in entry order, counts take their net change, the
@@ -861,7 +872,7 @@ __global__ void __launch_bounds__(kStepThreads) beam_step_kernel(const StepParam
         }
     }
     const bool early = policy == PA_POOL_FIFO && takes <= count;  // the same in every CTA
-    if (!early) go = grid_barrier(p, base + 3 * G, epoch, q.err, &s_go) && go;  // the freed blocks are listed
+    if (!early) go = grid_barrier(p, base + 3 * G, epoch, q.err, &s_go, blim) && go;  // the freed blocks are listed
     if (blockIdx.x == 0) {
         const bool ok4 = ok && go;
 #pragma unroll
@@ -933,8 +944,12 @@ cudaError_t launch_dpool_load(int32_t *state, int num_blocks, int block_size, in
 cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const int32_t *old_ctx, int num_old,
                              const int32_t *parents, int num_new, int32_t *new_tables, int32_t *new_ctx,
                              int max_blocks, int32_t *slots, int64_t *cow_pairs, int32_t *num_cow,
-                             int num_blocks, int block_size, unsigned int *err, cudaStream_t stream) {
+                             int num_blocks, int block_size, unsigned int *err, cudaStream_t stream,
+                             int withhold_cta, unsigned long long barrier_limit_ns) {
+    const bool hook = withhold_cta >= 0;
     beam::StepParams q;
+    q.withhold_cta = withhold_cta;
+    q.barrier_limit_ns = barrier_limit_ns;
     q.state = state;
     q.old_tables = old_tables;
     q.old_ctx = old_ctx;
@@ -968,9 +983,10 @@ cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const in
         const long long chunk = fused_chunk;
         q.chunk = (int)chunk;
         q.num_chunks = (int)std::max(1LL, (entries + chunk - 1) / chunk);
-        static AttrCache fused_attr;
-        cudaError_t e = ensure_smem_attr(reinterpret_cast<const void *>(beam::beam_step_kernel),
-                                         beam::kMaxStageBytes, &fused_attr);
+        static AttrCache fused_attr[2];
+        const void *fused = hook ? reinterpret_cast<const void *>(beam::beam_step_kernel<true>)
+                                 : reinterpret_cast<const void *>(beam::beam_step_kernel<false>);
+        cudaError_t e = ensure_smem_attr(fused, beam::kMaxStageBytes, &fused_attr[hook ? 1 : 0]);
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(q.num_chunks);
@@ -982,11 +998,13 @@ cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const in
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, beam::beam_step_kernel, q);
+        e = hook ? cudaLaunchKernelEx(&cfg, beam::beam_step_kernel<true>, q)
+                 : cudaLaunchKernelEx(&cfg, beam::beam_step_kernel<false>, q);
         if (e == cudaSuccess) return cudaSuccess;
         if (e != cudaErrorCooperativeLaunchTooLarge && e != cudaErrorNotSupported) return e;
         (void)cudaGetLastError();  // not launched: the four launches below instead
     }
+    if (hook) return cudaErrorNotSupported;  // the hook is the one-launch form's only
     // Four launches (launches 2-4 by programmatic dependent launch), chunks
     // of at least one entry per thread, at most kMaxChunks of them.
     const long long chunk = chunk_for(beam::kMaxChunks);

@@ -106,10 +106,12 @@ cudaError_t launch_dpool_init(int32_t *state, int num_blocks, int block_size, in
 cudaError_t launch_dpool_load(int32_t *state, int num_blocks, int block_size, int policy, const int32_t *ref_counts,
                               const int32_t *free_list, int num_free, unsigned int *err, cudaStream_t stream);
 
+// withhold_cta >= 0: the test hook (pa_beam_step_withhold_arrival), one-launch form only.
 cudaError_t launch_beam_step(int32_t *state, const int32_t *old_tables, const int32_t *old_ctx, int num_old,
                              const int32_t *parents, int num_new, int32_t *new_tables, int32_t *new_ctx,
                              int max_blocks, int32_t *slots, int64_t *cow_pairs, int32_t *num_cow,
-                             int num_blocks, int block_size, unsigned int *err, cudaStream_t stream);
+                             int num_blocks, int block_size, unsigned int *err, cudaStream_t stream,
+                             int withhold_cta = -1, unsigned long long barrier_limit_ns = 0);
 
 // A rank-2 TMA tensor map over `rows` rows of `inner` elements (row stride in
 // bytes), box box_inner x box_rows, zero fill. False if the encoder is

@@ -202,3 +202,90 @@ def test_prefill_hook_arguments_are_checked(pa):
         pa.pa_prefill_withhold_tile(out64, p64["q"], p64["qs"], p64["max_q"], p64["k"], p64["v"], p64["bt"], p64["cl"],
                                     p64["scale"], 0, 0, 0, 0, LIMIT_NS)
     assert e.value.status == -5
+
+
+# ---- beam step (one cooperative launch): a CTA that never reaches the first grid barrier
+
+def _beam_setup(pa, nb, bs, lengths, seed):
+    from oracle.block_pool import BlockPool as OPool, Sequence, append_tokens
+    order = np.random.default_rng(seed).permutation(nb).astype(np.int32)
+    opool = OPool(nb, bs, policy="fifo", free_order=order.tolist())
+    hpool = pa.BlockPool(nb, bs, pa.PA_POOL_FIFO, free_order=order)
+    beams = []
+    for n in lengths:
+        s = Sequence()
+        append_tokens(opool, s, n)
+        beams.append(s)
+        tab = np.full(nb, -1, np.int32)
+        hpool.append(tab, 0, n)
+    return opool, hpool, beams
+
+
+def _beam_args(beams, parents, mb):
+    tabs = np.full((len(beams), mb), -1, np.int32)
+    for i, b in enumerate(beams):
+        tabs[i, :len(b.block_table)] = b.block_table
+    n = len(parents)
+    return dict(old_t=torch.from_numpy(tabs).cuda(),
+                old_c=torch.tensor([b.num_tokens for b in beams], dtype=torch.int32, device="cuda"),
+                par=torch.tensor(parents, dtype=torch.int32, device="cuda"),
+                new_t=torch.full((n, mb), 7777, dtype=torch.int32, device="cuda"),
+                new_c=torch.full((n,), -5, dtype=torch.int32, device="cuda"),
+                slots=torch.full((n,), -5, dtype=torch.int32, device="cuda"),
+                cow=torch.full((n, 2), -5, dtype=torch.int64, device="cuda"),
+                ncow=torch.full((1,), -5, dtype=torch.int32, device="cuda"))
+
+
+def test_beam_barrier_wait_times_out_and_marks_the_state(pa):
+    from oracle.block_pool import beam_step
+    nb, bs, mb = 600, 16, 24
+    rng = np.random.default_rng(21)
+    lengths = [int(x) for x in rng.integers(1, 300, 40)]          # 40 beams x 24 entries: 4 CTAs of 256
+    parents = [int(x) for x in rng.integers(0, 40, 40)]
+    opool, hpool, beams = _beam_setup(pa, nb, bs, lengths, seed=21)
+    dpool = pa.DevicePool(nb, bs, pa.PA_POOL_FIFO, host_pool=hpool)
+    h = pa.PA_DPOOL_HEADER_WORDS
+    before = torch.cat([dpool.state[:5], dpool.state[h:h + 6 * nb]]).clone()
+    assert int(dpool.state[5].item()) != 0 and pa.pa_read_device_errors() == 0
+    a = _beam_args(beams, parents, mb)
+    t = time.perf_counter()
+    pa.pa_beam_step_withhold_arrival(dpool, a["old_t"], a["old_c"], a["par"], a["new_t"], a["new_c"], a["slots"],
+                                     a["cow"], a["ncow"], 2, LIMIT_NS)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t
+    assert wall < 2.0  # bounded waits of 5 ms, not the default 200 ms, and never a hang
+    assert pa.pa_read_device_errors() & pa.PA_DEVERR_TIMEOUT
+    assert (a["slots"].cpu().numpy() == -1).all() and int(a["ncow"].item()) == 0
+    # nothing applied; the state is marked unusable (header word 5)
+    assert torch.equal(torch.cat([dpool.state[:5], dpool.state[h:h + 6 * nb]]), before)
+    assert int(dpool.state[5].item()) == 0
+    # reloaded from the host pool, the same step runs clean and matches the oracle
+    dpool = pa.DevicePool(nb, bs, pa.PA_POOL_FIFO, host_pool=hpool)
+    a = _beam_args(beams, parents, mb)
+    pa.pa_beam_step(dpool, a["old_t"], a["old_c"], a["par"], a["new_t"], a["new_c"], a["slots"], a["cow"], a["ncow"])
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_errors() == 0
+    children, slots, cow = beam_step(opool, beams, parents)
+    assert a["slots"].cpu().tolist() == slots
+    assert int(a["ncow"].item()) == len(cow)
+    assert a["cow"].cpu().numpy()[:len(cow)].tolist() == [list(c) for c in cow]
+    assert dpool.ref.cpu().tolist() == opool.ref_counts and dpool.free_list() == opool.free_blocks
+
+
+def test_beam_hook_arguments_are_checked(pa):
+    opool, hpool, beams = _beam_setup(pa, 64, 16, [20, 5], seed=22)
+    dpool = pa.DevicePool(64, 16, pa.PA_POOL_FIFO, host_pool=hpool)
+    a = _beam_args(beams, [0, 1], 4)
+    for cta, lim in ((-1, LIMIT_NS), (0, 10), (0, 2_000_000_000)):
+        with pytest.raises(pa.PagedAttentionError) as e:
+            pa.pa_beam_step_withhold_arrival(dpool, a["old_t"], a["old_c"], a["par"], a["new_t"], a["new_c"],
+                                             a["slots"], a["cow"], a["ncow"], cta, lim)
+        assert e.value.status == -3
+    # a CTA past the launch withholds nothing: the step is pa_beam_step's
+    pa.pa_beam_step_withhold_arrival(dpool, a["old_t"], a["old_c"], a["par"], a["new_t"], a["new_c"], a["slots"],
+                                     a["cow"], a["ncow"], 50, LIMIT_NS)
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_errors() == 0
+    from oracle.block_pool import beam_step
+    _, slots, _ = beam_step(opool, beams, [0, 1])
+    assert a["slots"].cpu().tolist() == slots
