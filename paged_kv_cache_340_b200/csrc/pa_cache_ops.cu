@@ -59,7 +59,18 @@ __global__ void __launch_bounds__(256)
     const long long chunk = (vecs_per_block + gridDim.z - 1) / gridDim.z;
     const long long begin = blockIdx.z * chunk;
     const long long end = min(begin + chunk, vecs_per_block);
-    for (long long i = begin + threadIdx.x; i < end; i += blockDim.x) d[i] = s[i];
+    // kU loads in flight per thread before their stores (the read-only path
+    // is safe: within a call no block is both copied from and written to)
+    constexpr int kU = 8;
+    long long i = begin + threadIdx.x;
+    for (; i + (kU - 1) * (long long)blockDim.x < end; i += kU * (long long)blockDim.x) {
+        uint4 r[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) r[u] = __ldg(s + i + u * blockDim.x);
+#pragma unroll
+        for (int u = 0; u < kU; ++u) d[i + u * blockDim.x] = r[u];
+    }
+    for (; i < end; i += blockDim.x) d[i] = s[i];
 }
 
 cudaError_t launch_reshape_and_cache(const void *key, const void *value, void *k_cache,
@@ -85,8 +96,8 @@ cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *pair
                                unsigned int *err, cudaStream_t stream) {
     if (num_pairs == 0) return cudaSuccess;
     const long long vecs = (long long)(block_bytes / 16);
-    // about 16 KiB per CTA
-    long long chunks = (vecs + 1023) / 1024;
+    // about 32 KiB per CTA
+    long long chunks = (vecs + 2047) / 2048;
     if (chunks < 1) chunks = 1;
     if (chunks > 65535) chunks = 65535;
     dim3 grid((unsigned)num_pairs, 2, (unsigned)chunks);
