@@ -1142,18 +1142,32 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
     for (int i = lane; i < n; i += 32) M = fmaxf(M, ml[2 * i]);
 #pragma unroll
     for (int mk = 16; mk >= 1; mk >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, mk));
-    // this warp's partitions: weights e^(m_p - M), sum of w l, sum of w acc
+    // this warp's partitions (w, w + 8, ... in that order): weights
+    // e^(m_p - M), sum of w l, sum of w acc. Four partitions' loads are
+    // issued before any is used (one L2 round trip for four).
+    constexpr int kU = 4;
     float den = 0.f;
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = warp; i < n; i += kReduceWarps) {
-        const float w = fast_exp2((ml[2 * i] - M) * kLog2e);
-        den = fmaf(w, ml[2 * i + 1], den);
-        if (lane < vec) {
-            const float4 a = acc[(size_t)i * vec + lane];
-            num.x = fmaf(w, a.x, num.x);
-            num.y = fmaf(w, a.y, num.y);
-            num.z = fmaf(w, a.z, num.z);
-            num.w = fmaf(w, a.w, num.w);
+    for (int i = warp; i < n; i += kReduceWarps * kU) {
+        float m[kU], l[kU];
+        float4 a[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int iu = i + u * kReduceWarps;
+            const bool ok = iu < n;
+            m[u] = ok ? ml[2 * iu] : -INFINITY;
+            l[u] = ok ? ml[2 * iu + 1] : 0.f;
+            a[u] = (ok && lane < vec) ? acc[(size_t)iu * vec + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            if (i + u * kReduceWarps >= n) break;
+            const float w = fast_exp2((m[u] - M) * kLog2e);
+            den = fmaf(w, l[u], den);
+            num.x = fmaf(w, a[u].x, num.x);
+            num.y = fmaf(w, a[u].y, num.y);
+            num.z = fmaf(w, a[u].z, num.z);
+            num.w = fmaf(w, a[u].w, num.w);
         }
     }
     if (lane == 0) red_l[warp] = den;
