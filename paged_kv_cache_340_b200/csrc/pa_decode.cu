@@ -68,10 +68,14 @@ struct DecodeShape {
     static constexpr int kThreads = kWarps * 32;
     static constexpr int kTileBytes = kTS * D * kElt;  // 16 token rows of one kv head, K or V
     static constexpr int kScaleBytes = kInt8 ? kTS * 4 : 0;  // int8: the 16 rows' fp32 scales, K or V
-    // int8 with 128-byte rows: V tiles come by 2-D TMA in the 128-byte
-    // swizzled layout, in their own 1024-byte-aligned region; each stage
-    // buffer then holds K and the scales only.
-    static constexpr bool kVSwizzle = kInt8 && D == 128;
+    // The tensor-core consumers (int8 with 128-byte rows, 16-bit head groups
+    // of two or more): V tiles come by 2-D TMA in the 128-byte swizzled
+    // layout, as kVBoxes boxes of 16 rows x 128 bytes, in their own
+    // 1024-byte-aligned region; each stage buffer then holds K (and the
+    // scales) only. The V fragment loads read four rows per quarter-warp, a
+    // 4-way bank conflict in the plain layout and none in the swizzled one.
+    static constexpr bool kVSwizzle = (kInt8 && D == 128) || (kUseMma && kElt == 2);
+    static constexpr int kVBoxes = kInt8 ? 1 : D * kElt / 128;
     static constexpr int kStageBytes = (kVSwizzle ? 1 : 2) * kTileBytes + 2 * kScaleBytes;
     static constexpr int kScaleOff = (kVSwizzle ? 1 : 2) * kTileBytes;  // scales within a stage buffer
     // Buffers per warp (a ring of kWarps * kBufPerWarp stages). int8 stages
@@ -450,11 +454,24 @@ struct MmaConsumer {
         uint32_t a_lo[kMT][4];  // V^T A fragments of this stage
 #pragma unroll
         for (int ch = 0; ch < kCh; ++ch) {
-            const T *vcol = Vs + 64 * ch + 8 * r;
-            uint4 va = *reinterpret_cast<const uint4 *>(vcol + (2 * q4) * D);
-            uint4 vb = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 1) * D);
-            uint4 vc = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 8) * D);
-            uint4 vd = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 9) * D);
+            uint4 va, vb, vc, vd;
+            if constexpr (S::kVSwizzle) {
+                // box ch (dims 64 ch ..): row t at 128 t, its 16-byte chunk c at (c ^ t % 8) * 16
+                const unsigned char *vbox = Vb + ch * 2048;
+                auto row = [&](int t) {
+                    return *reinterpret_cast<const uint4 *>(vbox + t * 128 + ((r ^ (t & 7)) << 4));
+                };
+                va = row(2 * q4);
+                vb = row(2 * q4 + 1);
+                vc = row(2 * q4 + 8);
+                vd = row(2 * q4 + 9);
+            } else {
+                const T *vcol = Vs + 64 * ch + 8 * r;
+                va = *reinterpret_cast<const uint4 *>(vcol + (2 * q4) * D);
+                vb = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 1) * D);
+                vc = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 8) * D);
+                vd = *reinterpret_cast<const uint4 *>(vcol + (2 * q4 + 9) * D);
+            }
             if (nvalid < S::kTS) {  // rows past the context may hold anything
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
                 if (2 * q4 >= nvalid) va = z;
@@ -948,9 +965,12 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
             unsigned char *dst = ring + S::kVRegion + (size_t)buf * S::kStageBytes;
             mbar_arrive_expect_tx(full + buf, 2 * S::kTileBytes + 2 * S::kScaleBytes);
             bulk_load(dst, kc + src, S::kTileBytes, full + buf, pol);
-            if constexpr (S::kVSwizzle) {  // V: pool row (block, kv head, token) as a 2-D box
+            if constexpr (S::kVSwizzle) {  // V: pool rows (block, kv head, token) as 2-D boxes of 128 bytes
                 const int vrow = (int)(((long long)id * p.num_kv_heads + kvh) * BS + (k % S::kSubs) * S::kTS);
-                tma_load_2d(ring + (size_t)buf * S::kTileBytes, &p.v_map, 0, vrow, full + buf);
+#pragma unroll
+                for (int h = 0; h < S::kVBoxes; ++h)
+                    tma_load_2d(ring + (size_t)buf * S::kTileBytes + h * 2048, &p.v_map, h * (128 / S::kElt), vrow,
+                                full + buf);
             } else {
                 bulk_load(dst + S::kTileBytes, vc + src, S::kTileBytes, full + buf, pol);
             }
@@ -1034,7 +1054,13 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
                         if (c < 2 * kRowChunks) {
                             const bool isv = c >= kRowChunks;
                             const int cc = c % kRowChunks;
-                            reinterpret_cast<uint4 *>(Kw + (isv ? S::kTileBytes : 0) + (size_t)r * D * S::kElt)[cc] = nrow[i];
+                            if (S::kVSwizzle && isv) {  // the swizzled V box of chunk cc (128 bytes a box)
+                                unsigned char *vbox = ring + (size_t)buf * S::kTileBytes + (cc >> 3) * 2048;
+                                *reinterpret_cast<uint4 *>(vbox + r * 128 + (((cc & 7) ^ (r & 7)) << 4)) = nrow[i];
+                            } else {
+                                reinterpret_cast<uint4 *>(Kw + (isv ? S::kTileBytes : 0) + (size_t)r * D * S::kElt)[cc] =
+                                    nrow[i];
+                            }
                             if (sub == 0) {  // one CTA of the kv head writes the pool
                                 const unsigned char *pool = reinterpret_cast<const unsigned char *>(isv ? vc : kc);
                                 reinterpret_cast<uint4 *>(const_cast<unsigned char *>(pool) + prow)[cc] = nrow[i];
@@ -1248,9 +1274,21 @@ static cudaError_t dispatch_append(const DecodeParams &p, int head_dim, int bloc
                      : dispatch_shape<T, T, false>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream);
 }
 
-cudaError_t launch_decode(const DecodeParams &p, pa_dtype kv_dtype, int head_dim, int block_size,
+cudaError_t launch_decode(const DecodeParams &p0, pa_dtype kv_dtype, int head_dim, int block_size,
                           int group, int grid_x, int num_kv_heads, int num_seqs,
                           cudaStream_t stream) {
+    DecodeParams p = p0;
+    if ((kv_dtype == PA_F16 || kv_dtype == PA_BF16) && padded_group(group) >= 2) {
+        // the tensor-core consumer's V tiles: the V pool as rows of head_dim
+        // 16-bit elements, boxes of 64 elements x 16 rows, 128-byte swizzle
+        const long long rows = (long long)p.num_blocks * num_kv_heads * block_size;
+        if (rows >= INT_MAX) return cudaErrorInvalidValue;  // TMA row coordinates are 32-bit
+        if (rows > 0 &&
+            !encode_rows_2d(&p.v_map, kv_dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                            p.v_cache, (unsigned long long)head_dim, (unsigned long long)rows,
+                            (unsigned long long)head_dim * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
     switch (kv_dtype) {
         case PA_F32: return dispatch_append<float>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream);
         case PA_F16: return dispatch_append<__half>(p, head_dim, block_size, group, grid_x, num_kv_heads, num_seqs, stream);
