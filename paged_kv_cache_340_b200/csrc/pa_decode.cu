@@ -347,9 +347,11 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
 //   O^T += V^T P^T: M = 16 head dims per tile, N = 8 query-head columns,
 //     K = 16 tokens. P^T's B fragment is the S^T accumulator, packed to 16
 //     bits and transposed in registers (movmatrix). V^T's A fragment is built
-//     with byte permutes from 16-byte loads of V rows (no transposing load,
-//     no bank conflicts): tile mt row m holds d = 8 (m % 8) + E % 8 +
-//     64 (E / 8) with E = mt for m < 8 and E = mt + D/16 for m >= 8.
+//     with byte permutes from 16-byte loads of V rows (no transposing load;
+//     the V tile is in the 128-byte swizzled layout, so the four rows a
+//     quarter-warp reads fall in different banks): tile mt row m holds
+//     d = 8 (m % 8) + E % 8 + 64 (E / 8) with E = mt for m < 8 and
+//     E = mt + D/16 for m >= 8.
 // Running max / sum per (query head, warp); tokens past the context are
 // masked to -inf and their V rows zeroed (they may hold NaN).
 template <typename T, int D, int G, typename S>

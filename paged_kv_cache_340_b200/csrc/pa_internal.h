@@ -64,9 +64,11 @@ struct DecodeParams {
     int withhold_kvh = -1;
     int withhold_stage = -1;
     unsigned long long wait_limit_ns = 0;
-    // int8 caches with head_dim 128: the V pool as rows of 128 bytes, 16-row
-    // boxes in the 128-byte swizzled layout (the kernel's V fragment loads are
-    // then free of shared-memory bank conflicts)
+    // The tensor-core consumers (int8 caches with head_dim 128; 16-bit caches
+    // with head groups of two or more, set by launch_decode): the V pool as
+    // 2-D rows, boxes of 128 bytes x 16 rows in the 128-byte swizzled layout
+    // (the kernel's V fragment loads are then free of shared-memory bank
+    // conflicts)
     alignas(64) CUtensorMap v_map;
 };
 
