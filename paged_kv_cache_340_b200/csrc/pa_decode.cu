@@ -76,6 +76,10 @@ struct DecodeShape {
     // 4-way bank conflict in the plain layout and none in the swizzled one.
     static constexpr bool kVSwizzle = (kInt8 && D == 128) || (kUseMma && kElt == 2);
     static constexpr int kVBoxes = kInt8 ? 1 : D * kElt / 128;
+    // 16-bit tensor-core consumer: K comes the same way, into the stage
+    // buffer (1024-byte aligned there), and its lanes take the chunks of a
+    // row in an order that keeps a quarter-warp's two rows on different banks
+    static constexpr bool kKSwizzle = kUseMma && kElt == 2;
     static constexpr int kStageBytes = (kVSwizzle ? 1 : 2) * kTileBytes + 2 * kScaleBytes;
     static constexpr int kScaleOff = (kVSwizzle ? 1 : 2) * kTileBytes;  // scales within a stage buffer
     // Buffers per warp (a ring of kWarps * kBufPerWarp stages). int8 stages
@@ -111,6 +115,7 @@ struct DecodeShape {
     static_assert(kUseMma || G <= kLpt, "a lane's kept scores must belong to one query head");
     static_assert(kUseMma || kNvl <= kTc, "kept scores within one head");
     static_assert(kDataBytes % 16 == 0, "barriers, flags, hook and query fragments stay 16-byte aligned");
+    static_assert(!kKSwizzle || (kVRegion % 1024 == 0 && kStageBytes % 1024 == 0), "swizzled K boxes 1024-byte aligned");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -341,14 +346,15 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
 // group's 2-8 query heads. Per 16-token stage, with lane = 4 r + q:
 //   S^T = K Q^T: M = the stage's 16 tokens, N = 8 query-head columns (the
 //     group, zero-padded), K = head_dim. The k -> d map of each k-step is
-//     chosen so that one 16-byte shared load of a K row (d = 8q + 32i .. +8)
-//     feeds two k-steps; Q's B fragment, loaded once, uses the same map.
+//     chosen so that one 16-byte shared load of a K row (chunk kchunk(i),
+//     d = 8 kchunk(i) .. +8) feeds two k-steps; Q's B fragment, loaded once,
+//     uses the same map.
 //     Lane holds S^T[t][g] for t in {r, r + 8}, g in {2q, 2q + 1}.
 //   O^T += V^T P^T: M = 16 head dims per tile, N = 8 query-head columns,
 //     K = 16 tokens. P^T's B fragment is the S^T accumulator, packed to 16
 //     bits and transposed in registers (movmatrix). V^T's A fragment is built
 //     with byte permutes from 16-byte loads of V rows (no transposing load;
-//     the V tile is in the 128-byte swizzled layout, so the four rows a
+//     the K and V tiles are in the 128-byte swizzled layout, so the rows a
 //     quarter-warp reads fall in different banks): tile mt row m holds
 //     d = 8 (m % 8) + E % 8 + 64 (E / 8) with E = mt for m < 8 and
 //     E = mt + D/16 for m >= 8.
@@ -365,6 +371,9 @@ struct MmaConsumer {
     float o[kMT][4];
     float m_run[2], l_lane[2];
 
+    // 16-byte chunk (of a K or Q row) a lane of quarter q takes in QK step i
+    __device__ __forceinline__ int kchunk(int i) const { return 2 * q4 + (i & 1) + 8 * (i >> 1); }
+
     static __device__ __forceinline__ int dim_of(int m, int mt) {  // head dim of m-tile mt, row m
         const int E = m < 8 ? mt : mt + kMT;
         return 8 * (m & 7) + (E & 7) + 64 * (E >> 3);
@@ -376,9 +385,9 @@ struct MmaConsumer {
 #pragma unroll
         for (int i = 0; i < kI; ++i) {
             uint4 u = make_uint4(0u, 0u, 0u, 0u);
-            if (r < g_valid)
+            if (r < g_valid)  // the 16-byte chunk K's lanes take in step i (see stage())
                 u = *reinterpret_cast<const uint4 *>(static_cast<const T *>(p.query) + (head0 + r) * D +
-                                                     8 * q4 + 32 * i);
+                                                     8 * kchunk(i));
             qb[i][0] = u.x;
             qb[i][1] = u.y;
             qb[i][2] = u.z;
@@ -392,16 +401,18 @@ struct MmaConsumer {
 
     __device__ __forceinline__ void stage(const unsigned char *Kb, const unsigned char *Vb, int nvalid, int,
                                           float scale_log2) {
-        const T *Ks = reinterpret_cast<const T *>(Kb);
         const T *Vs = reinterpret_cast<const T *>(Vb);
-        // ---- S^T = K Q^T
+        // ---- S^T = K Q^T. The K tile is in the 128-byte swizzled layout
+        // (boxes of 64 dims x 16 rows, chunk c of row t at c ^ t % 8); in step
+        // i a lane takes 16-byte chunk kchunk(i) of rows r and r + 8, so the
+        // quarter-warp's rows r = 0, 1 read the even and the odd chunks.
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
-        const T *k0 = Ks + r * D + 8 * q4;
-        const T *k1 = k0 + 8 * D;
 #pragma unroll
         for (int i = 0; i < kI; ++i) {
-            const uint4 u0 = *reinterpret_cast<const uint4 *>(k0 + 32 * i);
-            const uint4 u1 = *reinterpret_cast<const uint4 *>(k1 + 32 * i);
+            const int c = kchunk(i);
+            const unsigned char *kbox = Kb + (c >> 3) * 2048;
+            const uint4 u0 = *reinterpret_cast<const uint4 *>(kbox + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+            const uint4 u1 = *reinterpret_cast<const uint4 *>(kbox + (r + 8) * 128 + (((c & 7) ^ (r & 7)) << 4));
             M::mma(sc, u0.x, u1.x, u0.y, u1.y, qb[i][0], qb[i][1]);
             M::mma(sc, u0.z, u1.z, u0.w, u1.w, qb[i][2], qb[i][3]);
         }
@@ -966,7 +977,14 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
             const size_t src = (size_t)id * block_elems + (size_t)(k % S::kSubs) * S::kTS * D;
             unsigned char *dst = ring + S::kVRegion + (size_t)buf * S::kStageBytes;
             mbar_arrive_expect_tx(full + buf, 2 * S::kTileBytes + 2 * S::kScaleBytes);
-            bulk_load(dst, kc + src, S::kTileBytes, full + buf, pol);
+            if constexpr (S::kKSwizzle) {  // K: the same pool rows as V, boxes of 128 bytes
+                const int krow = (int)(((long long)id * p.num_kv_heads + kvh) * BS + (k % S::kSubs) * S::kTS);
+#pragma unroll
+                for (int h = 0; h < S::kVBoxes; ++h)
+                    tma_load_2d(dst + h * 2048, &p.k_map, h * (128 / S::kElt), krow, full + buf);
+            } else {
+                bulk_load(dst, kc + src, S::kTileBytes, full + buf, pol);
+            }
             if constexpr (S::kVSwizzle) {  // V: pool rows (block, kv head, token) as 2-D boxes of 128 bytes
                 const int vrow = (int)(((long long)id * p.num_kv_heads + kvh) * BS + (k % S::kSubs) * S::kTS);
 #pragma unroll
@@ -1059,6 +1077,9 @@ __global__ void __launch_bounds__(DecodeShape<T, D, BS, G>::kThreads, DecodeShap
                             if (S::kVSwizzle && isv) {  // the swizzled V box of chunk cc (128 bytes a box)
                                 unsigned char *vbox = ring + (size_t)buf * S::kTileBytes + (cc >> 3) * 2048;
                                 *reinterpret_cast<uint4 *>(vbox + r * 128 + (((cc & 7) ^ (r & 7)) << 4)) = nrow[i];
+                            } else if (S::kKSwizzle && !isv) {  // the swizzled K box
+                                *reinterpret_cast<uint4 *>(Kw + (cc >> 3) * 2048 + r * 128 + (((cc & 7) ^ (r & 7)) << 4)) =
+                                    nrow[i];
                             } else {
                                 reinterpret_cast<uint4 *>(Kw + (isv ? S::kTileBytes : 0) + (size_t)r * D * S::kElt)[cc] =
                                     nrow[i];
@@ -1285,10 +1306,13 @@ cudaError_t launch_decode(const DecodeParams &p0, pa_dtype kv_dtype, int head_di
         // 16-bit elements, boxes of 64 elements x 16 rows, 128-byte swizzle
         const long long rows = (long long)p.num_blocks * num_kv_heads * block_size;
         if (rows >= INT_MAX) return cudaErrorInvalidValue;  // TMA row coordinates are 32-bit
+        const CUtensorMapDataType dt =
+            kv_dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
         if (rows > 0 &&
-            !encode_rows_2d(&p.v_map, kv_dtype == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                            p.v_cache, (unsigned long long)head_dim, (unsigned long long)rows,
-                            (unsigned long long)head_dim * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+            (!encode_rows_2d(&p.v_map, dt, p.v_cache, (unsigned long long)head_dim, (unsigned long long)rows,
+                             (unsigned long long)head_dim * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B) ||
+             !encode_rows_2d(&p.k_map, dt, p.k_cache, (unsigned long long)head_dim, (unsigned long long)rows,
+                             (unsigned long long)head_dim * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B)))
             return cudaErrorInvalidValue;
     }
     switch (kv_dtype) {

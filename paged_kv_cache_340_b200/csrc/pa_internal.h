@@ -70,6 +70,9 @@ struct DecodeParams {
     // (the kernel's V fragment loads are then free of shared-memory bank
     // conflicts)
     alignas(64) CUtensorMap v_map;
+    // The 16-bit tensor-core consumer: the K pool the same way (set by
+    // launch_decode)
+    alignas(64) CUtensorMap k_map;
 };
 
 cudaError_t launch_decode(const DecodeParams &p, pa_dtype kv_dtype, int head_dim, int block_size,
