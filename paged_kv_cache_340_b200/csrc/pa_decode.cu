@@ -94,11 +94,11 @@ struct DecodeShape {
     static constexpr int kAgStride = kUseMma ? D + 1 : D;  // floats per merged accumulator row
     static constexpr int kMergeBytes = kRowGroups * G * (kAgStride + 2) * 4;
     static constexpr int kDataBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
-    // int8 groups of two or more heads keep the query's fixed-point MMA
+    // int8 groups of more than four heads keep the query's fixed-point MMA
     // fragments (2 D/64 16-byte words per lane) in shared memory and read
     // them once per stage: every O column is live there, and the registers
     // this frees let five CTAs share an SM without spilling.
-    static constexpr bool kQShared = kInt8 && G >= 2;
+    static constexpr bool kQShared = kInt8 && G > 4;
     static constexpr int kQBytes = kQShared ? 2 * (D / 64) * 32 * 16 : 0;
     // ring (or merge area), full barriers, per-buffer "skipped" flags, the
     // test hook and head range (32 bytes) and the shared query fragments
@@ -570,18 +570,24 @@ __device__ __forceinline__ uint32_t i8pair_to_h2(uint32_t biased, unsigned sel) 
 //     mt row m holds dim W (m % 8) + mt + (m >= 8 ? W/2 : 0).
 // Tokens past the context have p = 0 and P' = 0 (their scales may hold
 // anything; int8 codes are always finite).
+// Groups of at most four heads put head g in column 2g (kSpread): every
+// lane's even column is a head (lane q: head q) and its odd column padding,
+// so a lane runs the softmax, the rescale and the O update of one head
+// instead of two, for four heads as for one.
 template <typename TQ, int D, int G, typename S>
 struct MmaConsumerQ8 {
     static constexpr int kJ = D / 64;    // 16-byte K chunks per lane per row
     static constexpr int kMT = D / 16;   // PV m-tiles
     static constexpr int kW = D / 8;     // V dims per lane
     static constexpr bool kQShared = S::kQShared;
+    static constexpr bool kSpread = G <= 4;
+    static constexpr int kH = kSpread ? 1 : 2;  // live columns (heads) per lane
     int q4, r;
     // query as 16-bit fixed point: signed high bytes, unsigned low bytes; in
     // registers (kQShared false) or as words [2 j + 0/1][lane] of qsm
     uint32_t qhi[kQShared ? 1 : kJ][4], qlo[kQShared ? 1 : kJ][4];
     const uint4 *qsm;                    // this lane's word 0 of the shared fragments
-    float qs[2];                         // fixed-point step of heads 2q, 2q + 1
+    float qs[2];                         // fixed-point step of columns 2q, 2q + 1
     float o[kMT][4];
     float m_run[2], l_lane[2];
 
@@ -618,13 +624,16 @@ struct MmaConsumerQ8 {
         r = lane >> 2;
         float f[kJ][16];
         float amax = 0.f;
+        // this lane's B column r holds head hq (kSpread: even columns only)
+        const int hq = kSpread ? r >> 1 : r;
+        const bool live = (!kSpread || (r & 1) == 0) && hq < g_valid;
 #pragma unroll
         for (int j = 0; j < kJ; ++j) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint4 u = make_uint4(0u, 0u, 0u, 0u);
-                if (r < g_valid)
-                    u = *reinterpret_cast<const uint4 *>(static_cast<const TQ *>(p.query) + (head0 + r) * D +
+                if (live)
+                    u = *reinterpret_cast<const uint4 *>(static_cast<const TQ *>(p.query) + (head0 + hq) * D +
                                                          16 * (q4 + 4 * j) + 8 * h);
                 Elt<TQ>::unpack(u, f[j] + 8 * h);
             }
@@ -714,29 +723,32 @@ struct MmaConsumerQ8 {
         const float s1 = v1 ? ksc[r + 8] * scale_log2 : 0.f;
         float x[4];
         x[0] = v0 ? sc[0] * s0 : -INFINITY;
-        x[1] = v0 ? sc[1] * s0 : -INFINITY;
+        x[1] = (v0 && !kSpread) ? sc[1] * s0 : -INFINITY;
         x[2] = v1 ? sc[2] * s1 : -INFINITY;
-        x[3] = v1 ? sc[3] * s1 : -INFINITY;
+        x[3] = (v1 && !kSpread) ? sc[3] * s1 : -INFINITY;
         float mx0 = fmaxf(x[0], x[2]);
-        float mx1 = fmaxf(x[1], x[3]);
 #pragma unroll
-        for (int mk = 4; mk < 32; mk <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, mk));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, mk));
-        }
+        for (int mk = 4; mk < 32; mk <<= 1) mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, mk));
         const float mn0 = fmaxf(m_run[0], mx0);
-        const float mn1 = fmaxf(m_run[1], mx1);
         const float al0 = (mn0 == -INFINITY) ? 1.f : fast_exp2(m_run[0] - mn0);
-        const float al1 = (mn1 == -INFINITY) ? 1.f : fast_exp2(m_run[1] - mn1);
         m_run[0] = mn0;
-        m_run[1] = mn1;
         float pr[4];
         pr[0] = (x[0] == -INFINITY) ? 0.f : fast_exp2(x[0] - mn0);
-        pr[1] = (x[1] == -INFINITY) ? 0.f : fast_exp2(x[1] - mn1);
         pr[2] = (x[2] == -INFINITY) ? 0.f : fast_exp2(x[2] - mn0);
-        pr[3] = (x[3] == -INFINITY) ? 0.f : fast_exp2(x[3] - mn1);
         l_lane[0] = l_lane[0] * al0 + pr[0] + pr[2];
-        l_lane[1] = l_lane[1] * al1 + pr[1] + pr[3];
+        float al1 = 1.f;
+        pr[1] = pr[3] = 0.f;
+        if constexpr (!kSpread) {
+            float mx1 = fmaxf(x[1], x[3]);
+#pragma unroll
+            for (int mk = 4; mk < 32; mk <<= 1) mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, mk));
+            const float mn1 = fmaxf(m_run[1], mx1);
+            al1 = (mn1 == -INFINITY) ? 1.f : fast_exp2(m_run[1] - mn1);
+            m_run[1] = mn1;
+            pr[1] = (x[1] == -INFINITY) ? 0.f : fast_exp2(x[1] - mn1);
+            pr[3] = (x[3] == -INFINITY) ? 0.f : fast_exp2(x[3] - mn1);
+            l_lane[1] = l_lane[1] * al1 + pr[1] + pr[3];
+        }
         // ---- V scales: P' = p * sv / svmax
         const float sv0 = v0 ? vsc[r] : 0.f;
         const float sv1 = v1 ? vsc[r + 8] : 0.f;
@@ -810,21 +822,23 @@ struct MmaConsumerQ8 {
             // row r: dim mt; row r + 8: dim kW/2 + mt (of this lane's W dims)
             mma_f16(t, plo[mt], plo[kW / 2 + mt], phi[mt], phi[kW / 2 + mt], bh0, bh1);
             o[mt][0] = fmaf(svmax, t[0], o[mt][0] * al0);
-            o[mt][1] = fmaf(svmax, t[1], o[mt][1] * al1);
             o[mt][2] = fmaf(svmax, t[2], o[mt][2] * al0);
-            o[mt][3] = fmaf(svmax, t[3], o[mt][3] * al1);
+            if constexpr (!kSpread) {  // else the odd (padding) columns are never stored
+                o[mt][1] = fmaf(svmax, t[1], o[mt][1] * al1);
+                o[mt][3] = fmaf(svmax, t[3], o[mt][3] * al1);
+            }
         }
     }
 
     __device__ __forceinline__ void store(float *mg, float *lg, float *ag, int warp, int) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < kH; ++h) {
 #pragma unroll
             for (int mk = 4; mk < 32; mk <<= 1) l_lane[h] += __shfl_xor_sync(0xffffffffu, l_lane[h], mk);
         }
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int g = 2 * q4 + h;
+        for (int h = 0; h < kH; ++h) {
+            const int g = kSpread ? q4 : 2 * q4 + h;  // the head of column 2 q4 + h
             if (g < G) {
                 if (r == 0) {
                     mg[warp * G + g] = m_run[h];
