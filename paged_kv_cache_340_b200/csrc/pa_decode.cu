@@ -349,7 +349,9 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
 //     chosen so that one 16-byte shared load of a K row (chunk kchunk(i),
 //     d = 8 kchunk(i) .. +8) feeds two k-steps; Q's B fragment, loaded once,
 //     uses the same map.
-//     Lane holds S^T[t][g] for t in {r, r + 8}, g in {2q, 2q + 1}.
+//     Lane holds S^T[t][n] for t in {r, r + 8}, columns n in {2q, 2q + 1};
+//     column n is head n, or for groups of at most four heads head n / 2 on
+//     even n and padding on odd n (one head per lane, kSpread).
 //   O^T += V^T P^T: M = 16 head dims per tile, N = 8 query-head columns,
 //     K = 16 tokens. P^T's B fragment is the S^T accumulator, packed to 16
 //     bits and transposed in registers (movmatrix). V^T's A fragment is built
@@ -366,6 +368,10 @@ struct MmaConsumer {
     static constexpr int kI = D / 32;    // 16-byte chunks of a K row per lane (2 k-steps each)
     static constexpr int kMT = D / 16;   // PV m-tiles
     static constexpr int kCh = D / 64;   // 16-byte V chunks per token row per lane
+    // groups of at most four heads: head g in column 2g, one head per lane
+    // (see MmaConsumerQ8)
+    static constexpr bool kSpread = G <= 4;
+    static constexpr int kH = kSpread ? 1 : 2;  // live columns (heads) per lane
     int q4, r;
     uint32_t qb[kI][4];
     float o[kMT][4];
@@ -382,11 +388,13 @@ struct MmaConsumer {
     __device__ __forceinline__ void init(const DecodeParams &p, size_t head0, int g_valid, int, int lane) {
         q4 = lane & 3;
         r = lane >> 2;
+        const int hq = kSpread ? r >> 1 : r;  // the head of this lane's B column r
+        const bool live = (!kSpread || (r & 1) == 0) && hq < g_valid;
 #pragma unroll
         for (int i = 0; i < kI; ++i) {
             uint4 u = make_uint4(0u, 0u, 0u, 0u);
-            if (r < g_valid)  // the 16-byte chunk K's lanes take in step i (see stage())
-                u = *reinterpret_cast<const uint4 *>(static_cast<const T *>(p.query) + (head0 + r) * D +
+            if (live)  // the 16-byte chunk K's lanes take in step i (see stage())
+                u = *reinterpret_cast<const uint4 *>(static_cast<const T *>(p.query) + (head0 + hq) * D +
                                                      8 * kchunk(i));
             qb[i][0] = u.x;
             qb[i][1] = u.y;
@@ -421,35 +429,40 @@ struct MmaConsumer {
         const bool v1 = r + 8 < nvalid;
         float x[4];
         x[0] = v0 ? sc[0] * scale_log2 : -INFINITY;  // t = r,     g = 2q
-        x[1] = v0 ? sc[1] * scale_log2 : -INFINITY;  // t = r,     g = 2q + 1
+        x[1] = (v0 && !kSpread) ? sc[1] * scale_log2 : -INFINITY;  // t = r,     g = 2q + 1
         x[2] = v1 ? sc[2] * scale_log2 : -INFINITY;  // t = r + 8, g = 2q
-        x[3] = v1 ? sc[3] * scale_log2 : -INFINITY;  // t = r + 8, g = 2q + 1
+        x[3] = (v1 && !kSpread) ? sc[3] * scale_log2 : -INFINITY;  // t = r + 8, g = 2q + 1
         float mx0 = fmaxf(x[0], x[2]);
-        float mx1 = fmaxf(x[1], x[3]);
 #pragma unroll
-        for (int mk = 4; mk < 32; mk <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, mk));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, mk));
-        }
+        for (int mk = 4; mk < 32; mk <<= 1) mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, mk));
         const float mn0 = fmaxf(m_run[0], mx0);
-        const float mn1 = fmaxf(m_run[1], mx1);
         const float al0 = (mn0 == -INFINITY) ? 1.f : fast_exp2(m_run[0] - mn0);
-        const float al1 = (mn1 == -INFINITY) ? 1.f : fast_exp2(m_run[1] - mn1);
         m_run[0] = mn0;
-        m_run[1] = mn1;
         float pr[4];
         pr[0] = (x[0] == -INFINITY) ? 0.f : fast_exp2(x[0] - mn0);
-        pr[1] = (x[1] == -INFINITY) ? 0.f : fast_exp2(x[1] - mn1);
         pr[2] = (x[2] == -INFINITY) ? 0.f : fast_exp2(x[2] - mn0);
-        pr[3] = (x[3] == -INFINITY) ? 0.f : fast_exp2(x[3] - mn1);
         l_lane[0] = l_lane[0] * al0 + pr[0] + pr[2];
-        l_lane[1] = l_lane[1] * al1 + pr[1] + pr[3];
+        pr[1] = pr[3] = 0.f;
+        float al1 = 1.f;
+        if constexpr (!kSpread) {
+            float mx1 = fmaxf(x[1], x[3]);
+#pragma unroll
+            for (int mk = 4; mk < 32; mk <<= 1) mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, mk));
+            const float mn1 = fmaxf(m_run[1], mx1);
+            al1 = (mn1 == -INFINITY) ? 1.f : fast_exp2(m_run[1] - mn1);
+            m_run[1] = mn1;
+            pr[1] = (x[1] == -INFINITY) ? 0.f : fast_exp2(x[1] - mn1);
+            pr[3] = (x[3] == -INFINITY) ? 0.f : fast_exp2(x[3] - mn1);
+            l_lane[1] = l_lane[1] * al1 + pr[1] + pr[3];
+        }
 #pragma unroll
         for (int mt = 0; mt < kMT; ++mt) {
             o[mt][0] *= al0;
-            o[mt][1] *= al1;
             o[mt][2] *= al0;
-            o[mt][3] *= al1;
+            if constexpr (!kSpread) {  // else the odd (padding) columns stay 0 and are never stored
+                o[mt][1] *= al1;
+                o[mt][3] *= al1;
+            }
         }
         // ---- P^T fragments -> PV's B fragments (tokens 0-7 and 8-15)
         const uint32_t h01 = M::pack(pr[0], pr[1]);
@@ -518,13 +531,13 @@ struct MmaConsumer {
     // Row stride D + 1 keeps the scattered stores off a single bank.
     __device__ __forceinline__ void store(float *mg, float *lg, float *ag, int warp, int) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < kH; ++h) {
 #pragma unroll
             for (int mk = 4; mk < 32; mk <<= 1) l_lane[h] += __shfl_xor_sync(0xffffffffu, l_lane[h], mk);
         }
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int g = 2 * q4 + h;
+        for (int h = 0; h < kH; ++h) {
+            const int g = kSpread ? q4 : 2 * q4 + h;  // the head of column 2 q4 + h
             if (g < G) {
                 if (r == 0) {
                     mg[warp * G + g] = m_run[h];
