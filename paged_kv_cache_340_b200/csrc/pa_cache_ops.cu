@@ -8,35 +8,77 @@ namespace pa {
 // Slot write ([P3 "Ascend C ... PagedAttention融合算子", §3.1 and §4.2:
 // block = slot / block_size, offset = slot % block_size]; [P4 "PagedAttention
 // 实现细节", §3.4: each new token's K/V goes into its block).
-// One thread moves one 16-byte vector of one (token, kv head) row of both key
-// and value; consecutive threads cover consecutive vectors of the source, so
-// loads and stores are coalesced per row.
+// A token's K (or V) is num_kv_heads rows of 2^kVShift 16-byte vectors, in the
+// source contiguous (per_token vectors) and in the pool one row per kv head.
+// Thread t of a CTA always moves vector j of (token group member) tin, with
+// (tin, j) fixed for the whole kernel, so no index is divided in the loop:
+// CTAs of 256 threads take tpi = 256 / per_token tokens at a time when a
+// token has at most 256 vectors, else one token in rounds of 256 vectors.
+// Each thread keeps kU tokens' (or rounds') loads in flight before storing.
+template <int kVShift>
 __global__ void __launch_bounds__(256)
     reshape_and_cache_kernel(const uint4 *__restrict__ key, const uint4 *__restrict__ value,
                              uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
                              const int32_t *__restrict__ slot_mapping, int num_tokens,
-                             int num_blocks, int num_kv_heads, int vecs_per_row, int block_size,
-                             unsigned int *err) {
-    const long long per_token = (long long)num_kv_heads * vecs_per_row;
-    const long long total = per_token * num_tokens;
-    const long long slots = (long long)num_blocks * block_size;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-         i += (long long)gridDim.x * blockDim.x) {
-        const int token = (int)(i / per_token);
-        const int rem = (int)(i - (long long)token * per_token);
-        const int h = rem / vecs_per_row;
-        const int v = rem - h * vecs_per_row;
+                             int num_blocks, int num_kv_heads, int bs_shift, unsigned int *err) {
+    constexpr int kU = 4;
+    const int per_token = num_kv_heads << kVShift;
+    const long long slots = (long long)num_blocks << bs_shift;
+    // one 16-byte vector: source index, token, vector j within the token
+    auto move_one = [&](int token, int j, uint4 &kr, uint4 &vr, long long &dst) {
+        dst = -1;
+        if (token >= num_tokens) return;
         const int slot = __ldg(slot_mapping + token);
-        if (slot < 0) continue;
+        if (slot < 0) return;
         if (slot >= slots) {
-            if (h == 0 && v == 0) record_error(err, PA_DEVERR_SLOT);
-            continue;
+            if (j == 0) record_error(err, PA_DEVERR_SLOT);
+            return;
         }
-        const int block = slot / block_size;
-        const int offset = slot - block * block_size;
-        const size_t dst = (((size_t)block * num_kv_heads + h) * block_size + offset) * vecs_per_row + v;
-        k_cache[dst] = __ldg(key + i);
-        v_cache[dst] = __ldg(value + i);
+        const int h = j >> kVShift;
+        const int v = j & ((1 << kVShift) - 1);
+        const long long block = slot >> bs_shift;
+        const int offset = slot & ((1 << bs_shift) - 1);
+        dst = ((((block * num_kv_heads + h) << bs_shift) + offset) << kVShift) + v;
+        const size_t src = (size_t)token * per_token + j;
+        kr = __ldg(key + src);
+        vr = __ldg(value + src);
+    };
+    if (per_token <= 256) {
+        const int tpi = 256 / per_token;  // tokens per CTA round
+        const int tin = threadIdx.x / per_token;
+        const int j = threadIdx.x - tin * per_token;
+        if (tin >= tpi) return;
+        const int step = gridDim.x * tpi;
+        for (int t0 = blockIdx.x * tpi + tin; t0 < num_tokens; t0 += kU * step) {
+            uint4 kr[kU], vr[kU];
+            long long dst[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) move_one(t0 + u * step, j, kr[u], vr[u], dst[u]);
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+                if (dst[u] >= 0) {
+                    k_cache[dst[u]] = kr[u];
+                    v_cache[dst[u]] = vr[u];
+                }
+        }
+    } else {
+        for (int token = blockIdx.x; token < num_tokens; token += gridDim.x) {
+            for (int j0 = threadIdx.x; j0 < per_token; j0 += kU * 256) {
+                uint4 kr[kU], vr[kU];
+                long long dst[kU];
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    dst[u] = -1;
+                    if (j0 + u * 256 < per_token) move_one(token, j0 + u * 256, kr[u], vr[u], dst[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < kU; ++u)
+                    if (dst[u] >= 0) {
+                        k_cache[dst[u]] = kr[u];
+                        v_cache[dst[u]] = vr[u];
+                    }
+            }
+        }
     }
 }
 
@@ -78,16 +120,33 @@ cudaError_t launch_reshape_and_cache(const void *key, const void *value, void *k
                                      int num_blocks, int num_kv_heads, int row_bytes,
                                      int block_size, unsigned int *err, cudaStream_t stream) {
     if (num_tokens == 0) return cudaSuccess;
-    const int vecs_per_row = row_bytes / 16;
-    const long long total = (long long)num_tokens * num_kv_heads * vecs_per_row;
-    const int threads = 256;
-    long long blocks = (total + threads - 1) / threads;
+    const int vecs_per_row = row_bytes / 16;  // 8, 16 or 32
+    const int bs_shift = block_size == 16 ? 4 : 5;
+    if ((long long)num_kv_heads * vecs_per_row > INT_MAX / 2) return cudaErrorInvalidValue;
+    const int per_token = num_kv_heads * vecs_per_row;
+    const long long tpi = per_token <= 256 ? 256 / per_token : 1;
+    long long blocks = (num_tokens + tpi - 1) / tpi;  // one token (or one token's rounds) a thread, up to the cap
     const long long cap = (long long)sm_count() * 8;
     if (blocks > cap) blocks = cap;
-    reshape_and_cache_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
-        static_cast<const uint4 *>(key), static_cast<const uint4 *>(value),
-        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), slot_mapping, num_tokens,
-        num_blocks, num_kv_heads, vecs_per_row, block_size, err);
+    if (blocks < 1) blocks = 1;
+    const uint4 *k = static_cast<const uint4 *>(key), *v = static_cast<const uint4 *>(value);
+    uint4 *kc = static_cast<uint4 *>(k_cache), *vc = static_cast<uint4 *>(v_cache);
+    switch (vecs_per_row) {
+        case 8:
+            reshape_and_cache_kernel<3><<<(unsigned)blocks, 256, 0, stream>>>(k, v, kc, vc, slot_mapping, num_tokens,
+                                                                              num_blocks, num_kv_heads, bs_shift, err);
+            break;
+        case 16:
+            reshape_and_cache_kernel<4><<<(unsigned)blocks, 256, 0, stream>>>(k, v, kc, vc, slot_mapping, num_tokens,
+                                                                              num_blocks, num_kv_heads, bs_shift, err);
+            break;
+        case 32:
+            reshape_and_cache_kernel<5><<<(unsigned)blocks, 256, 0, stream>>>(k, v, kc, vc, slot_mapping, num_tokens,
+                                                                              num_blocks, num_kv_heads, bs_shift, err);
+            break;
+        default:
+            return cudaErrorInvalidValue;
+    }
     return cudaGetLastError();
 }
 
