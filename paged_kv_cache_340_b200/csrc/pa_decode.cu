@@ -1196,7 +1196,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
                          const int32_t *context_lens, int num_heads, int head_dim,
                          int partition_size, int max_parts, int max_context_len,
                          pa_dtype out_dtype) {
-    __shared__ float red_l[kReduceWarps];
+    __shared__ float red_m[kReduceWarps], red_l[kReduceWarps];
     __shared__ float4 red_acc[kReduceWarps][32];
     const int h = blockIdx.x;
     const int s = blockIdx.y;
@@ -1213,16 +1213,13 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
     }
     const float *ml = ws_ml + row * max_parts * 2;
     const float4 *acc = reinterpret_cast<const float4 *>(ws_acc + row * max_parts * head_dim);
-    // M = max_p m_p (every warp computes it; n is small)
-    float M = -INFINITY;
-    for (int i = lane; i < n; i += 32) M = fmaxf(M, ml[2 * i]);
-#pragma unroll
-    for (int mk = 16; mk >= 1; mk >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, mk));
-    // this warp's partitions (w, w + 8, ... in that order): weights
-    // e^(m_p - M), sum of w l, sum of w acc. Four partitions' loads are
-    // issued before any is used (one L2 round trip for four).
-    constexpr int kU = 4;
-    float den = 0.f;
+    // One pass: warp w takes partitions w, w + 8, ... in batches of kU whose
+    // loads are all issued before any is used (one L2 round trip per batch),
+    // keeping its own running max m_w: sum of e^(m_p - m_w) l_p and of
+    // e^(m_p - m_w) acc_p, rescaled when m_w grows. The warps then merge with
+    // weights e^(m_w - M), M the largest m_w.
+    constexpr int kU = 8;
+    float m_w = -INFINITY, den = 0.f;
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int i = warp; i < n; i += kReduceWarps * kU) {
         float m[kU], l[kU];
@@ -1235,10 +1232,21 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
             l[u] = ok ? ml[2 * iu + 1] : 0.f;
             a[u] = (ok && lane < vec) ? acc[(size_t)iu * vec + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        float mb = m_w;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) mb = fmaxf(mb, m[u]);
+        if (mb == -INFINITY) continue;  // nothing finite yet
+        const float r = fast_exp2((m_w - mb) * kLog2e);  // 0 while m_w is -inf
+        den *= r;
+        num.x *= r;
+        num.y *= r;
+        num.z *= r;
+        num.w *= r;
+        m_w = mb;
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
             if (i + u * kReduceWarps >= n) break;
-            const float w = fast_exp2((m[u] - M) * kLog2e);
+            const float w = fast_exp2((m[u] - m_w) * kLog2e);
             den = fmaf(w, l[u], den);
             num.x = fmaf(w, a[u].x, num.x);
             num.y = fmaf(w, a[u].y, num.y);
@@ -1246,20 +1254,28 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
             num.w = fmaf(w, a[u].w, num.w);
         }
     }
-    if (lane == 0) red_l[warp] = den;
+    if (lane == 0) {
+        red_m[warp] = m_w;
+        red_l[warp] = den;
+    }
     red_acc[warp][lane] = num;
     __syncthreads();
     if (warp == 0) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kReduceWarps; ++w) M = fmaxf(M, red_m[w]);
         float dsum = 0.f;
         float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int w = 0; w < kReduceWarps; ++w) {
-            dsum += red_l[w];
+            const float mw = red_m[w];
+            const float f = (mw == -INFINITY) ? 0.f : fast_exp2((mw - M) * kLog2e);
+            dsum = fmaf(f, red_l[w], dsum);
             const float4 a = red_acc[w][lane];
-            t.x += a.x;
-            t.y += a.y;
-            t.z += a.z;
-            t.w += a.w;
+            t.x = fmaf(f, a.x, t.x);
+            t.y = fmaf(f, a.y, t.y);
+            t.z = fmaf(f, a.z, t.z);
+            t.w = fmaf(f, a.w, t.w);
         }
         if (lane < vec) {
             const float inv = dsum > 0.f ? 1.f / dsum : 0.f;
