@@ -424,14 +424,14 @@ struct MmaConsumer {
             M::mma(sc, u0.x, u1.x, u0.y, u1.y, qb[i][0], qb[i][1]);
             M::mma(sc, u0.z, u1.z, u0.w, u1.w, qb[i][2], qb[i][3]);
         }
-        // ---- online softmax per query head g = 2q + h (h = 0, 1) over tokens r, r + 8
+        // ---- online softmax per column n = 2q + h (h = 0, 1) over tokens r, r + 8
         const bool v0 = r < nvalid;
         const bool v1 = r + 8 < nvalid;
         float x[4];
-        x[0] = v0 ? sc[0] * scale_log2 : -INFINITY;  // t = r,     g = 2q
-        x[1] = (v0 && !kSpread) ? sc[1] * scale_log2 : -INFINITY;  // t = r,     g = 2q + 1
-        x[2] = v1 ? sc[2] * scale_log2 : -INFINITY;  // t = r + 8, g = 2q
-        x[3] = (v1 && !kSpread) ? sc[3] * scale_log2 : -INFINITY;  // t = r + 8, g = 2q + 1
+        x[0] = v0 ? sc[0] * scale_log2 : -INFINITY;  // t = r,     n = 2q
+        x[1] = (v0 && !kSpread) ? sc[1] * scale_log2 : -INFINITY;  // t = r,     n = 2q + 1
+        x[2] = v1 ? sc[2] * scale_log2 : -INFINITY;  // t = r + 8, n = 2q
+        x[3] = (v1 && !kSpread) ? sc[3] * scale_log2 : -INFINITY;  // t = r + 8, n = 2q + 1
         float mx0 = fmaxf(x[0], x[2]);
 #pragma unroll
         for (int mk = 4; mk < 32; mk <<= 1) mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, mk));
@@ -729,7 +729,7 @@ struct MmaConsumerQ8 {
         float sc[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) sc[i] = (float)((chi[i] << 8) + clo[i]) * qs[i & 1];
-        // ---- online softmax per query head g = 2q + h over tokens r, r + 8
+        // ---- online softmax per column n = 2q + h over tokens r, r + 8
         const bool v0 = r < nvalid;
         const bool v1 = r + 8 < nvalid;
         const float s0 = v0 ? ksc[r] * scale_log2 : 0.f;
