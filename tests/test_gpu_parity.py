@@ -388,3 +388,41 @@ def test_largest_batch_grid(pa):
     with pytest.raises(pa.PagedAttentionError):
         pa.pa_decode(big, big.to(torch.float16), k.cuda(), v.cuda(), torch.cat([tables, tables[:1]]).cuda(),
                      torch.cat([ctx, ctx[:1]]).cuda(), 0.125)
+
+
+# (dtype, Hkv, D, block_size, tokens): 16-byte vectors per token Hkv * D * elt / 16
+# at most 256 (several tokens per CTA round; 256 not always a multiple of it)
+# and above 256 (a token in rounds of 256 vectors, the last one partial), with
+# token counts that span many rounds of the grid and end mid-round.
+SLOT_WRITE_SHAPES = [
+    ("f16", 3, 128, 16, 3001),    # 48 vectors a token: 5 tokens a round, 16 threads idle
+    ("f32", 1, 64, 32, 777),      # 16 vectors
+    ("bf16", 24, 128, 16, 2500),  # 384 vectors: rounds of 256 and 128
+    ("f32", 8, 128, 32, 1500),    # 256 vectors: exactly one round
+    ("f32", 32, 128, 16, 9000),   # 1024 vectors: four rounds, and more tokens than the grid
+]
+
+
+@pytest.mark.parametrize("dt,Hkv,D,BS,T", SLOT_WRITE_SHAPES)
+def test_slot_write_shapes_bitwise(pa, dt, Hkv, D, BS, T):
+    """pa_reshape_and_cache against the oracle's byte copies: every pool byte
+    equal, including rows no slot names (left as they were) and tokens whose
+    slot is -1 (skipped)."""
+    dtype = DT[dt]
+    g = torch.Generator().manual_seed(1000 + Hkv * 7 + T)
+    NB = -(-T // BS) + 5
+    kp = torch.randn((NB, Hkv, BS, D), generator=g).to(dtype)
+    vp = torch.randn((NB, Hkv, BS, D), generator=g).to(dtype)
+    nk = torch.randn((T, Hkv, D), generator=g).to(dtype)
+    nv = torch.randn((T, Hkv, D), generator=g).to(dtype)
+    rng = np.random.default_rng(T)
+    slots = rng.permutation(NB * BS)[:T].astype(np.int32)  # distinct slots, any block and offset
+    slots[rng.random(T) < 0.05] = -1                        # padding tokens
+    okp, ovp = raw(kp).copy(), raw(vp).copy()
+    oracle.reshape_and_cache(okp, ovp, raw(nk), raw(nv), slots)
+    dk, dv = kp.cuda(), vp.cuda()
+    pa.pa_reshape_and_cache(nk.cuda(), nv.cuda(), dk, dv, torch.from_numpy(slots).cuda())
+    torch.cuda.synchronize()
+    assert pa.pa_read_device_errors() == 0
+    assert np.array_equal(raw(dk), okp)
+    assert np.array_equal(raw(dv), ovp)
