@@ -107,6 +107,7 @@ SHAPES = [
     (5, 16, 2, 64, 16, [15, 16, 1, 90, 257]),
     (2, 32, 4, 128, 16, [1000, 7]),
     (3, 8, 8, 64, 32, [31, 32, 129]),
+    (4, 8, 4, 128, 16, [2, 16, 33, 517]),   # head group 2 (two heads, one per lane)
 ]
 
 

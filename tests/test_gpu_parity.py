@@ -132,6 +132,7 @@ SHAPES = [
     ("bf16", 128, 32, 16, 4),
     ("bf16", 64, 32, 4, 4),
     ("bf16", 128, 16, 16, 2),
+    ("bf16", 64, 32, 8, 4),
 ]
 
 
