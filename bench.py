@@ -594,6 +594,33 @@ def measure_prefill(name: str, steps: int, warmup: int):
     return res
 
 
+def event_floor_ms(stream, reps: int = 50):
+    """Event-to-event time (median, ms) of an empty kernel between two events
+    inside a CUDA graph, the arrangement the beam step's per-kernel times are
+    read in: the part of such a time any kernel there pays. The empty kernel
+    is PyTorch's spin kernel with a zero-cycle spin (not this library's).
+    None if it cannot be measured."""
+    try:
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(0)
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                ev[0].record(stream)
+                torch.cuda._sleep(0)
+                ev[1].record(stream)
+        xs = []
+        for _ in range(reps):
+            g.replay()
+            torch.cuda.synchronize()
+            xs.append(ev[0].elapsed_time(ev[1]))
+        del g
+        return statistics.median(xs)
+    except Exception:  # a measurement aid only
+        return None
+
+
 def measure_beam(name: str, steps: int, warmup: int, host_steps: int = 30):
     """Beam-search decode steps with the beam step on the device (beam step,
     counted copy, slot write, decode; no host round trip), each step replayed
@@ -693,11 +720,13 @@ def measure_beam(name: str, steps: int, warmup: int, host_steps: int = 30):
                          spec.scale)
         torch.cuda.synchronize()
         host.append(time.perf_counter() - t)
+    floor = event_floor_ms(stream)  # what an empty kernel measures between two events in a graph
     res = {"ms_per_step": round(ms, 4), "beams": W, "steps_timed": steps, "launch": "one CUDA graph per step",
            "decode_kernel_ms": round(kern[3], 4), "decode_GBps_logical": round(dec_by / kern[3] / 1e6, 1),
            "step_GBps_logical": round(by / ms / 1e6, 1),
            "kernels_ms": {"beam_step": round(kern[0], 5), "copy_blocks_counted": round(kern[1], 5),
                           "decode_append": round(kern[3], 5)},
+           "event_floor_ms": None if floor is None else round(floor, 5),
            "device_path_wall_ms_with_sync": round(1e3 * statistics.median(wall), 4),
            "host_pool_path_wall_ms": round(1e3 * statistics.median(host), 4),
            "note": "decode bytes are logical: beams of a prompt share their prefix blocks (read from L2)"}
