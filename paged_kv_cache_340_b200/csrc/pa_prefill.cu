@@ -635,10 +635,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (!softmax_sync_and(done)) {
                 if (r == 0) record_error(p.err, PA_DEVERR_TIMEOUT);
             } else {
-                const int cpr = row_bytes / 16;  // 16-byte pieces per row
+                // 16-byte pieces per row: 2^cshift (8, 16 or 32)
+                const int cshift = (kD == 128 ? 4 : 3) + (ebytes == 4 ? 1 : 0);
+                const int cpr = 1 << cshift;
                 unsigned char *out = static_cast<unsigned char *>(p.out);
                 for (int i = r; i < rows_valid * cpr; i += kSoftmaxWarps * 32) {
-                    const int row = i / cpr, c = i % cpr;
+                    const int row = i >> cshift, c = i & (cpr - 1);
                     if ((row & (G - 1)) >= g_valid) continue;  // a padding slot
                     const size_t orow =
                         (size_t)(q0 + tok0 + (row >> gshift)) * p.num_heads + (size_t)head_base + (row & (G - 1));
