@@ -259,6 +259,33 @@ def test_splitk_reduce_on_oracle_partials(pa):
     np.testing.assert_allclose(f64(out), ref, rtol=2e-6, atol=2e-6)
 
 
+def test_splitk_reduce_many_partitions_rising_max(pa):
+    """The merge over hundreds of partitions per head, with the partitions'
+    maxima rising along the sequence (a random walk with drift) and also
+    falling in places, so each warp of the merge kernel folds several batches
+    and raises its running maximum between them; against the oracle's
+    closed-form merge."""
+    rng = np.random.default_rng(61)
+    S, H, D, P = 2, 3, 64, 16
+    ctx = np.array([P * 300 - 5, P * 97 + 1], np.int32)
+    mx = int(ctx.max())
+    mp = -(-mx // P)
+    m = np.cumsum(rng.normal(0.05, 1.5, size=(S, H, mp)), axis=-1)
+    l = rng.uniform(0.5, 40, size=(S, H, mp))
+    acc = rng.normal(size=(S, H, mp, D)) * l[..., None]
+    m32, l32, acc32 = m.astype(np.float32), l.astype(np.float32), acc.astype(np.float32)
+    ref = oracle.splitk_merge(m32.astype(np.float64), l32.astype(np.float64), acc32.astype(np.float64), ctx, P)
+    ws = torch.zeros(pa.pa_splitk_workspace_bytes(S, H, D, mx, P), dtype=torch.uint8, device="cuda")
+    wml, wacc = pa.splitk_views(ws, S, H, D, mx, P)
+    wml[..., 0] = torch.from_numpy(m32).cuda()
+    wml[..., 1] = torch.from_numpy(l32).cuda()
+    wacc.copy_(torch.from_numpy(acc32).cuda())
+    out = torch.empty((S, H, D), dtype=torch.float32, device="cuda")
+    pa.pa_splitk_reduce(out, ws, torch.from_numpy(ctx).cuda(), mx, P)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(f64(out), ref, rtol=2e-6, atol=2e-6)
+
+
 def test_partition_covering_context_equals_unsplit(pa):
     ctx = [300, 17, 999]
     c = Case(pa, torch.float16, 3, 8, 8, 128, 16, ctx, seed=7, out_dtype=torch.float32)
